@@ -1,0 +1,367 @@
+"""Pins of the CPU oracle to facts outside itself (no GPU).
+
+Each test checks one oracle function against a closed form, a hand-worked
+fixture, brute force on tiny inputs, an invariant stated by the pages, or a
+library routine on a special case — chosen so that a dropped term, a wrong
+sign or index, or a transposed operand fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+F64 = torch.float64
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------- rounding
+def test_bf16_round_matches_library_on_fp32_inputs():
+    g = torch.Generator().manual_seed(1)
+    v = torch.randn(100000, generator=g, dtype=torch.float32) * 10
+    ref = v.to(torch.bfloat16).to(F64)          # torch's fp32 -> bf16 is RNE
+    assert torch.equal(O.bf16_round(v.to(F64)), ref)
+
+
+def test_bf16_round_ties_and_no_double_rounding():
+    one = 1.0
+    assert O.bf16_round(torch.tensor([one + 2 ** -8], dtype=F64)).item() == 1.0        # tie -> even
+    assert O.bf16_round(torch.tensor([one + 3 * 2 ** -8], dtype=F64)).item() == 1.015625
+    # just above the midpoint: fp32 would first round onto the midpoint, then to 1.0
+    assert O.bf16_round(torch.tensor([one + 2 ** -8 + 2 ** -40], dtype=F64)).item() == 1.0078125
+    assert O.bf16_round(torch.tensor([-(one + 2 ** -8 + 2 ** -40)], dtype=F64)).item() == -1.0078125
+    assert O.bf16_round(torch.tensor([0.0], dtype=F64)).item() == 0.0
+
+
+# ------------------------------------------------------------ projections
+def test_linear_selection_matrix_closed_form():
+    # W = [I | 0] picks the first L input channels: z = x[:, :L] exactly.
+    T, D, L = 5, 12, 4
+    x = torch.randn(T, D, dtype=torch.float32).to(torch.bfloat16)
+    w = torch.zeros(L, D)
+    w[:, :L] = torch.eye(L)
+    z = O.linear_bf16(x, w.to(torch.bfloat16))
+    assert torch.equal(z, x[:, :L].to(F64))
+    # a permutation matrix permutes channels: catches a transposed operand
+    p = torch.tensor([2, 0, 3, 1])
+    wp = torch.zeros(L, D)
+    wp[torch.arange(L), p] = 1.0
+    assert torch.equal(O.linear_bf16(x, wp.to(torch.bfloat16)), x[:, p].to(F64))
+
+
+def test_linear_brute_force_loops():
+    g = torch.Generator().manual_seed(2)
+    T, D, L = 3, 7, 5
+    x = torch.randn(T, D, generator=g).to(torch.bfloat16)
+    w = torch.randn(L, D, generator=g).to(torch.bfloat16)
+    z = O.linear_bf16(x, w)
+    for t in range(T):
+        for o in range(L):
+            acc = math.fsum(float(x[t, i]) * float(w[o, i]) for i in range(D))
+            assert z[t, o].item() == O.bf16_round(torch.tensor([acc], dtype=F64)).item()
+
+
+# ----------------------------------------------------------------- routers
+def _sig(v):
+    return 1.0 / (1.0 + math.exp(-v))
+
+
+def test_single_router_reduces_to_sigmoid():
+    g = torch.Generator().manual_seed(3)
+    T, L, E = 4, 6, 5
+    z = torch.randn(T, L, generator=g).to(torch.bfloat16)
+    wr = torch.randn(1, E, L, generator=g).to(torch.bfloat16)
+    s = O.router_scores(z, wr)
+    for t in range(T):
+        for e in range(E):
+            logit = math.fsum(float(z[t, i]) * float(wr[0, e, i]) for i in range(L))
+            assert s[t, e].item() == np.float32(_sig(logit))
+
+
+def test_identical_routers_equal_one_router():
+    g = torch.Generator().manual_seed(4)
+    z = torch.randn(8, 16, generator=g).to(torch.bfloat16)
+    w1 = torch.randn(1, 6, 16, generator=g).to(torch.bfloat16)
+    s1 = O.router_scores(z, w1)
+    s4 = O.router_scores(z, w1.repeat(4, 1, 1))
+    assert torch.allclose(s1.to(F64), s4.to(F64), rtol=0, atol=1e-7)
+
+
+def test_router_aggregation_is_the_mean():
+    # routers r and -r: sigmoid(a) + sigmoid(-a) = 1, so the mean is 1/2 exactly
+    # (a sum would give 1, a max would give sigmoid(|a|)).
+    g = torch.Generator().manual_seed(5)
+    z = torch.randn(6, 8, generator=g).to(torch.bfloat16)
+    w = torch.randn(1, 5, 8, generator=g).to(torch.bfloat16)
+    s = O.router_scores(z, torch.cat([w, -w]))
+    assert torch.all(s == 0.5)
+    # zero weights: every router says sigmoid(0) = 1/2
+    assert torch.all(O.router_scores(z, torch.zeros(3, 5, 8, dtype=torch.bfloat16)) == 0.5)
+
+
+# --------------------------------------------------------------- selection
+def _valid_topk(sb, sel, k):
+    E = sb.shape[0]
+    S = set(sel)
+    if len(S) != k:
+        return False
+    for i in S:
+        for j in range(E):
+            if j in S:
+                continue
+            if not (sb[i] > sb[j] or (sb[i] == sb[j] and i < j)):
+                return False
+    return True
+
+
+def test_select_brute_force_E16_k2_with_ties():
+    rng = np.random.default_rng(6)
+    E, k = 16, 2
+    # dyadic scores on a coarse grid: many exact ties
+    s = torch.from_numpy(rng.integers(0, 6, size=(200, E)).astype(np.float32) / 8)
+    b = torch.from_numpy(rng.integers(-2, 3, size=E).astype(np.float32) / 16)
+    idx = O.select_topk(s, b, k)
+    sb = (s + b).numpy()
+    for t in range(s.shape[0]):
+        sel = idx[t].tolist()
+        assert _valid_topk(sb[t], sel, k), (t, sel)
+        # maximises the sum over all k-subsets
+        best = max(sum(sb[t][list(c)]) for c in itertools.combinations(range(E), k))
+        assert sum(sb[t][sel]) == best
+        # output order: descending biased score, ties by index
+        keys = [(-sb[t][e], e) for e in sel]
+        assert keys == sorted(keys)
+
+
+def test_select_crafted_ties():
+    E, k = 8, 3
+    # all equal -> the k lowest indices
+    assert O.select_topk(torch.full((1, E), 0.5), torch.zeros(E), k).tolist() == [[0, 1, 2]]
+    # +0 and -0 tie: lower index wins
+    s = torch.tensor([[-0.0, 0.0, -1.0, -1.0, -1.0, -1.0, -1.0, -1.0]])
+    assert O.select_topk(s, torch.zeros(E), 2).tolist() == [[0, 1]]
+    s = torch.tensor([[-1.0, 0.0, -1.0, -0.0, -1.0, -1.0, -1.0, -1.0]])
+    assert O.select_topk(s, torch.zeros(E), 2).tolist() == [[1, 3]]
+    # duplicates straddling the k-th boundary
+    s = torch.tensor([[0.1, 0.9, 0.5, 0.5, 0.5, 0.2, 0.5, 0.0]])
+    assert O.select_topk(s, torch.zeros(E), 3).tolist() == [[1, 2, 3]]
+    # bias breaks a tie the other way
+    b = torch.zeros(E)
+    b[6] = 0.25
+    assert O.select_topk(s, b, 3).tolist() == [[1, 6, 2]]      # 0.9 > 0.75 > 0.5
+
+
+def test_select_bias_zero_and_constant_shift():
+    rng = np.random.default_rng(7)
+    s = torch.from_numpy(rng.integers(0, 64, size=(50, 32)).astype(np.float32) / 64)
+    base = O.select_topk(s, torch.zeros(32), 5)
+    ref = torch.from_numpy(np.argsort(-s.numpy(), axis=1, kind="stable")[:, :5])
+    assert torch.equal(base, ref)
+    # an exactly representable constant shift of b keeps the selection
+    assert torch.equal(O.select_topk(s, torch.full((32,), 0.5), 5), base)
+
+
+# ----------------------------------------------------------------- weights
+def test_route_weights_sum_and_closed_form():
+    s = torch.tensor([[0.75, 0.1, 0.25, 0.0]], dtype=torch.float32)
+    idx = torch.tensor([[0, 2]])
+    w, ws = O.route_weights(s, idx, torch.ones(4))
+    assert w.tolist() == [[0.75, 0.25]] and torch.equal(w, ws)
+    w, ws = O.route_weights(s, idx, torch.tensor([2.0, 1.0, 0.5, 1.0]))
+    assert ws.tolist() == [[1.5, 0.125]]
+    g = torch.Generator().manual_seed(8)
+    s = torch.rand(100, 64, generator=g)
+    idx = O.select_topk(s, torch.zeros(64), 10)
+    w, _ = O.route_weights(s, idx, torch.ones(64))
+    assert torch.all((w.sum(1).to(F64) - 1).abs() <= 10 * 2 ** -23)
+    # the denominator is accumulated in slot order in fp32
+    ssel = torch.gather(s, 1, idx).numpy()
+    den = np.float32(0)
+    for j in range(10):
+        den = np.float32(den + ssel[0, j])
+    assert w[0, 3].item() == np.float32(ssel[0, 3] / den)
+
+
+# -------------------------------------------------------------- dispatch
+def test_permutation_golden():
+    g = _gold("permutation_small.json")
+    c, off, perm, inv = O.permutation(torch.tensor(g["topk_idx"]), g["n_experts"])
+    assert c.tolist() == g["counts"] and off.tolist() == g["offsets"]
+    assert perm.tolist() == g["perm"] and inv.tolist() == g["inv_perm"]
+
+
+def test_permutation_invariants():
+    g = torch.Generator().manual_seed(9)
+    T, E, k = 300, 40, 6
+    s = torch.rand(T, E, generator=g)
+    idx = O.select_topk(s, torch.zeros(E), k)
+    c, off, perm, inv = O.permutation(idx, E)
+    assert int(c.sum()) == T * k
+    assert torch.all(off[1:] >= off[:-1]) and int(off[-1]) == T * k
+    assert torch.equal(torch.sort(perm).values, torch.arange(T * k))
+    assert torch.equal(inv[perm], torch.arange(T * k))
+    flat = idx.reshape(-1)
+    for e in range(E):
+        rows = perm[off[e]:off[e + 1]]
+        assert torch.all(flat[rows] == e)
+        tok = rows // k
+        assert torch.all(tok[1:] > tok[:-1])       # ascending tokens, no repeats
+
+
+# ----------------------------------------------------------------- experts
+def test_glu_closed_form_and_operand_roles():
+    z = torch.ones(1, 1, dtype=torch.bfloat16)
+    one = torch.ones(1, 1, dtype=torch.bfloat16)
+    two = torch.full((1, 1), 2.0, dtype=torch.bfloat16)
+    # g=1, u=1: h = bf16(silu(1)) = bf16(0.7310585786...) = 0.73046875; o = h
+    assert O.expert_glu(z, one, one, one).item() == 0.73046875
+    # g=1,u=2 vs g=2,u=1 differ: silu(1)*2 = 1.4621 -> 1.4609375 ; silu(2) = 1.7616 -> 1.7578125
+    assert O.expert_glu(z, one, two, one).item() == 1.4609375
+    assert O.expert_glu(z, two, one, one).item() == 1.7578125
+    # g = 0 -> h = 0 regardless of u
+    assert O.expert_glu(z, torch.zeros(1, 1, dtype=torch.bfloat16), two, one).item() == 0.0
+
+
+def _tiny_layer(seed=0, T=24):
+    s = W.CONFIGS["c0_tiny"].with_T(T)
+    w = W.make_weights(s, "cpu", seed=seed)
+    x = W.make_x(s, "cpu", seed=seed)
+    return s, w, x
+
+
+def test_sparse_dispatch_equals_dense_brute_force():
+    s, w, x = _tiny_layer()
+    b = torch.zeros(s.n_experts)
+    r = O.forward(x, w, b, s.top_k, s.rms_eps)
+    # dense: every expert on every token, masked by the routing weights
+    z = r.z
+    T, E = z.shape[0], s.n_experts
+    mask = torch.zeros(T, E, dtype=F64)
+    _, ws = O.route_weights(r.s, r.topk_idx, w["expert_scale"])
+    for t in range(T):
+        for j in range(s.top_k):
+            mask[t, r.topk_idx[t, j]] = ws[t, j].double()
+    c = torch.zeros(T, s.d_lat, dtype=F64)
+    for t in range(T):
+        zt = z[t:t + 1]
+        for e in range(E):
+            o = O.expert_glu(zt, w["w_gate"][e], w["w_up_e"][e], w["w_down_e"][e])
+            c[t] += mask[t, e] * o[0]
+        c[t] += O.expert_glu(zt, w["w_sh_gate"], w["w_sh_up"], w["w_sh_down"])[0]
+    assert torch.allclose(c, r.c, rtol=1e-12, atol=1e-12)
+
+
+def test_identical_experts_make_output_routing_independent():
+    s, w, x = _tiny_layer(T=16)
+    for nm in ("w_gate", "w_up_e", "w_down_e"):
+        w[nm] = w[nm][:1].repeat(s.n_experts, 1, 1)
+    w["expert_scale"] = torch.full((s.n_experts,), 0.75)
+    r0 = O.forward(x, w, torch.zeros(s.n_experts), s.top_k)
+    b = torch.linspace(-1, 1, s.n_experts)            # changes the selection
+    r1 = O.forward(x, w, b, s.top_k)
+    assert not torch.equal(r0.topk_idx, r1.topk_idx)
+    assert torch.allclose(r0.c, r1.c, rtol=1e-6, atol=1e-7)
+
+
+def test_shared_expert_always_on():
+    # zero routed experts: the output is RMSNorm(shared expert) -> up-proj
+    s, w, x = _tiny_layer(T=8)
+    for nm in ("w_gate", "w_up_e", "w_down_e"):
+        w[nm] = torch.zeros_like(w[nm])
+    r = O.forward(x, w, torch.zeros(s.n_experts), s.top_k)
+    sh = O.expert_glu(r.z, w["w_sh_gate"], w["w_sh_up"], w["w_sh_down"])
+    assert torch.allclose(r.c, sh, rtol=0, atol=0)
+
+
+# ------------------------------------------------------------------- norm
+def test_rmsnorm_closed_form_and_scale_invariance():
+    L, eps = 16, 1e-6
+    gain = torch.linspace(0.5, 2.0, L)
+    lam = 3.0
+    n = O.rmsnorm(torch.full((1, L), lam, dtype=F64), gain, eps)
+    assert torch.allclose(n[0], gain.to(F64) * lam / math.sqrt(lam * lam + eps), rtol=1e-15)
+    c = torch.randn(4, L, dtype=F64)
+    assert torch.allclose(O.rmsnorm(c * 7.0, gain, 0.0), O.rmsnorm(c, gain, 0.0), rtol=1e-13)
+    assert torch.allclose(O.rmsnorm(-c, gain, eps), -O.rmsnorm(c, gain, eps), rtol=0)
+
+
+# ------------------------------------------------------------ bias update
+def test_bias_update_golden_and_uniform():
+    g = _gold("bias_update_small.json")
+    out = O.bias_update(torch.tensor(g["bias_in"]), torch.tensor(g["counts"]), g["T"],
+                        g["top_k"], g["gamma"])
+    assert out.tolist() == g["bias_out"]
+    b = torch.randn(32)
+    assert torch.equal(O.bias_update(b, torch.full((32,), 5), 16, 10, 1e-3), b)
+
+
+# -------------------------------------------------------------------- FP8
+def test_e4m3_decode_known_values_and_roundtrip():
+    dec = O.e4m3_decode(torch.arange(256))
+    assert dec[0x38].item() == 1.0 and dec[0x7E].item() == 448.0
+    assert dec[0x08].item() == 2.0 ** -6 and dec[0x01].item() == 2.0 ** -9
+    assert dec[0xB8].item() == -1.0 and math.isnan(dec[0x7F].item())
+    ok = ~torch.isnan(dec)
+    codes = O.e4m3_encode(dec[ok])
+    assert torch.equal(codes.to(torch.int64), torch.arange(256)[ok])
+
+
+def test_e4m3_encode_matches_library_in_range_and_saturates():
+    g = torch.Generator().manual_seed(10)
+    v = (torch.randn(200000, generator=g) * torch.exp(torch.randn(200000, generator=g) * 3))
+    v = v.clamp(-448, 448).to(torch.float32)
+    lib = v.to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(O.e4m3_encode(v.to(F64)), lib)
+    # midpoints round to even: 1 + 1/16 lies between 1 and 1.125
+    assert O.e4m3_encode(torch.tensor([1.0625], dtype=F64)).item() == 0x38
+    assert O.e4m3_encode(torch.tensor([1.1875], dtype=F64)).item() == 0x3A
+    assert O.e4m3_decode(O.e4m3_encode(torch.tensor([500.0, -1e6], dtype=F64))).tolist() == [448.0, -448.0]
+
+
+def test_quantize_act_block_scaling():
+    g = torch.Generator().manual_seed(11)
+    v = torch.randn(3, 256, generator=g, dtype=F64)
+    v[1, :128] = 0.0
+    q = O.quantize_act_1x128(v)
+    assert torch.all(q[1, :128] == 0)
+    for r in range(3):
+        for b in range(2):
+            blk = v[r, b * 128:(b + 1) * 128].to(torch.float32)
+            amax = blk.abs().max()
+            if amax == 0:
+                continue
+            qb = q[r, b * 128:(b + 1) * 128]
+            j = int(blk.abs().argmax())
+            # the block maximum maps to code 448 exactly: deq = 448 * fp32(amax/448)
+            sc = (amax / torch.tensor(448.0)).item()
+            assert abs(qb[j].item()) == 448.0 * sc
+            # relative error of e4m3 rounding: at most 2^-4 of the block's scale 2^e grid
+            assert torch.all((qb - blk.to(F64)).abs() <= amax.item() / 448 * 2 ** -1 * 32 + 1e-12)
+
+
+def test_weight_dequant_blocks():
+    codes = torch.full((256, 128), 0x38, dtype=torch.uint8)     # all 1.0
+    sc = torch.tensor([[2.0], [0.5]])
+    wd = O.dequantize_weight_128x128(codes, sc)
+    assert torch.all(wd[:128] == 2.0) and torch.all(wd[128:] == 0.5)
+
+
+# ----------------------------------------------------- consistency with pages
+def test_full_width_shapes_consistent_with_page_totals():
+    s = W.CONFIGS["c2_prefill"]
+    routed = 42 * s.n_experts * 3 * s.d_lat * s.d_ff        # 42 MoE layers (all but the first)
+    assert routed <= 280e9                                    # 280B total parameters
+    assert abs(routed / 42 * 2 / 1e9 - 12.88) < 0.01          # ~12.9 GB bf16 per layer
+    assert W.flops_per_token(s) == 318_767_104
+    assert W.flops_per_token(W.CONFIGS["c0_tiny"]) == 434_176
