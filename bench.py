@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Multi-Router Latent MoE layer forward: tokens/s on B200, and its roofline.
+
+One step = one forward of the whole layer (down-projection, routers + top-k,
+dispatch, gate/up + SiLU-GLU, expert down-projection, combine + RMSNorm,
+up-projection) over one batch of T synthetic tokens already in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2_prefill]
+    python bench.py --impl reference ...     # the CPU oracle on a bounded sample
+
+For N > 1 launch with torchrun; every rank runs its own batch on its own GPU
+(weak scaling, no data-path collective) and rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200 (T=8192, full width); % of roofline"
+UNIT = "tokens/s"
+KERNELS_PER_STEP = 11          # launches of this library's kernels per forward
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="c2_prefill")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (small profiling runs)")
+    ap.add_argument("--cpu-sample", type=int, default=24,
+                    help="tokens of the workload the CPU oracle baseline runs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "sparse_moe_layer_mean_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("csrc_hash") != csrc_hash():
+        return None
+    return d.get("dram_bytes_per_launch_full")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.samples = []
+        self.window = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.th = threading.Thread(target=self._read, daemon=True)
+        self.th.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def begin(self):
+        self.window = [time.time(), None]
+
+    def end(self):
+        if self.window:
+            self.window[1] = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        t0, t1 = self.window
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons, power = [], None, set(), []
+        for ts, line in self.samples:
+            if not (t0 - 0.05 <= ts <= t1 + 0.15):
+                continue
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_median": statistics.median(power) if power else None}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def layer_bytes_flops(s, counts):
+    """Algorithmic bytes and FLOPs of one forward (weights of touched experts,
+    the dense weights, x read and y written)."""
+    import workloads as W
+    touched = int((counts > 0).sum())
+    D, L, E, F, R, T = s.d_model, s.d_lat, s.n_experts, s.d_ff, s.n_routers, s.T
+    expert = 3 * F * L * 2
+    byts = (touched + 1) * expert + (L * D + R * E * L + D * L) * 2 + L * 4 + 2 * T * D * 2
+    return byts, W.flops_per_token(s) * T, touched
+
+
+def glu_kernel_bytes(s, touched):
+    """Algorithmic bytes of one gate/up + SiLU-GLU launch: gate and up weights
+    of the touched experts and the shared expert, the dispatched latent rows
+    read once, and h written once."""
+    rows = s.T * s.top_k + s.T
+    return (touched + 1) * 2 * s.d_ff * s.d_lat * 2 + rows * s.d_lat * 2 + rows * s.d_ff * 2
+
+
+def cpu_baseline(s, weights_dev, x_dev, bias_dev, ntok):
+    """The CPU oracle, as it stands, on the first ntok tokens of the batch."""
+    import torch
+    import oracle as O
+    wh = {k: v.cpu() for k, v in weights_dev.items()}
+    xs = x_dev[:ntok].cpu()
+    b = bias_dev.cpu()
+    t0 = time.perf_counter()
+    O.forward(xs, wh, b, s.top_k, s.rms_eps)
+    dt = time.perf_counter() - t0
+    return {"value": ntok / dt, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": f"first {ntok} tokens of the {s.name} batch (fp64 oracle, {dt:.1f} s)"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle timed on the host cores, one bounded
+    sample of the workload per step."""
+    world, rank, local = dist_setup()
+    if rank != 0:
+        return
+    import torch
+    import oracle as O
+    import workloads as W
+    s = W.CONFIGS[args.config]
+    if args.tokens:
+        s = s.with_T(args.tokens)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = {k: v.cpu() for k, v in W.make_weights(s, dev).items()}
+    per_step = 1
+    n = args.warmup + args.steps
+    x = W.make_x(s, dev, T=min(s.T, n * per_step)).cpu()
+    b = W.make_bias(s, "cpu")
+    for i in range(args.warmup):
+        O.forward(x[i:i + 1], w, b, s.top_k, s.rms_eps)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        j = (args.warmup + i) % x.shape[0]
+        O.forward(x[j:j + per_step], w, b, s.top_k, s.rms_eps)
+    dt = time.perf_counter() - t0
+    v = args.steps * per_step / dt
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": s.name, "T": s.T, "sample_tokens_per_step": per_step},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": torch.get_num_threads(),
+                             "kind": "oracle",
+                             "sample": f"{per_step} token of the {s.name} batch per step"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    world, rank, local = dist_setup()
+    import torch
+    import torch.distributed as dist
+
+    import sparse_moe_layer_mean_b200 as M
+    import workloads as W
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    s = W.CONFIGS[args.config]
+    if args.tokens:
+        s = s.with_T(args.tokens)
+    weights = W.make_weights(s, dev)
+    x = W.make_x(s, dev, seed=s.seed + rank)
+    bias = W.make_bias(s, dev)
+    layer = M.MRLMoELayer(s, weights, device=dev)
+    y = torch.empty(s.T, s.d_model, dtype=torch.bfloat16, device=dev)
+    routing = layer.routing_buffers()
+
+    # warm-up (also yields this batch's routing for the byte counts)
+    for _ in range(max(1, args.warmup)):
+        layer(x, bias, y=y, routing=routing)
+    torch.cuda.synchronize()
+    st = layer.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    counts = routing["counts"].cpu()
+    byts, flops, touched = layer_bytes_flops(s, counts)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(M._native.NUM_STAGE_EVENTS)]
+           for _ in range(args.steps)]
+    for row in evs:          # materialise the event handles
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    time.sleep(0.6)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.begin()
+    start.record()
+    for i in range(args.steps):
+        M.mrlmoe_forward_timed(layer.cfg, layer.cw, bias, x, y, None, layer.workspace, layer.ws_bytes,
+                               evs[i])
+    stop.record()
+    torch.cuda.synchronize()
+    clocks.end()
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    clk = clocks.stop()
+    ms = start.elapsed_time(stop)
+    stage_ms = [0.0] * (M._native.NUM_STAGE_EVENTS - 1)
+    for row in evs:
+        for j in range(len(stage_ms)):
+            stage_ms[j] += row[j].elapsed_time(row[j + 1])
+    stage_ms = [v / args.steps for v in stage_ms]
+    if layer.device_status() != 0:
+        raise RuntimeError("device status non-zero after the timed region")
+
+    # e2e: pinned host x -> device, forward, y -> pinned host, every step
+    e2e = None
+    if not args.no_e2e:
+        xh = x.cpu().pin_memory()
+        yh = torch.empty_like(y, device="cpu").pin_memory()
+        xd = torch.empty_like(x)
+        for _ in range(2):
+            xd.copy_(xh, non_blocking=True)
+            layer(xd, bias, y=y)
+            yh.copy_(y, non_blocking=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            xd.copy_(xh, non_blocking=True)
+            layer(xd, bias, y=y)
+            yh.copy_(y, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b)
+        e2e = [e2e_ms, x.numel() * x.element_size(), y.numel() * y.element_size()]
+
+    # max over ranks
+    if world > 1:
+        t = torch.tensor([ms, e2e[0] if e2e else 0.0] + stage_ms, device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t[0].item()
+        if e2e:
+            e2e[0] = t[1].item()
+        stage_ms = t[2:].tolist()
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        glu_ms = stage_ms[M._native.STAGES.index("gate_up_glu")]
+        glu_bytes = glu_kernel_bytes(s, touched)
+        achieved = glu_bytes / (glu_ms * 1e-3) / 1e9
+        step_s = ms / args.steps * 1e-3
+        t_bytes = byts / (peaks["hbm_gbs"] * 1e9)
+        t_flops = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+        workload = s.name
+        line = {
+            "metric": METRIC, "value": world * s.T * args.steps / (ms * 1e-3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": f"{workload}: T={s.T} tokens, d_model {s.d_model} -> d_lat {s.d_lat}, "
+                            f"{s.n_experts} experts top-{s.top_k} + 1 shared, d_ff {s.d_ff}, "
+                            f"R={s.n_routers} routers, bf16",
+                "T": s.T, "parallelism": f"replicas x{world} (expert weights replicated, own batch per GPU)",
+                "l2": "inputs larger than L2 (expert weights streamed every step)",
+                "touched_experts": touched,
+                "layer_roofline": {"bytes": byts, "flops": flops,
+                                   "t_bytes_ms": t_bytes * 1e3, "t_flops_ms": t_flops * 1e3,
+                                   "frac": max(t_bytes, t_flops) / step_s,
+                                   "tensor_frac_of_bf16_peak": flops / step_s / (peaks["bf16_tflops"] * 1e12),
+                                   "peaks": peak_kind},
+                "stage_ms": dict(zip(M._native.STAGES, [round(v, 4) for v in stage_ms])),
+            },
+            "roofline": {"kernel": "gate_up_glu (grouped tcgen05 GEMM, SiLU-GLU epilogue)",
+                         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": profiled_traffic("gate_up_glu", workload),
+                         "algorithmic_bytes": glu_bytes, "peak_kind": f"of {peak_kind}"},
+            "clocks": clk,
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+        }
+        if e2e:
+            line["e2e"] = {"value": world * s.T * args.steps / (e2e[0] * 1e-3), "unit": UNIT,
+                           "h2d_bytes_per_step": e2e[1], "d2h_bytes_per_step": e2e[2]}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(s, weights, x, bias, min(args.cpu_sample, s.T))
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * mrlmoe.h — C ABI of the Multi-Router Latent MoE layer forward pass (sm_100a).
+ *
+ * The layer (ERNIE 5.5 Flash release pages: blog.derekhsu.net "ERNIE-5.5-Flash-Base"
+ * translation, section "多路由潛在 MoE (Multi-Router Latent MoE)"; aitest123.com
+ * "ERNIE-5.5-Flash-Base开源", section "模型结构"; lininn.cn "2800 亿参数的模型，每次只叫醒
+ * 140 亿", section "路由器，不止一个"):
+ *
+ *   z   = x W_down^T                        tokens projected d_model -> d_lat (4096 -> 2048)
+ *   s   = mean_r sigmoid(z W_router[r]^T)   R sigmoid routers on the latent, aggregated
+ *   sel = top-k of (s + bias)               aux-loss-free balancing bias: selection only
+ *   w   = s_sel / sum(s_sel);  w' = w * alpha[e]   renormalised, per-expert learnable scalar
+ *   o_e = (SiLU(z W_gate,e^T) * (z W_up,e^T)) W_down,e^T     latent experts, d_ff = 2048
+ *   c   = sum_j w'_j o_{e_j} + o_shared     one always-on shared expert (weight 1)
+ *   y   = RMSNorm(c; gain, eps) W_up^T      shared up-projection d_lat -> d_model
+ *   bias[e] += gamma * sign(T*k/E - count[e])          balancing-bias update
+ *
+ * The mean aggregation, R, the renormalisation, the lower-index tie rule and
+ * the bias-update rule are this library's readings of pages that fix none of
+ * them.  The printed activation name "SiTU-GLU" is read as SiLU-GLU.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; matrices are
+ *    row-major and weights are stored [out, in] (the reduction dim contiguous).
+ *  - bf16 = IEEE bfloat16 (2 bytes); e4m3 = OCP FP8 E4M3 (1 byte).
+ *  - `stream` is a cudaStream_t (0 = legacy default stream).  Calls only
+ *    enqueue work on it; none synchronises except mrlmoe_get_device_status.
+ *  - Argument problems found on the host return a non-zero status before
+ *    anything is enqueued.  Faults found on the device (a bounded wait that
+ *    gave up, a failed check) are written to a status word inside the
+ *    workspace; read it with mrlmoe_get_device_status.  No kernel traps.
+ *  - The library allocates no device memory: all scratch lives in the
+ *    caller's workspace of mrlmoe_workspace_size() bytes (256-byte aligned).
+ *  - The library keeps no state between calls; two calls that share a
+ *    workspace must be ordered on one stream.
+ */
+#ifndef MRLMOE_H_
+#define MRLMOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MRLMOE_OK = 0,
+  MRLMOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad dims            */
+  MRLMOE_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. dtype)      */
+  MRLMOE_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned  */
+  MRLMOE_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed         */
+  MRLMOE_ERR_TIMEOUT = 5,       /* device: a bounded wait gave up              */
+  MRLMOE_ERR_CHECK = 6          /* device: a consistency check failed          */
+} mrlmoe_status;
+
+typedef enum {
+  MRLMOE_BF16 = 0,              /* bf16 weights and activations, fp32 accumulate */
+  MRLMOE_FP8_E4M3_BLOCK128 = 1  /* e4m3 weights with fp32 scales per 128x128 block,
+                                   activations quantised e4m3 per 1x128 block;
+                                   the routers stay bf16, y is bf16               */
+} mrlmoe_dtype;
+
+/* Layer shape.  Limits checked on the host:
+ *   T >= 1; d_model, d_lat, d_ff multiples of 128; 1 <= n_routers <= 8;
+ *   16 <= n_experts <= 1024 with n_experts a multiple of 16;
+ *   1 <= top_k <= min(n_experts, 16); rms_eps >= 0.                            */
+typedef struct {
+  int T;            /* tokens in this call                                       */
+  int d_model;      /* hidden size (4096 at full width)                          */
+  int d_lat;        /* latent size (2048)                                        */
+  int n_experts;    /* routed experts E (512)                                    */
+  int top_k;        /* experts selected per token k (10)                         */
+  int d_ff;         /* expert intermediate size F (2048)                         */
+  int n_routers;    /* sigmoid routers R (4)                                     */
+  float rms_eps;    /* RMSNorm epsilon (1e-6)                                    */
+  mrlmoe_dtype dtype;
+} mrlmoe_config;
+
+/* Weights: device pointers, caller-owned.  Element type is bf16 in BF16 mode;
+ * in FP8 mode every matrix except w_router is e4m3 and carries a scale array
+ * s_* of fp32 [ceil(out/128), ceil(in/128)] per matrix (per expert for the
+ * routed experts: [E, ...]).                                                   */
+typedef struct {
+  const void *w_down;      /* [d_lat, d_model]                                    */
+  const void *w_router;    /* [R, E, d_lat]   always bf16                         */
+  const void *w_gate;      /* [E, d_ff, d_lat]  routed experts, gate projection    */
+  const void *w_up_e;      /* [E, d_ff, d_lat]  routed experts, up projection      */
+  const void *w_down_e;    /* [E, d_lat, d_ff]  routed experts, down projection    */
+  const void *w_sh_gate;   /* [d_ff, d_lat]     shared expert                      */
+  const void *w_sh_up;     /* [d_ff, d_lat]                                        */
+  const void *w_sh_down;   /* [d_lat, d_ff]                                        */
+  const float *rms_gain;   /* [d_lat] fp32                                         */
+  const void *w_up;        /* [d_model, d_lat]  shared up-projection               */
+  const float *expert_scale; /* alpha [E] fp32                                     */
+  const float *s_down, *s_gate, *s_up_e, *s_down_e,
+              *s_sh_gate, *s_sh_up, *s_sh_down, *s_up;   /* FP8 only, else NULL   */
+} mrlmoe_weights;
+
+/* Routing record.  Every pointer is optional (NULL = keep it in the workspace
+ * only).  Sizes: topk_idx, topk_w, perm, inv_perm: T*k; counts: E;
+ * offsets: E+1; scores: T*E.
+ *   topk_idx[t*k+j] expert of rank j for token t (descending biased score,
+ *                   ties to the lower index);
+ *   topk_w[t*k+j]   normalised weight BEFORE alpha (sums to 1 per token);
+ *   counts[e]       (token, slot) pairs routed to e; offsets = exclusive scan;
+ *   perm[row]       t*k+j of dispatch row `row` (expert-major, tokens ascending);
+ *   inv_perm[t*k+j] its dispatch row;
+ *   scores[t*E+e]   fp32 aggregated router score s (output of mrlmoe_route /
+ *                   mrlmoe_forward when non-NULL; INPUT when scores_in = 1).  */
+typedef struct {
+  int32_t *topk_idx;
+  float   *topk_w;
+  int32_t *counts;
+  int32_t *offsets;
+  int32_t *perm;
+  int32_t *inv_perm;
+  float   *scores;
+} mrlmoe_routing;
+
+/* Bytes of device workspace that mrlmoe_route / mrlmoe_forward need for cfg
+ * (0 if cfg is invalid).  Dominant terms: the dispatched latent rows and
+ * expert activations, (T*k + T) * (d_lat + d_ff) * 2 bytes, and the
+ * per-slot expert outputs T * (k+1) * d_lat * 4 bytes.                       */
+size_t mrlmoe_workspace_size(const mrlmoe_config *cfg);
+
+/* Routing only (projection, routers, aggregation, bias, top-k, weights,
+ * dispatch record).  x: [T, d_model] bf16, unused (may be NULL) when
+ * scores_in != 0, in which case out->scores must hold the fp32 scores s
+ * [T, E] to route from (this mode is bit-exact against a CPU definition).
+ * bias: [E] fp32.  out: the routing record to fill (non-NULL struct).        */
+mrlmoe_status mrlmoe_route(const mrlmoe_config *cfg, const mrlmoe_weights *w,
+                           const float *bias, const void *x, int scores_in,
+                           mrlmoe_routing *out, void *workspace, size_t ws_bytes,
+                           void *stream);
+
+/* The full layer forward: y [T, d_model] bf16 from x [T, d_model] bf16.
+ * route_out may be NULL; otherwise its non-NULL fields receive the routing
+ * record of this call (scores, if non-NULL, are an output here).              */
+mrlmoe_status mrlmoe_forward(const mrlmoe_config *cfg, const mrlmoe_weights *w,
+                             const float *bias, const void *x, void *y,
+                             mrlmoe_routing *route_out, void *workspace,
+                             size_t ws_bytes, void *stream);
+
+/* Same as mrlmoe_forward, and records caller-created CUDA events
+ * (cudaEvent_t, cast to void*) on `stream` at the stage boundaries, so a
+ * caller can time each kernel of the layer without a profiler:
+ *   events[0] before the down-projection      events[5] after the gate/up GEMM
+ *   events[1] after the down-projection       events[6] after the down GEMM
+ *   events[2] after the router + top-k        events[7] after combine + RMSNorm
+ *   events[3] after the dispatch record       events[8] after the up-projection
+ *   events[4] after the row gather
+ * n_events must be MRLMOE_NUM_STAGE_EVENTS.                                  */
+#define MRLMOE_NUM_STAGE_EVENTS 9
+mrlmoe_status mrlmoe_forward_timed(const mrlmoe_config *cfg, const mrlmoe_weights *w,
+                                   const float *bias, const void *x, void *y,
+                                   mrlmoe_routing *route_out, void *workspace,
+                                   size_t ws_bytes, void *stream,
+                                   void *const *events, int n_events);
+
+/* Balancing-bias step, in place: bias[e] += gamma * sgn(T*k - E*counts[e])
+ * (sign taken exactly in 64-bit integers, sign(0) = 0; one fp32 add).
+ * counts: [E] int32 from a routing record of cfg->T tokens.                  */
+mrlmoe_status mrlmoe_bias_update(const mrlmoe_config *cfg, const int32_t *counts,
+                                 float *bias, float gamma, void *stream);
+
+/* One bf16 projection, out[M, N] = bf16(a[M, K] w[N, K]^T) with fp32
+ * accumulation: the layer's down-projection and shared up-projection steps
+ * on their own.  M >= 1; N, K multiples of 128.  No workspace.               */
+mrlmoe_status mrlmoe_linear(const void *a, const void *w, void *out,
+                            int M, int N, int K, void *stream);
+
+/* Synchronises `stream`, then returns the device status word of `workspace`
+ * written by the last call that used it (MRLMOE_OK if none failed).          */
+mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream);
+
+/* Static, human-readable name of a status code.                              */
+const char *mrlmoe_status_string(mrlmoe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MRLMOE_H_ */

@@ -1,0 +1,186 @@
+// gemm_sm100.cuh — persistent, warp-specialised tcgen05 GEMM for sm_100a.
+//
+// D[128 x N] += A[128 x K] * B[N x K]^T, both operands K-major bf16 staged by
+// SWIZZLE_128B TMA tile loads into a STAGES-deep shared-memory ring; the fp32
+// accumulator lives in tensor memory, double-buffered (2 x 256 columns) so the
+// epilogue of one tile overlaps the main loop of the next.
+//
+//   warp 0   : TMA producer (one thread)
+//   warp 1   : TMEM allocator + UMMA issuer (one thread issues, commits)
+//   warps 2-5: epilogue (warp w reads TMEM lanes 32*(w%4) .. +31)
+//
+// A policy class P describes the problem: how many work units there are, what
+// each unit loads per 64-wide K block, the MMA N of each unit, and the
+// epilogue.  A unit may hold several sub-tiles that share one A operand and
+// one epilogue state (the router walks its expert chunks that way).  Units
+// are dealt round-robin over the persistent CTAs.
+//
+// Every wait is bounded (see mbar_wait); on a timeout the CTA raises an abort
+// flag, every role unwinds, TMEM is freed, and the status word records it.
+#pragma once
+#include "common.cuh"
+
+namespace mrl {
+
+constexpr int kGemmThreads = 192;
+constexpr int kAccCols = 256;   // TMEM columns per accumulator buffer
+constexpr int kTmemCols = 512;  // two buffers
+constexpr int kBK = 64;         // bf16 elements per K block (128 bytes = one swizzle row)
+
+struct Unit {
+  int g;     // group (routed expert e < E, or E for the shared expert); 0 for dense
+  int m;     // M tile
+  int n0;    // first N column of the unit
+  int nv;    // valid N columns in the unit
+  int nsub;  // sub-tiles
+};
+
+__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+template <class P>
+struct GemmSmem {
+  static constexpr int kStageBytes = P::kABytes + P::kBBytesMax;
+  static constexpr int kBarOff = P::kStages * kStageBytes;
+  static constexpr int kNumBars = 2 * P::kStages + 4;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kEpiOff = (kMiscOff + 16 + 127) & ~127;
+  static constexpr int kTotal = kEpiOff + P::kEpiSmem + 1024;  // + alignment slack
+};
+
+template <class P>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ typename P::Params p) {
+  using L = GemmSmem<P>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+  uint8_t *epi_smem = smem + L::kEpiOff;
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * P::kStages;
+  const uint32_t accf0 = empty0 + 8 * P::kStages;
+  const uint32_t acce0 = accf0 + 16;
+  const uint32_t stage0 = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint32_t *status = p.status;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P::kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf0 + 8 * a, 1);
+      mbar_init(acce0 + 8 * a, 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nunits = P::num_units(p);
+  const int kblocks = P::k_blocks(p);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      P::prefetch(p);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const Unit U = P::unit(p, u);
+        for (int sub = 0; sub < U.nsub; ++sub) {
+          const uint32_t bytes = P::stage_bytes(p, U, sub);
+          for (int kb = 0; kb < kblocks; ++kb) {
+            if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, status)) goto done;
+            mbar_arrive_expect_tx(full0 + 8 * s, bytes);
+            const uint32_t sa = stage0 + s * L::kStageBytes;
+            P::load(p, U, sub, kb, sa, sa + P::kABytes, full0 + 8 * s);
+            if (++s == P::kStages) { s = 0; ph ^= 1; }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const Unit U = P::unit(p, u);
+        for (int sub = 0; sub < U.nsub; ++sub) {
+          if (!mbar_wait(acce0 + 8 * acc, aph ^ 1, abort_flag, status)) goto done;
+          tc_fence_after();
+          const uint32_t tacc = tmem_base + acc * kAccCols;
+          const uint32_t idesc = P::idesc(p, U, sub);
+          for (int kb = 0; kb < kblocks; ++kb) {
+            if (!mbar_wait(full0 + 8 * s, ph, abort_flag, status)) goto done;
+            tc_fence_after();
+            const uint32_t sa = stage0 + s * L::kStageBytes;
+            const uint32_t sb = sa + P::kABytes;
+#pragma unroll
+            for (int kk = 0; kk < kBK * 2 / P::kUmmaKBytes; ++kk)
+              P::mma(tacc, sdesc_sw128(sa + kk * P::kUmmaKBytes), sdesc_sw128(sb + kk * P::kUmmaKBytes),
+                     idesc, (kb | kk) != 0);
+            umma_commit(empty0 + 8 * s);
+            if (++s == P::kStages) { s = 0; ph ^= 1; }
+          }
+          umma_commit(accf0 + 8 * acc);
+          acc ^= 1;
+          if (acc == 0) aph ^= 1;
+        }
+      }
+    }
+  } else {
+    // epilogue warps 2..5; TMEM lane quarter = warp % 4
+    const int q = warp & 3;
+    const int etid = threadIdx.x - 64;
+    typename P::EpiState st;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const Unit U = P::unit(p, u);
+      for (int sub = 0; sub < U.nsub; ++sub) {
+        const bool ok = mbar_wait(accf0 + 8 * acc, aph, abort_flag, status);
+        // all four warps take the same decision, so none is left at a named barrier
+        if (bar_red_or(1, 128, !ok || *abort_flag)) goto done;
+        tc_fence_after();
+        P::epilogue(p, U, sub, tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16), q, lane,
+                    etid, st, epi_smem);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acce0 + 8 * acc);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace mrl

@@ -1,0 +1,469 @@
+// mrlmoe_api.cu — the C ABI: host-side validation, workspace layout, TMA
+// descriptor set-up and the launch sequence of the layer on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mrlmoe.h"
+#include "policies.cuh"
+#include "routing.cuh"
+
+using namespace mrl;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------ validation
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mrlmoe_status check_config(const mrlmoe_config *c) {
+  if (!c) return MRLMOE_ERR_INVALID_ARG;
+  if (c->T < 1 || c->d_model < 128 || c->d_lat < 128 || c->d_ff < 128) return MRLMOE_ERR_INVALID_ARG;
+  if (c->d_model % 128 || c->d_lat % 128 || c->d_ff % 128) return MRLMOE_ERR_INVALID_ARG;
+  if (c->d_lat > 8192) return MRLMOE_ERR_UNSUPPORTED;
+  if (c->n_experts < 16 || c->n_experts > 1024 || c->n_experts % 16) return MRLMOE_ERR_INVALID_ARG;
+  if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > kTopKMax) return MRLMOE_ERR_INVALID_ARG;
+  if (c->n_routers < 1 || c->n_routers > 8) return MRLMOE_ERR_INVALID_ARG;
+  if (!(c->rms_eps >= 0.f)) return MRLMOE_ERR_INVALID_ARG;
+  if (c->dtype != MRLMOE_BF16 && c->dtype != MRLMOE_FP8_E4M3_BLOCK128) return MRLMOE_ERR_INVALID_ARG;
+  // dispatched rows are addressed with 32-bit indices
+  const long long rows = static_cast<long long>(c->T) * (c->top_k + 1);
+  if (rows * 256 >= (1ll << 31)) return MRLMOE_ERR_UNSUPPORTED;
+  return MRLMOE_OK;
+}
+
+// Router chunk: experts per accumulator so that R * ec <= 256 and ec | E.
+int router_ec(int E, int R) {
+  for (int ec = 256; ec >= 16; ec >>= 1)
+    if (ec * R <= 256 && E % ec == 0) return ec;
+  return 16;
+}
+
+// ------------------------------------------------------------ workspace
+struct Layout {
+  size_t status, topk_idx, topk_w, wscaled, counts, offsets, grp_off, grp_cnt, unit1, unit2, perm, inv, mask,
+      base, zbuf, hbuf, slots, nbuf, total;
+};
+
+Layout layout_of(const mrlmoe_config &c) {
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  };
+  const size_t T = c.T, k = c.top_k, E = c.n_experts, Ld = c.d_lat, F = c.d_ff;
+  const size_t Tk = T * k, nch = (T + kChunk - 1) / kChunk;
+  L.status = take(256);
+  L.topk_idx = take(Tk * 4);
+  L.topk_w = take(Tk * 4);
+  L.wscaled = take(Tk * 4);
+  L.counts = take((E + 2) * 4);
+  L.offsets = take((E + 2) * 4);
+  L.grp_off = take((E + 2) * 4);
+  L.grp_cnt = take((E + 2) * 4);
+  L.unit1 = take((E + 2) * 4);
+  L.unit2 = take((E + 2) * 4);
+  L.perm = take(Tk * 4);
+  L.inv = take(Tk * 4);
+  L.mask = take(nch * E * 4);
+  L.base = take(nch * E * 4);
+  L.zbuf = take((Tk + T) * Ld * 2);
+  L.hbuf = take((Tk + T) * F * 2);
+  L.slots = take(T * (k + 1) * Ld * 4);
+  L.nbuf = take(T * Ld * 2);
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------ CUDA helpers
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [rows, inner] matrix of `esize`-byte elements,
+// box = box_rows x (128 / esize) elements (one 128-byte swizzle row).
+bool make_map(CUtensorMap *m, const void *base, int esize, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * esize};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt = esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Make the device that owns `p` current; reject host/unknown pointers.
+mrlmoe_status bind_device(const void *p, int *sm_count) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return MRLMOE_ERR_CUDA;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return MRLMOE_ERR_INVALID_ARG;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != a.device)
+    if (cudaSetDevice(a.device) != cudaSuccess) return MRLMOE_ERR_CUDA;
+  static int sms[kMaxDevices] = {0};
+  if (a.device < 0 || a.device >= kMaxDevices) return MRLMOE_ERR_UNSUPPORTED;
+  if (!sms[a.device]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, a.device) != cudaSuccess) return MRLMOE_ERR_CUDA;
+    sms[a.device] = n;
+  }
+  *sm_count = sms[a.device];
+  return MRLMOE_OK;
+}
+
+template <class P>
+cudaError_t launch_gemm(const typename P::Params &p, int grid, cudaStream_t st) {
+  static bool configured[kMaxDevices] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         GemmSmem<P>::kTotal);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  gemm_kernel<P><<<grid, kGemmThreads, GemmSmem<P>::kTotal, st>>>(p);
+  return cudaGetLastError();
+}
+
+#define MRL_TRY(expr)                                  \
+  do {                                                 \
+    if ((expr) != cudaSuccess) return MRLMOE_ERR_CUDA; \
+  } while (0)
+
+struct Ptrs {
+  uint32_t *status;
+  int32_t *topk_idx, *counts_e, *offsets_e, *grp_off, *grp_cnt, *unit1, *unit2, *perm, *inv, *base;
+  float *topk_w, *wscaled, *scores, *slots;
+  uint32_t *mask;
+  __nv_bfloat16 *zbuf, *hbuf, *nbuf;
+  int32_t *out_counts, *out_offsets;
+};
+
+Ptrs carve(const mrlmoe_config &c, void *ws, const mrlmoe_routing *r) {
+  const Layout L = layout_of(c);
+  uint8_t *b = static_cast<uint8_t *>(ws);
+  Ptrs P{};
+  P.status = reinterpret_cast<uint32_t *>(b + L.status);
+  P.topk_idx = (r && r->topk_idx) ? r->topk_idx : reinterpret_cast<int32_t *>(b + L.topk_idx);
+  P.topk_w = (r && r->topk_w) ? r->topk_w : reinterpret_cast<float *>(b + L.topk_w);
+  P.wscaled = reinterpret_cast<float *>(b + L.wscaled);
+  P.counts_e = reinterpret_cast<int32_t *>(b + L.counts);
+  P.offsets_e = reinterpret_cast<int32_t *>(b + L.offsets);
+  P.grp_off = reinterpret_cast<int32_t *>(b + L.grp_off);
+  P.grp_cnt = reinterpret_cast<int32_t *>(b + L.grp_cnt);
+  P.unit1 = reinterpret_cast<int32_t *>(b + L.unit1);
+  P.unit2 = reinterpret_cast<int32_t *>(b + L.unit2);
+  P.perm = (r && r->perm) ? r->perm : reinterpret_cast<int32_t *>(b + L.perm);
+  P.inv = (r && r->inv_perm) ? r->inv_perm : reinterpret_cast<int32_t *>(b + L.inv);
+  P.mask = reinterpret_cast<uint32_t *>(b + L.mask);
+  P.base = reinterpret_cast<int32_t *>(b + L.base);
+  P.zbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.zbuf);
+  P.hbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.hbuf);
+  P.slots = reinterpret_cast<float *>(b + L.slots);
+  P.nbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.nbuf);
+  P.scores = r ? r->scores : nullptr;
+  P.out_counts = r ? r->counts : nullptr;
+  P.out_offsets = r ? r->offsets : nullptr;
+  return P;
+}
+
+constexpr int kExpertBN = 256;  // token tile of the grouped GEMMs (GluPolicy/DownPolicy kBN)
+
+// counts -> offsets/group tables -> stable scatter (from topk_idx).
+mrlmoe_status launch_dispatch(const mrlmoe_config &c, const Ptrs &P, cudaStream_t st) {
+  const int T = c.T, E = c.n_experts, k = c.top_k;
+  const int nch = (T + kChunk - 1) / kChunk;
+  const int wpb = 8;
+  expert_mask_kernel<<<(nch + wpb - 1) / wpb, 32 * wpb, wpb * E * sizeof(uint32_t), st>>>(P.topk_idx, T, E, k,
+                                                                                         P.mask, nch);
+  MRL_TRY(cudaGetLastError());
+  expert_colscan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(P.mask, E, nch, P.base, P.counts_e);
+  MRL_TRY(cudaGetLastError());
+  expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, kExpertBN, c.d_ff / 64, c.d_lat / 128, P.grp_off,
+                                            P.grp_cnt, P.unit1, P.unit2, P.out_counts, P.out_offsets);
+  MRL_TRY(cudaGetLastError());
+  expert_scatter_kernel<<<(nch * 32 + 255) / 256, 256, 0, st>>>(P.topk_idx, P.mask, P.base, P.grp_off, T, E, k,
+                                                                 nch, P.perm, P.inv);
+  MRL_TRY(cudaGetLastError());
+  return MRLMOE_OK;
+}
+
+mrlmoe_status check_weights_bf16(const mrlmoe_weights *w, bool need_all) {
+  if (!w || !w->w_router || !w->expert_scale) return MRLMOE_ERR_INVALID_ARG;
+  if (need_all) {
+    const void *ps[] = {w->w_down, w->w_gate, w->w_up_e, w->w_down_e, w->w_sh_gate,
+                        w->w_sh_up, w->w_sh_down, w->rms_gain, w->w_up};
+    for (const void *p : ps)
+      if (!p || !aligned16(p)) return MRLMOE_ERR_INVALID_ARG;
+  }
+  if (!aligned16(w->w_router)) return MRLMOE_ERR_INVALID_ARG;
+  return MRLMOE_OK;
+}
+
+// Routing from x: down-projection into the tail of zbuf, then the fused router.
+mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weights *w, const float *bias,
+                                       const void *x, const Ptrs &P, int sms, cudaStream_t st,
+                                       void *const *ev = nullptr) {
+  const int T = c.T, D = c.d_model, Ld = c.d_lat, E = c.n_experts, R = c.n_routers, k = c.top_k;
+  __nv_bfloat16 *z = P.zbuf + static_cast<size_t>(T) * k * Ld;  // z rows live after the T*k dispatched rows
+  {
+    DensePolicy::Params p{};
+    if (!make_map(&p.ta, x, 2, D, T, 128) || !make_map(&p.tb, w->w_down, 2, D, Ld, DensePolicy::kBN))
+      return MRLMOE_ERR_CUDA;
+    p.out = z;
+    p.ldo = Ld;
+    p.M = T; p.N = Ld; p.K = D;
+    p.m_tiles = (T + 127) / 128;
+    p.n_tiles = (Ld + DensePolicy::kBN - 1) / DensePolicy::kBN;
+    p.status = P.status;
+    MRL_TRY(launch_gemm<DensePolicy>(p, std::min(sms, p.m_tiles * p.n_tiles), st));
+  }
+  if (ev) MRL_TRY(cudaEventRecord(static_cast<cudaEvent_t>(ev[1]), st));
+  {
+    RouterPolicy::Params p{};
+    const int ec = router_ec(E, R);
+    if (!make_map(&p.ta, z, 2, Ld, T, 128) ||
+        !make_map(&p.tb, w->w_router, 2, Ld, static_cast<uint64_t>(R) * E, ec))
+      return MRLMOE_ERR_CUDA;
+    p.bias = bias;
+    p.alpha = w->expert_scale;
+    p.topk_idx = P.topk_idx;
+    p.topk_w = P.topk_w;
+    p.wscaled = P.wscaled;
+    p.scores = P.scores;
+    p.T = T; p.L = Ld; p.E = E; p.R = R; p.ec = ec; p.k = k;
+    p.m_tiles = (T + 127) / 128;
+    p.status = P.status;
+    MRL_TRY(launch_gemm<RouterPolicy>(p, std::min(sms, p.m_tiles), st));
+  }
+  return MRLMOE_OK;
+}
+
+mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, const float *bias, const void *x,
+                           void *y, mrlmoe_routing *route_out, void *workspace, size_t ws_bytes, void *stream,
+                           void *const *ev) {
+  mrlmoe_status s = check_config(cfg);
+  if (s != MRLMOE_OK) return s;
+  if (!bias || !x || !y || !aligned16(x) || !aligned16(y)) return MRLMOE_ERR_INVALID_ARG;
+  if ((s = check_weights_bf16(w, true)) != MRLMOE_OK) return s;
+  if (cfg->dtype != MRLMOE_BF16) return MRLMOE_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
+  if (ws_bytes < layout_of(*cfg).total) return MRLMOE_ERR_WORKSPACE;
+  int sms = 0;
+  if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ptrs P = carve(*cfg, workspace, route_out);
+  const int T = cfg->T, D = cfg->d_model, Ld = cfg->d_lat, F = cfg->d_ff, E = cfg->n_experts, k = cfg->top_k;
+  const int Tk = T * k;
+  MRL_TRY(cudaMemsetAsync(P.status, 0, 4, st));
+  auto mark = [&](int i) -> bool {
+    return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
+  };
+
+  if (!mark(0)) return MRLMOE_ERR_CUDA;
+  if ((s = launch_project_and_route(*cfg, w, bias, x, P, sms, st, ev)) != MRLMOE_OK) return s;
+  if (!mark(2)) return MRLMOE_ERR_CUDA;
+  if ((s = launch_dispatch(*cfg, P, st)) != MRLMOE_OK) return s;
+  if (!mark(3)) return MRLMOE_ERR_CUDA;
+
+  // gather the dispatched latent rows (rows [0, T*k) of zbuf) from z (rows [T*k, T*k+T))
+  {
+    const int row_u4 = Ld * 2 / 16;
+    gather_rows_kernel<<<(Tk * 32 + 255) / 256, 256, 0, st>>>(
+        P.perm, Tk, k, reinterpret_cast<const uint4 *>(P.zbuf + static_cast<size_t>(Tk) * Ld),
+        reinterpret_cast<uint4 *>(P.zbuf), row_u4);
+    MRL_TRY(cudaGetLastError());
+  }
+  if (!mark(4)) return MRLMOE_ERR_CUDA;
+  GroupTable gt1{P.grp_off, P.grp_cnt, P.unit1, E, F / 64};
+  GroupTable gt2{P.grp_off, P.grp_cnt, P.unit2, E, Ld / 128};
+  {
+    GluPolicy::Params p{};
+    if (!make_map(&p.wg, w->w_gate, 2, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !make_map(&p.wu, w->w_up_e, 2, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !make_map(&p.sg, w->w_sh_gate, 2, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 2, Ld, F, 64) ||
+        !make_map(&p.tz, P.zbuf, 2, Ld, static_cast<uint64_t>(Tk) + T, 32))
+      return MRLMOE_ERR_CUDA;
+    p.gt = gt1;
+    p.h = P.hbuf;
+    p.F = F; p.L = Ld;
+    p.status = P.status;
+    MRL_TRY(launch_gemm<GluPolicy>(p, sms, st));
+  }
+  if (!mark(5)) return MRLMOE_ERR_CUDA;
+  {
+    DownPolicy::Params p{};
+    if (!make_map(&p.wd, w->w_down_e, 2, F, static_cast<uint64_t>(E) * Ld, 128) ||
+        !make_map(&p.sd, w->w_sh_down, 2, F, Ld, 128) ||
+        !make_map(&p.th, P.hbuf, 2, F, static_cast<uint64_t>(Tk) + T, 32))
+      return MRLMOE_ERR_CUDA;
+    p.gt = gt2;
+    p.perm = P.perm;
+    p.wscaled = P.wscaled;
+    p.slots = P.slots;
+    p.L = Ld; p.F = F; p.k = k; p.Tk = Tk;
+    p.status = P.status;
+    MRL_TRY(launch_gemm<DownPolicy>(p, sms, st));
+  }
+  if (!mark(6)) return MRLMOE_ERR_CUDA;
+  combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k,
+                                                        cfg->rms_eps,
+                                                        reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf);
+  MRL_TRY(cudaGetLastError());
+  if (!mark(7)) return MRLMOE_ERR_CUDA;
+  {
+    DensePolicy::Params p{};
+    if (!make_map(&p.ta, P.nbuf, 2, Ld, T, 128) || !make_map(&p.tb, w->w_up, 2, Ld, D, DensePolicy::kBN))
+      return MRLMOE_ERR_CUDA;
+    p.out = static_cast<__nv_bfloat16 *>(y);
+    p.ldo = D;
+    p.M = T; p.N = D; p.K = Ld;
+    p.m_tiles = (T + 127) / 128;
+    p.n_tiles = (D + DensePolicy::kBN - 1) / DensePolicy::kBN;
+    p.status = P.status;
+    MRL_TRY(launch_gemm<DensePolicy>(p, std::min(sms, p.m_tiles * p.n_tiles), st));
+  }
+  if (!mark(8)) return MRLMOE_ERR_CUDA;
+  return MRLMOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mrlmoe_workspace_size(const mrlmoe_config *cfg) {
+  if (check_config(cfg) != MRLMOE_OK) return 0;
+  return layout_of(*cfg).total;
+}
+
+const char *mrlmoe_status_string(mrlmoe_status s) {
+  switch (s) {
+    case MRLMOE_OK: return "ok";
+    case MRLMOE_ERR_INVALID_ARG: return "invalid argument";
+    case MRLMOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MRLMOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MRLMOE_ERR_CUDA: return "CUDA runtime error";
+    case MRLMOE_ERR_TIMEOUT: return "device wait timed out";
+    case MRLMOE_ERR_CHECK: return "device consistency check failed";
+  }
+  return "unknown status";
+}
+
+mrlmoe_status mrlmoe_route(const mrlmoe_config *cfg, const mrlmoe_weights *w, const float *bias, const void *x,
+                           int scores_in, mrlmoe_routing *out, void *workspace, size_t ws_bytes, void *stream) {
+  mrlmoe_status s = check_config(cfg);
+  if (s != MRLMOE_OK) return s;
+  if (!out || !bias || !w || !w->expert_scale) return MRLMOE_ERR_INVALID_ARG;
+  if (scores_in) {
+    if (!out->scores) return MRLMOE_ERR_INVALID_ARG;
+  } else {
+    if (!x || !aligned16(x)) return MRLMOE_ERR_INVALID_ARG;
+    if ((s = check_weights_bf16(w, false)) != MRLMOE_OK) return s;
+    if (!w->w_down || !aligned16(w->w_down)) return MRLMOE_ERR_INVALID_ARG;
+    if (cfg->dtype != MRLMOE_BF16) return MRLMOE_ERR_UNSUPPORTED;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
+  if (ws_bytes < layout_of(*cfg).total) return MRLMOE_ERR_WORKSPACE;
+  int sms = 0;
+  if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ptrs P = carve(*cfg, workspace, out);
+  MRL_TRY(cudaMemsetAsync(P.status, 0, 4, st));
+  if (scores_in) {
+    const int warps_per_block = 8;
+    topk_from_scores_kernel<kTopKMax><<<(cfg->T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0,
+                                        st>>>(out->scores, bias, w->expert_scale, cfg->T, cfg->n_experts,
+                                              cfg->top_k, P.topk_idx, P.topk_w, P.wscaled);
+    MRL_TRY(cudaGetLastError());
+  } else {
+    if ((s = launch_project_and_route(*cfg, w, bias, x, P, sms, st)) != MRLMOE_OK) return s;
+  }
+  return launch_dispatch(*cfg, P, st);
+}
+
+mrlmoe_status mrlmoe_forward(const mrlmoe_config *cfg, const mrlmoe_weights *w, const float *bias, const void *x,
+                             void *y, mrlmoe_routing *route_out, void *workspace, size_t ws_bytes, void *stream) {
+  return forward_impl(cfg, w, bias, x, y, route_out, workspace, ws_bytes, stream, nullptr);
+}
+
+mrlmoe_status mrlmoe_forward_timed(const mrlmoe_config *cfg, const mrlmoe_weights *w, const float *bias,
+                                   const void *x, void *y, mrlmoe_routing *route_out, void *workspace,
+                                   size_t ws_bytes, void *stream, void *const *events, int n_events) {
+  if (!events || n_events != MRLMOE_NUM_STAGE_EVENTS) return MRLMOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return MRLMOE_ERR_INVALID_ARG;
+  return forward_impl(cfg, w, bias, x, y, route_out, workspace, ws_bytes, stream, events);
+}
+
+mrlmoe_status mrlmoe_bias_update(const mrlmoe_config *cfg, const int32_t *counts, float *bias, float gamma,
+                                 void *stream) {
+  mrlmoe_status s = check_config(cfg);
+  if (s != MRLMOE_OK) return s;
+  if (!counts || !bias) return MRLMOE_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((s = bind_device(bias, &sms)) != MRLMOE_OK) return s;
+  const int E = cfg->n_experts;
+  bias_update_kernel<<<(E + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      counts, bias, E, static_cast<long long>(cfg->T) * cfg->top_k, gamma);
+  MRL_TRY(cudaGetLastError());
+  return MRLMOE_OK;
+}
+
+mrlmoe_status mrlmoe_linear(const void *a, const void *w, void *out, int M, int N, int K, void *stream) {
+  if (!a || !w || !out || M < 1 || N < 128 || K < 128 || N % 128 || K % 128) return MRLMOE_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return MRLMOE_ERR_INVALID_ARG;
+  int sms = 0;
+  mrlmoe_status s = bind_device(w, &sms);
+  if (s != MRLMOE_OK) return s;
+  DensePolicy::Params p{};
+  if (!make_map(&p.ta, a, 2, K, M, 128) || !make_map(&p.tb, w, 2, K, N, DensePolicy::kBN)) return MRLMOE_ERR_CUDA;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.ldo = N;
+  p.M = M; p.N = N; p.K = K;
+  p.m_tiles = (M + 127) / 128;
+  p.n_tiles = (N + DensePolicy::kBN - 1) / DensePolicy::kBN;
+  p.status = nullptr;
+  MRL_TRY(launch_gemm<DensePolicy>(p, std::min(sms, p.m_tiles * p.n_tiles), static_cast<cudaStream_t>(stream)));
+  return MRLMOE_OK;
+}
+
+mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream) {
+  if (!workspace) return MRLMOE_ERR_WORKSPACE;
+  uint32_t v = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MRL_TRY(cudaStreamSynchronize(st));
+  MRL_TRY(cudaMemcpy(&v, workspace, 4, cudaMemcpyDeviceToHost));
+  if (v == DEV_TIMEOUT) return MRLMOE_ERR_TIMEOUT;
+  if (v == DEV_CHECK) return MRLMOE_ERR_CHECK;
+  return v == 0 ? MRLMOE_OK : MRLMOE_ERR_CHECK;
+}
+
+}  // extern "C"

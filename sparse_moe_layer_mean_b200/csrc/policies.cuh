@@ -1,0 +1,374 @@
+// policies.cuh — the layer's GEMMs expressed as policies of gemm_kernel.
+//
+//  DensePolicy  : out[M,N] = bf16(a[M,K] w[N,K]^T)           (down-/up-projection)
+//  RouterPolicy : per token tile, R sigmoid routers x all experts, fused with
+//                 mean over routers, + bias, running top-k, renormalisation, alpha
+//  GluPolicy    : per (expert, 64-wide d_ff slice, token tile):
+//                 h = bf16(SiLU(z W_gate^T) * (z W_up^T))      (swap-AB: weights on M)
+//  DownPolicy   : per (expert, 128-wide d_lat slice, token tile):
+//                 slot[t, j] = w'_{t,j} * (h W_down^T)          (swap-AB)
+#pragma once
+#include "gemm_sm100.cuh"
+#include "topk.cuh"
+
+namespace mrl {
+
+constexpr int kTopKMax = 16;
+
+__device__ __forceinline__ int round16(int n) { return (n + 15) & ~15; }
+
+// ---------------------------------------------------------------- dense
+struct DensePolicy {
+  static constexpr int kStages = 4;
+  static constexpr int kBN = 256;
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytesMax = kBN * 128;
+  static constexpr int kEpiSmem = 0;
+  static constexpr int kUmmaKBytes = 32;
+  struct Params {
+    CUtensorMap ta;  // a [M, K], box 64 x 128
+    CUtensorMap tb;  // w [N, K], box 64 x 256
+    __nv_bfloat16 *out;
+    long ldo;
+    int M, N, K, m_tiles, n_tiles;
+    uint32_t *status;
+  };
+  struct EpiState {};
+  static __device__ __forceinline__ void prefetch(const Params &p) {
+    prefetch_tmap(&p.ta);
+    prefetch_tmap(&p.tb);
+  }
+  static __device__ __forceinline__ int num_units(const Params &p) { return p.m_tiles * p.n_tiles; }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.K / kBK; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u) {
+    Unit U;
+    U.g = 0;
+    U.m = u / p.n_tiles;
+    U.n0 = (u % p.n_tiles) * kBN;
+    U.nv = min(kBN, p.N - U.n0);
+    U.nsub = 1;
+    return U;
+  }
+  static __device__ __forceinline__ uint32_t stage_bytes(const Params &, const Unit &, int) {
+    return kABytes + kBBytesMax;
+  }
+  static __device__ __forceinline__ void load(const Params &p, const Unit &U, int, int kb, uint32_t sa,
+                                              uint32_t sb, uint32_t bar) {
+    tma_load_2d(sa, &p.ta, bar, kb * kBK, U.m * 128);
+    tma_load_2d(sb, &p.tb, bar, kb * kBK, U.n0);
+  }
+  static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
+    return idesc_bf16(128, round16(U.nv));
+  }
+  static __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    umma_f16(d, a, b, id, acc);
+  }
+  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
+                                                  int lane, int, EpiState &, uint8_t *) {
+    const int row = U.m * 128 + q * 32 + lane;
+    for (int c0 = 0; c0 < U.nv; c0 += 32) {
+      float v[32];
+      tmem_ld32(taddr + c0, v);
+      tmem_ld_wait();
+      if (row < p.M) {
+        uint4 *dst = reinterpret_cast<uint4 *>(p.out + row * p.ldo + U.n0 + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint4 w;
+          w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+          w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+          w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+          w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+          dst[i] = w;
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------- router
+// B tile = R boxes of `ec` router rows (experts [sub*ec, sub*ec+ec) of router r),
+// so accumulator column r*ec + j holds router r's logit for expert sub*ec + j.
+struct RouterPolicy {
+  static constexpr int kStages = 4;
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytesMax = 256 * 128;
+  static constexpr int kEpiSmem = 0;
+  static constexpr int kUmmaKBytes = 32;
+  struct Params {
+    CUtensorMap ta;  // z [T, L], box 64 x 128
+    CUtensorMap tb;  // w_router [R*E, L], box 64 x ec
+    const float *bias, *alpha;
+    int32_t *topk_idx;
+    float *topk_w, *wscaled, *scores;
+    int T, L, E, R, ec, k, m_tiles;
+    uint32_t *status;
+  };
+  struct EpiState {
+    TopK<kTopKMax> tk;
+  };
+  static __device__ __forceinline__ void prefetch(const Params &p) {
+    prefetch_tmap(&p.ta);
+    prefetch_tmap(&p.tb);
+  }
+  static __device__ __forceinline__ int num_units(const Params &p) { return p.m_tiles; }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.L / kBK; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u) {
+    Unit U;
+    U.g = 0;
+    U.m = u;
+    U.n0 = 0;
+    U.nv = p.R * p.ec;
+    U.nsub = p.E / p.ec;
+    return U;
+  }
+  static __device__ __forceinline__ uint32_t stage_bytes(const Params &p, const Unit &, int) {
+    return kABytes + p.R * p.ec * 128;
+  }
+  static __device__ __forceinline__ void load(const Params &p, const Unit &U, int sub, int kb, uint32_t sa,
+                                              uint32_t sb, uint32_t bar) {
+    tma_load_2d(sa, &p.ta, bar, kb * kBK, U.m * 128);
+    for (int r = 0; r < p.R; ++r) tma_load_2d(sb + r * p.ec * 128, &p.tb, bar, kb * kBK, r * p.E + sub * p.ec);
+  }
+  static __device__ __forceinline__ uint32_t idesc(const Params &p, const Unit &, int) {
+    return idesc_bf16(128, p.R * p.ec);
+  }
+  static __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    umma_f16(d, a, b, id, acc);
+  }
+  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int sub, uint32_t taddr, int q,
+                                                  int lane, int, EpiState &st, uint8_t *) {
+    const int t = U.m * 128 + q * 32 + lane;
+    const bool valid = t < p.T;
+    if (sub == 0) st.tk.init();
+    const float invR = 1.0f / static_cast<float>(p.R);
+    for (int j0 = 0; j0 < p.ec; j0 += 16) {
+      float acc[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+      for (int r = 0; r < p.R; ++r) {
+        float v[16];
+        tmem_ld16(taddr + r * p.ec + j0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] += sigmoidf_(v[i]);
+      }
+      const int e0 = sub * p.ec + j0;
+      float s16[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        // mean of the R router scores: (sum) / R; R = 2^n makes this exact scaling
+        s16[i] = (p.R & (p.R - 1)) == 0 ? acc[i] * invR : acc[i] / static_cast<float>(p.R);
+        const float sb = s16[i] + __ldg(p.bias + e0 + i);
+        st.tk.offer(sb, e0 + i, s16[i]);
+      }
+      if (valid && p.scores) {
+        float4 *dst = reinterpret_cast<float4 *>(p.scores + static_cast<size_t>(t) * p.E + e0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_float4(s16[4 * i], s16[4 * i + 1], s16[4 * i + 2], s16[4 * i + 3]);
+      }
+    }
+    if (sub == U.nsub - 1 && valid) {
+      float den = 0.f;
+#pragma unroll
+      for (int j = 0; j < kTopKMax; ++j)
+        if (j < p.k) den = (j == 0) ? st.tk.s[0] : den + st.tk.s[j];
+#pragma unroll
+      for (int j = 0; j < kTopKMax; ++j) {
+        if (j < p.k) {
+          const size_t o = static_cast<size_t>(t) * p.k + j;
+          const float w = st.tk.s[j] / den;
+          p.topk_idx[o] = st.tk.i[j];
+          p.topk_w[o] = w;
+          p.wscaled[o] = w * __ldg(p.alpha + st.tk.i[j]);
+        }
+      }
+    }
+  }
+};
+
+// --------------------------------------------------------- grouped helpers
+// Dispatch groups: g < E routed expert g, g == E the shared expert.  Rows of
+// group g start at grp_off[g] in the dispatched activation buffers and number
+// grp_cnt[g]; unit_off[g] is the exclusive prefix of units per group.
+struct GroupTable {
+  const int32_t *grp_off, *grp_cnt, *unit_off;
+  int E, m_tiles;  // M tiles per group
+};
+
+__device__ __forceinline__ Unit grouped_unit(const GroupTable &gt, int u, int BN) {
+  // largest g with unit_off[g] <= u
+  int lo = 0, hi = gt.E;  // g in [0, E]
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(gt.unit_off + mid) <= u) lo = mid; else hi = mid - 1;
+  }
+  Unit U;
+  U.g = lo;
+  const int local = u - __ldg(gt.unit_off + lo);
+  const int cnt = __ldg(gt.grp_cnt + lo);
+  const int ntiles = (cnt + BN - 1) / BN;
+  U.m = local / ntiles;
+  U.n0 = (local % ntiles) * BN;
+  U.nv = min(BN, cnt - U.n0);
+  U.nsub = 1;
+  return U;
+}
+
+// B operand: the unit's dispatched rows, loaded as 32-row boxes.
+__device__ __forceinline__ void load_rows(const CUtensorMap *tm, const GroupTable &gt, const Unit &U, int kb,
+                                          uint32_t sb, uint32_t bar) {
+  const int row0 = __ldg(gt.grp_off + U.g) + U.n0;
+  const int nb = (U.nv + 31) >> 5;
+  for (int i = 0; i < nb; ++i) tma_load_2d(sb + i * 4096, tm, bar, kb * kBK, row0 + 32 * i);
+}
+
+// --------------------------------------------------------------- gate/up
+struct GluPolicy {
+  static constexpr int kStages = 4;
+  static constexpr int kBN = 256;
+  static constexpr int kABytes = 128 * 128;  // 64 gate rows + 64 up rows
+  static constexpr int kBBytesMax = kBN * 128;
+  static constexpr int kEpiSmem = 4 * 32 * 17 * 4;
+  static constexpr int kUmmaKBytes = 32;
+  struct Params {
+    CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 64
+    CUtensorMap sg, su;  // shared gate/up [F, L], box 64 x 64
+    CUtensorMap tz;      // dispatched z [(T*k+T), L], box 64 x 32
+    GroupTable gt;
+    __nv_bfloat16 *h;    // [(T*k+T), F]
+    int F, L;
+    uint32_t *status;
+  };
+  struct EpiState {};
+  static __device__ __forceinline__ void prefetch(const Params &p) {
+    prefetch_tmap(&p.wg); prefetch_tmap(&p.wu); prefetch_tmap(&p.sg); prefetch_tmap(&p.su);
+    prefetch_tmap(&p.tz);
+  }
+  static __device__ __forceinline__ int num_units(const Params &p) { return __ldg(p.gt.unit_off + p.gt.E + 1); }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.L / kBK; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u) { return grouped_unit(p.gt, u, kBN); }
+  static __device__ __forceinline__ uint32_t stage_bytes(const Params &, const Unit &U, int) {
+    return kABytes + ((U.nv + 31) >> 5) * 4096;
+  }
+  static __device__ __forceinline__ void load(const Params &p, const Unit &U, int, int kb, uint32_t sa,
+                                              uint32_t sb, uint32_t bar) {
+    const bool sh = U.g == p.gt.E;
+    const int row = (sh ? 0 : U.g * p.F) + U.m * 64;
+    tma_load_2d(sa, sh ? &p.sg : &p.wg, bar, kb * kBK, row);
+    tma_load_2d(sa + 64 * 128, sh ? &p.su : &p.wu, bar, kb * kBK, row);
+    load_rows(&p.tz, p.gt, U, kb, sb, bar);
+  }
+  static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
+    return idesc_bf16(128, round16(U.nv));
+  }
+  static __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    umma_f16(d, a, b, id, acc);
+  }
+  // Lanes 0-63 hold gate rows f = m*64 + lane, lanes 64-127 the matching up
+  // rows.  Warp pair (q, q+2) swaps half a chunk through shared memory so each
+  // warp owns complete (g, u) pairs for 16 of the chunk's 32 token columns.
+  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
+                                                  int lane, int, EpiState &, uint8_t *epi) {
+    float *xb = reinterpret_cast<float *>(epi);  // [4][32][17]
+    const bool is_gate = q < 2;
+    const int pair = q & 1;
+    const int f = U.m * 64 + pair * 32 + lane;
+    const size_t row0 = static_cast<size_t>(__ldg(p.gt.grp_off + U.g)) + U.n0;
+    for (int c0 = 0; c0 < U.nv; c0 += 32) {
+      float v[32];
+      tmem_ld32(taddr + c0, v);
+      tmem_ld_wait();
+      // gate warps give away columns 16..31, up warps give away columns 0..15
+      float *mine = xb + (q * 32 + lane) * 17;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) mine[c] = is_gate ? v[16 + c] : v[c];
+      named_bar_sync(2, 128);
+      const float *other = xb + (((q + 2) & 3) * 32 + lane) * 17;
+      const int cbase = c0 + (is_gate ? 0 : 16);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float g = is_gate ? v[c] : other[c];
+        const float u = is_gate ? other[c] : v[16 + c];
+        if (cbase + c < U.nv) p.h[(row0 + cbase + c) * p.F + f] = __float2bfloat16_rn(siluf_(g) * u);
+      }
+      named_bar_sync(2, 128);
+    }
+  }
+};
+
+// ------------------------------------------------------------------ down
+struct DownPolicy {
+  static constexpr int kStages = 4;
+  static constexpr int kBN = 256;
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytesMax = kBN * 128;
+  static constexpr int kEpiSmem = 0;
+  static constexpr int kUmmaKBytes = 32;
+  struct Params {
+    CUtensorMap wd;  // routed down [E*L, F], box 64 x 128
+    CUtensorMap sd;  // shared down [L, F], box 64 x 128
+    CUtensorMap th;  // h [(T*k+T), F], box 64 x 32
+    GroupTable gt;
+    const int32_t *perm;
+    const float *wscaled;
+    float *slots;    // [T, k+1, L]
+    int L, F, k, Tk;
+    uint32_t *status;
+  };
+  struct EpiState {};
+  static __device__ __forceinline__ void prefetch(const Params &p) {
+    prefetch_tmap(&p.wd); prefetch_tmap(&p.sd); prefetch_tmap(&p.th);
+  }
+  static __device__ __forceinline__ int num_units(const Params &p) { return __ldg(p.gt.unit_off + p.gt.E + 1); }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.F / kBK; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u) { return grouped_unit(p.gt, u, kBN); }
+  static __device__ __forceinline__ uint32_t stage_bytes(const Params &, const Unit &U, int) {
+    return kABytes + ((U.nv + 31) >> 5) * 4096;
+  }
+  static __device__ __forceinline__ void load(const Params &p, const Unit &U, int, int kb, uint32_t sa,
+                                              uint32_t sb, uint32_t bar) {
+    const bool sh = U.g == p.gt.E;
+    tma_load_2d(sa, sh ? &p.sd : &p.wd, bar, kb * kBK, (sh ? 0 : U.g * p.L) + U.m * 128);
+    load_rows(&p.th, p.gt, U, kb, sb, bar);
+  }
+  static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
+    return idesc_bf16(128, round16(U.nv));
+  }
+  static __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    umma_f16(d, a, b, id, acc);
+  }
+  // Lane = output dim l; column = token.  For each token column the warp
+  // writes 32 consecutive fp32 of that token's slot row (128 B, coalesced).
+  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
+                                                  int lane, int, EpiState &, uint8_t *) {
+    const int l = U.m * 128 + q * 32 + lane;
+    const bool sh = U.g == p.gt.E;
+    const int row0 = __ldg(p.gt.grp_off + U.g) + U.n0;
+    for (int c0 = 0; c0 < U.nv; c0 += 32) {
+      float v[32];
+      tmem_ld32(taddr + c0, v);
+      tmem_ld_wait();
+      const int nc = min(32, U.nv - c0);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        if (c >= nc) break;
+        const int row = row0 + c0 + c;
+        size_t slot;
+        float wt;
+        if (sh) {
+          slot = static_cast<size_t>(row - p.Tk) * (p.k + 1) + p.k;
+          wt = 1.0f;
+        } else {
+          const int flat = __ldg(p.perm + row);
+          const int t = flat / p.k;
+          slot = static_cast<size_t>(t) * (p.k + 1) + (flat - t * p.k);
+          wt = __ldg(p.wscaled + flat);
+        }
+        p.slots[slot * p.L + l] = v[c] * wt;
+      }
+    }
+  }
+};
+
+}  // namespace mrl

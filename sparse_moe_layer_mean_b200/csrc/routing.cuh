@@ -1,0 +1,283 @@
+// routing.cuh — dispatch-record kernels: top-k from given scores, the
+// per-chunk expert bitmask histogram, the exclusive scans, the stable
+// scatter, the row gather, the fixed-order combine + RMSNorm and the
+// balancing-bias step.  No atomics decide any output order.
+#pragma once
+#include "common.cuh"
+#include "topk.cuh"
+
+namespace mrl {
+
+constexpr int kChunk = 32;  // tokens per histogram chunk (one warp, one bit per token)
+
+// ---------------------------------------------------------------------------
+// Top-k from caller-given fp32 scores s [T, E]: one warp per token.  Lane l
+// keeps the best of experts l, l+32, ... (ascending), then k rounds of a warp
+// arg-max (larger biased score, then lower index) emit the selection in rank
+// order.  sb = s + bias is one fp32 add, as in the CPU definition.
+template <int KMAX>
+__global__ void topk_from_scores_kernel(const float *__restrict__ s, const float *__restrict__ bias,
+                                        const float *__restrict__ alpha, int T, int E, int k,
+                                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                                        float *__restrict__ wscaled) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  TopK<KMAX> tk;
+  tk.init();
+  const float *row = s + static_cast<size_t>(warp) * E;
+  for (int e = lane; e < E; e += 32) {
+    const float sv = __ldg(row + e);
+    tk.offer(sv + __ldg(bias + e), e, sv);
+  }
+  float sel_s[KMAX];
+  int sel_i[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j < k) {
+      float bv = tk.v[0], bs = tk.s[0];
+      int bi = tk.i[0];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (ranks_before(ov, oi, bv, bi)) { bv = ov; bs = os; bi = oi; }
+      }
+      if (tk.i[0] == bi) tk.pop();
+      sel_s[j] = bs;
+      sel_i[j] = bi;
+    }
+  }
+  if (lane == 0) {
+    float den = sel_s[0];
+#pragma unroll
+    for (int j = 1; j < KMAX; ++j)
+      if (j < k) den = den + sel_s[j];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < k) {
+        const size_t o = static_cast<size_t>(warp) * k + j;
+        const float w = sel_s[j] / den;
+        topk_idx[o] = sel_i[j];
+        topk_w[o] = w;
+        wscaled[o] = w * __ldg(alpha + sel_i[j]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Histogram: for chunk c (tokens 32c .. 32c+31) and expert e, mask[c*E + e]
+// has bit i set iff token 32c+i selected e.  One warp per chunk; the warp's
+// table lives in shared memory (E <= 1024 words).
+__global__ void expert_mask_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int k,
+                                   uint32_t *__restrict__ mask, int nchunks) {
+  extern __shared__ uint32_t tab_all[];
+  const int wib = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int c = blockIdx.x * (blockDim.x >> 5) + wib;
+  if (c >= nchunks) return;
+  uint32_t *tab = tab_all + wib * E;
+  for (int e = lane; e < E; e += 32) tab[e] = 0u;
+  __syncwarp();
+  const int t = c * kChunk + lane;
+  if (t < T)
+    for (int j = 0; j < k; ++j) atomicOr(&tab[__ldg(topk_idx + static_cast<size_t>(t) * k + j)], 1u << lane);
+  __syncwarp();
+  uint32_t *dst = mask + static_cast<size_t>(c) * E;
+  for (int e = lane; e < E; e += 32) dst[e] = tab[e];
+}
+
+// Column scan: base[c*E + e] = sum over chunks c' < c of popc(mask[c'*E + e]);
+// counts[e] = total.  Block (32 x 32): lane = expert of a 32-expert group,
+// warp = a contiguous run of chunks.
+__global__ void expert_colscan_kernel(const uint32_t *__restrict__ mask, int E, int nchunks,
+                                      int32_t *__restrict__ base, int32_t *__restrict__ counts) {
+  __shared__ int tot[32][33];
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  const int cpw = (nchunks + 31) / 32;
+  const int c0 = w * cpw, c1 = min(nchunks, c0 + cpw);
+  int sum = 0;
+  if (e < E)
+    for (int c = c0; c < c1; ++c) sum += __popc(__ldg(mask + static_cast<size_t>(c) * E + e));
+  tot[w][lane] = sum;
+  __syncthreads();
+  int run = 0;
+  for (int i = 0; i < w; ++i) run += tot[i][lane];
+  if (e < E) {
+    for (int c = c0; c < c1; ++c) {
+      base[static_cast<size_t>(c) * E + e] = run;
+      run += __popc(__ldg(mask + static_cast<size_t>(c) * E + e));
+    }
+    if (w == 31) counts[e] = run;
+  }
+}
+
+// Block-wide exclusive scan of one int per thread (blockDim.x == 1024).
+__device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int *total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_tot[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int t = warp_tot[lane];
+    int ti = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ti, off);
+      if (lane >= off) ti += y;
+    }
+    warp_tot[lane] = ti - t;  // exclusive prefix of warps
+    if (lane == 31) *total = ti;
+  }
+  __syncthreads();
+  const int r = warp_tot[w] + x - v;
+  __syncthreads();
+  return r;
+}
+
+// Offsets and the grouped-GEMM tables.  Group g < E is routed expert g
+// (rows offsets[g] .. + counts[g]); group E is the shared expert over all T
+// tokens, whose rows start at T*k.  unit_off{1,2}[g] = exclusive prefix of
+// m_tiles{1,2} * ceil(cnt_g / BN).  Single block of 1024 threads (E <= 1024).
+__global__ void expert_offsets_kernel(const int32_t *__restrict__ counts_in, int T, int E, int k, int BN,
+                                      int mt1, int mt2, int32_t *__restrict__ grp_off,
+                                      int32_t *__restrict__ grp_cnt, int32_t *__restrict__ unit1,
+                                      int32_t *__restrict__ unit2, int32_t *__restrict__ out_counts,
+                                      int32_t *__restrict__ out_offsets) {
+  __shared__ int wt[32];
+  __shared__ int tot[3];
+  const int e = threadIdx.x;
+  const int cnt = e < E ? counts_in[e] : 0;
+  const int nt = (cnt + BN - 1) / BN;
+  const int off = block_excl_scan(cnt, wt, &tot[0]);
+  const int u1 = block_excl_scan(nt * mt1, wt, &tot[1]);
+  const int u2 = block_excl_scan(nt * mt2, wt, &tot[2]);
+  if (e < E) {
+    grp_off[e] = off;
+    grp_cnt[e] = cnt;
+    unit1[e] = u1;
+    unit2[e] = u2;
+    if (out_counts) out_counts[e] = cnt;
+    if (out_offsets) out_offsets[e] = off;
+  }
+  if (e == 0) {
+    const int ntS = (T + BN - 1) / BN;
+    grp_off[E] = T * k;
+    grp_cnt[E] = T;
+    grp_off[E + 1] = T * k + T;
+    grp_cnt[E + 1] = 0;
+    unit1[E] = tot[1];
+    unit2[E] = tot[2];
+    unit1[E + 1] = tot[1] + ntS * mt1;
+    unit2[E + 1] = tot[2] + ntS * mt2;
+    if (out_offsets) out_offsets[E] = tot[0];
+  }
+}
+
+// Stable scatter: entry (t, j) with expert e goes to row
+// offsets[e] + base[c*E + e] + popc(mask[c*E + e] & lanes below t's lane):
+// expert-major, ascending tokens within an expert.
+__global__ void expert_scatter_kernel(const int32_t *__restrict__ topk_idx, const uint32_t *__restrict__ mask,
+                                      const int32_t *__restrict__ base, const int32_t *__restrict__ offsets,
+                                      int T, int E, int k, int nchunks, int32_t *__restrict__ perm,
+                                      int32_t *__restrict__ inv_perm) {
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (c >= nchunks) return;
+  const int t = c * kChunk + lane;
+  if (t >= T) return;
+  const uint32_t below = (1u << lane) - 1u;
+  for (int j = 0; j < k; ++j) {
+    const int flat = t * k + j;
+    const int e = __ldg(topk_idx + flat);
+    const size_t ce = static_cast<size_t>(c) * E + e;
+    const int row = __ldg(offsets + e) + __ldg(base + ce) + __popc(__ldg(mask + ce) & below);
+    perm[row] = flat;
+    inv_perm[flat] = row;
+  }
+}
+
+// Row gather: zd[row] = zs[perm[row] / k] for row < T*k (one warp per row).
+__global__ void gather_rows_kernel(const int32_t *__restrict__ perm, int rows, int k,
+                                   const uint4 *__restrict__ zs, uint4 *__restrict__ zd, int row_u4) {
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const int t = __ldg(perm + r) / k;
+  const uint4 *src = zs + static_cast<size_t>(t) * row_u4;
+  uint4 *dst = zd + static_cast<size_t>(r) * row_u4;
+  for (int i = lane; i < row_u4; i += 32) dst[i] = __ldg(src + i);
+}
+
+// ---------------------------------------------------------------------------
+// Combine + RMSNorm, one block (256 threads) per token:
+//   c = slot[t,0] + slot[t,1] + ... + slot[t,k-1] + slot[t,k]   (rank order, then shared)
+//   n = bf16(c * (1 / sqrt(mean(c^2) + eps)) * gain)
+// All sums run in a fixed order, so the result is bitwise reproducible.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineMaxV4 = 8;  // d_lat <= 8192
+
+__global__ void __launch_bounds__(kCombineThreads) combine_rmsnorm_kernel(
+    const float4 *__restrict__ slots, int L, int k, float eps, const float4 *__restrict__ gain,
+    __nv_bfloat16 *__restrict__ n) {
+  __shared__ float red[kCombineThreads / 32];
+  const int t = blockIdx.x;
+  const int L4 = L >> 2;
+  const float4 *base = slots + static_cast<size_t>(t) * (k + 1) * L4;
+  float4 c[kCombineMaxV4];
+  float ss = 0.f;
+#pragma unroll
+  for (int v = 0; v < kCombineMaxV4; ++v) {
+    const int i = threadIdx.x + v * kCombineThreads;
+    if (i < L4) {
+      float4 a = __ldg(base + i);
+      for (int j = 1; j <= k; ++j) {
+        const float4 b = __ldg(base + static_cast<size_t>(j) * L4 + i);
+        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+      }
+      c[v] = a;
+      ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCombineThreads / 32; ++w) tot += red[w];
+  const float inv = 1.0f / sqrtf(tot / static_cast<float>(L) + eps);
+  uint2 *dst = reinterpret_cast<uint2 *>(n + static_cast<size_t>(t) * L);
+#pragma unroll
+  for (int v = 0; v < kCombineMaxV4; ++v) {
+    const int i = threadIdx.x + v * kCombineThreads;
+    if (i < L4) {
+      const float4 g = __ldg(gain + i);
+      uint2 o;
+      o.x = pack_bf16x2(c[v].x * inv * g.x, c[v].y * inv * g.y);
+      o.y = pack_bf16x2(c[v].z * inv * g.z, c[v].w * inv * g.w);
+      dst[i] = o;
+    }
+  }
+}
+
+// bias[e] += gamma * sgn(T*k - E*counts[e]) (exact integer sign; sign(0) = 0).
+__global__ void bias_update_kernel(const int32_t *__restrict__ counts, float *__restrict__ bias, int E,
+                                   long long Tk, float gamma) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  const long long d = Tk - static_cast<long long>(E) * counts[e];
+  const float sgn = d > 0 ? 1.0f : (d < 0 ? -1.0f : 0.0f);
+  bias[e] = bias[e] + gamma * sgn;
+}
+
+}  // namespace mrl

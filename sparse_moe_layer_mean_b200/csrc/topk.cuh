@@ -1,0 +1,67 @@
+// topk.cuh — register-resident running top-k with the lower-index tie rule.
+#pragma once
+#include <math.h>
+
+namespace mrl {
+
+// Sorted (descending value) list of the best candidates seen so far.
+// Candidates must be offered in ascending index order: a candidate equal in
+// value to a kept one is placed after it, so ties resolve to the lower index
+// under IEEE equality (+0 == -0).  The list holds the best KMAX candidates
+// offered so far, so its first k (<= KMAX) entries are the top k.
+template <int KMAX>
+struct TopK {
+  float v[KMAX];  // biased score used for selection
+  float s[KMAX];  // unbiased score carried along for the weights
+  int i[KMAX];    // expert index
+  float thr;
+
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      v[j] = -INFINITY;
+      s[j] = 0.f;
+      i[j] = 0x7fffffff;
+    }
+    thr = -INFINITY;
+  }
+
+  __device__ __forceinline__ void offer(float cv, int ci, float cs) {
+    if (cv > thr) {
+      bool take = false;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        take = take || (cv > v[j]);
+        const float tv = v[j], ts = s[j];
+        const int ti = i[j];
+        v[j] = take ? cv : tv;
+        s[j] = take ? cs : ts;
+        i[j] = take ? ci : ti;
+        cv = take ? tv : cv;
+        cs = take ? ts : cs;
+        ci = take ? ti : ci;
+      }
+      // Admission threshold: the KMAX-th best so far.  It is never above the
+      // k-th best, so no candidate that belongs in the top k is turned away.
+      thr = v[KMAX - 1];
+    }
+  }
+
+  // Remove the head (used by the warp merge).
+  __device__ __forceinline__ void pop() {
+#pragma unroll
+    for (int j = 0; j < KMAX - 1; ++j) {
+      v[j] = v[j + 1]; s[j] = s[j + 1]; i[j] = i[j + 1];
+    }
+    v[KMAX - 1] = -INFINITY;
+    s[KMAX - 1] = 0.f;
+    i[KMAX - 1] = 0x7fffffff;
+  }
+};
+
+// (va, ia) ranks before (vb, ib): larger value, or equal value and lower index.
+__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
+  return (va > vb) || (va == vb && ia < ib);
+}
+
+}  // namespace mrl

@@ -1,0 +1,80 @@
+"""Shared helpers for the GPU parity tests: seeded inputs on the device, host
+copies for the oracle, and the parity metrics."""
+from __future__ import annotations
+
+import functools
+
+import torch
+
+import oracle as O
+import workloads as W
+
+# Output bounds for the bf16 layer: max|dy| / max|y_ref| and sum|dy| / sum|y_ref|.
+BF16_MAX_REL = 1e-2
+BF16_MEAN_REL = 2e-3
+# A routing mismatch is legitimate only where the oracle's k-th vs (k+1)-th
+# biased-score gap is below this.
+GAP_TOL = 1e-5
+
+
+def _wkey(name: str) -> str:
+    """Configs with the same layer shape share one set of weights."""
+    s = W.CONFIGS[name]
+    return "c0_tiny" if s.d_model == 256 else "c2_prefill"
+
+
+@functools.lru_cache(maxsize=2)
+def _device_weights(key: str, seed: int):
+    return W.make_weights(W.CONFIGS[key], "cuda", seed=seed)
+
+
+@functools.lru_cache(maxsize=2)
+def _host_weights(key: str, seed: int):
+    return {k: v.cpu() for k, v in _device_weights(key, seed).items()}
+
+
+def device_weights(name: str, seed: int = 0):
+    return _device_weights(_wkey(name), seed)
+
+
+def host_weights(name: str, seed: int = 0):
+    return _host_weights(_wkey(name), seed)
+
+
+def rel_errors(y: torch.Tensor, ref: torch.Tensor):
+    d = (y.double() - ref.double()).abs()
+    r = ref.double().abs()
+    return (d.max() / r.max()).item(), (d.sum() / r.sum()).item()
+
+
+def routing_audit(gpu_idx: torch.Tensor, s_ref: torch.Tensor, bias: torch.Tensor, k: int):
+    """Tokens whose GPU top-k set differs from the oracle's, and the oracle's
+    boundary gap at each of them."""
+    ref_idx = O.select_topk(s_ref, bias.cpu(), k)
+    g = torch.sort(gpu_idx.cpu().long().view(-1, k), dim=1).values
+    r = torch.sort(ref_idx, dim=1).values
+    bad = (g != r).any(dim=1).nonzero().flatten()
+    gaps = O.topk_boundary_gap(s_ref[bad], bias.cpu(), k) if bad.numel() else torch.zeros(0)
+    return bad, gaps, ref_idx
+
+
+def check_dispatch_properties(r, T: int, E: int, k: int):
+    """Invariants of the dispatch record at any size."""
+    idx = r["topk_idx"].cpu().long().view(T, k)
+    counts = r["counts"].cpu().long()
+    offsets = r["offsets"].cpu().long()
+    perm = r["perm"].cpu().long()
+    inv = r["inv_perm"].cpu().long()
+    assert torch.all((idx >= 0) & (idx < E))
+    assert torch.all(torch.sort(idx, dim=1).values[:, 1:] != torch.sort(idx, dim=1).values[:, :-1])
+    assert torch.equal(counts, torch.bincount(idx.flatten(), minlength=E))
+    assert int(counts.sum()) == T * k
+    assert int(offsets[0]) == 0 and torch.equal(offsets[1:], torch.cumsum(counts, 0))
+    assert torch.equal(torch.sort(perm).values, torch.arange(T * k))
+    assert torch.equal(inv[perm], torch.arange(T * k))
+    e_of_row = idx.flatten()[perm]
+    rows_e = torch.repeat_interleave(torch.arange(E), counts)
+    assert torch.equal(e_of_row, rows_e)
+    tok = perm // k
+    same = e_of_row[1:] == e_of_row[:-1]
+    assert torch.all(tok[1:][same] > tok[:-1][same])

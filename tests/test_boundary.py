@@ -1,0 +1,117 @@
+"""The C ABI on the host (no GPU): the library loads, exports every entry
+point include/mrlmoe.h declares, and rejects bad arguments with the
+documented status before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sparse_moe_layer_mean_b200 as M
+from sparse_moe_layer_mean_b200 import _native as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mrlmoe.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mrlmoe_[a-z_]+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = N.lib()
+    names = _declared()
+    assert set(names) == set(N.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", N.LIB_PATH], capture_output=True, text=True).stdout
+    for n in names:
+        assert re.search(rf"\bT {n}\b", out), n
+
+
+def test_status_strings():
+    for code in range(7):
+        assert M.status_string(code)
+    assert M.status_string(99) == "unknown status"
+
+
+def _cfg(**kw):
+    d = dict(T=64, d_model=256, d_lat=128, n_experts=16, top_k=2, d_ff=128, n_routers=2,
+             rms_eps=1e-6, dtype=0)
+    d.update(kw)
+    return N.Config(**d)
+
+
+def test_workspace_size_valid_and_invalid():
+    assert M.mrlmoe_workspace_size(_cfg()) > 0
+    for bad in (dict(T=0), dict(d_model=200), dict(d_lat=0), dict(d_ff=100), dict(n_experts=8),
+                dict(n_experts=24 + 1), dict(top_k=0), dict(top_k=17), dict(top_k=17, n_experts=16),
+                dict(n_routers=0), dict(n_routers=9), dict(rms_eps=-1.0), dict(dtype=7)):
+        assert M.mrlmoe_workspace_size(_cfg(**bad)) == 0, bad
+    # grows with T
+    assert M.mrlmoe_workspace_size(_cfg(T=128)) > M.mrlmoe_workspace_size(_cfg(T=64))
+
+
+def _raw_forward(cfg, w, bias, x, y, ws, nbytes):
+    return N.lib().mrlmoe_forward(ctypes.byref(cfg) if cfg is not None else None,
+                                  ctypes.byref(w) if w is not None else None,
+                                  bias, x, y, None, ws, nbytes, None)
+
+
+def test_forward_rejects_bad_arguments_before_cuda():
+    cfg = _cfg()
+    full = N.Weights(*([4096] * 11 + [None] * 8))   # fake, 16-byte aligned "pointers"
+    need = M.mrlmoe_workspace_size(cfg)
+    assert _raw_forward(None, full, 4096, 4096, 4096, 4096, need) == 1
+    assert _raw_forward(_cfg(T=0), full, 4096, 4096, 4096, 4096, need) == 1
+    assert _raw_forward(cfg, None, 4096, 4096, 4096, 4096, need) == 1
+    assert _raw_forward(cfg, full, None, 4096, 4096, 4096, need) == 1      # bias
+    assert _raw_forward(cfg, full, 4096, None, 4096, 4096, need) == 1      # x
+    assert _raw_forward(cfg, full, 4096, 4104, 4096, 4096, need) == 1      # x misaligned
+    partial = N.Weights(*([4096] * 2 + [None] + [4096] * 8 + [None] * 8))
+    assert _raw_forward(cfg, partial, 4096, 4096, 4096, 4096, need) == 1   # w_gate missing
+    assert _raw_forward(cfg, full, 4096, 4096, 4096, None, need) == 3      # no workspace
+    assert _raw_forward(cfg, full, 4096, 4096, 4096, 4096 + 16, need) == 3  # misaligned
+    assert _raw_forward(cfg, full, 4096, 4096, 4096, 4096, need - 1) == 3  # too small
+    assert _raw_forward(_cfg(dtype=1), full, 4096, 4096, 4096, 4096, need) == 2  # FP8 not built yet
+
+
+def test_route_rejects_bad_arguments_before_cuda():
+    cfg = _cfg()
+    w = N.Weights(*([4096] * 11 + [None] * 8))
+    r = N.Routing(*([None] * 7))
+    need = M.mrlmoe_workspace_size(cfg)
+    L = N.lib()
+    # scores_in without scores
+    assert L.mrlmoe_route(ctypes.byref(cfg), ctypes.byref(w), 4096, None, 1, ctypes.byref(r), 4096,
+                          need, None) == 1
+    # routing from x without x
+    assert L.mrlmoe_route(ctypes.byref(cfg), ctypes.byref(w), 4096, None, 0, ctypes.byref(r), 4096,
+                          need, None) == 1
+    # no routing struct
+    assert L.mrlmoe_route(ctypes.byref(cfg), ctypes.byref(w), 4096, 4096, 0, None, 4096, need, None) == 1
+    r2 = N.Routing(*([None] * 6 + [4096]))
+    assert L.mrlmoe_route(ctypes.byref(cfg), ctypes.byref(w), 4096, None, 1, ctypes.byref(r2), 4096,
+                          need - 256, None) == 3
+
+
+def test_bias_update_and_linear_reject_bad_arguments():
+    L = N.lib()
+    cfg = _cfg()
+    assert L.mrlmoe_bias_update(ctypes.byref(cfg), None, 4096, 1e-3, None) == 1
+    assert L.mrlmoe_bias_update(ctypes.byref(cfg), 4096, None, 1e-3, None) == 1
+    assert L.mrlmoe_bias_update(None, 4096, 4096, 1e-3, None) == 1
+    assert L.mrlmoe_linear(4096, 4096, 4096, 0, 128, 128, None) == 1
+    assert L.mrlmoe_linear(4096, 4096, 4096, 8, 100, 128, None) == 1
+    assert L.mrlmoe_linear(4096, 4096, 4096, 8, 128, 64, None) == 1
+    assert L.mrlmoe_linear(None, 4096, 4096, 8, 128, 128, None) == 1
+    assert L.mrlmoe_linear(4096 + 2, 4096, 4096, 8, 128, 128, None) == 1
+
+
+def test_python_binding_raises_on_error():
+    with pytest.raises(M.MrlmoeError) as ei:
+        M.mrlmoe_linear(0, 0, 0, 8, 128, 128, stream=0)
+    assert ei.value.code == 1

@@ -1,0 +1,185 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle."""
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+import sparse_moe_layer_mean_b200 as M
+from helpers import (BF16_MAX_REL, BF16_MEAN_REL, GAP_TOL, check_dispatch_properties,
+                     device_weights, host_weights, rel_errors, routing_audit)
+
+pytestmark = pytest.mark.gpu
+
+
+def _require_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    _require_gpu()
+    yield
+
+
+# ------------------------------------------------------------------ linear
+@pytest.mark.parametrize("M_,N_,K_", [(1, 128, 128), (127, 256, 256), (129, 384, 640),
+                                      (300, 2048, 4096), (1000, 4096, 2048)])
+def test_linear_matches_oracle(M_, N_, K_):
+    a = W.normal((M_, K_), 7, 100, "cuda")
+    w = W.normal((N_, K_), 7, 101, "cuda", std=K_ ** -0.5)
+    out = torch.empty(M_, N_, dtype=torch.bfloat16, device="cuda")
+    M.mrlmoe_linear(a, w, out, M_, N_, K_)
+    torch.cuda.synchronize()
+    ref = O.linear_bf16(a.cpu(), w.cpu())
+    d = (out.cpu().double() - ref).abs()
+    # fp32 accumulation vs exact: at most one bf16 step apart
+    assert torch.all(d <= ref.abs() * 2 ** -7 + 1e-30)
+    assert (d.sum() / ref.abs().sum()).item() < 1e-3
+
+
+# ------------------------------------------------- routing: scores given
+def _scores_case(name, T, E, k):
+    if name == "uniform":
+        s = W.uniform((T, E), 0.0, 1.0, 11, 200, "cpu")
+        b = W.uniform((E,), -0.05, 0.05, 11, 201, "cpu")
+    elif name == "dyadic_ties":
+        s = (W.uniform((T, E), 0.0, 8.0, 12, 200, "cpu").floor() / 8).float()
+        b = (W.uniform((E,), -2.0, 2.0, 12, 201, "cpu").floor() / 16).float()
+    elif name == "all_equal":
+        s = torch.full((T, E), 0.5)
+        b = torch.zeros(E)
+    elif name == "signed_zeros":
+        u = W.uniform((T, E), 0.0, 3.0, 13, 200, "cpu").floor()
+        s = torch.where(u == 0, torch.tensor(0.0), torch.where(u == 1, torch.tensor(-0.0), torch.tensor(-1.0)))
+        b = torch.zeros(E)
+    return s.float().contiguous(), b.float().contiguous()
+
+
+@pytest.mark.parametrize("case", ["uniform", "dyadic_ties", "all_equal", "signed_zeros"])
+@pytest.mark.parametrize("T,E,k", [(64, 16, 2), (1, 16, 2), (33, 512, 10), (1000, 512, 10),
+                                   (257, 1024, 16)])
+def test_route_scores_in_bit_exact(case, T, E, k):
+    shape = W.LayerShape("t", T=T, d_model=256, d_lat=128, n_experts=E, top_k=k, d_ff=128, n_routers=1)
+    s, b = _scores_case(case, T, E, k)
+    alpha = W.uniform((E,), 0.5, 1.5, 3, 300, "cpu")
+    dev = "cuda"
+    w = {"w_router": torch.zeros(1, E, 128, dtype=torch.bfloat16, device=dev),
+         "expert_scale": alpha.to(dev)}
+    layer = M.MRLMoELayer(shape, w)
+    r = layer.routing_buffers(scores=False)
+    r["scores"] = s.to(dev).flatten()
+    layer.route(b.to(dev), routing=r, scores_in=True)
+    torch.cuda.synchronize()
+    ref = O.forward(None, {"expert_scale": alpha}, b, k, scores=s)
+    assert torch.equal(r["topk_idx"].cpu().long().view(T, k), ref.topk_idx)
+    assert torch.equal(r["topk_w"].cpu().view(T, k), ref.topk_w)          # bitwise
+    assert torch.equal(r["counts"].cpu().long(), ref.counts)
+    assert torch.equal(r["offsets"].cpu().long(), ref.offsets)
+    assert torch.equal(r["perm"].cpu().long(), ref.perm)
+    assert torch.equal(r["inv_perm"].cpu().long(), ref.inv_perm)
+    assert layer.device_status() == 0
+
+
+# ------------------------------------------------------- full layer, tiny
+def _run_layer(name, T=None, x=None, bias=None, seed=0, scores=True):
+    s = W.CONFIGS[name] if T is None else W.CONFIGS[name].with_T(T)
+    w = device_weights(name, seed)
+    if x is None:
+        x = W.make_x(s, "cuda", seed=seed)
+    if bias is None:
+        bias = torch.zeros(s.n_experts, dtype=torch.float32, device="cuda")
+    layer = M.MRLMoELayer(s, w)
+    r = layer.routing_buffers(scores=scores)
+    y = layer(x, bias, routing=r)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    return s, x, bias, y, r, layer
+
+
+def _compare_layer(s, x, bias, y, r, wh, tokens=None):
+    """Oracle on the given tokens; output parity on tokens routed alike."""
+    xs = x.cpu() if tokens is None else x.cpu()[tokens]
+    ref = O.forward(xs, wh, bias.cpu(), s.top_k, s.rms_eps)
+    gidx = r["topk_idx"].view(-1, s.top_k)
+    if tokens is not None:
+        gidx = gidx[tokens.to(gidx.device)]
+    bad, gaps, _ = routing_audit(gidx, ref.s, bias, s.top_k)
+    assert torch.all(gaps < GAP_TOL), (bad, gaps)
+    keep = torch.ones(xs.shape[0], dtype=torch.bool)
+    keep[bad] = False
+    yg = y.cpu() if tokens is None else y.cpu()[tokens]
+    mx, mean = rel_errors(yg[keep], ref.y[keep])
+    assert mx <= BF16_MAX_REL and mean <= BF16_MEAN_REL, (mx, mean)
+    if "scores" in r:
+        sg = r["scores"].view(-1, s.n_experts).cpu()
+        if tokens is not None:
+            sg = sg[tokens]
+        assert (sg.double() - ref.s.double()).abs().max().item() < 2e-6
+    return ref, bad
+
+
+def test_forward_c0_tiny():
+    s, x, bias, y, r, _ = _run_layer("c0_tiny")
+    ref, bad = _compare_layer(s, x, bias, y, r, host_weights("c0_tiny"))
+    assert bad.numel() == 0
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+    assert torch.equal(r["counts"].cpu().long(), ref.counts)
+    assert torch.equal(r["perm"].cpu().long(), ref.perm)
+    g = r["topk_w"].view(-1, s.top_k).cpu().double()
+    assert (g - ref.topk_w.double()).abs().max().item() < 1e-6
+
+
+@pytest.mark.parametrize("T", [1, 31, 200])
+def test_forward_c0_ragged_T(T):
+    s, x, bias, y, r, _ = _run_layer("c0_tiny", T=T)
+    _compare_layer(s, x, bias, y, r, host_weights("c0_tiny"))
+
+
+def test_forward_c0_with_bias():
+    s = W.CONFIGS["c0_tiny"]
+    bias = W.uniform((s.n_experts,), -0.1, 0.1, 5, 400, "cuda")
+    s, x, bias, y, r, _ = _run_layer("c0_tiny", bias=bias)
+    _compare_layer(s, x, bias, y, r, host_weights("c0_tiny"))
+
+
+def test_forward_deterministic():
+    s, x, bias, y1, r1, layer = _run_layer("c0_tiny", T=200)
+    y2 = layer(x, bias)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+# -------------------------------------------------- full layer, full width
+def test_forward_full_width_ragged():
+    s, x, bias, y, r, _ = _run_layer("c2_prefill", T=300)
+    _compare_layer(s, x, bias, y, r, host_weights("c2_prefill"))
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+
+
+def test_forward_c2_sampled_tokens():
+    s, x, bias, y, r, _ = _run_layer("c2_prefill")
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+    tokens = torch.tensor([0, 1, 127, 128, 1000, 4095, 4096, 8191])
+    _compare_layer(s, x, bias, y, r, host_weights("c2_prefill"), tokens=tokens)
+
+
+def test_forward_c1_decode():
+    s, x, bias, y, r, _ = _run_layer("c1_decode")
+    _compare_layer(s, x, bias, y, r, host_weights("c2_prefill"))
+
+
+# ---------------------------------------------------------------- bias
+def test_bias_update_bit_exact():
+    shape = W.CONFIGS["c3_skew"]
+    E, T, k = shape.n_experts, shape.T, shape.top_k
+    counts = (W.uniform((E,), 0, 1300, 9, 500, "cpu").floor()).to(torch.int32)
+    counts[:5] = T * k // E                                                   # exact mean load
+    bias = W.uniform((E,), -0.3, 0.3, 9, 501, "cpu")
+    bias[5] = -0.0
+    cfg = M.make_config(shape)
+    b_dev = bias.cuda()
+    M.mrlmoe_bias_update(cfg, counts.cuda(), b_dev, 1e-3)
+    torch.cuda.synchronize()
+    ref = O.bias_update(bias, counts, T, k, 1e-3)
+    assert torch.equal(b_dev.cpu().view(torch.int32), ref.view(torch.int32))
