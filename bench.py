@@ -41,6 +41,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="c2_prefill")
     ap.add_argument("--tokens", type=int, default=None, help="override T (small profiling runs)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override the routed expert count (small profiling runs only)")
     ap.add_argument("--cpu-sample", type=int, default=24,
                     help="tokens of the workload the CPU oracle baseline runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -147,6 +149,17 @@ def dist_setup():
     return world, rank, local
 
 
+def shape_from_args(args):
+    import dataclasses
+    import workloads as W
+    s = W.CONFIGS[args.config]
+    if args.tokens:
+        s = s.with_T(args.tokens)
+    if args.experts:
+        s = dataclasses.replace(s, n_experts=args.experts, name=f"{s.name}_E{args.experts}")
+    return s
+
+
 def layer_bytes_flops(s, counts):
     """Algorithmic bytes and FLOPs of one forward (weights of touched experts,
     the dense weights, x read and y written)."""
@@ -189,9 +202,7 @@ def run_reference(args):
     import torch
     import oracle as O
     import workloads as W
-    s = W.CONFIGS[args.config]
-    if args.tokens:
-        s = s.with_T(args.tokens)
+    s = shape_from_args(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     w = {k: v.cpu() for k, v in W.make_weights(s, dev).items()}
     per_step = 1
@@ -235,9 +246,7 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    s = W.CONFIGS[args.config]
-    if args.tokens:
-        s = s.with_T(args.tokens)
+    s = shape_from_args(args)
     weights = W.make_weights(s, dev)
     x = W.make_x(s, dev, seed=s.seed + rank)
     bias = W.make_bias(s, dev)

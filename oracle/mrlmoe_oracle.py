@@ -33,7 +33,9 @@ the design notes):
   * RMSNorm eps 1e-6 with a learnable gain; no norm after the down-projection;
   * bias update b += gamma * sign(T*k - E*count[e]) with sign(0) = 0;
   * rounding points: z, h, n, y are bf16 (round to nearest even);
-    s, w, and the FP8 quantiser inputs are fp32; everything else fp64.
+    s, w, and the FP8 quantiser inputs are fp32; everything else fp64;
+  * the routers read the latent before its bf16 rounding (the experts read
+    bf16 z), so that top-k decisions do not hinge on bf16 rounding of z.
 PARITY UNPINNED by the pages: the choice of mean (vs sum/max), R=4, eps, gamma.
 Those are stated assumptions; the tests pin only the arithmetic under them.
 """
@@ -310,7 +312,8 @@ def forward(x: torch.Tensor, weights: Dict[str, torch.Tensor], bias: torch.Tenso
     """The layer on CPU, step by step.
 
     1. z = bf16(x W_dn^T)                          down-projection 4096 -> 2048
-    2-3. s = mean_r sigmoid(z W_r^T) (fp32)         multi-router scores
+    2-3. s = mean_r sigmoid(zx W_r^T) (fp32)        multi-router scores, where zx
+         is the unrounded latent x W_dn^T (the routers read it at full precision)
     4-5. top-k of s + b; w = renormalised s; w' = w * alpha
     6. dispatch record (counts, offsets, perm, inv_perm)
     7-9. routed experts on their rows, shared expert on every token
@@ -334,8 +337,9 @@ def forward(x: torch.Tensor, weights: Dict[str, torch.Tensor], bias: torch.Tenso
                                       "w_sh_gate", "w_sh_up", "w_sh_down", "w_up")}
     if scores is None:
         xin = quantize_act_1x128(_as_f64(x)) if fp8 else _as_f64(x)
-        z = bf16_round(xin @ _as_f64(_w(weights, "w_down", deq)).T)
-        s = router_scores(z, weights["w_router"])
+        zx = xin @ _as_f64(_w(weights, "w_down", deq)).T
+        z = bf16_round(zx)
+        s = router_scores(zx, weights["w_router"])
     else:
         z, s = None, scores.to(F32)
     T = s.shape[0]

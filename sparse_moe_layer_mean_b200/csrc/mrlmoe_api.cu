@@ -46,7 +46,7 @@ int router_ec(int E, int R) {
 // ------------------------------------------------------------ workspace
 struct Layout {
   size_t status, topk_idx, topk_w, wscaled, counts, offsets, grp_off, grp_cnt, unit1, unit2, perm, inv, mask,
-      base, zbuf, hbuf, slots, nbuf, total;
+      base, zbuf, zlo, hbuf, slots, nbuf, total;
 };
 
 Layout layout_of(const mrlmoe_config &c) {
@@ -74,6 +74,7 @@ Layout layout_of(const mrlmoe_config &c) {
   L.mask = take(nch * E * 4);
   L.base = take(nch * E * 4);
   L.zbuf = take((Tk + T) * Ld * 2);
+  L.zlo = take(T * Ld * 2);
   L.hbuf = take((Tk + T) * F * 2);
   L.slots = take(T * (k + 1) * Ld * 4);
   L.nbuf = take(T * Ld * 2);
@@ -163,7 +164,7 @@ struct Ptrs {
   int32_t *topk_idx, *counts_e, *offsets_e, *grp_off, *grp_cnt, *unit1, *unit2, *perm, *inv, *base;
   float *topk_w, *wscaled, *scores, *slots;
   uint32_t *mask;
-  __nv_bfloat16 *zbuf, *hbuf, *nbuf;
+  __nv_bfloat16 *zbuf, *zlo, *hbuf, *nbuf;
   int32_t *out_counts, *out_offsets;
 };
 
@@ -186,6 +187,7 @@ Ptrs carve(const mrlmoe_config &c, void *ws, const mrlmoe_routing *r) {
   P.mask = reinterpret_cast<uint32_t *>(b + L.mask);
   P.base = reinterpret_cast<int32_t *>(b + L.base);
   P.zbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.zbuf);
+  P.zlo = reinterpret_cast<__nv_bfloat16 *>(b + L.zlo);
   P.hbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.hbuf);
   P.slots = reinterpret_cast<float *>(b + L.slots);
   P.nbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.nbuf);
@@ -239,6 +241,7 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
     if (!make_map(&p.ta, x, 2, D, T, 128) || !make_map(&p.tb, w->w_down, 2, D, Ld, DensePolicy::kBN))
       return MRLMOE_ERR_CUDA;
     p.out = z;
+    p.out_lo = P.zlo;
     p.ldo = Ld;
     p.M = T; p.N = Ld; p.K = D;
     p.m_tiles = (T + 127) / 128;
@@ -250,7 +253,7 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
   {
     RouterPolicy::Params p{};
     const int ec = router_ec(E, R);
-    if (!make_map(&p.ta, z, 2, Ld, T, 128) ||
+    if (!make_map(&p.ta, z, 2, Ld, T, 128) || !make_map(&p.ta_lo, P.zlo, 2, Ld, T, 128) ||
         !make_map(&p.tb, w->w_router, 2, Ld, static_cast<uint64_t>(R) * E, ec))
       return MRLMOE_ERR_CUDA;
     p.bias = bias;

@@ -29,6 +29,7 @@ struct DensePolicy {
     CUtensorMap ta;  // a [M, K], box 64 x 128
     CUtensorMap tb;  // w [N, K], box 64 x 256
     __nv_bfloat16 *out;
+    __nv_bfloat16 *out_lo;  // optional: bf16(acc - float(out)), the residual of the rounding
     long ldo;
     int M, N, K, m_tiles, n_tiles;
     uint32_t *status;
@@ -81,6 +82,21 @@ struct DensePolicy {
           w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
           dst[i] = w;
         }
+        if (p.out_lo) {
+          // residual of the bf16 rounding: hi + lo carries the fp32 accumulator to ~2^-17
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] -= __bfloat162float(__float2bfloat16_rn(v[i]));
+          uint4 *dlo = reinterpret_cast<uint4 *>(p.out_lo + row * p.ldo + U.n0 + c0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 w;
+            w.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
+            w.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
+            w.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
+            w.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
+            dlo[i] = w;
+          }
+        }
       }
     }
   }
@@ -89,6 +105,9 @@ struct DensePolicy {
 // ---------------------------------------------------------------- router
 // B tile = R boxes of `ec` router rows (experts [sub*ec, sub*ec+ec) of router r),
 // so accumulator column r*ec + j holds router r's logit for expert sub*ec + j.
+// The routers read the latent at the down-projection's fp32 precision: z is
+// given as bf16 hi + bf16 lo parts and the K loop runs over both (2 * d_lat),
+// reusing each router tile for the hi and the lo half.
 struct RouterPolicy {
   static constexpr int kStages = 4;
   static constexpr int kABytes = 128 * 128;
@@ -96,8 +115,9 @@ struct RouterPolicy {
   static constexpr int kEpiSmem = 0;
   static constexpr int kUmmaKBytes = 32;
   struct Params {
-    CUtensorMap ta;  // z [T, L], box 64 x 128
-    CUtensorMap tb;  // w_router [R*E, L], box 64 x ec
+    CUtensorMap ta;     // z hi [T, L], box 64 x 128
+    CUtensorMap ta_lo;  // z lo [T, L], box 64 x 128
+    CUtensorMap tb;     // w_router [R*E, L], box 64 x ec
     const float *bias, *alpha;
     int32_t *topk_idx;
     float *topk_w, *wscaled, *scores;
@@ -109,10 +129,11 @@ struct RouterPolicy {
   };
   static __device__ __forceinline__ void prefetch(const Params &p) {
     prefetch_tmap(&p.ta);
+    prefetch_tmap(&p.ta_lo);
     prefetch_tmap(&p.tb);
   }
   static __device__ __forceinline__ int num_units(const Params &p) { return p.m_tiles; }
-  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.L / kBK; }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return 2 * (p.L / kBK); }
   static __device__ __forceinline__ Unit unit(const Params &p, int u) {
     Unit U;
     U.g = 0;
@@ -127,8 +148,11 @@ struct RouterPolicy {
   }
   static __device__ __forceinline__ void load(const Params &p, const Unit &U, int sub, int kb, uint32_t sa,
                                               uint32_t sb, uint32_t bar) {
-    tma_load_2d(sa, &p.ta, bar, kb * kBK, U.m * 128);
-    for (int r = 0; r < p.R; ++r) tma_load_2d(sb + r * p.ec * 128, &p.tb, bar, kb * kBK, r * p.E + sub * p.ec);
+    const int nk = p.L / kBK;
+    const bool lo = kb >= nk;
+    const int x = (lo ? kb - nk : kb) * kBK;
+    tma_load_2d(sa, lo ? &p.ta_lo : &p.ta, bar, x, U.m * 128);
+    for (int r = 0; r < p.R; ++r) tma_load_2d(sb + r * p.ec * 128, &p.tb, bar, x, r * p.E + sub * p.ec);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &p, const Unit &, int) {
     return idesc_bf16(128, p.R * p.ec);
@@ -303,7 +327,7 @@ struct DownPolicy {
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
-  static constexpr int kEpiSmem = 0;
+  static constexpr int kEpiSmem = kBN * 8;
   static constexpr int kUmmaKBytes = 32;
   struct Params {
     CUtensorMap wd;  // routed down [E*L, F], box 64 x 128
@@ -338,36 +362,41 @@ struct DownPolicy {
   static __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
     umma_f16(d, a, b, id, acc);
   }
-  // Lane = output dim l; column = token.  For each token column the warp
-  // writes 32 consecutive fp32 of that token's slot row (128 B, coalesced).
+  // Lane = output dim l; column = token.  The unit's per-column slot row and
+  // weight are first staged in shared memory (one parallel pass over the
+  // dispatch record), then for each token column the warp writes 32
+  // consecutive fp32 of that token's slot row (128 B, coalesced).
   static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
-                                                  int lane, int, EpiState &, uint8_t *) {
+                                                  int lane, int etid, EpiState &, uint8_t *epi) {
+    int *s_slot = reinterpret_cast<int *>(epi);
+    float *s_wt = reinterpret_cast<float *>(epi + kBN * sizeof(int));
     const int l = U.m * 128 + q * 32 + lane;
     const bool sh = U.g == p.gt.E;
     const int row0 = __ldg(p.gt.grp_off + U.g) + U.n0;
+    for (int c = etid; c < U.nv; c += 128) {
+      const int row = row0 + c;
+      if (sh) {
+        s_slot[c] = (row - p.Tk) * (p.k + 1) + p.k;
+        s_wt[c] = 1.0f;
+      } else {
+        const int flat = __ldg(p.perm + row);
+        const int t = flat / p.k;
+        s_slot[c] = t * (p.k + 1) + (flat - t * p.k);
+        s_wt[c] = __ldg(p.wscaled + flat);
+      }
+    }
+    named_bar_sync(2, 128);
     for (int c0 = 0; c0 < U.nv; c0 += 32) {
       float v[32];
       tmem_ld32(taddr + c0, v);
       tmem_ld_wait();
-      const int nc = min(32, U.nv - c0);
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        if (c >= nc) break;
-        const int row = row0 + c0 + c;
-        size_t slot;
-        float wt;
-        if (sh) {
-          slot = static_cast<size_t>(row - p.Tk) * (p.k + 1) + p.k;
-          wt = 1.0f;
-        } else {
-          const int flat = __ldg(p.perm + row);
-          const int t = flat / p.k;
-          slot = static_cast<size_t>(t) * (p.k + 1) + (flat - t * p.k);
-          wt = __ldg(p.wscaled + flat);
-        }
-        p.slots[slot * p.L + l] = v[c] * wt;
+        if (c0 + c < U.nv)
+          p.slots[static_cast<size_t>(s_slot[c0 + c]) * p.L + l] = v[c] * s_wt[c0 + c];
       }
     }
+    named_bar_sync(2, 128);  // s_slot/s_wt are rewritten by the next unit
   }
 };
 

@@ -33,8 +33,11 @@ def test_linear_matches_oracle(M_, N_, K_):
     torch.cuda.synchronize()
     ref = O.linear_bf16(a.cpu(), w.cpu())
     d = (out.cpu().double() - ref).abs()
-    # fp32 accumulation vs exact: at most one bf16 step apart
-    assert torch.all(d <= ref.abs() * 2 ** -7 + 1e-30)
+    # bf16 output rounding (one step) plus fp32 accumulation error, which is
+    # bounded by the sum of |products|, not by |result|
+    acc = (a.cpu().double().abs() @ w.cpu().double().abs().T) * 2 ** -16
+    bad = d > ref.abs() * 2 ** -7 + acc
+    assert not bool(bad.any()), (int(bad.sum()), d[bad][:5], ref[bad][:5])
     assert (d.sum() / ref.abs().sum()).item() < 1e-3
 
 
@@ -52,6 +55,7 @@ def _scores_case(name, T, E, k):
     elif name == "signed_zeros":
         u = W.uniform((T, E), 0.0, 3.0, 13, 200, "cpu").floor()
         s = torch.where(u == 0, torch.tensor(0.0), torch.where(u == 1, torch.tensor(-0.0), torch.tensor(-1.0)))
+        s[:, E // 2] = 0.75          # a positive selected score keeps the weights finite
         b = torch.zeros(E)
     return s.float().contiguous(), b.float().contiguous()
 
@@ -73,7 +77,7 @@ def test_route_scores_in_bit_exact(case, T, E, k):
     torch.cuda.synchronize()
     ref = O.forward(None, {"expert_scale": alpha}, b, k, scores=s)
     assert torch.equal(r["topk_idx"].cpu().long().view(T, k), ref.topk_idx)
-    assert torch.equal(r["topk_w"].cpu().view(T, k), ref.topk_w)          # bitwise
+    assert torch.equal(r["topk_w"].cpu().view(T, k).view(torch.int32), ref.topk_w.view(torch.int32))
     assert torch.equal(r["counts"].cpu().long(), ref.counts)
     assert torch.equal(r["offsets"].cpu().long(), ref.offsets)
     assert torch.equal(r["perm"].cpu().long(), ref.perm)
@@ -115,7 +119,8 @@ def _compare_layer(s, x, bias, y, r, wh, tokens=None):
         sg = r["scores"].view(-1, s.n_experts).cpu()
         if tokens is not None:
             sg = sg[tokens]
-        assert (sg.double() - ref.s.double()).abs().max().item() < 2e-6
+        # routers read the fp32 latent (bf16 hi + lo): only accumulation-order noise remains
+        assert (sg.double() - ref.s.double()).abs().max().item() < 5e-6
     return ref, bad
 
 
