@@ -29,7 +29,24 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer fwd tokens/s on 1 B200 (T=8192, full width); % of roofline"
 UNIT = "tokens/s"
-KERNELS_PER_STEP = 11          # launches of this library's kernels per forward
+KERNELS_PER_STEP = 11          # launches of this library's kernels per forward (+1 router merge)
+
+
+def kernels_per_step(s, sms: int) -> int:
+    """Kernel launches of one forward: 11, plus the router's merge kernel when
+    the library splits the expert chunks of a token tile over several CTAs
+    (same rule as router_parts in the library)."""
+    ec = 16
+    for c in (256, 128, 64, 32, 16):
+        if c * s.n_routers <= 256 and s.n_experts % c == 0:
+            ec = c
+            break
+    chunks = s.n_experts // ec
+    m_tiles = (s.T + 127) // 128
+    parts = 1
+    while parts * 2 <= chunks and chunks % (parts * 2) == 0 and m_tiles * parts * 2 <= sms:
+        parts *= 2
+    return KERNELS_PER_STEP + (1 if parts > 1 else 0)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -43,7 +60,7 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=None, help="override T (small profiling runs)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override the routed expert count (small profiling runs only)")
-    ap.add_argument("--cpu-sample", type=int, default=24,
+    ap.add_argument("--cpu-sample", type=int, default=256,
                     help="tokens of the workload the CPU oracle baseline runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -365,7 +382,8 @@ def main():
                          "traffic": profiled_traffic("gate_up_glu", workload),
                          "algorithmic_bytes": glu_bytes, "peak_kind": f"of {peak_kind}"},
             "clocks": clk,
-            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "gpu_launches": kernels_per_step(s, torch.cuda.get_device_properties(dev).multi_processor_count)
+            * args.steps,
         }
         if e2e:
             line["e2e"] = {"value": world * s.T * args.steps / (e2e[0] * 1e-3), "unit": UNIT,

@@ -33,6 +33,7 @@ struct Unit {
   int n0;    // first N column of the unit
   int nv;    // valid N columns in the unit
   int nsub;  // sub-tiles
+  int row0;  // grouped GEMMs: first dispatched row of the unit
 };
 
 __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
@@ -55,7 +56,8 @@ struct GemmSmem {
   static constexpr int kNumBars = 2 * P::kStages + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kEpiOff = (kMiscOff + 16 + 127) & ~127;
-  static constexpr int kTotal = kEpiOff + P::kEpiSmem + 1024;  // + alignment slack
+  static constexpr int kAuxOff = (kEpiOff + P::kEpiSmem + 127) & ~127;
+  static constexpr int kTotal = kAuxOff + P::kAuxSmem + 1024;  // + alignment slack
 };
 
 template <class P>
@@ -67,6 +69,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
   uint8_t *epi_smem = smem + L::kEpiOff;
+  uint8_t *aux = smem + L::kAuxOff;  // per-launch tables staged once per CTA
 
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * P::kStages;
@@ -90,6 +93,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     *abort_flag = 0;
     fence_mbar_init();
   }
+  P::stage_aux(p, aux);
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -98,7 +102,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int nunits = P::num_units(p);
+  const int nunits = P::num_units(p, aux);
   const int kblocks = P::k_blocks(p);
 
   if (warp == 0) {
@@ -107,7 +111,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       int s = 0;
       uint32_t ph = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-        const Unit U = P::unit(p, u);
+        const Unit U = P::unit(p, u, aux);
         for (int sub = 0; sub < U.nsub; ++sub) {
           const uint32_t bytes = P::stage_bytes(p, U, sub);
           for (int kb = 0; kb < kblocks; ++kb) {
@@ -125,7 +129,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       int s = 0, acc = 0;
       uint32_t ph = 0, aph = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-        const Unit U = P::unit(p, u);
+        const Unit U = P::unit(p, u, aux);
         for (int sub = 0; sub < U.nsub; ++sub) {
           if (!mbar_wait(acce0 + 8 * acc, aph ^ 1, abort_flag, status)) goto done;
           tc_fence_after();
@@ -157,7 +161,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     int acc = 0;
     uint32_t aph = 0;
     for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-      const Unit U = P::unit(p, u);
+      const Unit U = P::unit(p, u, aux);
       for (int sub = 0; sub < U.nsub; ++sub) {
         const bool ok = mbar_wait(accf0 + 8 * acc, aph, abort_flag, status);
         // all four warps take the same decision, so none is left at a named barrier

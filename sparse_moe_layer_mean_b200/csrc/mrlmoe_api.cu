@@ -43,10 +43,21 @@ int router_ec(int E, int R) {
   return 16;
 }
 
+// Router split: the E/ec expert chunks of a token tile are shared by `parts`
+// CTAs (a power of two dividing the chunk count) so that m_tiles * parts
+// fills the SMs; parts > 1 adds a small merge of the partial selections.
+int router_parts(const mrlmoe_config &c, int sms) {
+  const int chunks = c.n_experts / router_ec(c.n_experts, c.n_routers);
+  const int m_tiles = (c.T + 127) / 128;
+  int parts = 1;
+  while (parts * 2 <= chunks && chunks % (parts * 2) == 0 && m_tiles * parts * 2 <= std::max(sms, 1)) parts *= 2;
+  return parts;
+}
+
 // ------------------------------------------------------------ workspace
 struct Layout {
   size_t status, topk_idx, topk_w, wscaled, counts, offsets, grp_off, grp_cnt, unit1, unit2, perm, inv, mask,
-      base, zbuf, zlo, hbuf, slots, nbuf, total;
+      base, cand_v, cand_s, cand_i, zbuf, zlo, hbuf, slots, nbuf, total;
 };
 
 Layout layout_of(const mrlmoe_config &c) {
@@ -73,6 +84,10 @@ Layout layout_of(const mrlmoe_config &c) {
   L.inv = take(Tk * 4);
   L.mask = take(nch * E * 4);
   L.base = take(nch * E * 4);
+  const size_t parts = router_parts(c, 1 << 30);  // upper bound over SM counts
+  L.cand_v = take(T * parts * k * 4);
+  L.cand_s = take(T * parts * k * 4);
+  L.cand_i = take(T * parts * k * 4);
   L.zbuf = take((Tk + T) * Ld * 2);
   L.zlo = take(T * Ld * 2);
   L.hbuf = take((Tk + T) * F * 2);
@@ -141,6 +156,7 @@ mrlmoe_status bind_device(const void *p, int *sm_count) {
 
 template <class P>
 cudaError_t launch_gemm(const typename P::Params &p, int grid, cudaStream_t st) {
+  static_assert(GemmSmem<P>::kTotal <= 232448, "GEMM shared memory above the 227 KB per-block limit");
   static bool configured[kMaxDevices] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -162,7 +178,8 @@ cudaError_t launch_gemm(const typename P::Params &p, int grid, cudaStream_t st) 
 struct Ptrs {
   uint32_t *status;
   int32_t *topk_idx, *counts_e, *offsets_e, *grp_off, *grp_cnt, *unit1, *unit2, *perm, *inv, *base;
-  float *topk_w, *wscaled, *scores, *slots;
+  float *topk_w, *wscaled, *scores, *slots, *cand_v, *cand_s;
+  int32_t *cand_i;
   uint32_t *mask;
   __nv_bfloat16 *zbuf, *zlo, *hbuf, *nbuf;
   int32_t *out_counts, *out_offsets;
@@ -186,6 +203,9 @@ Ptrs carve(const mrlmoe_config &c, void *ws, const mrlmoe_routing *r) {
   P.inv = (r && r->inv_perm) ? r->inv_perm : reinterpret_cast<int32_t *>(b + L.inv);
   P.mask = reinterpret_cast<uint32_t *>(b + L.mask);
   P.base = reinterpret_cast<int32_t *>(b + L.base);
+  P.cand_v = reinterpret_cast<float *>(b + L.cand_v);
+  P.cand_s = reinterpret_cast<float *>(b + L.cand_s);
+  P.cand_i = reinterpret_cast<int32_t *>(b + L.cand_i);
   P.zbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.zbuf);
   P.zlo = reinterpret_cast<__nv_bfloat16 *>(b + L.zlo);
   P.hbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.hbuf);
@@ -262,10 +282,19 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
     p.topk_w = P.topk_w;
     p.wscaled = P.wscaled;
     p.scores = P.scores;
+    p.cand_v = P.cand_v;
+    p.cand_s = P.cand_s;
+    p.cand_i = P.cand_i;
     p.T = T; p.L = Ld; p.E = E; p.R = R; p.ec = ec; p.k = k;
     p.m_tiles = (T + 127) / 128;
+    p.parts = router_parts(c, sms);
     p.status = P.status;
-    MRL_TRY(launch_gemm<RouterPolicy>(p, std::min(sms, p.m_tiles), st));
+    MRL_TRY(launch_gemm<RouterPolicy>(p, std::min(sms, p.m_tiles * p.parts), st));
+    if (p.parts > 1) {
+      topk_merge_kernel<kTopKMax><<<(T + 127) / 128, 128, 0, st>>>(P.cand_v, P.cand_s, P.cand_i, T, p.parts, k,
+                                                                  w->expert_scale, P.topk_idx, P.topk_w, P.wscaled);
+      MRL_TRY(cudaGetLastError());
+    }
   }
   return MRLMOE_OK;
 }

@@ -24,6 +24,7 @@ struct DensePolicy {
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
   static constexpr int kEpiSmem = 0;
+  static constexpr int kAuxSmem = 0;
   static constexpr int kUmmaKBytes = 32;
   struct Params {
     CUtensorMap ta;  // a [M, K], box 64 x 128
@@ -39,11 +40,13 @@ struct DensePolicy {
     prefetch_tmap(&p.ta);
     prefetch_tmap(&p.tb);
   }
-  static __device__ __forceinline__ int num_units(const Params &p) { return p.m_tiles * p.n_tiles; }
+  static __device__ __forceinline__ void stage_aux(const Params &, uint8_t *) {}
+  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *) { return p.m_tiles * p.n_tiles; }
   static __device__ __forceinline__ int k_blocks(const Params &p) { return p.K / kBK; }
-  static __device__ __forceinline__ Unit unit(const Params &p, int u) {
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *) {
     Unit U;
     U.g = 0;
+    U.row0 = 0;
     U.m = u / p.n_tiles;
     U.n0 = (u % p.n_tiles) * kBN;
     U.nv = min(kBN, p.N - U.n0);
@@ -113,6 +116,7 @@ struct RouterPolicy {
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = 256 * 128;
   static constexpr int kEpiSmem = 0;
+  static constexpr int kAuxSmem = 0;
   static constexpr int kUmmaKBytes = 32;
   struct Params {
     CUtensorMap ta;     // z hi [T, L], box 64 x 128
@@ -121,7 +125,11 @@ struct RouterPolicy {
     const float *bias, *alpha;
     int32_t *topk_idx;
     float *topk_w, *wscaled, *scores;
-    int T, L, E, R, ec, k, m_tiles;
+    // parts > 1: the expert chunks are split over `parts` CTAs per token tile;
+    // each leaves its best k candidates here for topk_merge_kernel
+    float *cand_v, *cand_s;
+    int32_t *cand_i;
+    int T, L, E, R, ec, k, m_tiles, parts;
     uint32_t *status;
   };
   struct EpiState {
@@ -132,15 +140,17 @@ struct RouterPolicy {
     prefetch_tmap(&p.ta_lo);
     prefetch_tmap(&p.tb);
   }
-  static __device__ __forceinline__ int num_units(const Params &p) { return p.m_tiles; }
+  static __device__ __forceinline__ void stage_aux(const Params &, uint8_t *) {}
+  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *) { return p.m_tiles * p.parts; }
   static __device__ __forceinline__ int k_blocks(const Params &p) { return 2 * (p.L / kBK); }
-  static __device__ __forceinline__ Unit unit(const Params &p, int u) {
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *) {
     Unit U;
-    U.g = 0;
-    U.m = u;
+    U.m = u / p.parts;
+    U.g = u - U.m * p.parts;                 // part
+    U.row0 = 0;
     U.n0 = 0;
     U.nv = p.R * p.ec;
-    U.nsub = p.E / p.ec;
+    U.nsub = p.E / p.ec / p.parts;
     return U;
   }
   static __device__ __forceinline__ uint32_t stage_bytes(const Params &p, const Unit &, int) {
@@ -152,7 +162,8 @@ struct RouterPolicy {
     const bool lo = kb >= nk;
     const int x = (lo ? kb - nk : kb) * kBK;
     tma_load_2d(sa, lo ? &p.ta_lo : &p.ta, bar, x, U.m * 128);
-    for (int r = 0; r < p.R; ++r) tma_load_2d(sb + r * p.ec * 128, &p.tb, bar, x, r * p.E + sub * p.ec);
+    const int chunk = U.g * U.nsub + sub;
+    for (int r = 0; r < p.R; ++r) tma_load_2d(sb + r * p.ec * 128, &p.tb, bar, x, r * p.E + chunk * p.ec);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &p, const Unit &, int) {
     return idesc_bf16(128, p.R * p.ec);
@@ -177,7 +188,7 @@ struct RouterPolicy {
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[i] += sigmoidf_(v[i]);
       }
-      const int e0 = sub * p.ec + j0;
+      const int e0 = (U.g * U.nsub + sub) * p.ec + j0;
       float s16[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -193,18 +204,18 @@ struct RouterPolicy {
       }
     }
     if (sub == U.nsub - 1 && valid) {
-      float den = 0.f;
+      if (p.parts == 1) {
+        write_selection<kTopKMax>(st.tk.s, st.tk.i, p.k, static_cast<size_t>(t), p.alpha, p.topk_idx, p.topk_w,
+                                  p.wscaled);
+      } else {
+        const size_t o = (static_cast<size_t>(t) * p.parts + U.g) * p.k;
 #pragma unroll
-      for (int j = 0; j < kTopKMax; ++j)
-        if (j < p.k) den = (j == 0) ? st.tk.s[0] : den + st.tk.s[j];
-#pragma unroll
-      for (int j = 0; j < kTopKMax; ++j) {
-        if (j < p.k) {
-          const size_t o = static_cast<size_t>(t) * p.k + j;
-          const float w = st.tk.s[j] / den;
-          p.topk_idx[o] = st.tk.i[j];
-          p.topk_w[o] = w;
-          p.wscaled[o] = w * __ldg(p.alpha + st.tk.i[j]);
+        for (int j = 0; j < kTopKMax; ++j) {
+          if (j < p.k) {
+            p.cand_v[o + j] = st.tk.v[j];
+            p.cand_s[o + j] = st.tk.s[j];
+            p.cand_i[o + j] = st.tk.i[j];
+          }
         }
       }
     }
@@ -214,37 +225,59 @@ struct RouterPolicy {
 // --------------------------------------------------------- grouped helpers
 // Dispatch groups: g < E routed expert g, g == E the shared expert.  Rows of
 // group g start at grp_off[g] in the dispatched activation buffers and number
-// grp_cnt[g]; unit_off[g] is the exclusive prefix of units per group.
+// grp_cnt[g]; unit_off[g] is the exclusive prefix of units per group
+// (unit_off[E+1] = total).  The three tables (E+2 ints each) are staged in
+// shared memory once per CTA, so mapping a unit to its group costs a short
+// binary search in shared memory instead of dependent global loads.
 struct GroupTable {
   const int32_t *grp_off, *grp_cnt, *unit_off;
   int E, m_tiles;  // M tiles per group
 };
 
-__device__ __forceinline__ Unit grouped_unit(const GroupTable &gt, int u, int BN) {
-  // largest g with unit_off[g] <= u
-  int lo = 0, hi = gt.E;  // g in [0, E]
+constexpr int kMaxGroups = 1024 + 2;
+constexpr int kGroupAuxSmem = 3 * kMaxGroups * 4;
+
+__device__ __forceinline__ void stage_group_table(const GroupTable &gt, uint8_t *aux) {
+  int *s = reinterpret_cast<int *>(aux);
+  const int n = gt.E + 2;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    s[i] = __ldg(gt.unit_off + i);
+    s[kMaxGroups + i] = __ldg(gt.grp_off + i);
+    s[2 * kMaxGroups + i] = __ldg(gt.grp_cnt + i);
+  }
+}
+
+__device__ __forceinline__ int grouped_num_units(const GroupTable &gt, const uint8_t *aux) {
+  return reinterpret_cast<const int *>(aux)[gt.E + 1];
+}
+
+__device__ __forceinline__ Unit grouped_unit(const GroupTable &gt, const uint8_t *aux, int u, int BN) {
+  const int *uo = reinterpret_cast<const int *>(aux);
+  const int *go = uo + kMaxGroups;
+  const int *gc = uo + 2 * kMaxGroups;
+  // largest g in [0, E] with unit_off[g] <= u (zero-unit groups share the next offset)
+  int lo = 0, hi = gt.E;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(gt.unit_off + mid) <= u) lo = mid; else hi = mid - 1;
+    if (uo[mid] <= u) lo = mid; else hi = mid - 1;
   }
   Unit U;
   U.g = lo;
-  const int local = u - __ldg(gt.unit_off + lo);
-  const int cnt = __ldg(gt.grp_cnt + lo);
+  const int local = u - uo[lo];
+  const int cnt = gc[lo];
   const int ntiles = (cnt + BN - 1) / BN;
   U.m = local / ntiles;
-  U.n0 = (local % ntiles) * BN;
+  U.n0 = (local - U.m * ntiles) * BN;
   U.nv = min(BN, cnt - U.n0);
   U.nsub = 1;
+  U.row0 = go[lo] + U.n0;
   return U;
 }
 
 // B operand: the unit's dispatched rows, loaded as 32-row boxes.
-__device__ __forceinline__ void load_rows(const CUtensorMap *tm, const GroupTable &gt, const Unit &U, int kb,
-                                          uint32_t sb, uint32_t bar) {
-  const int row0 = __ldg(gt.grp_off + U.g) + U.n0;
+__device__ __forceinline__ void load_rows(const CUtensorMap *tm, const Unit &U, int kb, uint32_t sb, uint32_t bar) {
   const int nb = (U.nv + 31) >> 5;
-  for (int i = 0; i < nb; ++i) tma_load_2d(sb + i * 4096, tm, bar, kb * kBK, row0 + 32 * i);
+  for (int i = 0; i < nb; ++i) tma_load_2d(sb + i * 4096, tm, bar, kb * kBK, U.row0 + 32 * i);
 }
 
 // --------------------------------------------------------------- gate/up
@@ -254,6 +287,7 @@ struct GluPolicy {
   static constexpr int kABytes = 128 * 128;  // 64 gate rows + 64 up rows
   static constexpr int kBBytesMax = kBN * 128;
   static constexpr int kEpiSmem = 4 * 32 * 17 * 4;
+  static constexpr int kAuxSmem = kGroupAuxSmem;
   static constexpr int kUmmaKBytes = 32;
   struct Params {
     CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 64
@@ -269,9 +303,14 @@ struct GluPolicy {
     prefetch_tmap(&p.wg); prefetch_tmap(&p.wu); prefetch_tmap(&p.sg); prefetch_tmap(&p.su);
     prefetch_tmap(&p.tz);
   }
-  static __device__ __forceinline__ int num_units(const Params &p) { return __ldg(p.gt.unit_off + p.gt.E + 1); }
+  static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
+  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
+    return grouped_num_units(p.gt, aux);
+  }
   static __device__ __forceinline__ int k_blocks(const Params &p) { return p.L / kBK; }
-  static __device__ __forceinline__ Unit unit(const Params &p, int u) { return grouped_unit(p.gt, u, kBN); }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
+    return grouped_unit(p.gt, aux, u, kBN);
+  }
   static __device__ __forceinline__ uint32_t stage_bytes(const Params &, const Unit &U, int) {
     return kABytes + ((U.nv + 31) >> 5) * 4096;
   }
@@ -281,7 +320,7 @@ struct GluPolicy {
     const int row = (sh ? 0 : U.g * p.F) + U.m * 64;
     tma_load_2d(sa, sh ? &p.sg : &p.wg, bar, kb * kBK, row);
     tma_load_2d(sa + 64 * 128, sh ? &p.su : &p.wu, bar, kb * kBK, row);
-    load_rows(&p.tz, p.gt, U, kb, sb, bar);
+    load_rows(&p.tz, U, kb, sb, bar);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
     return idesc_bf16(128, round16(U.nv));
@@ -298,7 +337,7 @@ struct GluPolicy {
     const bool is_gate = q < 2;
     const int pair = q & 1;
     const int f = U.m * 64 + pair * 32 + lane;
-    const size_t row0 = static_cast<size_t>(__ldg(p.gt.grp_off + U.g)) + U.n0;
+    const size_t row0 = static_cast<size_t>(U.row0);
     for (int c0 = 0; c0 < U.nv; c0 += 32) {
       float v[32];
       tmem_ld32(taddr + c0, v);
@@ -328,6 +367,7 @@ struct DownPolicy {
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
   static constexpr int kEpiSmem = kBN * 8;
+  static constexpr int kAuxSmem = kGroupAuxSmem;
   static constexpr int kUmmaKBytes = 32;
   struct Params {
     CUtensorMap wd;  // routed down [E*L, F], box 64 x 128
@@ -344,9 +384,14 @@ struct DownPolicy {
   static __device__ __forceinline__ void prefetch(const Params &p) {
     prefetch_tmap(&p.wd); prefetch_tmap(&p.sd); prefetch_tmap(&p.th);
   }
-  static __device__ __forceinline__ int num_units(const Params &p) { return __ldg(p.gt.unit_off + p.gt.E + 1); }
+  static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
+  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
+    return grouped_num_units(p.gt, aux);
+  }
   static __device__ __forceinline__ int k_blocks(const Params &p) { return p.F / kBK; }
-  static __device__ __forceinline__ Unit unit(const Params &p, int u) { return grouped_unit(p.gt, u, kBN); }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
+    return grouped_unit(p.gt, aux, u, kBN);
+  }
   static __device__ __forceinline__ uint32_t stage_bytes(const Params &, const Unit &U, int) {
     return kABytes + ((U.nv + 31) >> 5) * 4096;
   }
@@ -354,7 +399,7 @@ struct DownPolicy {
                                               uint32_t sb, uint32_t bar) {
     const bool sh = U.g == p.gt.E;
     tma_load_2d(sa, sh ? &p.sd : &p.wd, bar, kb * kBK, (sh ? 0 : U.g * p.L) + U.m * 128);
-    load_rows(&p.th, p.gt, U, kb, sb, bar);
+    load_rows(&p.th, U, kb, sb, bar);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
     return idesc_bf16(128, round16(U.nv));
@@ -372,7 +417,7 @@ struct DownPolicy {
     float *s_wt = reinterpret_cast<float *>(epi + kBN * sizeof(int));
     const int l = U.m * 128 + q * 32 + lane;
     const bool sh = U.g == p.gt.E;
-    const int row0 = __ldg(p.gt.grp_off + U.g) + U.n0;
+    const int row0 = U.row0;
     for (int c = etid; c < U.nv; c += 128) {
       const int row = row0 + c;
       if (sh) {

@@ -49,22 +49,25 @@ __global__ void topk_from_scores_kernel(const float *__restrict__ s, const float
       sel_i[j] = bi;
     }
   }
-  if (lane == 0) {
-    float den = sel_s[0];
-#pragma unroll
-    for (int j = 1; j < KMAX; ++j)
-      if (j < k) den = den + sel_s[j];
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      if (j < k) {
-        const size_t o = static_cast<size_t>(warp) * k + j;
-        const float w = sel_s[j] / den;
-        topk_idx[o] = sel_i[j];
-        topk_w[o] = w;
-        wscaled[o] = w * __ldg(alpha + sel_i[j]);
-      }
-    }
-  }
+  if (lane == 0) write_selection<KMAX>(sel_s, sel_i, k, static_cast<size_t>(warp), alpha, topk_idx, topk_w, wscaled);
+}
+
+// Merge of the router's partial selections: part p of token t left its best k
+// candidates (biased score, score, expert) at [(t * parts + p) * k + j].
+// One thread per token keeps the best k of all parts (same ranking rule).
+template <int KMAX>
+__global__ void topk_merge_kernel(const float *__restrict__ cand_v, const float *__restrict__ cand_s,
+                                  const int32_t *__restrict__ cand_i, int T, int parts, int k,
+                                  const float *__restrict__ alpha, int32_t *__restrict__ topk_idx,
+                                  float *__restrict__ topk_w, float *__restrict__ wscaled) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  TopK<KMAX> tk;
+  tk.init();
+  const size_t base = static_cast<size_t>(t) * parts * k;
+  for (int c = 0; c < parts * k; ++c)
+    topk_offer_any<KMAX>(tk, __ldg(cand_v + base + c), __ldg(cand_i + base + c), __ldg(cand_s + base + c));
+  write_selection<KMAX>(tk.s, tk.i, k, static_cast<size_t>(t), alpha, topk_idx, topk_w, wscaled);
 }
 
 // ---------------------------------------------------------------------------

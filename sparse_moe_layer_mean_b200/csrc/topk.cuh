@@ -64,4 +64,47 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
   return (va > vb) || (va == vb && ia < ib);
 }
 
+// Insert a candidate offered in any index order (the merge of partial lists):
+// it goes before the first kept entry it ranks before.
+template <int KMAX>
+__device__ __forceinline__ void topk_offer_any(TopK<KMAX> &tk, float cv, int ci, float cs) {
+  if (!ranks_before(cv, ci, tk.v[KMAX - 1], tk.i[KMAX - 1])) return;
+  bool take = false;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    take = take || ranks_before(cv, ci, tk.v[j], tk.i[j]);
+    const float tv = tk.v[j], ts = tk.s[j];
+    const int ti = tk.i[j];
+    tk.v[j] = take ? cv : tv;
+    tk.s[j] = take ? cs : ts;
+    tk.i[j] = take ? ci : ti;
+    cv = take ? tv : cv;
+    cs = take ? ts : cs;
+    ci = take ? ti : ci;
+  }
+}
+
+// Final step of routing for one token: w_j = s_j / (s_0 + ... + s_{k-1})
+// (fp32, summed in rank order), w'_j = w_j * alpha[e_j].
+template <int KMAX>
+__device__ __forceinline__ void write_selection(const float (&sel_s)[KMAX], const int (&sel_i)[KMAX], int k,
+                                                size_t t, const float *__restrict__ alpha,
+                                                int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                                                float *__restrict__ wscaled) {
+  float den = sel_s[0];
+#pragma unroll
+  for (int j = 1; j < KMAX; ++j)
+    if (j < k) den = den + sel_s[j];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j < k) {
+      const size_t o = t * k + j;
+      const float w = sel_s[j] / den;
+      topk_idx[o] = sel_i[j];
+      topk_w[o] = w;
+      wscaled[o] = w * __ldg(alpha + sel_i[j]);
+    }
+  }
+}
+
 }  // namespace mrl
