@@ -1,19 +1,23 @@
 // gemm_sm100.cuh — persistent, warp-specialised tcgen05 GEMM for sm_100a.
 //
 // D[128 x N] += A[128 x K] * B[N x K]^T, both operands K-major bf16 staged by
-// SWIZZLE_128B TMA tile loads into a STAGES-deep shared-memory ring; the fp32
-// accumulator lives in tensor memory, double-buffered (2 x 256 columns) so the
-// epilogue of one tile overlaps the main loop of the next.
+// SWIZZLE_128B TMA tile loads into shared memory; the fp32 accumulator lives
+// in tensor memory, double-buffered (2 x 256 columns) so the epilogue of one
+// tile overlaps the main loop of the next.  A and B have rings of their own
+// depths: the grouped expert GEMMs stream A (expert weights) from HBM and
+// re-read B (dispatched token rows) from L2, so A gets the deeper ring and
+// more HBM bytes stay in flight per SM.
 //
-//   warp 0   : TMA producer (one thread)
+//   warp 0   : TMA producer for A (one thread)
 //   warp 1   : TMEM allocator + UMMA issuer (one thread issues, commits)
 //   warps 2-5: epilogue (warp w reads TMEM lanes 32*(w%4) .. +31)
+//   warp 6   : TMA producer for B (one thread)
 //
 // A policy class P describes the problem: how many work units there are, what
 // each unit loads per 64-wide K block, the MMA N of each unit, and the
-// epilogue.  A unit may hold several sub-tiles that share one A operand and
-// one epilogue state (the router walks its expert chunks that way).  Units
-// are dealt round-robin over the persistent CTAs.
+// epilogue.  A unit may hold several sub-tiles that share one epilogue state
+// (the router walks its expert chunks that way).  Units are dealt round-robin
+// over the persistent CTAs.
 //
 // Every wait is bounded (see mbar_wait); on a timeout the CTA raises an abort
 // flag, every role unwinds, TMEM is freed, and the status word records it.
@@ -22,7 +26,7 @@
 
 namespace mrl {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;
 constexpr int kAccCols = 256;   // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 512;  // two buffers
 constexpr int kBK = 64;         // bf16 elements per K block (128 bytes = one swizzle row)
@@ -51,9 +55,10 @@ __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
 
 template <class P>
 struct GemmSmem {
-  static constexpr int kStageBytes = P::kABytes + P::kBBytesMax;
-  static constexpr int kBarOff = P::kStages * kStageBytes;
-  static constexpr int kNumBars = 2 * P::kStages + 4;
+  static constexpr int kARing = P::kStagesA * P::kABytes;
+  static constexpr int kBRing = P::kStagesB * P::kBBytesMax;
+  static constexpr int kBarOff = kARing + kBRing;
+  static constexpr int kNumBars = 2 * P::kStagesA + 2 * P::kStagesB + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kEpiOff = (kMiscOff + 16 + 127) & ~127;
   static constexpr int kAuxOff = (kEpiOff + P::kEpiSmem + 127) & ~127;
@@ -63,6 +68,7 @@ struct GemmSmem {
 template <class P>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ typename P::Params p) {
   using L = GemmSmem<P>;
+  constexpr int SA = P::kStagesA, SB = P::kStagesB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
@@ -71,20 +77,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint8_t *epi_smem = smem + L::kEpiOff;
   uint8_t *aux = smem + L::kAuxOff;  // per-launch tables staged once per CTA
 
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = full0 + 8 * P::kStages;
-  const uint32_t accf0 = empty0 + 8 * P::kStages;
+  const uint32_t fullA0 = smem_u32(bars);
+  const uint32_t emptyA0 = fullA0 + 8 * SA;
+  const uint32_t fullB0 = emptyA0 + 8 * SA;
+  const uint32_t emptyB0 = fullB0 + 8 * SB;
+  const uint32_t accf0 = emptyB0 + 8 * SB;
   const uint32_t acce0 = accf0 + 16;
-  const uint32_t stage0 = smem_u32(smem);
+  const uint32_t ringA = smem_u32(smem);
+  const uint32_t ringB = ringA + L::kARing;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   uint32_t *status = p.status;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < P::kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(fullA0 + 8 * s, 1);
+      mbar_init(emptyA0 + 8 * s, 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(fullB0 + 8 * s, 1);
+      mbar_init(emptyB0 + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf0 + 8 * a, 1);
@@ -105,29 +118,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const int nunits = P::num_units(p, aux);
   const int kblocks = P::k_blocks(p);
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 6) {
     if (lane == 0) {
+      // producers: warp 0 fills the A ring, warp 6 the B ring
+      const bool isA = warp == 0;
+      const int S = isA ? SA : SB;
+      const uint32_t full0 = isA ? fullA0 : fullB0, empty0 = isA ? emptyA0 : emptyB0;
+      const uint32_t ring = isA ? ringA : ringB;
+      const uint32_t sbytes = isA ? P::kABytes : P::kBBytesMax;
       P::prefetch(p);
       int s = 0;
       uint32_t ph = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         const Unit U = P::unit(p, u, aux);
         for (int sub = 0; sub < U.nsub; ++sub) {
-          const uint32_t bytes = P::stage_bytes(p, U, sub);
+          const uint32_t bytes = isA ? P::kABytes : P::b_bytes(p, U, sub);
           for (int kb = 0; kb < kblocks; ++kb) {
             if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, status)) goto done;
             mbar_arrive_expect_tx(full0 + 8 * s, bytes);
-            const uint32_t sa = stage0 + s * L::kStageBytes;
-            P::load(p, U, sub, kb, sa, sa + P::kABytes, full0 + 8 * s);
-            if (++s == P::kStages) { s = 0; ph ^= 1; }
+            if (isA)
+              P::load_a(p, U, sub, kb, ring + s * sbytes, full0 + 8 * s);
+            else
+              P::load_b(p, U, sub, kb, ring + s * sbytes, full0 + 8 * s);
+            if (++s == S) { s = 0; ph ^= 1; }
           }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      int s = 0, acc = 0;
-      uint32_t ph = 0, aph = 0;
+      int sa = 0, sb = 0, acc = 0;
+      uint32_t pa = 0, pb = 0, aph = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         const Unit U = P::unit(p, u, aux);
         for (int sub = 0; sub < U.nsub; ++sub) {
@@ -136,16 +157,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           const uint32_t tacc = tmem_base + acc * kAccCols;
           const uint32_t idesc = P::idesc(p, U, sub);
           for (int kb = 0; kb < kblocks; ++kb) {
-            if (!mbar_wait(full0 + 8 * s, ph, abort_flag, status)) goto done;
+            if (!mbar_wait(fullA0 + 8 * sa, pa, abort_flag, status)) goto done;
+            if (!mbar_wait(fullB0 + 8 * sb, pb, abort_flag, status)) goto done;
             tc_fence_after();
-            const uint32_t sa = stage0 + s * L::kStageBytes;
-            const uint32_t sb = sa + P::kABytes;
+            const uint32_t a_s = ringA + sa * P::kABytes;
+            const uint32_t b_s = ringB + sb * P::kBBytesMax;
 #pragma unroll
             for (int kk = 0; kk < kBK * 2 / P::kUmmaKBytes; ++kk)
-              P::mma(tacc, sdesc_sw128(sa + kk * P::kUmmaKBytes), sdesc_sw128(sb + kk * P::kUmmaKBytes),
+              P::mma(tacc, sdesc_sw128(a_s + kk * P::kUmmaKBytes), sdesc_sw128(b_s + kk * P::kUmmaKBytes),
                      idesc, (kb | kk) != 0);
-            umma_commit(empty0 + 8 * s);
-            if (++s == P::kStages) { s = 0; ph ^= 1; }
+            umma_commit(emptyA0 + 8 * sa);
+            umma_commit(emptyB0 + 8 * sb);
+            if (++sa == SA) { sa = 0; pa ^= 1; }
+            if (++sb == SB) { sb = 0; pb ^= 1; }
           }
           umma_commit(accf0 + 8 * acc);
           acc ^= 1;

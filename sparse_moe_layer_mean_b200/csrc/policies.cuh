@@ -19,7 +19,8 @@ __device__ __forceinline__ int round16(int n) { return (n + 15) & ~15; }
 
 // ---------------------------------------------------------------- dense
 struct DensePolicy {
-  static constexpr int kStages = 4;
+  static constexpr int kStagesA = 4;
+  static constexpr int kStagesB = 4;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
@@ -53,12 +54,13 @@ struct DensePolicy {
     U.nsub = 1;
     return U;
   }
-  static __device__ __forceinline__ uint32_t stage_bytes(const Params &, const Unit &, int) {
-    return kABytes + kBBytesMax;
-  }
-  static __device__ __forceinline__ void load(const Params &p, const Unit &U, int, int kb, uint32_t sa,
-                                              uint32_t sb, uint32_t bar) {
+  static __device__ __forceinline__ uint32_t b_bytes(const Params &, const Unit &, int) { return kBBytesMax; }
+  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int, int kb, uint32_t sa,
+                                                uint32_t bar) {
     tma_load_2d(sa, &p.ta, bar, kb * kBK, U.m * 128);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int, int kb, uint32_t sb,
+                                                uint32_t bar) {
     tma_load_2d(sb, &p.tb, bar, kb * kBK, U.n0);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
@@ -112,7 +114,8 @@ struct DensePolicy {
 // given as bf16 hi + bf16 lo parts and the K loop runs over both (2 * d_lat),
 // reusing each router tile for the hi and the lo half.
 struct RouterPolicy {
-  static constexpr int kStages = 4;
+  static constexpr int kStagesA = 4;
+  static constexpr int kStagesB = 4;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = 256 * 128;
   static constexpr int kEpiSmem = 0;
@@ -153,15 +156,19 @@ struct RouterPolicy {
     U.nsub = p.E / p.ec / p.parts;
     return U;
   }
-  static __device__ __forceinline__ uint32_t stage_bytes(const Params &p, const Unit &, int) {
-    return kABytes + p.R * p.ec * 128;
+  static __device__ __forceinline__ uint32_t b_bytes(const Params &p, const Unit &, int) {
+    return p.R * p.ec * 128;
   }
-  static __device__ __forceinline__ void load(const Params &p, const Unit &U, int sub, int kb, uint32_t sa,
-                                              uint32_t sb, uint32_t bar) {
+  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int, int kb, uint32_t sa,
+                                                uint32_t bar) {
     const int nk = p.L / kBK;
     const bool lo = kb >= nk;
-    const int x = (lo ? kb - nk : kb) * kBK;
-    tma_load_2d(sa, lo ? &p.ta_lo : &p.ta, bar, x, U.m * 128);
+    tma_load_2d(sa, lo ? &p.ta_lo : &p.ta, bar, (lo ? kb - nk : kb) * kBK, U.m * 128);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int sub, int kb, uint32_t sb,
+                                                uint32_t bar) {
+    const int nk = p.L / kBK;
+    const int x = (kb >= nk ? kb - nk : kb) * kBK;
     const int chunk = U.g * U.nsub + sub;
     for (int r = 0; r < p.R; ++r) tma_load_2d(sb + r * p.ec * 128, &p.tb, bar, x, r * p.E + chunk * p.ec);
   }
@@ -235,15 +242,16 @@ struct GroupTable {
 };
 
 constexpr int kMaxGroups = 1024 + 2;
-constexpr int kGroupAuxSmem = 3 * kMaxGroups * 4;
+constexpr int kGroupAuxSmem = 2 * kMaxGroups * 4;
 
+// unit_off and grp_off (E+2 entries each; grp_off[E+1] ends the shared
+// group, so a group's row count is grp_off[g+1] - grp_off[g]).
 __device__ __forceinline__ void stage_group_table(const GroupTable &gt, uint8_t *aux) {
   int *s = reinterpret_cast<int *>(aux);
   const int n = gt.E + 2;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     s[i] = __ldg(gt.unit_off + i);
     s[kMaxGroups + i] = __ldg(gt.grp_off + i);
-    s[2 * kMaxGroups + i] = __ldg(gt.grp_cnt + i);
   }
 }
 
@@ -254,7 +262,6 @@ __device__ __forceinline__ int grouped_num_units(const GroupTable &gt, const uin
 __device__ __forceinline__ Unit grouped_unit(const GroupTable &gt, const uint8_t *aux, int u, int BN) {
   const int *uo = reinterpret_cast<const int *>(aux);
   const int *go = uo + kMaxGroups;
-  const int *gc = uo + 2 * kMaxGroups;
   // largest g in [0, E] with unit_off[g] <= u (zero-unit groups share the next offset)
   int lo = 0, hi = gt.E;
   while (lo < hi) {
@@ -264,7 +271,7 @@ __device__ __forceinline__ Unit grouped_unit(const GroupTable &gt, const uint8_t
   Unit U;
   U.g = lo;
   const int local = u - uo[lo];
-  const int cnt = gc[lo];
+  const int cnt = go[lo + 1] - go[lo];
   const int ntiles = (cnt + BN - 1) / BN;
   U.m = local / ntiles;
   U.n0 = (local - U.m * ntiles) * BN;
@@ -282,7 +289,8 @@ __device__ __forceinline__ void load_rows(const CUtensorMap *tm, const Unit &U, 
 
 // --------------------------------------------------------------- gate/up
 struct GluPolicy {
-  static constexpr int kStages = 4;
+  static constexpr int kStagesA = 7;
+  static constexpr int kStagesB = 3;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;  // 64 gate rows + 64 up rows
   static constexpr int kBBytesMax = kBN * 128;
@@ -311,15 +319,18 @@ struct GluPolicy {
   static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
     return grouped_unit(p.gt, aux, u, kBN);
   }
-  static __device__ __forceinline__ uint32_t stage_bytes(const Params &, const Unit &U, int) {
-    return kABytes + ((U.nv + 31) >> 5) * 4096;
+  static __device__ __forceinline__ uint32_t b_bytes(const Params &, const Unit &U, int) {
+    return ((U.nv + 31) >> 5) * 4096;
   }
-  static __device__ __forceinline__ void load(const Params &p, const Unit &U, int, int kb, uint32_t sa,
-                                              uint32_t sb, uint32_t bar) {
+  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int, int kb, uint32_t sa,
+                                                uint32_t bar) {
     const bool sh = U.g == p.gt.E;
     const int row = (sh ? 0 : U.g * p.F) + U.m * 64;
     tma_load_2d(sa, sh ? &p.sg : &p.wg, bar, kb * kBK, row);
     tma_load_2d(sa + 64 * 128, sh ? &p.su : &p.wu, bar, kb * kBK, row);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int, int kb, uint32_t sb,
+                                                uint32_t bar) {
     load_rows(&p.tz, U, kb, sb, bar);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
@@ -362,7 +373,8 @@ struct GluPolicy {
 
 // ------------------------------------------------------------------ down
 struct DownPolicy {
-  static constexpr int kStages = 4;
+  static constexpr int kStagesA = 7;
+  static constexpr int kStagesB = 3;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
@@ -392,13 +404,16 @@ struct DownPolicy {
   static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
     return grouped_unit(p.gt, aux, u, kBN);
   }
-  static __device__ __forceinline__ uint32_t stage_bytes(const Params &, const Unit &U, int) {
-    return kABytes + ((U.nv + 31) >> 5) * 4096;
+  static __device__ __forceinline__ uint32_t b_bytes(const Params &, const Unit &U, int) {
+    return ((U.nv + 31) >> 5) * 4096;
   }
-  static __device__ __forceinline__ void load(const Params &p, const Unit &U, int, int kb, uint32_t sa,
-                                              uint32_t sb, uint32_t bar) {
+  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int, int kb, uint32_t sa,
+                                                uint32_t bar) {
     const bool sh = U.g == p.gt.E;
     tma_load_2d(sa, sh ? &p.sd : &p.wd, bar, kb * kBK, (sh ? 0 : U.g * p.L) + U.m * 128);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int, int kb, uint32_t sb,
+                                                uint32_t bar) {
     load_rows(&p.th, U, kb, sb, bar);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
