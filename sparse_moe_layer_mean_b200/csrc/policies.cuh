@@ -288,18 +288,23 @@ __device__ __forceinline__ void load_rows(const CUtensorMap *tm, const Unit &U, 
 }
 
 // --------------------------------------------------------------- gate/up
+// A tile (128 rows) for the unit's 64 d_ff columns f0 = m*64 .. +63: TMEM lane
+// quarter q holds gate rows f0+16q .. +15 in its lanes 0-15 and the matching up
+// rows in lanes 16-31 (eight 16-row TMA boxes per K block).  In the epilogue
+// each warp therefore owns complete (gate, up) pairs and pairs them with one
+// shuffle across the half-warps.
 struct GluPolicy {
   static constexpr int kStagesA = 7;
   static constexpr int kStagesB = 3;
   static constexpr int kBN = 256;
-  static constexpr int kABytes = 128 * 128;  // 64 gate rows + 64 up rows
+  static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
-  static constexpr int kEpiSmem = 4 * 32 * 17 * 4;
+  static constexpr int kEpiSmem = 0;
   static constexpr int kAuxSmem = kGroupAuxSmem;
   static constexpr int kUmmaKBytes = 32;
   struct Params {
-    CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 64
-    CUtensorMap sg, su;  // shared gate/up [F, L], box 64 x 64
+    CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 16
+    CUtensorMap sg, su;  // shared gate/up [F, L], box 64 x 16
     CUtensorMap tz;      // dispatched z [(T*k+T), L], box 64 x 32
     GroupTable gt;
     __nv_bfloat16 *h;    // [(T*k+T), F]
@@ -325,9 +330,14 @@ struct GluPolicy {
   static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int, int kb, uint32_t sa,
                                                 uint32_t bar) {
     const bool sh = U.g == p.gt.E;
+    const CUtensorMap *mg = sh ? &p.sg : &p.wg;
+    const CUtensorMap *mu = sh ? &p.su : &p.wu;
     const int row = (sh ? 0 : U.g * p.F) + U.m * 64;
-    tma_load_2d(sa, sh ? &p.sg : &p.wg, bar, kb * kBK, row);
-    tma_load_2d(sa + 64 * 128, sh ? &p.su : &p.wu, bar, kb * kBK, row);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      tma_load_2d(sa + (32 * q) * 128, mg, bar, kb * kBK, row + 16 * q);
+      tma_load_2d(sa + (32 * q + 16) * 128, mu, bar, kb * kBK, row + 16 * q);
+    }
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int, int kb, uint32_t sb,
                                                 uint32_t bar) {
@@ -339,34 +349,27 @@ struct GluPolicy {
   static __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
     umma_f16(d, a, b, id, acc);
   }
-  // Lanes 0-63 hold gate rows f = m*64 + lane, lanes 64-127 the matching up
-  // rows.  Warp pair (q, q+2) swaps half a chunk through shared memory so each
-  // warp owns complete (g, u) pairs for 16 of the chunk's 32 token columns.
   static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
-                                                  int lane, int, EpiState &, uint8_t *epi) {
-    float *xb = reinterpret_cast<float *>(epi);  // [4][32][17]
-    const bool is_gate = q < 2;
-    const int pair = q & 1;
-    const int f = U.m * 64 + pair * 32 + lane;
-    const size_t row0 = static_cast<size_t>(U.row0);
+                                                  int lane, int, EpiState &, uint8_t *) {
+    const bool up_half = lane >= 16;
+    const int f = U.m * 64 + q * 16 + (lane & 15);
+    __nv_bfloat16 *hcol = p.h + static_cast<size_t>(U.row0) * p.F + f;
     for (int c0 = 0; c0 < U.nv; c0 += 32) {
       float v[32];
       tmem_ld32(taddr + c0, v);
       tmem_ld_wait();
-      // gate warps give away columns 16..31, up warps give away columns 0..15
-      float *mine = xb + (q * 32 + lane) * 17;
+      // gate lanes keep tokens c0..c0+15 and receive their up values; up lanes
+      // keep tokens c0+16..c0+31 and receive their gate values
+      const int tbase = c0 + (up_half ? 16 : 0);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) mine[c] = is_gate ? v[16 + c] : v[c];
-      named_bar_sync(2, 128);
-      const float *other = xb + (((q + 2) & 3) * 32 + lane) * 17;
-      const int cbase = c0 + (is_gate ? 0 : 16);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float g = is_gate ? v[c] : other[c];
-        const float u = is_gate ? other[c] : v[16 + c];
-        if (cbase + c < U.nv) p.h[(row0 + cbase + c) * p.F + f] = __float2bfloat16_rn(siluf_(g) * u);
+      for (int i = 0; i < 16; ++i) {
+        const float give = up_half ? v[i] : v[16 + i];
+        const float got = __shfl_xor_sync(0xffffffffu, give, 16);
+        const float g = up_half ? got : v[i];
+        const float u = up_half ? v[16 + i] : got;
+        if (tbase + i < U.nv)
+          hcol[static_cast<size_t>(tbase + i) * p.F] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
       }
-      named_bar_sync(2, 128);
     }
   }
 };
