@@ -159,6 +159,20 @@ class ClockSampler:
                 "power_w_median": statistics.median(power) if power else None}
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of a list of floats over all ranks of the default group."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, tokens_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch each step."""
+    return world * tokens_per_rank * steps / (max_ms * 1e-3)
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -341,12 +355,11 @@ def main():
 
     # max over ranks
     if world > 1:
-        t = torch.tensor([ms, e2e[0] if e2e else 0.0] + stage_ms, device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t[0].item()
+        red = max_over_ranks([ms, e2e[0] if e2e else 0.0] + stage_ms, dev)
+        ms = red[0]
         if e2e:
-            e2e[0] = t[1].item()
-        stage_ms = t[2:].tolist()
+            e2e[0] = red[1]
+        stage_ms = red[2:]
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
@@ -358,7 +371,7 @@ def main():
         t_flops = flops / (peaks["bf16_tflops_sustained"] * 1e12)
         workload = s.name
         line = {
-            "metric": METRIC, "value": world * s.T * args.steps / (ms * 1e-3), "unit": UNIT,
+            "metric": METRIC, "value": job_throughput(world, s.T, args.steps, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -386,7 +399,7 @@ def main():
             * args.steps,
         }
         if e2e:
-            line["e2e"] = {"value": world * s.T * args.steps / (e2e[0] * 1e-3), "unit": UNIT,
+            line["e2e"] = {"value": job_throughput(world, s.T, args.steps, e2e[0]), "unit": UNIT,
                            "h2d_bytes_per_step": e2e[1], "d2h_bytes_per_step": e2e[2]}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(s, weights, x, bias, min(args.cpu_sample, s.T))
