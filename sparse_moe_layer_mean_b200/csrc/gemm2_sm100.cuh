@@ -1,0 +1,294 @@
+// gemm2_sm100.cuh — CTA-pair (cta_group::2) persistent tcgen05 GEMM for the
+// grouped expert GEMMs.
+//
+// Two CTAs of a cluster form one M = 256 UMMA: each holds 128 rows of A (its
+// own expert-weight rows) and half of the unit's N token rows in its shared
+// memory; the even CTA issues tcgen05.mma.cta_group::2 for both, and each CTA
+// receives its 128 rows of the accumulator in its own TMEM.  The token tile is
+// therefore read from L2 once per pair instead of once per CTA.
+//
+// Synchronisation (all waits bounded, as in gemm_sm100.cuh):
+//  - both CTAs' TMA loads (cta_group::2 form, no multicast) complete on the
+//    even CTA's full barriers; the even CTA's producers set the expected bytes
+//    of both halves;
+//  - the even CTA's commits arrive on the empty / accumulator-full barriers of
+//    both CTAs (tcgen05.commit multicast);
+//  - each CTA's epilogue warps arrive on the even CTA's accumulator-empty
+//    barrier (count 8) once they have drained their TMEM rows.
+#pragma once
+#include "gemm_sm100.cuh"
+#include "policies.cuh"
+
+namespace mrl {
+
+template <class P>
+struct Gemm2Smem {
+  static constexpr int kARing = P::kStagesA * P::kABytes;
+  static constexpr int kBRing = P::kStagesB * P::kBBytesMax;
+  static constexpr int kBarOff = kARing + kBRing;
+  static constexpr int kNumBars = 2 * P::kStagesA + 2 * P::kStagesB + 4;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kEpiOff = (kMiscOff + 16 + 127) & ~127;
+  static constexpr int kAuxOff = (kEpiOff + P::kEpiSmem + 127) & ~127;
+  static constexpr int kTotal = kAuxOff + P::kAuxSmem + 1024;
+};
+
+template <class P>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm2_kernel(const __grid_constant__ typename P::Params p) {
+  using L = Gemm2Smem<P>;
+  constexpr int SA = P::kStagesA, SB = P::kStagesB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+  uint8_t *epi_smem = smem + L::kEpiOff;
+  uint8_t *aux = smem + L::kAuxOff;
+
+  const uint32_t fullA0 = smem_u32(bars);
+  const uint32_t emptyA0 = fullA0 + 8 * SA;
+  const uint32_t fullB0 = emptyA0 + 8 * SA;
+  const uint32_t emptyB0 = fullB0 + 8 * SB;
+  const uint32_t accf0 = emptyB0 + 8 * SB;
+  const uint32_t acce0 = accf0 + 16;
+  const uint32_t ringA = smem_u32(smem);
+  const uint32_t ringB = ringA + L::kARing;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = static_cast<int>(cluster_id_x());
+  const int ncl = static_cast<int>(nclusters_x());
+  uint32_t *status = p.status;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(fullA0 + 8 * s, 1);
+      mbar_init(emptyA0 + 8 * s, 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(fullB0 + 8 * s, 1);
+      mbar_init(emptyB0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf0 + 8 * a, 1);
+      mbar_init(acce0 + 8 * a, 8);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  P::stage_aux(p, aux);
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barrier initialisation visible to the peer before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nunits = P::num_units(p, aux);
+  const int kblocks = P::k_blocks(p);
+
+  if (warp == 0 || warp == 6) {
+    if (lane == 0) {
+      const bool isA = warp == 0;
+      const int S = isA ? SA : SB;
+      const uint32_t full0 = isA ? fullA0 : fullB0, empty0 = isA ? emptyA0 : emptyB0;
+      const uint32_t ring = isA ? ringA : ringB;
+      const uint32_t sbytes = isA ? P::kABytes : P::kBBytesMax;
+      P::prefetch(p);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int u = cid; u < nunits; u += ncl) {
+        const Unit U = P::unit(p, u, aux);
+        const uint32_t pair_bytes = isA ? 2u * P::kABytes : P::b_bytes_pair(p, U);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, status)) goto done;
+          const uint32_t full_local = full0 + 8 * s;
+          if (leader) mbar_arrive_expect_tx(full_local, pair_bytes);
+          const uint32_t full_cl = mapa_shared(full_local, 0);
+          if (isA)
+            P::load_a(p, U, kb, ring + s * sbytes, full_cl, rank);
+          else
+            P::load_b(p, U, kb, ring + s * sbytes, full_cl, rank);
+          if (++s == S) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      int sa = 0, sb = 0, acc = 0;
+      uint32_t pa = 0, pb = 0, aph = 0;
+      for (int u = cid; u < nunits; u += ncl) {
+        const Unit U = P::unit(p, u, aux);
+        if (!mbar_wait(acce0 + 8 * acc, aph ^ 1, abort_flag, status)) goto done;
+        tc_fence_after();
+        const uint32_t tacc = tmem_base + acc * kAccCols;
+        const uint32_t idesc = P::idesc(p, U);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(fullA0 + 8 * sa, pa, abort_flag, status)) goto done;
+          if (!mbar_wait(fullB0 + 8 * sb, pb, abort_flag, status)) goto done;
+          tc_fence_after();
+          const uint32_t a_s = ringA + sa * P::kABytes;
+          const uint32_t b_s = ringB + sb * P::kBBytesMax;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16_pair(tacc, sdesc_sw128(a_s + kk * 32), sdesc_sw128(b_s + kk * 32), idesc, (kb | kk) != 0);
+          umma_commit_pair(emptyA0 + 8 * sa, 0x3);
+          umma_commit_pair(emptyB0 + 8 * sb, 0x3);
+          if (++sa == SA) { sa = 0; pa ^= 1; }
+          if (++sb == SB) { sb = 0; pb ^= 1; }
+        }
+        umma_commit_pair(accf0 + 8 * acc, 0x3);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int etid = threadIdx.x - 64;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int u = cid; u < nunits; u += ncl) {
+      const Unit U = P::unit(p, u, aux);
+      const bool ok = mbar_wait(accf0 + 8 * acc, aph, abort_flag, status);
+      if (bar_red_or(1, 128, !ok || *abort_flag)) goto done;
+      tc_fence_after();
+      P::epilogue(p, U, tmem_base + acc * kAccCols + (static_cast<uint32_t>(q * 32) << 16), q, lane, etid, rank,
+                  epi_smem);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(acce0 + 8 * acc);
+        else
+          mbar_arrive_remote(mapa_shared(acce0 + 8 * acc, 0));
+      }
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still signal its barriers
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------- policies
+__device__ __forceinline__ int round32(int n) { return (n + 31) & ~31; }
+
+// B half of CTA `rank`: rows row0 + rank*N/2 .. + N/2 (N = MMA N, multiple of
+// 32), as 16-row boxes.
+__device__ __forceinline__ void load_rows_half(const CUtensorMap *tm, const Unit &U, int kb, uint32_t sb,
+                                               uint32_t bar_cl, uint32_t rank) {
+  const int half = round32(U.nv) >> 1;
+  const int r0 = U.row0 + static_cast<int>(rank) * half;
+  for (int i = 0; i < (half >> 4); ++i) tma_load_2d_pair(sb + i * 2048, tm, bar_cl, kb * kBK, r0 + 16 * i);
+}
+
+// gate/up over a CTA pair: unit = (group, 128-wide d_ff slice, <= 256 tokens);
+// CTA r owns d_ff columns f0 = m*128 + r*64 .. +63 with the same gate/up row
+// interleave as GluPolicy, so its epilogue is the same.
+struct Glu2Policy {
+  static constexpr int kStagesA = 6;
+  static constexpr int kStagesB = 6;
+  static constexpr int kBN = 256;
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytesMax = (kBN / 2) * 128;
+  static constexpr int kEpiSmem = 0;
+  static constexpr int kAuxSmem = kGroupAuxSmem;
+  using Params = GluPolicy::Params;
+  static __device__ __forceinline__ void prefetch(const Params &p) { GluPolicy::prefetch(p); }
+  static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
+  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
+    return grouped_num_units(p.gt, aux);
+  }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.L / kBK; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
+    return grouped_unit(p.gt, aux, u, kBN);
+  }
+  static __device__ __forceinline__ uint32_t b_bytes_pair(const Params &, const Unit &U) {
+    return round32(U.nv) * 128;
+  }
+  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int kb, uint32_t sa,
+                                                uint32_t bar_cl, uint32_t rank) {
+    const bool sh = U.g == p.gt.E;
+    const CUtensorMap *mg = sh ? &p.sg : &p.wg;
+    const CUtensorMap *mu = sh ? &p.su : &p.wu;
+    const int row = (sh ? 0 : U.g * p.F) + U.m * 128 + static_cast<int>(rank) * 64;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      tma_load_2d_pair(sa + (32 * q) * 128, mg, bar_cl, kb * kBK, row + 16 * q);
+      tma_load_2d_pair(sa + (32 * q + 16) * 128, mu, bar_cl, kb * kBK, row + 16 * q);
+    }
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb,
+                                                uint32_t bar_cl, uint32_t rank) {
+    load_rows_half(&p.tz, U, kb, sb, bar_cl, rank);
+  }
+  static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U) {
+    return idesc_bf16(256, round32(U.nv));
+  }
+  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, uint32_t taddr, int q, int lane,
+                                                  int etid, uint32_t rank, uint8_t *epi) {
+    Unit V = U;
+    V.m = U.m * 2 + static_cast<int>(rank);  // the CTA's 64-wide d_ff slice
+    GluPolicy::EpiState st;
+    GluPolicy::epilogue(p, V, 0, taddr, q, lane, etid, st, epi);
+  }
+};
+
+// expert down over a CTA pair: unit = (group, 256-wide d_lat slice, <= 256
+// tokens); CTA r owns output rows l = m*256 + r*128 .. +127.
+struct Down2Policy {
+  static constexpr int kStagesA = 6;
+  static constexpr int kStagesB = 6;
+  static constexpr int kBN = 256;
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytesMax = (kBN / 2) * 128;
+  static constexpr int kEpiSmem = DownPolicy::kEpiSmem;
+  static constexpr int kAuxSmem = kGroupAuxSmem;
+  using Params = DownPolicy::Params;
+  static __device__ __forceinline__ void prefetch(const Params &p) { DownPolicy::prefetch(p); }
+  static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
+  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
+    return grouped_num_units(p.gt, aux);
+  }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.F / kBK; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
+    return grouped_unit(p.gt, aux, u, kBN);
+  }
+  static __device__ __forceinline__ uint32_t b_bytes_pair(const Params &, const Unit &U) {
+    return round32(U.nv) * 128;
+  }
+  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int kb, uint32_t sa,
+                                                uint32_t bar_cl, uint32_t rank) {
+    const bool sh = U.g == p.gt.E;
+    tma_load_2d_pair(sa, sh ? &p.sd : &p.wd, bar_cl, kb * kBK,
+                     (sh ? 0 : U.g * p.L) + U.m * 256 + static_cast<int>(rank) * 128);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb,
+                                                uint32_t bar_cl, uint32_t rank) {
+    load_rows_half(&p.th, U, kb, sb, bar_cl, rank);
+  }
+  static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U) {
+    return idesc_bf16(256, round32(U.nv));
+  }
+  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, uint32_t taddr, int q, int lane,
+                                                  int etid, uint32_t rank, uint8_t *epi) {
+    Unit V = U;
+    V.m = U.m * 2 + static_cast<int>(rank);  // the CTA's 128-wide d_lat slice
+    DownPolicy::EpiState st;
+    DownPolicy::epilogue(p, V, 0, taddr, q, lane, etid, st, epi);
+  }
+};
+
+}  // namespace mrl

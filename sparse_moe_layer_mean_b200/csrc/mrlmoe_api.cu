@@ -9,6 +9,7 @@
 
 #include "mrlmoe.h"
 #include "policies.cuh"
+#include "gemm2_sm100.cuh"
 #include "routing.cuh"
 
 using namespace mrl;
@@ -170,6 +171,28 @@ cudaError_t launch_gemm(const typename P::Params &p, int grid, cudaStream_t st) 
   return cudaGetLastError();
 }
 
+template <class P>
+cudaError_t launch_gemm_pair(const typename P::Params &p, int grid, cudaStream_t st) {
+  static_assert(Gemm2Smem<P>::kTotal <= 232448, "GEMM shared memory above the 227 KB per-block limit");
+  static bool configured[kMaxDevices] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm2_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Gemm2Smem<P>::kTotal);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  gemm2_kernel<P><<<grid & ~1, kGemmThreads, Gemm2Smem<P>::kTotal, st>>>(p);
+  return cudaGetLastError();
+}
+
+// The expert GEMMs run on CTA pairs (M = 256) whenever the slice widths allow:
+// gate/up needs d_ff % 128 == 0 (always true), the down GEMM d_lat % 256 == 0.
+bool down_uses_pairs(const mrlmoe_config &c) { return c.d_lat % 256 == 0; }
+int glu_m_tiles(const mrlmoe_config &c) { return c.d_ff / 128; }
+int down_m_tiles(const mrlmoe_config &c) { return down_uses_pairs(c) ? c.d_lat / 256 : c.d_lat / 128; }
+
 #define MRL_TRY(expr)                                  \
   do {                                                 \
     if ((expr) != cudaSuccess) return MRLMOE_ERR_CUDA; \
@@ -229,7 +252,7 @@ mrlmoe_status launch_dispatch(const mrlmoe_config &c, const Ptrs &P, cudaStream_
   MRL_TRY(cudaGetLastError());
   expert_colscan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(P.mask, E, nch, P.base, P.counts_e);
   MRL_TRY(cudaGetLastError());
-  expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, kExpertBN, c.d_ff / 64, c.d_lat / 128, P.grp_off,
+  expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, kExpertBN, glu_m_tiles(c), down_m_tiles(c), P.grp_off,
                                             P.grp_cnt, P.unit1, P.unit2, P.out_counts, P.out_offsets);
   MRL_TRY(cudaGetLastError());
   expert_scatter_kernel<<<(nch * 32 + 255) / 256, 256, 0, st>>>(P.topk_idx, P.mask, P.base, P.grp_off, T, E, k,
@@ -335,27 +358,27 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
     MRL_TRY(cudaGetLastError());
   }
   if (!mark(4)) return MRLMOE_ERR_CUDA;
-  GroupTable gt1{P.grp_off, P.grp_cnt, P.unit1, E, F / 64};
-  GroupTable gt2{P.grp_off, P.grp_cnt, P.unit2, E, Ld / 128};
+  GroupTable gt1{P.grp_off, P.grp_cnt, P.unit1, E, glu_m_tiles(*cfg)};
+  GroupTable gt2{P.grp_off, P.grp_cnt, P.unit2, E, down_m_tiles(*cfg)};
   {
     GluPolicy::Params p{};
     if (!make_map(&p.wg, w->w_gate, 2, Ld, static_cast<uint64_t>(E) * F, 16) ||
         !make_map(&p.wu, w->w_up_e, 2, Ld, static_cast<uint64_t>(E) * F, 16) ||
         !make_map(&p.sg, w->w_sh_gate, 2, Ld, F, 16) || !make_map(&p.su, w->w_sh_up, 2, Ld, F, 16) ||
-        !make_map(&p.tz, P.zbuf, 2, Ld, static_cast<uint64_t>(Tk) + T, 32))
+        !make_map(&p.tz, P.zbuf, 2, Ld, static_cast<uint64_t>(Tk) + T, 16))
       return MRLMOE_ERR_CUDA;
     p.gt = gt1;
     p.h = P.hbuf;
     p.F = F; p.L = Ld;
     p.status = P.status;
-    MRL_TRY(launch_gemm<GluPolicy>(p, sms, st));
+    MRL_TRY(launch_gemm_pair<Glu2Policy>(p, sms, st));
   }
   if (!mark(5)) return MRLMOE_ERR_CUDA;
   {
     DownPolicy::Params p{};
     if (!make_map(&p.wd, w->w_down_e, 2, F, static_cast<uint64_t>(E) * Ld, 128) ||
         !make_map(&p.sd, w->w_sh_down, 2, F, Ld, 128) ||
-        !make_map(&p.th, P.hbuf, 2, F, static_cast<uint64_t>(Tk) + T, 32))
+        !make_map(&p.th, P.hbuf, 2, F, static_cast<uint64_t>(Tk) + T, down_uses_pairs(*cfg) ? 16 : 32))
       return MRLMOE_ERR_CUDA;
     p.gt = gt2;
     p.perm = P.perm;
@@ -363,7 +386,10 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
     p.slots = P.slots;
     p.L = Ld; p.F = F; p.k = k; p.Tk = Tk;
     p.status = P.status;
-    MRL_TRY(launch_gemm<DownPolicy>(p, sms, st));
+    if (down_uses_pairs(*cfg))
+      MRL_TRY(launch_gemm_pair<Down2Policy>(p, sms, st));
+    else
+      MRL_TRY(launch_gemm<DownPolicy>(p, sms, st));
   }
   if (!mark(6)) return MRLMOE_ERR_CUDA;
   combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k,
