@@ -9,10 +9,11 @@
 //
 // Synchronisation (all waits bounded, as in gemm_sm100.cuh):
 //  - both CTAs' TMA loads (cta_group::2 form, no multicast) complete on the
-//    even CTA's full barriers; the even CTA's producers set the expected bytes
-//    of both halves;
-//  - the even CTA's commits arrive on the empty / accumulator-full barriers of
-//    both CTAs (tcgen05.commit multicast);
+//    even CTA's full barriers; the even CTA's two producers set the expected
+//    bytes of both halves;
+//  - one commit of the even CTA per group of stages, and one per tile, arrive
+//    on the release / accumulator-full barriers of both CTAs (tcgen05.commit
+//    multicast);
 //  - each CTA's epilogue warps arrive on the even CTA's accumulator-empty
 //    barrier (count 8) once they have drained their TMEM rows.
 #pragma once
@@ -23,10 +24,11 @@ namespace mrl {
 
 template <class P>
 struct Gemm2Smem {
-  static constexpr int kARing = P::kStagesA * P::kABytes;
-  static constexpr int kBRing = P::kStagesB * P::kBBytesMax;
-  static constexpr int kBarOff = kARing + kBRing;
-  static constexpr int kNumBars = 2 * P::kStagesA + 2 * P::kStagesB + 4;
+  static_assert(P::kStages % P::kGroup == 0, "ring depth must be a multiple of the release group");
+  static constexpr int kStageBytes = P::kABytes + P::kBBytesMax;
+  static constexpr int kRing = P::kStages * kStageBytes;
+  static constexpr int kBarOff = kRing;
+  static constexpr int kNumBars = P::kStages + P::kStages / P::kGroup + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kEpiOff = (kMiscOff + 16 + 127) & ~127;
   static constexpr int kAuxOff = (kEpiOff + P::kEpiSmem + 127) & ~127;
@@ -37,7 +39,7 @@ template <class P>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm2_kernel(const __grid_constant__ typename P::Params p) {
   using L = Gemm2Smem<P>;
-  constexpr int SA = P::kStagesA, SB = P::kStagesB;
+  constexpr int S = P::kStages, G = P::kGroup;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
@@ -46,14 +48,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint8_t *epi_smem = smem + L::kEpiOff;
   uint8_t *aux = smem + L::kAuxOff;
 
-  const uint32_t fullA0 = smem_u32(bars);
-  const uint32_t emptyA0 = fullA0 + 8 * SA;
-  const uint32_t fullB0 = emptyA0 + 8 * SA;
-  const uint32_t emptyB0 = fullB0 + 8 * SB;
-  const uint32_t accf0 = emptyB0 + 8 * SB;
+  const uint32_t full0 = smem_u32(bars);   // used in the even CTA only
+  const uint32_t empty0 = full0 + 8 * S;   // one per group of G stages, in both CTAs
+  const uint32_t accf0 = empty0 + 8 * (S / G);
   const uint32_t acce0 = accf0 + 16;
-  const uint32_t ringA = smem_u32(smem);
-  const uint32_t ringB = ringA + L::kARing;
+  const uint32_t ring = smem_u32(smem);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -64,14 +63,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint32_t *status = p.status;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SA; ++s) {
-      mbar_init(fullA0 + 8 * s, 1);
-      mbar_init(emptyA0 + 8 * s, 1);
-    }
-    for (int s = 0; s < SB; ++s) {
-      mbar_init(fullB0 + 8 * s, 1);
-      mbar_init(emptyB0 + 8 * s, 1);
-    }
+    for (int s = 0; s < S; ++s) mbar_init(full0 + 8 * s, 2);
+    for (int g = 0; g < S / G; ++g) mbar_init(empty0 + 8 * g, 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf0 + 8 * a, 1);
       mbar_init(acce0 + 8 * a, 8);
@@ -95,10 +88,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 || warp == 6) {
     if (lane == 0) {
       const bool isA = warp == 0;
-      const int S = isA ? SA : SB;
-      const uint32_t full0 = isA ? fullA0 : fullB0, empty0 = isA ? emptyA0 : emptyB0;
-      const uint32_t ring = isA ? ringA : ringB;
-      const uint32_t sbytes = isA ? P::kABytes : P::kBBytesMax;
       P::prefetch(p);
       int s = 0;
       uint32_t ph = 0;
@@ -106,22 +95,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const Unit U = P::unit(p, u, aux);
         const uint32_t pair_bytes = isA ? 2u * P::kABytes : P::b_bytes_pair(p, U);
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, status)) goto done;
+          if (s % G == 0 && !mbar_wait(empty0 + 8 * (s / G), ph ^ 1, abort_flag, status)) goto done;
           const uint32_t full_local = full0 + 8 * s;
           if (leader) mbar_arrive_expect_tx(full_local, pair_bytes);
           const uint32_t full_cl = mapa_shared(full_local, 0);
+          const uint32_t st = ring + s * L::kStageBytes;
           if (isA)
-            P::load_a(p, U, kb, ring + s * sbytes, full_cl, rank);
+            P::load_a(p, U, kb, st, full_cl, rank);
           else
-            P::load_b(p, U, kb, ring + s * sbytes, full_cl, rank);
+            P::load_b(p, U, kb, st + P::kABytes, full_cl, rank);
           if (++s == S) { s = 0; ph ^= 1; }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      int sa = 0, sb = 0, acc = 0;
-      uint32_t pa = 0, pb = 0, aph = 0;
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
       for (int u = cid; u < nunits; u += ncl) {
         const Unit U = P::unit(p, u, aux);
         if (!mbar_wait(acce0 + 8 * acc, aph ^ 1, abort_flag, status)) goto done;
@@ -129,18 +119,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const uint32_t tacc = tmem_base + acc * kAccCols;
         const uint32_t idesc = P::idesc(p, U);
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(fullA0 + 8 * sa, pa, abort_flag, status)) goto done;
-          if (!mbar_wait(fullB0 + 8 * sb, pb, abort_flag, status)) goto done;
+          if (!mbar_wait(full0 + 8 * s, ph, abort_flag, status)) goto done;
           tc_fence_after();
-          const uint32_t a_s = ringA + sa * P::kABytes;
-          const uint32_t b_s = ringB + sb * P::kBBytesMax;
+          const uint32_t a_s = ring + s * L::kStageBytes;
+          const uint32_t b_s = a_s + P::kABytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_f16_pair(tacc, sdesc_sw128(a_s + kk * 32), sdesc_sw128(b_s + kk * 32), idesc, (kb | kk) != 0);
-          umma_commit_pair(emptyA0 + 8 * sa, 0x3);
-          umma_commit_pair(emptyB0 + 8 * sb, 0x3);
-          if (++sa == SA) { sa = 0; pa ^= 1; }
-          if (++sb == SB) { sb = 0; pb ^= 1; }
+          if (s % G == G - 1) umma_commit_pair(empty0 + 8 * (s / G), 0x3);
+          if (++s == S) { s = 0; ph ^= 1; }
         }
         umma_commit_pair(accf0 + 8 * acc, 0x3);
         acc ^= 1;
@@ -198,8 +185,8 @@ __device__ __forceinline__ void load_rows_half(const CUtensorMap *tm, const Unit
 // CTA r owns d_ff columns f0 = m*128 + r*64 .. +63 with the same gate/up row
 // interleave as GluPolicy, so its epilogue is the same.
 struct Glu2Policy {
-  static constexpr int kStagesA = 6;
-  static constexpr int kStagesB = 6;
+  static constexpr int kStages = 6;
+  static constexpr int kGroup = 2;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = (kBN / 2) * 128;
@@ -249,8 +236,8 @@ struct Glu2Policy {
 // expert down over a CTA pair: unit = (group, 256-wide d_lat slice, <= 256
 // tokens); CTA r owns output rows l = m*256 + r*128 .. +127.
 struct Down2Policy {
-  static constexpr int kStagesA = 6;
-  static constexpr int kStagesB = 6;
+  static constexpr int kStages = 6;
+  static constexpr int kGroup = 2;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = (kBN / 2) * 128;

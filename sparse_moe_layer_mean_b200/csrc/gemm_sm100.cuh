@@ -3,10 +3,8 @@
 // D[128 x N] += A[128 x K] * B[N x K]^T, both operands K-major bf16 staged by
 // SWIZZLE_128B TMA tile loads into shared memory; the fp32 accumulator lives
 // in tensor memory, double-buffered (2 x 256 columns) so the epilogue of one
-// tile overlaps the main loop of the next.  A and B have rings of their own
-// depths: the grouped expert GEMMs stream A (expert weights) from HBM and
-// re-read B (dispatched token rows) from L2, so A gets the deeper ring and
-// more HBM bytes stay in flight per SM.
+// tile overlaps the main loop of the next.  A and B are loaded by producer
+// warps of their own into the same ring stages.
 //
 //   warp 0   : TMA producer for A (one thread)
 //   warp 1   : TMEM allocator + UMMA issuer (one thread issues, commits)
@@ -53,12 +51,19 @@ __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
   return r != 0;
 }
 
+// Ring: P::kStages stages, each holding one 64-wide K block of A and of B.
+// A stage's full barrier completes when both producers' loads have landed
+// (arrival count 2 plus the transaction bytes).  Stages are released in
+// groups of P::kGroup by a single tcgen05.commit: every commit costs the MMA
+// pipe about 100 cycles, so committing once per group instead of once per
+// operand per stage keeps the tensor pipe busy.
 template <class P>
 struct GemmSmem {
-  static constexpr int kARing = P::kStagesA * P::kABytes;
-  static constexpr int kBRing = P::kStagesB * P::kBBytesMax;
-  static constexpr int kBarOff = kARing + kBRing;
-  static constexpr int kNumBars = 2 * P::kStagesA + 2 * P::kStagesB + 4;
+  static_assert(P::kStages % P::kGroup == 0, "ring depth must be a multiple of the release group");
+  static constexpr int kStageBytes = P::kABytes + P::kBBytesMax;
+  static constexpr int kRing = P::kStages * kStageBytes;
+  static constexpr int kBarOff = kRing;
+  static constexpr int kNumBars = P::kStages + P::kStages / P::kGroup + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kEpiOff = (kMiscOff + 16 + 127) & ~127;
   static constexpr int kAuxOff = (kEpiOff + P::kEpiSmem + 127) & ~127;
@@ -68,7 +73,7 @@ struct GemmSmem {
 template <class P>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ typename P::Params p) {
   using L = GemmSmem<P>;
-  constexpr int SA = P::kStagesA, SB = P::kStagesB;
+  constexpr int S = P::kStages, G = P::kGroup;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
@@ -77,28 +82,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint8_t *epi_smem = smem + L::kEpiOff;
   uint8_t *aux = smem + L::kAuxOff;  // per-launch tables staged once per CTA
 
-  const uint32_t fullA0 = smem_u32(bars);
-  const uint32_t emptyA0 = fullA0 + 8 * SA;
-  const uint32_t fullB0 = emptyA0 + 8 * SA;
-  const uint32_t emptyB0 = fullB0 + 8 * SB;
-  const uint32_t accf0 = emptyB0 + 8 * SB;
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * S;  // one per group of G stages
+  const uint32_t accf0 = empty0 + 8 * (S / G);
   const uint32_t acce0 = accf0 + 16;
-  const uint32_t ringA = smem_u32(smem);
-  const uint32_t ringB = ringA + L::kARing;
+  const uint32_t ring = smem_u32(smem);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   uint32_t *status = p.status;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SA; ++s) {
-      mbar_init(fullA0 + 8 * s, 1);
-      mbar_init(emptyA0 + 8 * s, 1);
-    }
-    for (int s = 0; s < SB; ++s) {
-      mbar_init(fullB0 + 8 * s, 1);
-      mbar_init(emptyB0 + 8 * s, 1);
-    }
+    for (int s = 0; s < S; ++s) mbar_init(full0 + 8 * s, 2);
+    for (int g = 0; g < S / G; ++g) mbar_init(empty0 + 8 * g, 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf0 + 8 * a, 1);
       mbar_init(acce0 + 8 * a, 4);
@@ -120,12 +116,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 
   if (warp == 0 || warp == 6) {
     if (lane == 0) {
-      // producers: warp 0 fills the A ring, warp 6 the B ring
+      // producers: warp 0 loads A, warp 6 loads B, into the same stages
       const bool isA = warp == 0;
-      const int S = isA ? SA : SB;
-      const uint32_t full0 = isA ? fullA0 : fullB0, empty0 = isA ? emptyA0 : emptyB0;
-      const uint32_t ring = isA ? ringA : ringB;
-      const uint32_t sbytes = isA ? P::kABytes : P::kBBytesMax;
       P::prefetch(p);
       int s = 0;
       uint32_t ph = 0;
@@ -134,12 +126,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         for (int sub = 0; sub < U.nsub; ++sub) {
           const uint32_t bytes = isA ? P::kABytes : P::b_bytes(p, U, sub);
           for (int kb = 0; kb < kblocks; ++kb) {
-            if (!mbar_wait(empty0 + 8 * s, ph ^ 1, abort_flag, status)) goto done;
+            if (s % G == 0 && !mbar_wait(empty0 + 8 * (s / G), ph ^ 1, abort_flag, status)) goto done;
             mbar_arrive_expect_tx(full0 + 8 * s, bytes);
+            const uint32_t st = ring + s * L::kStageBytes;
             if (isA)
-              P::load_a(p, U, sub, kb, ring + s * sbytes, full0 + 8 * s);
+              P::load_a(p, U, sub, kb, st, full0 + 8 * s);
             else
-              P::load_b(p, U, sub, kb, ring + s * sbytes, full0 + 8 * s);
+              P::load_b(p, U, sub, kb, st + P::kABytes, full0 + 8 * s);
             if (++s == S) { s = 0; ph ^= 1; }
           }
         }
@@ -147,8 +140,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      int sa = 0, sb = 0, acc = 0;
-      uint32_t pa = 0, pb = 0, aph = 0;
+      int s = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         const Unit U = P::unit(p, u, aux);
         for (int sub = 0; sub < U.nsub; ++sub) {
@@ -157,19 +150,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           const uint32_t tacc = tmem_base + acc * kAccCols;
           const uint32_t idesc = P::idesc(p, U, sub);
           for (int kb = 0; kb < kblocks; ++kb) {
-            if (!mbar_wait(fullA0 + 8 * sa, pa, abort_flag, status)) goto done;
-            if (!mbar_wait(fullB0 + 8 * sb, pb, abort_flag, status)) goto done;
+            if (!mbar_wait(full0 + 8 * s, ph, abort_flag, status)) goto done;
             tc_fence_after();
-            const uint32_t a_s = ringA + sa * P::kABytes;
-            const uint32_t b_s = ringB + sb * P::kBBytesMax;
+            const uint32_t a_s = ring + s * L::kStageBytes;
+            const uint32_t b_s = a_s + P::kABytes;
 #pragma unroll
             for (int kk = 0; kk < kBK * 2 / P::kUmmaKBytes; ++kk)
               P::mma(tacc, sdesc_sw128(a_s + kk * P::kUmmaKBytes), sdesc_sw128(b_s + kk * P::kUmmaKBytes),
                      idesc, (kb | kk) != 0);
-            umma_commit(emptyA0 + 8 * sa);
-            umma_commit(emptyB0 + 8 * sb);
-            if (++sa == SA) { sa = 0; pa ^= 1; }
-            if (++sb == SB) { sb = 0; pb ^= 1; }
+            if (s % G == G - 1) umma_commit(empty0 + 8 * (s / G));
+            if (++s == S) { s = 0; ph ^= 1; }
           }
           umma_commit(accf0 + 8 * acc);
           acc ^= 1;

@@ -19,8 +19,8 @@ __device__ __forceinline__ int round16(int n) { return (n + 15) & ~15; }
 
 // ---------------------------------------------------------------- dense
 struct DensePolicy {
-  static constexpr int kStagesA = 4;
-  static constexpr int kStagesB = 4;
+  static constexpr int kStages = 4;
+  static constexpr int kGroup = 2;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
@@ -114,8 +114,8 @@ struct DensePolicy {
 // given as bf16 hi + bf16 lo parts and the K loop runs over both (2 * d_lat),
 // reusing each router tile for the hi and the lo half.
 struct RouterPolicy {
-  static constexpr int kStagesA = 4;
-  static constexpr int kStagesB = 4;
+  static constexpr int kStages = 4;
+  static constexpr int kGroup = 2;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = 256 * 128;
   static constexpr int kEpiSmem = 0;
@@ -294,8 +294,8 @@ __device__ __forceinline__ void load_rows(const CUtensorMap *tm, const Unit &U, 
 // each warp therefore owns complete (gate, up) pairs and pairs them with one
 // shuffle across the half-warps.
 struct GluPolicy {
-  static constexpr int kStagesA = 7;
-  static constexpr int kStagesB = 3;
+  static constexpr int kStages = 4;
+  static constexpr int kGroup = 2;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
@@ -376,8 +376,8 @@ struct GluPolicy {
 
 // ------------------------------------------------------------------ down
 struct DownPolicy {
-  static constexpr int kStagesA = 7;
-  static constexpr int kStagesB = 3;
+  static constexpr int kStages = 4;
+  static constexpr int kGroup = 2;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
