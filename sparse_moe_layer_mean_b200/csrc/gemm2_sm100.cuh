@@ -182,15 +182,19 @@ __device__ __forceinline__ void load_rows_half(const CUtensorMap *tm, const Unit
 }
 
 // gate/up over a CTA pair: unit = (group, 128-wide d_ff slice, <= 256 tokens);
-// CTA r owns d_ff columns f0 = m*128 + r*64 .. +63 with the same gate/up row
-// interleave as GluPolicy, so its epilogue is the same.
+// CTA r owns d_ff columns f0 = m*128 + r*64 .. +63: its A tile is 64 gate
+// rows (TMEM lanes 0-63) then the 64 matching up rows (lanes 64-127), two
+// 64-row TMA boxes per K block (a 64-row box streams at full HBM rate; 16-row
+// boxes did not).  In the epilogue, warp pair (q, q+2) swaps half of each
+// 32-token chunk through shared memory so each warp owns complete (gate, up)
+// pairs for 16 of the chunk's tokens.
 struct Glu2Policy {
   static constexpr int kStages = 6;
   static constexpr int kGroup = 2;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = (kBN / 2) * 128;
-  static constexpr int kEpiSmem = 0;
+  static constexpr int kEpiSmem = 4 * 32 * 17 * 4;
   static constexpr int kAuxSmem = kGroupAuxSmem;
   using Params = GluPolicy::Params;
   static __device__ __forceinline__ void prefetch(const Params &p) { GluPolicy::prefetch(p); }
@@ -208,14 +212,9 @@ struct Glu2Policy {
   static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int kb, uint32_t sa,
                                                 uint32_t bar_cl, uint32_t rank) {
     const bool sh = U.g == p.gt.E;
-    const CUtensorMap *mg = sh ? &p.sg : &p.wg;
-    const CUtensorMap *mu = sh ? &p.su : &p.wu;
     const int row = (sh ? 0 : U.g * p.F) + U.m * 128 + static_cast<int>(rank) * 64;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      tma_load_2d_pair(sa + (32 * q) * 128, mg, bar_cl, kb * kBK, row + 16 * q);
-      tma_load_2d_pair(sa + (32 * q + 16) * 128, mu, bar_cl, kb * kBK, row + 16 * q);
-    }
+    tma_load_2d_pair(sa, sh ? &p.sg : &p.wg, bar_cl, kb * kBK, row);
+    tma_load_2d_pair(sa + 64 * 128, sh ? &p.su : &p.wu, bar_cl, kb * kBK, row);
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb,
                                                 uint32_t bar_cl, uint32_t rank) {
@@ -226,10 +225,29 @@ struct Glu2Policy {
   }
   static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, uint32_t taddr, int q, int lane,
                                                   int etid, uint32_t rank, uint8_t *epi) {
-    Unit V = U;
-    V.m = U.m * 2 + static_cast<int>(rank);  // the CTA's 64-wide d_ff slice
-    GluPolicy::EpiState st;
-    GluPolicy::epilogue(p, V, 0, taddr, q, lane, etid, st, epi);
+    float *xb = reinterpret_cast<float *>(epi);  // [4][32][17]
+    const bool is_gate = q < 2;
+    const int pair = q & 1;
+    const int f = (U.m * 2 + static_cast<int>(rank)) * 64 + pair * 32 + lane;
+    const size_t row0 = static_cast<size_t>(U.row0);
+    for (int c0 = 0; c0 < U.nv; c0 += 32) {
+      float v[32];
+      tmem_ld32(taddr + c0, v);
+      tmem_ld_wait();
+      float *mine = xb + (q * 32 + lane) * 17;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) mine[c] = is_gate ? v[16 + c] : v[c];
+      named_bar_sync(2, 128);
+      const float *other = xb + (((q + 2) & 3) * 32 + lane) * 17;
+      const int cbase = c0 + (is_gate ? 0 : 16);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float g = is_gate ? v[c] : other[c];
+        const float u = is_gate ? other[c] : v[16 + c];
+        if (cbase + c < U.nv) p.h[(row0 + cbase + c) * p.F + f] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
+      }
+      named_bar_sync(2, 128);
+    }
   }
 };
 

@@ -303,8 +303,8 @@ struct GluPolicy {
   static constexpr int kAuxSmem = kGroupAuxSmem;
   static constexpr int kUmmaKBytes = 32;
   struct Params {
-    CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 16
-    CUtensorMap sg, su;  // shared gate/up [F, L], box 64 x 16
+    CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 64 (pairs) / 64 x 16 (single CTA)
+    CUtensorMap sg, su;  // shared gate/up [F, L], box 64 x 64 (pairs) / 64 x 16 (single CTA)
     CUtensorMap tz;      // dispatched z [(T*k+T), L], box 64 x 32
     GroupTable gt;
     __nv_bfloat16 *h;    // [(T*k+T), F]
