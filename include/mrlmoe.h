@@ -51,7 +51,9 @@ typedef enum {
   MRLMOE_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned  */
   MRLMOE_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed         */
   MRLMOE_ERR_TIMEOUT = 5,       /* device: a bounded wait gave up              */
-  MRLMOE_ERR_CHECK = 6          /* device: a consistency check failed          */
+  MRLMOE_ERR_CHECK = 6,         /* device: a consistency check failed          */
+  MRLMOE_ERR_SCRATCH_LIMIT = 7  /* problem larger than the built-in scratch of
+                                   mrlmoe_route_scores_static                    */
 } mrlmoe_status;
 
 typedef enum {
@@ -169,6 +171,27 @@ mrlmoe_status mrlmoe_bias_update(const mrlmoe_config *cfg, const int32_t *counts
  * on their own.  M >= 1; N, K multiples of 128.  No workspace.               */
 mrlmoe_status mrlmoe_linear(const void *a, const void *w, void *out,
                             int M, int N, int K, void *stream);
+
+/* Routing from caller-given fp32 scores WITHOUT a workspace (no counterpart in
+ * the paper: an entry point for callers that cannot allocate device memory,
+ * e.g. code running inside a framework that owns every allocation, or a
+ * graph of pre-planned buffers).  Same results as mrlmoe_route with
+ * scores_in = 1: out->scores holds s [T, E]; out->topk_idx, topk_w, counts,
+ * offsets, perm and inv_perm must all be non-NULL and receive the record.
+ * Its scratch (per-chunk expert masks and prefixes, scaled weights, group
+ * tables) lives in one static device array of MRLMOE_STATIC_SCRATCH_BYTES
+ * that every GPU which loads this library holds until process exit; the
+ * library allocates nothing.  Problems whose scratch would not fit (about
+ * T * (8*E/32 + 4*k) bytes) are rejected with MRLMOE_ERR_SCRATCH_LIMIT before
+ * anything is enqueued.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  All calls share the one array, so calls that overlap on
+ * the GPU (different streams, or graphs replayed concurrently) race: order
+ * them on one stream.                                                        */
+#define MRLMOE_STATIC_SCRATCH_BYTES (2u * 1024u * 1024u)
+mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *bias,
+                                         const float *expert_scale, mrlmoe_routing *out,
+                                         void *stream);
 
 /* Synchronises `stream`, then returns the device status word of `workspace`
  * written by the last call that used it (MRLMOE_OK if none failed).          */

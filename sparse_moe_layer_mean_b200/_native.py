@@ -20,11 +20,12 @@ MRLMOE_FP8_E4M3_BLOCK128 = 1
 
 STATUS = {0: "MRLMOE_OK", 1: "MRLMOE_ERR_INVALID_ARG", 2: "MRLMOE_ERR_UNSUPPORTED",
           3: "MRLMOE_ERR_WORKSPACE", 4: "MRLMOE_ERR_CUDA", 5: "MRLMOE_ERR_TIMEOUT",
-          6: "MRLMOE_ERR_CHECK"}
+          6: "MRLMOE_ERR_CHECK", 7: "MRLMOE_ERR_SCRATCH_LIMIT"}
 
 EXPORTED = ("mrlmoe_workspace_size", "mrlmoe_route", "mrlmoe_forward", "mrlmoe_forward_timed",
             "mrlmoe_bias_update", "mrlmoe_linear", "mrlmoe_get_device_status",
-            "mrlmoe_status_string")
+            "mrlmoe_status_string", "mrlmoe_route_scores_static")
+STATIC_SCRATCH_BYTES = 2 * 1024 * 1024
 NUM_STAGE_EVENTS = 9
 STAGES = ("down_proj", "router_topk", "dispatch", "gather", "gate_up_glu", "expert_down",
           "combine_rmsnorm", "up_proj")
@@ -85,6 +86,9 @@ def lib() -> ctypes.CDLL:
         L.mrlmoe_bias_update.restype = c_int
         L.mrlmoe_linear.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]
         L.mrlmoe_linear.restype = c_int
+        L.mrlmoe_route_scores_static.argtypes = [POINTER(Config), c_void_p, c_void_p, POINTER(Routing),
+                                                 c_void_p]
+        L.mrlmoe_route_scores_static.restype = c_int
         L.mrlmoe_get_device_status.argtypes = [c_void_p, c_void_p]
         L.mrlmoe_get_device_status.restype = c_int
         L.mrlmoe_status_string.argtypes = [c_int]
@@ -180,6 +184,13 @@ def mrlmoe_bias_update(cfg: Config, counts, bias, gamma: float, stream=None) -> 
 def mrlmoe_linear(a, w, out, M: int, N: int, K: int, stream=None) -> None:
     _check(lib().mrlmoe_linear(_ptr(a), _ptr(w), _ptr(out), int(M), int(N), int(K),
                                _stream_ptr(stream)), "mrlmoe_linear")
+
+
+def mrlmoe_route_scores_static(cfg: Config, bias, expert_scale, routing: Routing, stream=None) -> None:
+    """Routing from given scores with the library's static scratch (no workspace)."""
+    _check(lib().mrlmoe_route_scores_static(ctypes.byref(cfg), _ptr(bias), _ptr(expert_scale),
+                                            ctypes.byref(routing), _stream_ptr(stream)),
+           "mrlmoe_route_scores_static")
 
 
 def mrlmoe_get_device_status(workspace, stream=None) -> int:

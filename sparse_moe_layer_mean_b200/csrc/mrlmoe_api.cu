@@ -413,6 +413,55 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   return MRLMOE_OK;
 }
 
+// ------------------------------------------------ static-scratch routing
+// Scratch for mrlmoe_route_scores_static: one array per device that loads
+// the library.  Host code never dereferences this symbol; it asks the runtime
+// for the device address once per device (static_scratch()).
+static __device__ __align__(256) uint8_t g_route_scratch[MRLMOE_STATIC_SCRATCH_BYTES];
+
+struct StaticRouteLayout {
+  size_t status, wscaled, counts, grp_off, grp_cnt, unit1, unit2, mask, base, total;
+};
+
+StaticRouteLayout static_route_layout(const mrlmoe_config &c) {
+  StaticRouteLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  };
+  const size_t T = c.T, k = c.top_k, E = c.n_experts, nch = (T + kChunk - 1) / kChunk;
+  L.status = take(256);
+  L.wscaled = take(T * k * 4);
+  L.counts = take((E + 2) * 4);
+  L.grp_off = take((E + 2) * 4);
+  L.grp_cnt = take((E + 2) * 4);
+  L.unit1 = take((E + 2) * 4);
+  L.unit2 = take((E + 2) * 4);
+  L.mask = take(nch * E * 4);
+  L.base = take(nch * E * 4);
+  L.total = off;
+  return L;
+}
+
+// Device address of g_route_scratch on the current device (looked up once per
+// device, with that device current).  nullptr if the lookup failed.
+uint8_t *static_scratch(int dev) {
+  static std::mutex mu;
+  static uint8_t *addr[kMaxDevices] = {nullptr};
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<uint8_t *>(p);
+  }
+  return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -431,6 +480,7 @@ const char *mrlmoe_status_string(mrlmoe_status s) {
     case MRLMOE_ERR_CUDA: return "CUDA runtime error";
     case MRLMOE_ERR_TIMEOUT: return "device wait timed out";
     case MRLMOE_ERR_CHECK: return "device consistency check failed";
+    case MRLMOE_ERR_SCRATCH_LIMIT: return "problem exceeds the static scratch of mrlmoe_route_scores_static";
   }
   return "unknown status";
 }
@@ -511,6 +561,48 @@ mrlmoe_status mrlmoe_linear(const void *a, const void *w, void *out, int M, int 
   p.status = nullptr;
   MRL_TRY(launch_gemm<DensePolicy>(p, std::min(sms, p.m_tiles * p.n_tiles), static_cast<cudaStream_t>(stream)));
   return MRLMOE_OK;
+}
+
+mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *bias, const float *expert_scale,
+                                         mrlmoe_routing *out, void *stream) {
+  mrlmoe_status s = check_config(cfg);
+  if (s != MRLMOE_OK) return s;
+  if (!bias || !expert_scale || !out || !out->scores || !out->topk_idx || !out->topk_w || !out->counts ||
+      !out->offsets || !out->perm || !out->inv_perm)
+    return MRLMOE_ERR_INVALID_ARG;
+  const StaticRouteLayout SL = static_route_layout(*cfg);
+  if (SL.total > MRLMOE_STATIC_SCRATCH_BYTES) return MRLMOE_ERR_SCRATCH_LIMIT;
+  int sms = 0;
+  if ((s = bind_device(out->scores, &sms)) != MRLMOE_OK) return s;
+  int dev = 0;
+  MRL_TRY(cudaGetDevice(&dev));
+  uint8_t *b = static_scratch(dev);
+  if (!b) return MRLMOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Ptrs P{};
+  P.status = reinterpret_cast<uint32_t *>(b + SL.status);
+  P.topk_idx = out->topk_idx;
+  P.topk_w = out->topk_w;
+  P.wscaled = reinterpret_cast<float *>(b + SL.wscaled);
+  P.counts_e = reinterpret_cast<int32_t *>(b + SL.counts);
+  P.grp_off = reinterpret_cast<int32_t *>(b + SL.grp_off);
+  P.grp_cnt = reinterpret_cast<int32_t *>(b + SL.grp_cnt);
+  P.unit1 = reinterpret_cast<int32_t *>(b + SL.unit1);
+  P.unit2 = reinterpret_cast<int32_t *>(b + SL.unit2);
+  P.perm = out->perm;
+  P.inv = out->inv_perm;
+  P.mask = reinterpret_cast<uint32_t *>(b + SL.mask);
+  P.base = reinterpret_cast<int32_t *>(b + SL.base);
+  P.out_counts = out->counts;
+  P.out_offsets = out->offsets;
+  // the array keeps the previous call's contents: the status word must start
+  // at zero; every other region is fully rewritten below before it is read
+  MRL_TRY(cudaMemsetAsync(P.status, 0, 4, st));
+  const int warps_per_block = 8;
+  topk_from_scores_kernel<kTopKMax><<<(cfg->T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, st>>>(
+      out->scores, bias, expert_scale, cfg->T, cfg->n_experts, cfg->top_k, P.topk_idx, P.topk_w, P.wscaled);
+  MRL_TRY(cudaGetLastError());
+  return launch_dispatch(*cfg, P, st);
 }
 
 mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream) {
