@@ -188,3 +188,25 @@ def test_bias_update_bit_exact():
     torch.cuda.synchronize()
     ref = O.bias_update(bias, counts, T, k, 1e-3)
     assert torch.equal(b_dev.cpu().view(torch.int32), ref.view(torch.int32))
+
+
+def test_forward_c3_skew_sampled_tokens_and_bias_update():
+    s = W.CONFIGS["c3_skew"]
+    bias = W.make_bias(s, "cuda")
+    s, x, bias, y, r, layer = _run_layer("c3_skew", bias=bias, scores=False)
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+    counts = r["counts"].cpu().long()
+    ratio = (counts.max().double() / counts.double().mean()).item()
+    assert 20.0 < ratio < 45.0, ratio          # Zipf(1.1) skew, fitted to ~30x on the oracle
+    tokens = torch.tensor([0, 5, 4095, 16384, 30001, 32767])
+    _compare_layer(s, x, bias, y, r, host_weights("c3_skew"), tokens=tokens)
+    # one balancing step: every bias moves by exactly +-gamma or 0, against the load
+    gamma = 1e-3
+    b0 = bias.clone()
+    M.mrlmoe_bias_update(layer.cfg, r["counts"], bias, gamma)
+    torch.cuda.synchronize()
+    d = (bias - b0).cpu()
+    sgn = torch.sign(torch.tensor(s.T * s.top_k) - s.n_experts * counts)
+    want = (b0.cpu() + torch.tensor(gamma, dtype=torch.float32) * sgn.float()) - b0.cpu()
+    assert torch.equal(d, want)
+    assert int((sgn < 0).sum()) > 0 and int((sgn > 0).sum()) > 0
