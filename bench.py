@@ -46,7 +46,8 @@ def kernels_per_step(s, sms: int) -> int:
     parts = 1
     while parts * 2 <= chunks and chunks % (parts * 2) == 0 and m_tiles * parts * 2 <= sms:
         parts *= 2
-    return KERNELS_PER_STEP + (1 if parts > 1 else 0)
+    # FP8 variant: the x, h and n quantisers replace nothing and the z quantiser replaces the gather
+    return KERNELS_PER_STEP + (1 if parts > 1 else 0) + (3 if s.fp8 else 0)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -197,8 +198,9 @@ def layer_bytes_flops(s, counts):
     import workloads as W
     touched = int((counts > 0).sum())
     D, L, E, F, R, T = s.d_model, s.d_lat, s.n_experts, s.d_ff, s.n_routers, s.T
-    expert = 3 * F * L * 2
-    byts = (touched + 1) * expert + (L * D + R * E * L + D * L) * 2 + L * 4 + 2 * T * D * 2
+    wb = 1 if s.fp8 else 2                       # bytes per expert / projection weight
+    expert = 3 * F * L * wb
+    byts = (touched + 1) * expert + (L * D + D * L) * wb + R * E * L * 2 + L * 4 + 2 * T * D * 2
     return byts, W.flops_per_token(s) * T, touched
 
 
@@ -207,7 +209,13 @@ def glu_kernel_bytes(s, touched):
     of the touched experts and the shared expert, the dispatched latent rows
     read once, and h written once."""
     rows = s.T * s.top_k + s.T
-    return (touched + 1) * 2 * s.d_ff * s.d_lat * 2 + rows * s.d_lat * 2 + rows * s.d_ff * 2
+    wb = 1 if s.fp8 else 2
+    return (touched + 1) * 2 * s.d_ff * s.d_lat * wb + rows * s.d_lat * wb + rows * s.d_ff * 2
+
+
+def glu_kernel_flops(s):
+    """FLOPs of one gate/up launch: 2 * rows * d_lat * 2 d_ff."""
+    return 2 * (s.T * s.top_k + s.T) * s.d_lat * 2 * s.d_ff
 
 
 def cpu_baseline(s, weights_dev, x_dev, bias_dev, ntok):
@@ -218,7 +226,7 @@ def cpu_baseline(s, weights_dev, x_dev, bias_dev, ntok):
     xs = x_dev[:ntok].cpu()
     b = bias_dev.cpu()
     t0 = time.perf_counter()
-    O.forward(xs, wh, b, s.top_k, s.rms_eps)
+    O.forward(xs, wh, b, s.top_k, s.rms_eps, fp8=s.fp8)
     dt = time.perf_counter() - t0
     return {"value": ntok / dt, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
             "sample": f"first {ntok} tokens of the {s.name} batch (fp64 oracle, {dt:.1f} s)"}
@@ -235,17 +243,17 @@ def run_reference(args):
     import workloads as W
     s = shape_from_args(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    w = {k: v.cpu() for k, v in W.make_weights(s, dev).items()}
+    w = {k: v.cpu() for k, v in (W.make_weights_fp8 if s.fp8 else W.make_weights)(s, dev).items()}
     per_step = 1
     n = args.warmup + args.steps
     x = W.make_x(s, dev, T=min(s.T, n * per_step)).cpu()
     b = W.make_bias(s, "cpu")
     for i in range(args.warmup):
-        O.forward(x[i:i + 1], w, b, s.top_k, s.rms_eps)
+        O.forward(x[i:i + 1], w, b, s.top_k, s.rms_eps, fp8=s.fp8)
     t0 = time.perf_counter()
     for i in range(args.steps):
         j = (args.warmup + i) % x.shape[0]
-        O.forward(x[j:j + per_step], w, b, s.top_k, s.rms_eps)
+        O.forward(x[j:j + per_step], w, b, s.top_k, s.rms_eps, fp8=s.fp8)
     dt = time.perf_counter() - t0
     v = args.steps * per_step / dt
     line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
@@ -278,7 +286,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     s = shape_from_args(args)
-    weights = W.make_weights(s, dev)
+    weights = (W.make_weights_fp8 if s.fp8 else W.make_weights)(s, dev)
     x = W.make_x(s, dev, seed=s.seed + rank)
     bias = W.make_bias(s, dev)
     layer = M.MRLMoELayer(s, weights, device=dev)
@@ -365,16 +373,20 @@ def main():
         peaks, peak_kind = load_peaks()
         glu_ms = stage_ms[M._native.STAGES.index("gate_up_glu")]
         glu_bytes = glu_kernel_bytes(s, touched)
+        glu_flops = glu_kernel_flops(s)
+        # the gate/up kernel's bound: HBM bytes or tensor FLOPs (FP8 peak taken as 2x bf16)
+        tensor_peak = peaks["bf16_tflops_sustained"] * (2 if s.fp8 else 1)
+        glu_tensor_bound = glu_flops / (tensor_peak * 1e12) > glu_bytes / (peaks["hbm_gbs"] * 1e9)
         achieved = glu_bytes / (glu_ms * 1e-3) / 1e9
         step_s = ms / args.steps * 1e-3
         t_bytes = byts / (peaks["hbm_gbs"] * 1e9)
-        t_flops = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+        t_flops = flops / (peaks["bf16_tflops_sustained"] * (2 if s.fp8 else 1) * 1e12)
         workload = s.name
         line = {
             "metric": METRIC, "value": job_throughput(world, s.T, args.steps, ms), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "e4m3" if s.fp8 else "bf16", "data": "synthetic",
             "config": {
                 "workload": f"{workload}: T={s.T} tokens, d_model {s.d_model} -> d_lat {s.d_lat}, "
                             f"{s.n_experts} experts top-{s.top_k} + 1 shared, d_ff {s.d_ff}, "
@@ -389,11 +401,19 @@ def main():
                                    "peaks": peak_kind},
                 "stage_ms": dict(zip(M._native.STAGES, [round(v, 4) for v in stage_ms])),
             },
-            "roofline": {"kernel": "gate_up_glu (grouped tcgen05 GEMM, SiLU-GLU epilogue)",
-                         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": profiled_traffic("gate_up_glu", workload),
-                         "algorithmic_bytes": glu_bytes, "peak_kind": f"of {peak_kind}"},
+            "roofline": ({"kernel": "gate_up_glu (grouped tcgen05 GEMM, SiLU-GLU epilogue)",
+                          "bound": "tensor", "achieved": glu_flops / (glu_ms * 1e-3) / 1e12,
+                          "peak": tensor_peak, "unit": "TFLOP/s",
+                          "frac": glu_flops / (glu_ms * 1e-3) / 1e12 / tensor_peak,
+                          "traffic": profiled_traffic("gate_up_glu", workload),
+                          "algorithmic_flops": glu_flops,
+                          "peak_kind": f"of {peak_kind} (sustained bf16" + (" x 2 for e4m3, assumed)" if s.fp8 else ")")}
+                         if glu_tensor_bound else
+                         {"kernel": "gate_up_glu (grouped tcgen05 GEMM, SiLU-GLU epilogue)",
+                          "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                          "traffic": profiled_traffic("gate_up_glu", workload),
+                          "algorithmic_bytes": glu_bytes, "peak_kind": f"of {peak_kind}"}),
             "clocks": clk,
             "gpu_launches": kernels_per_step(s, torch.cuda.get_device_properties(dev).multi_processor_count)
             * args.steps,

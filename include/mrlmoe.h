@@ -193,6 +193,15 @@ mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *
                                          const float *expert_scale, mrlmoe_routing *out,
                                          void *stream);
 
+/* FP8 activation quantiser of the FP8 variant: for each row r and 128-wide
+ * block b of in [rows, K] bf16 (K a multiple of 128), amax = max |v|;
+ * scale[r*K/128 + b] = amax / 448 (1 if amax == 0) and
+ * q[r*K + b*128 + i] = e4m3(v_i * 448 / amax) rounded to nearest even with
+ * saturation (0 if amax == 0).  q: [rows, K] e4m3 bytes; scale: fp32.
+ * The variant's reading of "activations quantised e4m3 per 1x128 block".    */
+mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, float *scale,
+                                   void *stream);
+
 /* Synchronises `stream`, then returns the device status word of `workspace`
  * written by the last call that used it (MRLMOE_OK if none failed).          */
 mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream);

@@ -33,7 +33,10 @@ the design notes):
   * RMSNorm eps 1e-6 with a learnable gain; no norm after the down-projection;
   * bias update b += gamma * sign(T*k - E*count[e]) with sign(0) = 0;
   * rounding points: z, h, n, y are bf16 (round to nearest even);
-    s, w, and the FP8 quantiser inputs are fp32; everything else fp64;
+    s, w fp32; everything else fp64;
+  * FP8 variant: every GEMM input is a bf16 tensor (x, z, h, n) quantised
+    per 1x128 block from those bf16 values; weights are e4m3 codes with fp32
+    scales per 128x128 block;
   * the routers read the latent before its bf16 rounding (the experts read
     bf16 z), so that top-k decisions do not hinge on bf16 rounding of z.
 PARITY UNPINNED by the pages: the choice of mean (vs sum/max), R=4, eps, gamma.
@@ -176,8 +179,8 @@ def expert_glu(zrows: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
     """One latent expert on its rows: h = bf16(SiLU(z W_g^T) * (z W_u^T)),
     o = h W_d^T (fp64).  Intermediate size d_ff, operating in the latent space
     [derekhsu, 潛在專家]; the gated activation is SiLU-GLU (reading of the
-    garbled "SiTU-GLU").  In FP8 mode the inputs z and h are fake-quantised per
-    1x128 block and h is not rounded to bf16; the weights passed are already
+    garbled "SiTU-GLU").  In FP8 mode the GEMM inputs (bf16 z, bf16 h) are
+    fake-quantised per 1x128 block and the weights passed are already
     dequantised.
     """
     a = _as_f64(zrows)
@@ -185,8 +188,9 @@ def expert_glu(zrows: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
         a = quantize_act_1x128(a)
     g = a @ _as_f64(w_gate).T
     u = a @ _as_f64(w_up).T
-    hv = g / (1.0 + torch.exp(-g)) * u
-    h = quantize_act_1x128(hv) if quant else bf16_round(hv)
+    h = bf16_round(g / (1.0 + torch.exp(-g)) * u)
+    if quant:
+        h = quantize_act_1x128(h)
     return h @ _as_f64(w_down).T
 
 
@@ -322,14 +326,14 @@ def forward(x: torch.Tensor, weights: Dict[str, torch.Tensor], bias: torch.Tenso
     12. y = bf16(n W_up^T)                         shared up-projection 2048 -> 4096
     ``scores`` replaces steps 1-3 with the given fp32 s (routing-only use; z,
     c, n and y are then not computed).  In FP8 mode ``weights`` carries e4m3
-    codes and 128x128 scales for every projection and expert matrix; the
-    router stays bf16.
+    codes for every projection and expert matrix w_<x> and its 128x128 block
+    scales as s_<x>; the routers stay bf16.
     """
     E = weights["expert_scale"].numel()
     deq = None
     if fp8:
         def mk(nm):
-            codes, sc = weights[nm], weights[nm + "_scale"]
+            codes, sc = weights[nm], weights["s_" + nm[2:]]   # scale array: w_<x> -> s_<x>
             if codes.dim() == 3:
                 return lambda e: dequantize_weight_128x128(codes[e], sc[e])
             return lambda: dequantize_weight_128x128(codes, sc)
@@ -362,12 +366,7 @@ def forward(x: torch.Tensor, weights: Dict[str, torch.Tensor], bias: torch.Tenso
         c.index_add_(0, tok, o * wsc[tok, slot].to(F64)[:, None])
     c += expert_glu(z, _w(weights, "w_sh_gate", deq), _w(weights, "w_sh_up", deq),
                     _w(weights, "w_sh_down", deq), quant=fp8)
-    nv = rmsnorm(c, weights["rms_gain"], rms_eps)
-    if fp8:
-        n = quantize_act_1x128(nv)
-        y = bf16_round(n @ _as_f64(_w(weights, "w_up", deq)).T)
-        n = bf16_round(nv)
-    else:
-        n = bf16_round(nv)
-        y = bf16_round(n @ _as_f64(_w(weights, "w_up", deq)).T)
+    n = bf16_round(rmsnorm(c, weights["rms_gain"], rms_eps))
+    nin = quantize_act_1x128(n) if fp8 else n
+    y = bf16_round(nin @ _as_f64(_w(weights, "w_up", deq)).T)
     return OracleResult(z, s, idx, w, counts, offsets, perm, inv, c, n, y)

@@ -12,13 +12,13 @@ from . import _native
 from ._native import (MRLMOE_BF16, MRLMOE_FP8_E4M3_BLOCK128, Config, MrlmoeError, Routing,
                       Weights, make_config, make_routing, make_weights, mrlmoe_bias_update,
                       mrlmoe_forward, mrlmoe_forward_timed, mrlmoe_get_device_status, mrlmoe_linear, mrlmoe_route,
-                      mrlmoe_route_scores_static,
+                      mrlmoe_route_scores_static, mrlmoe_quantize_e4m3,
                       mrlmoe_workspace_size, status_string)
 
 __all__ = ["MRLMoELayer", "Config", "Weights", "Routing", "MrlmoeError", "make_config",
            "make_weights", "make_routing", "mrlmoe_route", "mrlmoe_forward", "mrlmoe_forward_timed",
            "mrlmoe_bias_update", "mrlmoe_linear", "mrlmoe_workspace_size",
-           "mrlmoe_get_device_status", "mrlmoe_route_scores_static", "status_string", "MRLMOE_BF16",
+           "mrlmoe_get_device_status", "mrlmoe_route_scores_static", "mrlmoe_quantize_e4m3", "status_string", "MRLMOE_BF16",
            "MRLMOE_FP8_E4M3_BLOCK128"]
 
 

@@ -24,7 +24,7 @@ STATUS = {0: "MRLMOE_OK", 1: "MRLMOE_ERR_INVALID_ARG", 2: "MRLMOE_ERR_UNSUPPORTE
 
 EXPORTED = ("mrlmoe_workspace_size", "mrlmoe_route", "mrlmoe_forward", "mrlmoe_forward_timed",
             "mrlmoe_bias_update", "mrlmoe_linear", "mrlmoe_get_device_status",
-            "mrlmoe_status_string", "mrlmoe_route_scores_static")
+            "mrlmoe_status_string", "mrlmoe_route_scores_static", "mrlmoe_quantize_e4m3")
 STATIC_SCRATCH_BYTES = 2 * 1024 * 1024
 NUM_STAGE_EVENTS = 9
 STAGES = ("down_proj", "router_topk", "dispatch", "gather", "gate_up_glu", "expert_down",
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.mrlmoe_route_scores_static.argtypes = [POINTER(Config), c_void_p, c_void_p, POINTER(Routing),
                                                  c_void_p]
         L.mrlmoe_route_scores_static.restype = c_int
+        L.mrlmoe_quantize_e4m3.argtypes = [c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]
+        L.mrlmoe_quantize_e4m3.restype = c_int
         L.mrlmoe_get_device_status.argtypes = [c_void_p, c_void_p]
         L.mrlmoe_get_device_status.restype = c_int
         L.mrlmoe_status_string.argtypes = [c_int]
@@ -191,6 +193,11 @@ def mrlmoe_route_scores_static(cfg: Config, bias, expert_scale, routing: Routing
     _check(lib().mrlmoe_route_scores_static(ctypes.byref(cfg), _ptr(bias), _ptr(expert_scale),
                                             ctypes.byref(routing), _stream_ptr(stream)),
            "mrlmoe_route_scores_static")
+
+
+def mrlmoe_quantize_e4m3(x, rows: int, K: int, q, scale, stream=None) -> None:
+    _check(lib().mrlmoe_quantize_e4m3(_ptr(x), int(rows), int(K), _ptr(q), _ptr(scale), _stream_ptr(stream)),
+           "mrlmoe_quantize_e4m3")
 
 
 def mrlmoe_get_device_status(workspace, stream=None) -> int:

@@ -10,6 +10,7 @@
 #include "mrlmoe.h"
 #include "policies.cuh"
 #include "gemm2_sm100.cuh"
+#include "gemm8_sm100.cuh"
 #include "routing.cuh"
 
 using namespace mrl;
@@ -58,7 +59,7 @@ int router_parts(const mrlmoe_config &c, int sms) {
 // ------------------------------------------------------------ workspace
 struct Layout {
   size_t status, topk_idx, topk_w, wscaled, counts, offsets, grp_off, grp_cnt, unit1, unit2, perm, inv, mask,
-      base, cand_v, cand_s, cand_i, zbuf, zlo, hbuf, slots, nbuf, total;
+      base, cand_v, cand_s, cand_i, zbuf, zlo, hbuf, slots, nbuf, xq, xs, zq, zs, hq, hs, nq, ns, total;
 };
 
 Layout layout_of(const mrlmoe_config &c) {
@@ -94,6 +95,17 @@ Layout layout_of(const mrlmoe_config &c) {
   L.hbuf = take((Tk + T) * F * 2);
   L.slots = take(T * (k + 1) * Ld * 4);
   L.nbuf = take(T * Ld * 2);
+  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) {  // e4m3 copies of the GEMM inputs and their 1x128 scales
+    const size_t D = c.d_model;
+    L.xq = take(T * D);
+    L.xs = take(T * (D / 128) * 4);
+    L.zq = take((Tk + T) * Ld);
+    L.zs = take((Tk + T) * (Ld / 128) * 4);
+    L.hq = take((Tk + T) * F);
+    L.hs = take((Tk + T) * (F / 128) * 4);
+    L.nq = take(T * Ld);
+    L.ns = take(T * (Ld / 128) * 4);
+  }
   L.total = off;
   return L;
 }
@@ -205,6 +217,8 @@ struct Ptrs {
   int32_t *cand_i;
   uint32_t *mask;
   __nv_bfloat16 *zbuf, *zlo, *hbuf, *nbuf;
+  uint8_t *xq, *zq, *hq, *nq;  // FP8 variant only
+  float *xs, *zs, *hs, *ns;
   int32_t *out_counts, *out_offsets;
 };
 
@@ -234,16 +248,33 @@ Ptrs carve(const mrlmoe_config &c, void *ws, const mrlmoe_routing *r) {
   P.hbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.hbuf);
   P.slots = reinterpret_cast<float *>(b + L.slots);
   P.nbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.nbuf);
+  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) {
+    P.xq = b + L.xq; P.zq = b + L.zq; P.hq = b + L.hq; P.nq = b + L.nq;
+    P.xs = reinterpret_cast<float *>(b + L.xs);
+    P.zs = reinterpret_cast<float *>(b + L.zs);
+    P.hs = reinterpret_cast<float *>(b + L.hs);
+    P.ns = reinterpret_cast<float *>(b + L.ns);
+  }
   P.scores = r ? r->scores : nullptr;
   P.out_counts = r ? r->counts : nullptr;
   P.out_offsets = r ? r->offsets : nullptr;
   return P;
 }
 
-constexpr int kExpertBN = 256;  // token tile of the grouped GEMMs (GluPolicy/DownPolicy kBN)
+constexpr int kExpertBN = 256;  // token tile of the bf16 grouped GEMMs (Glu2Policy/Down2Policy kBN)
+
+// Token tile and M tiles per group of the grouped GEMMs that follow.
+struct GroupTiling {
+  int bn, mt1, mt2;
+};
+GroupTiling group_tiling(const mrlmoe_config &c) {
+  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) return {kF8MaxN, c.d_ff / 64, c.d_lat / 128};
+  return {kExpertBN, glu_m_tiles(c), down_m_tiles(c)};
+}
 
 // counts -> offsets/group tables -> stable scatter (from topk_idx).
 mrlmoe_status launch_dispatch(const mrlmoe_config &c, const Ptrs &P, cudaStream_t st) {
+  const GroupTiling gtl = group_tiling(c);
   const int T = c.T, E = c.n_experts, k = c.top_k;
   const int nch = (T + kChunk - 1) / kChunk;
   const int wpb = 8;
@@ -252,7 +283,7 @@ mrlmoe_status launch_dispatch(const mrlmoe_config &c, const Ptrs &P, cudaStream_
   MRL_TRY(cudaGetLastError());
   expert_colscan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(P.mask, E, nch, P.base, P.counts_e);
   MRL_TRY(cudaGetLastError());
-  expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, kExpertBN, glu_m_tiles(c), down_m_tiles(c), P.grp_off,
+  expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, gtl.bn, gtl.mt1, gtl.mt2, P.grp_off,
                                             P.grp_cnt, P.unit1, P.unit2, P.out_counts, P.out_offsets);
   MRL_TRY(cudaGetLastError());
   expert_scatter_kernel<<<(nch * 32 + 255) / 256, 256, 0, st>>>(P.topk_idx, P.mask, P.base, P.grp_off, T, E, k,
@@ -273,13 +304,70 @@ mrlmoe_status check_weights_bf16(const mrlmoe_weights *w, bool need_all) {
   return MRLMOE_OK;
 }
 
+mrlmoe_status check_weights_fp8(const mrlmoe_weights *w) {
+  if (!w || !w->w_router || !w->expert_scale || !w->rms_gain || !aligned16(w->w_router)) return MRLMOE_ERR_INVALID_ARG;
+  const void *codes[] = {w->w_down, w->w_gate, w->w_up_e, w->w_down_e, w->w_sh_gate, w->w_sh_up, w->w_sh_down, w->w_up};
+  const float *scales[] = {w->s_down, w->s_gate, w->s_up_e, w->s_down_e, w->s_sh_gate, w->s_sh_up, w->s_sh_down, w->s_up};
+  for (const void *p : codes)
+    if (!p || !aligned16(p)) return MRLMOE_ERR_INVALID_ARG;
+  for (const float *p : scales)
+    if (!p) return MRLMOE_ERR_INVALID_ARG;
+  return MRLMOE_OK;
+}
+
+cudaError_t launch_quant(const __nv_bfloat16 *in, long ld_in, int rows, int K, const int32_t *perm, int k, int Tk,
+                         uint8_t *q, float *sc, cudaStream_t st) {
+  const long warps = static_cast<long>(rows) * (K / 128);
+  quant_rows_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(in, ld_in, rows, K, perm, k, Tk,
+                                                                                    q, sc);
+  return cudaGetLastError();
+}
+
+template <class P>
+cudaError_t launch_gemm8(const typename P::Params &p, int grid, cudaStream_t st) {
+  static_assert(Gemm8Smem<P>::kTotal <= 232448, "GEMM shared memory above the 227 KB per-block limit");
+  static bool configured[kMaxDevices] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm8_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Gemm8Smem<P>::kTotal);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  gemm8_kernel<P><<<grid, kGemmThreads, Gemm8Smem<P>::kTotal, st>>>(p);
+  return cudaGetLastError();
+}
+
+// FP8 projection out = bf16(q(a) w^T) from e4m3 codes + scales.
+mrlmoe_status launch_dense8(const uint8_t *aq, const float *as, const void *wq, const float *ws, int M, int N, int K,
+                            __nv_bfloat16 *out, __nv_bfloat16 *out_lo, const Ptrs &P, int sms, cudaStream_t st) {
+  Dense8Policy::Params p{};
+  if (!make_map(&p.ta, aq, 1, K, M, 128) || !make_map(&p.tb, wq, 1, K, N, kF8MaxN)) return MRLMOE_ERR_CUDA;
+  p.as = as;
+  p.ws = ws;
+  p.out = out;
+  p.out_lo = out_lo;
+  p.ldo = N;
+  p.M = M; p.N = N; p.K = K;
+  p.m_tiles = (M + 127) / 128;
+  p.n_tiles = (N + kF8MaxN - 1) / kF8MaxN;
+  p.status = P.status;
+  MRL_TRY(launch_gemm8<Dense8Policy>(p, std::min(sms, p.m_tiles * p.n_tiles), st));
+  return MRLMOE_OK;
+}
+
 // Routing from x: down-projection into the tail of zbuf, then the fused router.
 mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weights *w, const float *bias,
                                        const void *x, const Ptrs &P, int sms, cudaStream_t st,
                                        void *const *ev = nullptr) {
   const int T = c.T, D = c.d_model, Ld = c.d_lat, E = c.n_experts, R = c.n_routers, k = c.top_k;
   __nv_bfloat16 *z = P.zbuf + static_cast<size_t>(T) * k * Ld;  // z rows live after the T*k dispatched rows
-  {
+  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) {
+    MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(x), D, T, D, nullptr, 1, 0, P.xq, P.xs, st));
+    mrlmoe_status s = launch_dense8(P.xq, P.xs, w->w_down, w->s_down, T, Ld, D, z, P.zlo, P, sms, st);
+    if (s != MRLMOE_OK) return s;
+  } else {
     DensePolicy::Params p{};
     if (!make_map(&p.ta, x, 2, D, T, 128) || !make_map(&p.tb, w->w_down, 2, D, Ld, DensePolicy::kBN))
       return MRLMOE_ERR_CUDA;
@@ -322,14 +410,20 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
   return MRLMOE_OK;
 }
 
+// FP8 variant after the dispatch record: quantised gather of the dispatched
+// latent rows, gate/up, quantised h, expert down, combine + RMSNorm,
+// quantised n, up-projection.  Stage events 4..7 as in the bf16 sequence.
+mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *w, const Ptrs &P, int sms,
+                                  cudaStream_t st, void *const *ev, void *y_out = nullptr);
+
 mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, const float *bias, const void *x,
                            void *y, mrlmoe_routing *route_out, void *workspace, size_t ws_bytes, void *stream,
                            void *const *ev) {
   mrlmoe_status s = check_config(cfg);
   if (s != MRLMOE_OK) return s;
   if (!bias || !x || !y || !aligned16(x) || !aligned16(y)) return MRLMOE_ERR_INVALID_ARG;
-  if ((s = check_weights_bf16(w, true)) != MRLMOE_OK) return s;
-  if (cfg->dtype != MRLMOE_BF16) return MRLMOE_ERR_UNSUPPORTED;
+  const bool fp8 = cfg->dtype == MRLMOE_FP8_E4M3_BLOCK128;
+  if ((s = fp8 ? check_weights_fp8(w) : check_weights_bf16(w, true)) != MRLMOE_OK) return s;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
   if (ws_bytes < layout_of(*cfg).total) return MRLMOE_ERR_WORKSPACE;
   int sms = 0;
@@ -348,6 +442,11 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   if (!mark(2)) return MRLMOE_ERR_CUDA;
   if ((s = launch_dispatch(*cfg, P, st)) != MRLMOE_OK) return s;
   if (!mark(3)) return MRLMOE_ERR_CUDA;
+  if (fp8) {
+    if ((s = forward_experts_fp8(*cfg, w, P, sms, st, ev, y)) != MRLMOE_OK) return s;
+    if (!mark(8)) return MRLMOE_ERR_CUDA;
+    return MRLMOE_OK;
+  }
 
   // gather the dispatched latent rows (rows [0, T*k) of zbuf) from z (rows [T*k, T*k+T))
   {
@@ -411,6 +510,60 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   }
   if (!mark(8)) return MRLMOE_ERR_CUDA;
   return MRLMOE_OK;
+}
+
+mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *w, const Ptrs &P, int sms,
+                                  cudaStream_t st, void *const *ev, void *y_out) {
+  const int T = c.T, D = c.d_model, Ld = c.d_lat, F = c.d_ff, E = c.n_experts, k = c.top_k;
+  const int Tk = T * k;
+  auto mark = [&](int i) -> bool {
+    return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
+  };
+  // quantised dispatched latent rows (rows < T*k) and the shared expert's rows (all T tokens)
+  MRL_TRY(launch_quant(P.zbuf + static_cast<size_t>(Tk) * Ld, Ld, Tk + T, Ld, P.perm, k, Tk, P.zq, P.zs, st));
+  if (!mark(4)) return MRLMOE_ERR_CUDA;
+  const GroupTiling gtl = group_tiling(c);
+  {
+    Glu8Policy::Params p{};
+    if (!make_map(&p.wg, w->w_gate, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !make_map(&p.wu, w->w_up_e, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !make_map(&p.sg, w->w_sh_gate, 1, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 1, Ld, F, 64) ||
+        !make_map(&p.tz, P.zq, 1, Ld, static_cast<uint64_t>(Tk) + T, 32))
+      return MRLMOE_ERR_CUDA;
+    p.wg_s = w->s_gate; p.wu_s = w->s_up_e; p.sg_s = w->s_sh_gate; p.su_s = w->s_sh_up;
+    p.zs = P.zs;
+    p.gt = GroupTable{P.grp_off, P.grp_cnt, P.unit1, E, gtl.mt1};
+    p.h = P.hbuf;
+    p.F = F; p.L = Ld;
+    p.status = P.status;
+    MRL_TRY(launch_gemm8<Glu8Policy>(p, sms, st));
+  }
+  MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, nullptr, 1, 0, P.hq, P.hs, st));
+  if (!mark(5)) return MRLMOE_ERR_CUDA;
+  {
+    Down8Policy::Params p{};
+    if (!make_map(&p.wd, w->w_down_e, 1, F, static_cast<uint64_t>(E) * Ld, 128) ||
+        !make_map(&p.sd, w->w_sh_down, 1, F, Ld, 128) ||
+        !make_map(&p.th, P.hq, 1, F, static_cast<uint64_t>(Tk) + T, 32))
+      return MRLMOE_ERR_CUDA;
+    p.wd_s = w->s_down_e; p.sd_s = w->s_sh_down;
+    p.hs = P.hs;
+    p.gt = GroupTable{P.grp_off, P.grp_cnt, P.unit2, E, gtl.mt2};
+    p.perm = P.perm;
+    p.wscaled = P.wscaled;
+    p.slots = P.slots;
+    p.L = Ld; p.F = F; p.k = k; p.Tk = Tk;
+    p.status = P.status;
+    MRL_TRY(launch_gemm8<Down8Policy>(p, sms, st));
+  }
+  if (!mark(6)) return MRLMOE_ERR_CUDA;
+  combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k, c.rms_eps,
+                                                        reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf);
+  MRL_TRY(cudaGetLastError());
+  MRL_TRY(launch_quant(P.nbuf, Ld, T, Ld, nullptr, 1, 0, P.nq, P.ns, st));
+  if (!mark(7)) return MRLMOE_ERR_CUDA;
+  return launch_dense8(P.nq, P.ns, w->w_up, w->s_up, T, D, Ld, static_cast<__nv_bfloat16 *>(y_out), nullptr, P, sms,
+                       st);
 }
 
 // ------------------------------------------------ static-scratch routing
@@ -496,7 +649,7 @@ mrlmoe_status mrlmoe_route(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
     if (!x || !aligned16(x)) return MRLMOE_ERR_INVALID_ARG;
     if ((s = check_weights_bf16(w, false)) != MRLMOE_OK) return s;
     if (!w->w_down || !aligned16(w->w_down)) return MRLMOE_ERR_INVALID_ARG;
-    if (cfg->dtype != MRLMOE_BF16) return MRLMOE_ERR_UNSUPPORTED;
+    if (cfg->dtype == MRLMOE_FP8_E4M3_BLOCK128 && !w->s_down) return MRLMOE_ERR_INVALID_ARG;
   }
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
   if (ws_bytes < layout_of(*cfg).total) return MRLMOE_ERR_WORKSPACE;
@@ -603,6 +756,19 @@ mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *
       out->scores, bias, expert_scale, cfg->T, cfg->n_experts, cfg->top_k, P.topk_idx, P.topk_w, P.wscaled);
   MRL_TRY(cudaGetLastError());
   return launch_dispatch(*cfg, P, st);
+}
+
+mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, float *scale, void *stream) {
+  if (!in || !q || !scale || rows < 1 || K < 128 || K % 128) return MRLMOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(in) & 7u) || (reinterpret_cast<uintptr_t>(q) & 3u) ||
+      (reinterpret_cast<uintptr_t>(scale) & 3u))
+    return MRLMOE_ERR_INVALID_ARG;
+  int sms = 0;
+  mrlmoe_status s = bind_device(in, &sms);
+  if (s != MRLMOE_OK) return s;
+  MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(in), K, rows, K, nullptr, 1, 0, static_cast<uint8_t *>(q),
+                       scale, static_cast<cudaStream_t>(stream)));
+  return MRLMOE_OK;
 }
 
 mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream) {

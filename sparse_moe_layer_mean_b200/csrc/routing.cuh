@@ -222,6 +222,47 @@ __global__ void gather_rows_kernel(const int32_t *__restrict__ perm, int rows, i
 }
 
 // ---------------------------------------------------------------------------
+// FP8 activation quantiser, one warp per (row, 128-wide K block): amax over
+// the block's bf16 values; amax == 0 -> scale 1, codes 0; else scale =
+// amax / 448 and code = e4m3_rn_satfinite(v * (448 / amax)) (fp32 IEEE ops).
+// With `perm`, output row r < Tk takes input row perm[r] / k (a dispatched
+// token) and rows Tk .. Tk+T-1 take input rows 0 .. T-1.
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));  // first source -> upper byte
+  return r;
+}
+
+__global__ void quant_rows_kernel(const __nv_bfloat16 *__restrict__ in, long ld_in, int rows, int K,
+                                  const int32_t *__restrict__ perm, int k, int Tk, uint8_t *__restrict__ q,
+                                  float *__restrict__ s) {
+  const int kbs = K >> 7;
+  const long wid = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= static_cast<long>(rows) * kbs) return;
+  const int r = static_cast<int>(wid / kbs);
+  const int b = static_cast<int>(wid - static_cast<long>(r) * kbs);
+  long src = r;
+  if (perm) src = r < Tk ? __ldg(perm + r) / k : r - Tk;
+  const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(in + src * ld_in + b * 128 + lane * 4));
+  const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
+  const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
+  const float v0 = __low2float(p0), v1 = __high2float(p0), v2 = __low2float(p1), v3 = __high2float(p1);
+  float amax = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  float scale = 1.0f, inv = 0.0f;
+  if (amax != 0.0f) {
+    scale = amax / 448.0f;
+    inv = 448.0f / amax;
+  }
+  const uint32_t codes = static_cast<uint32_t>(e4m3x2(v0 * inv, v1 * inv)) |
+                         (static_cast<uint32_t>(e4m3x2(v2 * inv, v3 * inv)) << 16);
+  *reinterpret_cast<uint32_t *>(q + static_cast<long>(r) * K + b * 128 + lane * 4) = codes;
+  if (lane == 0) s[static_cast<long>(r) * kbs + b] = scale;
+}
+
+// ---------------------------------------------------------------------------
 // Combine + RMSNorm, one block (256 threads) per token:
 //   c = slot[t,0] + slot[t,1] + ... + slot[t,k-1] + slot[t,k]   (rank order, then shared)
 //   n = bf16(c * (1 / sqrt(mean(c^2) + eps)) * gain)

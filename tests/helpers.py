@@ -12,20 +12,26 @@ import workloads as W
 # Output bounds for the bf16 layer: max|dy| / max|y_ref| and sum|dy| / sum|y_ref|.
 BF16_MAX_REL = 1e-2
 BF16_MEAN_REL = 2e-3
+# ... and for the FP8 variant
+FP8_MAX_REL = 3e-2
+FP8_MEAN_REL = 6e-3
 # A routing mismatch is legitimate only where the oracle's k-th vs (k+1)-th
 # biased-score gap is below this.
 GAP_TOL = 1e-5
 
 
 def _wkey(name: str) -> str:
-    """Configs with the same layer shape share one set of weights."""
+    """Configs with the same layer shape and weight type share one set of weights."""
     s = W.CONFIGS[name]
-    return "c0_tiny" if s.d_model == 256 else "c2_prefill"
+    if s.d_model == 256:
+        return "c0_fp8" if s.fp8 else "c0_tiny"
+    return "c4_fp8" if s.fp8 else "c2_prefill"
 
 
 @functools.lru_cache(maxsize=2)
 def _device_weights(key: str, seed: int):
-    return W.make_weights(W.CONFIGS[key], "cuda", seed=seed)
+    s = W.CONFIGS[key]
+    return (W.make_weights_fp8 if s.fp8 else W.make_weights)(s, "cuda", seed=seed)
 
 
 @functools.lru_cache(maxsize=2)

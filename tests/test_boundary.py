@@ -18,7 +18,7 @@ HEADER = os.path.join(ROOT, "include", "mrlmoe.h")
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(mrlmoe_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(mrlmoe_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_library_loads_and_exports_every_declared_symbol():
@@ -33,7 +33,7 @@ def test_library_loads_and_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(7):
+    for code in range(8):
         assert M.status_string(code)
     assert M.status_string(99) == "unknown status"
 
@@ -76,7 +76,13 @@ def test_forward_rejects_bad_arguments_before_cuda():
     assert _raw_forward(cfg, full, 4096, 4096, 4096, None, need) == 3      # no workspace
     assert _raw_forward(cfg, full, 4096, 4096, 4096, 4096 + 16, need) == 3  # misaligned
     assert _raw_forward(cfg, full, 4096, 4096, 4096, 4096, need - 1) == 3  # too small
-    assert _raw_forward(_cfg(dtype=1), full, 4096, 4096, 4096, 4096, need) == 2  # FP8 not built yet
+    # the FP8 variant needs the block-scale arrays too
+    cfg8 = _cfg(dtype=1)
+    need8 = M.mrlmoe_workspace_size(cfg8)
+    assert need8 > need                                                    # e4m3 copies of the GEMM inputs
+    assert _raw_forward(cfg8, full, 4096, 4096, 4096, 4096, need8) == 1
+    full8 = N.Weights(*([4096] * 11 + [8192] * 8))
+    assert _raw_forward(cfg8, full8, 4096, 4096, 4096, 4096, need8 - 1) == 3
 
 
 def test_route_rejects_bad_arguments_before_cuda():
@@ -109,6 +115,14 @@ def test_bias_update_and_linear_reject_bad_arguments():
     assert L.mrlmoe_linear(4096, 4096, 4096, 8, 128, 64, None) == 1
     assert L.mrlmoe_linear(None, 4096, 4096, 8, 128, 128, None) == 1
     assert L.mrlmoe_linear(4096 + 2, 4096, 4096, 8, 128, 128, None) == 1
+
+
+def test_quantize_rejects_bad_arguments():
+    L = N.lib()
+    assert L.mrlmoe_quantize_e4m3(None, 4, 128, 4096, 4096, None) == 1
+    assert L.mrlmoe_quantize_e4m3(4096, 0, 128, 4096, 4096, None) == 1
+    assert L.mrlmoe_quantize_e4m3(4096, 4, 100, 4096, 4096, None) == 1
+    assert L.mrlmoe_quantize_e4m3(4096 + 2, 4, 128, 4096, 4096, None) == 1
 
 
 def test_python_binding_raises_on_error():

@@ -5,7 +5,8 @@ import torch
 import oracle as O
 import workloads as W
 import sparse_moe_layer_mean_b200 as M
-from helpers import (BF16_MAX_REL, BF16_MEAN_REL, GAP_TOL, check_dispatch_properties,
+from helpers import (BF16_MAX_REL, BF16_MEAN_REL, FP8_MAX_REL, FP8_MEAN_REL, GAP_TOL,
+                     check_dispatch_properties,
                      device_weights, host_weights, rel_errors, routing_audit)
 
 pytestmark = pytest.mark.gpu
@@ -210,3 +211,60 @@ def test_forward_c3_skew_sampled_tokens_and_bias_update():
     want = (b0.cpu() + torch.tensor(gamma, dtype=torch.float32) * sgn.float()) - b0.cpu()
     assert torch.equal(d, want)
     assert int((sgn < 0).sum()) > 0 and int((sgn > 0).sum()) > 0
+
+
+# ------------------------------------------------------------------- FP8
+def test_quantize_e4m3_bit_exact():
+    g = torch.Generator().manual_seed(21)
+    rows, K = 300, 512
+    v = (torch.randn(rows, K, generator=g) * torch.exp(torch.randn(rows, 1, generator=g) * 2))
+    v[3, :128] = 0.0                                   # an all-zero block
+    v[5, 130] = 1e4                                    # an outlier
+    v[7, 256:384] = -0.0
+    xb = v.to(torch.bfloat16)
+    xd = xb.cuda()
+    q = torch.empty(rows, K, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(rows, K // 128, dtype=torch.float32, device="cuda")
+    M.mrlmoe_quantize_e4m3(xd, rows, K, q, sc)
+    torch.cuda.synchronize()
+    deq = O.e4m3_decode(q.cpu()) * sc.cpu().double().repeat_interleave(128, 1)
+    ref = O.quantize_act_1x128(xb.double())
+    assert torch.equal(deq, ref)
+    amax = xb.float().abs().reshape(rows, K // 128, 128).amax(-1)
+    want = torch.where(amax == 0, torch.ones_like(amax), amax / torch.tensor(448.0))
+    assert torch.equal(sc.cpu(), want)
+
+
+def _compare_fp8(s, x, bias, y, r, wh, tokens=None):
+    xs = x.cpu() if tokens is None else x.cpu()[tokens]
+    ref = O.forward(xs, wh, bias.cpu(), s.top_k, s.rms_eps, fp8=True)
+    gidx = r["topk_idx"].view(-1, s.top_k)
+    if tokens is not None:
+        gidx = gidx[tokens.to(gidx.device)]
+    bad, gaps, _ = routing_audit(gidx, ref.s, bias, s.top_k)
+    assert torch.all(gaps < GAP_TOL), (bad, gaps)
+    keep = torch.ones(xs.shape[0], dtype=torch.bool)
+    keep[bad] = False
+    yg = y.cpu() if tokens is None else y.cpu()[tokens]
+    mx, mean = rel_errors(yg[keep], ref.y[keep])
+    assert mx <= FP8_MAX_REL and mean <= FP8_MEAN_REL, (mx, mean)
+    return ref
+
+
+def test_forward_fp8_tiny():
+    s, x, bias, y, r, _ = _run_layer("c0_fp8")
+    ref = _compare_fp8(s, x, bias, y, r, host_weights("c0_fp8"))
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+
+
+@pytest.mark.parametrize("T", [1, 200])
+def test_forward_fp8_tiny_ragged(T):
+    s, x, bias, y, r, _ = _run_layer("c0_fp8", T=T)
+    _compare_fp8(s, x, bias, y, r, host_weights("c0_fp8"))
+
+
+def test_forward_c4_fp8_sampled_tokens():
+    s, x, bias, y, r, _ = _run_layer("c4_fp8", scores=False)
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+    tokens = torch.tensor([0, 1, 777, 8192, 16383])
+    _compare_fp8(s, x, bias, y, r, host_weights("c4_fp8"), tokens=tokens)

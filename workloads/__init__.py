@@ -75,6 +75,9 @@ CONFIGS: Dict[str, LayerShape] = {
     "c3_skew": LayerShape("c3_skew", T=32768, bias_kind="zipf", **_FULL),
     # full width, e4m3 experts/projections with 1% outlier channels in x
     "c4_fp8": LayerShape("c4_fp8", T=16384, fp8=True, outlier_frac=0.01, **_FULL),
+    # test case: the tiny layer in the FP8 variant (2 of the 256 x channels are outliers)
+    "c0_fp8": LayerShape("c0_fp8", T=64, d_model=256, d_lat=128, n_experts=16, top_k=2, d_ff=128,
+                         n_routers=2, fp8=True, outlier_frac=0.01),
 }
 
 # Scalar lambda for the c3_skew bias b_e = lambda * ln(p_rank(e) / p_1), with
@@ -230,6 +233,44 @@ def make_weights(s: LayerShape, device, seed: Optional[int] = None) -> Dict[str,
     w["rms_gain"] = torch.ones(L, dtype=torch.float32, device=device)
     w["expert_scale"] = uniform((E,), 0.5, 1.5, seed, _S_ALPHA, device)
     return w
+
+
+FP8_MATRICES = ("w_down", "w_gate", "w_up_e", "w_down_e", "w_sh_gate", "w_sh_up", "w_sh_down", "w_up")
+
+
+def to_fp8_blocks(w: torch.Tensor):
+    """e4m3 codes and fp32 scales per 128x128 block of the trailing [out, in]
+    dims: scale = fp32(amax / 448) (1 for an all-zero block), codes from the
+    library's float8_e4m3fn conversion of w / scale (clamped to +-448)."""
+    *lead, out, inn = w.shape
+    ob, ib = (out + 127) // 128, (inn + 127) // 128
+    wf = w.to(torch.float32)
+    pad = torch.zeros(*lead, ob * 128, ib * 128, dtype=torch.float32, device=w.device)
+    pad[..., :out, :inn] = wf
+    blk = pad.reshape(*lead, ob, 128, ib, 128)
+    amax = blk.abs().amax(dim=(-3, -1))                       # [..., ob, ib]
+    scale = torch.where(amax == 0, torch.ones_like(amax), amax / torch.tensor(448.0))
+    q = (blk / scale[..., :, None, :, None]).clamp(-448.0, 448.0)
+    codes = q.to(torch.float8_e4m3fn).reshape(*lead, ob * 128, ib * 128)[..., :out, :inn]
+    return codes.contiguous().view(torch.uint8), scale.contiguous()
+
+
+def make_weights_fp8(s: LayerShape, device, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """The FP8 variant's inputs: the bf16 weights of make_weights, with every
+    projection and expert matrix given as e4m3 codes (uint8) plus its fp32
+    128x128 block scales under the C ABI's name (w_down -> s_down, w_up_e ->
+    s_up_e, ...); the routers stay bf16."""
+    w = make_weights(s, device, seed)
+    for nm in FP8_MATRICES:
+        codes, scale = to_fp8_blocks(w[nm])
+        w[nm] = codes
+        w[fp8_scale_name(nm)] = scale
+    return w
+
+
+def fp8_scale_name(matrix: str) -> str:
+    """Name of a matrix's block-scale array: w_<x> -> s_<x>."""
+    return "s_" + matrix[2:]
 
 
 def outlier_channels(s: LayerShape, device, seed: Optional[int] = None) -> torch.Tensor:
