@@ -66,7 +66,9 @@ typedef enum {
 /* Layer shape.  Limits checked on the host:
  *   T >= 1; d_model, d_lat, d_ff multiples of 128; 1 <= n_routers <= 8;
  *   16 <= n_experts <= 1024 with n_experts a multiple of 16;
- *   1 <= top_k <= min(n_experts, 16); rms_eps >= 0.                            */
+ *   1 <= top_k <= min(n_experts, 16); rms_eps >= 0.  d_lat <= 8192, and in
+ *   FP8 mode d_model, d_lat, d_ff <= 4096; beyond those the status is
+ *   MRLMOE_ERR_UNSUPPORTED, otherwise MRLMOE_ERR_INVALID_ARG.                 */
 typedef struct {
   int T;            /* tokens in this call                                       */
   int d_model;      /* hidden size (4096 at full width)                          */
@@ -198,6 +200,8 @@ mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *
  * scale[r*K/128 + b] = amax / 448 (1 if amax == 0) and
  * q[r*K + b*128 + i] = e4m3(v_i * 448 / amax) rounded to nearest even with
  * saturation (0 if amax == 0).  q: [rows, K] e4m3 bytes; scale: fp32.
+ * Device pointers, caller-owned; in 16-byte, q 8-byte and scale 4-byte
+ * aligned, else MRLMOE_ERR_INVALID_ARG (as for rows < 1 or a bad K).
  * The variant's reading of "activations quantised e4m3 per 1x128 block".    */
 mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, float *scale,
                                    void *stream);

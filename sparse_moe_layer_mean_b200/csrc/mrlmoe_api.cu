@@ -32,6 +32,10 @@ mrlmoe_status check_config(const mrlmoe_config *c) {
   if (c->n_routers < 1 || c->n_routers > 8) return MRLMOE_ERR_INVALID_ARG;
   if (!(c->rms_eps >= 0.f)) return MRLMOE_ERR_INVALID_ARG;
   if (c->dtype != MRLMOE_BF16 && c->dtype != MRLMOE_FP8_E4M3_BLOCK128) return MRLMOE_ERR_INVALID_ARG;
+  // the FP8 GEMMs stage at most kF8MaxKB scales of 128-wide K blocks per unit
+  if (c->dtype == MRLMOE_FP8_E4M3_BLOCK128 &&
+      (c->d_model > 128 * kF8MaxKB || c->d_lat > 128 * kF8MaxKB || c->d_ff > 128 * kF8MaxKB))
+    return MRLMOE_ERR_UNSUPPORTED;
   // dispatched rows are addressed with 32-bit indices
   const long long rows = static_cast<long long>(c->T) * (c->top_k + 1);
   if (rows * 256 >= (1ll << 31)) return MRLMOE_ERR_UNSUPPORTED;
@@ -268,7 +272,7 @@ struct GroupTiling {
   int bn, mt1, mt2;
 };
 GroupTiling group_tiling(const mrlmoe_config &c) {
-  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) return {kF8MaxN, c.d_ff / 64, c.d_lat / 128};
+  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) return {kF8Tile, c.d_ff / 64, c.d_lat / 128};
   return {kExpertBN, glu_m_tiles(c), down_m_tiles(c)};
 }
 
@@ -315,11 +319,12 @@ mrlmoe_status check_weights_fp8(const mrlmoe_weights *w) {
   return MRLMOE_OK;
 }
 
+// Scales go to sc[rows][K/128], or transposed to sc[K/128][rows] (the layout
+// the FP8 GEMMs read) when `transposed`.
 cudaError_t launch_quant(const __nv_bfloat16 *in, long ld_in, int rows, int K, const int32_t *perm, int k, int Tk,
-                         uint8_t *q, float *sc, cudaStream_t st) {
-  const long warps = static_cast<long>(rows) * (K / 128);
-  quant_rows_kernel<<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(in, ld_in, rows, K, perm, k, Tk,
-                                                                                    q, sc);
+                         uint8_t *q, float *sc, bool transposed, cudaStream_t st) {
+  quant_rows_kernel<<<(rows + kQuantWarps - 1) / kQuantWarps, kQuantWarps * 32, 0, st>>>(
+      in, ld_in, rows, K, perm, k, Tk, q, sc, transposed ? static_cast<long>(rows) : 0L);
   return cudaGetLastError();
 }
 
@@ -335,23 +340,24 @@ cudaError_t launch_gemm8(const typename P::Params &p, int grid, cudaStream_t st)
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  gemm8_kernel<P><<<grid, kGemmThreads, Gemm8Smem<P>::kTotal, st>>>(p);
+  gemm8_kernel<P><<<grid, kF8Threads, Gemm8Smem<P>::kTotal, st>>>(p);
   return cudaGetLastError();
 }
 
-// FP8 projection out = bf16(q(a) w^T) from e4m3 codes + scales.
-mrlmoe_status launch_dense8(const uint8_t *aq, const float *as, const void *wq, const float *ws, int M, int N, int K,
+// FP8 projection out = bf16(q(a) w^T) from e4m3 codes + scales (as_t: the
+// activation scales transposed, [K/128, M]).
+mrlmoe_status launch_dense8(const uint8_t *aq, const float *as_t, const void *wq, const float *ws, int M, int N, int K,
                             __nv_bfloat16 *out, __nv_bfloat16 *out_lo, const Ptrs &P, int sms, cudaStream_t st) {
   Dense8Policy::Params p{};
-  if (!make_map(&p.ta, aq, 1, K, M, 128) || !make_map(&p.tb, wq, 1, K, N, kF8MaxN)) return MRLMOE_ERR_CUDA;
-  p.as = as;
+  if (!make_map(&p.ta, aq, 1, K, M, 128) || !make_map(&p.tb, wq, 1, K, N, kF8Tile)) return MRLMOE_ERR_CUDA;
+  p.as_t = as_t;
   p.ws = ws;
   p.out = out;
   p.out_lo = out_lo;
   p.ldo = N;
   p.M = M; p.N = N; p.K = K;
   p.m_tiles = (M + 127) / 128;
-  p.n_tiles = (N + kF8MaxN - 1) / kF8MaxN;
+  p.n_tiles = (N + kF8Tile - 1) / kF8Tile;
   p.status = P.status;
   MRL_TRY(launch_gemm8<Dense8Policy>(p, std::min(sms, p.m_tiles * p.n_tiles), st));
   return MRLMOE_OK;
@@ -364,7 +370,7 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
   const int T = c.T, D = c.d_model, Ld = c.d_lat, E = c.n_experts, R = c.n_routers, k = c.top_k;
   __nv_bfloat16 *z = P.zbuf + static_cast<size_t>(T) * k * Ld;  // z rows live after the T*k dispatched rows
   if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) {
-    MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(x), D, T, D, nullptr, 1, 0, P.xq, P.xs, st));
+    MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(x), D, T, D, nullptr, 1, 0, P.xq, P.xs, true, st));
     mrlmoe_status s = launch_dense8(P.xq, P.xs, w->w_down, w->s_down, T, Ld, D, z, P.zlo, P, sms, st);
     if (s != MRLMOE_OK) return s;
   } else {
@@ -520,7 +526,7 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
   };
   // quantised dispatched latent rows (rows < T*k) and the shared expert's rows (all T tokens)
-  MRL_TRY(launch_quant(P.zbuf + static_cast<size_t>(Tk) * Ld, Ld, Tk + T, Ld, P.perm, k, Tk, P.zq, P.zs, st));
+  MRL_TRY(launch_quant(P.zbuf + static_cast<size_t>(Tk) * Ld, Ld, Tk + T, Ld, P.perm, k, Tk, P.zq, P.zs, true, st));
   if (!mark(4)) return MRLMOE_ERR_CUDA;
   const GroupTiling gtl = group_tiling(c);
   {
@@ -528,26 +534,28 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     if (!make_map(&p.wg, w->w_gate, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
         !make_map(&p.wu, w->w_up_e, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
         !make_map(&p.sg, w->w_sh_gate, 1, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 1, Ld, F, 64) ||
-        !make_map(&p.tz, P.zq, 1, Ld, static_cast<uint64_t>(Tk) + T, 32))
+        !make_map(&p.tz, P.zq, 1, Ld, static_cast<uint64_t>(Tk) + T, kF8Tile))
       return MRLMOE_ERR_CUDA;
     p.wg_s = w->s_gate; p.wu_s = w->s_up_e; p.sg_s = w->s_sh_gate; p.su_s = w->s_sh_up;
-    p.zs = P.zs;
+    p.zs_t = P.zs;
+    p.rows = Tk + T;
     p.gt = GroupTable{P.grp_off, P.grp_cnt, P.unit1, E, gtl.mt1};
     p.h = P.hbuf;
     p.F = F; p.L = Ld;
     p.status = P.status;
     MRL_TRY(launch_gemm8<Glu8Policy>(p, sms, st));
   }
-  MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, nullptr, 1, 0, P.hq, P.hs, st));
+  MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, nullptr, 1, 0, P.hq, P.hs, true, st));
   if (!mark(5)) return MRLMOE_ERR_CUDA;
   {
     Down8Policy::Params p{};
     if (!make_map(&p.wd, w->w_down_e, 1, F, static_cast<uint64_t>(E) * Ld, 128) ||
         !make_map(&p.sd, w->w_sh_down, 1, F, Ld, 128) ||
-        !make_map(&p.th, P.hq, 1, F, static_cast<uint64_t>(Tk) + T, 32))
+        !make_map(&p.th, P.hq, 1, F, static_cast<uint64_t>(Tk) + T, kF8Tile))
       return MRLMOE_ERR_CUDA;
     p.wd_s = w->s_down_e; p.sd_s = w->s_sh_down;
-    p.hs = P.hs;
+    p.hs_t = P.hs;
+    p.rows = Tk + T;
     p.gt = GroupTable{P.grp_off, P.grp_cnt, P.unit2, E, gtl.mt2};
     p.perm = P.perm;
     p.wscaled = P.wscaled;
@@ -560,7 +568,7 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
   combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k, c.rms_eps,
                                                         reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf);
   MRL_TRY(cudaGetLastError());
-  MRL_TRY(launch_quant(P.nbuf, Ld, T, Ld, nullptr, 1, 0, P.nq, P.ns, st));
+  MRL_TRY(launch_quant(P.nbuf, Ld, T, Ld, nullptr, 1, 0, P.nq, P.ns, true, st));
   if (!mark(7)) return MRLMOE_ERR_CUDA;
   return launch_dense8(P.nq, P.ns, w->w_up, w->s_up, T, D, Ld, static_cast<__nv_bfloat16 *>(y_out), nullptr, P, sms,
                        st);
@@ -760,14 +768,14 @@ mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *
 
 mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, float *scale, void *stream) {
   if (!in || !q || !scale || rows < 1 || K < 128 || K % 128) return MRLMOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(in) & 7u) || (reinterpret_cast<uintptr_t>(q) & 3u) ||
+  if ((reinterpret_cast<uintptr_t>(in) & 15u) || (reinterpret_cast<uintptr_t>(q) & 7u) ||
       (reinterpret_cast<uintptr_t>(scale) & 3u))
     return MRLMOE_ERR_INVALID_ARG;
   int sms = 0;
   mrlmoe_status s = bind_device(in, &sms);
   if (s != MRLMOE_OK) return s;
   MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(in), K, rows, K, nullptr, 1, 0, static_cast<uint8_t *>(q),
-                       scale, static_cast<cudaStream_t>(stream)));
+                       scale, false, static_cast<cudaStream_t>(stream)));
   return MRLMOE_OK;
 }
 

@@ -222,44 +222,69 @@ __global__ void gather_rows_kernel(const int32_t *__restrict__ perm, int rows, i
 }
 
 // ---------------------------------------------------------------------------
-// FP8 activation quantiser, one warp per (row, 128-wide K block): amax over
-// the block's bf16 values; amax == 0 -> scale 1, codes 0; else scale =
-// amax / 448 and code = e4m3_rn_satfinite(v * (448 / amax)) (fp32 IEEE ops).
+// FP8 activation quantiser, one warp per row, a half-warp per 128-wide K
+// block (16 lanes x 8 bf16: 16-byte loads, 8-byte code stores): amax over the
+// block's bf16 values; amax == 0 -> scale 1, codes 0; else scale = amax / 448
+// and code = e4m3_rn_satfinite(v * (448 / amax)) (fp32 IEEE ops).
 // With `perm`, output row r < Tk takes input row perm[r] / k (a dispatched
-// token) and rows Tk .. Tk+T-1 take input rows 0 .. T-1.
+// token) and rows Tk .. Tk+T-1 take input rows 0 .. T-1.  Scales go to
+// s[r][K/128] (s_ld == 0) or, transposed, to s[b * s_ld + r].
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));  // first source -> upper byte
   return r;
 }
 
-__global__ void quant_rows_kernel(const __nv_bfloat16 *__restrict__ in, long ld_in, int rows, int K,
-                                  const int32_t *__restrict__ perm, int k, int Tk, uint8_t *__restrict__ q,
-                                  float *__restrict__ s) {
+constexpr int kQuantWarps = 8;
+
+__global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_kernel(
+    const __nv_bfloat16 *__restrict__ in, long ld_in, int rows, int K, const int32_t *__restrict__ perm, int k,
+    int Tk, uint8_t *__restrict__ q, float *__restrict__ s, long s_ld) {
   const int kbs = K >> 7;
-  const long wid = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int r = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+  if (r >= rows) return;  // whole warps leave together
   const int lane = threadIdx.x & 31;
-  if (wid >= static_cast<long>(rows) * kbs) return;
-  const int r = static_cast<int>(wid / kbs);
-  const int b = static_cast<int>(wid - static_cast<long>(r) * kbs);
+  const int half = lane >> 4, hl = lane & 15;
   long src = r;
   if (perm) src = r < Tk ? __ldg(perm + r) / k : r - Tk;
-  const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(in + src * ld_in + b * 128 + lane * 4));
-  const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
-  const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
-  const float v0 = __low2float(p0), v1 = __high2float(p0), v2 = __low2float(p1), v3 = __high2float(p1);
-  float amax = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
+  const __nv_bfloat16 *row_in = in + src * ld_in;
+  uint8_t *row_q = q + static_cast<long>(r) * K;
+  for (int b0 = 0; b0 < kbs; b0 += 2) {
+    const int b = b0 + half;
+    const bool live = b < kbs;
+    float v[8];
+    if (live) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(row_in + b * 128 + hl * 8));
+      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  float scale = 1.0f, inv = 0.0f;
-  if (amax != 0.0f) {
-    scale = amax / 448.0f;
-    inv = 448.0f / amax;
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __low2float(h2[i]);
+        v[2 * i + 1] = __high2float(h2[i]);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    float scale = 1.0f, inv = 0.0f;
+    if (amax != 0.0f) {
+      scale = amax / 448.0f;
+      inv = 448.0f / amax;
+    }
+    if (live) {
+      uint2 codes;
+      codes.x = static_cast<uint32_t>(e4m3x2(v[0] * inv, v[1] * inv)) |
+                (static_cast<uint32_t>(e4m3x2(v[2] * inv, v[3] * inv)) << 16);
+      codes.y = static_cast<uint32_t>(e4m3x2(v[4] * inv, v[5] * inv)) |
+                (static_cast<uint32_t>(e4m3x2(v[6] * inv, v[7] * inv)) << 16);
+      *reinterpret_cast<uint2 *>(row_q + b * 128 + hl * 8) = codes;
+      if (hl == 0) s[s_ld ? b * s_ld + r : static_cast<long>(r) * kbs + b] = scale;
+    }
   }
-  const uint32_t codes = static_cast<uint32_t>(e4m3x2(v0 * inv, v1 * inv)) |
-                         (static_cast<uint32_t>(e4m3x2(v2 * inv, v3 * inv)) << 16);
-  *reinterpret_cast<uint32_t *>(q + static_cast<long>(r) * K + b * 128 + lane * 4) = codes;
-  if (lane == 0) s[static_cast<long>(r) * kbs + b] = scale;
 }
 
 // ---------------------------------------------------------------------------

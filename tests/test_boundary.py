@@ -51,6 +51,11 @@ def test_workspace_size_valid_and_invalid():
                 dict(n_experts=24 + 1), dict(top_k=0), dict(top_k=17), dict(top_k=17, n_experts=16),
                 dict(n_routers=0), dict(n_routers=9), dict(rms_eps=-1.0), dict(dtype=7)):
         assert M.mrlmoe_workspace_size(_cfg(**bad)) == 0, bad
+    # the FP8 variant stages at most 32 K-block scales per GEMM unit: K <= 4096
+    for big in (dict(d_model=4224), dict(d_lat=4224), dict(d_ff=4224)):
+        assert M.mrlmoe_workspace_size(_cfg(dtype=1, **big)) == 0, big
+        assert M.mrlmoe_workspace_size(_cfg(dtype=0, **big)) > 0, big
+    assert M.mrlmoe_workspace_size(_cfg(dtype=1, d_model=4096, d_lat=4096, d_ff=4096)) > 0
     # grows with T
     assert M.mrlmoe_workspace_size(_cfg(T=128)) > M.mrlmoe_workspace_size(_cfg(T=64))
 
@@ -123,6 +128,8 @@ def test_quantize_rejects_bad_arguments():
     assert L.mrlmoe_quantize_e4m3(4096, 0, 128, 4096, 4096, None) == 1
     assert L.mrlmoe_quantize_e4m3(4096, 4, 100, 4096, 4096, None) == 1
     assert L.mrlmoe_quantize_e4m3(4096 + 2, 4, 128, 4096, 4096, None) == 1
+    assert L.mrlmoe_quantize_e4m3(4096 + 8, 4, 128, 4096, 4096, None) == 1   # in: 16-byte aligned
+    assert L.mrlmoe_quantize_e4m3(4096, 4, 128, 4096 + 4, 4096, None) == 1   # q: 8-byte aligned
 
 
 def test_python_binding_raises_on_error():

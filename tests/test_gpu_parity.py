@@ -214,9 +214,9 @@ def test_forward_c3_skew_sampled_tokens_and_bias_update():
 
 
 # ------------------------------------------------------------------- FP8
-def test_quantize_e4m3_bit_exact():
+@pytest.mark.parametrize("rows,K", [(300, 512), (37, 384)])   # even and odd block counts per row
+def test_quantize_e4m3_bit_exact(rows, K):
     g = torch.Generator().manual_seed(21)
-    rows, K = 300, 512
     v = (torch.randn(rows, K, generator=g) * torch.exp(torch.randn(rows, 1, generator=g) * 2))
     v[3, :128] = 0.0                                   # an all-zero block
     v[5, 130] = 1e4                                    # an outlier
