@@ -172,13 +172,12 @@ done:
 // --------------------------------------------------------------- policies
 __device__ __forceinline__ int round32(int n) { return (n + 31) & ~31; }
 
-// B half of CTA `rank`: rows row0 + rank*N/2 .. + N/2 (N = MMA N, multiple of
-// 32), as 16-row boxes.
-__device__ __forceinline__ void load_rows_half(const CUtensorMap *tm, const Unit &U, int kb, uint32_t sb,
+// B half of CTA `rank`: rows row0 + rank*N/2 .. + N/2 (N = MMA N, a multiple
+// of 32, so N/2 is a multiple of 16), as 64/32/16-row boxes.
+__device__ __forceinline__ void load_rows_half(const TokenMaps &t, const Unit &U, int kb, uint32_t sb,
                                                uint32_t bar_cl, uint32_t rank) {
   const int half = round32(U.nv) >> 1;
-  const int r0 = U.row0 + static_cast<int>(rank) * half;
-  for (int i = 0; i < (half >> 4); ++i) tma_load_2d_pair(sb + i * 2048, tm, bar_cl, kb * kBK, r0 + 16 * i);
+  load_token_rows<true>(t, kb * kBK, U.row0 + static_cast<int>(rank) * half, half, sb, bar_cl);
 }
 
 // gate/up over a CTA pair: unit = (group, 128-wide d_ff slice, <= 256 tokens);
@@ -218,7 +217,7 @@ struct Glu2Policy {
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb,
                                                 uint32_t bar_cl, uint32_t rank) {
-    load_rows_half(&p.tz, U, kb, sb, bar_cl, rank);
+    load_rows_half(p.tz, U, kb, sb, bar_cl, rank);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U) {
     return idesc_bf16(256, round32(U.nv));
@@ -282,7 +281,7 @@ struct Down2Policy {
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb,
                                                 uint32_t bar_cl, uint32_t rank) {
-    load_rows_half(&p.th, U, kb, sb, bar_cl, rank);
+    load_rows_half(p.th, U, kb, sb, bar_cl, rank);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U) {
     return idesc_bf16(256, round32(U.nv));

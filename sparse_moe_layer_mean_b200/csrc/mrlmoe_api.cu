@@ -149,6 +149,12 @@ bool make_map(CUtensorMap *m, const void *base, int esize, uint64_t inner, uint6
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The three box heights of a bf16 token tensor [rows, inner] (load_token_rows).
+bool make_token_maps(TokenMaps *t, const void *base, uint64_t inner, uint64_t rows) {
+  return make_map(&t->m16, base, 2, inner, rows, 16) && make_map(&t->m32, base, 2, inner, rows, 32) &&
+         make_map(&t->m64, base, 2, inner, rows, 64);
+}
+
 // Make the device that owns `p` current; reject host/unknown pointers.
 mrlmoe_status bind_device(const void *p, int *sm_count) {
   cudaPointerAttributes a;
@@ -470,7 +476,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
     if (!make_map(&p.wg, w->w_gate, 2, Ld, static_cast<uint64_t>(E) * F, 64) ||
         !make_map(&p.wu, w->w_up_e, 2, Ld, static_cast<uint64_t>(E) * F, 64) ||
         !make_map(&p.sg, w->w_sh_gate, 2, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 2, Ld, F, 64) ||
-        !make_map(&p.tz, P.zbuf, 2, Ld, static_cast<uint64_t>(Tk) + T, 16))
+        !make_token_maps(&p.tz, P.zbuf, Ld, static_cast<uint64_t>(Tk) + T))
       return MRLMOE_ERR_CUDA;
     p.gt = gt1;
     p.h = P.hbuf;
@@ -483,7 +489,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
     DownPolicy::Params p{};
     if (!make_map(&p.wd, w->w_down_e, 2, F, static_cast<uint64_t>(E) * Ld, 128) ||
         !make_map(&p.sd, w->w_sh_down, 2, F, Ld, 128) ||
-        !make_map(&p.th, P.hbuf, 2, F, static_cast<uint64_t>(Tk) + T, down_uses_pairs(*cfg) ? 16 : 32))
+        !make_token_maps(&p.th, P.hbuf, F, static_cast<uint64_t>(Tk) + T))
       return MRLMOE_ERR_CUDA;
     p.gt = gt2;
     p.perm = P.perm;

@@ -281,10 +281,39 @@ __device__ __forceinline__ Unit grouped_unit(const GroupTable &gt, const uint8_t
   return U;
 }
 
-// B operand: the unit's dispatched rows, loaded as 32-row boxes.
-__device__ __forceinline__ void load_rows(const CUtensorMap *tm, const Unit &U, int kb, uint32_t sb, uint32_t bar) {
-  const int nb = (U.nv + 31) >> 5;
-  for (int i = 0; i < nb; ++i) tma_load_2d(sb + i * 4096, tm, bar, kb * kBK, U.row0 + 32 * i);
+// Token rows y0 .. y0+n-1 (n a multiple of 16) of a K-major token tensor,
+// as 64-row boxes, then at most one 32-row and one 16-row box, back to back
+// in shared memory (128 B a row; every box is whole 8-row swizzle atoms).
+// One TMA copy costs its issuing thread on the order of a hundred cycles,
+// so a token tile of 160 rows takes 3 copies instead of 10 16-row ones.
+// PAIR: the cta_group::2 form, completing on the even CTA's barrier.
+struct TokenMaps {
+  CUtensorMap m16, m32, m64;  // the same tensor, boxes of 16 / 32 / 64 rows x 128 B
+};
+
+template <bool PAIR>
+__device__ __forceinline__ void load_token_rows(const TokenMaps &t, int x, int y0, int n, uint32_t sb, uint32_t bar) {
+  auto copy = [&](const CUtensorMap *m, int r) {
+    if constexpr (PAIR)
+      tma_load_2d_pair(sb + r * 128, m, bar, x, y0 + r);
+    else
+      tma_load_2d(sb + r * 128, m, bar, x, y0 + r);
+  };
+  int r = 0;
+  for (; r + 64 <= n; r += 64) copy(&t.m64, r);
+  if (r + 32 <= n) { copy(&t.m32, r); r += 32; }
+  if (r + 16 <= n) copy(&t.m16, r);
+}
+
+__device__ __forceinline__ void prefetch_token_maps(const TokenMaps &t) {
+  prefetch_tmap(&t.m16);
+  prefetch_tmap(&t.m32);
+  prefetch_tmap(&t.m64);
+}
+
+// B operand: the unit's dispatched rows, rounded up to a multiple of 32.
+__device__ __forceinline__ void load_rows(const TokenMaps &t, const Unit &U, int kb, uint32_t sb, uint32_t bar) {
+  load_token_rows<false>(t, kb * kBK, U.row0, (U.nv + 31) & ~31, sb, bar);
 }
 
 // --------------------------------------------------------------- gate/up
@@ -305,7 +334,7 @@ struct GluPolicy {
   struct Params {
     CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 64 (pairs) / 64 x 16 (single CTA)
     CUtensorMap sg, su;  // shared gate/up [F, L], box 64 x 64 (pairs) / 64 x 16 (single CTA)
-    CUtensorMap tz;      // dispatched z [(T*k+T), L], box 64 x 32
+    TokenMaps tz;        // dispatched z [(T*k+T), L], boxes 64 x 16/32/64
     GroupTable gt;
     __nv_bfloat16 *h;    // [(T*k+T), F]
     int F, L;
@@ -314,7 +343,7 @@ struct GluPolicy {
   struct EpiState {};
   static __device__ __forceinline__ void prefetch(const Params &p) {
     prefetch_tmap(&p.wg); prefetch_tmap(&p.wu); prefetch_tmap(&p.sg); prefetch_tmap(&p.su);
-    prefetch_tmap(&p.tz);
+    prefetch_token_maps(p.tz);
   }
   static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
   static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
@@ -341,7 +370,7 @@ struct GluPolicy {
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int, int kb, uint32_t sb,
                                                 uint32_t bar) {
-    load_rows(&p.tz, U, kb, sb, bar);
+    load_rows(p.tz, U, kb, sb, bar);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
     return idesc_bf16(128, round16(U.nv));
@@ -387,7 +416,7 @@ struct DownPolicy {
   struct Params {
     CUtensorMap wd;  // routed down [E*L, F], box 64 x 128
     CUtensorMap sd;  // shared down [L, F], box 64 x 128
-    CUtensorMap th;  // h [(T*k+T), F], box 64 x 32
+    TokenMaps th;    // h [(T*k+T), F], boxes 64 x 16/32/64
     GroupTable gt;
     const int32_t *perm;
     const float *wscaled;
@@ -397,7 +426,7 @@ struct DownPolicy {
   };
   struct EpiState {};
   static __device__ __forceinline__ void prefetch(const Params &p) {
-    prefetch_tmap(&p.wd); prefetch_tmap(&p.sd); prefetch_tmap(&p.th);
+    prefetch_tmap(&p.wd); prefetch_tmap(&p.sd); prefetch_token_maps(p.th);
   }
   static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
   static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
@@ -417,7 +446,7 @@ struct DownPolicy {
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int, int kb, uint32_t sb,
                                                 uint32_t bar) {
-    load_rows(&p.th, U, kb, sb, bar);
+    load_rows(p.th, U, kb, sb, bar);
   }
   static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
     return idesc_bf16(128, round16(U.nv));
