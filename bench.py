@@ -65,6 +65,9 @@ def parse_args():
                     help="tokens of the workload the CPU oracle baseline runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--route-only", action="store_true",
+                    help="time routing from x alone (down-projection, routers, top-k, dispatch: "
+                         "mrlmoe_route) and print its own JSON line; bf16 configs")
     return ap.parse_args()
 
 
@@ -268,10 +271,57 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_route_only(args):
+    """Routing from x (S1-S6 through mrlmoe_route) on one GPU: only the
+    down-projection and router weights are built.  Each call is timed alone
+    with CUDA events, an L2 flush (a 256 MB write) between calls."""
+    import torch
+    import sparse_moe_layer_mean_b200 as M
+    import workloads as W
+    s = shape_from_args(args)
+    if s.fp8:
+        raise SystemExit("--route-only runs the bf16 configs")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    weights = W.make_routing_weights(s, dev)
+    x = W.make_x(s, dev)
+    bias = W.make_bias(s, dev)
+    layer = M.MRLMoELayer(s, weights, device=dev)
+    routing = layer.routing_buffers()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        layer.route(bias, x=x, routing=routing)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        layer.route(bias, x=x, routing=routing)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    st = layer.device_status()
+    if st != 0:
+        raise SystemExit(f"device status {M.status_string(st)}")
+    ms = sum(times) / len(times)
+    print(json.dumps({"metric": "routing from x, tokens/s (down-projection, routers, top-k, dispatch)",
+                      "value": s.T / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+                      "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+                      "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": f"{s.name} routing: T={s.T} tokens, d_model {s.d_model} -> "
+                                             f"d_lat {s.d_lat}, {s.n_experts} experts top-{s.top_k}, "
+                                             f"R={s.n_routers} routers, bf16",
+                                 "T": s.T, "l2": "flushed between calls"}}),
+          flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.route_only:
+        return run_route_only(args)
     world, rank, local = dist_setup()
     import torch
     import torch.distributed as dist

@@ -235,6 +235,16 @@ def make_weights(s: LayerShape, device, seed: Optional[int] = None) -> Dict[str,
     return w
 
 
+def make_routing_weights(s: LayerShape, device, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """The tensors routing from x needs (down-projection, routers, alpha): the
+    same draws as make_weights, without the expert weights."""
+    seed = s.seed if seed is None else seed
+    D, L, E, R = s.d_model, s.d_lat, s.n_experts, s.n_routers
+    return {"w_down": normal((L, D), seed, _S_WDN, device, std=1.0 / math.sqrt(D)),
+            "w_router": normal((R, E, L), seed, _S_WR, device, std=1.0 / math.sqrt(L)),
+            "expert_scale": uniform((E,), 0.5, 1.5, seed, _S_ALPHA, device)}
+
+
 FP8_MATRICES = ("w_down", "w_gate", "w_up_e", "w_down_e", "w_sh_gate", "w_sh_up", "w_sh_down", "w_up")
 
 
