@@ -195,8 +195,8 @@ struct Glu2Policy {
   static constexpr int kBBytesMax = (kBN / 2) * 128;
   static constexpr int kEpiSmem = 4 * 32 * 17 * 4;
   static constexpr int kAuxSmem = kGroupAuxSmem;
-  using Params = GluPolicy::Params;
-  static __device__ __forceinline__ void prefetch(const Params &p) { GluPolicy::prefetch(p); }
+  using Params = GluParams;
+  static __device__ __forceinline__ void prefetch(const Params &p) { prefetch_glu(p); }
   static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
   static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
     return grouped_num_units(p.gt, aux);

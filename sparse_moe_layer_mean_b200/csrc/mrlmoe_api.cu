@@ -472,7 +472,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   GroupTable gt1{P.grp_off, P.grp_cnt, P.unit1, E, glu_m_tiles(*cfg)};
   GroupTable gt2{P.grp_off, P.grp_cnt, P.unit2, E, down_m_tiles(*cfg)};
   {
-    GluPolicy::Params p{};
+    GluParams p{};
     if (!make_map(&p.wg, w->w_gate, 2, Ld, static_cast<uint64_t>(E) * F, 64) ||
         !make_map(&p.wu, w->w_up_e, 2, Ld, static_cast<uint64_t>(E) * F, 64) ||
         !make_map(&p.sg, w->w_sh_gate, 2, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 2, Ld, F, 64) ||

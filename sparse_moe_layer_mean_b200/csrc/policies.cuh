@@ -3,8 +3,7 @@
 //  DensePolicy  : out[M,N] = bf16(a[M,K] w[N,K]^T)           (down-/up-projection)
 //  RouterPolicy : per token tile, R sigmoid routers x all experts, fused with
 //                 mean over routers, + bias, running top-k, renormalisation, alpha
-//  GluPolicy    : per (expert, 64-wide d_ff slice, token tile):
-//                 h = bf16(SiLU(z W_gate^T) * (z W_up^T))      (swap-AB: weights on M)
+//  GluParams    : parameters of the gate/up GEMM (Glu2Policy, gemm2_sm100.cuh)
 //  DownPolicy   : per (expert, 128-wide d_lat slice, token tile):
 //                 slot[t, j] = w'_{t,j} * (h W_down^T)          (swap-AB)
 #pragma once
@@ -317,91 +316,26 @@ __device__ __forceinline__ void load_rows(const TokenMaps &t, const Unit &U, int
 }
 
 // --------------------------------------------------------------- gate/up
-// A tile (128 rows) for the unit's 64 d_ff columns f0 = m*64 .. +63: TMEM lane
-// quarter q holds gate rows f0+16q .. +15 in its lanes 0-15 and the matching up
-// rows in lanes 16-31 (eight 16-row TMA boxes per K block).  In the epilogue
-// each warp therefore owns complete (gate, up) pairs and pairs them with one
-// shuffle across the half-warps.
-struct GluPolicy {
-  static constexpr int kStages = 4;
-  static constexpr int kGroup = 2;
-  static constexpr int kBN = 256;
-  static constexpr int kABytes = 128 * 128;
-  static constexpr int kBBytesMax = kBN * 128;
-  static constexpr int kEpiSmem = 0;
-  static constexpr int kAuxSmem = kGroupAuxSmem;
-  static constexpr int kUmmaKBytes = 32;
-  struct Params {
-    CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 64 (pairs) / 64 x 16 (single CTA)
-    CUtensorMap sg, su;  // shared gate/up [F, L], box 64 x 64 (pairs) / 64 x 16 (single CTA)
-    TokenMaps tz;        // dispatched z [(T*k+T), L], boxes 64 x 16/32/64
-    GroupTable gt;
-    __nv_bfloat16 *h;    // [(T*k+T), F]
-    int F, L;
-    uint32_t *status;
-  };
-  struct EpiState {};
-  static __device__ __forceinline__ void prefetch(const Params &p) {
-    prefetch_tmap(&p.wg); prefetch_tmap(&p.wu); prefetch_tmap(&p.sg); prefetch_tmap(&p.su);
-    prefetch_token_maps(p.tz);
-  }
-  static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
-  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
-    return grouped_num_units(p.gt, aux);
-  }
-  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.L / kBK; }
-  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
-    return grouped_unit(p.gt, aux, u, kBN);
-  }
-  static __device__ __forceinline__ uint32_t b_bytes(const Params &, const Unit &U, int) {
-    return ((U.nv + 31) >> 5) * 4096;
-  }
-  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int, int kb, uint32_t sa,
-                                                uint32_t bar) {
-    const bool sh = U.g == p.gt.E;
-    const CUtensorMap *mg = sh ? &p.sg : &p.wg;
-    const CUtensorMap *mu = sh ? &p.su : &p.wu;
-    const int row = (sh ? 0 : U.g * p.F) + U.m * 64;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      tma_load_2d(sa + (32 * q) * 128, mg, bar, kb * kBK, row + 16 * q);
-      tma_load_2d(sa + (32 * q + 16) * 128, mu, bar, kb * kBK, row + 16 * q);
-    }
-  }
-  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int, int kb, uint32_t sb,
-                                                uint32_t bar) {
-    load_rows(p.tz, U, kb, sb, bar);
-  }
-  static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U, int) {
-    return idesc_bf16(128, round16(U.nv));
-  }
-  static __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-    umma_f16(d, a, b, id, acc);
-  }
-  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
-                                                  int lane, int, EpiState &, uint8_t *) {
-    const bool up_half = lane >= 16;
-    const int f = U.m * 64 + q * 16 + (lane & 15);
-    __nv_bfloat16 *hcol = p.h + static_cast<size_t>(U.row0) * p.F + f;
-    for (int c0 = 0; c0 < U.nv; c0 += 32) {
-      float v[32];
-      tmem_ld32(taddr + c0, v);
-      tmem_ld_wait();
-      // gate lanes keep tokens c0..c0+15 and receive their up values; up lanes
-      // keep tokens c0+16..c0+31 and receive their gate values
-      const int tbase = c0 + (up_half ? 16 : 0);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float give = up_half ? v[i] : v[16 + i];
-        const float got = __shfl_xor_sync(0xffffffffu, give, 16);
-        const float g = up_half ? got : v[i];
-        const float u = up_half ? v[16 + i] : got;
-        if (tbase + i < U.nv)
-          hcol[static_cast<size_t>(tbase + i) * p.F] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
-      }
-    }
-  }
+// Parameters of the gate/up GEMM (run on CTA pairs by Glu2Policy in
+// gemm2_sm100.cuh): routed and shared gate/up weights, the dispatched latent
+// rows, and h.
+struct GluParams {
+  CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 64
+  CUtensorMap sg, su;  // shared gate/up [F, L], box 64 x 64
+  TokenMaps tz;        // dispatched z [(T*k+T), L], boxes 64 x 16/32/64
+  GroupTable gt;
+  __nv_bfloat16 *h;    // [(T*k+T), F]
+  int F, L;
+  uint32_t *status;
 };
+
+__device__ __forceinline__ void prefetch_glu(const GluParams &p) {
+  prefetch_tmap(&p.wg);
+  prefetch_tmap(&p.wu);
+  prefetch_tmap(&p.sg);
+  prefetch_tmap(&p.su);
+  prefetch_token_maps(p.tz);
+}
 
 // ------------------------------------------------------------------ down
 struct DownPolicy {
