@@ -221,6 +221,36 @@ def glu_kernel_flops(s):
     return 2 * (s.T * s.top_k + s.T) * s.d_lat * 2 * s.d_ff
 
 
+def fp8_peak_probe(dev, n=8192, seconds=1.0):
+    """Sustained e4m3 GEMM throughput of the vendor library on this GPU
+    (torch._scaled_mm, n x n x n, per-tensor scales), for context next to the
+    assumed e4m3 peak (2 x the measured sustained bf16 peak)."""
+    import torch
+    try:
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e1.record()
+        torch.cuda.synchronize()
+        reps = max(10, int(seconds * 1e3 / max(e0.elapsed_time(e1), 1e-3)))
+        e0.record()
+        for _ in range(reps):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e1.record()
+        torch.cuda.synchronize()
+        tflops = 2.0 * n ** 3 * reps / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        return {"tflops": round(tflops, 1), "gemm": f"{n}x{n}x{n} e4m3 -> bf16, torch._scaled_mm",
+                "reps": reps}
+    except (RuntimeError, AttributeError) as e:   # not available in this torch build
+        return {"unavailable": str(e).splitlines()[0][:200]}
+
+
 def cpu_baseline(s, weights_dev, x_dev, bias_dev, ntok):
     """The CPU oracle, as it stands, on the first ntok tokens of the batch."""
     import torch
@@ -411,6 +441,20 @@ def main():
         e2e_ms = a.elapsed_time(b)
         e2e = [e2e_ms, x.numel() * x.element_size(), y.numel() * y.element_size()]
 
+    # the balancing-bias update (the skewed workload's step after the forward), timed alone
+    bias_ms = None
+    if s.bias_kind == "zipf":
+        b2 = bias.clone()
+        for _ in range(3):
+            M.mrlmoe_bias_update(layer.cfg, routing["counts"], b2, 1e-3)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            M.mrlmoe_bias_update(layer.cfg, routing["counts"], b2, 1e-3)
+        b.record()
+        torch.cuda.synchronize()
+        bias_ms = a.elapsed_time(b) / args.steps
+
     # max over ranks
     if world > 1:
         red = max_over_ranks([ms, e2e[0] if e2e else 0.0] + stage_ms, dev)
@@ -440,7 +484,8 @@ def main():
             "config": {
                 "workload": f"{workload}: T={s.T} tokens, d_model {s.d_model} -> d_lat {s.d_lat}, "
                             f"{s.n_experts} experts top-{s.top_k} + 1 shared, d_ff {s.d_ff}, "
-                            f"R={s.n_routers} routers, bf16",
+                            f"R={s.n_routers} routers, "
+                            + ("e4m3 experts and projections (128x128 block scales), bf16 routers" if s.fp8 else "bf16"),
                 "T": s.T, "parallelism": f"replicas x{world} (expert weights replicated, own batch per GPU)",
                 "l2": "inputs larger than L2 (expert weights streamed every step)",
                 "touched_experts": touched,
@@ -471,6 +516,10 @@ def main():
         if e2e:
             line["e2e"] = {"value": job_throughput(world, s.T, args.steps, e2e[0]), "unit": UNIT,
                            "h2d_bytes_per_step": e2e[1], "d2h_bytes_per_step": e2e[2]}
+        if bias_ms is not None:
+            line["config"]["bias_update_ms"] = bias_ms
+        if s.fp8 and world == 1:
+            line["config"]["e4m3_peak_probe"] = fp8_peak_probe(dev)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(s, weights, x, bias, min(args.cpu_sample, s.T))
         print(json.dumps(line), flush=True)
