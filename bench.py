@@ -65,6 +65,9 @@ def parse_args():
                     help="tokens of the workload the CPU oracle baseline runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--aggregation", choices=["mean", "sum", "max"], default=None,
+                    help="router score aggregation (default: the config's, the mean)")
+    ap.add_argument("--routers", type=int, default=None, help="override the number of routers R")
     ap.add_argument("--route-only", action="store_true",
                     help="time routing from x alone (down-projection, routers, top-k, dispatch: "
                          "mrlmoe_route) and print its own JSON line; bf16 configs")
@@ -192,6 +195,10 @@ def shape_from_args(args):
         s = s.with_T(args.tokens)
     if args.experts:
         s = dataclasses.replace(s, n_experts=args.experts, name=f"{s.name}_E{args.experts}")
+    if args.routers:
+        s = dataclasses.replace(s, n_routers=args.routers, name=f"{s.name}_R{args.routers}")
+    if args.aggregation and args.aggregation != s.aggregation:
+        s = dataclasses.replace(s, aggregation=args.aggregation, name=f"{s.name}_{args.aggregation}")
     return s
 
 

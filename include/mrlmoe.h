@@ -63,10 +63,22 @@ typedef enum {
                                    the routers stay bf16, y is bf16               */
 } mrlmoe_dtype;
 
+/* How the R sigmoid router scores of a (token, expert) are aggregated into
+ * the score s used for selection and weights.  The pages say the routers'
+ * scores are aggregated without fixing the rule (aitest123, "模型结构";
+ * derekhsu, "多路由潛在 MoE"); MEAN is the layer's reading, SUM and MAX are
+ * the alternatives for sensitivity studies.                                   */
+typedef enum {
+  MRLMOE_AGG_MEAN = 0,          /* s = (sum_r sigmoid(l_r)) / R  (default)       */
+  MRLMOE_AGG_SUM = 1,           /* s = sum_r sigmoid(l_r)                        */
+  MRLMOE_AGG_MAX = 2            /* s = max_r sigmoid(l_r)                        */
+} mrlmoe_aggregation;
+
 /* Layer shape.  Limits checked on the host:
  *   T >= 1; d_model, d_lat, d_ff multiples of 128; 1 <= n_routers <= 8;
  *   16 <= n_experts <= 1024 with n_experts a multiple of 16;
- *   1 <= top_k <= min(n_experts, 16); rms_eps >= 0.  d_lat <= 8192, and in
+ *   1 <= top_k <= min(n_experts, 16); rms_eps >= 0; aggregation one of
+ *   mrlmoe_aggregation.  d_lat <= 8192, and in
  *   FP8 mode d_model, d_lat, d_ff <= 4096; beyond those the status is
  *   MRLMOE_ERR_UNSUPPORTED, otherwise MRLMOE_ERR_INVALID_ARG.                 */
 typedef struct {
@@ -79,6 +91,7 @@ typedef struct {
   int n_routers;    /* sigmoid routers R (4)                                     */
   float rms_eps;    /* RMSNorm epsilon (1e-6)                                    */
   mrlmoe_dtype dtype;
+  mrlmoe_aggregation aggregation;  /* router score aggregation (0 = mean)      */
 } mrlmoe_config;
 
 /* Weights: device pointers, caller-owned.  Element type is bf16 in BF16 mode;

@@ -98,20 +98,26 @@ def linear_bf16(a: torch.Tensor, w: torch.Tensor) -> torch.Tensor:
 # ---------------------------------------------------------------------------
 # routing
 # ---------------------------------------------------------------------------
-def router_scores(z: torch.Tensor, w_router: torch.Tensor) -> torch.Tensor:
-    """s[t, e] = fp32( (1/R) sum_r sigmoid(z[t] . w_router[r, e]) ).
+def router_scores(z: torch.Tensor, w_router: torch.Tensor, aggregation: str = "mean") -> torch.Tensor:
+    """s[t, e] = fp32( agg_r sigmoid(z[t] . w_router[r, e]) ), agg over the R
+    routers: "mean" (1/R) sum_r, "sum" sum_r, or "max" max_r (in fp64, one
+    rounding to fp32 at the end).
 
     R independently initialised sigmoid routers score every expert from the
     latent z [derekhsu; knowflow "关键信息"]; their scores are aggregated
-    [aitest123 "模型结构"] by the mean (an assumption).
+    [aitest123 "模型结构"] by a rule the pages do not give: the mean is the
+    layer's reading, sum and max are the alternatives it is compared with.
     """
+    if aggregation not in ("mean", "sum", "max"):
+        raise ValueError(f"unknown aggregation {aggregation!r}")
     z64 = _as_f64(z)
     R = w_router.shape[0]
     acc = torch.zeros(z.shape[0], w_router.shape[1], dtype=F64)
     for r in range(R):
         logit = z64 @ _as_f64(w_router[r]).T
-        acc += 1.0 / (1.0 + torch.exp(-logit))
-    return (acc / R).to(F32)
+        p = 1.0 / (1.0 + torch.exp(-logit))
+        acc = torch.maximum(acc, p) if aggregation == "max" else acc + p
+    return (acc / R if aggregation == "mean" else acc).to(F32)
 
 
 def select_topk(s: torch.Tensor, bias: torch.Tensor, k: int) -> torch.Tensor:
@@ -312,11 +318,12 @@ def _w(weights, name, fp8_deq, e=None):
 
 def forward(x: torch.Tensor, weights: Dict[str, torch.Tensor], bias: torch.Tensor,
             top_k: int, rms_eps: float = 1e-6, fp8: bool = False,
-            scores: Optional[torch.Tensor] = None) -> OracleResult:
+            scores: Optional[torch.Tensor] = None, aggregation: str = "mean") -> OracleResult:
     """The layer on CPU, step by step.
 
     1. z = bf16(x W_dn^T)                          down-projection 4096 -> 2048
-    2-3. s = mean_r sigmoid(zx W_r^T) (fp32)        multi-router scores, where zx
+    2-3. s = agg_r sigmoid(zx W_r^T) (fp32)         multi-router scores (agg: mean by
+         default, or sum / max, see router_scores), where zx
          is the unrounded latent x W_dn^T (the routers read it at full precision)
     4-5. top-k of s + b; w = renormalised s; w' = w * alpha
     6. dispatch record (counts, offsets, perm, inv_perm)
@@ -343,7 +350,7 @@ def forward(x: torch.Tensor, weights: Dict[str, torch.Tensor], bias: torch.Tenso
         xin = quantize_act_1x128(_as_f64(x)) if fp8 else _as_f64(x)
         zx = xin @ _as_f64(_w(weights, "w_down", deq)).T
         z = bf16_round(zx)
-        s = router_scores(zx, weights["w_router"])
+        s = router_scores(zx, weights["w_router"], aggregation)
     else:
         z, s = None, scores.to(F32)
     T = s.shape[0]

@@ -40,7 +40,7 @@ class MrlmoeError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("T", c_int), ("d_model", c_int), ("d_lat", c_int), ("n_experts", c_int),
                 ("top_k", c_int), ("d_ff", c_int), ("n_routers", c_int), ("rms_eps", c_float),
-                ("dtype", c_int)]
+                ("dtype", c_int), ("aggregation", c_int)]
 
 
 WEIGHT_FIELDS = ("w_down", "w_router", "w_gate", "w_up_e", "w_down_e", "w_sh_gate", "w_sh_up",
@@ -117,12 +117,17 @@ def _stream_ptr(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
+AGGREGATIONS = {"mean": 0, "sum": 1, "max": 2}   # mrlmoe_aggregation
+
+
 def make_config(shape, T: Optional[int] = None, fp8: Optional[bool] = None) -> Config:
-    """Config from a workloads.LayerShape-like object (duck-typed)."""
+    """Config from a workloads.LayerShape-like object (duck-typed; a missing
+    `aggregation` attribute means the mean)."""
     f8 = shape.fp8 if fp8 is None else fp8
     return Config(shape.T if T is None else T, shape.d_model, shape.d_lat, shape.n_experts,
                   shape.top_k, shape.d_ff, shape.n_routers, float(shape.rms_eps),
-                  MRLMOE_FP8_E4M3_BLOCK128 if f8 else MRLMOE_BF16)
+                  MRLMOE_FP8_E4M3_BLOCK128 if f8 else MRLMOE_BF16,
+                  AGGREGATIONS[getattr(shape, "aggregation", "mean")])
 
 
 def make_weights(w: Dict[str, object]) -> Weights:

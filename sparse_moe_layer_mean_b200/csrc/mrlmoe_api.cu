@@ -32,6 +32,8 @@ mrlmoe_status check_config(const mrlmoe_config *c) {
   if (c->n_routers < 1 || c->n_routers > 8) return MRLMOE_ERR_INVALID_ARG;
   if (!(c->rms_eps >= 0.f)) return MRLMOE_ERR_INVALID_ARG;
   if (c->dtype != MRLMOE_BF16 && c->dtype != MRLMOE_FP8_E4M3_BLOCK128) return MRLMOE_ERR_INVALID_ARG;
+  if (c->aggregation != MRLMOE_AGG_MEAN && c->aggregation != MRLMOE_AGG_SUM && c->aggregation != MRLMOE_AGG_MAX)
+    return MRLMOE_ERR_INVALID_ARG;
   // the FP8 GEMMs stage at most kF8MaxKB scales of 128-wide K blocks per unit
   if (c->dtype == MRLMOE_FP8_E4M3_BLOCK128 &&
       (c->d_model > 128 * kF8MaxKB || c->d_lat > 128 * kF8MaxKB || c->d_ff > 128 * kF8MaxKB))
@@ -409,6 +411,7 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
     p.cand_s = P.cand_s;
     p.cand_i = P.cand_i;
     p.T = T; p.L = Ld; p.E = E; p.R = R; p.ec = ec; p.k = k;
+    p.agg = static_cast<int>(c.aggregation);
     p.m_tiles = (T + 127) / 128;
     p.parts = router_parts(c, sms);
     p.status = P.status;

@@ -2,7 +2,8 @@
 //
 //  DensePolicy  : out[M,N] = bf16(a[M,K] w[N,K]^T)           (down-/up-projection)
 //  RouterPolicy : per token tile, R sigmoid routers x all experts, fused with
-//                 mean over routers, + bias, running top-k, renormalisation, alpha
+//                 the aggregation over routers (mean / sum / max), + bias,
+//                 running top-k, renormalisation, alpha
 //  GluParams    : parameters of the gate/up GEMM (Glu2Policy, gemm2_sm100.cuh)
 //  DownPolicy   : per (expert, 128-wide d_lat slice, token tile):
 //                 slot[t, j] = w'_{t,j} * (h W_down^T)          (swap-AB)
@@ -132,6 +133,7 @@ struct RouterPolicy {
     float *cand_v, *cand_s;
     int32_t *cand_i;
     int T, L, E, R, ec, k, m_tiles, parts;
+    int agg;  // mrlmoe_aggregation: 0 mean, 1 sum, 2 max of the R sigmoid scores
     uint32_t *status;
   };
   struct EpiState {
@@ -191,15 +193,20 @@ struct RouterPolicy {
         float v[16];
         tmem_ld16(taddr + r * p.ec + j0, v);
         tmem_ld_wait();
+        if (p.agg == 2) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] += sigmoidf_(v[i]);
+          for (int i = 0; i < 16; ++i) acc[i] = fmaxf(acc[i], sigmoidf_(v[i]));  // sigmoid >= 0
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] += sigmoidf_(v[i]);
+        }
       }
       const int e0 = (U.g * U.nsub + sub) * p.ec + j0;
       float s16[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        // mean of the R router scores: (sum) / R; R = 2^n makes this exact scaling
-        s16[i] = (p.R & (p.R - 1)) == 0 ? acc[i] * invR : acc[i] / static_cast<float>(p.R);
+        // mean: (sum) / R (R = 2^n makes this an exact scaling); sum and max as accumulated
+        s16[i] = p.agg != 0 ? acc[i] : (p.R & (p.R - 1)) == 0 ? acc[i] * invR : acc[i] / static_cast<float>(p.R);
         const float sb = s16[i] + __ldg(p.bias + e0 + i);
         st.tk.offer(sb, e0 + i, s16[i]);
       }

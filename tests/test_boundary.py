@@ -49,8 +49,11 @@ def test_workspace_size_valid_and_invalid():
     assert M.mrlmoe_workspace_size(_cfg()) > 0
     for bad in (dict(T=0), dict(d_model=200), dict(d_lat=0), dict(d_ff=100), dict(n_experts=8),
                 dict(n_experts=24 + 1), dict(top_k=0), dict(top_k=17), dict(top_k=17, n_experts=16),
-                dict(n_routers=0), dict(n_routers=9), dict(rms_eps=-1.0), dict(dtype=7)):
+                dict(n_routers=0), dict(n_routers=9), dict(rms_eps=-1.0), dict(dtype=7),
+                dict(aggregation=3), dict(aggregation=-1)):
         assert M.mrlmoe_workspace_size(_cfg(**bad)) == 0, bad
+    for agg in (0, 1, 2):                                       # mean, sum, max
+        assert M.mrlmoe_workspace_size(_cfg(aggregation=agg)) > 0
     # the FP8 variant stages at most 32 K-block scales per GEMM unit: K <= 4096
     for big in (dict(d_model=4224), dict(d_lat=4224), dict(d_ff=4224)):
         assert M.mrlmoe_workspace_size(_cfg(dtype=1, **big)) == 0, big

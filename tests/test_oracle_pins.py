@@ -110,6 +110,50 @@ def test_router_aggregation_is_the_mean():
     assert torch.all(O.router_scores(z, torch.zeros(3, 5, 8, dtype=torch.bfloat16)) == 0.5)
 
 
+def test_router_sum_and_max_closed_forms():
+    # the alternative aggregations on routers r and -r: the sum is exactly 1,
+    # the max is sigmoid(|a|), computed here from a hand-summed logit
+    g = torch.Generator().manual_seed(6)
+    z = torch.randn(5, 8, generator=g).to(torch.bfloat16)
+    w = torch.randn(1, 4, 8, generator=g).to(torch.bfloat16)
+    assert torch.all(O.router_scores(z, torch.cat([w, -w]), "sum") == 1.0)
+    smax = O.router_scores(z, torch.cat([w, -w]), "max")
+    for t in range(5):
+        for e in range(4):
+            a = math.fsum(float(z[t, i]) * float(w[0, e, i]) for i in range(8))
+            assert smax[t, e].item() == np.float32(_sig(abs(a)))
+
+
+def test_router_aggregations_relate_exactly():
+    g = torch.Generator().manual_seed(7)
+    z = torch.randn(16, 12, generator=g).to(torch.bfloat16)
+    w4 = torch.randn(4, 7, 12, generator=g).to(torch.bfloat16)
+    # R = 4: the sum is 4 x the mean (scaling by 2^2 commutes with the fp32 rounding)
+    assert torch.equal(O.router_scores(z, w4, "sum"), 4 * O.router_scores(z, w4, "mean"))
+    # R = 1: all three rules are the single router's sigmoid
+    w1 = w4[:1]
+    m = O.router_scores(z, w1, "mean")
+    assert torch.equal(m, O.router_scores(z, w1, "sum")) and torch.equal(m, O.router_scores(z, w1, "max"))
+    # the max is at least the mean and at most the sum
+    mx, mn, sm = (O.router_scores(z, w4, a) for a in ("max", "mean", "sum"))
+    assert torch.all(mx >= mn) and torch.all(mx <= sm)
+    with pytest.raises(ValueError):
+        O.router_scores(z, w4, "median")
+
+
+def test_router_max_brute_force():
+    g = torch.Generator().manual_seed(8)
+    T, L, E, R = 3, 10, 4, 3
+    z = torch.randn(T, L, generator=g).to(torch.bfloat16)
+    wr = torch.randn(R, E, L, generator=g).to(torch.bfloat16)
+    s = O.router_scores(z, wr, "max")
+    for t in range(T):
+        for e in range(E):
+            best = max(_sig(math.fsum(float(z[t, i]) * float(wr[r, e, i]) for i in range(L)))
+                       for r in range(R))
+            assert s[t, e].item() == np.float32(best)
+
+
 # --------------------------------------------------------------- selection
 def _valid_topk(sb, sel, k):
     E = sb.shape[0]

@@ -53,6 +53,7 @@ class LayerShape:
     rms_eps: float = 1e-6
     fp8: bool = False
     bias_kind: str = "zero"        # "zero" | "zipf"
+    aggregation: str = "mean"      # router score aggregation: "mean" | "sum" | "max"
     outlier_frac: float = 0.0      # fraction of x channels scaled by outlier_scale
     outlier_scale: float = 20.0
     seed: int = 0
