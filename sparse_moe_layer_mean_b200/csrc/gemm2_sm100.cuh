@@ -177,7 +177,7 @@ __device__ __forceinline__ int round32(int n) { return (n + 31) & ~31; }
 __device__ __forceinline__ void load_rows_half(const TokenMaps &t, const Unit &U, int kb, uint32_t sb,
                                                uint32_t bar_cl, uint32_t rank) {
   const int half = round32(U.nv) >> 1;
-  load_token_rows<true>(t, kb * kBK, U.row0 + static_cast<int>(rank) * half, half, sb, bar_cl);
+  load_token_rows<true>(t, kb, U.row0 + static_cast<int>(rank) * half, half, sb, bar_cl);
 }
 
 // gate/up over a CTA pair: unit = (group, 128-wide d_ff slice, <= 256 tokens);
@@ -227,7 +227,10 @@ struct Glu2Policy {
     float *xb = reinterpret_cast<float *>(epi);  // [4][32][17]
     const bool is_gate = q < 2;
     const int pair = q & 1;
-    const int f = (U.m * 2 + static_cast<int>(rank)) * 64 + pair * 32 + lane;
+    // h is K-blocked: the CTA's 64 d_ff columns are one plane, so the unit's
+    // rows land in one contiguous N x 128 B range of it
+    const int plane = U.m * 2 + static_cast<int>(rank);
+    __nv_bfloat16 *hp = p.h + static_cast<size_t>(plane) * p.rows * 64 + pair * 32 + lane;
     const size_t row0 = static_cast<size_t>(U.row0);
     for (int c0 = 0; c0 < U.nv; c0 += 32) {
       float v[32];
@@ -243,7 +246,7 @@ struct Glu2Policy {
       for (int c = 0; c < 16; ++c) {
         const float g = is_gate ? v[c] : other[c];
         const float u = is_gate ? other[c] : v[16 + c];
-        if (cbase + c < U.nv) p.h[(row0 + cbase + c) * p.F + f] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
+        if (cbase + c < U.nv) hp[(row0 + cbase + c) * 64] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
       }
       named_bar_sync(2, 128);
     }

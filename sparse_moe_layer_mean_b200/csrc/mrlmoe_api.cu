@@ -153,8 +153,16 @@ bool make_map(CUtensorMap *m, const void *base, int esize, uint64_t inner, uint6
 
 // The three box heights of a bf16 token tensor [rows, inner] (load_token_rows).
 bool make_token_maps(TokenMaps *t, const void *base, uint64_t inner, uint64_t rows) {
+  t->plane_rows = 0;
   return make_map(&t->m16, base, 2, inner, rows, 16) && make_map(&t->m32, base, 2, inner, rows, 32) &&
          make_map(&t->m64, base, 2, inner, rows, 64);
+}
+
+// The same for a K-blocked bf16 token tensor [K/64][rows][64].
+bool make_token_maps_blocked(TokenMaps *t, const void *base, uint64_t K, uint64_t rows) {
+  if (!make_token_maps(t, base, 64, (K / 64) * rows)) return false;
+  t->plane_rows = static_cast<int>(rows);
+  return true;
 }
 
 // Make the device that owns `p` current; reject host/unknown pointers.
@@ -483,7 +491,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
       return MRLMOE_ERR_CUDA;
     p.gt = gt1;
     p.h = P.hbuf;
-    p.F = F; p.L = Ld;
+    p.F = F; p.L = Ld; p.rows = Tk + T;
     p.status = P.status;
     MRL_TRY(launch_gemm_pair<Glu2Policy>(p, sms, st));
   }
@@ -492,7 +500,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
     DownPolicy::Params p{};
     if (!make_map(&p.wd, w->w_down_e, 2, F, static_cast<uint64_t>(E) * Ld, 128) ||
         !make_map(&p.sd, w->w_sh_down, 2, F, Ld, 128) ||
-        !make_token_maps(&p.th, P.hbuf, F, static_cast<uint64_t>(Tk) + T))
+        !make_token_maps_blocked(&p.th, P.hbuf, F, static_cast<uint64_t>(Tk) + T))
       return MRLMOE_ERR_CUDA;
     p.gt = gt2;
     p.perm = P.perm;

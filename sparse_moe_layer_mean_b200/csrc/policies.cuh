@@ -293,17 +293,27 @@ __device__ __forceinline__ Unit grouped_unit(const GroupTable &gt, const uint8_t
 // One TMA copy costs its issuing thread on the order of a hundred cycles,
 // so a token tile of 160 rows takes 3 copies instead of 10 16-row ones.
 // PAIR: the cta_group::2 form, completing on the even CTA's barrier.
+//
+// Two layouts of a bf16 token tensor [rows, K]: row-major (plane_rows == 0;
+// K block kb of row r at x = 64 kb, y = r), or K-blocked, [K/64][rows][64]
+// (plane_rows == rows; the tensor map sees [K/64 * rows, 64] and K block kb
+// of row r sits at x = 0, y = kb * rows + r).  In the blocked layout a tile of
+// consecutive rows is one contiguous range for every K block, for the TMA
+// loads here and for the epilogue that writes it.
 struct TokenMaps {
   CUtensorMap m16, m32, m64;  // the same tensor, boxes of 16 / 32 / 64 rows x 128 B
+  int plane_rows;             // 0: row-major; else rows per K-block plane
 };
 
 template <bool PAIR>
-__device__ __forceinline__ void load_token_rows(const TokenMaps &t, int x, int y0, int n, uint32_t sb, uint32_t bar) {
+__device__ __forceinline__ void load_token_rows(const TokenMaps &t, int kb, int y0, int n, uint32_t sb, uint32_t bar) {
+  const int x = t.plane_rows ? 0 : kb * kBK;
+  const int yb = t.plane_rows ? kb * t.plane_rows + y0 : y0;
   auto copy = [&](const CUtensorMap *m, int r) {
     if constexpr (PAIR)
-      tma_load_2d_pair(sb + r * 128, m, bar, x, y0 + r);
+      tma_load_2d_pair(sb + r * 128, m, bar, x, yb + r);
     else
-      tma_load_2d(sb + r * 128, m, bar, x, y0 + r);
+      tma_load_2d(sb + r * 128, m, bar, x, yb + r);
   };
   int r = 0;
   for (; r + 64 <= n; r += 64) copy(&t.m64, r);
@@ -319,7 +329,7 @@ __device__ __forceinline__ void prefetch_token_maps(const TokenMaps &t) {
 
 // B operand: the unit's dispatched rows, rounded up to a multiple of 32.
 __device__ __forceinline__ void load_rows(const TokenMaps &t, const Unit &U, int kb, uint32_t sb, uint32_t bar) {
-  load_token_rows<false>(t, kb * kBK, U.row0, (U.nv + 31) & ~31, sb, bar);
+  load_token_rows<false>(t, kb, U.row0, (U.nv + 31) & ~31, sb, bar);
 }
 
 // --------------------------------------------------------------- gate/up
@@ -329,10 +339,10 @@ __device__ __forceinline__ void load_rows(const TokenMaps &t, const Unit &U, int
 struct GluParams {
   CUtensorMap wg, wu;  // routed gate/up [E*F, L], box 64 x 64
   CUtensorMap sg, su;  // shared gate/up [F, L], box 64 x 64
-  TokenMaps tz;        // dispatched z [(T*k+T), L], boxes 64 x 16/32/64
+  TokenMaps tz;        // dispatched z [(T*k+T), L] row-major, boxes 64 x 16/32/64
   GroupTable gt;
-  __nv_bfloat16 *h;    // [(T*k+T), F]
-  int F, L;
+  __nv_bfloat16 *h;    // [F/64][T*k+T][64], K-blocked (see TokenMaps)
+  int F, L, rows;      // rows = T*k+T
   uint32_t *status;
 };
 
@@ -357,7 +367,7 @@ struct DownPolicy {
   struct Params {
     CUtensorMap wd;  // routed down [E*L, F], box 64 x 128
     CUtensorMap sd;  // shared down [L, F], box 64 x 128
-    TokenMaps th;    // h [(T*k+T), F], boxes 64 x 16/32/64
+    TokenMaps th;    // h [F/64][T*k+T][64] K-blocked, boxes 64 x 16/32/64
     GroupTable gt;
     const int32_t *perm;
     const float *wscaled;
