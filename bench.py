@@ -424,28 +424,58 @@ def main():
     if layer.device_status() != 0:
         raise RuntimeError("device status non-zero after the timed region")
 
-    # e2e: pinned host x -> device, forward, y -> pinned host, every step
+    # e2e: pinned host x -> device, forward, y -> pinned host, every step.  The
+    # copies run on the copy engines, pipelined as a server would run them:
+    # step i+1's x goes up (H2D stream) while step i computes, step i-1's y
+    # comes back (D2H stream); device x / y are double-buffered.  Every step's
+    # copies lie inside the timed region.
     e2e = None
     if not args.no_e2e:
         xh = x.cpu().pin_memory()
-        yh = torch.empty_like(y, device="cpu").pin_memory()
-        xd = torch.empty_like(x)
-        for _ in range(2):
-            xd.copy_(xh, non_blocking=True)
-            layer(xd, bias, y=y)
-            yh.copy_(y, non_blocking=True)
-        torch.cuda.synchronize()
+        yh = [torch.empty_like(y, device="cpu").pin_memory() for _ in range(2)]
+        xd = [torch.empty_like(x) for _ in range(2)]
+        yd = [torch.empty_like(y) for _ in range(2)]
+        comp = torch.cuda.current_stream()
+        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+
+        def pipelined(n):
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(comp)
+            h2d.wait_event(t0)
+            fwd_done, y_read = [None, None], [None, None]
+            for i in range(n):
+                j = i % 2
+                if fwd_done[j] is not None:          # step i-2 has read xd[j]
+                    h2d.wait_event(fwd_done[j])
+                with torch.cuda.stream(h2d):
+                    xd[j].copy_(xh, non_blocking=True)
+                up = torch.cuda.Event()
+                up.record(h2d)
+                comp.wait_event(up)
+                if y_read[j] is not None:            # step i-2's y has left yd[j]
+                    comp.wait_event(y_read[j])
+                layer(xd[j], bias, y=yd[j], stream=comp)
+                fwd_done[j] = torch.cuda.Event()
+                fwd_done[j].record(comp)
+                d2h.wait_event(fwd_done[j])
+                with torch.cuda.stream(d2h):
+                    yh[j].copy_(yd[j], non_blocking=True)
+                y_read[j] = torch.cuda.Event()
+                y_read[j].record(d2h)
+            for ev in y_read:
+                if ev is not None:
+                    comp.wait_event(ev)
+            t1.record(comp)
+            torch.cuda.synchronize()
+            return t0.elapsed_time(t1)
+
+        pipelined(3)
         if world > 1:
             dist.barrier(device_ids=[local])
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(args.steps):
-            xd.copy_(xh, non_blocking=True)
-            layer(xd, bias, y=y)
-            yh.copy_(y, non_blocking=True)
-        b.record()
-        torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b)
+        e2e_ms = pipelined(args.steps)
+        # the layer is bitwise reproducible: the last step read back equals the device-only result
+        if not torch.equal(yh[(args.steps - 1) % 2], y.cpu()):
+            raise RuntimeError("pipelined end-to-end result differs from the device-only forward")
         e2e = [e2e_ms, x.numel() * x.element_size(), y.numel() * y.element_size()]
 
     # the balancing-bias update (the skewed workload's step after the forward), timed alone
