@@ -14,7 +14,7 @@
 // Tokens are on M (TMEM lanes) and weights on N in every FP8 GEMM, and a
 // unit's 128 N columns fall in at most two weight blocks (one per column
 // half), so the scale a thread applies to its 64 columns is ONE scalar per K
-// block: two 4-byte shared loads and an FMUL, then 64 FFMAs.  (With tokens on
+// block: two 4-byte shared loads and an FMUL, then 32 packed fp32x2 FMAs.  (With tokens on
 // N every thread would need 64 distinct column scales per K block; as warp-
 // wide broadcast loads those cost 8 KB of shared-memory return bandwidth per
 // warp per K block and throttled the whole pipeline.)
@@ -207,8 +207,14 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(free0 + 8 * j);  // the partial is in registers
+        // packed fp32x2 FMAs (round to nearest per lane: the same values as fmaf)
+        const float2 s2 = make_float2(s, s);
 #pragma unroll
-        for (int i = 0; i < kF8Half; ++i) acc[i] = fmaf(v[i], s, acc[i]);
+        for (int i = 0; i < kF8Half; i += 2) {
+          const float2 r = __ffma2_rn(make_float2(v[i], v[i + 1]), s2, make_float2(acc[i], acc[i + 1]));
+          acc[i] = r.x;
+          acc[i + 1] = r.y;
+        }
       }
       Unit U;
       {
