@@ -236,7 +236,11 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 }
 
 constexpr int kQuantWarps = 8;
+constexpr int kQuantBatch = 4;   // warp iterations whose loads are in flight together
 
+// A warp's loads are issued kQuantBatch iterations (8 blocks) at a time before
+// those blocks are reduced, so a warp waits for memory once per 8 blocks
+// while the block keeps few registers (and many warps per SM).
 __global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_kernel(
     const __nv_bfloat16 *__restrict__ in, long ld_in, int rows, int K, const int32_t *__restrict__ perm, int k,
     int Tk, uint8_t *__restrict__ q, float *__restrict__ s, long s_ld) {
@@ -249,40 +253,44 @@ __global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_kernel(
   if (perm) src = r < Tk ? __ldg(perm + r) / k : r - Tk;
   const __nv_bfloat16 *row_in = in + src * ld_in;
   uint8_t *row_q = q + static_cast<long>(r) * K;
-  for (int b0 = 0; b0 < kbs; b0 += 2) {
-    const int b = b0 + half;
-    const bool live = b < kbs;
-    float v[8];
-    if (live) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(row_in + b * 128 + hl * 8));
-      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+  for (int it0 = 0; 2 * it0 < kbs; it0 += kQuantBatch) {
+    uint4 raw[kQuantBatch];
+#pragma unroll
+    for (int j = 0; j < kQuantBatch; ++j) {
+      const int b = 2 * (it0 + j) + half;
+      raw[j] = b < kbs ? __ldg(reinterpret_cast<const uint4 *>(row_in + b * 128 + hl * 8)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < kQuantBatch; ++j) {
+      if (2 * (it0 + j) >= kbs) break;  // uniform across the warp
+      const int b = 2 * (it0 + j) + half;
+      const bool live = b < kbs;
+      float v[8];
+      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[j]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         v[2 * i] = __low2float(h2[i]);
         v[2 * i + 1] = __high2float(h2[i]);
       }
-    } else {
+      float amax = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.f;
-    }
-    float amax = 0.f;
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    float scale = 1.0f, inv = 0.0f;
-    if (amax != 0.0f) {
-      scale = amax / 448.0f;
-      inv = 448.0f / amax;
-    }
-    if (live) {
-      uint2 codes;
-      codes.x = static_cast<uint32_t>(e4m3x2(v[0] * inv, v[1] * inv)) |
-                (static_cast<uint32_t>(e4m3x2(v[2] * inv, v[3] * inv)) << 16);
-      codes.y = static_cast<uint32_t>(e4m3x2(v[4] * inv, v[5] * inv)) |
-                (static_cast<uint32_t>(e4m3x2(v[6] * inv, v[7] * inv)) << 16);
-      *reinterpret_cast<uint2 *>(row_q + b * 128 + hl * 8) = codes;
-      if (hl == 0) s[s_ld ? b * s_ld + r : static_cast<long>(r) * kbs + b] = scale;
+      for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      float scale = 1.0f, inv = 0.0f;
+      if (amax != 0.0f) {
+        scale = amax / 448.0f;
+        inv = 448.0f / amax;
+      }
+      if (live) {
+        uint2 codes;
+        codes.x = static_cast<uint32_t>(e4m3x2(v[0] * inv, v[1] * inv)) |
+                  (static_cast<uint32_t>(e4m3x2(v[2] * inv, v[3] * inv)) << 16);
+        codes.y = static_cast<uint32_t>(e4m3x2(v[4] * inv, v[5] * inv)) |
+                  (static_cast<uint32_t>(e4m3x2(v[6] * inv, v[7] * inv)) << 16);
+        *reinterpret_cast<uint2 *>(row_q + b * 128 + hl * 8) = codes;
+        if (hl == 0) s[s_ld ? b * s_ld + r : static_cast<long>(r) * kbs + b] = scale;
+      }
     }
   }
 }
