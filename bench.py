@@ -41,8 +41,8 @@ def kernels_per_step(s, sms: int) -> int:
         if c * s.n_routers <= 256 and s.n_experts % c == 0:
             ec = c
             break
-    chunks = s.n_experts // ec
     m_tiles = (s.T + 127) // 128
+    chunks = s.n_experts // ec
     parts = 1
     while parts * 2 <= chunks and chunks % (parts * 2) == 0 and m_tiles * parts * 2 <= sms:
         parts *= 2

@@ -45,7 +45,11 @@ mrlmoe_status check_config(const mrlmoe_config *c) {
 }
 
 // Router chunk: experts per accumulator so that R * ec <= 256 and ec | E.
-int router_ec(int E, int R) {
+// The widest expert chunk that fits one accumulator (R * ec <= 256 columns).
+// (Narrower chunks for decode-sized T, to spread the router over more CTAs,
+// measured slower: more partial lists to merge and MMAs at the instruction's
+// minimum cost.)
+int router_ec(int E, int R, int) {
   for (int ec = 256; ec >= 16; ec >>= 1)
     if (ec * R <= 256 && E % ec == 0) return ec;
   return 16;
@@ -55,7 +59,7 @@ int router_ec(int E, int R) {
 // CTAs (a power of two dividing the chunk count) so that m_tiles * parts
 // fills the SMs; parts > 1 adds a small merge of the partial selections.
 int router_parts(const mrlmoe_config &c, int sms) {
-  const int chunks = c.n_experts / router_ec(c.n_experts, c.n_routers);
+  const int chunks = c.n_experts / router_ec(c.n_experts, c.n_routers, c.T);
   const int m_tiles = (c.T + 127) / 128;
   int parts = 1;
   while (parts * 2 <= chunks && chunks % (parts * 2) == 0 && m_tiles * parts * 2 <= std::max(sms, 1)) parts *= 2;
@@ -379,6 +383,33 @@ mrlmoe_status launch_dense8(const uint8_t *aq, const float *as_t, const void *wq
   return MRLMOE_OK;
 }
 
+// bf16 projection out = bf16(a w^T) (and optionally the residual of that
+// rounding): 256-column tiles, or 64-column tiles when the 256-wide grid would
+// occupy fewer than half the SMs (decode-sized M).
+template <class DP>
+mrlmoe_status launch_dense_with(const void *a, const void *w, __nv_bfloat16 *out, __nv_bfloat16 *out_lo, int M, int N,
+                                int K, uint32_t *status, int sms, cudaStream_t st) {
+  typename DP::Params p{};
+  if (!make_map(&p.ta, a, 2, K, M, 128) || !make_map(&p.tb, w, 2, K, N, DP::kBN)) return MRLMOE_ERR_CUDA;
+  p.out = out;
+  p.out_lo = out_lo;
+  p.ldo = N;
+  p.M = M; p.N = N; p.K = K;
+  p.m_tiles = (M + 127) / 128;
+  p.n_tiles = (N + DP::kBN - 1) / DP::kBN;
+  p.status = status;
+  MRL_TRY(launch_gemm<DP>(p, std::min(sms, p.m_tiles * p.n_tiles), st));
+  return MRLMOE_OK;
+}
+
+mrlmoe_status launch_dense_bf16(const void *a, const void *w, __nv_bfloat16 *out, __nv_bfloat16 *out_lo, int M,
+                                int N, int K, uint32_t *status, int sms, cudaStream_t st) {
+  const int wide_tiles = ((M + 127) / 128) * ((N + DensePolicy::kBN - 1) / DensePolicy::kBN);
+  if (2 * wide_tiles < sms && N % DenseNarrowPolicy::kBN == 0)
+    return launch_dense_with<DenseNarrowPolicy>(a, w, out, out_lo, M, N, K, status, sms, st);
+  return launch_dense_with<DensePolicy>(a, w, out, out_lo, M, N, K, status, sms, st);
+}
+
 // Routing from x: down-projection into the tail of zbuf, then the fused router.
 mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weights *w, const float *bias,
                                        const void *x, const Ptrs &P, int sms, cudaStream_t st,
@@ -390,22 +421,13 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
     mrlmoe_status s = launch_dense8(P.xq, P.xs, w->w_down, w->s_down, T, Ld, D, z, P.zlo, P, sms, st);
     if (s != MRLMOE_OK) return s;
   } else {
-    DensePolicy::Params p{};
-    if (!make_map(&p.ta, x, 2, D, T, 128) || !make_map(&p.tb, w->w_down, 2, D, Ld, DensePolicy::kBN))
-      return MRLMOE_ERR_CUDA;
-    p.out = z;
-    p.out_lo = P.zlo;
-    p.ldo = Ld;
-    p.M = T; p.N = Ld; p.K = D;
-    p.m_tiles = (T + 127) / 128;
-    p.n_tiles = (Ld + DensePolicy::kBN - 1) / DensePolicy::kBN;
-    p.status = P.status;
-    MRL_TRY(launch_gemm<DensePolicy>(p, std::min(sms, p.m_tiles * p.n_tiles), st));
+    mrlmoe_status s = launch_dense_bf16(x, w->w_down, z, P.zlo, T, Ld, D, P.status, sms, st);
+    if (s != MRLMOE_OK) return s;
   }
   if (ev) MRL_TRY(cudaEventRecord(static_cast<cudaEvent_t>(ev[1]), st));
   {
     RouterPolicy::Params p{};
-    const int ec = router_ec(E, R);
+    const int ec = router_ec(E, R, T);
     if (!make_map(&p.ta, z, 2, Ld, T, 128) || !make_map(&p.ta_lo, P.zlo, 2, Ld, T, 128) ||
         !make_map(&p.tb, w->w_router, 2, Ld, static_cast<uint64_t>(R) * E, ec))
       return MRLMOE_ERR_CUDA;
@@ -520,16 +542,9 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   MRL_TRY(cudaGetLastError());
   if (!mark(7)) return MRLMOE_ERR_CUDA;
   {
-    DensePolicy::Params p{};
-    if (!make_map(&p.ta, P.nbuf, 2, Ld, T, 128) || !make_map(&p.tb, w->w_up, 2, Ld, D, DensePolicy::kBN))
-      return MRLMOE_ERR_CUDA;
-    p.out = static_cast<__nv_bfloat16 *>(y);
-    p.ldo = D;
-    p.M = T; p.N = D; p.K = Ld;
-    p.m_tiles = (T + 127) / 128;
-    p.n_tiles = (D + DensePolicy::kBN - 1) / DensePolicy::kBN;
-    p.status = P.status;
-    MRL_TRY(launch_gemm<DensePolicy>(p, std::min(sms, p.m_tiles * p.n_tiles), st));
+    mrlmoe_status s = launch_dense_bf16(P.nbuf, w->w_up, static_cast<__nv_bfloat16 *>(y), nullptr, T, D, Ld,
+                                        P.status, sms, st);
+    if (s != MRLMOE_OK) return s;
   }
   if (!mark(8)) return MRLMOE_ERR_CUDA;
   return MRLMOE_OK;
@@ -729,16 +744,8 @@ mrlmoe_status mrlmoe_linear(const void *a, const void *w, void *out, int M, int 
   int sms = 0;
   mrlmoe_status s = bind_device(w, &sms);
   if (s != MRLMOE_OK) return s;
-  DensePolicy::Params p{};
-  if (!make_map(&p.ta, a, 2, K, M, 128) || !make_map(&p.tb, w, 2, K, N, DensePolicy::kBN)) return MRLMOE_ERR_CUDA;
-  p.out = static_cast<__nv_bfloat16 *>(out);
-  p.ldo = N;
-  p.M = M; p.N = N; p.K = K;
-  p.m_tiles = (M + 127) / 128;
-  p.n_tiles = (N + DensePolicy::kBN - 1) / DensePolicy::kBN;
-  p.status = nullptr;
-  MRL_TRY(launch_gemm<DensePolicy>(p, std::min(sms, p.m_tiles * p.n_tiles), static_cast<cudaStream_t>(stream)));
-  return MRLMOE_OK;
+  return launch_dense_bf16(a, w, static_cast<__nv_bfloat16 *>(out), nullptr, M, N, K, nullptr, sms,
+                           static_cast<cudaStream_t>(stream));
 }
 
 mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *bias, const float *expert_scale,

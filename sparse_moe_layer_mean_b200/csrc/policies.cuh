@@ -1,6 +1,6 @@
 // policies.cuh — the layer's GEMMs expressed as policies of gemm_kernel.
 //
-//  DensePolicy  : out[M,N] = bf16(a[M,K] w[N,K]^T)           (down-/up-projection)
+//  DensePolicyN : out[M,N] = bf16(a[M,K] w[N,K]^T)           (down-/up-projection)
 //  RouterPolicy : per token tile, R sigmoid routers x all experts, fused with
 //                 the aggregation over routers (mean / sum / max), + bias,
 //                 running top-k, renormalisation, alpha
@@ -18,10 +18,14 @@ constexpr int kTopKMax = 16;
 __device__ __forceinline__ int round16(int n) { return (n + 15) & ~15; }
 
 // ---------------------------------------------------------------- dense
-struct DensePolicy {
-  static constexpr int kStages = 4;
+// BN output columns per unit: 256 normally; 64 when the token count is small
+// (decode) and 256-wide tiles would leave most SMs idle, with a deeper ring of
+// the smaller stages.
+template <int BN>
+struct DensePolicyN {
+  static constexpr int kStages = BN >= 256 ? 4 : 8;
   static constexpr int kGroup = 2;
-  static constexpr int kBN = 256;
+  static constexpr int kBN = BN;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
   static constexpr int kEpiSmem = 0;
@@ -29,7 +33,7 @@ struct DensePolicy {
   static constexpr int kUmmaKBytes = 32;
   struct Params {
     CUtensorMap ta;  // a [M, K], box 64 x 128
-    CUtensorMap tb;  // w [N, K], box 64 x 256
+    CUtensorMap tb;  // w [N, K], box 64 x BN
     __nv_bfloat16 *out;
     __nv_bfloat16 *out_lo;  // optional: bf16(acc - float(out)), the residual of the rounding
     long ldo;
@@ -106,6 +110,8 @@ struct DensePolicy {
     }
   }
 };
+using DensePolicy = DensePolicyN<256>;
+using DenseNarrowPolicy = DensePolicyN<64>;
 
 // ---------------------------------------------------------------- router
 // B tile = R boxes of `ec` router rows (experts [sub*ec, sub*ec+ec) of router r),
