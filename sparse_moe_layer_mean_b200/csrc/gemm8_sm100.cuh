@@ -46,10 +46,13 @@ constexpr int kF8PromoWarp0 = 4;
 constexpr int kF8PromoThreads = 256;
 constexpr int kF8OpBytes = kF8Tile * 128;  // one operand tile per K block
 
-// One scale table: tok[kF8MaxKB][kF8Tile], w[2][kF8MaxKB], then the unit's
-// descriptor (so the promotion warps need not search the group table).
-constexpr int kF8TabFloats = kF8MaxKB * kF8Tile + 2 * kF8MaxKB + 8;
+// One scale table: tok[kF8MaxKB][kF8Tile], w[2][kF8MaxKB], the unit's
+// descriptor (so the promotion warps need not search the group table), and
+// 256 words a policy may fill for its epilogue (the expert-down GEMM: each
+// token's slot index and routing weight).
 constexpr int kF8TabUnit = kF8MaxKB * kF8Tile + 2 * kF8MaxKB;
+constexpr int kF8TabExtra = kF8TabUnit + 8;
+constexpr int kF8TabFloats = kF8TabExtra + 2 * kF8Tile;
 
 template <class P>
 struct Gemm8Smem {
@@ -173,7 +176,7 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
       if (ul >= 2 && !__all_sync(0xffffffffu, mbar_wait(sempty0 + 8 * b, ((ul >> 1) - 1) & 1, abort_flag, status)))
         goto done;
       float *tok = tabs + b * kF8TabFloats;
-      P::stage_scales(p, U, tok, tok + kF8MaxKB * kF8Tile, lane);
+      P::stage_scales(p, U, tok, tok + kF8MaxKB * kF8Tile, tok + kF8TabExtra, lane);
       if (lane == 0) {
         int *d = reinterpret_cast<int *>(tok + kF8TabUnit);
         d[0] = U.g; d[1] = U.m; d[2] = U.n0; d[3] = U.nv; d[4] = U.row0;
@@ -221,10 +224,10 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
         const int *d = reinterpret_cast<const int *>(tabs + b * kF8TabFloats + kF8TabUnit);
         U.g = d[0]; U.m = d[1]; U.n0 = d[2]; U.nv = d[3]; U.row0 = d[4]; U.nsub = 1;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sempty0 + 8 * b);
       if (bar_red_or(1, kF8PromoThreads, bad || *abort_flag)) goto done;
-      P::epilogue_regs(p, U, acc, q, h, lane, epi_smem);
+      P::epilogue_regs(p, U, acc, q, h, lane, epi_smem, tabs + b * kF8TabFloats + kF8TabExtra);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sempty0 + 8 * b);  // table b (read by the epilogue too) is free
     }
   }
 done:
@@ -315,13 +318,14 @@ struct Dense8Policy {
     tma_load_2d(sb, &p.tb, bar, kb * 128, U.n0);
   }
   static __device__ __forceinline__ int scale_class(int) { return 0; }
-  static __device__ __forceinline__ void stage_scales(const Params &p, const Unit &U, float *tok, float *w, int lane) {
+  static __device__ __forceinline__ void stage_scales(const Params &p, const Unit &U, float *tok, float *w, float *,
+                                                      int lane) {
     const int kbs = p.K / 128;
     stage_token_scales(p.as_t, p.M, U.row0, U.nv, kbs, tok, lane);
     stage_weight_scales(p.ws + static_cast<size_t>(U.n0 / 128) * kbs, nullptr, kbs, w, lane);
   }
   static __device__ __forceinline__ void epilogue_regs(const Params &p, const Unit &U, float (&acc)[kF8Half], int q,
-                                                       int h, int lane, uint8_t *) {
+                                                       int h, int lane, uint8_t *, const float *) {
     const int t = q * 32 + lane;
     if (t >= U.nv) return;
     const long row = U.row0 + t;
@@ -390,7 +394,8 @@ struct Glu8Policy {
     tma_load_2d(sb + 64 * 128, sh ? &p.su : &p.wu, bar, kb * 128, row);
   }
   static __device__ __forceinline__ int scale_class(int h) { return h; }
-  static __device__ __forceinline__ void stage_scales(const Params &p, const Unit &U, float *tok, float *w, int lane) {
+  static __device__ __forceinline__ void stage_scales(const Params &p, const Unit &U, float *tok, float *w, float *,
+                                                      int lane) {
     const bool sh = U.g == p.gt.E;
     const int kbs = p.L / 128;
     const size_t blk = (static_cast<size_t>(sh ? 0 : U.g) * (p.F / 128) + (U.m * 64) / 128) * kbs;
@@ -400,9 +405,11 @@ struct Glu8Policy {
   // Warp (q, 0) holds one token's gate values for f = 64m .. 64m+63, warp
   // (q, 1) the up values; each hands the other half of its row across
   // shared memory (named barrier 3 + q, 64 threads), then warp (q, hh)
-  // writes h for f = 64m + 32hh .. +31: 64 contiguous bytes per token.
+  // computes h for f = 64m + 32hh .. +31 of its 32 tokens and writes them
+  // through its own shared rows so that each store instruction covers 8
+  // tokens' 64 contiguous bytes.
   static __device__ __forceinline__ void epilogue_regs(const Params &p, const Unit &U, float (&acc)[kF8Half], int q,
-                                                       int hh, int lane, uint8_t *epi) {
+                                                       int hh, int lane, uint8_t *epi, const float *) {
     float *xb = reinterpret_cast<float *>(epi);  // [8 warps][32][33]
     const int pw = hh * 4 + q;
     float *mine = xb + (pw * 32 + lane) * 33;
@@ -410,34 +417,49 @@ struct Glu8Policy {
 #pragma unroll
     for (int i = 0; i < 32; ++i) mine[i] = hh == 0 ? acc[32 + i] : acc[i];
     named_bar_sync(3 + q, 64);
-    float out[32];
+    uint32_t packed[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float gv = hh == 0 ? acc[i] : other[i];
-      const float uv = hh == 0 ? other[i] : acc[32 + i];
-      out[i] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+    for (int i = 0; i < 16; ++i) {
+      float hv[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = 2 * i + e;
+        const float gv = hh == 0 ? acc[c] : other[c];
+        const float uv = hh == 0 ? other[c] : acc[32 + c];
+        hv[e] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+      }
+      packed[i] = pack_bf16x2(hv[0], hv[1]);
     }
-    const int t = q * 32 + lane;
-    if (t < U.nv) {
-      uint4 *dst = reinterpret_cast<uint4 *>(p.h + static_cast<size_t>(U.row0 + t) * p.F + U.m * 64 + hh * 32);
+    named_bar_sync(3 + q, 64);  // both warps of the pair are done reading the exchange rows
+    uint32_t *wrow = reinterpret_cast<uint32_t *>(xb + pw * 32 * 33);  // this warp's rows: [32 tokens][17 words]
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 16; ++i) wrow[lane * 17 + i] = packed[i];
+    __syncwarp();
+    const int chunk = lane & 3;  // 16-byte quarter of a token's 64 bytes
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int i = it * 8 + (lane >> 2);  // token within the warp
+      const int t = q * 32 + i;
+      if (t < U.nv) {
         uint4 w;
-        w.x = pack_bf16x2(out[8 * i + 0], out[8 * i + 1]);
-        w.y = pack_bf16x2(out[8 * i + 2], out[8 * i + 3]);
-        w.z = pack_bf16x2(out[8 * i + 4], out[8 * i + 5]);
-        w.w = pack_bf16x2(out[8 * i + 6], out[8 * i + 7]);
-        dst[i] = w;
+        w.x = wrow[i * 17 + chunk * 4 + 0];
+        w.y = wrow[i * 17 + chunk * 4 + 1];
+        w.z = wrow[i * 17 + chunk * 4 + 2];
+        w.w = wrow[i * 17 + chunk * 4 + 3];
+        *reinterpret_cast<uint4 *>(p.h + static_cast<size_t>(U.row0 + t) * p.F + U.m * 64 + hh * 32 + chunk * 8) = w;
       }
     }
-    named_bar_sync(3 + q, 64);  // the exchange rows are free for the next unit
+    __syncwarp();  // the rows are rewritten by the next unit's exchange
   }
 };
 
 // expert down: unit = (group, 128-wide d_lat slice m, <= 128 dispatched
-// tokens); each thread writes 64 contiguous fp32 of its token's slot row.
+// tokens).  The stager also looks up each token's slot index and routing
+// weight (dispatch permutation, scaled weights) into the table; the epilogue
+// scales its 64 columns and writes them through its own shared rows so that
+// each store instruction covers four tokens' 128 contiguous bytes.
 struct Down8Policy {
-  static constexpr int kEpiSmem = 0;
+  static constexpr int kEpiSmem = 8 * 32 * 33 * 4;
   static constexpr int kAuxSmem = kGroupAuxSmem;
   struct Params {
     CUtensorMap wd, sd;  // e4m3 [E*L, F] / [L, F], box 128 x 128
@@ -470,33 +492,65 @@ struct Down8Policy {
     tma_load_2d(sb, sh ? &p.sd : &p.wd, bar, kb * 128, (sh ? 0 : U.g * p.L) + U.m * 128);
   }
   static __device__ __forceinline__ int scale_class(int) { return 0; }
-  static __device__ __forceinline__ void stage_scales(const Params &p, const Unit &U, float *tok, float *w, int lane) {
+  static __device__ __forceinline__ void stage_scales(const Params &p, const Unit &U, float *tok, float *w,
+                                                      float *extra, int lane) {
     const bool sh = U.g == p.gt.E;
     const int kbs = p.F / 128;
     const size_t blk = (static_cast<size_t>(sh ? 0 : U.g) * (p.L / 128) + U.m) * kbs;
     stage_token_scales(p.hs_t, p.rows, U.row0, U.nv, kbs, tok, lane);
     stage_weight_scales((sh ? p.sd_s : p.wd_s) + blk, nullptr, kbs, w, lane);
+    // [128] slot row, then [128] weight; the loads go out in two batches
+    // (all permutation entries, then all weights) rather than as four
+    // dependent pairs
+    int *slot = reinterpret_cast<int *>(extra);
+    constexpr int C = kF8Tile / 32;
+    int flat[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      const int n = c * 32 + lane;
+      flat[c] = (!sh && n < U.nv) ? __ldg(p.perm + U.row0 + n) : 0;
+    }
+    float wv[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) wv[c] = (!sh && c * 32 + lane < U.nv) ? __ldg(p.wscaled + flat[c]) : 1.0f;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      const int n = c * 32 + lane;
+      if (n < U.nv) {
+        if (sh) {
+          slot[n] = (U.row0 + n - p.Tk) * (p.k + 1) + p.k;
+        } else {
+          const int tk = flat[c] / p.k;
+          slot[n] = tk * (p.k + 1) + (flat[c] - tk * p.k);
+        }
+        extra[kF8Tile + n] = wv[c];
+      }
+    }
   }
   static __device__ __forceinline__ void epilogue_regs(const Params &p, const Unit &U, float (&acc)[kF8Half], int q,
-                                                       int h, int lane, uint8_t *) {
-    const int t = q * 32 + lane;
-    if (t >= U.nv) return;
-    const int row = U.row0 + t;
-    int slot;
-    float wt;
-    if (U.g == p.gt.E) {
-      slot = (row - p.Tk) * (p.k + 1) + p.k;
-      wt = 1.0f;
-    } else {
-      const int flat = __ldg(p.perm + row);
-      const int tk = flat / p.k;
-      slot = tk * (p.k + 1) + (flat - tk * p.k);
-      wt = __ldg(p.wscaled + flat);
-    }
-    float4 *dst = reinterpret_cast<float4 *>(p.slots + static_cast<size_t>(slot) * p.L + U.m * 128 + h * kF8Half);
+                                                       int h, int lane, uint8_t *epi, const float *extra) {
+    const int *slot = reinterpret_cast<const int *>(extra);
+    const float *wt = extra + kF8Tile;
+    float *wrow = reinterpret_cast<float *>(epi) + (h * 4 + q) * 32 * 33;  // this warp's rows: [32 tokens][33]
+    const float my_wt = q * 32 + lane < U.nv ? wt[q * 32 + lane] : 0.f;
+    const int part = lane & 7;  // 16-byte eighth of a token's 128 bytes
 #pragma unroll
-    for (int i = 0; i < kF8Half / 4; ++i)
-      dst[i] = make_float4(acc[4 * i] * wt, acc[4 * i + 1] * wt, acc[4 * i + 2] * wt, acc[4 * i + 3] * wt);
+    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) wrow[lane * 33 + i] = acc[half * 32 + i] * my_wt;
+      __syncwarp();
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int i = it * 4 + (lane >> 3);  // token within the warp
+        const int t = q * 32 + i;
+        if (t < U.nv) {
+          const float *src = wrow + i * 33 + part * 4;
+          *reinterpret_cast<float4 *>(p.slots + static_cast<size_t>(slot[t]) * p.L + U.m * 128 + h * kF8Half +
+                                      half * 32 + part * 4) = make_float4(src[0], src[1], src[2], src[3]);
+        }
+      }
+      __syncwarp();
+    }
   }
 };
 
