@@ -29,6 +29,8 @@
  *    anything is enqueued.  Faults found on the device (a bounded wait that
  *    gave up, a failed check) are written to a status word inside the
  *    workspace; read it with mrlmoe_get_device_status.  No kernel traps.
+ *    Once a kernel of a call has failed, the call's later kernels do nothing,
+ *    so no kernel reads a record that a failed kernel left unwritten.
  *  - The library allocates no device memory: all scratch lives in the
  *    caller's workspace of mrlmoe_workspace_size() bytes (256-byte aligned).
  *  - The library keeps no state between calls; two calls that share a
@@ -92,7 +94,20 @@ typedef struct {
   float rms_eps;    /* RMSNorm epsilon (1e-6)                                    */
   mrlmoe_dtype dtype;
   mrlmoe_aggregation aggregation;  /* router score aggregation (0 = mean)      */
+  uint32_t hold;    /* 0 in normal use.  Test hook for the bounded waits: an OR
+                       of mrlmoe_hold bits; the GEMM kernels of those families
+                       issue no tile loads in this call, so their waits run out
+                       (after about 2 s) and the call ends with
+                       MRLMOE_ERR_TIMEOUT in the status word.  Other bits:
+                       MRLMOE_ERR_INVALID_ARG.                                 */
 } mrlmoe_config;
+
+/* GEMM families for mrlmoe_config.hold.                                       */
+typedef enum {
+  MRLMOE_HOLD_GEMM = 1,         /* one-CTA bf16 GEMMs: projections, routers, expert down */
+  MRLMOE_HOLD_GEMM_PAIR = 2,    /* CTA-pair bf16 grouped GEMMs: gate/up (and wide down)  */
+  MRLMOE_HOLD_GEMM_FP8 = 4      /* the FP8 variant's GEMMs                               */
+} mrlmoe_hold;
 
 /* Weights: device pointers, caller-owned.  Element type is bf16 in BF16 mode;
  * in FP8 mode every matrix except w_router is e4m3 and carries a scale array
@@ -222,6 +237,40 @@ mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, flo
 /* Synchronises `stream`, then returns the device status word of `workspace`
  * written by the last call that used it (MRLMOE_OK if none failed).          */
 mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream);
+
+/* Invariants of a routing record that mrlmoe_check_routing verifies; each
+ * failed one sets its bit (mrlmoe_get_device_detail).                         */
+typedef enum {
+  MRLMOE_CHECK_INDEX = 1,       /* an expert index outside [0, E)                   */
+  MRLMOE_CHECK_DUPLICATE = 2,   /* a token selects one expert twice                 */
+  MRLMOE_CHECK_OFFSETS = 4,     /* a negative count, or offsets not the exclusive
+                                   scan of counts ending at T*k                     */
+  MRLMOE_CHECK_PERM = 8,        /* perm, inv_perm not inverse bijections of [0,T*k) */
+  MRLMOE_CHECK_GROUP = 16,      /* a dispatch row outside its expert's row range    */
+  MRLMOE_CHECK_ORDER = 32,      /* an expert's rows not in ascending t*k+j order    */
+  MRLMOE_CHECK_WEIGHT = 64      /* a routing weight that is not finite              */
+} mrlmoe_check_bits;
+
+/* Device check of the routing record of cfg->T tokens: the invariants above,
+ * every index range-checked before use, so a corrupt record is reported and
+ * never dereferenced out of bounds.  r's non-NULL fields name the record (as
+ * filled by mrlmoe_route / mrlmoe_forward); NULL fields are read from the
+ * workspace copy that those calls keep.  If any of topk_idx, counts, offsets,
+ * perm, inv_perm is NULL, ws_bytes must be at least mrlmoe_workspace_size(cfg),
+ * else 256 (the status header).  The weights are checked from r->topk_w, or
+ * from the workspace copy when the workspace is full-sized, else skipped.  clear != 0
+ * zeroes the workspace's status header first; clear == 0 keeps the status of
+ * the call it follows on `stream`.  A failure sets MRLMOE_ERR_CHECK (if the
+ * status was clear) and the failed invariants' bits; read them with
+ * mrlmoe_get_device_detail.  Enqueues one kernel.                            */
+mrlmoe_status mrlmoe_check_routing(const mrlmoe_config *cfg, const mrlmoe_routing *r,
+                                   void *workspace, size_t ws_bytes, int clear,
+                                   void *stream);
+
+/* As mrlmoe_get_device_status; also stores the OR of the mrlmoe_check_bits
+ * that failed since the header was last cleared in *check_bits (non-NULL).   */
+mrlmoe_status mrlmoe_get_device_detail(const void *workspace, uint32_t *check_bits,
+                                       void *stream);
 
 /* Static, human-readable name of a status code.                              */
 const char *mrlmoe_status_string(mrlmoe_status s);

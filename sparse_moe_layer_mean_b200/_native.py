@@ -9,7 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from ctypes import POINTER, c_float, c_int, c_size_t, c_void_p
+from ctypes import POINTER, c_float, c_int, c_size_t, c_uint32, c_void_p
 from typing import Dict, Optional
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -24,7 +24,8 @@ STATUS = {0: "MRLMOE_OK", 1: "MRLMOE_ERR_INVALID_ARG", 2: "MRLMOE_ERR_UNSUPPORTE
 
 EXPORTED = ("mrlmoe_workspace_size", "mrlmoe_route", "mrlmoe_forward", "mrlmoe_forward_timed",
             "mrlmoe_bias_update", "mrlmoe_linear", "mrlmoe_get_device_status",
-            "mrlmoe_status_string", "mrlmoe_route_scores_static", "mrlmoe_quantize_e4m3")
+            "mrlmoe_status_string", "mrlmoe_route_scores_static", "mrlmoe_quantize_e4m3",
+            "mrlmoe_check_routing", "mrlmoe_get_device_detail")
 STATIC_SCRATCH_BYTES = 2 * 1024 * 1024
 NUM_STAGE_EVENTS = 9
 STAGES = ("down_proj", "router_topk", "dispatch", "gather", "gate_up_glu", "expert_down",
@@ -40,7 +41,14 @@ class MrlmoeError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("T", c_int), ("d_model", c_int), ("d_lat", c_int), ("n_experts", c_int),
                 ("top_k", c_int), ("d_ff", c_int), ("n_routers", c_int), ("rms_eps", c_float),
-                ("dtype", c_int), ("aggregation", c_int)]
+                ("dtype", c_int), ("aggregation", c_int), ("hold", c_uint32)]
+
+
+# mrlmoe_hold: GEMM families whose tile loads a call may hold (test hook)
+HOLD = {"gemm": 1, "gemm_pair": 2, "gemm_fp8": 4}
+
+# mrlmoe_check_bits: invariants of a routing record
+CHECK_BITS = {"index": 1, "duplicate": 2, "offsets": 4, "perm": 8, "group": 16, "order": 32, "weight": 64}
 
 
 WEIGHT_FIELDS = ("w_down", "w_router", "w_gate", "w_up_e", "w_down_e", "w_sh_gate", "w_sh_up",
@@ -93,6 +101,11 @@ def lib() -> ctypes.CDLL:
         L.mrlmoe_quantize_e4m3.restype = c_int
         L.mrlmoe_get_device_status.argtypes = [c_void_p, c_void_p]
         L.mrlmoe_get_device_status.restype = c_int
+        L.mrlmoe_get_device_detail.argtypes = [c_void_p, POINTER(c_uint32), c_void_p]
+        L.mrlmoe_get_device_detail.restype = c_int
+        L.mrlmoe_check_routing.argtypes = [POINTER(Config), POINTER(Routing), c_void_p, c_size_t, c_int,
+                                           c_void_p]
+        L.mrlmoe_check_routing.restype = c_int
         L.mrlmoe_status_string.argtypes = [c_int]
         L.mrlmoe_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -120,14 +133,15 @@ def _stream_ptr(stream) -> Optional[int]:
 AGGREGATIONS = {"mean": 0, "sum": 1, "max": 2}   # mrlmoe_aggregation
 
 
-def make_config(shape, T: Optional[int] = None, fp8: Optional[bool] = None) -> Config:
+def make_config(shape, T: Optional[int] = None, fp8: Optional[bool] = None, hold: int = 0) -> Config:
     """Config from a workloads.LayerShape-like object (duck-typed; a missing
-    `aggregation` attribute means the mean)."""
+    `aggregation` attribute means the mean).  ``hold``: mrlmoe_config.hold
+    (0 in normal use; an OR of HOLD values makes those GEMMs' waits run out)."""
     f8 = shape.fp8 if fp8 is None else fp8
     return Config(shape.T if T is None else T, shape.d_model, shape.d_lat, shape.n_experts,
                   shape.top_k, shape.d_ff, shape.n_routers, float(shape.rms_eps),
                   MRLMOE_FP8_E4M3_BLOCK128 if f8 else MRLMOE_BF16,
-                  AGGREGATIONS[getattr(shape, "aggregation", "mean")])
+                  AGGREGATIONS[getattr(shape, "aggregation", "mean")], int(hold))
 
 
 def make_weights(w: Dict[str, object]) -> Weights:
@@ -207,3 +221,19 @@ def mrlmoe_quantize_e4m3(x, rows: int, K: int, q, scale, stream=None) -> None:
 
 def mrlmoe_get_device_status(workspace, stream=None) -> int:
     return int(lib().mrlmoe_get_device_status(_ptr(workspace), _stream_ptr(stream)))
+
+
+def mrlmoe_get_device_detail(workspace, stream=None):
+    """(status, check_bits): the status word and the failed routing invariants."""
+    bits = c_uint32(0)
+    st = int(lib().mrlmoe_get_device_detail(_ptr(workspace), ctypes.byref(bits), _stream_ptr(stream)))
+    return st, int(bits.value)
+
+
+def mrlmoe_check_routing(cfg: Config, routing: Optional[Routing], workspace, ws_bytes: int, clear: bool,
+                         stream=None) -> None:
+    """Enqueue the device check of a routing record (read the verdict with
+    mrlmoe_get_device_detail)."""
+    rp = ctypes.byref(routing) if routing is not None else None
+    _check(lib().mrlmoe_check_routing(ctypes.byref(cfg), rp, _ptr(workspace), int(ws_bytes), int(bool(clear)),
+                                      _stream_ptr(stream)), "mrlmoe_check_routing")

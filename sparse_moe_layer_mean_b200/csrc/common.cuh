@@ -14,6 +14,27 @@ namespace mrl {
 // Status codes written to the device status word (mirror mrlmoe_status).
 enum : uint32_t { DEV_OK = 0, DEV_TIMEOUT = 5, DEV_CHECK = 6 };
 
+// Call header: the first words of the scratch every call uses.  [0] status
+// code, [1] this call's lost-arrival test mask (mrlmoe_config.hold: the GEMM
+// families below whose tile loads are not issued), [2] the routing checker's
+// failed-invariant bits.  The host zeroes it at the start of each call.
+enum : uint32_t { HOLD_GEMM = 1, HOLD_GEMM_PAIR = 2, HOLD_GEMM_FP8 = 4 };
+
+// Both first header words in one load (status may be null: no header).
+__device__ __forceinline__ uint2 call_header(const uint32_t *status) {
+  uint2 r = make_uint2(0u, 0u);
+  if (status) asm volatile("ld.volatile.global.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(status));
+  return r;
+}
+
+// True once an earlier kernel of the call has recorded a failure.  Kernels
+// that read what earlier kernels wrote return on entry then, so a record a
+// failed kernel left unwritten is never used as an index.  Within one launch
+// of such a kernel nothing writes the word, so every thread reads the same.
+__device__ __forceinline__ bool call_failed(const uint32_t *status) {
+  return status && *reinterpret_cast<const volatile uint32_t *>(status) != DEV_OK;
+}
+
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
@@ -123,6 +144,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
+}
+
+// 32-bit load from a shared::cluster address (this or another CTA of the cluster).
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
 }
 
 // Arrive on an mbarrier in another CTA of the cluster (shared::cluster address).

@@ -45,6 +45,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+  volatile int *entry = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 8);  // [0] skip, [1] hold
   uint8_t *epi_smem = smem + L::kEpiOff;
   uint8_t *aux = smem + L::kAuxOff;
 
@@ -63,6 +64,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint32_t *status = p.status;
 
   if (threadIdx.x == 0) {
+    // only the even CTA reads the call header; both CTAs act on its reading
+    const uint2 hdr = leader ? call_header(status) : make_uint2(0u, 0u);
     for (int s = 0; s < S; ++s) mbar_init(full0 + 8 * s, 2);
     for (int g = 0; g < S / G; ++g) mbar_init(empty0 + 8 * g, 1);
     for (int a = 0; a < 2; ++a) {
@@ -70,6 +73,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(acce0 + 8 * a, 8);
     }
     *abort_flag = 0;
+    entry[0] = hdr.x != DEV_OK;
+    entry[1] = (hdr.y & HOLD_GEMM_PAIR) != 0;
     fence_mbar_init();
   }
   P::stage_aux(p, aux);
@@ -84,9 +89,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int nunits = P::num_units(p, aux);
   const int kblocks = P::k_blocks(p);
+  // the even CTA's entry words, read after the cluster barrier that published them
+  const uint32_t entry_l = mapa_shared(smem_u32(const_cast<int *>(entry)), 0);
+  if (ld_shared_cluster_u32(entry_l)) goto done;  // an earlier kernel of the call failed
 
   if (warp == 0 || warp == 6) {
-    if (lane == 0) {
+    // loads held (test mask): nothing is issued in either CTA, so the bounded waits run out
+    if (lane == 0 && !ld_shared_cluster_u32(entry_l + 4)) {
       const bool isA = warp == 0;
       P::prefetch(p);
       int s = 0;

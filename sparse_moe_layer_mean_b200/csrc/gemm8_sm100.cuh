@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+  volatile int *hold_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 8);
   float *tabs = reinterpret_cast<float *>(smem + L::kTabOff);
   uint8_t *epi_smem = smem + L::kEpiOff;
   uint8_t *aux = smem + L::kAuxOff;
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
   uint32_t *status = p.status;
 
   if (threadIdx.x == 0) {
+    const uint2 hdr = call_header(status);  // loaded first: the barrier set-up hides its latency
     for (int j = 0; j < kF8Ring; ++j) {
       mbar_init(full0 + 8 * j, 2);
       mbar_init(done0 + 8 * j, 1);
@@ -108,7 +110,8 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
       mbar_init(sfull0 + 8 * b, 32);
       mbar_init(sempty0 + 8 * b, 8);
     }
-    *abort_flag = 0;
+    *abort_flag = hdr.x != DEV_OK;  // an earlier kernel of the call failed: do nothing
+    *hold_flag = (hdr.y & HOLD_GEMM_FP8) != 0;
     fence_mbar_init();
   }
   P::stage_aux(p, aux);
@@ -124,9 +127,12 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
   const int kblocks = P::k_blocks(p);
   int issued = -1;  // MMA issuer: last committed K block
   const uint32_t idesc = idesc_e4m3(kF8Tile, kF8Tile);
+  if (*abort_flag) goto done;
 
   if (warp == 0 || warp == 2) {
-    if (lane == 0) {
+    // with the call's loads held (test mask) nothing is issued, so the
+    // consumers' bounded waits run out and record DEV_TIMEOUT
+    if (lane == 0 && !*hold_flag) {
       const bool isA = warp == 0;
       P::prefetch(p);
       uint32_t g = 0;

@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+  volatile int *hold_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 8);
   uint8_t *epi_smem = smem + L::kEpiOff;
   uint8_t *aux = smem + L::kAuxOff;  // per-launch tables staged once per CTA
 
@@ -93,13 +94,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   uint32_t *status = p.status;
 
   if (threadIdx.x == 0) {
+    const uint2 hdr = call_header(status);  // loaded first: the barrier set-up hides its latency
     for (int s = 0; s < S; ++s) mbar_init(full0 + 8 * s, 2);
     for (int g = 0; g < S / G; ++g) mbar_init(empty0 + 8 * g, 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf0 + 8 * a, 1);
       mbar_init(acce0 + 8 * a, 4);
     }
-    *abort_flag = 0;
+    *abort_flag = hdr.x != DEV_OK;  // an earlier kernel of the call failed: do nothing
+    *hold_flag = (hdr.y & HOLD_GEMM) != 0;
     fence_mbar_init();
   }
   P::stage_aux(p, aux);
@@ -113,9 +116,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   const uint32_t tmem_base = *tmem_slot;
   const int nunits = P::num_units(p, aux);
   const int kblocks = P::k_blocks(p);
+  if (*abort_flag) goto done;
 
   if (warp == 0 || warp == 6) {
-    if (lane == 0) {
+    // with the call's loads held (test mask) nothing is issued, so the
+    // consumers' bounded waits run out and record DEV_TIMEOUT
+    if (lane == 0 && !*hold_flag) {
       // producers: warp 0 loads A, warp 6 loads B, into the same stages
       const bool isA = warp == 0;
       P::prefetch(p);

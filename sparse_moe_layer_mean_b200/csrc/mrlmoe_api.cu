@@ -12,6 +12,7 @@
 #include "gemm2_sm100.cuh"
 #include "gemm8_sm100.cuh"
 #include "routing.cuh"
+#include "check.cuh"
 
 using namespace mrl;
 
@@ -33,6 +34,8 @@ mrlmoe_status check_config(const mrlmoe_config *c) {
   if (!(c->rms_eps >= 0.f)) return MRLMOE_ERR_INVALID_ARG;
   if (c->dtype != MRLMOE_BF16 && c->dtype != MRLMOE_FP8_E4M3_BLOCK128) return MRLMOE_ERR_INVALID_ARG;
   if (c->aggregation != MRLMOE_AGG_MEAN && c->aggregation != MRLMOE_AGG_SUM && c->aggregation != MRLMOE_AGG_MAX)
+    return MRLMOE_ERR_INVALID_ARG;
+  if (c->hold & ~static_cast<uint32_t>(MRLMOE_HOLD_GEMM | MRLMOE_HOLD_GEMM_PAIR | MRLMOE_HOLD_GEMM_FP8))
     return MRLMOE_ERR_INVALID_ARG;
   // the FP8 GEMMs stage at most kF8MaxKB scales of 128-wide K blocks per unit
   if (c->dtype == MRLMOE_FP8_E4M3_BLOCK128 &&
@@ -234,6 +237,15 @@ int down_m_tiles(const mrlmoe_config &c) { return down_uses_pairs(c) ? c.d_lat /
     if ((expr) != cudaSuccess) return MRLMOE_ERR_CUDA; \
   } while (0)
 
+// Start of a call: zero the call header (status, hold mask, check bits) and
+// store the call's hold mask in the low byte of word 1.  Both are memsets, so
+// the call stays capturable in a CUDA graph.
+mrlmoe_status init_header(uint32_t *hdr, uint32_t hold, cudaStream_t st) {
+  MRL_TRY(cudaMemsetAsync(hdr, 0, 16, st));
+  if (hold) MRL_TRY(cudaMemsetAsync(reinterpret_cast<uint8_t *>(hdr) + 4, static_cast<int>(hold & 0xffu), 1, st));
+  return MRLMOE_OK;
+}
+
 struct Ptrs {
   uint32_t *status;
   int32_t *topk_idx, *counts_e, *offsets_e, *grp_off, *grp_cnt, *unit1, *unit2, *perm, *inv, *base;
@@ -303,15 +315,15 @@ mrlmoe_status launch_dispatch(const mrlmoe_config &c, const Ptrs &P, cudaStream_
   const int nch = (T + kChunk - 1) / kChunk;
   const int wpb = 8;
   expert_mask_kernel<<<(nch + wpb - 1) / wpb, 32 * wpb, wpb * E * sizeof(uint32_t), st>>>(P.topk_idx, T, E, k,
-                                                                                         P.mask, nch);
+                                                                                         P.mask, nch, P.status);
   MRL_TRY(cudaGetLastError());
-  expert_colscan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(P.mask, E, nch, P.base, P.counts_e);
+  expert_colscan_kernel<<<(E + 31) / 32, 1024, 0, st>>>(P.mask, E, nch, P.base, P.counts_e, P.status);
   MRL_TRY(cudaGetLastError());
   expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, gtl.bn, gtl.mt1, gtl.mt2, P.grp_off,
-                                            P.grp_cnt, P.unit1, P.unit2, P.out_counts, P.out_offsets);
+                                            P.grp_cnt, P.unit1, P.unit2, P.out_counts, P.out_offsets, P.status);
   MRL_TRY(cudaGetLastError());
   expert_scatter_kernel<<<(nch * 32 + 255) / 256, 256, 0, st>>>(P.topk_idx, P.mask, P.base, P.grp_off, T, E, k,
-                                                                 nch, P.perm, P.inv);
+                                                                 nch, P.perm, P.inv, P.status);
   MRL_TRY(cudaGetLastError());
   return MRLMOE_OK;
 }
@@ -342,9 +354,9 @@ mrlmoe_status check_weights_fp8(const mrlmoe_weights *w) {
 // Scales go to sc[rows][K/128], or transposed to sc[K/128][rows] (the layout
 // the FP8 GEMMs read) when `transposed`.
 cudaError_t launch_quant(const __nv_bfloat16 *in, long ld_in, int rows, int K, const int32_t *perm, int k, int Tk,
-                         uint8_t *q, float *sc, bool transposed, cudaStream_t st) {
+                         uint8_t *q, float *sc, bool transposed, const uint32_t *status, cudaStream_t st) {
   quant_rows_kernel<<<(rows + kQuantWarps - 1) / kQuantWarps, kQuantWarps * 32, 0, st>>>(
-      in, ld_in, rows, K, perm, k, Tk, q, sc, transposed ? static_cast<long>(rows) : 0L);
+      in, ld_in, rows, K, perm, k, Tk, q, sc, transposed ? static_cast<long>(rows) : 0L, status);
   return cudaGetLastError();
 }
 
@@ -417,7 +429,8 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
   const int T = c.T, D = c.d_model, Ld = c.d_lat, E = c.n_experts, R = c.n_routers, k = c.top_k;
   __nv_bfloat16 *z = P.zbuf + static_cast<size_t>(T) * k * Ld;  // z rows live after the T*k dispatched rows
   if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) {
-    MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(x), D, T, D, nullptr, 1, 0, P.xq, P.xs, true, st));
+    MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(x), D, T, D, nullptr, 1, 0, P.xq, P.xs, true, P.status,
+                         st));
     mrlmoe_status s = launch_dense8(P.xq, P.xs, w->w_down, w->s_down, T, Ld, D, z, P.zlo, P, sms, st);
     if (s != MRLMOE_OK) return s;
   } else {
@@ -448,7 +461,8 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
     MRL_TRY(launch_gemm<RouterPolicy>(p, std::min(sms, p.m_tiles * p.parts), st));
     if (p.parts > 1) {
       topk_merge_kernel<kTopKMax><<<(T + 127) / 128, 128, 0, st>>>(P.cand_v, P.cand_s, P.cand_i, T, p.parts, k,
-                                                                  w->expert_scale, P.topk_idx, P.topk_w, P.wscaled);
+                                                                  w->expert_scale, P.topk_idx, P.topk_w, P.wscaled,
+                                                                  P.status);
       MRL_TRY(cudaGetLastError());
     }
   }
@@ -477,7 +491,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   const Ptrs P = carve(*cfg, workspace, route_out);
   const int T = cfg->T, D = cfg->d_model, Ld = cfg->d_lat, F = cfg->d_ff, E = cfg->n_experts, k = cfg->top_k;
   const int Tk = T * k;
-  MRL_TRY(cudaMemsetAsync(P.status, 0, 4, st));
+  if ((s = init_header(P.status, cfg->hold, st)) != MRLMOE_OK) return s;
   auto mark = [&](int i) -> bool {
     return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
   };
@@ -498,7 +512,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
     const int row_u4 = Ld * 2 / 16;
     gather_rows_kernel<<<(Tk * 32 + 255) / 256, 256, 0, st>>>(
         P.perm, Tk, k, reinterpret_cast<const uint4 *>(P.zbuf + static_cast<size_t>(Tk) * Ld),
-        reinterpret_cast<uint4 *>(P.zbuf), row_u4);
+        reinterpret_cast<uint4 *>(P.zbuf), row_u4, P.status);
     MRL_TRY(cudaGetLastError());
   }
   if (!mark(4)) return MRLMOE_ERR_CUDA;
@@ -538,7 +552,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   if (!mark(6)) return MRLMOE_ERR_CUDA;
   combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k,
                                                         cfg->rms_eps,
-                                                        reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf);
+                                                        reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf, P.status);
   MRL_TRY(cudaGetLastError());
   if (!mark(7)) return MRLMOE_ERR_CUDA;
   {
@@ -558,7 +572,8 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
   };
   // quantised dispatched latent rows (rows < T*k) and the shared expert's rows (all T tokens)
-  MRL_TRY(launch_quant(P.zbuf + static_cast<size_t>(Tk) * Ld, Ld, Tk + T, Ld, P.perm, k, Tk, P.zq, P.zs, true, st));
+  MRL_TRY(launch_quant(P.zbuf + static_cast<size_t>(Tk) * Ld, Ld, Tk + T, Ld, P.perm, k, Tk, P.zq, P.zs, true,
+                       P.status, st));
   if (!mark(4)) return MRLMOE_ERR_CUDA;
   const GroupTiling gtl = group_tiling(c);
   {
@@ -577,7 +592,7 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     p.status = P.status;
     MRL_TRY(launch_gemm8<Glu8Policy>(p, sms, st));
   }
-  MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, nullptr, 1, 0, P.hq, P.hs, true, st));
+  MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, nullptr, 1, 0, P.hq, P.hs, true, P.status, st));
   if (!mark(5)) return MRLMOE_ERR_CUDA;
   {
     Down8Policy::Params p{};
@@ -598,9 +613,9 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
   }
   if (!mark(6)) return MRLMOE_ERR_CUDA;
   combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k, c.rms_eps,
-                                                        reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf);
+                                                        reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf, P.status);
   MRL_TRY(cudaGetLastError());
-  MRL_TRY(launch_quant(P.nbuf, Ld, T, Ld, nullptr, 1, 0, P.nq, P.ns, true, st));
+  MRL_TRY(launch_quant(P.nbuf, Ld, T, Ld, nullptr, 1, 0, P.nq, P.ns, true, P.status, st));
   if (!mark(7)) return MRLMOE_ERR_CUDA;
   return launch_dense8(P.nq, P.ns, w->w_up, w->s_up, T, D, Ld, static_cast<__nv_bfloat16 *>(y_out), nullptr, P, sms,
                        st);
@@ -697,12 +712,12 @@ mrlmoe_status mrlmoe_route(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ptrs P = carve(*cfg, workspace, out);
-  MRL_TRY(cudaMemsetAsync(P.status, 0, 4, st));
+  if ((s = init_header(P.status, cfg->hold, st)) != MRLMOE_OK) return s;
   if (scores_in) {
     const int warps_per_block = 8;
     topk_from_scores_kernel<kTopKMax><<<(cfg->T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0,
                                         st>>>(out->scores, bias, w->expert_scale, cfg->T, cfg->n_experts,
-                                              cfg->top_k, P.topk_idx, P.topk_w, P.wscaled);
+                                              cfg->top_k, P.topk_idx, P.topk_w, P.wscaled, P.status);
     MRL_TRY(cudaGetLastError());
   } else {
     if ((s = launch_project_and_route(*cfg, w, bias, x, P, sms, st)) != MRLMOE_OK) return s;
@@ -780,12 +795,13 @@ mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *
   P.base = reinterpret_cast<int32_t *>(b + SL.base);
   P.out_counts = out->counts;
   P.out_offsets = out->offsets;
-  // the array keeps the previous call's contents: the status word must start
-  // at zero; every other region is fully rewritten below before it is read
-  MRL_TRY(cudaMemsetAsync(P.status, 0, 4, st));
+  // the array keeps the previous call's contents: the header must start at
+  // zero; every other region is fully rewritten below before it is read
+  if ((s = init_header(P.status, 0, st)) != MRLMOE_OK) return s;
   const int warps_per_block = 8;
   topk_from_scores_kernel<kTopKMax><<<(cfg->T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, st>>>(
-      out->scores, bias, expert_scale, cfg->T, cfg->n_experts, cfg->top_k, P.topk_idx, P.topk_w, P.wscaled);
+      out->scores, bias, expert_scale, cfg->T, cfg->n_experts, cfg->top_k, P.topk_idx, P.topk_w, P.wscaled,
+      P.status);
   MRL_TRY(cudaGetLastError());
   return launch_dispatch(*cfg, P, st);
 }
@@ -799,19 +815,58 @@ mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, flo
   mrlmoe_status s = bind_device(in, &sms);
   if (s != MRLMOE_OK) return s;
   MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(in), K, rows, K, nullptr, 1, 0, static_cast<uint8_t *>(q),
-                       scale, false, static_cast<cudaStream_t>(stream)));
+                       scale, false, nullptr, static_cast<cudaStream_t>(stream)));
   return MRLMOE_OK;
 }
 
 mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream) {
+  uint32_t bits = 0;
+  return mrlmoe_get_device_detail(workspace, &bits, stream);
+}
+
+mrlmoe_status mrlmoe_get_device_detail(const void *workspace, uint32_t *check_bits, void *stream) {
   if (!workspace) return MRLMOE_ERR_WORKSPACE;
-  uint32_t v = 0;
+  if (!check_bits) return MRLMOE_ERR_INVALID_ARG;
+  uint32_t h[3] = {0, 0, 0};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   MRL_TRY(cudaStreamSynchronize(st));
-  MRL_TRY(cudaMemcpy(&v, workspace, 4, cudaMemcpyDeviceToHost));
-  if (v == DEV_TIMEOUT) return MRLMOE_ERR_TIMEOUT;
-  if (v == DEV_CHECK) return MRLMOE_ERR_CHECK;
-  return v == 0 ? MRLMOE_OK : MRLMOE_ERR_CHECK;
+  MRL_TRY(cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost));
+  *check_bits = h[2];
+  if (h[0] == DEV_TIMEOUT) return MRLMOE_ERR_TIMEOUT;
+  if (h[0] == DEV_CHECK) return MRLMOE_ERR_CHECK;
+  return h[0] == 0 ? MRLMOE_OK : MRLMOE_ERR_CHECK;
+}
+
+mrlmoe_status mrlmoe_check_routing(const mrlmoe_config *cfg, const mrlmoe_routing *r, void *workspace,
+                                   size_t ws_bytes, int clear, void *stream) {
+  mrlmoe_status s = check_config(cfg);
+  if (s != MRLMOE_OK) return s;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
+  const bool whole = r && r->topk_idx && r->counts && r->offsets && r->perm && r->inv_perm;
+  const bool full = ws_bytes >= layout_of(*cfg).total;
+  if (ws_bytes < 256 || (!whole && !full)) return MRLMOE_ERR_WORKSPACE;
+  int sms = 0;
+  if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t *hdr = static_cast<uint32_t *>(workspace);
+  // r's arrays where given, else the workspace copies that route/forward keep
+  // (counts and offsets from the group table, whose entry E is T*k)
+  Ptrs P{};
+  if (full) P = carve(*cfg, workspace, r);
+  const int32_t *idx = (r && r->topk_idx) ? r->topk_idx : P.topk_idx;
+  const int32_t *perm = (r && r->perm) ? r->perm : P.perm;
+  const int32_t *inv = (r && r->inv_perm) ? r->inv_perm : P.inv;
+  const int32_t *counts = (r && r->counts) ? r->counts : P.grp_cnt;
+  const int32_t *offsets = (r && r->offsets) ? r->offsets : P.grp_off;
+  const float *w = (r && r->topk_w) ? r->topk_w : P.topk_w;  // NULL: weights unchecked
+  if (clear) MRL_TRY(cudaMemsetAsync(hdr, 0, 16, st));
+  const long long Tk = static_cast<long long>(cfg->T) * cfg->top_k;
+  const long long n = std::max<long long>(Tk, cfg->n_experts + 1);
+  const long long blocks = std::min<long long>((n + kCheckThreads - 1) / kCheckThreads, 8ll * sms);
+  check_routing_kernel<<<static_cast<int>(blocks), kCheckThreads, 0, st>>>(idx, w, counts, offsets, perm, inv,
+                                                                          cfg->T, cfg->n_experts, cfg->top_k, hdr);
+  MRL_TRY(cudaGetLastError());
+  return MRLMOE_OK;
 }
 
 }  // extern "C"

@@ -19,7 +19,8 @@ template <int KMAX>
 __global__ void topk_from_scores_kernel(const float *__restrict__ s, const float *__restrict__ bias,
                                         const float *__restrict__ alpha, int T, int E, int k,
                                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
-                                        float *__restrict__ wscaled) {
+                                        float *__restrict__ wscaled, const uint32_t *status) {
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
@@ -59,7 +60,9 @@ template <int KMAX>
 __global__ void topk_merge_kernel(const float *__restrict__ cand_v, const float *__restrict__ cand_s,
                                   const int32_t *__restrict__ cand_i, int T, int parts, int k,
                                   const float *__restrict__ alpha, int32_t *__restrict__ topk_idx,
-                                  float *__restrict__ topk_w, float *__restrict__ wscaled) {
+                                  float *__restrict__ topk_w, float *__restrict__ wscaled,
+                                  const uint32_t *status) {
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
   TopK<KMAX> tk;
@@ -75,8 +78,9 @@ __global__ void topk_merge_kernel(const float *__restrict__ cand_v, const float 
 // has bit i set iff token 32c+i selected e.  One warp per chunk; the warp's
 // table lives in shared memory (E <= 1024 words).
 __global__ void expert_mask_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int k,
-                                   uint32_t *__restrict__ mask, int nchunks) {
+                                   uint32_t *__restrict__ mask, int nchunks, const uint32_t *status) {
   extern __shared__ uint32_t tab_all[];
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int wib = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int c = blockIdx.x * (blockDim.x >> 5) + wib;
@@ -96,8 +100,10 @@ __global__ void expert_mask_kernel(const int32_t *__restrict__ topk_idx, int T, 
 // counts[e] = total.  Block (32 x 32): lane = expert of a 32-expert group,
 // warp = a contiguous run of chunks.
 __global__ void expert_colscan_kernel(const uint32_t *__restrict__ mask, int E, int nchunks,
-                                      int32_t *__restrict__ base, int32_t *__restrict__ counts) {
+                                      int32_t *__restrict__ base, int32_t *__restrict__ counts,
+                                      const uint32_t *status) {
   __shared__ int tot[32][33];
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int lane = threadIdx.x & 31;
   const int w = threadIdx.x >> 5;
   const int e = blockIdx.x * 32 + lane;
@@ -155,8 +161,9 @@ __global__ void expert_offsets_kernel(const int32_t *__restrict__ counts_in, int
                                       int mt1, int mt2, int32_t *__restrict__ grp_off,
                                       int32_t *__restrict__ grp_cnt, int32_t *__restrict__ unit1,
                                       int32_t *__restrict__ unit2, int32_t *__restrict__ out_counts,
-                                      int32_t *__restrict__ out_offsets) {
+                                      int32_t *__restrict__ out_offsets, const uint32_t *status) {
   __shared__ int wt[32];
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
   __shared__ int tot[3];
   const int e = threadIdx.x;
   const int cnt = e < E ? counts_in[e] : 0;
@@ -192,7 +199,8 @@ __global__ void expert_offsets_kernel(const int32_t *__restrict__ counts_in, int
 __global__ void expert_scatter_kernel(const int32_t *__restrict__ topk_idx, const uint32_t *__restrict__ mask,
                                       const int32_t *__restrict__ base, const int32_t *__restrict__ offsets,
                                       int T, int E, int k, int nchunks, int32_t *__restrict__ perm,
-                                      int32_t *__restrict__ inv_perm) {
+                                      int32_t *__restrict__ inv_perm, const uint32_t *status) {
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (c >= nchunks) return;
@@ -211,7 +219,9 @@ __global__ void expert_scatter_kernel(const int32_t *__restrict__ topk_idx, cons
 
 // Row gather: zd[row] = zs[perm[row] / k] for row < T*k (one warp per row).
 __global__ void gather_rows_kernel(const int32_t *__restrict__ perm, int rows, int k,
-                                   const uint4 *__restrict__ zs, uint4 *__restrict__ zd, int row_u4) {
+                                   const uint4 *__restrict__ zs, uint4 *__restrict__ zd, int row_u4,
+                                   const uint32_t *status) {
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
@@ -243,7 +253,8 @@ constexpr int kQuantBatch = 4;   // warp iterations whose loads are in flight to
 // while the block keeps few registers (and many warps per SM).
 __global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_kernel(
     const __nv_bfloat16 *__restrict__ in, long ld_in, int rows, int K, const int32_t *__restrict__ perm, int k,
-    int Tk, uint8_t *__restrict__ q, float *__restrict__ s, long s_ld) {
+    int Tk, uint8_t *__restrict__ q, float *__restrict__ s, long s_ld, const uint32_t *status) {
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int kbs = K >> 7;
   const int r = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
   if (r >= rows) return;  // whole warps leave together
@@ -305,8 +316,9 @@ constexpr int kCombineMaxV4 = 8;  // d_lat <= 8192
 
 __global__ void __launch_bounds__(kCombineThreads) combine_rmsnorm_kernel(
     const float4 *__restrict__ slots, int L, int k, float eps, const float4 *__restrict__ gain,
-    __nv_bfloat16 *__restrict__ n) {
+    __nv_bfloat16 *__restrict__ n, const uint32_t *status) {
   __shared__ float red[kCombineThreads / 32];
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int t = blockIdx.x;
   const int L4 = L >> 2;
   const float4 *base = slots + static_cast<size_t>(t) * (k + 1) * L4;

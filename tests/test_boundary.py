@@ -50,8 +50,10 @@ def test_workspace_size_valid_and_invalid():
     for bad in (dict(T=0), dict(d_model=200), dict(d_lat=0), dict(d_ff=100), dict(n_experts=8),
                 dict(n_experts=24 + 1), dict(top_k=0), dict(top_k=17), dict(top_k=17, n_experts=16),
                 dict(n_routers=0), dict(n_routers=9), dict(rms_eps=-1.0), dict(dtype=7),
-                dict(aggregation=3), dict(aggregation=-1)):
+                dict(aggregation=3), dict(aggregation=-1), dict(hold=8), dict(hold=0x100)):
         assert M.mrlmoe_workspace_size(_cfg(**bad)) == 0, bad
+    for hold in (1, 2, 4, 7):                                    # the GEMM families of mrlmoe_hold
+        assert M.mrlmoe_workspace_size(_cfg(hold=hold)) > 0
     for agg in (0, 1, 2):                                       # mean, sum, max
         assert M.mrlmoe_workspace_size(_cfg(aggregation=agg)) > 0
     # the FP8 variant stages at most 32 K-block scales per GEMM unit: K <= 4096
@@ -133,6 +135,26 @@ def test_quantize_rejects_bad_arguments():
     assert L.mrlmoe_quantize_e4m3(4096 + 2, 4, 128, 4096, 4096, None) == 1
     assert L.mrlmoe_quantize_e4m3(4096 + 8, 4, 128, 4096, 4096, None) == 1   # in: 16-byte aligned
     assert L.mrlmoe_quantize_e4m3(4096, 4, 128, 4096 + 4, 4096, None) == 1   # q: 8-byte aligned
+
+
+def test_check_routing_and_detail_reject_bad_arguments():
+    L = N.lib()
+    cfg = _cfg()
+    need = M.mrlmoe_workspace_size(cfg)
+    whole = N.Routing(*([4096] * 6 + [None]))
+    part = N.Routing(*([4096] * 3 + [None] * 4))
+    chk = lambda c, r, ws, n: L.mrlmoe_check_routing(ctypes.byref(c) if c is not None else None,
+                                                     ctypes.byref(r) if r is not None else None, ws, n, 1, None)
+    assert chk(None, whole, 4096, 256) == 1
+    assert chk(_cfg(hold=16), whole, 4096, 256) == 1
+    assert chk(cfg, whole, None, 256) == 3          # no workspace
+    assert chk(cfg, whole, 4096 + 16, 256) == 3     # misaligned
+    assert chk(cfg, whole, 4096, 255) == 3          # smaller than the status header
+    assert chk(cfg, part, 4096, 256) == 3           # a field read from the workspace: full size needed
+    assert chk(cfg, None, 4096, need - 1) == 3
+    det = ctypes.c_uint32(0)
+    assert L.mrlmoe_get_device_detail(None, ctypes.byref(det), None) == 3
+    assert L.mrlmoe_get_device_detail(4096, None, None) == 1
 
 
 def test_python_binding_raises_on_error():
