@@ -160,10 +160,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             tc_fence_after();
             const uint32_t a_s = ring + s * L::kStageBytes;
             const uint32_t b_s = a_s + P::kABytes;
+            // kASub A tiles of the stage (each kASubBytes) share its B tile and the accumulator
 #pragma unroll
-            for (int kk = 0; kk < kBK * 2 / P::kUmmaKBytes; ++kk)
-              P::mma(tacc, sdesc_sw128(a_s + kk * P::kUmmaKBytes), sdesc_sw128(b_s + kk * P::kUmmaKBytes),
-                     idesc, (kb | kk) != 0);
+            for (int as = 0; as < P::kASub; ++as)
+#pragma unroll
+              for (int kk = 0; kk < kBK * 2 / P::kUmmaKBytes; ++kk)
+                P::mma(tacc, sdesc_sw128(a_s + as * P::kASubBytes + kk * P::kUmmaKBytes),
+                       sdesc_sw128(b_s + kk * P::kUmmaKBytes), idesc, (kb | kk | as) != 0);
             if (s % G == G - 1) umma_commit(empty0 + 8 * (s / G));
             if (++s == S) { s = 0; ph ^= 1; }
           }

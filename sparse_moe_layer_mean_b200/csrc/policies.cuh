@@ -31,6 +31,7 @@ struct DensePolicyN {
   static constexpr int kEpiSmem = 0;
   static constexpr int kAuxSmem = 0;
   static constexpr int kUmmaKBytes = 32;
+  static constexpr int kASub = 1, kASubBytes = 0;
   struct Params {
     CUtensorMap ta;  // a [M, K], box 64 x 128
     CUtensorMap tb;  // w [N, K], box 64 x BN
@@ -120,9 +121,14 @@ using DenseNarrowPolicy = DensePolicyN<64>;
 // given as bf16 hi + bf16 lo parts and the K loop runs over both (2 * d_lat),
 // reusing each router tile for the hi and the lo half.
 struct RouterPolicy {
-  static constexpr int kStages = 4;
-  static constexpr int kGroup = 2;
-  static constexpr int kABytes = 128 * 128;
+  // A stage holds both halves of the fp32 latent's 64-wide K block (z hi and
+  // z lo, 128 tokens each) and the router weights once: both MMAs of the
+  // block read the same B tile into one accumulator, so the weights cross
+  // from L2 once per K block instead of once per half.
+  static constexpr int kStages = 3;
+  static constexpr int kGroup = 1;
+  static constexpr int kASub = 2, kASubBytes = 128 * 128;
+  static constexpr int kABytes = kASub * kASubBytes;
   static constexpr int kBBytesMax = 256 * 128;
   static constexpr int kEpiSmem = 0;
   static constexpr int kAuxSmem = 0;
@@ -152,7 +158,7 @@ struct RouterPolicy {
   }
   static __device__ __forceinline__ void stage_aux(const Params &, uint8_t *) {}
   static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *) { return p.m_tiles * p.parts; }
-  static __device__ __forceinline__ int k_blocks(const Params &p) { return 2 * (p.L / kBK); }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.L / kBK; }
   static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *) {
     Unit U;
     U.m = u / p.parts;
@@ -168,14 +174,12 @@ struct RouterPolicy {
   }
   static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int, int kb, uint32_t sa,
                                                 uint32_t bar) {
-    const int nk = p.L / kBK;
-    const bool lo = kb >= nk;
-    tma_load_2d(sa, lo ? &p.ta_lo : &p.ta, bar, (lo ? kb - nk : kb) * kBK, U.m * 128);
+    tma_load_2d(sa, &p.ta, bar, kb * kBK, U.m * 128);
+    tma_load_2d(sa + kASubBytes, &p.ta_lo, bar, kb * kBK, U.m * 128);
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int sub, int kb, uint32_t sb,
                                                 uint32_t bar) {
-    const int nk = p.L / kBK;
-    const int x = (kb >= nk ? kb - nk : kb) * kBK;
+    const int x = kb * kBK;
     const int chunk = U.g * U.nsub + sub;
     for (int r = 0; r < p.R; ++r) tma_load_2d(sb + r * p.ec * 128, &p.tb, bar, x, r * p.E + chunk * p.ec);
   }
@@ -370,6 +374,7 @@ struct DownPolicy {
   static constexpr int kEpiSmem = kBN * 8;
   static constexpr int kAuxSmem = kGroupAuxSmem;
   static constexpr int kUmmaKBytes = 32;
+  static constexpr int kASub = 1, kASubBytes = 0;
   struct Params {
     CUtensorMap wd;  // routed down [E*L, F], box 64 x 128
     CUtensorMap sd;  // shared down [L, F], box 64 x 128
