@@ -46,6 +46,37 @@ constexpr int kF8PromoWarp0 = 4;
 constexpr int kF8PromoThreads = 256;
 constexpr int kF8OpBytes = kF8Tile * 128;  // one operand tile per K block
 
+// An e4m3 token tensor [rows, K] with four box heights (16 / 32 / 64 / 128
+// rows x 128 B): a unit loads only its dispatched rows, rounded up to 16, so
+// a group of a few tokens (decode) moves 2 KB per K block instead of 16 KB.
+// The tile's remaining smem rows keep older bytes; an accumulator row depends
+// on its own A row only, and rows >= the unit's count are never stored.
+struct TokenMaps8 {
+  CUtensorMap m16, m32, m64, m128;
+};
+
+__device__ __forceinline__ int token_rows16(int nv) { return (nv + 15) & ~15; }
+
+__device__ __forceinline__ void load_token_rows8(const TokenMaps8 &t, int kb, int y0, int n, uint32_t sa,
+                                                 uint32_t bar) {
+  const int x = kb * 128;
+  if (n == kF8Tile) {
+    tma_load_2d(sa, &t.m128, bar, x, y0);
+    return;
+  }
+  int r = 0;
+  if (r + 64 <= n) { tma_load_2d(sa + r * 128, &t.m64, bar, x, y0 + r); r += 64; }
+  if (r + 32 <= n) { tma_load_2d(sa + r * 128, &t.m32, bar, x, y0 + r); r += 32; }
+  if (r + 16 <= n) tma_load_2d(sa + r * 128, &t.m16, bar, x, y0 + r);
+}
+
+__device__ __forceinline__ void prefetch_token_maps8(const TokenMaps8 &t) {
+  prefetch_tmap(&t.m16);
+  prefetch_tmap(&t.m32);
+  prefetch_tmap(&t.m64);
+  prefetch_tmap(&t.m128);
+}
+
 // One scale table: tok[kF8MaxKB][kF8Tile], w[2][kF8MaxKB], the unit's
 // descriptor (so the promotion warps need not search the group table), and
 // 256 words a policy may fill for its epilogue (the expert-down GEMM: each
@@ -143,7 +174,7 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
         for (int kb = 0; kb < kblocks; ++kb, ++g) {
           const uint32_t j = g & (kF8Ring - 1);
           if (g >= kF8Ring && !mbar_wait(done0 + 8 * j, ((g / kF8Ring) - 1) & 1, abort_flag, status)) goto done;
-          mbar_arrive_expect_tx(full0 + 8 * j, kF8OpBytes);
+          mbar_arrive_expect_tx(full0 + 8 * j, isA ? P::a_bytes(U) : kF8OpBytes);
           const uint32_t st = ring + j * L::kStageBytes;
           if (isA)
             P::load_a(p, U, kb, st, full0 + 8 * j);
@@ -317,6 +348,7 @@ struct Dense8Policy {
     U.nsub = 1;
     return U;
   }
+  static __device__ __forceinline__ uint32_t a_bytes(const Unit &) { return kF8OpBytes; }
   static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int kb, uint32_t sa, uint32_t bar) {
     tma_load_2d(sa, &p.ta, bar, kb * 128, U.row0);
   }
@@ -371,7 +403,7 @@ struct Glu8Policy {
   static constexpr int kAuxSmem = kGroupAuxSmem;
   struct Params {
     CUtensorMap wg, wu, sg, su;  // e4m3 [E*F, L] / [F, L], box 64 x 128
-    CUtensorMap tz;              // quantised dispatched z [(T*k+T), L], box 128 x 128
+    TokenMaps8 tz;               // quantised dispatched z [(T*k+T), L], boxes 16..128 x 128
     const float *wg_s, *wu_s, *sg_s, *su_s;  // [E, F/128, L/128] / [F/128, L/128]
     const float *zs_t;                        // [L/128, T*k+T] (transposed)
     GroupTable gt;
@@ -380,7 +412,8 @@ struct Glu8Policy {
     uint32_t *status;
   };
   static __device__ __forceinline__ void prefetch(const Params &p) {
-    prefetch_tmap(&p.wg); prefetch_tmap(&p.wu); prefetch_tmap(&p.sg); prefetch_tmap(&p.su); prefetch_tmap(&p.tz);
+    prefetch_tmap(&p.wg); prefetch_tmap(&p.wu); prefetch_tmap(&p.sg); prefetch_tmap(&p.su);
+    prefetch_token_maps8(p.tz);
   }
   static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
   static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
@@ -390,8 +423,9 @@ struct Glu8Policy {
   static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
     return grouped_unit(p.gt, aux, u, kF8Tile);
   }
+  static __device__ __forceinline__ uint32_t a_bytes(const Unit &U) { return token_rows16(U.nv) * 128; }
   static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int kb, uint32_t sa, uint32_t bar) {
-    tma_load_2d(sa, &p.tz, bar, kb * 128, U.row0);
+    load_token_rows8(p.tz, kb, U.row0, token_rows16(U.nv), sa, bar);
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb, uint32_t bar) {
     const bool sh = U.g == p.gt.E;
@@ -469,7 +503,7 @@ struct Down8Policy {
   static constexpr int kAuxSmem = kGroupAuxSmem;
   struct Params {
     CUtensorMap wd, sd;  // e4m3 [E*L, F] / [L, F], box 128 x 128
-    CUtensorMap th;      // quantised h [(T*k+T), F], box 128 x 128
+    TokenMaps8 th;       // quantised h [(T*k+T), F], boxes 16..128 x 128
     const float *wd_s, *sd_s;  // [E, L/128, F/128] / [L/128, F/128]
     const float *hs_t;         // [F/128, T*k+T] (transposed)
     GroupTable gt;
@@ -480,7 +514,8 @@ struct Down8Policy {
     uint32_t *status;
   };
   static __device__ __forceinline__ void prefetch(const Params &p) {
-    prefetch_tmap(&p.wd); prefetch_tmap(&p.sd); prefetch_tmap(&p.th);
+    prefetch_tmap(&p.wd); prefetch_tmap(&p.sd);
+    prefetch_token_maps8(p.th);
   }
   static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
   static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
@@ -490,8 +525,9 @@ struct Down8Policy {
   static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
     return grouped_unit(p.gt, aux, u, kF8Tile);
   }
+  static __device__ __forceinline__ uint32_t a_bytes(const Unit &U) { return token_rows16(U.nv) * 128; }
   static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int kb, uint32_t sa, uint32_t bar) {
-    tma_load_2d(sa, &p.th, bar, kb * 128, U.row0);
+    load_token_rows8(p.th, kb, U.row0, token_rows16(U.nv), sa, bar);
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb, uint32_t bar) {
     const bool sh = U.g == p.gt.E;

@@ -172,6 +172,12 @@ bool make_token_maps_blocked(TokenMaps *t, const void *base, uint64_t K, uint64_
   return true;
 }
 
+// The four box heights of an e4m3 token tensor [rows, inner] (load_token_rows8).
+bool make_token_maps8(TokenMaps8 *t, const void *base, uint64_t inner, uint64_t rows) {
+  return make_map(&t->m16, base, 1, inner, rows, 16) && make_map(&t->m32, base, 1, inner, rows, 32) &&
+         make_map(&t->m64, base, 1, inner, rows, 64) && make_map(&t->m128, base, 1, inner, rows, kF8Tile);
+}
+
 // Make the device that owns `p` current; reject host/unknown pointers.
 mrlmoe_status bind_device(const void *p, int *sm_count) {
   cudaPointerAttributes a;
@@ -581,7 +587,7 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     if (!make_map(&p.wg, w->w_gate, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
         !make_map(&p.wu, w->w_up_e, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
         !make_map(&p.sg, w->w_sh_gate, 1, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 1, Ld, F, 64) ||
-        !make_map(&p.tz, P.zq, 1, Ld, static_cast<uint64_t>(Tk) + T, kF8Tile))
+        !make_token_maps8(&p.tz, P.zq, Ld, static_cast<uint64_t>(Tk) + T))
       return MRLMOE_ERR_CUDA;
     p.wg_s = w->s_gate; p.wu_s = w->s_up_e; p.sg_s = w->s_sh_gate; p.su_s = w->s_sh_up;
     p.zs_t = P.zs;
@@ -598,7 +604,7 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     Down8Policy::Params p{};
     if (!make_map(&p.wd, w->w_down_e, 1, F, static_cast<uint64_t>(E) * Ld, 128) ||
         !make_map(&p.sd, w->w_sh_down, 1, F, Ld, 128) ||
-        !make_map(&p.th, P.hq, 1, F, static_cast<uint64_t>(Tk) + T, kF8Tile))
+        !make_token_maps8(&p.th, P.hq, F, static_cast<uint64_t>(Tk) + T))
       return MRLMOE_ERR_CUDA;
     p.wd_s = w->s_down_e; p.sd_s = w->s_sh_down;
     p.hs_t = P.hs;
