@@ -69,10 +69,26 @@ int router_parts(const mrlmoe_config &c, int sms) {
   return parts;
 }
 
+// Router K split for small T: when token tiles x expert chunks would fill at
+// most half of a 148-SM GPU, the K range is split (a power of two dividing
+// the K blocks) so that about 148 units run at once.  The target is a fixed
+// number, not the device's SM count, so the workspace layout depends on the
+// config alone.
+constexpr int kRouterSplitUnits = 148;
+int router_ksplit(const mrlmoe_config &c) {
+  const int chunks = c.n_experts / router_ec(c.n_experts, c.n_routers, c.T);
+  const int base = ((c.T + 127) / 128) * chunks;
+  if (2 * base > kRouterSplitUnits) return 1;
+  const int kb = c.d_lat / kBK;
+  int ks = 1;
+  while (kb % (2 * ks) == 0 && base * 2 * ks <= kRouterSplitUnits) ks *= 2;
+  return ks;
+}
+
 // ------------------------------------------------------------ workspace
 struct Layout {
   size_t status, topk_idx, topk_w, wscaled, counts, offsets, grp_off, grp_cnt, unit1, unit2, perm, inv, mask,
-      base, cand_v, cand_s, cand_i, zbuf, zlo, hbuf, slots, nbuf, xq, xs, zq, zs, hq, hs, nq, ns, total;
+      base, cand_v, cand_s, cand_i, rpart, zbuf, zlo, hbuf, slots, nbuf, xq, xs, zq, zs, hq, hs, nq, ns, total;
 };
 
 Layout layout_of(const mrlmoe_config &c) {
@@ -103,6 +119,8 @@ Layout layout_of(const mrlmoe_config &c) {
   L.cand_v = take(T * parts * k * 4);
   L.cand_s = take(T * parts * k * 4);
   L.cand_i = take(T * parts * k * 4);
+  const size_t ks = router_ksplit(c);
+  L.rpart = take(ks > 1 ? (ks * T * c.n_routers * E + T * E) * 4 : 0);  // partial logits, then s
   L.zbuf = take((Tk + T) * Ld * 2);
   L.zlo = take(T * Ld * 2);
   L.hbuf = take((Tk + T) * F * 2);
@@ -255,7 +273,7 @@ mrlmoe_status init_header(uint32_t *hdr, uint32_t hold, cudaStream_t st) {
 struct Ptrs {
   uint32_t *status;
   int32_t *topk_idx, *counts_e, *offsets_e, *grp_off, *grp_cnt, *unit1, *unit2, *perm, *inv, *base;
-  float *topk_w, *wscaled, *scores, *slots, *cand_v, *cand_s;
+  float *topk_w, *wscaled, *scores, *slots, *cand_v, *cand_s, *rpart;
   int32_t *cand_i;
   uint32_t *mask;
   __nv_bfloat16 *zbuf, *zlo, *hbuf, *nbuf;
@@ -285,6 +303,7 @@ Ptrs carve(const mrlmoe_config &c, void *ws, const mrlmoe_routing *r) {
   P.cand_v = reinterpret_cast<float *>(b + L.cand_v);
   P.cand_s = reinterpret_cast<float *>(b + L.cand_s);
   P.cand_i = reinterpret_cast<int32_t *>(b + L.cand_i);
+  P.rpart = reinterpret_cast<float *>(b + L.rpart);
   P.zbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.zbuf);
   P.zlo = reinterpret_cast<__nv_bfloat16 *>(b + L.zlo);
   P.hbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.hbuf);
@@ -462,8 +481,26 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
     p.T = T; p.L = Ld; p.E = E; p.R = R; p.ec = ec; p.k = k;
     p.agg = static_cast<int>(c.aggregation);
     p.m_tiles = (T + 127) / 128;
-    p.parts = router_parts(c, sms);
     p.status = P.status;
+    const int ks = router_ksplit(c);
+    if (ks > 1) {
+      // few token tiles: split K over the CTAs, then finish per token
+      p.part = P.rpart;
+      p.ksplit = ks;
+      p.parts = 1;
+      MRL_TRY(launch_gemm<RouterSplitPolicy>(p, std::min(sms, p.m_tiles * (E / ec) * ks), st));
+      float *s = P.scores ? P.scores : P.rpart + static_cast<size_t>(ks) * T * R * E;
+      const long long n = static_cast<long long>(T) * E;
+      router_split_scores_kernel<<<static_cast<int>((n + 255) / 256), 256, 0, st>>>(P.rpart, ks, T, E, R, p.agg, s,
+                                                                                    P.status);
+      MRL_TRY(cudaGetLastError());
+      const int wpb = 8;
+      topk_from_scores_kernel<kTopKMax><<<(T + wpb - 1) / wpb, 32 * wpb, 0, st>>>(
+          s, bias, w->expert_scale, T, E, k, P.topk_idx, P.topk_w, P.wscaled, P.status);
+      MRL_TRY(cudaGetLastError());
+      return MRLMOE_OK;
+    }
+    p.parts = router_parts(c, sms);
     MRL_TRY(launch_gemm<RouterPolicy>(p, std::min(sms, p.m_tiles * p.parts), st));
     if (p.parts > 1) {
       topk_merge_kernel<kTopKMax><<<(T + 127) / 128, 128, 0, st>>>(P.cand_v, P.cand_s, P.cand_i, T, p.parts, k,

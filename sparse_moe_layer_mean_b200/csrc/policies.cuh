@@ -146,6 +146,9 @@ struct RouterPolicy {
     int32_t *cand_i;
     int T, L, E, R, ec, k, m_tiles, parts;
     int agg;  // mrlmoe_aggregation: 0 mean, 1 sum, 2 max of the R sigmoid scores
+    // K split (RouterSplitPolicy): part[ks][t][r*E + e], fp32 logits of K range ks
+    float *part;
+    int ksplit;
     uint32_t *status;
   };
   struct EpiState {
@@ -240,6 +243,59 @@ struct RouterPolicy {
             p.cand_i[o + j] = st.tk.i[j];
           }
         }
+      }
+    }
+  }
+};
+
+// Router with its K range split over CTAs, for token counts whose token tiles
+// times expert chunks would occupy few SMs (decode): unit = (token tile m,
+// expert chunk c, K range ks); the epilogue stores the tile's fp32 partial
+// logits, router_split_scores_kernel sums the K ranges in order and applies
+// the sigmoid and the aggregation, and topk_from_scores_kernel selects.
+struct RouterSplitPolicy : RouterPolicy {
+  struct EpiState {};
+  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *) {
+    return p.m_tiles * (p.E / p.ec) * p.ksplit;
+  }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.L / kBK / p.ksplit; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *) {
+    Unit U;
+    const int chunks = p.E / p.ec;
+    U.n0 = u % p.ksplit;            // K range
+    U.g = (u / p.ksplit) % chunks;  // expert chunk
+    U.m = u / (p.ksplit * chunks);  // token tile
+    U.row0 = 0;
+    U.nv = p.R * p.ec;
+    U.nsub = 1;
+    return U;
+  }
+  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int, int kb, uint32_t sa,
+                                                uint32_t bar) {
+    const int x = (U.n0 * k_blocks(p) + kb) * kBK;
+    tma_load_2d(sa, &p.ta, bar, x, U.m * 128);
+    tma_load_2d(sa + kASubBytes, &p.ta_lo, bar, x, U.m * 128);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int, int kb, uint32_t sb,
+                                                uint32_t bar) {
+    const int x = (U.n0 * k_blocks(p) + kb) * kBK;
+    for (int r = 0; r < p.R; ++r) tma_load_2d(sb + r * p.ec * 128, &p.tb, bar, x, r * p.E + U.g * p.ec);
+  }
+  // Accumulator column r*ec + i is router r's logit of expert U.g*ec + i.
+  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
+                                                  int lane, int, EpiState &, uint8_t *) {
+    const int t = U.m * 128 + q * 32 + lane;
+    const bool valid = t < p.T;
+    float *row = p.part + (static_cast<size_t>(U.n0) * p.T + t) * (static_cast<size_t>(p.R) * p.E) + U.g * p.ec;
+    for (int c0 = 0; c0 < p.R * p.ec; c0 += 16) {
+      float v[16];
+      tmem_ld16(taddr + c0, v);
+      tmem_ld_wait();
+      if (valid) {
+        const int r = c0 / p.ec, i0 = c0 - r * p.ec;
+        float4 *dst = reinterpret_cast<float4 *>(row + static_cast<size_t>(r) * p.E + i0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
       }
     }
   }

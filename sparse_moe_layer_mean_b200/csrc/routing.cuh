@@ -11,26 +11,14 @@ namespace mrl {
 constexpr int kChunk = 32;  // tokens per histogram chunk (one warp, one bit per token)
 
 // ---------------------------------------------------------------------------
-// Top-k from caller-given fp32 scores s [T, E]: one warp per token.  Lane l
-// keeps the best of experts l, l+32, ... (ascending), then k rounds of a warp
-// arg-max (larger biased score, then lower index) emit the selection in rank
-// order.  sb = s + bias is one fp32 add, as in the CPU definition.
+// The selection of one token by one warp: lane l has offered experts
+// l, l+32, ... (ascending) to its running list; k rounds of a warp arg-max
+// (larger biased score, then lower index) emit the selection in rank order,
+// and lane 0 writes it with its weights.
 template <int KMAX>
-__global__ void topk_from_scores_kernel(const float *__restrict__ s, const float *__restrict__ bias,
-                                        const float *__restrict__ alpha, int T, int E, int k,
-                                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
-                                        float *__restrict__ wscaled, const uint32_t *status) {
-  if (call_failed(status)) return;  // an earlier kernel of the call failed
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
-  TopK<KMAX> tk;
-  tk.init();
-  const float *row = s + static_cast<size_t>(warp) * E;
-  for (int e = lane; e < E; e += 32) {
-    const float sv = __ldg(row + e);
-    tk.offer(sv + __ldg(bias + e), e, sv);
-  }
+__device__ __forceinline__ void warp_select_and_write(TopK<KMAX> &tk, int k, int lane, size_t t,
+                                                      const float *__restrict__ alpha, int32_t *__restrict__ topk_idx,
+                                                      float *__restrict__ topk_w, float *__restrict__ wscaled) {
   float sel_s[KMAX];
   int sel_i[KMAX];
 #pragma unroll
@@ -50,7 +38,54 @@ __global__ void topk_from_scores_kernel(const float *__restrict__ s, const float
       sel_i[j] = bi;
     }
   }
-  if (lane == 0) write_selection<KMAX>(sel_s, sel_i, k, static_cast<size_t>(warp), alpha, topk_idx, topk_w, wscaled);
+  if (lane == 0) write_selection<KMAX>(sel_s, sel_i, k, t, alpha, topk_idx, topk_w, wscaled);
+}
+
+// Top-k from caller-given fp32 scores s [T, E]: one warp per token (see
+// warp_select_and_write).  sb = s + bias is one fp32 add, as in the CPU
+// definition.
+template <int KMAX>
+__global__ void topk_from_scores_kernel(const float *__restrict__ s, const float *__restrict__ bias,
+                                        const float *__restrict__ alpha, int T, int E, int k,
+                                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                                        float *__restrict__ wscaled, const uint32_t *status) {
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  TopK<KMAX> tk;
+  tk.init();
+  const float *row = s + static_cast<size_t>(warp) * E;
+  for (int e = lane; e < E; e += 32) {
+    const float sv = __ldg(row + e);
+    tk.offer(sv + __ldg(bias + e), e, sv);
+  }
+  warp_select_and_write<KMAX>(tk, k, lane, static_cast<size_t>(warp), alpha, topk_idx, topk_w, wscaled);
+}
+
+// Scores of the K-split router: part[ks][t][r*E + e] holds router r's logit
+// of expert e for token t over the ks-th K range.  One thread per (t, e):
+// each logit is the sum of its K ranges in order, then s[t*E + e] = the
+// aggregation (over r in order) of the routers' sigmoids, as in the router
+// GEMM's epilogue.  topk_from_scores_kernel then selects from s + bias.
+__global__ void router_split_scores_kernel(const float *__restrict__ part, int ksplit, int T, int E, int R, int agg,
+                                           float *__restrict__ s, const uint32_t *status) {
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<long long>(T) * E) return;
+  const int t = static_cast<int>(i / E), e = static_cast<int>(i - static_cast<long long>(t) * E);
+  const size_t RE = static_cast<size_t>(R) * E;
+  const size_t plane = static_cast<size_t>(T) * RE;
+  const float *l0 = part + static_cast<size_t>(t) * RE + e;
+  float acc = 0.f;
+  for (int r = 0; r < R; ++r) {
+    const float *l = l0 + static_cast<size_t>(r) * E;
+    float logit = __ldg(l);
+    for (int ks = 1; ks < ksplit; ++ks) logit += __ldg(l + ks * plane);
+    const float sg = sigmoidf_(logit);
+    acc = agg == 2 ? fmaxf(acc, sg) : acc + sg;  // sigmoid >= 0
+  }
+  s[i] = agg != 0 ? acc : (R & (R - 1)) == 0 ? acc * (1.0f / static_cast<float>(R)) : acc / static_cast<float>(R);
 }
 
 // Merge of the router's partial selections: part p of token t left its best k
