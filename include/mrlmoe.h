@@ -79,7 +79,7 @@ typedef enum {
 /* Layer shape.  Limits checked on the host:
  *   T >= 1; d_model, d_lat, d_ff multiples of 128; 1 <= n_routers <= 8;
  *   16 <= n_experts <= 1024 with n_experts a multiple of 16;
- *   1 <= top_k <= min(n_experts, 16); rms_eps >= 0; aggregation one of
+ *   1 <= top_k <= min(n_experts, 32); rms_eps >= 0; aggregation one of
  *   mrlmoe_aggregation.  d_lat <= 8192, and in
  *   FP8 mode d_model, d_lat, d_ff <= 4096; beyond those the status is
  *   MRLMOE_ERR_UNSUPPORTED, otherwise MRLMOE_ERR_INVALID_ARG.                 */

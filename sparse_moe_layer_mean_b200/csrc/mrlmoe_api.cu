@@ -385,6 +385,19 @@ cudaError_t launch_quant(const __nv_bfloat16 *in, long ld_in, int rows, int K, c
   return cudaGetLastError();
 }
 
+// Top-k from fp32 scores with the running-list length that k needs.
+cudaError_t launch_topk_from_scores(const float *s, const float *bias, const float *alpha, int T, int E, int k,
+                                    int32_t *idx, float *w, float *wscaled, const uint32_t *status,
+                                    cudaStream_t st) {
+  const int wpb = 8;
+  const int grid = (T + wpb - 1) / wpb;
+  if (k <= kTopKNarrow)
+    topk_from_scores_kernel<kTopKNarrow><<<grid, 32 * wpb, 0, st>>>(s, bias, alpha, T, E, k, idx, w, wscaled, status);
+  else
+    topk_from_scores_kernel<kTopKMax><<<grid, 32 * wpb, 0, st>>>(s, bias, alpha, T, E, k, idx, w, wscaled, status);
+  return cudaGetLastError();
+}
+
 template <class P>
 cudaError_t launch_gemm8(const typename P::Params &p, int grid, cudaStream_t st) {
   static_assert(Gemm8Smem<P>::kTotal <= 232448, "GEMM shared memory above the 227 KB per-block limit");
@@ -464,7 +477,7 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
   }
   if (ev) MRL_TRY(cudaEventRecord(static_cast<cudaEvent_t>(ev[1]), st));
   {
-    RouterPolicy::Params p{};
+    RouterParams p{};
     const int ec = router_ec(E, R, T);
     if (!make_map(&p.ta, z, 2, Ld, T, 128) || !make_map(&p.ta_lo, P.zlo, 2, Ld, T, 128) ||
         !make_map(&p.tb, w->w_router, 2, Ld, static_cast<uint64_t>(R) * E, ec))
@@ -494,18 +507,23 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
       router_split_scores_kernel<<<static_cast<int>((n + 255) / 256), 256, 0, st>>>(P.rpart, ks, T, E, R, p.agg, s,
                                                                                     P.status);
       MRL_TRY(cudaGetLastError());
-      const int wpb = 8;
-      topk_from_scores_kernel<kTopKMax><<<(T + wpb - 1) / wpb, 32 * wpb, 0, st>>>(
-          s, bias, w->expert_scale, T, E, k, P.topk_idx, P.topk_w, P.wscaled, P.status);
-      MRL_TRY(cudaGetLastError());
+      MRL_TRY(launch_topk_from_scores(s, bias, w->expert_scale, T, E, k, P.topk_idx, P.topk_w, P.wscaled, P.status,
+                                      st));
       return MRLMOE_OK;
     }
     p.parts = router_parts(c, sms);
-    MRL_TRY(launch_gemm<RouterPolicy>(p, std::min(sms, p.m_tiles * p.parts), st));
+    const int grid = std::min(sms, p.m_tiles * p.parts);
+    if (k <= kTopKNarrow)
+      MRL_TRY(launch_gemm<RouterPolicy>(p, grid, st));
+    else
+      MRL_TRY(launch_gemm<RouterPolicyWide>(p, grid, st));
     if (p.parts > 1) {
-      topk_merge_kernel<kTopKMax><<<(T + 127) / 128, 128, 0, st>>>(P.cand_v, P.cand_s, P.cand_i, T, p.parts, k,
-                                                                  w->expert_scale, P.topk_idx, P.topk_w, P.wscaled,
-                                                                  P.status);
+      if (k <= kTopKNarrow)
+        topk_merge_kernel<kTopKNarrow><<<(T + 127) / 128, 128, 0, st>>>(
+            P.cand_v, P.cand_s, P.cand_i, T, p.parts, k, w->expert_scale, P.topk_idx, P.topk_w, P.wscaled, P.status);
+      else
+        topk_merge_kernel<kTopKMax><<<(T + 127) / 128, 128, 0, st>>>(
+            P.cand_v, P.cand_s, P.cand_i, T, p.parts, k, w->expert_scale, P.topk_idx, P.topk_w, P.wscaled, P.status);
       MRL_TRY(cudaGetLastError());
     }
   }
@@ -757,11 +775,8 @@ mrlmoe_status mrlmoe_route(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   const Ptrs P = carve(*cfg, workspace, out);
   if ((s = init_header(P.status, cfg->hold, st)) != MRLMOE_OK) return s;
   if (scores_in) {
-    const int warps_per_block = 8;
-    topk_from_scores_kernel<kTopKMax><<<(cfg->T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0,
-                                        st>>>(out->scores, bias, w->expert_scale, cfg->T, cfg->n_experts,
-                                              cfg->top_k, P.topk_idx, P.topk_w, P.wscaled, P.status);
-    MRL_TRY(cudaGetLastError());
+    MRL_TRY(launch_topk_from_scores(out->scores, bias, w->expert_scale, cfg->T, cfg->n_experts, cfg->top_k,
+                                    P.topk_idx, P.topk_w, P.wscaled, P.status, st));
   } else {
     if ((s = launch_project_and_route(*cfg, w, bias, x, P, sms, st)) != MRLMOE_OK) return s;
   }
@@ -841,11 +856,8 @@ mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *
   // the array keeps the previous call's contents: the header must start at
   // zero; every other region is fully rewritten below before it is read
   if ((s = init_header(P.status, 0, st)) != MRLMOE_OK) return s;
-  const int warps_per_block = 8;
-  topk_from_scores_kernel<kTopKMax><<<(cfg->T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, st>>>(
-      out->scores, bias, expert_scale, cfg->T, cfg->n_experts, cfg->top_k, P.topk_idx, P.topk_w, P.wscaled,
-      P.status);
-  MRL_TRY(cudaGetLastError());
+  MRL_TRY(launch_topk_from_scores(out->scores, bias, expert_scale, cfg->T, cfg->n_experts, cfg->top_k, P.topk_idx,
+                                  P.topk_w, P.wscaled, P.status, st));
   return launch_dispatch(*cfg, P, st);
 }
 

@@ -13,7 +13,10 @@
 
 namespace mrl {
 
-constexpr int kTopKMax = 16;
+// Running top-k lists: k <= 16 uses 16-entry lists (fewer registers in the
+// router epilogue and the top-k kernels), 16 < k <= 32 the 32-entry ones.
+constexpr int kTopKNarrow = 16;
+constexpr int kTopKMax = 32;  // the largest k the library accepts
 
 __device__ __forceinline__ int round16(int n) { return (n + 15) & ~15; }
 
@@ -117,10 +120,31 @@ using DenseNarrowPolicy = DensePolicyN<64>;
 // ---------------------------------------------------------------- router
 // B tile = R boxes of `ec` router rows (experts [sub*ec, sub*ec+ec) of router r),
 // so accumulator column r*ec + j holds router r's logit for expert sub*ec + j.
+// Router GEMM parameters (RouterPolicyK, RouterSplitPolicy).
+struct RouterParams {
+  CUtensorMap ta;     // z hi [T, L], box 64 x 128
+  CUtensorMap ta_lo;  // z lo [T, L], box 64 x 128
+  CUtensorMap tb;     // w_router [R*E, L], box 64 x ec
+  const float *bias, *alpha;
+  int32_t *topk_idx;
+  float *topk_w, *wscaled, *scores;
+  // parts > 1: the expert chunks are split over `parts` CTAs per token tile;
+  // each leaves its best k candidates here for topk_merge_kernel
+  float *cand_v, *cand_s;
+  int32_t *cand_i;
+  int T, L, E, R, ec, k, m_tiles, parts;
+  int agg;  // mrlmoe_aggregation: 0 mean, 1 sum, 2 max of the R sigmoid scores
+  // K split (RouterSplitPolicy): part[ks][t][r*E + e], fp32 logits of K range ks
+  float *part;
+  int ksplit;
+  uint32_t *status;
+};
+
 // The routers read the latent at the down-projection's fp32 precision: z is
-// given as bf16 hi + bf16 lo parts and the K loop runs over both (2 * d_lat),
-// reusing each router tile for the hi and the lo half.
-struct RouterPolicy {
+// given as bf16 hi + bf16 lo parts, and both halves meet the same router
+// weight tile in one accumulator.  KMAX: length of the running top-k list.
+template <int KMAX>
+struct RouterPolicyK {
   // A stage holds both halves of the fp32 latent's 64-wide K block (z hi and
   // z lo, 128 tokens each) and the router weights once: both MMAs of the
   // block read the same B tile into one accumulator, so the weights cross
@@ -133,26 +157,9 @@ struct RouterPolicy {
   static constexpr int kEpiSmem = 0;
   static constexpr int kAuxSmem = 0;
   static constexpr int kUmmaKBytes = 32;
-  struct Params {
-    CUtensorMap ta;     // z hi [T, L], box 64 x 128
-    CUtensorMap ta_lo;  // z lo [T, L], box 64 x 128
-    CUtensorMap tb;     // w_router [R*E, L], box 64 x ec
-    const float *bias, *alpha;
-    int32_t *topk_idx;
-    float *topk_w, *wscaled, *scores;
-    // parts > 1: the expert chunks are split over `parts` CTAs per token tile;
-    // each leaves its best k candidates here for topk_merge_kernel
-    float *cand_v, *cand_s;
-    int32_t *cand_i;
-    int T, L, E, R, ec, k, m_tiles, parts;
-    int agg;  // mrlmoe_aggregation: 0 mean, 1 sum, 2 max of the R sigmoid scores
-    // K split (RouterSplitPolicy): part[ks][t][r*E + e], fp32 logits of K range ks
-    float *part;
-    int ksplit;
-    uint32_t *status;
-  };
+  using Params = RouterParams;
   struct EpiState {
-    TopK<kTopKMax> tk;
+    TopK<KMAX> tk;
   };
   static __device__ __forceinline__ void prefetch(const Params &p) {
     prefetch_tmap(&p.ta);
@@ -231,12 +238,12 @@ struct RouterPolicy {
     }
     if (sub == U.nsub - 1 && valid) {
       if (p.parts == 1) {
-        write_selection<kTopKMax>(st.tk.s, st.tk.i, p.k, static_cast<size_t>(t), p.alpha, p.topk_idx, p.topk_w,
+        write_selection<KMAX>(st.tk.s, st.tk.i, p.k, static_cast<size_t>(t), p.alpha, p.topk_idx, p.topk_w,
                                   p.wscaled);
       } else {
         const size_t o = (static_cast<size_t>(t) * p.parts + U.g) * p.k;
 #pragma unroll
-        for (int j = 0; j < kTopKMax; ++j) {
+        for (int j = 0; j < KMAX; ++j) {
           if (j < p.k) {
             p.cand_v[o + j] = st.tk.v[j];
             p.cand_s[o + j] = st.tk.s[j];
@@ -247,6 +254,9 @@ struct RouterPolicy {
     }
   }
 };
+
+using RouterPolicy = RouterPolicyK<kTopKNarrow>;
+using RouterPolicyWide = RouterPolicyK<kTopKMax>;
 
 // Router with its K range split over CTAs, for token counts whose token tiles
 // times expert chunks would occupy few SMs (decode): unit = (token tile m,

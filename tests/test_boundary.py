@@ -54,6 +54,10 @@ def test_workspace_size_valid_and_invalid():
         assert M.mrlmoe_workspace_size(_cfg(**bad)) == 0, bad
     for hold in (1, 2, 4, 7):                                    # the GEMM families of mrlmoe_hold
         assert M.mrlmoe_workspace_size(_cfg(hold=hold)) > 0
+    # k up to min(E, 32)
+    assert M.mrlmoe_workspace_size(_cfg(top_k=32, n_experts=32)) > 0
+    assert M.mrlmoe_workspace_size(_cfg(top_k=17, n_experts=64)) > 0
+    assert M.mrlmoe_workspace_size(_cfg(top_k=33, n_experts=64)) == 0
     for agg in (0, 1, 2):                                       # mean, sum, max
         assert M.mrlmoe_workspace_size(_cfg(aggregation=agg)) > 0
     # the FP8 variant stages at most 32 K-block scales per GEMM unit: K <= 4096

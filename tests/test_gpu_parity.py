@@ -63,7 +63,7 @@ def _scores_case(name, T, E, k):
 
 @pytest.mark.parametrize("case", ["uniform", "dyadic_ties", "all_equal", "signed_zeros"])
 @pytest.mark.parametrize("T,E,k", [(64, 16, 2), (1, 16, 2), (33, 512, 10), (1000, 512, 10),
-                                   (257, 1024, 16)])
+                                   (257, 1024, 16), (513, 512, 17), (300, 64, 24), (77, 32, 32)])
 def test_route_scores_in_bit_exact(case, T, E, k):
     shape = W.LayerShape("t", T=T, d_model=256, d_lat=128, n_experts=E, top_k=k, d_ff=128, n_routers=1)
     s, b = _scores_case(case, T, E, k)
