@@ -530,7 +530,11 @@ def main():
                                    "t_bytes_ms": t_bytes * 1e3, "t_flops_ms": t_flops * 1e3,
                                    "frac": max(t_bytes, t_flops) / step_s,
                                    "tensor_frac_of_bf16_peak": flops / step_s / (peaks["bf16_tflops"] * 1e12),
-                                   "peaks": peak_kind},
+                                   "peaks": peak_kind,
+                                   # the same against the nominal datasheet figures (HBM 8 TB/s,
+                                   # dense bf16 2.25 PFLOP/s, dense e4m3 4.5 PFLOP/s)
+                                   "frac_nominal": max(byts / 8.0e12,
+                                                       flops / ((4.5e15 if s.fp8 else 2.25e15))) / step_s},
                 "stage_ms": dict(zip(M._native.STAGES, [round(v, 4) for v in stage_ms])),
             },
             "roofline": ({"kernel": "gate_up_glu (grouped tcgen05 GEMM, SiLU-GLU epilogue)",
