@@ -268,3 +268,47 @@ def test_forward_c4_fp8_sampled_tokens():
     check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
     tokens = torch.tensor([0, 1, 777, 8192, 16383])
     _compare_fp8(s, x, bias, y, r, host_weights("c4_fp8"), tokens=tokens)
+
+
+def test_forward_fp8_groups_of_every_size():
+    # every token on expert 0 (300 rows: two full 128-row tiles and a ragged
+    # one), expert 5 favoured, a small ramp over the rest: groups of 1 to ~100
+    # rows, so the token tiles load 16, 32, 32+16, 64 and 64+32+16-row boxes
+    s = W.CONFIGS["c0_fp8"].with_T(300)
+    bias = torch.linspace(0.0, 0.05, s.n_experts, dtype=torch.float32)
+    bias[0] = 10.0
+    bias[5] += 0.2
+    s, x, bias, y, r, _ = _run_layer("c0_fp8", T=300, bias=bias.cuda())
+    counts = r["counts"].cpu()
+    assert int(counts.min()) < 16 and int(counts[0]) == 300
+    assert len(set((int(c) + 15) // 16 for c in counts)) >= 5
+    _compare_fp8(s, x, bias, y, r, host_weights("c0_fp8"))
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+
+
+def test_forward_fp8_decode_size_sampled_tokens():
+    s, x, bias, y, r, _ = _run_layer("c4_fp8", T=128, scores=False)
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+    _compare_fp8(s, x, bias, y, r, host_weights("c4_fp8"), tokens=torch.tensor([0, 63, 127]))
+
+
+@pytest.mark.parametrize("T", [1152, 1153])
+def test_route_either_side_of_the_router_k_split(T):
+    # E = 512, R = 4: 8 expert chunks; 9 token tiles (T = 1152) take the
+    # K-split router, 10 (T = 1153) the one that splits the expert range
+    s = W.LayerShape("split", T=T, d_model=256, d_lat=128, n_experts=512, top_k=10, d_ff=128, n_routers=4)
+    w = W.make_routing_weights(s, "cuda")
+    x = W.make_x(s, "cuda")
+    bias = W.uniform((s.n_experts,), -0.02, 0.02, 3, 940, "cuda")
+    layer = M.MRLMoELayer(s, w)
+    r = layer.routing_buffers(scores=True)
+    layer.route(bias, x=x, routing=r)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    zx = x.cpu().double() @ w["w_down"].cpu().double().T
+    s_ref = O.router_scores(zx, w["w_router"].cpu())
+    sg = r["scores"].view(T, s.n_experts).cpu().double()
+    assert (sg - s_ref.double()).abs().max().item() < 1e-5
+    bad, gaps, _ = routing_audit(r["topk_idx"].view(-1, s.top_k), s_ref, bias, s.top_k)
+    assert torch.all(gaps < GAP_TOL), (bad, gaps)
+    check_dispatch_properties(r, T, s.n_experts, s.top_k)
