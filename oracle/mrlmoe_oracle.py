@@ -55,6 +55,7 @@ __all__ = [
     "bf16_round", "linear_bf16", "router_scores", "select_topk", "route_weights",
     "permutation", "expert_glu", "rmsnorm", "forward", "bias_update",
     "e4m3_decode", "e4m3_encode", "quantize_act_1x128", "dequantize_weight_128x128",
+    "e2m1_decode", "unpack_e2m1", "dequantize_weight_fp4_128x128", "FP4_MATRICES",
     "OracleResult", "topk_boundary_gap",
 ]
 
@@ -292,6 +293,44 @@ def dequantize_weight_128x128(codes: torch.Tensor, scales: torch.Tensor) -> torc
 
 
 # ---------------------------------------------------------------------------
+# FP4 e2m1 (OCP Microscaling Formats v1.0, FP4 element type: 1 sign, 2
+# exponent bits with bias 1, 1 mantissa bit, no inf or NaN, max 6) for the
+# FP4 expert variant.  The pages say only that the post-trained release ships
+# FP4 weights; this variant's reading: every expert matrix (routed and
+# shared) holds e2m1 codes, two per byte along K (element 2i in the low
+# nibble), with one fp32 scale per 128x128 block as in the FP8 variant; the
+# projections, activations and routers are as in the FP8 variant.
+# ---------------------------------------------------------------------------
+FP4_MATRICES = ("w_gate", "w_up_e", "w_down_e", "w_sh_gate", "w_sh_up", "w_sh_down")
+
+
+def e2m1_decode(codes: torch.Tensor) -> torch.Tensor:
+    """Value of each 4-bit e2m1 code (low nibble of the input), float64:
+    exponent field 0 is subnormal (0 or 0.5), else (1 + m/2) 2^(e-1)."""
+    c = codes.to(torch.int64) & 0xF
+    e = (c >> 1) & 3
+    m = (c & 1).to(F64)
+    v = torch.where(e == 0, m * 0.5, (1.0 + m / 2.0) * torch.pow(2.0, (e - 1).to(F64)))
+    return torch.where((c >> 3) == 1, -v, v)
+
+
+def unpack_e2m1(packed: torch.Tensor) -> torch.Tensor:
+    """[..., n] bytes -> [..., 2n] codes: byte i holds element 2i in its low
+    nibble and element 2i + 1 in its high nibble."""
+    b = packed.to(torch.int64) & 0xFF
+    return torch.stack((b & 0xF, b >> 4), dim=-1).reshape(*b.shape[:-1], 2 * b.shape[-1])
+
+
+def dequantize_weight_fp4_128x128(packed: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
+    """W = e2m1(code) * scale[block] for 128x128 blocks of an [out, in]
+    matrix given as packed codes [out, in / 2]."""
+    codes = unpack_e2m1(packed)
+    out, inn = codes.shape
+    s = scales.to(F64).repeat_interleave(128, 0)[:out].repeat_interleave(128, 1)[:, :inn]
+    return e2m1_decode(codes) * s
+
+
+# ---------------------------------------------------------------------------
 # the layer
 # ---------------------------------------------------------------------------
 @dataclass
@@ -318,7 +357,8 @@ def _w(weights, name, fp8_deq, e=None):
 
 def forward(x: torch.Tensor, weights: Dict[str, torch.Tensor], bias: torch.Tensor,
             top_k: int, rms_eps: float = 1e-6, fp8: bool = False,
-            scores: Optional[torch.Tensor] = None, aggregation: str = "mean") -> OracleResult:
+            scores: Optional[torch.Tensor] = None, aggregation: str = "mean",
+            fp4: bool = False) -> OracleResult:
     """The layer on CPU, step by step.
 
     1. z = bf16(x W_dn^T)                          down-projection 4096 -> 2048
@@ -334,16 +374,21 @@ def forward(x: torch.Tensor, weights: Dict[str, torch.Tensor], bias: torch.Tenso
     ``scores`` replaces steps 1-3 with the given fp32 s (routing-only use; z,
     c, n and y are then not computed).  In FP8 mode ``weights`` carries e4m3
     codes for every projection and expert matrix w_<x> and its 128x128 block
-    scales as s_<x>; the routers stay bf16.
+    scales as s_<x>; the routers stay bf16.  FP4 mode (``fp4``) is FP8 mode
+    with the expert matrices (FP4_MATRICES) given as packed e2m1 codes
+    [.., out, in / 2] with the same 128x128 block scales.
     """
     E = weights["expert_scale"].numel()
     deq = None
+    if fp4:
+        fp8 = True                 # projections, activations and routers as in FP8 mode
     if fp8:
         def mk(nm):
             codes, sc = weights[nm], weights["s_" + nm[2:]]   # scale array: w_<x> -> s_<x>
+            dq = dequantize_weight_fp4_128x128 if (fp4 and nm in FP4_MATRICES) else dequantize_weight_128x128
             if codes.dim() == 3:
-                return lambda e: dequantize_weight_128x128(codes[e], sc[e])
-            return lambda: dequantize_weight_128x128(codes, sc)
+                return lambda e: dq(codes[e], sc[e])
+            return lambda: dq(codes, sc)
         deq = {nm: mk(nm) for nm in ("w_down", "w_gate", "w_up_e", "w_down_e",
                                       "w_sh_gate", "w_sh_up", "w_sh_down", "w_up")}
     if scores is None:

@@ -401,6 +401,89 @@ def test_weight_dequant_blocks():
     assert torch.all(wd[:128] == 2.0) and torch.all(wd[128:] == 0.5)
 
 
+# ------------------------------------------------------------- FP4 e2m1
+# OCP Microscaling Formats (MX) v1.0, FP4 E2M1: exponent bias 1, one mantissa
+# bit, exponent field 0 subnormal, no inf/NaN; the positive values are
+# 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+E2M1_POSITIVE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_decode_table():
+    dec = O.e2m1_decode(torch.arange(16))
+    assert dec[:8].tolist() == E2M1_POSITIVE
+    assert dec[8:].tolist() == [-v for v in E2M1_POSITIVE]
+    assert torch.signbit(dec[8])                                  # code 8 is -0
+    assert torch.equal(O.e2m1_decode(torch.arange(16) + 16 * 5), dec)   # only the low nibble counts
+
+
+def test_e2m1_values_are_exact_e4m3_values():
+    # every e2m1 value has an e4m3 code of exactly that value (the FP4 GEMM
+    # feeds its weights to the tensor core as e4m3 codes)
+    dec = O.e2m1_decode(torch.arange(16))
+    codes = O.e4m3_encode(dec)
+    assert torch.equal(O.e4m3_decode(codes), dec)
+    assert [int(c) for c in codes[:8]] == [0x00, 0x30, 0x38, 0x3C, 0x40, 0x44, 0x48, 0x4C]
+
+
+def test_unpack_order_low_nibble_first():
+    packed = torch.tensor([[0x21, 0xF8]], dtype=torch.uint8)
+    assert O.unpack_e2m1(packed).tolist() == [[1, 2, 8, 15]]
+    assert O.e2m1_decode(O.unpack_e2m1(packed)).tolist() == [[0.5, 1.0, -0.0, -6.0]]
+
+
+def test_fp4_weight_dequant_blocks():
+    # [200, 256]: two block rows (the second ragged) x two block columns
+    codes = torch.zeros(200, 256, dtype=torch.int64)
+    codes[:, :128] = 2                       # 1.0
+    codes[:, 128:] = 15                      # -6.0
+    codes[5, 7] = 1                          # 0.5
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).to(torch.uint8)
+    sc = torch.tensor([[2.0, 0.25], [0.5, 4.0]])
+    wd = O.dequantize_weight_fp4_128x128(packed, sc)
+    assert wd.shape == (200, 256)
+    assert torch.all(wd[:128, :128][codes[:128, :128] == 2] == 2.0) and wd[5, 7].item() == 1.0
+    assert torch.all(wd[:128, 128:] == -1.5) and torch.all(wd[128:, :128] == 0.5)
+    assert torch.all(wd[128:, 128:] == -24.0)
+
+
+def test_fp4_layer_equals_fp8_layer_on_the_same_values():
+    # the FP4 variant with e2m1 codes is the FP8 variant with the e4m3 codes
+    # of the same values and the same scales: the oracle's FP4 mode must give
+    # the FP8 mode's result exactly
+    s = W.CONFIGS["c0_fp4"]
+    w4 = W.make_layer_weights(s, "cpu")
+    w8 = dict(w4)
+    for nm in O.FP4_MATRICES:
+        w8[nm] = O.e4m3_encode(O.e2m1_decode(O.unpack_e2m1(w4[nm])))
+    x = W.make_x(s, "cpu")
+    bias = W.uniform((s.n_experts,), -0.01, 0.01, 4, 950, "cpu")
+    r4 = O.forward(x, w4, bias, s.top_k, s.rms_eps, fp4=True)
+    r8 = O.forward(x, w8, bias, s.top_k, s.rms_eps, fp8=True)
+    assert torch.equal(r4.y, r8.y) and torch.equal(r4.topk_idx, r8.topk_idx)
+    # and it is not the bf16 layer: the weights really are 4-bit
+    rb = O.forward(x, W.make_weights(s, "cpu"), bias, s.top_k, s.rms_eps)
+    assert not torch.equal(r4.y, rb.y)
+
+
+def test_fp4_input_quantiser_nearest_value():
+    # the input generator's e2m1 rounding: every weight lands on the nearest
+    # e2m1 multiple of its block scale (ties excepted), and the block maximum on +-6
+    g = torch.Generator().manual_seed(12)
+    w = torch.randn(256, 256, generator=g)
+    packed, sc = W.to_fp4_blocks(w)
+    wd = O.dequantize_weight_fp4_128x128(packed, sc)
+    grid = torch.tensor(E2M1_POSITIVE, dtype=F64)
+    for bi in range(2):
+        for bj in range(2):
+            blk = w[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128].to(F64)
+            s_ = sc[bi, bj].item()
+            dq = wd[bi * 128:(bi + 1) * 128, bj * 128:(bj + 1) * 128]
+            assert abs(dq.abs().max().item() - 6.0 * s_) < 1e-12
+            err = (dq - blk).abs()
+            best = ((blk.abs()[..., None] / s_ - grid).abs().min(dim=-1).values * s_)
+            assert torch.all(err <= best + 1e-9)
+
+
 # ----------------------------------------------------- consistency with pages
 def test_full_width_shapes_consistent_with_page_totals():
     s = W.CONFIGS["c2_prefill"]

@@ -40,7 +40,8 @@ class LayerShape:
 
     T tokens; d_model hidden; d_lat latent; n_experts routed experts; top_k
     selected per token; d_ff expert intermediate; n_routers sigmoid routers.
-    ``fp8`` selects the e4m3 block-scaled expert/projection variant.
+    ``fp8`` selects the e4m3 block-scaled expert/projection variant; ``fp4``
+    (with ``fp8``) gives the expert matrices as packed e2m1 codes instead.
     """
     name: str
     T: int
@@ -52,6 +53,7 @@ class LayerShape:
     n_routers: int
     rms_eps: float = 1e-6
     fp8: bool = False
+    fp4: bool = False              # expert matrices e2m1 (implies the FP8 variant elsewhere)
     bias_kind: str = "zero"        # "zero" | "zipf"
     aggregation: str = "mean"      # router score aggregation: "mean" | "sum" | "max"
     outlier_frac: float = 0.0      # fraction of x channels scaled by outlier_scale
@@ -79,6 +81,11 @@ CONFIGS: Dict[str, LayerShape] = {
     # test case: the tiny layer in the FP8 variant (2 of the 256 x channels are outliers)
     "c0_fp8": LayerShape("c0_fp8", T=64, d_model=256, d_lat=128, n_experts=16, top_k=2, d_ff=128,
                          n_routers=2, fp8=True, outlier_frac=0.01),
+    # FP4 expert weights (e2m1, 128x128 block scales), the rest as in the FP8
+    # variant: the decode-sized full-width layer, and the tiny test layer
+    "c1_fp4": LayerShape("c1_fp4", T=128, fp8=True, fp4=True, outlier_frac=0.01, **_FULL),
+    "c0_fp4": LayerShape("c0_fp4", T=64, d_model=256, d_lat=128, n_experts=16, top_k=2, d_ff=128,
+                         n_routers=2, fp8=True, fp4=True, outlier_frac=0.01),
 }
 
 # Scalar lambda for the c3_skew bias b_e = lambda * ln(p_rank(e) / p_1), with
@@ -277,6 +284,53 @@ def make_weights_fp8(s: LayerShape, device, seed: Optional[int] = None) -> Dict[
         w[nm] = codes
         w[fp8_scale_name(nm)] = scale
     return w
+
+
+FP4_MATRICES = ("w_gate", "w_up_e", "w_down_e", "w_sh_gate", "w_sh_up", "w_sh_down")
+_E2M1_UP = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)   # midpoints of the e2m1 magnitudes
+
+
+def to_fp4_blocks(w: torch.Tensor):
+    """Packed e2m1 codes and fp32 scales per 128x128 block of the trailing
+    [out, in] dims (in even): scale = fp32(amax / 6) (1 for an all-zero
+    block); each w / scale goes to the nearest of 0, 0.5, 1, 1.5, 2, 3, 4, 6
+    (the midpoint 0.75, 1.75 and 3.5 upward, the others downward) with its
+    sign; byte i of a row holds element 2i in its low nibble.  Codes [..,
+    out, in / 2] uint8."""
+    *lead, out, inn = w.shape
+    ob, ib = (out + 127) // 128, (inn + 127) // 128
+    pad = torch.zeros(*lead, ob * 128, ib * 128, dtype=torch.float32, device=w.device)
+    pad[..., :out, :inn] = w.to(torch.float32)
+    blk = pad.reshape(*lead, ob, 128, ib, 128)
+    amax = blk.abs().amax(dim=(-3, -1))
+    scale = torch.where(amax == 0, torch.ones_like(amax), amax / torch.tensor(6.0))
+    q = (blk / scale[..., :, None, :, None]).reshape(*lead, ob * 128, ib * 128)[..., :out, :inn]
+    a = q.abs()
+    mag = torch.zeros_like(a, dtype=torch.uint8)
+    for i, t in enumerate(_E2M1_UP):
+        mag += (a >= t) if i in (1, 3, 5) else (a > t)
+    code = mag | (torch.signbit(q).to(torch.uint8) << 3)
+    packed = code[..., 0::2] | (code[..., 1::2] << 4)
+    return packed.contiguous(), scale.contiguous()
+
+
+def make_weights_fp4(s: LayerShape, device, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """The FP4 expert variant's inputs: the FP8 variant's, with the expert
+    matrices (routed and shared) re-quantised from the bf16 draws as packed
+    e2m1 codes plus fp32 128x128 block scales under the same names."""
+    w = make_weights(s, device, seed)
+    for nm in FP8_MATRICES:
+        codes, scale = (to_fp4_blocks if nm in FP4_MATRICES else to_fp8_blocks)(w[nm])
+        w[nm] = codes
+        w[fp8_scale_name(nm)] = scale
+    return w
+
+
+def make_layer_weights(s: LayerShape, device, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """The weights of a config in its variant (bf16, FP8 or FP4 experts)."""
+    if s.fp4:
+        return make_weights_fp4(s, device, seed)
+    return (make_weights_fp8 if s.fp8 else make_weights)(s, device, seed)
 
 
 def fp8_scale_name(matrix: str) -> str:
