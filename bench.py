@@ -35,7 +35,9 @@ KERNELS_PER_STEP = 11          # launches of this library's kernels per forward 
 def kernels_per_step(s, sms: int) -> int:
     """Kernel launches of one forward: 11, plus the router's merge kernel when
     the library splits the expert chunks of a token tile over several CTAs
-    (same rule as router_parts in the library)."""
+    (same rule as router_parts in the library), or plus two (the score pass
+    and the top-k) when it splits the router's K range instead (small T; same
+    rule as router_ksplit)."""
     ec = 16
     for c in (256, 128, 64, 32, 16):
         if c * s.n_routers <= 256 and s.n_experts % c == 0:
@@ -43,6 +45,8 @@ def kernels_per_step(s, sms: int) -> int:
             break
     m_tiles = (s.T + 127) // 128
     chunks = s.n_experts // ec
+    if 2 * m_tiles * chunks <= 148 and s.d_lat // 64 % 2 == 0:
+        return KERNELS_PER_STEP + 2 + (3 if s.fp8 else 0)
     parts = 1
     while parts * 2 <= chunks and chunks % (parts * 2) == 0 and m_tiles * parts * 2 <= sms:
         parts *= 2
@@ -208,8 +212,9 @@ def layer_bytes_flops(s, counts):
     import workloads as W
     touched = int((counts > 0).sum())
     D, L, E, F, R, T = s.d_model, s.d_lat, s.n_experts, s.d_ff, s.n_routers, s.T
-    wb = 1 if s.fp8 else 2                       # bytes per expert / projection weight
-    expert = 3 * F * L * wb
+    wb = 1 if s.fp8 else 2                       # bytes per projection weight
+    we = 0.5 if s.fp4 else wb                    # bytes per expert weight (e2m1: half a byte)
+    expert = int(3 * F * L * we)
     byts = (touched + 1) * expert + (L * D + D * L) * wb + R * E * L * 2 + L * 4 + 2 * T * D * 2
     return byts, W.flops_per_token(s) * T, touched
 
@@ -220,7 +225,8 @@ def glu_kernel_bytes(s, touched):
     read once, and h written once."""
     rows = s.T * s.top_k + s.T
     wb = 1 if s.fp8 else 2
-    return (touched + 1) * 2 * s.d_ff * s.d_lat * wb + rows * s.d_lat * wb + rows * s.d_ff * 2
+    we = 0.5 if s.fp4 else wb
+    return int((touched + 1) * 2 * s.d_ff * s.d_lat * we) + rows * s.d_lat * wb + rows * s.d_ff * 2
 
 
 def glu_kernel_flops(s):
@@ -266,7 +272,7 @@ def cpu_baseline(s, weights_dev, x_dev, bias_dev, ntok):
     xs = x_dev[:ntok].cpu()
     b = bias_dev.cpu()
     t0 = time.perf_counter()
-    O.forward(xs, wh, b, s.top_k, s.rms_eps, fp8=s.fp8)
+    O.forward(xs, wh, b, s.top_k, s.rms_eps, fp8=s.fp8, fp4=s.fp4)
     dt = time.perf_counter() - t0
     return {"value": ntok / dt, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
             "sample": f"first {ntok} tokens of the {s.name} batch (fp64 oracle, {dt:.1f} s)"}
@@ -283,17 +289,17 @@ def run_reference(args):
     import workloads as W
     s = shape_from_args(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    w = {k: v.cpu() for k, v in (W.make_weights_fp8 if s.fp8 else W.make_weights)(s, dev).items()}
+    w = {k: v.cpu() for k, v in W.make_layer_weights(s, dev).items()}
     per_step = 1
     n = args.warmup + args.steps
     x = W.make_x(s, dev, T=min(s.T, n * per_step)).cpu()
     b = W.make_bias(s, "cpu")
     for i in range(args.warmup):
-        O.forward(x[i:i + 1], w, b, s.top_k, s.rms_eps, fp8=s.fp8)
+        O.forward(x[i:i + 1], w, b, s.top_k, s.rms_eps, fp8=s.fp8, fp4=s.fp4)
     t0 = time.perf_counter()
     for i in range(args.steps):
         j = (args.warmup + i) % x.shape[0]
-        O.forward(x[j:j + per_step], w, b, s.top_k, s.rms_eps, fp8=s.fp8)
+        O.forward(x[j:j + per_step], w, b, s.top_k, s.rms_eps, fp8=s.fp8, fp4=s.fp4)
     dt = time.perf_counter() - t0
     v = args.steps * per_step / dt
     line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
@@ -373,7 +379,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     s = shape_from_args(args)
-    weights = (W.make_weights_fp8 if s.fp8 else W.make_weights)(s, dev)
+    weights = W.make_layer_weights(s, dev)
     x = W.make_x(s, dev, seed=s.seed + rank)
     bias = W.make_bias(s, dev)
     layer = M.MRLMoELayer(s, weights, device=dev)
@@ -522,7 +528,9 @@ def main():
                 "workload": f"{workload}: T={s.T} tokens, d_model {s.d_model} -> d_lat {s.d_lat}, "
                             f"{s.n_experts} experts top-{s.top_k} + 1 shared, d_ff {s.d_ff}, "
                             f"R={s.n_routers} routers, "
-                            + ("e4m3 experts and projections (128x128 block scales), bf16 routers" if s.fp8 else "bf16"),
+                            + ("e2m1 experts, e4m3 projections (128x128 block scales), e4m3 activations, bf16 routers"
+                               if s.fp4 else
+                               "e4m3 experts and projections (128x128 block scales), bf16 routers" if s.fp8 else "bf16"),
                 "T": s.T, "parallelism": f"replicas x{world} (expert weights replicated, own batch per GPU)",
                 "l2": "inputs larger than L2 (expert weights streamed every step)",
                 "touched_experts": touched,

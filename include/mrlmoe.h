@@ -60,9 +60,18 @@ typedef enum {
 
 typedef enum {
   MRLMOE_BF16 = 0,              /* bf16 weights and activations, fp32 accumulate */
-  MRLMOE_FP8_E4M3_BLOCK128 = 1  /* e4m3 weights with fp32 scales per 128x128 block,
+  MRLMOE_FP8_E4M3_BLOCK128 = 1, /* e4m3 weights with fp32 scales per 128x128 block,
                                    activations quantised e4m3 per 1x128 block;
                                    the routers stay bf16, y is bf16               */
+  MRLMOE_FP4_E2M1_BLOCK128 = 2  /* as MRLMOE_FP8_E4M3_BLOCK128, but the six expert
+                                   matrices (routed gate/up/down, shared gate/up/
+                                   down) hold e2m1 codes (OCP MX FP4), two per
+                                   byte along K (lower index in the low nibble):
+                                   [.., out, in/2] bytes, 16-byte aligned, with
+                                   the same fp32 128x128 block scales s_*; the
+                                   projections stay e4m3.  Reading of "the
+                                   release ships FP4 weights"; tuned for
+                                   decode-sized batches (token tiles of 64)   */
 } mrlmoe_dtype;
 
 /* How the R sigmoid router scores of a (token, expert) are aggregated into

@@ -15,7 +15,7 @@ import os
 from typing import Dict, Optional
 
 from . import _native
-from ._native import (MRLMOE_BF16, MRLMOE_FP8_E4M3_BLOCK128, Config, MrlmoeError, Routing,
+from ._native import (MRLMOE_BF16, MRLMOE_FP8_E4M3_BLOCK128, MRLMOE_FP4_E2M1_BLOCK128, Config, MrlmoeError, Routing,
                       Weights, make_config, make_routing, make_weights, mrlmoe_bias_update,
                       mrlmoe_forward, mrlmoe_forward_timed, mrlmoe_get_device_status, mrlmoe_linear, mrlmoe_route,
                       mrlmoe_route_scores_static, mrlmoe_quantize_e4m3, mrlmoe_check_routing,
@@ -26,7 +26,7 @@ __all__ = ["MRLMoELayer", "Config", "Weights", "Routing", "MrlmoeError", "make_c
            "mrlmoe_bias_update", "mrlmoe_linear", "mrlmoe_workspace_size",
            "mrlmoe_get_device_status", "mrlmoe_route_scores_static", "mrlmoe_quantize_e4m3",
            "mrlmoe_check_routing", "mrlmoe_get_device_detail", "status_string", "MRLMOE_BF16",
-           "MRLMOE_FP8_E4M3_BLOCK128", "HOLD", "CHECK_BITS"]
+           "MRLMOE_FP8_E4M3_BLOCK128", "MRLMOE_FP4_E2M1_BLOCK128", "HOLD", "CHECK_BITS"]
 
 
 class MRLMoELayer:

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libmrlmoe.so")
 
 MRLMOE_BF16 = 0
 MRLMOE_FP8_E4M3_BLOCK128 = 1
+MRLMOE_FP4_E2M1_BLOCK128 = 2
 
 STATUS = {0: "MRLMOE_OK", 1: "MRLMOE_ERR_INVALID_ARG", 2: "MRLMOE_ERR_UNSUPPORTED",
           3: "MRLMOE_ERR_WORKSPACE", 4: "MRLMOE_ERR_CUDA", 5: "MRLMOE_ERR_TIMEOUT",
@@ -138,9 +139,10 @@ def make_config(shape, T: Optional[int] = None, fp8: Optional[bool] = None, hold
     `aggregation` attribute means the mean).  ``hold``: mrlmoe_config.hold
     (0 in normal use; an OR of HOLD values makes those GEMMs' waits run out)."""
     f8 = shape.fp8 if fp8 is None else fp8
+    f4 = bool(getattr(shape, "fp4", False))
     return Config(shape.T if T is None else T, shape.d_model, shape.d_lat, shape.n_experts,
                   shape.top_k, shape.d_ff, shape.n_routers, float(shape.rms_eps),
-                  MRLMOE_FP8_E4M3_BLOCK128 if f8 else MRLMOE_BF16,
+                  MRLMOE_FP4_E2M1_BLOCK128 if f4 else MRLMOE_FP8_E4M3_BLOCK128 if f8 else MRLMOE_BF16,
                   AGGREGATIONS[getattr(shape, "aggregation", "mean")], int(hold))
 
 

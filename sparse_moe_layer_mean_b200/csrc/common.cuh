@@ -99,6 +99,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (the tensor core reading them as an MMA operand).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion on an mbarrier.
 // x is the innermost (contiguous) coordinate in elements, y the row.

@@ -70,6 +70,53 @@ __device__ __forceinline__ void load_token_rows8(const TokenMaps8 &t, int kb, in
   if (r + 16 <= n) tma_load_2d(sa + r * 128, &t.m16, bar, x, y0 + r);
 }
 
+// ------------------------------------------------------------ FP4 weights
+// Expert weights given as packed e2m1 codes (two per byte, the lower K index
+// in the low nibble) are expanded in shared memory into the e4m3 B tile the
+// MMA reads.  The expansion is exact: every e2m1 value is an e4m3 value, so
+// it is a table lookup, done on the integer pipes with byte permutes.
+//   magnitude code 0..7 (0, 0.5, 1, 1.5, 2, 3, 4, 6) -> e4m3 byte
+//   00 30 38 3C 40 44 48 4C, and the code's sign bit (bit 3) -> bit 7.
+// c holds 4 codes in bits 0..15 (code i in nibble i); the result holds their
+// 4 e4m3 bytes (byte i from code i).  The second permute uses the selector's
+// bit 3 in its sign-replicating sense: a negative code's byte becomes 0xFF
+// (the table bytes 0x80 have their msb set), a positive one's 0x80.
+__device__ __forceinline__ uint32_t e2m1x4_to_e4m3x4(uint32_t c) {
+  uint32_t mag, sgn;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(mag) : "r"(0x3C383000u), "r"(0x4C484440u), "r"(c & 0x7777u));
+  asm("prmt.b32 %0, %1, %1, %2;" : "=r"(sgn) : "r"(0x80808080u), "r"(c & 0xFFFFu));
+  return mag | (((sgn & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u);
+}
+
+// 16 packed bytes (32 codes) -> 32 e4m3 bytes in the same element order.
+__device__ __forceinline__ void e2m1x32_to_e4m3(uint4 in, uint4 &lo, uint4 &hi) {
+  lo = make_uint4(e2m1x4_to_e4m3x4(in.x), e2m1x4_to_e4m3x4(in.x >> 16), e2m1x4_to_e4m3x4(in.y),
+                  e2m1x4_to_e4m3x4(in.y >> 16));
+  hi = make_uint4(e2m1x4_to_e4m3x4(in.z), e2m1x4_to_e4m3x4(in.z >> 16), e2m1x4_to_e4m3x4(in.w),
+                  e2m1x4_to_e4m3x4(in.w >> 16));
+}
+
+// One K block of packed weights (128 rows x 64 B, row-major at src) into the
+// e4m3 B tile at dst (128 rows x 128 B, 16-byte chunk c of row r at chunk
+// position c ^ (r & 7): the SWIZZLE_128B layout TMA would write; dst is
+// 1024-byte aligned).  Thread tid of the 256 promotion threads takes 16
+// packed bytes: row tid / 4 (+64 in the second pass), quarter tid % 4.
+__device__ __forceinline__ void expand_fp4_tile(const uint8_t *src, uint8_t *dst, int tid) {
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int r = pass * 64 + (tid >> 2), q = tid & 3;
+    const uint4 in = *reinterpret_cast<const uint4 *>(src + r * 64 + q * 16);
+    uint4 lo, hi;
+    e2m1x32_to_e4m3(in, lo, hi);
+    const int sw = r & 7;
+    *reinterpret_cast<uint4 *>(dst + r * 128 + (((2 * q) ^ sw) << 4)) = lo;
+    *reinterpret_cast<uint4 *>(dst + r * 128 + (((2 * q + 1) ^ sw) << 4)) = hi;
+  }
+}
+
+// K blocks the promotion warps expand ahead of the one they promote.
+constexpr int kF4Ahead = 3;
+
 __device__ __forceinline__ void prefetch_token_maps8(const TokenMaps8 &t) {
   prefetch_tmap(&t.m16);
   prefetch_tmap(&t.m32);
@@ -91,7 +138,7 @@ struct Gemm8Smem {
   static constexpr int kRing = kF8Ring * kStageBytes;
   static constexpr int kTabOff = kRing;
   static constexpr int kBarOff = kTabOff + 2 * kF8TabFloats * 4;
-  static constexpr int kNumBars = 3 * kF8Ring + 4;
+  static constexpr int kNumBars = 4 * kF8Ring + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kEpiOff = (kMiscOff + 16 + 127) & ~127;
   static constexpr int kAuxOff = (kEpiOff + P::kEpiSmem + 127) & ~127;
@@ -122,7 +169,8 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
   const uint32_t full0 = smem_u32(bars);
   const uint32_t done0 = full0 + 8 * kF8Ring;   // MMAs of the K block completed
   const uint32_t free0 = done0 + 8 * kF8Ring;   // partial buffer promoted
-  const uint32_t sfull0 = free0 + 8 * kF8Ring;  // scale table b written
+  const uint32_t ready0 = free0 + 8 * kF8Ring;  // FP4: the stage's B tile expanded
+  const uint32_t sfull0 = ready0 + 8 * kF8Ring; // scale table b written
   const uint32_t sempty0 = sfull0 + 16;         // scale table b read
   const uint32_t ring = smem_u32(smem);
 
@@ -136,6 +184,7 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
       mbar_init(full0 + 8 * j, 2);
       mbar_init(done0 + 8 * j, 1);
       mbar_init(free0 + 8 * j, 8);
+      mbar_init(ready0 + 8 * j, kF8PromoThreads / 32);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(sfull0 + 8 * b, 32);
@@ -174,12 +223,12 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
         for (int kb = 0; kb < kblocks; ++kb, ++g) {
           const uint32_t j = g & (kF8Ring - 1);
           if (g >= kF8Ring && !mbar_wait(done0 + 8 * j, ((g / kF8Ring) - 1) & 1, abort_flag, status)) goto done;
-          mbar_arrive_expect_tx(full0 + 8 * j, isA ? P::a_bytes(U) : kF8OpBytes);
+          mbar_arrive_expect_tx(full0 + 8 * j, isA ? P::a_bytes(U) : P::b_bytes());
           const uint32_t st = ring + j * L::kStageBytes;
           if (isA)
             P::load_a(p, U, kb, st, full0 + 8 * j);
-          else
-            P::load_b(p, U, kb, st + kF8OpBytes, full0 + 8 * j);
+          else  // FP4: the packed tile lands in the A slot's upper half (token tiles <= 64 rows)
+            P::load_b(p, U, kb, st + (P::kFp4B ? kF8OpBytes / 2 : kF8OpBytes), full0 + 8 * j);
           // the next unit's descriptor, while this unit's loads are in flight
           if (kb == 0 && u + static_cast<int>(gridDim.x) < nunits) Un = P::unit(p, u + gridDim.x, aux);
         }
@@ -192,7 +241,8 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
       for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
         for (int kb = 0; kb < kblocks; ++kb, ++g) {
           const uint32_t j = g & (kF8Ring - 1);
-          if (!mbar_wait(full0 + 8 * j, (g / kF8Ring) & 1, abort_flag, status)) goto done;
+          // FP4: the stage is ready once the promotion warps have expanded its B tile
+          if (!mbar_wait((P::kFp4B ? ready0 : full0) + 8 * j, (g / kF8Ring) & 1, abort_flag, status)) goto done;
           if (g >= kF8Ring && !mbar_wait(free0 + 8 * j, ((g / kF8Ring) - 1) & 1, abort_flag, status)) goto done;
           tc_fence_after();
           const uint32_t a_s = ring + j * L::kStageBytes;
@@ -228,16 +278,42 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
     const int cls = P::scale_class(h);
     uint32_t g = 0;
     int ul = 0;
+    // FP4: K block c of this CTA's sequence (c < ctot) is expanded while block
+    // c - kF4Ahead is promoted; its stage was last read by the MMA of block
+    // c - 4, complete once block c - kF4Ahead - 1 <= c - 4 was seen done.
+    uint32_t cx = 0;
+    const uint32_t ctot =
+        static_cast<int>(blockIdx.x) < nunits
+            ? static_cast<uint32_t>((nunits - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1) *
+                  static_cast<uint32_t>(kblocks)
+            : 0u;
+    auto expand_to = [&](uint32_t lim) -> bool {
+      for (; cx < lim && cx < ctot; ++cx) {
+        const uint32_t j = cx & (kF8Ring - 1);
+        if (!__all_sync(0xffffffffu, mbar_wait(full0 + 8 * j, (cx / kF8Ring) & 1, abort_flag, status))) return false;
+        uint8_t *stg = smem + j * L::kStageBytes;
+        expand_fp4_tile(stg + kF8OpBytes / 2, stg + kF8OpBytes, pw * 32 + lane);
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ready0 + 8 * j);
+      }
+      return true;
+    };
+    bool lost = false;  // FP4: an expansion wait gave up
+    if constexpr (P::kFp4B) lost = !expand_to(kF4Ahead);
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++ul) {
       const int b = ul & 1;
       const float *tok = tabs + b * kF8TabFloats + q * 32 + lane;
       const float *wsc = tabs + b * kF8TabFloats + kF8MaxKB * kF8Tile + cls * kF8MaxKB;
-      bool bad = !__all_sync(0xffffffffu, mbar_wait(sfull0 + 8 * b, (ul >> 1) & 1, abort_flag, status));
+      bool bad = !__all_sync(0xffffffffu, mbar_wait(sfull0 + 8 * b, (ul >> 1) & 1, abort_flag, status)) || lost;
       float acc[kF8Half];
 #pragma unroll
       for (int i = 0; i < kF8Half; ++i) acc[i] = 0.f;
       for (int kb = 0; kb < kblocks; ++kb, ++g) {
         const uint32_t j = g & (kF8Ring - 1);
+        if constexpr (P::kFp4B) {
+          if (!bad && !expand_to(g + 1 + kF4Ahead)) bad = lost = true;
+        }
         if (!bad) bad = !__all_sync(0xffffffffu, mbar_wait(done0 + 8 * j, (g / kF8Ring) & 1, abort_flag, status));
         if (bad) continue;
         const float s = tok[kb * kF8Tile] * wsc[kb];
@@ -322,6 +398,8 @@ __device__ __forceinline__ void stage_weight_scales(const float *ws0, const floa
 struct Dense8Policy {
   static constexpr int kEpiSmem = 0;
   static constexpr int kAuxSmem = 0;
+  static constexpr bool kFp4B = false;  // weights arrive as e4m3 tiles
+  static __device__ __forceinline__ uint32_t b_bytes() { return kF8OpBytes; }
   struct Params {
     CUtensorMap ta;  // a codes [M, K], box 128 x 128
     CUtensorMap tb;  // w codes [N, K], box 128 x 128
@@ -401,6 +479,8 @@ struct Dense8Policy {
 struct Glu8Policy {
   static constexpr int kEpiSmem = 8 * 32 * 33 * 4;
   static constexpr int kAuxSmem = kGroupAuxSmem;
+  static constexpr bool kFp4B = false;  // weights arrive as e4m3 tiles
+  static __device__ __forceinline__ uint32_t b_bytes() { return kF8OpBytes; }
   struct Params {
     CUtensorMap wg, wu, sg, su;  // e4m3 [E*F, L] / [F, L], box 64 x 128
     TokenMaps8 tz;               // quantised dispatched z [(T*k+T), L], boxes 16..128 x 128
@@ -501,6 +581,8 @@ struct Glu8Policy {
 struct Down8Policy {
   static constexpr int kEpiSmem = 8 * 32 * 33 * 4;
   static constexpr int kAuxSmem = kGroupAuxSmem;
+  static constexpr bool kFp4B = false;  // weights arrive as e4m3 tiles
+  static __device__ __forceinline__ uint32_t b_bytes() { return kF8OpBytes; }
   struct Params {
     CUtensorMap wd, sd;  // e4m3 [E*L, F] / [L, F], box 128 x 128
     TokenMaps8 th;       // quantised h [(T*k+T), F], boxes 16..128 x 128
@@ -593,6 +675,40 @@ struct Down8Policy {
       }
       __syncwarp();
     }
+  }
+};
+
+// FP4 expert weights: Glu8Policy / Down8Policy with each weight matrix given as
+// packed e2m1 codes [rows, K / 2] (maps with 64-byte boxes, no swizzle) and
+// token tiles of at most 64 rows, so that a K block's packed weight tile
+// (8 KB) fits in the upper half of the stage's token slot; the promotion
+// warps expand it into the stage's e4m3 B tile (expand_fp4_tile).  Scales,
+// promotion and epilogues are the FP8 policies'.
+constexpr int kF4TokTile = 64;
+
+struct Glu4Policy : Glu8Policy {
+  static constexpr bool kFp4B = true;
+  static __device__ __forceinline__ uint32_t b_bytes() { return kF8OpBytes / 2; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
+    return grouped_unit(p.gt, aux, u, kF4TokTile);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb, uint32_t bar) {
+    const bool sh = U.g == p.gt.E;
+    const int row = (sh ? 0 : U.g * p.F) + U.m * 64;
+    tma_load_2d(sb, sh ? &p.sg : &p.wg, bar, kb * 64, row);            // 64 gate rows x 64 B
+    tma_load_2d(sb + 64 * 64, sh ? &p.su : &p.wu, bar, kb * 64, row);  // then the 64 up rows
+  }
+};
+
+struct Down4Policy : Down8Policy {
+  static constexpr bool kFp4B = true;
+  static __device__ __forceinline__ uint32_t b_bytes() { return kF8OpBytes / 2; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
+    return grouped_unit(p.gt, aux, u, kF4TokTile);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb, uint32_t bar) {
+    const bool sh = U.g == p.gt.E;
+    tma_load_2d(sb, sh ? &p.sd : &p.wd, bar, kb * 64, (sh ? 0 : U.g * p.L) + U.m * 128);  // 128 rows x 64 B
   }
 };
 

@@ -32,13 +32,14 @@ mrlmoe_status check_config(const mrlmoe_config *c) {
   if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > kTopKMax) return MRLMOE_ERR_INVALID_ARG;
   if (c->n_routers < 1 || c->n_routers > 8) return MRLMOE_ERR_INVALID_ARG;
   if (!(c->rms_eps >= 0.f)) return MRLMOE_ERR_INVALID_ARG;
-  if (c->dtype != MRLMOE_BF16 && c->dtype != MRLMOE_FP8_E4M3_BLOCK128) return MRLMOE_ERR_INVALID_ARG;
+  if (c->dtype != MRLMOE_BF16 && c->dtype != MRLMOE_FP8_E4M3_BLOCK128 && c->dtype != MRLMOE_FP4_E2M1_BLOCK128)
+    return MRLMOE_ERR_INVALID_ARG;
   if (c->aggregation != MRLMOE_AGG_MEAN && c->aggregation != MRLMOE_AGG_SUM && c->aggregation != MRLMOE_AGG_MAX)
     return MRLMOE_ERR_INVALID_ARG;
   if (c->hold & ~static_cast<uint32_t>(MRLMOE_HOLD_GEMM | MRLMOE_HOLD_GEMM_PAIR | MRLMOE_HOLD_GEMM_FP8))
     return MRLMOE_ERR_INVALID_ARG;
   // the FP8 GEMMs stage at most kF8MaxKB scales of 128-wide K blocks per unit
-  if (c->dtype == MRLMOE_FP8_E4M3_BLOCK128 &&
+  if (c->dtype != MRLMOE_BF16 &&
       (c->d_model > 128 * kF8MaxKB || c->d_lat > 128 * kF8MaxKB || c->d_ff > 128 * kF8MaxKB))
     return MRLMOE_ERR_UNSUPPORTED;
   // dispatched rows are addressed with 32-bit indices
@@ -126,7 +127,7 @@ Layout layout_of(const mrlmoe_config &c) {
   L.hbuf = take((Tk + T) * F * 2);
   L.slots = take(T * (k + 1) * Ld * 4);
   L.nbuf = take(T * Ld * 2);
-  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) {  // e4m3 copies of the GEMM inputs and their 1x128 scales
+  if (c.dtype != MRLMOE_BF16) {  // e4m3 copies of the GEMM inputs and their 1x128 scales
     const size_t D = c.d_model;
     L.xq = take(T * D);
     L.xs = take(T * (D / 128) * 4);
@@ -188,6 +189,20 @@ bool make_token_maps_blocked(TokenMaps *t, const void *base, uint64_t K, uint64_
   if (!make_token_maps(t, base, 64, (K / 64) * rows)) return false;
   t->plane_rows = static_cast<int>(rows);
   return true;
+}
+
+// Packed e2m1 weights [rows, inner_bytes]: boxes of 64 bytes (128 codes) x
+// box_rows, row-major in shared memory (no swizzle; expand_fp4_tile reads it).
+bool make_map_packed(CUtensorMap *m, const void *base, uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner_bytes, rows};
+  const cuuint64_t strides[1] = {inner_bytes};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // The four box heights of an e4m3 token tensor [rows, inner] (load_token_rows8).
@@ -309,7 +324,7 @@ Ptrs carve(const mrlmoe_config &c, void *ws, const mrlmoe_routing *r) {
   P.hbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.hbuf);
   P.slots = reinterpret_cast<float *>(b + L.slots);
   P.nbuf = reinterpret_cast<__nv_bfloat16 *>(b + L.nbuf);
-  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) {
+  if (c.dtype != MRLMOE_BF16) {
     P.xq = b + L.xq; P.zq = b + L.zq; P.hq = b + L.hq; P.nq = b + L.nq;
     P.xs = reinterpret_cast<float *>(b + L.xs);
     P.zs = reinterpret_cast<float *>(b + L.zs);
@@ -330,6 +345,7 @@ struct GroupTiling {
 };
 GroupTiling group_tiling(const mrlmoe_config &c) {
   if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) return {kF8Tile, c.d_ff / 64, c.d_lat / 128};
+  if (c.dtype == MRLMOE_FP4_E2M1_BLOCK128) return {kF4TokTile, c.d_ff / 64, c.d_lat / 128};
   return {kExpertBN, glu_m_tiles(c), down_m_tiles(c)};
 }
 
@@ -466,7 +482,7 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
                                        void *const *ev = nullptr) {
   const int T = c.T, D = c.d_model, Ld = c.d_lat, E = c.n_experts, R = c.n_routers, k = c.top_k;
   __nv_bfloat16 *z = P.zbuf + static_cast<size_t>(T) * k * Ld;  // z rows live after the T*k dispatched rows
-  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) {
+  if (c.dtype != MRLMOE_BF16) {
     MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(x), D, T, D, nullptr, 1, 0, P.xq, P.xs, true, P.status,
                          st));
     mrlmoe_status s = launch_dense8(P.xq, P.xs, w->w_down, w->s_down, T, Ld, D, z, P.zlo, P, sms, st);
@@ -542,7 +558,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   mrlmoe_status s = check_config(cfg);
   if (s != MRLMOE_OK) return s;
   if (!bias || !x || !y || !aligned16(x) || !aligned16(y)) return MRLMOE_ERR_INVALID_ARG;
-  const bool fp8 = cfg->dtype == MRLMOE_FP8_E4M3_BLOCK128;
+  const bool fp8 = cfg->dtype != MRLMOE_BF16;  // e4m3 projections and activations (FP8 and FP4 variants)
   if ((s = fp8 ? check_weights_fp8(w) : check_weights_bf16(w, true)) != MRLMOE_OK) return s;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
   if (ws_bytes < layout_of(*cfg).total) return MRLMOE_ERR_WORKSPACE;
@@ -637,11 +653,16 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
                        P.status, st));
   if (!mark(4)) return MRLMOE_ERR_CUDA;
   const GroupTiling gtl = group_tiling(c);
+  const bool fp4 = c.dtype == MRLMOE_FP4_E2M1_BLOCK128;  // expert matrices as packed e2m1 codes
+  // an expert weight map: e4m3 [rows, K] with 128-byte boxes, or packed e2m1 [rows, K/2] with 64-byte boxes
+  auto wmap = [&](CUtensorMap *m, const void *base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+    return fp4 ? make_map_packed(m, base, K / 2, rows, box_rows) : make_map(m, base, 1, K, rows, box_rows);
+  };
   {
     Glu8Policy::Params p{};
-    if (!make_map(&p.wg, w->w_gate, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
-        !make_map(&p.wu, w->w_up_e, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
-        !make_map(&p.sg, w->w_sh_gate, 1, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 1, Ld, F, 64) ||
+    if (!wmap(&p.wg, w->w_gate, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !wmap(&p.wu, w->w_up_e, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !wmap(&p.sg, w->w_sh_gate, Ld, F, 64) || !wmap(&p.su, w->w_sh_up, Ld, F, 64) ||
         !make_token_maps8(&p.tz, P.zq, Ld, static_cast<uint64_t>(Tk) + T))
       return MRLMOE_ERR_CUDA;
     p.wg_s = w->s_gate; p.wu_s = w->s_up_e; p.sg_s = w->s_sh_gate; p.su_s = w->s_sh_up;
@@ -651,14 +672,16 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     p.h = P.hbuf;
     p.F = F; p.L = Ld;
     p.status = P.status;
-    MRL_TRY(launch_gemm8<Glu8Policy>(p, sms, st));
+    if (fp4)
+      MRL_TRY(launch_gemm8<Glu4Policy>(p, sms, st));
+    else
+      MRL_TRY(launch_gemm8<Glu8Policy>(p, sms, st));
   }
   MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, nullptr, 1, 0, P.hq, P.hs, true, P.status, st));
   if (!mark(5)) return MRLMOE_ERR_CUDA;
   {
     Down8Policy::Params p{};
-    if (!make_map(&p.wd, w->w_down_e, 1, F, static_cast<uint64_t>(E) * Ld, 128) ||
-        !make_map(&p.sd, w->w_sh_down, 1, F, Ld, 128) ||
+    if (!wmap(&p.wd, w->w_down_e, F, static_cast<uint64_t>(E) * Ld, 128) || !wmap(&p.sd, w->w_sh_down, F, Ld, 128) ||
         !make_token_maps8(&p.th, P.hq, F, static_cast<uint64_t>(Tk) + T))
       return MRLMOE_ERR_CUDA;
     p.wd_s = w->s_down_e; p.sd_s = w->s_sh_down;
@@ -670,7 +693,10 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     p.slots = P.slots;
     p.L = Ld; p.F = F; p.k = k; p.Tk = Tk;
     p.status = P.status;
-    MRL_TRY(launch_gemm8<Down8Policy>(p, sms, st));
+    if (fp4)
+      MRL_TRY(launch_gemm8<Down4Policy>(p, sms, st));
+    else
+      MRL_TRY(launch_gemm8<Down8Policy>(p, sms, st));
   }
   if (!mark(6)) return MRLMOE_ERR_CUDA;
   combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k, c.rms_eps,
@@ -765,7 +791,7 @@ mrlmoe_status mrlmoe_route(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
     if (!x || !aligned16(x)) return MRLMOE_ERR_INVALID_ARG;
     if ((s = check_weights_bf16(w, false)) != MRLMOE_OK) return s;
     if (!w->w_down || !aligned16(w->w_down)) return MRLMOE_ERR_INVALID_ARG;
-    if (cfg->dtype == MRLMOE_FP8_E4M3_BLOCK128 && !w->s_down) return MRLMOE_ERR_INVALID_ARG;
+    if (cfg->dtype != MRLMOE_BF16 && !w->s_down) return MRLMOE_ERR_INVALID_ARG;
   }
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
   if (ws_bytes < layout_of(*cfg).total) return MRLMOE_ERR_WORKSPACE;

@@ -24,14 +24,13 @@ def _wkey(name: str) -> str:
     """Configs with the same layer shape and weight type share one set of weights."""
     s = W.CONFIGS[name]
     if s.d_model == 256:
-        return "c0_fp8" if s.fp8 else "c0_tiny"
-    return "c4_fp8" if s.fp8 else "c2_prefill"
+        return "c0_fp4" if s.fp4 else "c0_fp8" if s.fp8 else "c0_tiny"
+    return "c1_fp4" if s.fp4 else "c4_fp8" if s.fp8 else "c2_prefill"
 
 
 @functools.lru_cache(maxsize=2)
 def _device_weights(key: str, seed: int):
-    s = W.CONFIGS[key]
-    return (W.make_weights_fp8 if s.fp8 else W.make_weights)(s, "cuda", seed=seed)
+    return W.make_layer_weights(W.CONFIGS[key], "cuda", seed=seed)
 
 
 @functools.lru_cache(maxsize=2)

@@ -237,7 +237,7 @@ def test_quantize_e4m3_bit_exact(rows, K):
 
 def _compare_fp8(s, x, bias, y, r, wh, tokens=None):
     xs = x.cpu() if tokens is None else x.cpu()[tokens]
-    ref = O.forward(xs, wh, bias.cpu(), s.top_k, s.rms_eps, fp8=True)
+    ref = O.forward(xs, wh, bias.cpu(), s.top_k, s.rms_eps, fp8=True, fp4=s.fp4)
     gidx = r["topk_idx"].view(-1, s.top_k)
     if tokens is not None:
         gidx = gidx[tokens.to(gidx.device)]
@@ -312,3 +312,34 @@ def test_route_either_side_of_the_router_k_split(T):
     bad, gaps, _ = routing_audit(r["topk_idx"].view(-1, s.top_k), s_ref, bias, s.top_k)
     assert torch.all(gaps < GAP_TOL), (bad, gaps)
     check_dispatch_properties(r, T, s.n_experts, s.top_k)
+
+
+# ------------------------------------------------ FP4 expert weights (e2m1)
+def test_forward_fp4_tiny():
+    s, x, bias, y, r, _ = _run_layer("c0_fp4")
+    _compare_fp8(s, x, bias, y, r, host_weights("c0_fp4"))
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+
+
+@pytest.mark.parametrize("T", [1, 200])
+def test_forward_fp4_tiny_ragged(T):
+    s, x, bias, y, r, _ = _run_layer("c0_fp4", T=T)
+    _compare_fp8(s, x, bias, y, r, host_weights("c0_fp4"))
+
+
+def test_forward_fp4_groups_of_every_size():
+    # as the FP8 case: expert 0 takes all 300 tokens (five 64-row token
+    # tiles, the last ragged), the other groups hold 1 to ~100 rows
+    bias = torch.linspace(0.0, 0.05, 16, dtype=torch.float32)
+    bias[0] = 10.0
+    bias[5] += 0.2
+    s, x, bias, y, r, _ = _run_layer("c0_fp4", T=300, bias=bias.cuda())
+    assert int(r["counts"][0]) == 300
+    _compare_fp8(s, x, bias, y, r, host_weights("c0_fp4"))
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+
+
+def test_forward_c1_fp4_sampled_tokens():
+    s, x, bias, y, r, _ = _run_layer("c1_fp4", scores=False)
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+    _compare_fp8(s, x, bias, y, r, host_weights("c1_fp4"), tokens=torch.tensor([0, 64, 127]))
