@@ -73,18 +73,19 @@ __device__ __forceinline__ void load_token_rows8(const TokenMaps8 &t, int kb, in
 // ------------------------------------------------------------ FP4 weights
 // Expert weights given as packed e2m1 codes (two per byte, the lower K index
 // in the low nibble) are expanded in shared memory into the e4m3 B tile the
-// MMA reads.  The expansion is exact: every e2m1 value is an e4m3 value, so
-// it is a table lookup, done on the integer pipes with byte permutes.
+// MMA reads.  The expansion is exact (every e2m1 value is an e4m3 value): a
+// table lookup on the integer pipes with byte permutes,
 //   magnitude code 0..7 (0, 0.5, 1, 1.5, 2, 3, 4, 6) -> e4m3 byte
 //   00 30 38 3C 40 44 48 4C, and the code's sign bit (bit 3) -> bit 7.
-// c holds 4 codes in bits 0..15 (code i in nibble i); the result holds their
-// 4 e4m3 bytes (byte i from code i).  The second permute uses the selector's
-// bit 3 in its sign-replicating sense: a negative code's byte becomes 0xFF
-// (the table bytes 0x80 have their msb set), a positive one's 0x80.
+// c holds 4 codes in bits 0..15 (code i in nibble i; the permutes read only
+// those bits); the result holds their 4 e4m3 bytes (byte i from code i).  The
+// second permute uses the selector's bit 3 in its sign-replicating sense: a
+// negative code's byte becomes 0xFF (the table bytes 0x80 have their msb
+// set), a positive one's 0x80.
 __device__ __forceinline__ uint32_t e2m1x4_to_e4m3x4(uint32_t c) {
   uint32_t mag, sgn;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(mag) : "r"(0x3C383000u), "r"(0x4C484440u), "r"(c & 0x7777u));
-  asm("prmt.b32 %0, %1, %1, %2;" : "=r"(sgn) : "r"(0x80808080u), "r"(c & 0xFFFFu));
+  asm("prmt.b32 %0, %1, %1, %2;" : "=r"(sgn) : "r"(0x80808080u), "r"(c));
   return mag | (((sgn & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u);
 }
 
