@@ -307,6 +307,14 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
       const float *tok = tabs + b * kF8TabFloats + q * 32 + lane;
       const float *wsc = tabs + b * kF8TabFloats + kF8MaxKB * kF8Tile + cls * kF8MaxKB;
       bool bad = !__all_sync(0xffffffffu, mbar_wait(sfull0 + 8 * b, (ul >> 1) & 1, abort_flag, status)) || lost;
+      Unit U;
+      {
+        const int *d = reinterpret_cast<const int *>(tabs + b * kF8TabFloats + kF8TabUnit);
+        U.g = d[0]; U.m = d[1]; U.n0 = d[2]; U.nv = d[3]; U.row0 = d[4]; U.nsub = 1;
+      }
+      // no token of the unit in this warp's 32 rows (decode-sized groups):
+      // its partials need no promotion, and the epilogue stores nothing for it
+      const bool idle = q * 32 >= U.nv;
       float acc[kF8Half];
 #pragma unroll
       for (int i = 0; i < kF8Half; ++i) acc[i] = 0.f;
@@ -317,6 +325,11 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
         }
         if (!bad) bad = !__all_sync(0xffffffffu, mbar_wait(done0 + 8 * j, (g / kF8Ring) & 1, abort_flag, status));
         if (bad) continue;
+        if (idle) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(free0 + 8 * j);
+          continue;
+        }
         const float s = tok[kb * kF8Tile] * wsc[kb];
         tc_fence_after();
         float v[kF8Half];
@@ -332,11 +345,6 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8_kernel(const __grid_const
           acc[i] = r.x;
           acc[i + 1] = r.y;
         }
-      }
-      Unit U;
-      {
-        const int *d = reinterpret_cast<const int *>(tabs + b * kF8TabFloats + kF8TabUnit);
-        U.g = d[0]; U.m = d[1]; U.n0 = d[2]; U.nv = d[3]; U.row0 = d[4]; U.nsub = 1;
       }
       if (bar_red_or(1, kF8PromoThreads, bad || *abort_flag)) goto done;
       P::epilogue_regs(p, U, acc, q, h, lane, epi_smem, tabs + b * kF8TabFloats + kF8TabExtra);
