@@ -37,7 +37,7 @@ def _bias(E):
 
 
 @pytest.mark.parametrize("family,config", [("gemm", "c0_tiny"), ("gemm_pair", "c0_tiny"),
-                                           ("gemm_fp8", "c0_fp8")])
+                                           ("gemm_fp8", "c0_fp8"), ("gemm_fp8", "c0_fp4")])
 def test_held_loads_run_out_the_bounded_waits(family, config):
     s = W.CONFIGS[config]
     x = W.make_x(s, "cuda")
@@ -61,7 +61,7 @@ def test_held_loads_run_out_the_bounded_waits(family, config):
 
 
 @pytest.mark.parametrize("config,T", [("c0_tiny", None), ("c0_tiny", 1), ("c0_tiny", 17),
-                                      ("c2_prefill", 300), ("c0_fp8", None)])
+                                      ("c2_prefill", 300), ("c0_fp8", None), ("c0_fp4", None)])
 def test_checker_passes_the_layers_records(config, T):
     s = W.CONFIGS[config] if T is None else W.CONFIGS[config].with_T(T)
     x = W.make_x(s, "cuda")
@@ -126,7 +126,7 @@ def _padded(n, dtype, pad, canary):
     return buf, buf[pad:pad + n].view(dtype)
 
 
-@pytest.mark.parametrize("config,T", [("c0_tiny", 37), ("c0_fp8", 37)])
+@pytest.mark.parametrize("config,T", [("c0_tiny", 37), ("c0_fp8", 37), ("c0_fp4", 37)])
 def test_outputs_and_workspace_stay_inside_their_buffers(config, T):
     s = W.CONFIGS[config].with_T(T)
     x = W.make_x(s, "cuda")
