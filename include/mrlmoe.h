@@ -243,6 +243,62 @@ mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *
 mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, float *scale,
                                    void *stream);
 
+/* ------------------------------------------------------------ training
+ * Backward pass of the layer (bf16 mode only).  The pages train the model
+ * with this layer and motivate the several routers by how they learn
+ * (derekhsu, "多路由潛在 MoE"), but give no gradient formulas; the library's
+ * readings: the top-k selection and the balancing bias carry no gradient;
+ * the selected experts' scores get it through the renormalised weights
+ * w = s_sel / sum(s_sel); the bf16 rounding points of the forward pass it
+ * through unchanged; alpha and the RMSNorm gain are learnable; with MAX
+ * aggregation the router attaining the maximum (the lowest index on ties)
+ * takes the gradient.
+ *
+ * Gradients: device pointers, caller-owned, all required.  Weight gradients
+ * are fp32 with the shapes of mrlmoe_weights (written, not accumulated);
+ * dx is bf16 [T, d_model].                                                    */
+typedef struct {
+  void  *dx;              /* [T, d_model] bf16                                  */
+  float *d_w_down;        /* [d_lat, d_model]                                   */
+  float *d_w_router;      /* [R, E, d_lat]                                      */
+  float *d_w_gate;        /* [E, d_ff, d_lat]                                   */
+  float *d_w_up_e;        /* [E, d_ff, d_lat]                                   */
+  float *d_w_down_e;      /* [E, d_lat, d_ff]                                   */
+  float *d_w_sh_gate;     /* [d_ff, d_lat]                                      */
+  float *d_w_sh_up;       /* [d_ff, d_lat]                                      */
+  float *d_w_sh_down;     /* [d_lat, d_ff]                                      */
+  float *d_rms_gain;      /* [d_lat]                                            */
+  float *d_w_up;          /* [d_model, d_lat]                                   */
+  float *d_expert_scale;  /* [E]                                                */
+} mrlmoe_grads;
+
+/* Workspace bytes for mrlmoe_forward_train + mrlmoe_backward (0 if cfg is
+ * invalid or not bf16).  Beyond mrlmoe_workspace_size: the kept gate/up
+ * pre-activations (T*k + T) * d_ff * 4 bytes and the backward's buffers,
+ * about (T*k + T) * (2 * d_lat + 2 * d_ff) * 2 bytes more.                    */
+size_t mrlmoe_train_workspace_size(const mrlmoe_config *cfg);
+
+/* mrlmoe_forward that also keeps, in `workspace`, what mrlmoe_backward reads
+ * (the forward's own scratch plus the bf16 gate and up pre-activations).
+ * ws_bytes >= mrlmoe_train_workspace_size(cfg).  bf16 mode only
+ * (MRLMOE_ERR_UNSUPPORTED otherwise), d_ff <= 8192.                           */
+mrlmoe_status mrlmoe_forward_train(const mrlmoe_config *cfg, const mrlmoe_weights *w,
+                                   const float *bias, const void *x, void *y,
+                                   mrlmoe_routing *route_out, void *workspace,
+                                   size_t ws_bytes, void *stream);
+
+/* Gradients of a loss L with respect to x and every learnable tensor, given
+ * dy = dL/dy [T, d_model] bf16, for the mrlmoe_forward_train call that last
+ * used `workspace` on `stream` with the same cfg, w and x.  Nothing is
+ * re-validated against that call: a different cfg, w or x gives wrong
+ * gradients.  The call continues the forward's status word (it does not
+ * clear it): if the forward failed, every backward kernel does nothing and
+ * the status stays the forward's.  cfg->hold applies to the backward's GEMMs
+ * (MRLMOE_HOLD_GEMM).  Enqueues about 14 kernels; allocates nothing.          */
+mrlmoe_status mrlmoe_backward(const mrlmoe_config *cfg, const mrlmoe_weights *w,
+                              const void *x, const void *dy, const mrlmoe_grads *grads,
+                              void *workspace, size_t ws_bytes, void *stream);
+
 /* Synchronises `stream`, then returns the device status word of `workspace`
  * written by the last call that used it (MRLMOE_OK if none failed).          */
 mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream);

@@ -130,8 +130,15 @@ def forward_for_grad(x: torch.Tensor, w: Dict[str, torch.Tensor], bias: torch.Te
 
 
 def backward(fc: ForwardCache, w: Dict[str, torch.Tensor], dy: torch.Tensor, top_k: int,
-             aggregation: str = "mean") -> Dict[str, torch.Tensor]:
-    """Gradients of sum(y * dy) for the names in GRAD_NAMES (fp64)."""
+             aggregation: str = "mean", experts=None) -> Dict[str, torch.Tensor]:
+    """Gradients of sum(y * dy) for the names in GRAD_NAMES (fp64).
+
+    ``experts`` (a list of routed expert indices) limits the routed experts'
+    weight gradients to those experts, stacked in that order (the full
+    tensors at full width do not fit a host's memory in fp64); every other
+    gradient is complete either way."""
+    sel = None if experts is None else [int(e) for e in experts]
+    slot_of = None if sel is None else {e: i for i, e in enumerate(sel)}
     dy = _f(dy)
     gain = _f(w["rms_gain"])
     alpha = _f(w["expert_scale"])
@@ -149,8 +156,9 @@ def backward(fc: ForwardCache, w: Dict[str, torch.Tensor], dy: torch.Tensor, top
     # c = sum_j ws_j o_j + o_shared
     dws = torch.zeros(T * top_k, dtype=F64)
     dz = torch.zeros(T, L, dtype=F64)
-    shapes = {"w_gate": (E,) + tuple(w["w_gate"].shape[1:]), "w_up_e": (E,) + tuple(w["w_up_e"].shape[1:]),
-              "w_down_e": (E,) + tuple(w["w_down_e"].shape[1:])}
+    ne = E if sel is None else len(sel)
+    shapes = {"w_gate": (ne,) + tuple(w["w_gate"].shape[1:]), "w_up_e": (ne,) + tuple(w["w_up_e"].shape[1:]),
+              "w_down_e": (ne,) + tuple(w["w_down_e"].shape[1:])}
     for nm, shp in shapes.items():
         grads[nm] = torch.zeros(shp, dtype=F64)
     for e, rows in fc.rows.items():
@@ -173,7 +181,9 @@ def backward(fc: ForwardCache, w: Dict[str, torch.Tensor], dy: torch.Tensor, top
         dwg, dwu = dg.T @ zr, du.T @ zr
         dz.index_add_(0, tok, dg @ wg + du @ wu)
         if e >= 0:
-            grads["w_gate"][e], grads["w_up_e"][e], grads["w_down_e"][e] = dwg, dwu, dwd
+            if slot_of is None or e in slot_of:
+                i = e if slot_of is None else slot_of[e]
+                grads["w_gate"][i], grads["w_up_e"][i], grads["w_down_e"][i] = dwg, dwu, dwd
         else:
             grads["w_sh_gate"], grads["w_sh_up"], grads["w_sh_down"] = dwg, dwu, dwd
     for nm in ("w_sh_gate", "w_sh_up", "w_sh_down"):

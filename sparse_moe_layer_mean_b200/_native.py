@@ -26,7 +26,8 @@ STATUS = {0: "MRLMOE_OK", 1: "MRLMOE_ERR_INVALID_ARG", 2: "MRLMOE_ERR_UNSUPPORTE
 EXPORTED = ("mrlmoe_workspace_size", "mrlmoe_route", "mrlmoe_forward", "mrlmoe_forward_timed",
             "mrlmoe_bias_update", "mrlmoe_linear", "mrlmoe_get_device_status",
             "mrlmoe_status_string", "mrlmoe_route_scores_static", "mrlmoe_quantize_e4m3",
-            "mrlmoe_check_routing", "mrlmoe_get_device_detail")
+            "mrlmoe_check_routing", "mrlmoe_get_device_detail", "mrlmoe_train_workspace_size",
+            "mrlmoe_forward_train", "mrlmoe_backward")
 STATIC_SCRATCH_BYTES = 2 * 1024 * 1024
 NUM_STAGE_EVENTS = 9
 STAGES = ("down_proj", "router_topk", "dispatch", "gather", "gate_up_glu", "expert_down",
@@ -68,6 +69,14 @@ class Routing(ctypes.Structure):
     _fields_ = [(n, c_void_p) for n in ROUTING_FIELDS]
 
 
+GRAD_FIELDS = ("dx", "d_w_down", "d_w_router", "d_w_gate", "d_w_up_e", "d_w_down_e", "d_w_sh_gate",
+               "d_w_sh_up", "d_w_sh_down", "d_rms_gain", "d_w_up", "d_expert_scale")
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in GRAD_FIELDS]
+
+
 _lib = None
 
 
@@ -107,6 +116,14 @@ def lib() -> ctypes.CDLL:
         L.mrlmoe_check_routing.argtypes = [POINTER(Config), POINTER(Routing), c_void_p, c_size_t, c_int,
                                            c_void_p]
         L.mrlmoe_check_routing.restype = c_int
+        L.mrlmoe_train_workspace_size.argtypes = [POINTER(Config)]
+        L.mrlmoe_train_workspace_size.restype = c_size_t
+        L.mrlmoe_forward_train.argtypes = [POINTER(Config), POINTER(Weights), c_void_p, c_void_p, c_void_p,
+                                           POINTER(Routing), c_void_p, c_size_t, c_void_p]
+        L.mrlmoe_forward_train.restype = c_int
+        L.mrlmoe_backward.argtypes = [POINTER(Config), POINTER(Weights), c_void_p, c_void_p, POINTER(Grads),
+                                      c_void_p, c_size_t, c_void_p]
+        L.mrlmoe_backward.restype = c_int
         L.mrlmoe_status_string.argtypes = [c_int]
         L.mrlmoe_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -197,6 +214,29 @@ def mrlmoe_forward_timed(cfg: Config, weights: Weights, bias, x, y, routing: Opt
                                       _ptr(y), rp, _ptr(workspace), int(ws_bytes),
                                       _stream_ptr(stream), arr, len(events)),
            "mrlmoe_forward_timed")
+
+
+def make_grads(g: Dict[str, object]) -> Grads:
+    return Grads(*[_ptr(g.get(n)) for n in GRAD_FIELDS])
+
+
+def mrlmoe_train_workspace_size(cfg: Config) -> int:
+    return int(lib().mrlmoe_train_workspace_size(ctypes.byref(cfg)))
+
+
+def mrlmoe_forward_train(cfg: Config, weights: Weights, bias, x, y, routing: Optional[Routing],
+                         workspace, ws_bytes: int, stream=None) -> None:
+    rp = ctypes.byref(routing) if routing is not None else None
+    _check(lib().mrlmoe_forward_train(ctypes.byref(cfg), ctypes.byref(weights), _ptr(bias), _ptr(x),
+                                      _ptr(y), rp, _ptr(workspace), int(ws_bytes), _stream_ptr(stream)),
+           "mrlmoe_forward_train")
+
+
+def mrlmoe_backward(cfg: Config, weights: Weights, x, dy, grads: Grads, workspace, ws_bytes: int,
+                    stream=None) -> None:
+    _check(lib().mrlmoe_backward(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(dy),
+                                 ctypes.byref(grads), _ptr(workspace), int(ws_bytes), _stream_ptr(stream)),
+           "mrlmoe_backward")
 
 
 def mrlmoe_bias_update(cfg: Config, counts, bias, gamma: float, stream=None) -> None:

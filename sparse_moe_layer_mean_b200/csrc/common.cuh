@@ -278,11 +278,34 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor: MN-major operand (the M or N index
+// contiguous) staged by SWIZZLE_128B TMA boxes of 64 elements x 64 K rows:
+// each box is 64 K rows of 128 bytes (8-row atoms of 1024 bytes), and the
+// tile's 64-wide M/N blocks follow one another `mn_stride` bytes apart.
+// Fields: leading byte offset = mn_stride (between 64-wide M/N blocks),
+// stride byte offset = 1024 (between 8-row K groups); a K step of 16 rows
+// advances the start address by 2048 bytes (whole atoms).
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t mn_stride) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
 // Instruction descriptor for kind::f16: D fp32 [4,6)=1, A bf16 [7,10)=1,
 // B bf16 [10,13)=1, both K-major, N>>3 at [17,23), M>>4 at [24,29).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// As idesc_bf16, with the operands' major-ness: bit 15 set = A MN-major,
+// bit 16 set = B MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_major(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16(M, N) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
 }
 
 // Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format 0), D fp32.

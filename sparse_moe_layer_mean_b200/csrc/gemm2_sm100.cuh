@@ -239,7 +239,8 @@ struct Glu2Policy {
     // h is K-blocked: the CTA's 64 d_ff columns are one plane, so the unit's
     // rows land in one contiguous N x 128 B range of it
     const int plane = U.m * 2 + static_cast<int>(rank);
-    __nv_bfloat16 *hp = p.h + static_cast<size_t>(plane) * p.rows * 64 + pair * 32 + lane;
+    const size_t hoff = static_cast<size_t>(plane) * p.rows * 64 + pair * 32 + lane;
+    __nv_bfloat16 *hp = p.h + hoff;
     const size_t row0 = static_cast<size_t>(U.row0);
     for (int c0 = 0; c0 < U.nv; c0 += 32) {
       float v[32];
@@ -255,7 +256,14 @@ struct Glu2Policy {
       for (int c = 0; c < 16; ++c) {
         const float g = is_gate ? v[c] : other[c];
         const float u = is_gate ? other[c] : v[16 + c];
-        if (cbase + c < U.nv) hp[(row0 + cbase + c) * 64] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
+        if (cbase + c < U.nv) {
+          const size_t o = (row0 + cbase + c) * 64;
+          hp[o] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
+          if (p.gs) {
+            p.gs[hoff + o] = __float2bfloat16_rn(g);
+            p.us[hoff + o] = __float2bfloat16_rn(u);
+          }
+        }
       }
       named_bar_sync(2, 128);
     }

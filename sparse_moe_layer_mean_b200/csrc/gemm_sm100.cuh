@@ -36,7 +36,54 @@ struct Unit {
   int nv;    // valid N columns in the unit
   int nsub;  // sub-tiles
   int row0;  // grouped GEMMs: first dispatched row of the unit
+  int krows; // ragged-K policies: rows of the unit's reduction
 };
+
+// Operand major-ness of a policy: P::kAMN / P::kBMN (true = the M or N index
+// is contiguous in memory, staged as 64-wide MN blocks of P::kAMNStride /
+// P::kBMNStride bytes); policies without them are K-major on both sides.
+template <class P, class = void>
+struct OperandMajor {
+  static constexpr bool a_mn = false, b_mn = false;
+  static constexpr uint32_t a_stride = 0, b_stride = 0;
+};
+template <class P>
+struct OperandMajor<P, decltype(void(P::kAMN))> {
+  static constexpr bool a_mn = P::kAMN, b_mn = P::kBMN;
+  static constexpr uint32_t a_stride = P::kAMNStride, b_stride = P::kBMNStride;
+};
+
+// Ragged K (P::kRaggedK): each unit has its own number of K blocks,
+// P::unit_k_blocks(p, U) (possibly 0), and only the first
+// P::tail_rows(p, U) rows of its last K block belong to it; the MMA warp
+// zeroes the rest of that block's tiles in shared memory (P::zero_tail)
+// before the MMAs read it.  A unit with no K blocks leaves a zero tile
+// (P::epilogue is told through U and writes zeros without reading TMEM).
+template <class P, class = void>
+struct RaggedK {
+  static constexpr bool on = false;
+};
+template <class P>
+struct RaggedK<P, decltype(void(P::kRaggedK))> {
+  static constexpr bool on = P::kRaggedK;
+};
+
+template <class P>
+__device__ __forceinline__ int unit_k_blocks(const typename P::Params &p, const Unit &U, int kblocks) {
+  if constexpr (RaggedK<P>::on)
+    return P::unit_k_blocks(p, U);
+  else
+    return kblocks;
+}
+
+// Descriptor of the kk-th 16-deep K step of an operand tile at `base`.
+template <bool MN, uint32_t STRIDE, int UMMA_K_BYTES>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
+  if constexpr (MN)
+    return sdesc_mn_sw128(base + kk * 2048, STRIDE);
+  else
+    return sdesc_sw128(base + kk * UMMA_K_BYTES);
+}
 
 __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
   uint32_t r;
@@ -131,7 +178,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const Unit U = P::unit(p, u, aux);
         for (int sub = 0; sub < U.nsub; ++sub) {
           const uint32_t bytes = isA ? P::kABytes : P::b_bytes(p, U, sub);
-          for (int kb = 0; kb < kblocks; ++kb) {
+          const int kbu = unit_k_blocks<P>(p, U, kblocks);
+          for (int kb = 0; kb < kbu; ++kb) {
             if (s % G == 0 && !mbar_wait(empty0 + 8 * (s / G), ph ^ 1, abort_flag, status)) goto done;
             mbar_arrive_expect_tx(full0 + 8 * s, bytes);
             const uint32_t st = ring + s * L::kStageBytes;
@@ -145,6 +193,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       }
     }
   } else if (warp == 1) {
+   if constexpr (RaggedK<P>::on) {
+    // the whole warp walks the ring (it zeroes the ragged tails); lane 0 issues
+    int s = 0, acc = 0;
+    uint32_t ph = 0, aph = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const Unit U = P::unit(p, u, aux);
+      const int kbu = unit_k_blocks<P>(p, U, kblocks);
+      if (!__all_sync(0xffffffffu, mbar_wait(acce0 + 8 * acc, aph ^ 1, abort_flag, status))) goto done;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + acc * kAccCols;
+      const uint32_t idesc = P::idesc(p, U, 0);
+      for (int kb = 0; kb < kbu; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(full0 + 8 * s, ph, abort_flag, status))) goto done;
+        tc_fence_after();
+        const uint32_t a_s = ring + s * L::kStageBytes;
+        const uint32_t b_s = a_s + P::kABytes;
+        if (kb == kbu - 1) {
+          const int tail = P::tail_rows(p, U);
+          if (tail < kBK) {
+            P::zero_tail(p, U, smem + (a_s - ring), smem + (b_s - ring), tail, lane);
+            fence_proxy_async_shared();  // the zeros are read by the tensor core (async proxy)
+          }
+          __syncwarp();
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < kBK * 2 / P::kUmmaKBytes; ++kk)
+            P::mma(tacc, operand_desc<OperandMajor<P>::a_mn, OperandMajor<P>::a_stride, P::kUmmaKBytes>(a_s, kk),
+                   operand_desc<OperandMajor<P>::b_mn, OperandMajor<P>::b_stride, P::kUmmaKBytes>(b_s, kk), idesc,
+                   (kb | kk) != 0);
+          if (s % G == G - 1) umma_commit(empty0 + 8 * (s / G));
+        }
+        __syncwarp();
+        if (++s == S) { s = 0; ph ^= 1; }
+      }
+      if (lane == 0) {
+        if (kbu > 0)
+          umma_commit(accf0 + 8 * acc);
+        else
+          mbar_arrive(accf0 + 8 * acc);  // nothing to wait for: the epilogue writes a zero tile
+      }
+      __syncwarp();
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+   } else {
     if (lane == 0) {
       int s = 0, acc = 0;
       uint32_t ph = 0, aph = 0;
@@ -165,8 +259,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             for (int as = 0; as < P::kASub; ++as)
 #pragma unroll
               for (int kk = 0; kk < kBK * 2 / P::kUmmaKBytes; ++kk)
-                P::mma(tacc, sdesc_sw128(a_s + as * P::kASubBytes + kk * P::kUmmaKBytes),
-                       sdesc_sw128(b_s + kk * P::kUmmaKBytes), idesc, (kb | kk | as) != 0);
+                P::mma(tacc,
+                       operand_desc<OperandMajor<P>::a_mn, OperandMajor<P>::a_stride, P::kUmmaKBytes>(
+                           a_s + as * P::kASubBytes, kk),
+                       operand_desc<OperandMajor<P>::b_mn, OperandMajor<P>::b_stride, P::kUmmaKBytes>(b_s, kk),
+                       idesc, (kb | kk | as) != 0);
             if (s % G == G - 1) umma_commit(empty0 + 8 * (s / G));
             if (++s == S) { s = 0; ph ^= 1; }
           }
@@ -176,6 +273,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         }
       }
     }
+   }
   } else {
     // epilogue warps 2..5; TMEM lane quarter = warp % 4
     const int q = warp & 3;

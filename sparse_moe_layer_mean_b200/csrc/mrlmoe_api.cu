@@ -13,6 +13,7 @@
 #include "gemm8_sm100.cuh"
 #include "routing.cuh"
 #include "check.cuh"
+#include "backward.cuh"
 
 using namespace mrl;
 
@@ -90,9 +91,16 @@ int router_ksplit(const mrlmoe_config &c) {
 struct Layout {
   size_t status, topk_idx, topk_w, wscaled, counts, offsets, grp_off, grp_cnt, unit1, unit2, perm, inv, mask,
       base, cand_v, cand_s, cand_i, rpart, zbuf, zlo, hbuf, slots, nbuf, xq, xs, zq, zs, hq, hs, nq, ns, total;
+  // training forward + backward (bf16): kept pre-activations and the backward's buffers
+  size_t gsave, usave, dn, dcd, dod, dgu, dwsp, dzx, dl, aw, gpart, bgrp_off, bgrp_cnt, bunit1, bunit2;
 };
 
-Layout layout_of(const mrlmoe_config &c) {
+// Blocks of rms_combine_bwd_kernel (a fixed number, so the gain gradient's
+// summation order depends on the config alone).
+constexpr int kRmsBwdBlocks = 296;
+int rms_bwd_blocks(const mrlmoe_config &c) { return std::min(c.T, kRmsBwdBlocks); }
+
+Layout layout_of(const mrlmoe_config &c, bool train = false) {
   Layout L{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -137,6 +145,24 @@ Layout layout_of(const mrlmoe_config &c) {
     L.hs = take((Tk + T) * (F / 128) * 4);
     L.nq = take(T * Ld);
     L.ns = take(T * (Ld / 128) * 4);
+  }
+  if (train) {
+    const size_t rows = Tk + T;
+    L.gsave = take(rows * F * 2);
+    L.usave = take(rows * F * 2);
+    L.dn = take(T * Ld * 4);
+    L.dcd = take(rows * Ld * 2);
+    L.dod = take(rows * Ld * 2);
+    L.dgu = take(rows * 2 * F * 2);
+    L.dwsp = take((F / 128) * Tk * 4);
+    L.dzx = take(T * Ld * 2);
+    L.dl = take(Tk * c.n_routers * 4);
+    L.aw = take(Tk * 4);
+    L.gpart = take(static_cast<size_t>(rms_bwd_blocks(c)) * Ld * 4);
+    L.bgrp_off = take((E + 2) * 4);
+    L.bgrp_cnt = take((E + 2) * 4);
+    L.bunit1 = take((E + 2) * 4);
+    L.bunit2 = take((E + 2) * 4);
   }
   L.total = off;
   return L;
@@ -554,19 +580,28 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
 
 mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, const float *bias, const void *x,
                            void *y, mrlmoe_routing *route_out, void *workspace, size_t ws_bytes, void *stream,
-                           void *const *ev) {
+                           void *const *ev, bool train = false) {
   mrlmoe_status s = check_config(cfg);
   if (s != MRLMOE_OK) return s;
+  if (train && (cfg->dtype != MRLMOE_BF16 || cfg->d_ff > 128 * kBwdMaxSlices)) return MRLMOE_ERR_UNSUPPORTED;
   if (!bias || !x || !y || !aligned16(x) || !aligned16(y)) return MRLMOE_ERR_INVALID_ARG;
   const bool fp8 = cfg->dtype != MRLMOE_BF16;  // e4m3 projections and activations (FP8 and FP4 variants)
   if ((s = fp8 ? check_weights_fp8(w) : check_weights_bf16(w, true)) != MRLMOE_OK) return s;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
-  if (ws_bytes < layout_of(*cfg).total) return MRLMOE_ERR_WORKSPACE;
+  if (ws_bytes < layout_of(*cfg, train).total) return MRLMOE_ERR_WORKSPACE;
   int sms = 0;
   if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Ptrs P = carve(*cfg, workspace, route_out);
+  // the training forward keeps the routing record in the workspace (the
+  // backward reads it there) and copies it to route_out afterwards
+  Ptrs P = carve(*cfg, workspace, train ? nullptr : route_out);
+  if (train && route_out) {
+    P.scores = route_out->scores;
+    P.out_counts = route_out->counts;
+    P.out_offsets = route_out->offsets;
+  }
   const int T = cfg->T, D = cfg->d_model, Ld = cfg->d_lat, F = cfg->d_ff, E = cfg->n_experts, k = cfg->top_k;
+  const Layout LT = layout_of(*cfg, train);
   const int Tk = T * k;
   if ((s = init_header(P.status, cfg->hold, st)) != MRLMOE_OK) return s;
   auto mark = [&](int i) -> bool {
@@ -577,6 +612,13 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   if ((s = launch_project_and_route(*cfg, w, bias, x, P, sms, st, ev)) != MRLMOE_OK) return s;
   if (!mark(2)) return MRLMOE_ERR_CUDA;
   if ((s = launch_dispatch(*cfg, P, st)) != MRLMOE_OK) return s;
+  if (train && route_out) {
+    const size_t n = static_cast<size_t>(T) * k * 4;
+    if (route_out->topk_idx) MRL_TRY(cudaMemcpyAsync(route_out->topk_idx, P.topk_idx, n, cudaMemcpyDeviceToDevice, st));
+    if (route_out->topk_w) MRL_TRY(cudaMemcpyAsync(route_out->topk_w, P.topk_w, n, cudaMemcpyDeviceToDevice, st));
+    if (route_out->perm) MRL_TRY(cudaMemcpyAsync(route_out->perm, P.perm, n, cudaMemcpyDeviceToDevice, st));
+    if (route_out->inv_perm) MRL_TRY(cudaMemcpyAsync(route_out->inv_perm, P.inv, n, cudaMemcpyDeviceToDevice, st));
+  }
   if (!mark(3)) return MRLMOE_ERR_CUDA;
   if (fp8) {
     if ((s = forward_experts_fp8(*cfg, w, P, sms, st, ev, y)) != MRLMOE_OK) return s;
@@ -604,6 +646,10 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
       return MRLMOE_ERR_CUDA;
     p.gt = gt1;
     p.h = P.hbuf;
+    if (train) {
+      p.gs = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(workspace) + LT.gsave);
+      p.us = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(workspace) + LT.usave);
+    }
     p.F = F; p.L = Ld; p.rows = Tk + T;
     p.status = P.status;
     MRL_TRY(launch_gemm_pair<Glu2Policy>(p, sms, st));
@@ -706,6 +752,149 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
   if (!mark(7)) return MRLMOE_ERR_CUDA;
   return launch_dense8(P.nq, P.ns, w->w_up, w->s_up, T, D, Ld, static_cast<__nv_bfloat16 *>(y_out), nullptr, P, sms,
                        st);
+}
+
+// ------------------------------------------------------------ backward
+template <class DP>
+mrlmoe_status launch_dense_grad(const CUtensorMap &ta, const CUtensorMap &tb, void *out, int M, int N, int K,
+                                uint32_t *status, int sms, cudaStream_t st) {
+  typename DP::Params p{};
+  p.ta = ta;
+  p.tb = tb;
+  p.out = out;
+  p.ldo = N;
+  p.M = M; p.N = N; p.K = K;
+  p.m_tiles = (M + 127) / 128;
+  p.n_tiles = (N + DP::kBN - 1) / DP::kBN;
+  p.status = status;
+  MRL_TRY(launch_gemm<DP>(p, std::min(sms, p.m_tiles * p.n_tiles), st));
+  return MRLMOE_OK;
+}
+
+mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, const void *x, const void *dy,
+                            const mrlmoe_grads *g, void *workspace, size_t ws_bytes, void *stream) {
+  mrlmoe_status s = check_config(cfg);
+  if (s != MRLMOE_OK) return s;
+  if (cfg->dtype != MRLMOE_BF16 || cfg->d_ff > 128 * kBwdMaxSlices) return MRLMOE_ERR_UNSUPPORTED;
+  if (!x || !dy || !g || !aligned16(x) || !aligned16(dy)) return MRLMOE_ERR_INVALID_ARG;
+  if ((s = check_weights_bf16(w, true)) != MRLMOE_OK) return s;
+  {
+    const void *outs[] = {g->dx, g->d_w_down, g->d_w_router, g->d_w_gate, g->d_w_up_e, g->d_w_down_e,
+                          g->d_w_sh_gate, g->d_w_sh_up, g->d_w_sh_down, g->d_rms_gain, g->d_w_up, g->d_expert_scale};
+    for (const void *o : outs)
+      if (!o || !aligned16(o)) return MRLMOE_ERR_INVALID_ARG;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
+  const Layout LT = layout_of(*cfg, true);
+  if (ws_bytes < LT.total) return MRLMOE_ERR_WORKSPACE;
+  int sms = 0;
+  if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ptrs P = carve(*cfg, workspace, nullptr);
+  uint8_t *b = static_cast<uint8_t *>(workspace);
+  const int T = cfg->T, D = cfg->d_model, Ld = cfg->d_lat, F = cfg->d_ff, E = cfg->n_experts, k = cfg->top_k;
+  const int R = cfg->n_routers, Tk = T * k, rows = Tk + T;
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16 *>(b + off); };
+  auto f32 = [&](size_t off) { return reinterpret_cast<float *>(b + off); };
+  auto i32 = [&](size_t off) { return reinterpret_cast<int32_t *>(b + off); };
+  __nv_bfloat16 *gsave = bf(LT.gsave), *usave = bf(LT.usave), *dcd = bf(LT.dcd), *dod = bf(LT.dod);
+  __nv_bfloat16 *dgu = bf(LT.dgu), *dzx = bf(LT.dzx);
+  float *dn = f32(LT.dn), *dwsp = f32(LT.dwsp), *dl = f32(LT.dl), *aw = f32(LT.aw), *gpart = f32(LT.gpart);
+  const __nv_bfloat16 *zhi = P.zbuf + static_cast<size_t>(Tk) * Ld;
+  // the call continues the forward's status word; only this call's hold mask is set
+  MRL_TRY(cudaMemsetAsync(reinterpret_cast<uint8_t *>(P.status) + 4, static_cast<int>(cfg->hold & 0xffu), 1, st));
+
+  // dn = dy W_up (W_up [D, Ld] MN-major); dW_up = dy^T n (both MN-major, K = T)
+  {
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, dy, 2, D, T, 128) || !make_map(&tb, w->w_up, 2, Ld, D, 64)) return MRLMOE_ERR_CUDA;
+    if ((s = launch_dense_grad<DenseGradPolicy<false, true, true>>(ta, tb, dn, T, Ld, D, P.status, sms, st)) !=
+        MRLMOE_OK)
+      return s;
+    if (!make_map(&ta, dy, 2, D, T, 64) || !make_map(&tb, P.nbuf, 2, Ld, T, 64)) return MRLMOE_ERR_CUDA;
+    if ((s = launch_dense_grad<DenseGradPolicy<true, true, true>>(ta, tb, g->d_w_up, D, Ld, T, P.status, sms, st)) !=
+        MRLMOE_OK)
+      return s;
+  }
+  // RMSNorm + combine backward: dc rows (plain and weighted) per dispatch row
+  const int nb = rms_bwd_blocks(*cfg);
+  rms_combine_bwd_kernel<<<nb, kBwdThreads, 0, st>>>(
+      reinterpret_cast<const float4 *>(P.slots), reinterpret_cast<const float4 *>(dn),
+      reinterpret_cast<const float4 *>(w->rms_gain), P.inv, P.wscaled, T, Ld, k, cfg->rms_eps, dcd, dod,
+      reinterpret_cast<float4 *>(gpart), P.status);
+  MRL_TRY(cudaGetLastError());
+  gain_reduce_kernel<<<(Ld + 255) / 256, 256, 0, st>>>(gpart, nb, Ld, g->d_rms_gain, P.status);
+  MRL_TRY(cudaGetLastError());
+  // unit tables of the two grouped dgrad GEMMs (token tiles of 256; d_ff / 128 and d_lat / 128 M tiles)
+  int32_t *bgo = i32(LT.bgrp_off), *bgc = i32(LT.bgrp_cnt), *bu1 = i32(LT.bunit1), *bu2 = i32(LT.bunit2);
+  expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, DhPolicy::kBN, F / 128, Ld / 128, bgo, bgc, bu1,
+                                            bu2, nullptr, nullptr, P.status);
+  MRL_TRY(cudaGetLastError());
+  {
+    DhPolicy::Params p{};
+    if (!make_map(&p.wd, w->w_down_e, 2, F, static_cast<uint64_t>(E) * Ld, 64) ||
+        !make_map(&p.sd, w->w_sh_down, 2, F, Ld, 64) || !make_token_maps(&p.tc, dcd, Ld, rows))
+      return MRLMOE_ERR_CUDA;
+    p.gt = GroupTable{bgo, bgc, bu1, E, F / 128};
+    p.perm = P.perm;
+    p.wscaled = P.wscaled;
+    p.g = gsave; p.u = usave; p.h = P.hbuf;
+    p.dgu = dgu;
+    p.dwsp = dwsp;
+    p.L = Ld; p.F = F; p.Tk = Tk; p.rows = rows;
+    p.status = P.status;
+    MRL_TRY(launch_gemm<DhPolicy>(p, sms, st));
+  }
+  {
+    DzPolicy::Params p{};
+    if (!make_map(&p.wg, w->w_gate, 2, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !make_map(&p.wu, w->w_up_e, 2, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !make_map(&p.sg, w->w_sh_gate, 2, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 2, Ld, F, 64) ||
+        !make_token_maps_blocked(&p.tgu, dgu, 2 * F, rows))
+      return MRLMOE_ERR_CUDA;
+    p.gt = GroupTable{bgo, bgc, bu2, E, Ld / 128};
+    p.perm = P.perm;
+    p.dzs = P.slots;  // the forward's slots were consumed by rms_combine_bwd_kernel
+    p.L = Ld; p.F = F; p.k = k; p.Tk = Tk;
+    p.status = P.status;
+    MRL_TRY(launch_gemm<DzPolicy>(p, sms, st));
+  }
+  // routers, combine weights, alpha; dz reduced per token
+  token_bwd_kernel<<<T, kBwdThreads, Ld * sizeof(float), st>>>(
+      dwsp, F / 128, P.topk_idx, P.topk_w, w->expert_scale, zhi, P.zlo,
+      static_cast<const __nv_bfloat16 *>(w->w_router), P.slots, T, Ld, E, R, k, static_cast<int>(cfg->aggregation),
+      dzx, dl, aw, P.status);
+  MRL_TRY(cudaGetLastError());
+  expert_param_bwd_kernel<<<E, kBwdThreads, 0, st>>>(P.grp_off, P.grp_cnt, P.perm, dl, aw, zhi, P.zlo, Ld, E, R, k,
+                                                     g->d_w_router, g->d_expert_scale, P.status);
+  MRL_TRY(cudaGetLastError());
+  // expert weight gradients (K = each group's rows)
+  {
+    WgradPolicy::Params p{};
+    if (!make_map(&p.tdgu, dgu, 2, 64, static_cast<uint64_t>(2 * F / 64) * rows, 64) ||
+        !make_map(&p.tz, P.zbuf, 2, Ld, rows, 64) || !make_map(&p.tdo, dod, 2, Ld, rows, 64) ||
+        !make_map(&p.th, P.hbuf, 2, 64, static_cast<uint64_t>(F / 64) * rows, 64))
+      return MRLMOE_ERR_CUDA;
+    p.grp_off = P.grp_off;
+    p.dwg = g->d_w_gate; p.dwu = g->d_w_up_e; p.dwd = g->d_w_down_e;
+    p.dsg = g->d_w_sh_gate; p.dsu = g->d_w_sh_up; p.dsd = g->d_w_sh_down;
+    p.E = E; p.F = F; p.L = Ld; p.rows = rows;
+    p.status = P.status;
+    MRL_TRY(launch_gemm<WgradPolicy>(p, sms, st));
+  }
+  // dx = dzx W_dn (W_dn [Ld, D] MN-major); dW_dn = dzx^T x (K = T)
+  {
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, dzx, 2, Ld, T, 128) || !make_map(&tb, w->w_down, 2, D, Ld, 64)) return MRLMOE_ERR_CUDA;
+    if ((s = launch_dense_grad<DenseGradPolicy<false, true, false>>(ta, tb, g->dx, T, D, Ld, P.status, sms, st)) !=
+        MRLMOE_OK)
+      return s;
+    if (!make_map(&ta, dzx, 2, Ld, T, 64) || !make_map(&tb, x, 2, D, T, 64)) return MRLMOE_ERR_CUDA;
+    if ((s = launch_dense_grad<DenseGradPolicy<true, true, true>>(ta, tb, g->d_w_down, Ld, D, T, P.status, sms,
+                                                                    st)) != MRLMOE_OK)
+      return s;
+  }
+  return MRLMOE_OK;
 }
 
 // ------------------------------------------------ static-scratch routing
@@ -821,6 +1010,22 @@ mrlmoe_status mrlmoe_forward_timed(const mrlmoe_config *cfg, const mrlmoe_weight
   for (int i = 0; i < n_events; ++i)
     if (!events[i]) return MRLMOE_ERR_INVALID_ARG;
   return forward_impl(cfg, w, bias, x, y, route_out, workspace, ws_bytes, stream, events);
+}
+
+size_t mrlmoe_train_workspace_size(const mrlmoe_config *cfg) {
+  if (check_config(cfg) != MRLMOE_OK || cfg->dtype != MRLMOE_BF16 || cfg->d_ff > 128 * kBwdMaxSlices) return 0;
+  return layout_of(*cfg, true).total;
+}
+
+mrlmoe_status mrlmoe_forward_train(const mrlmoe_config *cfg, const mrlmoe_weights *w, const float *bias,
+                                   const void *x, void *y, mrlmoe_routing *route_out, void *workspace,
+                                   size_t ws_bytes, void *stream) {
+  return forward_impl(cfg, w, bias, x, y, route_out, workspace, ws_bytes, stream, nullptr, true);
+}
+
+mrlmoe_status mrlmoe_backward(const mrlmoe_config *cfg, const mrlmoe_weights *w, const void *x, const void *dy,
+                              const mrlmoe_grads *grads, void *workspace, size_t ws_bytes, void *stream) {
+  return backward_impl(cfg, w, x, dy, grads, workspace, ws_bytes, stream);
 }
 
 mrlmoe_status mrlmoe_bias_update(const mrlmoe_config *cfg, const int32_t *counts, float *bias, float gamma,

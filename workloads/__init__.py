@@ -221,7 +221,7 @@ def _perm(n: int, seed: int, stream: int, device) -> torch.Tensor:
 
 # Stream ids, one per tensor.
 _S_X, _S_WDN, _S_WR, _S_WG, _S_WU, _S_WD, _S_SG, _S_SU, _S_SD, _S_WUP, _S_ALPHA, \
-    _S_ZIPF_PERM, _S_OUTLIER = range(1, 14)
+    _S_ZIPF_PERM, _S_OUTLIER, _S_DY, _S_GAIN = range(1, 16)
 
 
 def make_weights(s: LayerShape, device, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
@@ -363,6 +363,21 @@ def make_x(s: LayerShape, device, seed: Optional[int] = None, T: Optional[int] =
     # window: generate the covering range and slice (elements are position-addressed)
     full = normal(((token0 + T), s.d_model), seed, _S_X, device, col_scale=col_scale)
     return full[token0:].contiguous()
+
+
+def make_dy(s: LayerShape, device, seed: Optional[int] = None, T: Optional[int] = None) -> torch.Tensor:
+    """Incoming gradient of the layer output for the backward pass: dy ~ N(0,1)
+    [T, d_model] bf16 (a loss with unit-variance output gradients)."""
+    seed = s.seed if seed is None else seed
+    T = s.T if T is None else T
+    return normal((T, s.d_model), seed, _S_DY, device)
+
+
+def make_train_gain(s: LayerShape, device, seed: Optional[int] = None) -> torch.Tensor:
+    """A trained-looking RMSNorm gain for the backward tests: 1 + 0.1 N(0,1)
+    (fp32), so that a gain dropped or misplaced in a gradient shows."""
+    seed = s.seed if seed is None else seed
+    return 1.0 + 0.1 * normal((s.d_lat,), seed, _S_GAIN, device, dtype=torch.float32)
 
 
 def zipf_ln_ratio(s: LayerShape, device, seed: Optional[int] = None) -> torch.Tensor:
