@@ -72,6 +72,8 @@ def parse_args():
     ap.add_argument("--aggregation", choices=["mean", "sum", "max"], default=None,
                     help="router score aggregation (default: the config's, the mean)")
     ap.add_argument("--routers", type=int, default=None, help="override the number of routers R")
+    ap.add_argument("--train", action="store_true",
+                    help="time a training step (forward that keeps its activations + backward) instead")
     ap.add_argument("--route-only", action="store_true",
                     help="time routing from x alone (down-projection, routers, top-k, dispatch: "
                          "mrlmoe_route) and print its own JSON line; bf16 configs")
@@ -359,12 +361,163 @@ def run_route_only(args):
           flush=True)
 
 
+TRAIN_METRIC = "MoE-layer training step (fwd + bwd) tokens/s on 1 B200 (full width); % of roofline"
+BACKWARD_KERNELS = 12          # launches of this library's kernels per backward
+
+
+def wgrad_kernel_bytes(s):
+    """Algorithmic bytes of the expert weight-gradient launch: the fp32
+    gradients of gate, up and down for every routed expert and the shared
+    one written once, and its operands (dg, du, z, do, h rows) read once."""
+    rows = s.T * s.top_k + s.T
+    return 3 * (s.n_experts + 1) * s.d_ff * s.d_lat * 4 + rows * (3 * s.d_ff + 2 * s.d_lat) * 2
+
+
+def train_flops(s):
+    """FLOPs of one training step: the forward plus twice its GEMM FLOPs
+    (dgrad and wgrad of every GEMM)."""
+    import workloads as W
+    return 3 * W.flops_per_token(s) * s.T
+
+
+def run_train(args):
+    """--train: one step = mrlmoe_forward_train + mrlmoe_backward over one batch
+    (fp32 weight gradients of every expert, bf16 dx)."""
+    import torch
+    import sparse_moe_layer_mean_b200 as M
+    import workloads as W
+    world, rank, local = dist_setup()
+    if world > 1:
+        raise SystemExit("--train runs on one GPU")
+    s = shape_from_args(args)
+    if s.fp8:
+        raise SystemExit("--train runs the bf16 configs")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    weights = W.make_layer_weights(s, dev)
+    weights["rms_gain"] = W.make_train_gain(s, dev)
+    x = W.make_x(s, dev)
+    bias = W.make_bias(s, dev)
+    dy = W.make_dy(s, dev)
+    layer = M.MRLMoELayer(s, weights, device=dev, train=True)
+    y = torch.empty(s.T, s.d_model, dtype=torch.bfloat16, device=dev)
+    grads = M.grad_buffers(layer.cfg, dev)
+    cg = M.make_grads(grads)
+    for _ in range(max(3, args.warmup)):
+        layer.forward_train(x, bias, y=y)
+        M.mrlmoe_backward(layer.cfg, layer.cw, x, dy, cg, layer.workspace, layer.ws_bytes)
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status non-zero after warm-up")
+    NB = M._native.NUM_BACKWARD_EVENTS
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NB + 1)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    time.sleep(0.6)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.begin()
+    start.record()
+    for i in range(args.steps):
+        evs[i][0].record()
+        layer.forward_train(x, bias, y=y)
+        M.mrlmoe_backward_timed(layer.cfg, layer.cw, x, dy, cg, layer.workspace, layer.ws_bytes, evs[i][1:])
+    stop.record()
+    torch.cuda.synchronize()
+    clocks.end()
+    clk = clocks.stop()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status non-zero after the timed region")
+    ms = start.elapsed_time(stop)
+    fwd_ms = sum(r[0].elapsed_time(r[1]) for r in evs) / args.steps
+    stage = [sum(r[j + 1].elapsed_time(r[j + 2]) for r in evs) / args.steps for j in range(NB - 1)]
+    bwd_ms = sum(stage)
+
+    # e2e: x and dy from pinned host memory, the step, dx back to pinned host memory, every step
+    e2e = None
+    if not args.no_e2e:
+        xh, dyh = x.cpu().pin_memory(), dy.cpu().pin_memory()
+        dxh = torch.empty_like(grads["dx"], device="cpu").pin_memory()
+        xd, dyd = torch.empty_like(x), torch.empty_like(dy)
+
+        def e2e_run(n):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(n):
+                xd.copy_(xh, non_blocking=True)
+                dyd.copy_(dyh, non_blocking=True)
+                layer.forward_train(xd, bias, y=y)
+                M.mrlmoe_backward(layer.cfg, layer.cw, xd, dyd, cg, layer.workspace, layer.ws_bytes)
+                dxh.copy_(grads["dx"], non_blocking=True)
+            b.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(b)
+
+        e2e_run(2)
+        e2e_ms = e2e_run(args.steps)
+        e2e = {"value": s.T * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": 2 * x.numel() * x.element_size(),
+               "d2h_bytes_per_step": grads["dx"].numel() * grads["dx"].element_size()}
+
+    peaks, peak_kind = load_peaks()
+    wg_ms = stage[M._native.BACKWARD_STAGES.index("expert_wgrad")]
+    wg_bytes = wgrad_kernel_bytes(s)
+    flops = train_flops(s)
+    line = {
+        "metric": TRAIN_METRIC, "value": s.T * args.steps / (ms * 1e-3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{s.name} training step: T={s.T} tokens, d_model {s.d_model} -> d_lat {s.d_lat}, "
+                               f"{s.n_experts} experts top-{s.top_k} + 1 shared, d_ff {s.d_ff}, "
+                               f"R={s.n_routers} routers, bf16 operands, fp32 weight gradients",
+                   "T": s.T, "l2": "inputs larger than L2 (expert weights and gradients streamed every step)",
+                   "forward_train_ms": round(fwd_ms, 4), "backward_ms": round(bwd_ms, 4),
+                   "backward_stage_ms": dict(zip(M._native.BACKWARD_STAGES, [round(v, 4) for v in stage])),
+                   "step_tensor_frac_of_bf16_peak": flops / (ms / args.steps * 1e-3) / (peaks["bf16_tflops"] * 1e12)},
+        "roofline": {"kernel": "expert_wgrad (grouped tcgen05 GEMM over ragged token K, fp32 gradients)",
+                     "bound": "hbm", "achieved": wg_bytes / (wg_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": wg_bytes / (wg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "traffic": None, "algorithmic_bytes": wg_bytes, "peak_kind": f"of {peak_kind}"},
+        "clocks": clk,
+        "gpu_launches": (kernels_per_step(s, torch.cuda.get_device_properties(dev).multi_processor_count)
+                         + BACKWARD_KERNELS) * args.steps,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_train(s, weights, x, bias, dy, min(args.cpu_sample, 4))
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_train(s, weights_dev, x_dev, bias_dev, dy_dev, ntok):
+    """The oracle's forward + backward, as they stand, on the first ntok
+    tokens (the routed experts' weight gradients for the experts those
+    tokens select; the others are zero)."""
+    import torch
+    from oracle import mrlmoe_backward as OB
+    wh = {k: v.cpu() for k, v in weights_dev.items()}
+    t0 = time.perf_counter()
+    fc = OB.forward_for_grad(x_dev[:ntok].cpu(), wh, bias_dev.cpu(), s.top_k, rms_eps=s.rms_eps,
+                             aggregation=s.aggregation)
+    used = torch.unique(fc.idx).tolist()
+    OB.backward(fc, wh, dy_dev[:ntok].cpu(), s.top_k, aggregation=s.aggregation, experts=used)
+    dt = time.perf_counter() - t0
+    return {"value": ntok / dt, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": f"first {ntok} tokens of the {s.name} batch, forward + backward (fp64 oracle, {dt:.1f} s)"}
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.route_only:
         return run_route_only(args)
+    if args.train:
+        return run_train(args)
     world, rank, local = dist_setup()
     import torch
     import torch.distributed as dist

@@ -299,6 +299,21 @@ mrlmoe_status mrlmoe_backward(const mrlmoe_config *cfg, const mrlmoe_weights *w,
                               const void *x, const void *dy, const mrlmoe_grads *grads,
                               void *workspace, size_t ws_bytes, void *stream);
 
+/* Same as mrlmoe_backward, and records caller-created CUDA events on `stream`
+ * at its stage boundaries (as mrlmoe_forward_timed does):
+ *   events[0]  before the first kernel     events[6]  after the router/token backward
+ *   events[1]  after dn = dy W_up          events[7]  after dW_router and dalpha
+ *   events[2]  after dW_up                 events[8]  after the expert weight gradients
+ *   events[3]  after RMSNorm/combine bwd   events[9]  after dx
+ *   events[4]  after dh (W_down dgrad)     events[10] after dW_down
+ *   events[5]  after dz (W_gate/W_up dgrad)
+ * n_events must be MRLMOE_NUM_BACKWARD_EVENTS.                               */
+#define MRLMOE_NUM_BACKWARD_EVENTS 11
+mrlmoe_status mrlmoe_backward_timed(const mrlmoe_config *cfg, const mrlmoe_weights *w,
+                                    const void *x, const void *dy, const mrlmoe_grads *grads,
+                                    void *workspace, size_t ws_bytes, void *stream,
+                                    void *const *events, int n_events);
+
 /* Synchronises `stream`, then returns the device status word of `workspace`
  * written by the last call that used it (MRLMOE_OK if none failed).          */
 mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream);

@@ -21,7 +21,7 @@ from ._native import (MRLMOE_BF16, MRLMOE_FP8_E4M3_BLOCK128, MRLMOE_FP4_E2M1_BLO
                       mrlmoe_route_scores_static, mrlmoe_quantize_e4m3, mrlmoe_check_routing,
                       mrlmoe_get_device_detail, mrlmoe_workspace_size, status_string, HOLD, CHECK_BITS,
                       Grads, GRAD_FIELDS, make_grads, mrlmoe_train_workspace_size, mrlmoe_forward_train,
-                      mrlmoe_backward)
+                      mrlmoe_backward, mrlmoe_backward_timed)
 
 __all__ = ["MRLMoELayer", "Config", "Weights", "Routing", "MrlmoeError", "make_config",
            "make_weights", "make_routing", "mrlmoe_route", "mrlmoe_forward", "mrlmoe_forward_timed",
@@ -30,7 +30,7 @@ __all__ = ["MRLMoELayer", "Config", "Weights", "Routing", "MrlmoeError", "make_c
            "mrlmoe_check_routing", "mrlmoe_get_device_detail", "status_string", "MRLMOE_BF16",
            "MRLMOE_FP8_E4M3_BLOCK128", "MRLMOE_FP4_E2M1_BLOCK128", "HOLD", "CHECK_BITS",
            "Grads", "GRAD_FIELDS", "make_grads", "mrlmoe_train_workspace_size", "mrlmoe_forward_train",
-           "mrlmoe_backward", "grad_buffers"]
+           "mrlmoe_backward", "mrlmoe_backward_timed", "grad_buffers"]
 
 
 def grad_buffers(cfg: Config, device="cuda"):

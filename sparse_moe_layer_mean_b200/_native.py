@@ -27,9 +27,12 @@ EXPORTED = ("mrlmoe_workspace_size", "mrlmoe_route", "mrlmoe_forward", "mrlmoe_f
             "mrlmoe_bias_update", "mrlmoe_linear", "mrlmoe_get_device_status",
             "mrlmoe_status_string", "mrlmoe_route_scores_static", "mrlmoe_quantize_e4m3",
             "mrlmoe_check_routing", "mrlmoe_get_device_detail", "mrlmoe_train_workspace_size",
-            "mrlmoe_forward_train", "mrlmoe_backward")
+            "mrlmoe_forward_train", "mrlmoe_backward", "mrlmoe_backward_timed")
 STATIC_SCRATCH_BYTES = 2 * 1024 * 1024
 NUM_STAGE_EVENTS = 9
+NUM_BACKWARD_EVENTS = 11
+BACKWARD_STAGES = ("dn", "dw_up", "rms_combine_bwd", "dh_glu_bwd", "dz", "token_router_bwd",
+                   "dw_router_alpha", "expert_wgrad", "dx", "dw_down")
 STAGES = ("down_proj", "router_topk", "dispatch", "gather", "gate_up_glu", "expert_down",
           "combine_rmsnorm", "up_proj")
 
@@ -124,6 +127,9 @@ def lib() -> ctypes.CDLL:
         L.mrlmoe_backward.argtypes = [POINTER(Config), POINTER(Weights), c_void_p, c_void_p, POINTER(Grads),
                                       c_void_p, c_size_t, c_void_p]
         L.mrlmoe_backward.restype = c_int
+        L.mrlmoe_backward_timed.argtypes = [POINTER(Config), POINTER(Weights), c_void_p, c_void_p, POINTER(Grads),
+                                            c_void_p, c_size_t, c_void_p, c_void_p, c_int]
+        L.mrlmoe_backward_timed.restype = c_int
         L.mrlmoe_status_string.argtypes = [c_int]
         L.mrlmoe_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -237,6 +243,19 @@ def mrlmoe_backward(cfg: Config, weights: Weights, x, dy, grads: Grads, workspac
     _check(lib().mrlmoe_backward(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(dy),
                                  ctypes.byref(grads), _ptr(workspace), int(ws_bytes), _stream_ptr(stream)),
            "mrlmoe_backward")
+
+
+def mrlmoe_backward_timed(cfg: Config, weights: Weights, x, dy, grads: Grads, workspace, ws_bytes: int,
+                          events, stream=None) -> None:
+    """``events``: NUM_BACKWARD_EVENTS timing events, recorded at the
+    backward's stage boundaries (BACKWARD_STAGES lie between them)."""
+    arr = (c_void_p * NUM_BACKWARD_EVENTS)()
+    for i, e in enumerate(events):
+        arr[i] = e.cuda_event if hasattr(e, "cuda_event") else int(e)
+    _check(lib().mrlmoe_backward_timed(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(dy),
+                                       ctypes.byref(grads), _ptr(workspace), int(ws_bytes), _stream_ptr(stream),
+                                       arr, len(events)),
+           "mrlmoe_backward_timed")
 
 
 def mrlmoe_bias_update(cfg: Config, counts, bias, gamma: float, stream=None) -> None:

@@ -130,6 +130,22 @@ __device__ __forceinline__ void load_mn_pair(uint32_t sa, const CUtensorMap *m, 
   tma_load_2d(sa + 8192, m, bar, x0 + 64, y);
 }
 
+// a[c] summed over the warp's 32 lanes, for all 32 c at once: lane i returns
+// the sum for c = i (31 shuffles instead of 32 x 5).
+__device__ __forceinline__ float transpose_sum32(float (&a)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? a[i] : a[i + off];
+      const float keep = upper ? a[i + off] : a[i];
+      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return a[0];
+}
+
 // ------------------------------------------ expert dgrad through W_down
 // Swap-AB over the dispatch groups: unit = (group, 128-wide d_ff slice m,
 // <= 256 dispatch rows); D[f, row] = sum_l W_d[l, f] dc[row, l], so W_d is
@@ -218,24 +234,34 @@ struct DhPolicy {
     for (int c0 = 0; c0 < U.nv; c0 += 32) {
       float v[32];
       tmem_ld32(taddr + c0, v);
+      // the chunk's g, u, h loads are all issued before any is used
+      __nv_bfloat16 gr[32], ur[32], hr[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const size_t o = static_cast<size_t>(U.row0 + c0 + c) * 64;
+        const bool in = c0 + c < U.nv;
+        gr[c] = in ? gp[o] : __float2bfloat16_rn(0.f);
+        ur[c] = in ? up[o] : __float2bfloat16_rn(0.f);
+        hr[c] = in ? hp[o] : __float2bfloat16_rn(0.f);
+      }
       tmem_ld_wait();
+      float part[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         const int col = c0 + c;
-        if (col >= U.nv) continue;  // uniform over the warp
-        const size_t o = static_cast<size_t>(U.row0 + col) * 64;
-        const float g = __bfloat162float(gp[o]);
-        const float u = __bfloat162float(up[o]);
-        const float h = __bfloat162float(hp[o]);
-        float part = h * v[c];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-        if (lane == 0) red[q * kBN + col] = part;
-        const float dh = s_ws[col] * v[c];
-        const float sg = 1.0f / (1.0f + __expf(-g));
-        dgp[o] = __float2bfloat16_rn(dh * u * sg * (1.0f + g * (1.0f - sg)));
-        dup[o] = __float2bfloat16_rn(dh * g * sg);
+        const float g = __bfloat162float(gr[c]);
+        const float u = __bfloat162float(ur[c]);
+        part[c] = __bfloat162float(hr[c]) * v[c];
+        if (col < U.nv) {  // uniform over the warp
+          const size_t o = static_cast<size_t>(U.row0 + col) * 64;
+          const float dh = s_ws[col] * v[c];
+          const float sg = 1.0f / (1.0f + __expf(-g));
+          dgp[o] = __float2bfloat16_rn(dh * u * sg * (1.0f + g * (1.0f - sg)));
+          dup[o] = __float2bfloat16_rn(dh * g * sg);
+        }
       }
+      const float tot = transpose_sum32(part, lane);  // lane i: column c0 + i summed over the warp's 32 f
+      if (c0 + lane < U.nv) red[q * kBN + c0 + lane] = tot;
     }
     named_bar_sync(2, 128);
     if (!sh) {
@@ -346,16 +372,19 @@ struct DzPolicy {
 //   dW_d[l, f] = sum_rows do[row, l] h[row, f]    A: do rows,   B: h planes
 // with do = w' dc.  Rows past the group's end in its last K block belong to
 // the next group (or are the TMA zero fill); they are zeroed in shared
-// memory before the MMAs.  A group without rows writes zero tiles.
+// memory before the MMAs.  A group without rows writes zero tiles.  The fp32
+// tiles leave through TMA stores: each epilogue warp stages its 32 rows x 32
+// columns in a swizzled 4 KB buffer (two per warp, alternating) and one lane
+// issues the bulk store, so the gradient writes go out as whole lines.
 struct WgradPolicy {
   static constexpr bool kAMN = true, kBMN = true, kRaggedK = true;
   static constexpr uint32_t kAMNStride = 8192, kBMNStride = 8192;
-  static constexpr int kStages = 4;
-  static constexpr int kGroup = 2;
+  static constexpr int kStages = 3;
+  static constexpr int kGroup = 1;
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
-  static constexpr int kEpiSmem = 0;
+  static constexpr int kEpiSmem = 4 * 2 * 4096 + 1024;  // + alignment of the swizzled buffers
   static constexpr int kAuxSmem = kMaxGroups * 4;
   static constexpr int kUmmaKBytes = 32;
   static constexpr int kASub = 1, kASubBytes = 0;
@@ -364,17 +393,21 @@ struct WgradPolicy {
     CUtensorMap tz;    // z rows [rows, L], boxes 64 x 64
     CUtensorMap tdo;   // do rows [rows, L], boxes 64 x 64
     CUtensorMap th;    // h [F/64 * rows, 64], boxes 64 x 64
+    // fp32 gradients, boxes of 32 columns x 32 rows, SWIZZLE_128B:
+    CUtensorMap og, ou, od;    // routed [E*F, L], [E*F, L], [E*L, F]
+    CUtensorMap sog, sou, sod; // shared [F, L], [F, L], [L, F]
     const int32_t *grp_off;  // E + 2 entries
-    float *dwg, *dwu, *dwd;  // routed [E, F, L], [E, F, L], [E, L, F]
-    float *dsg, *dsu, *dsd;  // shared [F, L], [F, L], [L, F]
     int E, F, L, rows;
     uint32_t *status;
   };
-  struct EpiState {};
+  struct EpiState {
+    int n = 0;  // chunks this thread's warp has staged (selects the buffer)
+  };
   static __device__ __forceinline__ int tiles_gu(const Params &p) { return (p.F / 128) * ((p.L + kBN - 1) / kBN); }
   static __device__ __forceinline__ int tiles_d(const Params &p) { return (p.L / 128) * ((p.F + kBN - 1) / kBN); }
   static __device__ __forceinline__ void prefetch(const Params &p) {
     prefetch_tmap(&p.tdgu); prefetch_tmap(&p.tz); prefetch_tmap(&p.tdo); prefetch_tmap(&p.th);
+    prefetch_tmap(&p.og); prefetch_tmap(&p.ou); prefetch_tmap(&p.od);
   }
   static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) {
     int *s = reinterpret_cast<int *>(aux);
@@ -453,16 +486,15 @@ struct WgradPolicy {
   }
   // Lane = output row (f for dW_g/dW_u, l for dW_d), columns = the tile's N.
   static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
-                                                  int lane, int, EpiState &, uint8_t *) {
+                                                  int lane, int, EpiState &st, uint8_t *epi) {
     const int which = U.g % 3, g = U.g / 3;
     const bool sh = g == p.E;
-    const size_t FL = static_cast<size_t>(p.F) * p.L;
-    float *base = which == 0 ? (sh ? p.dsg : p.dwg + g * FL)
-                : which == 1 ? (sh ? p.dsu : p.dwu + g * FL)
-                             : (sh ? p.dsd : p.dwd + g * FL);
-    const int ld = which < 2 ? p.L : p.F;
-    const int row = U.m * 128 + q * 32 + lane;
-    float4 *dst = reinterpret_cast<float4 *>(base + static_cast<size_t>(row) * ld + U.n0);
+    const CUtensorMap *map = which == 0 ? (sh ? &p.sog : &p.og) : which == 1 ? (sh ? &p.sou : &p.ou)
+                                                                               : (sh ? &p.sod : &p.od);
+    const int y = (sh ? 0 : g * (which < 2 ? p.F : p.L)) + U.m * 128 + q * 32;
+    const uint32_t e0 = smem_u32(epi);
+    const uint32_t bufs = ((e0 + 1023u) & ~1023u) + static_cast<uint32_t>(q) * 8192u;
+    uint8_t *bufp = epi + (bufs - e0);
     const bool empty = U.krows == 0;
     for (int c0 = 0; c0 < U.nv; c0 += 32) {
       float v[32];
@@ -473,8 +505,20 @@ struct WgradPolicy {
         tmem_ld32(taddr + c0, v);
         tmem_ld_wait();
       }
+      const int b = st.n & 1;
+      if (lane == 0) bulk_wait_read<1>();  // the store issued two chunks ago has read this buffer
+      __syncwarp();
+      float4 *row = reinterpret_cast<float4 *>(bufp + b * 4096 + lane * 128);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dst[c0 / 4 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int j = 0; j < 8; ++j)  // 16-byte chunk j of row `lane` sits at chunk j ^ (lane % 8)
+        row[j ^ (lane & 7)] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      fence_proxy_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(map, bufs + b * 4096, U.n0 + c0, y);
+        bulk_commit();
+      }
+      ++st.n;
     }
   }
 };
@@ -505,6 +549,7 @@ __device__ __forceinline__ uint2 pack_bf16x4(float4 v) {
 // dispatch row of the token (dcd: as is; dod: times the row's w'), the
 // shared row Tk + t included (weight 1).  gpart[block] = sum over the
 // block's tokens of dn cn (the gain's gradient, reduced by gain_reduce_kernel).
+template <int MAXV4>  // float4 columns per thread: d_lat <= 4 * kBwdThreads * MAXV4
 __global__ void __launch_bounds__(kBwdThreads) rms_combine_bwd_kernel(
     const float4 *__restrict__ slots, const float4 *__restrict__ dn, const float4 *__restrict__ gain,
     const int32_t *__restrict__ inv, const float *__restrict__ wscaled, int T, int L, int k, float eps,
@@ -514,15 +559,15 @@ __global__ void __launch_bounds__(kBwdThreads) rms_combine_bwd_kernel(
   if (call_failed(status)) return;
   const int L4 = L >> 2;
   const size_t Tk = static_cast<size_t>(T) * k;
-  float4 gacc[kBwdMaxV4];
+  float4 gacc[MAXV4];
 #pragma unroll
-  for (int v = 0; v < kBwdMaxV4; ++v) gacc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int v = 0; v < MAXV4; ++v) gacc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     const float4 *base = slots + static_cast<size_t>(t) * (k + 1) * L4;
-    float4 c[kBwdMaxV4];
+    float4 c[MAXV4];
     float ss = 0.f;
 #pragma unroll
-    for (int v = 0; v < kBwdMaxV4; ++v) {
+    for (int v = 0; v < MAXV4; ++v) {
       const int i = threadIdx.x + v * kBwdThreads;
       if (i < L4) {
         float4 a = __ldg(base + i);
@@ -535,10 +580,10 @@ __global__ void __launch_bounds__(kBwdThreads) rms_combine_bwd_kernel(
       }
     }
     const float r = 1.0f / sqrtf(block_sum(ss, red) / static_cast<float>(L) + eps);
-    float4 dcn[kBwdMaxV4];
+    float4 dcn[MAXV4];
     float dot = 0.f;
 #pragma unroll
-    for (int v = 0; v < kBwdMaxV4; ++v) {
+    for (int v = 0; v < MAXV4; ++v) {
       const int i = threadIdx.x + v * kBwdThreads;
       if (i < L4) {
         const float4 d = __ldg(dn + static_cast<size_t>(t) * L4 + i);
@@ -558,7 +603,7 @@ __global__ void __launch_bounds__(kBwdThreads) rms_combine_bwd_kernel(
       uint2 *d1 = reinterpret_cast<uint2 *>(dcd + row * L);
       uint2 *d2 = reinterpret_cast<uint2 *>(dod + row * L);
 #pragma unroll
-      for (int v = 0; v < kBwdMaxV4; ++v) {
+      for (int v = 0; v < MAXV4; ++v) {
         const int i = threadIdx.x + v * kBwdThreads;
         if (i < L4) {
           const float4 dc = make_float4(r * (dcn[v].x - c[v].x * m), r * (dcn[v].y - c[v].y * m),
@@ -570,7 +615,7 @@ __global__ void __launch_bounds__(kBwdThreads) rms_combine_bwd_kernel(
     }
   }
 #pragma unroll
-  for (int v = 0; v < kBwdMaxV4; ++v) {
+  for (int v = 0; v < MAXV4; ++v) {
     const int i = threadIdx.x + v * kBwdThreads;
     if (i < L4) gpart[static_cast<size_t>(blockIdx.x) * L4 + i] = gacc[v];
   }

@@ -299,6 +299,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
   }
 done:
+  // bulk tensor stores an epilogue issued finish before the CTA's shared memory goes away
+  if (lane == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -203,6 +203,20 @@ bool make_map(CUtensorMap *m, const void *base, int esize, uint64_t inner, uint6
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 [rows, inner] written by TMA stores: boxes of 32 columns x 32 rows
+// (128-byte rows, SWIZZLE_128B).
+bool make_map_f32_out(CUtensorMap *m, void *base, uint64_t inner, uint64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The three box heights of a bf16 token tensor [rows, inner] (load_token_rows).
 bool make_token_maps(TokenMaps *t, const void *base, uint64_t inner, uint64_t rows) {
   t->plane_rows = 0;
@@ -772,7 +786,8 @@ mrlmoe_status launch_dense_grad(const CUtensorMap &ta, const CUtensorMap &tb, vo
 }
 
 mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, const void *x, const void *dy,
-                            const mrlmoe_grads *g, void *workspace, size_t ws_bytes, void *stream) {
+                            const mrlmoe_grads *g, void *workspace, size_t ws_bytes, void *stream,
+                            void *const *ev = nullptr) {
   mrlmoe_status s = check_config(cfg);
   if (s != MRLMOE_OK) return s;
   if (cfg->dtype != MRLMOE_BF16 || cfg->d_ff > 128 * kBwdMaxSlices) return MRLMOE_ERR_UNSUPPORTED;
@@ -801,8 +816,12 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
   __nv_bfloat16 *dgu = bf(LT.dgu), *dzx = bf(LT.dzx);
   float *dn = f32(LT.dn), *dwsp = f32(LT.dwsp), *dl = f32(LT.dl), *aw = f32(LT.aw), *gpart = f32(LT.gpart);
   const __nv_bfloat16 *zhi = P.zbuf + static_cast<size_t>(Tk) * Ld;
+  auto mark = [&](int i) -> bool {
+    return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
+  };
   // the call continues the forward's status word; only this call's hold mask is set
   MRL_TRY(cudaMemsetAsync(reinterpret_cast<uint8_t *>(P.status) + 4, static_cast<int>(cfg->hold & 0xffu), 1, st));
+  if (!mark(0)) return MRLMOE_ERR_CUDA;
 
   // dn = dy W_up (W_up [D, Ld] MN-major); dW_up = dy^T n (both MN-major, K = T)
   {
@@ -811,20 +830,26 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
     if ((s = launch_dense_grad<DenseGradPolicy<false, true, true>>(ta, tb, dn, T, Ld, D, P.status, sms, st)) !=
         MRLMOE_OK)
       return s;
+    if (!mark(1)) return MRLMOE_ERR_CUDA;
     if (!make_map(&ta, dy, 2, D, T, 64) || !make_map(&tb, P.nbuf, 2, Ld, T, 64)) return MRLMOE_ERR_CUDA;
     if ((s = launch_dense_grad<DenseGradPolicy<true, true, true>>(ta, tb, g->d_w_up, D, Ld, T, P.status, sms, st)) !=
         MRLMOE_OK)
       return s;
   }
+  if (!mark(2)) return MRLMOE_ERR_CUDA;
   // RMSNorm + combine backward: dc rows (plain and weighted) per dispatch row
   const int nb = rms_bwd_blocks(*cfg);
-  rms_combine_bwd_kernel<<<nb, kBwdThreads, 0, st>>>(
-      reinterpret_cast<const float4 *>(P.slots), reinterpret_cast<const float4 *>(dn),
-      reinterpret_cast<const float4 *>(w->rms_gain), P.inv, P.wscaled, T, Ld, k, cfg->rms_eps, dcd, dod,
-      reinterpret_cast<float4 *>(gpart), P.status);
+  {
+    auto kern = Ld <= 4 * kBwdThreads * 2 ? rms_combine_bwd_kernel<2>
+              : Ld <= 4 * kBwdThreads * 4 ? rms_combine_bwd_kernel<4> : rms_combine_bwd_kernel<kBwdMaxV4>;
+    kern<<<nb, kBwdThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), reinterpret_cast<const float4 *>(dn),
+                                     reinterpret_cast<const float4 *>(w->rms_gain), P.inv, P.wscaled, T, Ld, k,
+                                     cfg->rms_eps, dcd, dod, reinterpret_cast<float4 *>(gpart), P.status);
+  }
   MRL_TRY(cudaGetLastError());
   gain_reduce_kernel<<<(Ld + 255) / 256, 256, 0, st>>>(gpart, nb, Ld, g->d_rms_gain, P.status);
   MRL_TRY(cudaGetLastError());
+  if (!mark(3)) return MRLMOE_ERR_CUDA;
   // unit tables of the two grouped dgrad GEMMs (token tiles of 256; d_ff / 128 and d_lat / 128 M tiles)
   int32_t *bgo = i32(LT.bgrp_off), *bgc = i32(LT.bgrp_cnt), *bu1 = i32(LT.bunit1), *bu2 = i32(LT.bunit2);
   expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, DhPolicy::kBN, F / 128, Ld / 128, bgo, bgc, bu1,
@@ -845,6 +870,7 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
     p.status = P.status;
     MRL_TRY(launch_gemm<DhPolicy>(p, sms, st));
   }
+  if (!mark(4)) return MRLMOE_ERR_CUDA;
   {
     DzPolicy::Params p{};
     if (!make_map(&p.wg, w->w_gate, 2, Ld, static_cast<uint64_t>(E) * F, 64) ||
@@ -859,15 +885,18 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
     p.status = P.status;
     MRL_TRY(launch_gemm<DzPolicy>(p, sms, st));
   }
+  if (!mark(5)) return MRLMOE_ERR_CUDA;
   // routers, combine weights, alpha; dz reduced per token
   token_bwd_kernel<<<T, kBwdThreads, Ld * sizeof(float), st>>>(
       dwsp, F / 128, P.topk_idx, P.topk_w, w->expert_scale, zhi, P.zlo,
       static_cast<const __nv_bfloat16 *>(w->w_router), P.slots, T, Ld, E, R, k, static_cast<int>(cfg->aggregation),
       dzx, dl, aw, P.status);
   MRL_TRY(cudaGetLastError());
+  if (!mark(6)) return MRLMOE_ERR_CUDA;
   expert_param_bwd_kernel<<<E, kBwdThreads, 0, st>>>(P.grp_off, P.grp_cnt, P.perm, dl, aw, zhi, P.zlo, Ld, E, R, k,
                                                      g->d_w_router, g->d_expert_scale, P.status);
   MRL_TRY(cudaGetLastError());
+  if (!mark(7)) return MRLMOE_ERR_CUDA;
   // expert weight gradients (K = each group's rows)
   {
     WgradPolicy::Params p{};
@@ -875,13 +904,17 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
         !make_map(&p.tz, P.zbuf, 2, Ld, rows, 64) || !make_map(&p.tdo, dod, 2, Ld, rows, 64) ||
         !make_map(&p.th, P.hbuf, 2, 64, static_cast<uint64_t>(F / 64) * rows, 64))
       return MRLMOE_ERR_CUDA;
+    const uint64_t EF = static_cast<uint64_t>(E) * F, EL = static_cast<uint64_t>(E) * Ld;
+    if (!make_map_f32_out(&p.og, g->d_w_gate, Ld, EF) || !make_map_f32_out(&p.ou, g->d_w_up_e, Ld, EF) ||
+        !make_map_f32_out(&p.od, g->d_w_down_e, F, EL) || !make_map_f32_out(&p.sog, g->d_w_sh_gate, Ld, F) ||
+        !make_map_f32_out(&p.sou, g->d_w_sh_up, Ld, F) || !make_map_f32_out(&p.sod, g->d_w_sh_down, F, Ld))
+      return MRLMOE_ERR_CUDA;
     p.grp_off = P.grp_off;
-    p.dwg = g->d_w_gate; p.dwu = g->d_w_up_e; p.dwd = g->d_w_down_e;
-    p.dsg = g->d_w_sh_gate; p.dsu = g->d_w_sh_up; p.dsd = g->d_w_sh_down;
     p.E = E; p.F = F; p.L = Ld; p.rows = rows;
     p.status = P.status;
     MRL_TRY(launch_gemm<WgradPolicy>(p, sms, st));
   }
+  if (!mark(8)) return MRLMOE_ERR_CUDA;
   // dx = dzx W_dn (W_dn [Ld, D] MN-major); dW_dn = dzx^T x (K = T)
   {
     CUtensorMap ta, tb;
@@ -889,11 +922,13 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
     if ((s = launch_dense_grad<DenseGradPolicy<false, true, false>>(ta, tb, g->dx, T, D, Ld, P.status, sms, st)) !=
         MRLMOE_OK)
       return s;
+    if (!mark(9)) return MRLMOE_ERR_CUDA;
     if (!make_map(&ta, dzx, 2, Ld, T, 64) || !make_map(&tb, x, 2, D, T, 64)) return MRLMOE_ERR_CUDA;
     if ((s = launch_dense_grad<DenseGradPolicy<true, true, true>>(ta, tb, g->d_w_down, Ld, D, T, P.status, sms,
                                                                     st)) != MRLMOE_OK)
       return s;
   }
+  if (!mark(10)) return MRLMOE_ERR_CUDA;
   return MRLMOE_OK;
 }
 
@@ -1026,6 +1061,15 @@ mrlmoe_status mrlmoe_forward_train(const mrlmoe_config *cfg, const mrlmoe_weight
 mrlmoe_status mrlmoe_backward(const mrlmoe_config *cfg, const mrlmoe_weights *w, const void *x, const void *dy,
                               const mrlmoe_grads *grads, void *workspace, size_t ws_bytes, void *stream) {
   return backward_impl(cfg, w, x, dy, grads, workspace, ws_bytes, stream);
+}
+
+mrlmoe_status mrlmoe_backward_timed(const mrlmoe_config *cfg, const mrlmoe_weights *w, const void *x,
+                                    const void *dy, const mrlmoe_grads *grads, void *workspace, size_t ws_bytes,
+                                    void *stream, void *const *events, int n_events) {
+  if (!events || n_events != MRLMOE_NUM_BACKWARD_EVENTS) return MRLMOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return MRLMOE_ERR_INVALID_ARG;
+  return backward_impl(cfg, w, x, dy, grads, workspace, ws_bytes, stream, events);
 }
 
 mrlmoe_status mrlmoe_bias_update(const mrlmoe_config *cfg, const int32_t *counts, float *bias, float gamma,
