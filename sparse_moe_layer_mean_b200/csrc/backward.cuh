@@ -9,7 +9,7 @@
 //   dc  = r (dn g - cn mean(cn dn g)) dgain = sum_t dn cn           (per token)
 //   per dispatch row of expert e (token t, weight w' = w alpha):
 //   dh' = dc_t W_d,e                  dw'  = <h, dh'>                (grouped)
-//   dh  = w' dh';  dg = dh u SiLU'(g);  du = dh SiLU(g)
+//   dh  = w' dh';  dg = dh u SiLU'(g);  du = dh SiLU(g)   (h = SiLU(g) u from the kept bf16 g, u)
 //   dz  = dg W_g,e + du W_u,e                                          (grouped)
 //   dW_g,e = dg^T z, dW_u,e = du^T z, dW_d,e = (w' dc)^T h            (grouped, K = rows)
 //   dalpha_e = sum over e's rows of w dw';  dw = alpha dw'
@@ -151,7 +151,10 @@ __device__ __forceinline__ float transpose_sum32(float (&a)[32], int lane) {
 // <= 256 dispatch rows); D[f, row] = sum_l W_d[l, f] dc[row, l], so W_d is
 // read MN-major straight from its [d_lat, d_ff] storage.  The epilogue
 // finishes the GLU backward on the tile and leaves dg, du (K-blocked, as h)
-// and the slice's share of dw' = <h, dh'> per row.
+// and the slice's share of dw' = <h, dh'> per row, with h = SiLU(g) u
+// recomputed from the bf16 g and u that the training forward kept (one
+// 4-byte word per element; the next 32 rows' words load while the current
+// ones are used).
 struct DhPolicy {
   static constexpr bool kAMN = true, kBMN = false;
   static constexpr uint32_t kAMNStride = 8192, kBMNStride = 0;
@@ -169,12 +172,11 @@ struct DhPolicy {
     CUtensorMap sd;  // shared W_down [L, F]
     TokenMaps tc;    // dc rows [rows, L] row-major, boxes 64 x 16/32/64
     GroupTable gt;   // M tiles per group: F / 128
-    const int32_t *perm;
-    const float *wscaled;
-    const __nv_bfloat16 *g, *u, *h;  // [F/64][rows][64]
+    const float *wrow;               // [rows]: w' of each dispatch row (1 for the shared expert's)
+    const uint32_t *gu;              // [F/64][rows][64] words: bf16 g (low), u (high)
     __nv_bfloat16 *dgu;              // [2F/64][rows][64]: dg planes, then du planes
-    float *dwsp;                     // [F/128][T*k]: per-slice share of dw'
-    int L, F, Tk, rows;
+    float *dwsp;                     // [F/128][rows]: per-slice share of dw' by dispatch row
+    int L, F, rows;
     uint32_t *status;
   };
   struct EpiState {};
@@ -211,65 +213,54 @@ struct DhPolicy {
   // consecutive f of one K-blocked plane (64 contiguous bytes of g, u, h).
   static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
                                                   int lane, int etid, EpiState &, uint8_t *epi) {
-    int *s_flat = reinterpret_cast<int *>(epi);
     float *s_ws = reinterpret_cast<float *>(epi + kBN * 4);
     float *red = reinterpret_cast<float *>(epi + kBN * 8);  // [4][kBN]
-    const bool sh = U.g == p.gt.E;
-    for (int c = etid; c < U.nv; c += 128) {
-      const int row = U.row0 + c;
-      const int flat = sh ? -1 : __ldg(p.perm + row);
-      s_flat[c] = flat;
-      s_ws[c] = sh ? 1.0f : __ldg(p.wscaled + flat);
-    }
+    for (int c = etid; c < U.nv; c += 128) s_ws[c] = __ldg(p.wrow + U.row0 + c);
     named_bar_sync(2, 128);
     const int f = U.m * 128 + q * 32 + lane;
     const size_t plane = static_cast<size_t>(f >> 6);
     const size_t prow = static_cast<size_t>(p.rows) * 64;
     const int within = f & 63;
-    const __nv_bfloat16 *gp = p.g + plane * prow + within;
-    const __nv_bfloat16 *up = p.u + plane * prow + within;
-    const __nv_bfloat16 *hp = p.h + plane * prow + within;
+    const uint32_t *gup = p.gu + plane * prow + within;
     __nv_bfloat16 *dgp = p.dgu + plane * prow + within;
     __nv_bfloat16 *dup = p.dgu + (static_cast<size_t>(p.F >> 6) + plane) * prow + within;
+    uint32_t cur[32], nxt[32];
+    auto load_chunk = [&](uint32_t (&dst)[32], int c0) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        dst[c] = c0 + c < U.nv ? __ldg(gup + static_cast<size_t>(U.row0 + c0 + c) * 64) : 0u;
+    };
+    load_chunk(cur, 0);
     for (int c0 = 0; c0 < U.nv; c0 += 32) {
       float v[32];
       tmem_ld32(taddr + c0, v);
-      // the chunk's g, u, h loads are all issued before any is used
-      __nv_bfloat16 gr[32], ur[32], hr[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const size_t o = static_cast<size_t>(U.row0 + c0 + c) * 64;
-        const bool in = c0 + c < U.nv;
-        gr[c] = in ? gp[o] : __float2bfloat16_rn(0.f);
-        ur[c] = in ? up[o] : __float2bfloat16_rn(0.f);
-        hr[c] = in ? hp[o] : __float2bfloat16_rn(0.f);
-      }
+      if (c0 + 32 < U.nv) load_chunk(nxt, c0 + 32);
       tmem_ld_wait();
       float part[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         const int col = c0 + c;
-        const float g = __bfloat162float(gr[c]);
-        const float u = __bfloat162float(ur[c]);
-        part[c] = __bfloat162float(hr[c]) * v[c];
+        const float g = __uint_as_float(cur[c] << 16);
+        const float u = __uint_as_float(cur[c] & 0xFFFF0000u);
+        const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
+        part[c] = g * sg * u * v[c];
         if (col < U.nv) {  // uniform over the warp
           const size_t o = static_cast<size_t>(U.row0 + col) * 64;
           const float dh = s_ws[col] * v[c];
-          const float sg = 1.0f / (1.0f + __expf(-g));
           dgp[o] = __float2bfloat16_rn(dh * u * sg * (1.0f + g * (1.0f - sg)));
           dup[o] = __float2bfloat16_rn(dh * g * sg);
         }
       }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
       const float tot = transpose_sum32(part, lane);  // lane i: column c0 + i summed over the warp's 32 f
       if (c0 + lane < U.nv) red[q * kBN + c0 + lane] = tot;
     }
     named_bar_sync(2, 128);
-    if (!sh) {
-      for (int c = etid; c < U.nv; c += 128)
-        p.dwsp[static_cast<size_t>(U.m) * p.Tk + s_flat[c]] =
-            (red[c] + red[kBN + c]) + (red[2 * kBN + c] + red[3 * kBN + c]);
-    }
-    named_bar_sync(2, 128);  // s_flat/s_ws/red are rewritten by the next unit
+    for (int c = etid; c < U.nv; c += 128)
+      p.dwsp[static_cast<size_t>(U.m) * p.rows + U.row0 + c] =
+          (red[c] + red[kBN + c]) + (red[2 * kBN + c] + red[3 * kBN + c]);
+    named_bar_sync(2, 128);  // s_ws/red are rewritten by the next unit
   }
 };
 
@@ -549,12 +540,13 @@ __device__ __forceinline__ uint2 pack_bf16x4(float4 v) {
 // dispatch row of the token (dcd: as is; dod: times the row's w'), the
 // shared row Tk + t included (weight 1).  gpart[block] = sum over the
 // block's tokens of dn cn (the gain's gradient, reduced by gain_reduce_kernel).
+// wrow[row] = the row's weight w' (1 for the shared expert's row).
 template <int MAXV4>  // float4 columns per thread: d_lat <= 4 * kBwdThreads * MAXV4
 __global__ void __launch_bounds__(kBwdThreads) rms_combine_bwd_kernel(
     const float4 *__restrict__ slots, const float4 *__restrict__ dn, const float4 *__restrict__ gain,
     const int32_t *__restrict__ inv, const float *__restrict__ wscaled, int T, int L, int k, float eps,
-    __nv_bfloat16 *__restrict__ dcd, __nv_bfloat16 *__restrict__ dod, float4 *__restrict__ gpart,
-    const uint32_t *status) {
+    __nv_bfloat16 *__restrict__ dcd, __nv_bfloat16 *__restrict__ dod, float *__restrict__ wrow,
+    float4 *__restrict__ gpart, const uint32_t *status) {
   __shared__ float red[kBwdThreads / 32];
   if (call_failed(status)) return;
   const int L4 = L >> 2;
@@ -600,6 +592,7 @@ __global__ void __launch_bounds__(kBwdThreads) rms_combine_bwd_kernel(
       const bool shared = j == k;
       const size_t row = shared ? Tk + t : static_cast<size_t>(__ldg(inv + static_cast<size_t>(t) * k + j));
       const float w = shared ? 1.0f : __ldg(wscaled + static_cast<size_t>(t) * k + j);
+      if (threadIdx.x == 0) wrow[row] = w;
       uint2 *d1 = reinterpret_cast<uint2 *>(dcd + row * L);
       uint2 *d2 = reinterpret_cast<uint2 *>(dod + row * L);
 #pragma unroll
@@ -645,7 +638,8 @@ constexpr int kBwdMaxRouters = 8;
 //   dzx = sum_{j <= k} dzs[t][j] + sum_{j,r} dl_{j,r} W_router[r, e_j]  (in that order)
 // Dynamic shared memory: d_lat floats (zx).
 __global__ void __launch_bounds__(kBwdThreads) token_bwd_kernel(
-    const float *__restrict__ dwsp, int nsl, const int32_t *__restrict__ topk_idx,
+    const float *__restrict__ dwsp, int nsl, int rows, const int32_t *__restrict__ inv,
+    const int32_t *__restrict__ topk_idx,
     const float *__restrict__ topk_w, const float *__restrict__ alpha, const __nv_bfloat16 *__restrict__ zhi,
     const __nv_bfloat16 *__restrict__ zlo, const __nv_bfloat16 *__restrict__ wr, const float *__restrict__ dzs,
     int T, int L, int E, int R, int k, int agg, __nv_bfloat16 *__restrict__ dzx, float *__restrict__ dl,
@@ -671,7 +665,8 @@ __global__ void __launch_bounds__(kBwdThreads) token_bwd_kernel(
   if (threadIdx.x < k) eidx[threadIdx.x] = __ldg(topk_idx + static_cast<size_t>(t) * k + threadIdx.x);
   for (int i = threadIdx.x; i < k * nsl; i += kBwdThreads) {
     const int j = i / nsl, m = i - j * nsl;
-    part[i] = __ldg(dwsp + static_cast<size_t>(m) * Tk + static_cast<size_t>(t) * k + j);
+    const int row = __ldg(inv + static_cast<size_t>(t) * k + j);
+    part[i] = __ldg(dwsp + static_cast<size_t>(m) * rows + row);
   }
   __syncthreads();
   for (int idx = warp; idx < k * R; idx += kBwdThreads / 32) {

@@ -259,10 +259,7 @@ struct Glu2Policy {
         if (cbase + c < U.nv) {
           const size_t o = (row0 + cbase + c) * 64;
           hp[o] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
-          if (p.gs) {
-            p.gs[hoff + o] = __float2bfloat16_rn(g);
-            p.us[hoff + o] = __float2bfloat16_rn(u);
-          }
+          if (p.gu) p.gu[hoff + o] = pack_bf16x2(g, u);
         }
       }
       named_bar_sync(2, 128);

@@ -92,7 +92,7 @@ struct Layout {
   size_t status, topk_idx, topk_w, wscaled, counts, offsets, grp_off, grp_cnt, unit1, unit2, perm, inv, mask,
       base, cand_v, cand_s, cand_i, rpart, zbuf, zlo, hbuf, slots, nbuf, xq, xs, zq, zs, hq, hs, nq, ns, total;
   // training forward + backward (bf16): kept pre-activations and the backward's buffers
-  size_t gsave, usave, dn, dcd, dod, dgu, dwsp, dzx, dl, aw, gpart, bgrp_off, bgrp_cnt, bunit1, bunit2;
+  size_t gusave, dn, dcd, dod, dgu, dwsp, wrow, dzx, dl, aw, gpart, bgrp_off, bgrp_cnt, bunit1, bunit2;
 };
 
 // Blocks of rms_combine_bwd_kernel (a fixed number, so the gain gradient's
@@ -148,13 +148,13 @@ Layout layout_of(const mrlmoe_config &c, bool train = false) {
   }
   if (train) {
     const size_t rows = Tk + T;
-    L.gsave = take(rows * F * 2);
-    L.usave = take(rows * F * 2);
+    L.gusave = take(rows * F * 4);
     L.dn = take(T * Ld * 4);
     L.dcd = take(rows * Ld * 2);
     L.dod = take(rows * Ld * 2);
     L.dgu = take(rows * 2 * F * 2);
-    L.dwsp = take((F / 128) * Tk * 4);
+    L.dwsp = take((F / 128) * rows * 4);
+    L.wrow = take(rows * 4);
     L.dzx = take(T * Ld * 2);
     L.dl = take(Tk * c.n_routers * 4);
     L.aw = take(Tk * 4);
@@ -660,10 +660,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
       return MRLMOE_ERR_CUDA;
     p.gt = gt1;
     p.h = P.hbuf;
-    if (train) {
-      p.gs = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(workspace) + LT.gsave);
-      p.us = reinterpret_cast<__nv_bfloat16 *>(static_cast<uint8_t *>(workspace) + LT.usave);
-    }
+    if (train) p.gu = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + LT.gusave);
     p.F = F; p.L = Ld; p.rows = Tk + T;
     p.status = P.status;
     MRL_TRY(launch_gemm_pair<Glu2Policy>(p, sms, st));
@@ -812,9 +809,10 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16 *>(b + off); };
   auto f32 = [&](size_t off) { return reinterpret_cast<float *>(b + off); };
   auto i32 = [&](size_t off) { return reinterpret_cast<int32_t *>(b + off); };
-  __nv_bfloat16 *gsave = bf(LT.gsave), *usave = bf(LT.usave), *dcd = bf(LT.dcd), *dod = bf(LT.dod);
+  const uint32_t *gusave = reinterpret_cast<const uint32_t *>(b + LT.gusave);
+  __nv_bfloat16 *dcd = bf(LT.dcd), *dod = bf(LT.dod);
   __nv_bfloat16 *dgu = bf(LT.dgu), *dzx = bf(LT.dzx);
-  float *dn = f32(LT.dn), *dwsp = f32(LT.dwsp), *dl = f32(LT.dl), *aw = f32(LT.aw), *gpart = f32(LT.gpart);
+  float *dn = f32(LT.dn), *dwsp = f32(LT.dwsp), *wrow = f32(LT.wrow), *dl = f32(LT.dl), *aw = f32(LT.aw), *gpart = f32(LT.gpart);
   const __nv_bfloat16 *zhi = P.zbuf + static_cast<size_t>(Tk) * Ld;
   auto mark = [&](int i) -> bool {
     return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
@@ -844,7 +842,7 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
               : Ld <= 4 * kBwdThreads * 4 ? rms_combine_bwd_kernel<4> : rms_combine_bwd_kernel<kBwdMaxV4>;
     kern<<<nb, kBwdThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), reinterpret_cast<const float4 *>(dn),
                                      reinterpret_cast<const float4 *>(w->rms_gain), P.inv, P.wscaled, T, Ld, k,
-                                     cfg->rms_eps, dcd, dod, reinterpret_cast<float4 *>(gpart), P.status);
+                                     cfg->rms_eps, dcd, dod, wrow, reinterpret_cast<float4 *>(gpart), P.status);
   }
   MRL_TRY(cudaGetLastError());
   gain_reduce_kernel<<<(Ld + 255) / 256, 256, 0, st>>>(gpart, nb, Ld, g->d_rms_gain, P.status);
@@ -861,12 +859,11 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
         !make_map(&p.sd, w->w_sh_down, 2, F, Ld, 64) || !make_token_maps(&p.tc, dcd, Ld, rows))
       return MRLMOE_ERR_CUDA;
     p.gt = GroupTable{bgo, bgc, bu1, E, F / 128};
-    p.perm = P.perm;
-    p.wscaled = P.wscaled;
-    p.g = gsave; p.u = usave; p.h = P.hbuf;
+    p.wrow = wrow;
+    p.gu = gusave;
     p.dgu = dgu;
     p.dwsp = dwsp;
-    p.L = Ld; p.F = F; p.Tk = Tk; p.rows = rows;
+    p.L = Ld; p.F = F; p.rows = rows;
     p.status = P.status;
     MRL_TRY(launch_gemm<DhPolicy>(p, sms, st));
   }
@@ -888,7 +885,7 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
   if (!mark(5)) return MRLMOE_ERR_CUDA;
   // routers, combine weights, alpha; dz reduced per token
   token_bwd_kernel<<<T, kBwdThreads, Ld * sizeof(float), st>>>(
-      dwsp, F / 128, P.topk_idx, P.topk_w, w->expert_scale, zhi, P.zlo,
+      dwsp, F / 128, rows, P.inv, P.topk_idx, P.topk_w, w->expert_scale, zhi, P.zlo,
       static_cast<const __nv_bfloat16 *>(w->w_router), P.slots, T, Ld, E, R, k, static_cast<int>(cfg->aggregation),
       dzx, dl, aw, P.status);
   MRL_TRY(cudaGetLastError());

@@ -418,7 +418,8 @@ struct GluParams {
   TokenMaps tz;        // dispatched z [(T*k+T), L] row-major, boxes 64 x 16/32/64
   GroupTable gt;
   __nv_bfloat16 *h;    // [F/64][T*k+T][64], K-blocked (see TokenMaps)
-  __nv_bfloat16 *gs, *us;  // training forward: bf16 gate and up pre-activations, laid out as h (else null)
+  uint32_t *gu;        // training forward: bf16 gate (low half) and up (high half) pre-activations,
+                       // one word per element laid out as h (else null)
   int F, L, rows;      // rows = T*k+T
   uint32_t *status;
 };
