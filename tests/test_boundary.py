@@ -165,3 +165,44 @@ def test_python_binding_raises_on_error():
     with pytest.raises(M.MrlmoeError) as ei:
         M.mrlmoe_linear(0, 0, 0, 8, 128, 128, stream=0)
     assert ei.value.code == 1
+
+
+def test_training_entry_points_reject_bad_arguments_before_cuda():
+    L = N.lib()
+    cfg = _cfg()
+    fwd = M.mrlmoe_workspace_size(cfg)
+    train = M.mrlmoe_train_workspace_size(cfg)
+    assert train > fwd                                  # + kept pre-activations and backward buffers
+    assert M.mrlmoe_train_workspace_size(_cfg(T=128)) > train
+    assert M.mrlmoe_train_workspace_size(_cfg(dtype=1)) == 0   # bf16 only
+    assert M.mrlmoe_train_workspace_size(_cfg(dtype=2)) == 0
+    assert M.mrlmoe_train_workspace_size(_cfg(T=0)) == 0
+    assert M.mrlmoe_train_workspace_size(_cfg(d_ff=8320)) == 0  # d_ff <= 8192
+    w = N.Weights(*([4096] * 11 + [None] * 8))
+    g = N.Grads(*([4096] * 12))
+    bwd = lambda c, w_, x, dy, g_, ws, n: L.mrlmoe_backward(
+        ctypes.byref(c) if c is not None else None, ctypes.byref(w_) if w_ is not None else None, x, dy,
+        ctypes.byref(g_) if g_ is not None else None, ws, n, None)
+    assert bwd(None, w, 4096, 4096, g, 4096, train) == 1
+    assert bwd(_cfg(dtype=1), w, 4096, 4096, g, 4096, train) == 2       # unsupported: FP8
+    assert bwd(cfg, w, None, 4096, g, 4096, train) == 1                 # x
+    assert bwd(cfg, w, 4096, None, g, 4096, train) == 1                 # dy
+    assert bwd(cfg, w, 4096, 4096 + 2, g, 4096, train) == 1             # dy misaligned
+    assert bwd(cfg, w, 4096, 4096, None, 4096, train) == 1              # no grads struct
+    for i in range(12):                                                 # every gradient is required
+        gi = N.Grads(*([4096] * i + [None] + [4096] * (11 - i)))
+        assert bwd(cfg, w, 4096, 4096, gi, 4096, train) == 1, N.GRAD_FIELDS[i]
+    partial = N.Weights(*([4096] * 2 + [None] + [4096] * 8 + [None] * 8))
+    assert bwd(cfg, partial, 4096, 4096, g, 4096, train) == 1          # w_gate missing
+    assert bwd(cfg, w, 4096, 4096, g, None, train) == 3                 # no workspace
+    assert bwd(cfg, w, 4096, 4096, g, 4096 + 16, train) == 3            # misaligned
+    assert bwd(cfg, w, 4096, 4096, g, 4096, train - 1) == 3             # forward-sized is too small
+    ft = lambda c, ws, n: L.mrlmoe_forward_train(ctypes.byref(c), ctypes.byref(w), 4096, 4096, 4096, None,
+                                                 ws, n, None)
+    assert ft(_cfg(dtype=1), 4096, train) == 2
+    assert ft(cfg, 4096, train - 1) == 3
+    ev = (ctypes.c_void_p * N.NUM_BACKWARD_EVENTS)(*([4096] * N.NUM_BACKWARD_EVENTS))
+    assert L.mrlmoe_backward_timed(ctypes.byref(cfg), ctypes.byref(w), 4096, 4096, ctypes.byref(g), 4096, train,
+                                   None, ev, N.NUM_BACKWARD_EVENTS - 1) == 1
+    assert L.mrlmoe_backward_timed(ctypes.byref(cfg), ctypes.byref(w), 4096, 4096, ctypes.byref(g), 4096, train,
+                                   None, None, N.NUM_BACKWARD_EVENTS) == 1

@@ -153,3 +153,85 @@ def test_outputs_and_workspace_stay_inside_their_buffers(config, T):
         assert torch.equal(r[name].cpu(), ref_r[name].cpu()), name
     assert torch.all(wsbuf[layer.ws_bytes:] == 0xA5)
     assert torch.equal(y.view(T, s.d_model), y_ref)
+
+
+def _train_setup(config="c0_tiny", T=96):
+    s = W.CONFIGS[config].with_T(T)
+    x = W.make_x(s, "cuda")
+    dy = W.make_dy(s, "cuda")
+    bias = _bias(s.n_experts)
+    layer = M.MRLMoELayer(s, device_weights(config), train=True)
+    return s, x, dy, bias, layer
+
+
+def _sentinel_grads(cfg):
+    g = M.grad_buffers(cfg)
+    for t in g.values():
+        t.fill_(7.0)
+    return g
+
+
+def test_backward_with_held_loads_times_out_and_writes_nothing():
+    s, x, dy, bias, layer = _train_setup()
+    layer.forward_train(x, bias)
+    ref = {k: v.clone() for k, v in layer.backward(x, dy).items()}
+    assert layer.device_status() == OK
+    layer.forward_train(x, bias)
+    layer.cfg.hold = M.HOLD["gemm"]             # the backward's GEMMs issue no loads
+    g = _sentinel_grads(layer.cfg)
+    t0 = time.monotonic()
+    layer.backward(x, dy, grads=g)
+    status = layer.device_status()
+    dt = time.monotonic() - t0
+    assert status == TIMEOUT, M.status_string(status)
+    assert 1.5 < dt < 60.0, dt
+    for k, t in g.items():                      # the first GEMM timed out; no later kernel wrote
+        assert torch.all(t == 7.0), k
+    layer.cfg.hold = 0
+    layer.forward_train(x, bias)
+    again = layer.backward(x, dy)
+    assert layer.device_status() == OK
+    for k in ref:
+        assert torch.equal(again[k], ref[k]), k
+
+
+def test_backward_after_a_failed_training_forward_does_nothing():
+    # the backward continues the forward's status word: a forward whose
+    # gate/up GEMM timed out leaves the kept activations unwritten, and
+    # every backward kernel then returns without reading them
+    s, x, dy, bias, layer = _train_setup()
+    layer.cfg.hold = M.HOLD["gemm_pair"]
+    layer.forward_train(x, bias)
+    layer.cfg.hold = 0
+    g = _sentinel_grads(layer.cfg)
+    layer.backward(x, dy, grads=g)
+    assert layer.device_status() == TIMEOUT
+    for k, t in g.items():
+        assert torch.all(t == 7.0), k
+
+
+def test_backward_buffers_stay_inside_their_bounds():
+    s, x, dy, bias, layer = _train_setup(T=37)
+    layer.forward_train(x, bias)
+    ref = layer.backward(x, dy)
+    torch.cuda.synchronize()
+    assert layer.device_status() == OK
+    pad = 64
+    bufs, g = {}, {}
+    for name, t in ref.items():
+        it = torch.int16 if t.dtype == torch.bfloat16 else torch.int32
+        canary = CANARY16 if it == torch.int16 else CANARY32
+        buf = torch.full((t.numel() + 2 * pad,), canary, dtype=it, device="cuda")
+        bufs[name] = (buf, canary)
+        g[name] = buf[pad:pad + t.numel()].view(t.dtype).view(t.shape)
+    wsbuf = torch.full((layer.ws_bytes + 4096,), 0xA5, dtype=torch.uint8, device="cuda")
+    wsbuf[:layer.ws_bytes].copy_(layer.workspace)
+    layer.workspace = wsbuf[:layer.ws_bytes]
+    layer.forward_train(x, bias)
+    layer.backward(x, dy, grads=g)
+    assert layer.device_status() == OK
+    torch.cuda.synchronize()
+    for name, (buf, canary) in bufs.items():
+        assert torch.all(buf[:pad] == canary) and torch.all(buf[-pad:] == canary), name
+        assert torch.equal(g[name], ref[name]), name
+    assert torch.all(wsbuf[layer.ws_bytes:] == 0xA5)
