@@ -365,8 +365,8 @@ struct DzPolicy {
 // the next group (or are the TMA zero fill); they are zeroed in shared
 // memory before the MMAs.  A group without rows writes zero tiles.  The fp32
 // tiles leave through TMA stores: each epilogue warp stages its 32 rows x 32
-// columns in a swizzled 4 KB buffer (two per warp, alternating) and one lane
-// issues the bulk store, so the gradient writes go out as whole lines.
+// columns in a swizzled 4 KB buffer (kStoreBufs per warp, in rotation) and one
+// lane issues the bulk store, so the gradient writes go out as whole lines.
 struct WgradPolicy {
   static constexpr bool kAMN = true, kBMN = true, kRaggedK = true;
   static constexpr uint32_t kAMNStride = 8192, kBMNStride = 8192;
@@ -375,7 +375,8 @@ struct WgradPolicy {
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
-  static constexpr int kEpiSmem = 4 * 2 * 4096 + 1024;  // + alignment of the swizzled buffers
+  static constexpr int kStoreBufs = 4;
+  static constexpr int kEpiSmem = 4 * kStoreBufs * 4096 + 1024;  // + alignment of the swizzled buffers
   static constexpr int kAuxSmem = kMaxGroups * 4;
   static constexpr int kUmmaKBytes = 32;
   static constexpr int kASub = 1, kASubBytes = 0;
@@ -484,7 +485,7 @@ struct WgradPolicy {
                                                                                : (sh ? &p.sod : &p.od);
     const int y = (sh ? 0 : g * (which < 2 ? p.F : p.L)) + U.m * 128 + q * 32;
     const uint32_t e0 = smem_u32(epi);
-    const uint32_t bufs = ((e0 + 1023u) & ~1023u) + static_cast<uint32_t>(q) * 8192u;
+    const uint32_t bufs = ((e0 + 1023u) & ~1023u) + static_cast<uint32_t>(q) * (kStoreBufs * 4096u);
     uint8_t *bufp = epi + (bufs - e0);
     const bool empty = U.krows == 0;
     for (int c0 = 0; c0 < U.nv; c0 += 32) {
@@ -496,8 +497,8 @@ struct WgradPolicy {
         tmem_ld32(taddr + c0, v);
         tmem_ld_wait();
       }
-      const int b = st.n & 1;
-      if (lane == 0) bulk_wait_read<1>();  // the store issued two chunks ago has read this buffer
+      const int b = st.n & (kStoreBufs - 1);
+      if (lane == 0) bulk_wait_read<kStoreBufs - 1>();  // this buffer's previous store has read it
       __syncwarp();
       float4 *row = reinterpret_cast<float4 *>(bufp + b * 4096 + lane * 128);
 #pragma unroll
@@ -563,6 +564,7 @@ __global__ void __launch_bounds__(kBwdThreads) rms_combine_bwd_kernel(
       const int i = threadIdx.x + v * kBwdThreads;
       if (i < L4) {
         float4 a = __ldg(base + i);
+#pragma unroll 4
         for (int j = 1; j <= k; ++j) {
           const float4 b = __ldg(base + static_cast<size_t>(j) * L4 + i);
           a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
@@ -648,6 +650,7 @@ __global__ void __launch_bounds__(kBwdThreads) token_bwd_kernel(
   __shared__ float part[kTopKMax * kBwdMaxSlices];
   __shared__ float logit[kTopKMax * kBwdMaxRouters];
   __shared__ float coef[kTopKMax * kBwdMaxRouters];
+  __shared__ float s_sel[kTopKMax], s_dw[kTopKMax], s_w[kTopKMax], s_tot[2];
   __shared__ int eidx[kTopKMax];
   if (call_failed(status)) return;
   const int t = blockIdx.x;
@@ -684,42 +687,46 @@ __global__ void __launch_bounds__(kBwdThreads) token_bwd_kernel(
     if (lane == 0) logit[idx] = a;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float ssel[kTopKMax], dws[kTopKMax];
-    float S = 0.f;
-    for (int j = 0; j < k; ++j) {
-      float sj = 0.f;
-      for (int r = 0; r < R; ++r) {
-        const float pr = sigmoidf_(logit[j * R + r]);
-        sj = agg == 2 ? fmaxf(sj, pr) : sj + pr;
-      }
-      ssel[j] = agg == 0 ? sj / static_cast<float>(R) : sj;
-      S += ssel[j];
-      float d = 0.f;
-      for (int m = 0; m < nsl; ++m) d += part[j * nsl + m];
-      dws[j] = d;
+  // slot j (thread j): its score s_j, dw'_j, aw_j and dw_j
+  if (threadIdx.x < k) {
+    const int j = threadIdx.x;
+    float sj = 0.f;
+    for (int r = 0; r < R; ++r) {
+      const float pr = sigmoidf_(logit[j * R + r]);
+      sj = agg == 2 ? fmaxf(sj, pr) : sj + pr;
     }
-    float swdw = 0.f;
+    s_sel[j] = agg == 0 ? sj / static_cast<float>(R) : sj;
+    float d = 0.f;
+    for (int m = 0; m < nsl; ++m) d += part[j * nsl + m];
+    const float wj = __ldg(topk_w + static_cast<size_t>(t) * k + j);
+    aw[static_cast<size_t>(t) * k + j] = wj * d;
+    s_w[j] = wj;
+    s_dw[j] = d * __ldg(alpha + eidx[j]);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // sums over the slots, in slot order
+    float S = 0.f, swdw = 0.f;
     for (int j = 0; j < k; ++j) {
-      const float wj = __ldg(topk_w + static_cast<size_t>(t) * k + j);
-      aw[static_cast<size_t>(t) * k + j] = wj * dws[j];
-      dws[j] *= __ldg(alpha + eidx[j]);  // dw_j
-      swdw += wj * dws[j];
+      S += s_sel[j];
+      swdw += s_w[j] * s_dw[j];
     }
-    for (int j = 0; j < k; ++j) {
-      const float ds = (dws[j] - swdw) / S;
-      int rmax = 0;
-      if (agg == 2)
-        for (int r = 1; r < R; ++r)
-          if (logit[j * R + r] > logit[j * R + rmax]) rmax = r;
-      for (int r = 0; r < R; ++r) {
-        const float pr = sigmoidf_(logit[j * R + r]);
-        const float dp = agg == 0 ? ds / static_cast<float>(R) : (agg == 1 || r == rmax ? ds : 0.f);
-        const float d = dp * pr * (1.0f - pr);
-        coef[j * R + r] = d;
-        dl[(static_cast<size_t>(t) * k + j) * R + r] = d;
-      }
-    }
+    s_tot[0] = S;
+    s_tot[1] = swdw;
+  }
+  __syncthreads();
+  // (slot j, router r): dl
+  if (threadIdx.x < k * R) {
+    const int j = threadIdx.x / R, r = threadIdx.x - j * R;
+    const float ds = (s_dw[j] - s_tot[1]) / s_tot[0];
+    int rmax = 0;
+    if (agg == 2)
+      for (int q = 1; q < R; ++q)
+        if (logit[j * R + q] > logit[j * R + rmax]) rmax = q;
+    const float pr = sigmoidf_(logit[j * R + r]);
+    const float dp = agg == 0 ? ds / static_cast<float>(R) : (agg == 1 || r == rmax ? ds : 0.f);
+    const float d = dp * pr * (1.0f - pr);
+    coef[j * R + r] = d;
+    dl[(static_cast<size_t>(t) * k + j) * R + r] = d;
   }
   __syncthreads();
   const float *zs = dzs + static_cast<size_t>(t) * (k + 1) * L;
@@ -730,11 +737,13 @@ __global__ void __launch_bounds__(kBwdThreads) token_bwd_kernel(
       const float4 x1 = __ldg(reinterpret_cast<const float4 *>(zs) + 2 * i + 1);
       a[0] = x0.x; a[1] = x0.y; a[2] = x0.z; a[3] = x0.w; a[4] = x1.x; a[5] = x1.y; a[6] = x1.z; a[7] = x1.w;
     }
+#pragma unroll 4
     for (int j = 1; j <= k; ++j) {
       const float4 *src = reinterpret_cast<const float4 *>(zs + static_cast<size_t>(j) * L) + 2 * i;
       const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
       a[0] += x0.x; a[1] += x0.y; a[2] += x0.z; a[3] += x0.w; a[4] += x1.x; a[5] += x1.y; a[6] += x1.z; a[7] += x1.w;
     }
+#pragma unroll 8
     for (int jr = 0; jr < k * R; ++jr) {
       const int j = jr / R, r = jr - j * R;
       const uint4 v = __ldg(reinterpret_cast<const uint4 *>(wr + (static_cast<size_t>(r) * E + eidx[j]) * L) + i);

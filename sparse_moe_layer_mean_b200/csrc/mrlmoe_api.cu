@@ -97,7 +97,7 @@ struct Layout {
 
 // Blocks of rms_combine_bwd_kernel (a fixed number, so the gain gradient's
 // summation order depends on the config alone).
-constexpr int kRmsBwdBlocks = 296;
+constexpr int kRmsBwdBlocks = 592;
 int rms_bwd_blocks(const mrlmoe_config &c) { return std::min(c.T, kRmsBwdBlocks); }
 
 Layout layout_of(const mrlmoe_config &c, bool train = false) {
