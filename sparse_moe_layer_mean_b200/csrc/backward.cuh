@@ -22,6 +22,7 @@
 // with no transposed copy of any weight or activation.
 #pragma once
 #include "policies.cuh"
+#include "gemm2_sm100.cuh"
 
 namespace mrl {
 
@@ -352,6 +353,60 @@ struct DzPolicy {
         if (c0 + c < U.nv) p.dzs[static_cast<size_t>(s_slot[c0 + c]) * p.L + l] = v[c];
     }
     named_bar_sync(2, 128);
+  }
+};
+
+// DzPolicy over a CTA pair (gemm2_kernel): unit = (group, 256-wide d_lat
+// slice, <= 256 rows); CTA r owns d_lat rows m*256 + r*128 .. +127 (its A
+// tile: W_g / W_u MN-major at that offset) and loads half of the unit's dg/du
+// rows, so the rows cross from L2 once per pair.
+struct Dz2Policy {
+  static constexpr bool kAMN = true, kBMN = false;
+  static constexpr uint32_t kAMNStride = 8192, kBMNStride = 0;
+  static constexpr int kStages = 6;
+  static constexpr int kGroup = 2;
+  static constexpr int kBN = 256;
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytesMax = (kBN / 2) * 128;
+  static constexpr int kEpiSmem = DzPolicy::kEpiSmem;
+  static constexpr int kAuxSmem = kGroupAuxSmem;
+  using Params = DzPolicy::Params;  // gt: M tiles per group = d_lat / 256
+  static __device__ __forceinline__ void prefetch(const Params &p) { DzPolicy::prefetch(p); }
+  static __device__ __forceinline__ void stage_aux(const Params &p, uint8_t *aux) { stage_group_table(p.gt, aux); }
+  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *aux) {
+    return grouped_num_units(p.gt, aux);
+  }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return 2 * p.F / kBK; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
+    return grouped_unit(p.gt, aux, u, kBN);
+  }
+  static __device__ __forceinline__ uint32_t b_bytes_pair(const Params &, const Unit &U) {
+    return round32(U.nv) * 128;
+  }
+  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int kb, uint32_t sa,
+                                                uint32_t bar_cl, uint32_t rank) {
+    const bool sh = U.g == p.gt.E;
+    const int fb = p.F / kBK;
+    const bool up = kb >= fb;
+    const CUtensorMap *m = sh ? (up ? &p.su : &p.sg) : (up ? &p.wu : &p.wg);
+    const int x0 = U.m * 256 + static_cast<int>(rank) * 128;
+    const int y = (sh ? 0 : U.g * p.F) + (kb - (up ? fb : 0)) * kBK;
+    tma_load_2d_pair(sa, m, bar_cl, x0, y);
+    tma_load_2d_pair(sa + 8192, m, bar_cl, x0 + 64, y);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb,
+                                                uint32_t bar_cl, uint32_t rank) {
+    load_rows_half(p.tgu, U, kb, sb, bar_cl, rank);
+  }
+  static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U) {
+    return idesc_bf16_major(256, round32(U.nv), true, false);
+  }
+  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, uint32_t taddr, int q, int lane,
+                                                  int etid, uint32_t rank, uint8_t *epi) {
+    Unit V = U;
+    V.m = U.m * 2 + static_cast<int>(rank);  // this CTA's 128-row d_lat slice
+    DzPolicy::EpiState st;
+    DzPolicy::epilogue(p, V, 0, taddr, q, lane, etid, st, epi);
   }
 };
 

@@ -134,7 +134,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint32_t b_s = a_s + P::kABytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_f16_pair(tacc, sdesc_sw128(a_s + kk * 32), sdesc_sw128(b_s + kk * 32), idesc, (kb | kk) != 0);
+            umma_f16_pair(tacc, operand_desc<OperandMajor<P>::a_mn, OperandMajor<P>::a_stride, 32>(a_s, kk),
+                          operand_desc<OperandMajor<P>::b_mn, OperandMajor<P>::b_stride, 32>(b_s, kk), idesc,
+                          (kb | kk) != 0);
           if (s % G == G - 1) umma_commit_pair(empty0 + 8 * (s / G), 0x3);
           if (++s == S) { s = 0; ph ^= 1; }
         }

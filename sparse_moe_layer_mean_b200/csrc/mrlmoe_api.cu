@@ -850,8 +850,10 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
   if (!mark(3)) return MRLMOE_ERR_CUDA;
   // unit tables of the two grouped dgrad GEMMs (token tiles of 256; d_ff / 128 and d_lat / 128 M tiles)
   int32_t *bgo = i32(LT.bgrp_off), *bgc = i32(LT.bgrp_cnt), *bu1 = i32(LT.bunit1), *bu2 = i32(LT.bunit2);
-  expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, DhPolicy::kBN, F / 128, Ld / 128, bgo, bgc, bu1,
-                                            bu2, nullptr, nullptr, P.status);
+  const bool dz_pairs = Ld % 256 == 0;  // the dz GEMM on CTA pairs (256-wide d_lat slices)
+  expert_offsets_kernel<<<1, 1024, 0, st>>>(P.counts_e, T, E, k, DhPolicy::kBN, F / 128,
+                                            dz_pairs ? Ld / 256 : Ld / 128, bgo, bgc, bu1, bu2, nullptr, nullptr,
+                                            P.status);
   MRL_TRY(cudaGetLastError());
   {
     DhPolicy::Params p{};
@@ -875,12 +877,15 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
         !make_map(&p.sg, w->w_sh_gate, 2, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 2, Ld, F, 64) ||
         !make_token_maps_blocked(&p.tgu, dgu, 2 * F, rows))
       return MRLMOE_ERR_CUDA;
-    p.gt = GroupTable{bgo, bgc, bu2, E, Ld / 128};
+    p.gt = GroupTable{bgo, bgc, bu2, E, dz_pairs ? Ld / 256 : Ld / 128};
     p.perm = P.perm;
     p.dzs = P.slots;  // the forward's slots were consumed by rms_combine_bwd_kernel
     p.L = Ld; p.F = F; p.k = k; p.Tk = Tk;
     p.status = P.status;
-    MRL_TRY(launch_gemm<DzPolicy>(p, sms, st));
+    if (dz_pairs)
+      MRL_TRY(launch_gemm_pair<Dz2Policy>(p, sms, st));
+    else
+      MRL_TRY(launch_gemm<DzPolicy>(p, sms, st));
   }
   if (!mark(5)) return MRLMOE_ERR_CUDA;
   // routers, combine weights, alpha; dz reduced per token
