@@ -117,6 +117,27 @@ def test_backward_matches_oracle(config, T, agg):
     _compare(s, grads, ref, experts=experts)
 
 
+EDGE = [  # (overrides of c0_tiny, T)
+    (dict(n_routers=1), 64),                  # one router
+    (dict(n_routers=8), 64),                  # eight routers
+    (dict(top_k=1), 64),                      # k = 1: w = 1, no router gradient
+    (dict(top_k=16), 40),                     # k = E: every expert selected
+    (dict(n_experts=64, top_k=17), 50),       # the wide (32-entry) top-k lists
+    (dict(n_experts=1024, top_k=4), 200),     # most experts without rows (zero gradient tiles)
+]
+
+
+@pytest.mark.parametrize("over,T", EDGE)
+def test_backward_edge_cases(over, T):
+    s = dataclasses.replace(W.CONFIGS["c0_tiny"], T=T, **over)
+    layer, w, x, bias, dy, r, y, grads = _run(s)
+    fc, ref = _oracle(s, w, x, bias, dy)
+    assert torch.equal(r["topk_idx"].cpu().long().view(T, s.top_k), fc.idx)
+    _compare(s, grads, ref)
+    if s.top_k == 1:
+        assert float(grads["d_w_router"].abs().max()) < 1e-6 * float(grads["d_w_gate"].abs().max())
+
+
 def test_training_forward_output_equals_forward():
     s = W.CONFIGS["c0_tiny"].with_T(300)
     w = _weights(s)
