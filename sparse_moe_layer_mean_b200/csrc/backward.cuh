@@ -731,6 +731,7 @@ __global__ void __launch_bounds__(kBwdThreads) token_bwd_kernel(
     const int j = idx / R, r = idx - j * R;
     const uint4 *row = reinterpret_cast<const uint4 *>(wr + (static_cast<size_t>(r) * E + eidx[j]) * L);
     float a = 0.f;
+#pragma unroll 4
     for (int i = lane; i < L8; i += 32) {
       const uint4 v = __ldg(row + i);
       const __nv_bfloat16 *hv = reinterpret_cast<const __nv_bfloat16 *>(&v);
@@ -819,7 +820,7 @@ __global__ void __launch_bounds__(kBwdThreads) token_bwd_kernel(
 // Per expert e (one block): dalpha[e] = sum over e's dispatch rows of aw,
 // dW_router[r, e, :] = sum over e's rows (ascending, as in the dispatch
 // record) of dl[row, r] zx[t(row)].
-__global__ void __launch_bounds__(kBwdThreads) expert_param_bwd_kernel(
+__global__ void __launch_bounds__(kBwdThreads, 2) expert_param_bwd_kernel(
     const int32_t *__restrict__ grp_off, const int32_t *__restrict__ grp_cnt, const int32_t *__restrict__ perm,
     const float *__restrict__ dl, const float *__restrict__ aw, const __nv_bfloat16 *__restrict__ zhi,
     const __nv_bfloat16 *__restrict__ zlo, int L, int E, int R, int k, float *__restrict__ dwr,
@@ -839,6 +840,7 @@ __global__ void __launch_bounds__(kBwdThreads) expert_param_bwd_kernel(
     for (int r = 0; r < kBwdMaxRouters; ++r)
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[r][q] = 0.f;
+#pragma unroll 4
     for (int i = 0; i < n; ++i) {
       const int flat = __ldg(perm + r0 + i);
       const size_t t = static_cast<size_t>(flat / k);
