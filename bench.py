@@ -481,7 +481,8 @@ def run_train(args):
         "roofline": {"kernel": "expert_wgrad (grouped tcgen05 GEMM over ragged token K, fp32 gradients)",
                      "bound": "hbm", "achieved": wg_bytes / (wg_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": wg_bytes / (wg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                     "traffic": None, "algorithmic_bytes": wg_bytes, "peak_kind": f"of {peak_kind}"},
+                     "traffic": profiled_traffic("expert_wgrad", s.name), "algorithmic_bytes": wg_bytes,
+                     "peak_kind": f"of {peak_kind}"},
         "clocks": clk,
         "gpu_launches": (kernels_per_step(s, torch.cuda.get_device_properties(dev).multi_processor_count)
                          + BACKWARD_KERNELS) * args.steps,
