@@ -273,7 +273,7 @@ typedef struct {
 } mrlmoe_grads;
 
 /* Workspace bytes for mrlmoe_forward_train + mrlmoe_backward (0 if cfg is
- * invalid or not bf16).  Beyond mrlmoe_workspace_size: the kept gate/up
+ * invalid, not bf16, or d_ff > 8192).  Beyond mrlmoe_workspace_size: the kept gate/up
  * pre-activations (T*k + T) * d_ff * 4 bytes and the backward's buffers,
  * about (T*k + T) * (2 * d_lat + 2 * d_ff) * 2 bytes more.                    */
 size_t mrlmoe_train_workspace_size(const mrlmoe_config *cfg);
