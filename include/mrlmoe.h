@@ -255,8 +255,10 @@ mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, flo
  * takes the gradient.
  *
  * Gradients: device pointers, caller-owned, all required.  Weight gradients
- * are fp32 with the shapes of mrlmoe_weights (written, not accumulated);
- * dx is bf16 [T, d_model].                                                    */
+ * are fp32 with the shapes of mrlmoe_weights; accumulate = 0 overwrites
+ * them, accumulate != 0 adds this call's gradients to their contents (one
+ * fp32 add per element, e.g. for micro-batches).  dx is bf16 [T, d_model]
+ * and always overwritten.                                                     */
 typedef struct {
   void  *dx;              /* [T, d_model] bf16                                  */
   float *d_w_down;        /* [d_lat, d_model]                                   */
@@ -270,6 +272,7 @@ typedef struct {
   float *d_rms_gain;      /* [d_lat]                                            */
   float *d_w_up;          /* [d_model, d_lat]                                   */
   float *d_expert_scale;  /* [E]                                                */
+  int    accumulate;      /* 0: write the weight gradients; else add to them   */
 } mrlmoe_grads;
 
 /* Workspace bytes for mrlmoe_forward_train + mrlmoe_backward (0 if cfg is

@@ -100,10 +100,12 @@ class MRLMoELayer:
                              stream)
         return y
 
-    def backward(self, x, dy, grads: Optional[Dict[str, object]] = None, stream=None):
-        """Gradients for the last forward_train(x, ...) of this layer."""
+    def backward(self, x, dy, grads: Optional[Dict[str, object]] = None, accumulate: bool = False, stream=None):
+        """Gradients for the last forward_train(x, ...) of this layer; with
+        ``accumulate`` the weight gradients are added to ``grads``."""
         grads = grads if grads is not None else grad_buffers(self.cfg, self.workspace.device)
-        mrlmoe_backward(self.cfg, self.cw, x, dy, make_grads(grads), self.workspace, self.ws_bytes, stream)
+        mrlmoe_backward(self.cfg, self.cw, x, dy, make_grads(grads, accumulate), self.workspace, self.ws_bytes,
+                        stream)
         return grads
 
     def route(self, bias, x=None, routing: Optional[Dict[str, object]] = None,

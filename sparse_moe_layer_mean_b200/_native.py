@@ -77,7 +77,7 @@ GRAD_FIELDS = ("dx", "d_w_down", "d_w_router", "d_w_gate", "d_w_up_e", "d_w_down
 
 
 class Grads(ctypes.Structure):
-    _fields_ = [(n, c_void_p) for n in GRAD_FIELDS]
+    _fields_ = [(n, c_void_p) for n in GRAD_FIELDS] + [("accumulate", c_int)]
 
 
 _lib = None
@@ -222,8 +222,8 @@ def mrlmoe_forward_timed(cfg: Config, weights: Weights, bias, x, y, routing: Opt
            "mrlmoe_forward_timed")
 
 
-def make_grads(g: Dict[str, object]) -> Grads:
-    return Grads(*[_ptr(g.get(n)) for n in GRAD_FIELDS])
+def make_grads(g: Dict[str, object], accumulate: bool = False) -> Grads:
+    return Grads(*[_ptr(g.get(n)) for n in GRAD_FIELDS], int(bool(accumulate)))
 
 
 def mrlmoe_train_workspace_size(cfg: Config) -> int:

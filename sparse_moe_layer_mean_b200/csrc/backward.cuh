@@ -50,6 +50,7 @@ struct DenseGradPolicy {
     void *out;  // fp32 or bf16 [M, ldo]
     long ldo;
     int M, N, K, m_tiles, n_tiles;
+    int accumulate;  // fp32 output: add to it instead of overwriting
     uint32_t *status;
   };
   struct EpiState {};
@@ -106,6 +107,13 @@ struct DenseGradPolicy {
       if (row >= p.M) continue;
       if constexpr (OUTF32) {
         float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + row * p.ldo + U.n0 + c0);
+        if (p.accumulate) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 o = dst[i];
+            v[4 * i] += o.x; v[4 * i + 1] += o.y; v[4 * i + 2] += o.z; v[4 * i + 3] += o.w;
+          }
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
       } else {
@@ -445,6 +453,7 @@ struct WgradPolicy {
     CUtensorMap sog, sou, sod; // shared [F, L], [F, L], [L, F]
     const int32_t *grp_off;  // E + 2 entries
     int E, F, L, rows;
+    int accumulate;          // add the tiles to the gradients (TMA reduce-add) instead of storing
     uint32_t *status;
   };
   struct EpiState {
@@ -562,7 +571,10 @@ struct WgradPolicy {
       fence_proxy_async_shared();
       __syncwarp();
       if (lane == 0) {
-        tma_store_2d(map, bufs + b * 4096, U.n0 + c0, y);
+        if (p.accumulate)
+          tma_reduce_add_2d(map, bufs + b * 4096, U.n0 + c0, y);
+        else
+          tma_store_2d(map, bufs + b * 4096, U.n0 + c0, y);
         bulk_commit();
       }
       ++st.n;
@@ -673,13 +685,13 @@ __global__ void __launch_bounds__(kBwdThreads) rms_combine_bwd_kernel(
 
 // dgain[l] = sum over blocks b (in order) of gpart[b][l].
 __global__ void gain_reduce_kernel(const float *__restrict__ gpart, int nb, int L, float *__restrict__ dgain,
-                                   const uint32_t *status) {
+                                   int accumulate, const uint32_t *status) {
   if (call_failed(status)) return;
   const int l = blockIdx.x * blockDim.x + threadIdx.x;
   if (l >= L) return;
   float a = 0.f;
   for (int b = 0; b < nb; ++b) a += __ldg(gpart + static_cast<size_t>(b) * L + l);
-  dgain[l] = a;
+  dgain[l] = accumulate ? dgain[l] + a : a;
 }
 
 constexpr int kBwdMaxSlices = 64;  // d_ff / 128 at d_ff <= 8192
@@ -824,7 +836,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) expert_param_bwd_kernel(
     const int32_t *__restrict__ grp_off, const int32_t *__restrict__ grp_cnt, const int32_t *__restrict__ perm,
     const float *__restrict__ dl, const float *__restrict__ aw, const __nv_bfloat16 *__restrict__ zhi,
     const __nv_bfloat16 *__restrict__ zlo, int L, int E, int R, int k, float *__restrict__ dwr,
-    float *__restrict__ dalpha, const uint32_t *status) {
+    float *__restrict__ dalpha, int accumulate, const uint32_t *status) {
   __shared__ float red[kBwdThreads / 32];
   if (call_failed(status)) return;
   const int e = blockIdx.x;
@@ -832,7 +844,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) expert_param_bwd_kernel(
   float a = 0.f;
   for (int i = threadIdx.x; i < n; i += kBwdThreads) a += __ldg(aw + __ldg(perm + r0 + i));
   a = block_sum(a, red);
-  if (threadIdx.x == 0) dalpha[e] = a;
+  if (threadIdx.x == 0) dalpha[e] = accumulate ? dalpha[e] + a : a;
   const int L8 = L >> 3;
   for (int c = threadIdx.x; c < L8; c += kBwdThreads) {
     float acc[kBwdMaxRouters][8];
@@ -864,6 +876,11 @@ __global__ void __launch_bounds__(kBwdThreads, 2) expert_param_bwd_kernel(
     for (int r = 0; r < kBwdMaxRouters; ++r) {
       if (r < R) {
         float4 *dst = reinterpret_cast<float4 *>(dwr + (static_cast<size_t>(r) * E + e) * L + 8 * c);
+        if (accumulate) {
+          const float4 o0 = dst[0], o1 = dst[1];
+          acc[r][0] += o0.x; acc[r][1] += o0.y; acc[r][2] += o0.z; acc[r][3] += o0.w;
+          acc[r][4] += o1.x; acc[r][5] += o1.y; acc[r][6] += o1.z; acc[r][7] += o1.w;
+        }
         dst[0] = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
         dst[1] = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
       }

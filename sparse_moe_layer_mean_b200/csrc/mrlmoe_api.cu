@@ -778,8 +778,9 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
 // ------------------------------------------------------------ backward
 template <class DP>
 mrlmoe_status launch_dense_grad(const CUtensorMap &ta, const CUtensorMap &tb, void *out, int M, int N, int K,
-                                uint32_t *status, int sms, cudaStream_t st) {
+                                uint32_t *status, int sms, cudaStream_t st, int accumulate = 0) {
   typename DP::Params p{};
+  p.accumulate = accumulate;
   p.ta = ta;
   p.tb = tb;
   p.out = out;
@@ -816,6 +817,7 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
   uint8_t *b = static_cast<uint8_t *>(workspace);
   const int T = cfg->T, D = cfg->d_model, Ld = cfg->d_lat, F = cfg->d_ff, E = cfg->n_experts, k = cfg->top_k;
   const int R = cfg->n_routers, Tk = T * k, rows = Tk + T;
+  const int acc = g->accumulate != 0;  // weight gradients: add instead of overwrite
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16 *>(b + off); };
   auto f32 = [&](size_t off) { return reinterpret_cast<float *>(b + off); };
   auto i32 = [&](size_t off) { return reinterpret_cast<int32_t *>(b + off); };
@@ -840,8 +842,8 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
       return s;
     if (!mark(1)) return MRLMOE_ERR_CUDA;
     if (!make_map(&ta, dy, 2, D, T, 64) || !make_map(&tb, P.nbuf, 2, Ld, T, 64)) return MRLMOE_ERR_CUDA;
-    if ((s = launch_dense_grad<DenseGradPolicy<true, true, true>>(ta, tb, g->d_w_up, D, Ld, T, P.status, sms, st)) !=
-        MRLMOE_OK)
+    if ((s = launch_dense_grad<DenseGradPolicy<true, true, true>>(ta, tb, g->d_w_up, D, Ld, T, P.status, sms, st,
+                                                                    acc)) != MRLMOE_OK)
       return s;
   }
   if (!mark(2)) return MRLMOE_ERR_CUDA;
@@ -855,7 +857,7 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
                                      cfg->rms_eps, dcd, dod, wrow, reinterpret_cast<float4 *>(gpart), P.status);
   }
   MRL_TRY(cudaGetLastError());
-  gain_reduce_kernel<<<(Ld + 255) / 256, 256, 0, st>>>(gpart, nb, Ld, g->d_rms_gain, P.status);
+  gain_reduce_kernel<<<(Ld + 255) / 256, 256, 0, st>>>(gpart, nb, Ld, g->d_rms_gain, acc, P.status);
   MRL_TRY(cudaGetLastError());
   if (!mark(3)) return MRLMOE_ERR_CUDA;
   // unit tables of the two grouped dgrad GEMMs (token tiles of 256; d_ff / 128 and d_lat / 128 M tiles)
@@ -906,7 +908,7 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
   MRL_TRY(cudaGetLastError());
   if (!mark(6)) return MRLMOE_ERR_CUDA;
   expert_param_bwd_kernel<<<E, kBwdThreads, 0, st>>>(P.grp_off, P.grp_cnt, P.perm, dl, aw, zhi, P.zlo, Ld, E, R, k,
-                                                     g->d_w_router, g->d_expert_scale, P.status);
+                                                     g->d_w_router, g->d_expert_scale, acc, P.status);
   MRL_TRY(cudaGetLastError());
   if (!mark(7)) return MRLMOE_ERR_CUDA;
   // expert weight gradients (K = each group's rows)
@@ -922,6 +924,7 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
         !make_map_f32_out(&p.sou, g->d_w_sh_up, Ld, F) || !make_map_f32_out(&p.sod, g->d_w_sh_down, F, Ld))
       return MRLMOE_ERR_CUDA;
     p.grp_off = P.grp_off;
+    p.accumulate = acc;
     p.E = E; p.F = F; p.L = Ld; p.rows = rows;
     p.status = P.status;
     MRL_TRY(launch_gemm<WgradPolicy>(p, sms, st));
@@ -937,7 +940,7 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
     if (!mark(9)) return MRLMOE_ERR_CUDA;
     if (!make_map(&ta, dzx, 2, Ld, T, 64) || !make_map(&tb, x, 2, D, T, 64)) return MRLMOE_ERR_CUDA;
     if ((s = launch_dense_grad<DenseGradPolicy<true, true, true>>(ta, tb, g->d_w_down, Ld, D, T, P.status, sms,
-                                                                    st)) != MRLMOE_OK)
+                                                                    st, acc)) != MRLMOE_OK)
       return s;
   }
   if (!mark(10)) return MRLMOE_ERR_CUDA;

@@ -188,3 +188,24 @@ def test_backward_rejects_fp8_and_small_workspace():
     with pytest.raises(M.MrlmoeError):
         M.mrlmoe_backward(layer.cfg, layer.cw, x, W.make_dy(s, "cuda"), M.make_grads(M.grad_buffers(layer.cfg)),
                           layer.workspace, layer.ws_bytes)
+
+
+@pytest.mark.parametrize("config,T", [("c0_tiny", 300), ("c2_prefill", 64)])
+def test_accumulated_gradients_add_up(config, T):
+    # zeroed buffers, two accumulating calls = twice the written gradients,
+    # bit for bit (g + g is exact in fp32); dx is overwritten each time
+    s = W.CONFIGS[config].with_T(T)
+    layer, w, x, bias, dy, r, y, g1 = _run(s)
+    g1 = {k: v.clone() for k, v in g1.items()}
+    acc = M.grad_buffers(layer.cfg)
+    for t in acc.values():
+        t.zero_()
+    for _ in range(2):
+        layer.forward_train(x, bias)
+        layer.backward(x, dy, grads=acc, accumulate=True)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert torch.equal(acc["dx"], g1["dx"])
+    for k in g1:
+        if k != "dx":
+            assert torch.equal(acc[k], 2 * g1[k]), k
