@@ -172,7 +172,7 @@ struct DhPolicy {
   static constexpr int kBN = 256;
   static constexpr int kABytes = 128 * 128;
   static constexpr int kBBytesMax = kBN * 128;
-  static constexpr int kEpiSmem = kBN * 8 + 4 * kBN * 4;
+  static constexpr int kEpiSmem = kBN * 4 + 4 * kBN * 4;  // row weights, per-warp partial sums
   static constexpr int kAuxSmem = kGroupAuxSmem;
   static constexpr int kUmmaKBytes = 32;
   static constexpr int kASub = 1, kASubBytes = 0;
@@ -222,8 +222,8 @@ struct DhPolicy {
   // consecutive f of one K-blocked plane (64 contiguous bytes of g, u, h).
   static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
                                                   int lane, int etid, EpiState &, uint8_t *epi) {
-    float *s_ws = reinterpret_cast<float *>(epi + kBN * 4);
-    float *red = reinterpret_cast<float *>(epi + kBN * 8);  // [4][kBN]
+    float *s_ws = reinterpret_cast<float *>(epi);
+    float *red = reinterpret_cast<float *>(epi + kBN * 4);  // [4][kBN]
     for (int c = etid; c < U.nv; c += 128) s_ws[c] = __ldg(p.wrow + U.row0 + c);
     named_bar_sync(2, 128);
     const int f = U.m * 128 + q * 32 + lane;
@@ -721,7 +721,6 @@ __global__ void __launch_bounds__(kBwdThreads) token_bwd_kernel(
   __shared__ int eidx[kTopKMax];
   if (call_failed(status)) return;
   const int t = blockIdx.x;
-  const size_t Tk = static_cast<size_t>(T) * k;
   const int L8 = L >> 3;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < L8; i += kBwdThreads) {
