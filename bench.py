@@ -72,6 +72,8 @@ def parse_args():
     ap.add_argument("--aggregation", choices=["mean", "sum", "max"], default=None,
                     help="router score aggregation (default: the config's, the mean)")
     ap.add_argument("--routers", type=int, default=None, help="override the number of routers R")
+    ap.add_argument("--no-train-summary", action="store_true",
+                    help="leave the training-step summary out of the forward's line")
     ap.add_argument("--train", action="store_true",
                     help="time a training step (forward that keeps its activations + backward) instead")
     ap.add_argument("--route-only", action="store_true",
@@ -380,6 +382,80 @@ def train_flops(s):
     return 3 * W.flops_per_token(s) * s.T
 
 
+def _time_training(layer, x, bias, dy, cg, steps, warmup, clocks=None):
+    """Warm-up, then `steps` training steps (forward_train + backward) between
+    CUDA events on the current stream; returns (total ms, mean forward_train
+    ms, mean ms of each backward stage)."""
+    import torch
+    import sparse_moe_layer_mean_b200 as M
+    y = torch.empty(layer.cfg.T, layer.cfg.d_model, dtype=torch.bfloat16, device=x.device)
+    for _ in range(max(3, warmup)):
+        layer.forward_train(x, bias, y=y)
+        M.mrlmoe_backward(layer.cfg, layer.cw, x, dy, cg, layer.workspace, layer.ws_bytes)
+    torch.cuda.synchronize()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status non-zero after warm-up")
+    NB = M._native.NUM_BACKWARD_EVENTS
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NB + 1)] for _ in range(steps)]
+    for row in evs:
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+    if clocks is not None:
+        time.sleep(0.6)
+        clocks.begin()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        evs[i][0].record()
+        layer.forward_train(x, bias, y=y)
+        M.mrlmoe_backward_timed(layer.cfg, layer.cw, x, dy, cg, layer.workspace, layer.ws_bytes, evs[i][1:])
+    stop.record()
+    torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.end()
+    if layer.device_status() != 0:
+        raise RuntimeError("device status non-zero after the timed region")
+    ms = start.elapsed_time(stop)
+    fwd_ms = sum(r[0].elapsed_time(r[1]) for r in evs) / steps
+    stage = [sum(r[j + 1].elapsed_time(r[j + 2]) for r in evs) / steps for j in range(NB - 1)]
+    return ms, fwd_ms, stage
+
+
+def train_summary(s, dev, weights, x, bias, steps=10, warmup=3):
+    """The training step (forward_train + backward) on the same workload,
+    timed on its own after the forward's timed region: a summary object for
+    the forward's JSON line."""
+    import torch
+    import sparse_moe_layer_mean_b200 as M
+    import workloads as W
+    try:
+        w = dict(weights)
+        w["rms_gain"] = W.make_train_gain(s, dev)
+        dy = W.make_dy(s, dev)
+        layer = M.MRLMoELayer(s, w, device=dev, train=True)
+        grads = M.grad_buffers(layer.cfg, dev)
+        ms, fwd_ms, stage = _time_training(layer, x, bias, dy, M.make_grads(grads), steps, warmup)
+        peaks, peak_kind = load_peaks()
+        wg_ms = stage[M._native.BACKWARD_STAGES.index("expert_wgrad")]
+        wg_bytes = wgrad_kernel_bytes(s)
+        out = {"metric": "training step (forward_train + backward) tokens/s", "value": s.T * steps / (ms * 1e-3),
+               "unit": UNIT, "ms_per_step": ms / steps, "steps": steps, "warmup": max(3, warmup),
+               "forward_train_ms": round(fwd_ms, 4), "backward_ms": round(sum(stage), 4),
+               "backward_stage_ms": dict(zip(M._native.BACKWARD_STAGES, [round(v, 4) for v in stage])),
+               "roofline": {"kernel": "expert_wgrad", "bound": "hbm",
+                            "achieved": wg_bytes / (wg_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": wg_bytes / (wg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                            "traffic": profiled_traffic("expert_wgrad", s.name), "peak_kind": f"of {peak_kind}"},
+               "gpu_launches": BACKWARD_KERNELS * steps,
+               "note": "python bench.py --train gives the full line (e2e, clocks, CPU baseline)"}
+        del layer, grads
+        torch.cuda.empty_cache()
+        return out
+    except Exception as e:  # the forward's line is printed either way
+        return {"error": str(e).splitlines()[0][:200] if str(e) else type(e).__name__}
+
+
 def run_train(args):
     """--train: one step = mrlmoe_forward_train + mrlmoe_backward over one batch
     (fp32 weight gradients of every expert, bf16 dx)."""
@@ -403,37 +479,10 @@ def run_train(args):
     y = torch.empty(s.T, s.d_model, dtype=torch.bfloat16, device=dev)
     grads = M.grad_buffers(layer.cfg, dev)
     cg = M.make_grads(grads)
-    for _ in range(max(3, args.warmup)):
-        layer.forward_train(x, bias, y=y)
-        M.mrlmoe_backward(layer.cfg, layer.cw, x, dy, cg, layer.workspace, layer.ws_bytes)
-    torch.cuda.synchronize()
-    if layer.device_status() != 0:
-        raise RuntimeError("device status non-zero after warm-up")
-    NB = M._native.NUM_BACKWARD_EVENTS
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NB + 1)] for _ in range(args.steps)]
-    for row in evs:
-        for e in row:
-            e.record()
-    torch.cuda.synchronize()
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     clocks = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
-    time.sleep(0.6)
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks.begin()
-    start.record()
-    for i in range(args.steps):
-        evs[i][0].record()
-        layer.forward_train(x, bias, y=y)
-        M.mrlmoe_backward_timed(layer.cfg, layer.cw, x, dy, cg, layer.workspace, layer.ws_bytes, evs[i][1:])
-    stop.record()
-    torch.cuda.synchronize()
-    clocks.end()
+    ms, fwd_ms, stage = _time_training(layer, x, bias, dy, cg, args.steps, args.warmup, clocks)
     clk = clocks.stop()
-    if layer.device_status() != 0:
-        raise RuntimeError("device status non-zero after the timed region")
-    ms = start.elapsed_time(stop)
-    fwd_ms = sum(r[0].elapsed_time(r[1]) for r in evs) / args.steps
-    stage = [sum(r[j + 1].elapsed_time(r[j + 2]) for r in evs) / args.steps for j in range(NB - 1)]
     bwd_ms = sum(stage)
 
     # e2e: x and dy from pinned host memory, the step, dx back to pinned host memory, every step
@@ -725,6 +774,8 @@ def main():
             line["config"]["e4m3_peak_probe"] = fp8_peak_probe(dev)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(s, weights, x, bias, min(args.cpu_sample, s.T))
+        if world == 1 and not s.fp8 and not args.no_train_summary:
+            line["train_step"] = train_summary(s, dev, weights, x, bias)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier(device_ids=[local])
