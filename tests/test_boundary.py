@@ -206,3 +206,11 @@ def test_training_entry_points_reject_bad_arguments_before_cuda():
                                    None, ev, N.NUM_BACKWARD_EVENTS - 1) == 1
     assert L.mrlmoe_backward_timed(ctypes.byref(cfg), ctypes.byref(w), 4096, 4096, ctypes.byref(g), 4096, train,
                                    None, None, N.NUM_BACKWARD_EVENTS) == 1
+
+
+def test_gradient_fields_cover_every_learnable_tensor():
+    from oracle import mrlmoe_backward as OB
+    # dx -> x, d_<name> -> <name>: the same twelve tensors as the oracle's backward
+    assert sorted("x" if f == "dx" else f[2:] for f in N.GRAD_FIELDS) == sorted(OB.GRAD_NAMES)
+    # and the C struct: twelve pointers then the accumulate flag
+    assert [n for n, _ in N.Grads._fields_] == list(N.GRAD_FIELDS) + ["accumulate"]

@@ -204,3 +204,16 @@ def test_gradient_descent_lowers_the_loss():
     losses = _train_loop_oracle(12)
     assert all(b < a for a, b in zip(losses, losses[1:])), losses
     assert losses[-1] < 0.2 * losses[0], losses
+
+
+def test_expert_subset_equals_the_full_gradients():
+    # the memory-saving `experts` option computes the same numbers, stacked in the given order
+    x, w, bias, dy = _params(T=6, E=8, seed=9)
+    fc = B.forward_for_grad(x, w, bias, 2, round_points=False)
+    full = B.backward(fc, w, dy, 2)
+    pick = [5, 0, 3, 7]
+    sub = B.backward(fc, w, dy, 2, experts=pick)
+    for nm in ("w_gate", "w_up_e", "w_down_e"):
+        assert torch.equal(sub[nm], full[nm][pick]), nm
+    for nm in set(B.GRAD_NAMES) - {"w_gate", "w_up_e", "w_down_e"}:
+        assert torch.equal(sub[nm], full[nm]), nm
