@@ -1,5 +1,6 @@
 /*
- * mrlmoe.h — C ABI of the Multi-Router Latent MoE layer forward pass (sm_100a).
+ * mrlmoe.h — C ABI of the Multi-Router Latent MoE layer (sm_100a): the forward
+ * pass, its balancing-bias update, and the backward pass for training.
  *
  * The layer (ERNIE 5.5 Flash release pages: blog.derekhsu.net "ERNIE-5.5-Flash-Base"
  * translation, section "多路由潛在 MoE (Multi-Router Latent MoE)"; aitest123.com

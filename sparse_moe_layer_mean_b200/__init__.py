@@ -1,4 +1,5 @@
-"""Multi-Router Latent MoE layer forward for B200 (sm_100a).
+"""Multi-Router Latent MoE layer for B200 (sm_100a): forward, balancing-bias
+update and backward.
 
 The compute lives in libmrlmoe.so (CUDA, C ABI in include/mrlmoe.h); this
 package is its binding.  ``MRLMoELayer`` bundles a config, device weights
