@@ -83,3 +83,28 @@ def check_dispatch_properties(r, T: int, E: int, k: int):
     tok = perm // k
     same = e_of_row[1:] == e_of_row[:-1]
     assert torch.all(tok[1:][same] > tok[:-1][same])
+
+
+def train_loop_oracle(steps, lr=7.8125e-4, gamma=1e-3):
+    """SGD on fp32 master weights (bf16 copies in the forward, as the layer
+    stores them) towards a teacher layer's output, with the balancing-bias
+    update after every step; returns the loss of each step."""
+    from oracle import mrlmoe_backward as B
+    s = W.CONFIGS["c0_tiny"]
+    bf = lambda w: {k: v.to(torch.bfloat16) if v.dim() > 1 else v.float() for k, v in w.items()}
+    master = {k: v.double() for k, v in W.make_weights(s, "cpu").items()}
+    teacher = bf({k: v.double() for k, v in W.make_weights(s, "cpu", seed=5).items()})
+    x = W.make_x(s, "cpu")
+    bias = torch.zeros(s.n_experts)
+    target = B.forward_for_grad(x, teacher, bias, s.top_k).y
+    losses = []
+    for _ in range(steps):
+        w = bf(master)
+        fc = B.forward_for_grad(x, w, bias, s.top_k)
+        d = fc.y - target
+        losses.append(0.5 * float((d * d).mean()))
+        g = B.backward(fc, w, d.to(torch.bfloat16), s.top_k)
+        for k in master:
+            master[k] -= lr * g[k]
+        bias = O.bias_update(bias, torch.bincount(fc.idx.flatten(), minlength=s.n_experts), s.T, s.top_k, gamma)
+    return losses

@@ -2,7 +2,7 @@
 backward, an SGD step on fp32 master weights (their bf16 copies are what the
 layer reads) and the balancing-bias update from the step's expert counts.
 The loss falls at every step and follows the oracle's loop
-(tests/test_oracle_backward.py, same teacher target, learning rate and
+(helpers.train_loop_oracle, same teacher target, learning rate and
 bias step) to within the drift that bf16 gradients accumulate."""
 import pytest
 import torch
@@ -10,7 +10,7 @@ import torch
 import sparse_moe_layer_mean_b200 as M
 import workloads as W
 from oracle import mrlmoe_backward as B
-from test_oracle_backward import _train_loop_oracle
+from helpers import train_loop_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -45,7 +45,7 @@ def test_training_loop_lowers_the_loss_and_follows_the_oracle():
             master[k] -= LR * g["d_" + k]
             w[k].copy_(master[k])          # in place: the layer keeps its pointers
         assert layer.device_status() == 0
-    ref = _train_loop_oracle(STEPS, LR, GAMMA)
+    ref = train_loop_oracle(STEPS, LR, GAMMA)
     print([f"{a:.4f}/{b:.4f}" for a, b in zip(losses, ref)])
     assert all(b < a for a, b in zip(losses, losses[1:])), losses
     assert losses[-1] < 0.2 * losses[0], losses

@@ -15,6 +15,7 @@ do not share its arithmetic:
 import pytest
 import torch
 
+from helpers import train_loop_oracle
 from oracle import mrlmoe_backward as B
 from oracle import mrlmoe_oracle as O
 
@@ -174,34 +175,9 @@ def test_kept_forward_matches_the_forward_oracle():
     assert torch.allclose(fc.y, ref.y, rtol=2 ** -6, atol=1e-3)
 
 
-def _train_loop_oracle(steps, lr=7.8125e-4, gamma=1e-3):
-    """SGD on fp32 master weights (bf16 copies in the forward, as the layer
-    stores them) towards a teacher layer's output, with the balancing-bias
-    update after every step; returns the loss of each step."""
-    import workloads as W
-    s = W.CONFIGS["c0_tiny"]
-    bf = lambda w: {k: v.to(torch.bfloat16) if v.dim() > 1 else v.float() for k, v in w.items()}
-    master = {k: v.double() for k, v in W.make_weights(s, "cpu").items()}
-    teacher = bf({k: v.double() for k, v in W.make_weights(s, "cpu", seed=5).items()})
-    x = W.make_x(s, "cpu")
-    bias = torch.zeros(s.n_experts)
-    target = B.forward_for_grad(x, teacher, bias, s.top_k).y
-    losses = []
-    for _ in range(steps):
-        w = bf(master)
-        fc = B.forward_for_grad(x, w, bias, s.top_k)
-        d = fc.y - target
-        losses.append(0.5 * float((d * d).mean()))
-        g = B.backward(fc, w, d.to(torch.bfloat16), s.top_k)
-        for k in master:
-            master[k] -= lr * g[k]
-        bias = O.bias_update(bias, torch.bincount(fc.idx.flatten(), minlength=s.n_experts), s.T, s.top_k, gamma)
-    return losses
-
-
 def test_gradient_descent_lowers_the_loss():
     # the oracle's gradients, used as a training step, lower the loss at every step
-    losses = _train_loop_oracle(12)
+    losses = train_loop_oracle(12)
     assert all(b < a for a, b in zip(losses, losses[1:])), losses
     assert losses[-1] < 0.2 * losses[0], losses
 
