@@ -1,4 +1,6 @@
-"""CPU oracle for the Multi-Router Latent MoE layer forward pass.
+"""CPU oracle for the Multi-Router Latent MoE layer: the forward pass
+(mrlmoe_oracle), its backward (mrlmoe_backward) and its expert-parallel form
+(mrlmoe_ep).
 
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  The product path
