@@ -193,3 +193,49 @@ def test_expert_subset_equals_the_full_gradients():
         assert torch.equal(sub[nm], full[nm][pick]), nm
     for nm in set(B.GRAD_NAMES) - {"w_gate", "w_up_e", "w_down_e"}:
         assert torch.equal(sub[nm], full[nm]), nm
+
+
+def _autograd_loss(x, w, idx, top_k, eps, aggregation):
+    """The layer written again, densely (every expert on every token, masked
+    by the given selection), differentiable by torch.autograd; fp64, no
+    rounding points."""
+    zx = x @ w["w_down"].T
+    logits = torch.einsum("tl,rel->rte", zx, w["w_router"])
+    p = torch.sigmoid(logits)
+    if aggregation == "mean":
+        s = p.mean(0)
+    elif aggregation == "sum":
+        s = p.sum(0)
+    else:
+        s = p.max(0).values
+    T, E = s.shape
+    mask = torch.zeros(T, E, dtype=F64)
+    mask.scatter_(1, idx, 1.0)
+    ssel = s * mask
+    wts = ssel / ssel.sum(1, keepdim=True) * w["expert_scale"][None, :]   # zero off the selection
+    g = torch.einsum("tl,efl->tef", zx, w["w_gate"])
+    u = torch.einsum("tl,efl->tef", zx, w["w_up_e"])
+    o = torch.einsum("tef,elf->tel", torch.nn.functional.silu(g) * u, w["w_down_e"])
+    c = (o * wts[:, :, None]).sum(1)
+    gs, us = zx @ w["w_sh_gate"].T, zx @ w["w_sh_up"].T
+    c = c + (torch.nn.functional.silu(gs) * us) @ w["w_sh_down"].T
+    n = c * torch.rsqrt((c * c).mean(1, keepdim=True) + eps) * w["rms_gain"][None, :]
+    return n @ w["w_up"].T
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_matches_automatic_differentiation(case):
+    T, D, L, E, F, R, k, agg, seed = case
+    x, w, bias, dy = _params(T, D, L, E, F, R, seed)
+    eps = 1e-6
+    fc = B.forward_for_grad(x, w, bias, k, rms_eps=eps, aggregation=agg, round_points=False)
+    grads = B.backward(fc, w, dy, k, aggregation=agg)
+    xa = x.clone().requires_grad_(True)
+    wa = {n: t.clone().requires_grad_(True) for n, t in w.items()}
+    y = _autograd_loss(xa, wa, fc.idx, k, eps, agg)
+    assert torch.allclose(y, fc.y, rtol=1e-12, atol=1e-12)
+    (y * dy).sum().backward()
+    for name in B.GRAD_NAMES:
+        ref = xa.grad if name == "x" else wa[name].grad
+        d = (grads[name] - ref).abs().max().item()
+        assert d <= 1e-10 * max(1.0, ref.abs().max().item()), (name, d)
