@@ -2,6 +2,7 @@
 // descriptor set-up and the launch sequence of the layer on the caller's stream.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstdint>
 #include <cstring>
@@ -20,6 +21,36 @@ using namespace mrl;
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------ NVTX ranges
+// One range per call of an entry point and, inside it, one per stage (the
+// stages that the *_timed entry points time with events), so a profiler can
+// attribute or filter kernels by stage.  Host-side only: no-ops unless a
+// profiling tool is attached, and invisible to a CUDA graph capture.
+thread_local bool t_stage_open = false;
+
+void nvtx_stage(const char *name) {
+  if (t_stage_open) nvtxRangePop();
+  t_stage_open = name != nullptr;
+  if (name) nvtxRangePushA(name);
+}
+
+struct NvtxCall {
+  explicit NvtxCall(const char *name) {
+    nvtxRangePushA(name);
+    t_stage_open = false;
+  }
+  ~NvtxCall() {
+    nvtx_stage(nullptr);
+    nvtxRangePop();
+  }
+};
+
+constexpr const char *kForwardStages[8] = {"down_proj",   "router_topk", "dispatch",        "gather",
+                                           "gate_up_glu", "expert_down", "combine_rmsnorm", "up_proj"};
+constexpr const char *kBackwardStages[10] = {"dn", "dw_up", "rms_combine_bwd", "dh_glu_bwd", "dz",
+                                             "token_router_bwd", "dw_router_alpha", "expert_wgrad", "dx",
+                                             "dw_down"};
 
 // ------------------------------------------------------------ validation
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -541,6 +572,7 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
     mrlmoe_status s = launch_dense_bf16(x, w->w_down, z, P.zlo, T, Ld, D, P.status, sms, st);
     if (s != MRLMOE_OK) return s;
   }
+  nvtx_stage(kForwardStages[1]);
   if (ev) MRL_TRY(cudaEventRecord(static_cast<cudaEvent_t>(ev[1]), st));
   {
     RouterParams p{};
@@ -628,7 +660,9 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   const Layout LT = layout_of(*cfg, train);
   const int Tk = T * k;
   if ((s = init_header(P.status, cfg->hold, st)) != MRLMOE_OK) return s;
+  NvtxCall nvtx_call(train ? "mrlmoe_forward_train" : "mrlmoe_forward");
   auto mark = [&](int i) -> bool {
+    nvtx_stage(i < 8 ? kForwardStages[i] : nullptr);
     return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
   };
 
@@ -713,6 +747,7 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
   const int T = c.T, D = c.d_model, Ld = c.d_lat, F = c.d_ff, E = c.n_experts, k = c.top_k;
   const int Tk = T * k;
   auto mark = [&](int i) -> bool {
+    nvtx_stage(i < 8 ? kForwardStages[i] : nullptr);
     return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
   };
   // quantised dispatched latent rows (rows < T*k) and the shared expert's rows (all T tokens)
@@ -826,7 +861,9 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
   __nv_bfloat16 *dgu = bf(LT.dgu), *dzx = bf(LT.dzx);
   float *dn = f32(LT.dn), *dwsp = f32(LT.dwsp), *wrow = f32(LT.wrow), *dl = f32(LT.dl), *aw = f32(LT.aw), *gpart = f32(LT.gpart);
   const __nv_bfloat16 *zhi = P.zbuf + static_cast<size_t>(Tk) * Ld;
+  NvtxCall nvtx_call("mrlmoe_backward");
   auto mark = [&](int i) -> bool {
+    nvtx_stage(i < 10 ? kBackwardStages[i] : nullptr);
     return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
   };
   // the call continues the forward's status word; only this call's hold mask is set
@@ -1039,6 +1076,7 @@ mrlmoe_status mrlmoe_route(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ptrs P = carve(*cfg, workspace, out);
   if ((s = init_header(P.status, cfg->hold, st)) != MRLMOE_OK) return s;
+  NvtxCall nvtx_call("mrlmoe_route");
   if (scores_in) {
     MRL_TRY(launch_topk_from_scores(out->scores, bias, w->expert_scale, cfg->T, cfg->n_experts, cfg->top_k,
                                     P.topk_idx, P.topk_w, P.wscaled, P.status, st));
