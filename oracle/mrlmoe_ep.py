@@ -1,4 +1,5 @@
-"""Expert-parallel form of the layer forward, plain CPU reference.
+"""Expert-parallel form of the layer (forward, and the backward of a training
+step), plain CPU reference.
 
 TEST INFRASTRUCTURE ONLY, like the rest of this package.
 
@@ -41,7 +42,7 @@ from .mrlmoe_oracle import (_as_f64, bf16_round, expert_glu, permutation, rmsnor
 F64 = torch.float64
 
 __all__ = ["owned_range", "RankRecord", "route_and_dispatch", "send_buffers", "run_local_experts", "combine",
-           "ep_forward", "exchange_bytes"]
+           "ep_forward", "exchange_bytes", "ep_backward"]
 
 
 def owned_range(E: int, n_ranks: int, d: int) -> Tuple[int, int]:
@@ -163,3 +164,138 @@ def exchange_bytes(recs: Sequence[RankRecord], n_ranks: int, width: int, elem_by
             else:
                 remote += rows.shape[0]
     return {"remote_rows": remote, "local_rows": local, "bytes": remote * width * elem_bytes}
+
+
+# ---------------------------------------------------------------------------
+# backward (training step) in the expert-parallel layout
+# ---------------------------------------------------------------------------
+def ep_backward(xs: Sequence[torch.Tensor], dys: Sequence[torch.Tensor], weights: Dict[str, torch.Tensor],
+                bias: torch.Tensor, top_k: int, rms_eps: float = 1e-6, aggregation: str = "mean"):
+    """Gradients of sum_r <y_r, dy_r> with every rank holding its own tokens.
+
+    Exchange plan (the forward's, run backwards): each token's rank computes
+    dc (the RMSNorm and combine backward are per token) and sends, for every
+    dispatch row, dc of the row's token and the row's weight w' to the
+    expert's owner, in the same slices as the forward's latent rows.  The
+    owner, from what it received (the forward's z rows and these), forms
+    dh' = dc W_d, dw' = <h, dh'>, dg, du and dz = dg W_g + du W_u per row,
+    accumulates its experts' weight gradients over all sources, and returns
+    dz and dw' per row.  The token's rank finishes the router and alpha terms
+    and dx.  Replicated tensors (projections, routers, gain, alpha, shared
+    expert) get one partial gradient per rank, summed here as an all-reduce
+    would; the routed experts' gradients are complete on their owner.
+
+    Returns (per-rank dx list, dict of the summed gradients)."""
+    from .mrlmoe_backward import forward_for_grad
+
+    n = len(xs)
+    f64 = lambda t: _as_f64(t)
+    E = weights["expert_scale"].numel()
+    alpha = f64(weights["expert_scale"])
+    Wr = f64(weights["w_router"])
+    R = Wr.shape[0]
+    # forward on every rank (the kept activations a training forward leaves)
+    fcs = [forward_for_grad(x, weights, bias, top_k, rms_eps, aggregation, round_points=True) for x in xs]
+    recs = [route_and_dispatch(x, weights, bias, top_k, aggregation) for x in xs]
+    grads = {k: torch.zeros(weights[k].shape, dtype=F64) for k in
+             ("w_down", "w_router", "w_gate", "w_up_e", "w_down_e", "w_sh_gate", "w_sh_up", "w_sh_down",
+              "rms_gain", "w_up", "expert_scale")}
+    # 1) token side, up to dc, and the shared expert
+    dcs, sends = [], []
+    for s in range(n):
+        fc, rec, dy = fcs[s], recs[s], f64(dys[s])
+        dn = dy @ f64(weights["w_up"])
+        grads["w_up"] += dy.T @ fc.n
+        cn = fc.c * fc.r
+        grads["rms_gain"] += (dn * cn).sum(0)
+        dcn = dn * f64(weights["rms_gain"])[None, :]
+        dc = fc.r * (dcn - cn * (cn * dcn).mean(1, keepdim=True))
+        dcs.append(dc)
+        flat = rec.perm
+        tok, slot = flat // top_k, flat % top_k
+        wrow = fc.ws[tok, slot]                      # w' per dispatch row (as the forward kept it)
+        out = []
+        for d in range(n):
+            lo, hi = owned_range(E, n, d)
+            a, b = int(rec.offsets[lo]), int(rec.offsets[hi])
+            out.append((dc[tok[a:b]], wrow[a:b], rec.counts[lo:hi].clone()))
+        sends.append(out)
+    fwd_rows = [send_buffers(rec, n) for rec in recs]   # what each owner received in the forward
+    # 2) owners
+    back = [[None] * n for _ in range(n)]
+    for d in range(n):
+        lo, hi = owned_range(E, n, d)
+        res = [(torch.zeros(sends[s][d][0].shape, dtype=F64), torch.zeros(sends[s][d][1].shape, dtype=F64))
+               for s in range(n)]
+        for s in range(n):
+            z_rows, cnt = fwd_rows[s][d]
+            dc_rows, w_rows, _ = sends[s][d]
+            start = 0
+            for e in range(lo, hi):
+                m = int(cnt[e - lo])
+                if m == 0:
+                    continue
+                z = z_rows[start:start + m]
+                wg, wu, wd = f64(weights["w_gate"][e]), f64(weights["w_up_e"][e]), f64(weights["w_down_e"][e])
+                g, u = z @ wg.T, z @ wu.T
+                h = bf16_round(g / (1.0 + torch.exp(-g)) * u)
+                dcr, wr_ = dc_rows[start:start + m], w_rows[start:start + m]
+                dhp = dcr @ wd
+                dws = (h * dhp).sum(1)
+                dh = wr_[:, None] * dhp
+                sg = 1.0 / (1.0 + torch.exp(-g))
+                dg = dh * u * sg * (1.0 + g * (1.0 - sg))
+                du = dh * (g * sg)
+                grads["w_gate"][e] += dg.T @ z
+                grads["w_up_e"][e] += du.T @ z
+                grads["w_down_e"][e] += (wr_[:, None] * dcr).T @ h
+                res[s][0][start:start + m] = dg @ wg + du @ wu
+                res[s][1][start:start + m] = dws
+                start += m
+        for s in range(n):
+            back[s][d] = res[s]
+    # 3) token side: router, alpha, dx
+    dxs = []
+    for s in range(n):
+        fc, rec, dc = fcs[s], recs[s], dcs[s]
+        T, L = dc.shape
+        dz_rows = torch.cat([back[s][d][0] for d in range(n)])
+        dws_rows = torch.cat([back[s][d][1] for d in range(n)])
+        flat = rec.perm
+        tok = flat // top_k
+        dz = torch.zeros(T, L, dtype=F64).index_add_(0, tok, dz_rows)
+        # shared expert (replicated), on every token
+        zs = fc.z
+        gs, us = zs @ f64(weights["w_sh_gate"]).T, zs @ f64(weights["w_sh_up"]).T
+        hs = bf16_round(gs / (1.0 + torch.exp(-gs)) * us)
+        dhs = dc @ f64(weights["w_sh_down"])
+        sgs = 1.0 / (1.0 + torch.exp(-gs))
+        dgs = dhs * us * sgs * (1.0 + gs * (1.0 - sgs))
+        dus = dhs * (gs * sgs)
+        grads["w_sh_down"] += dc.T @ hs
+        grads["w_sh_gate"] += dgs.T @ zs
+        grads["w_sh_up"] += dus.T @ zs
+        dz += dgs @ f64(weights["w_sh_gate"]) + dus @ f64(weights["w_sh_up"])
+        # weights and routers
+        dws = torch.zeros(T * top_k, dtype=F64)
+        dws[flat] = dws_rows
+        idxf = fc.idx.reshape(-1)
+        grads["expert_scale"] += torch.zeros(E, dtype=F64).index_add_(0, idxf, fc.w.reshape(-1) * dws)
+        dw = (dws * alpha[idxf]).view(T, top_k)
+        S = fc.ssel.sum(1, keepdim=True)
+        dssel = (dw - (fc.w * dw).sum(1, keepdim=True)) / S
+        ds = torch.zeros(T, E, dtype=F64).scatter_add_(1, fc.idx, dssel)
+        dzx = dz.clone()
+        for r in range(R):
+            if aggregation == "mean":
+                dp = ds / R
+            elif aggregation == "sum":
+                dp = ds
+            else:
+                dp = torch.where(fc.rmax == r, ds, torch.zeros_like(ds))
+            dl = dp * fc.p[r] * (1.0 - fc.p[r])
+            grads["w_router"][r] += dl.T @ fc.zx
+            dzx += dl @ Wr[r]
+        dxs.append(dzx @ f64(weights["w_down"]))
+        grads["w_down"] += dzx.T @ fc.x
+    return dxs, grads

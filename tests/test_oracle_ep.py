@@ -136,3 +136,22 @@ def test_expert_parallel_over_gloo_ranks(world):
         # the same operations on the same rows as in one process: bit for bit
         assert torch.equal(got[r][0], outs[r]["c"]) and torch.equal(got[r][1], outs[r]["y"]), r
     _check_against_single_gpu(s, w, bias, xs, outs)
+
+
+@pytest.mark.parametrize("n,agg", [(1, "mean"), (2, "mean"), (4, "sum"), (4, "max")])
+def test_expert_parallel_backward_equals_single_gpu(n, agg):
+    # the owners see only the rows they received; summed over ranks the
+    # gradients are the single-GPU ones of the whole batch
+    import dataclasses
+    from oracle import mrlmoe_backward as B
+    s, w, bias, xs = _setup(n)
+    s = dataclasses.replace(s, aggregation=agg)
+    dys = [W.make_dy(s, "cpu", seed=31 + r, T=x.shape[0]) for r, x in enumerate(xs)]
+    dxs, grads = EP.ep_backward(xs, dys, w, bias, s.top_k, s.rms_eps, agg)
+    fc = B.forward_for_grad(torch.cat(xs), w, bias, s.top_k, rms_eps=s.rms_eps, aggregation=agg)
+    ref = B.backward(fc, w, torch.cat(dys), s.top_k, aggregation=agg)
+    d = (torch.cat(dxs) - ref["x"]).abs().max().item()
+    assert d <= 1e-10 * ref["x"].abs().max().item(), d
+    for name, g in grads.items():
+        d = (g - ref[name]).abs().max().item()
+        assert d <= 1e-10 * max(1e-30, ref[name].abs().max().item()), (name, d)
