@@ -214,3 +214,42 @@ def test_gradient_fields_cover_every_learnable_tensor():
     assert sorted("x" if f == "dx" else f[2:] for f in N.GRAD_FIELDS) == sorted(OB.GRAD_NAMES)
     # and the C struct: twelve pointers then the accumulate flag
     assert [n for n, _ in N.Grads._fields_] == list(N.GRAD_FIELDS) + ["accumulate"]
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "mrlmoe.h"
+int main(void) {
+  mrlmoe_config c;
+  memset(&c, 0, sizeof c);
+  c.T = 64; c.d_model = 256; c.d_lat = 128; c.n_experts = 16; c.top_k = 2; c.d_ff = 128; c.n_routers = 2;
+  c.rms_eps = 1e-6f; c.dtype = MRLMOE_BF16; c.aggregation = MRLMOE_AGG_MEAN;
+  size_t f = mrlmoe_workspace_size(&c), t = mrlmoe_train_workspace_size(&c);
+  mrlmoe_grads g;
+  memset(&g, 0, sizeof g);
+  /* host-side rejection before any CUDA work: a null x */
+  mrlmoe_status s = mrlmoe_backward(&c, NULL, NULL, NULL, &g, NULL, t, NULL);
+  printf("%zu %zu %d %s\n", f, t, (int)s, mrlmoe_status_string(s));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    # the ABI from C itself: the header compiles as strict C99, a C program
+    # links against the library and calls its host-only entry points
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    lib_dir = os.path.dirname(N.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), str(src), "-L", lib_dir, "-lmrlmoe",
+                        f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    f, t, code, *msg = out.stdout.split()
+    assert int(f) == M.mrlmoe_workspace_size(_cfg())
+    assert int(t) == M.mrlmoe_train_workspace_size(_cfg()) > int(f)
+    assert int(code) == 1 and " ".join(msg) == M.status_string(1)
