@@ -144,7 +144,9 @@ typedef struct {
  * offsets: E+1; scores: T*E.
  *   topk_idx[t*k+j] expert of rank j for token t (descending biased score,
  *                   ties to the lower index);
- *   topk_w[t*k+j]   normalised weight BEFORE alpha (sums to 1 per token);
+ *   topk_w[t*k+j]   normalised weight BEFORE alpha (sums to 1 per token; if
+ *                   the k selected scores sum to exactly 0, every weight is
+ *                   the uniform fp32(1/k));
  *   counts[e]       (token, slot) pairs routed to e; offsets = exclusive scan;
  *   perm[row]       t*k+j of dispatch row `row` (expert-major, tokens ascending);
  *   inv_perm[t*k+j] its dispatch row;
@@ -170,7 +172,15 @@ size_t mrlmoe_workspace_size(const mrlmoe_config *cfg);
  * dispatch record).  x: [T, d_model] bf16, unused (may be NULL) when
  * scores_in != 0, in which case out->scores must hold the fp32 scores s
  * [T, E] to route from (this mode is bit-exact against a CPU definition).
- * bias: [E] fp32.  out: the routing record to fill (non-NULL struct).        */
+ * bias: [E] fp32.  out: the routing record to fill (non-NULL struct).
+ *
+ * Precondition on the values (every routing entry point, and the routers of
+ * mrlmoe_forward): scores, x and bias are finite, or at least every token has
+ * k experts whose biased score s + bias is a number above -inf (NaN scores
+ * and -inf biases are never selected).  A token without k such experts gets
+ * expert -1 and weight 0 in its empty slots; the device status becomes
+ * MRLMOE_ERR_CHECK, the call's later kernels do nothing (the dispatch record
+ * and y are left unwritten), and no index outside [0, E) is ever used.       */
 mrlmoe_status mrlmoe_route(const mrlmoe_config *cfg, const mrlmoe_weights *w,
                            const float *bias, const void *x, int scores_in,
                            mrlmoe_routing *out, void *workspace, size_t ws_bytes,
@@ -227,7 +237,11 @@ mrlmoe_status mrlmoe_linear(const void *a, const void *w, void *out,
  * device address (cudaGetSymbolAddress); make that first call before any
  * stream capture.  All calls share the one array, so calls that overlap on
  * the GPU (different streams, or graphs replayed concurrently) race: order
- * them on one stream.                                                        */
+ * them on one stream.  Its device status word lives in the static array and
+ * cannot be read directly: scores that break the routing precondition above
+ * leave expert -1 in topk_idx and the rest of the record unwritten, which
+ * mrlmoe_check_routing (with a 256-byte status workspace) reports as
+ * MRLMOE_ERR_CHECK.                                                          */
 #define MRLMOE_STATIC_SCRATCH_BYTES (2u * 1024u * 1024u)
 mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *bias,
                                          const float *expert_scale, mrlmoe_routing *out,

@@ -96,7 +96,9 @@ def forward_for_grad(x: torch.Tensor, w: Dict[str, torch.Tensor], bias: torch.Te
         s = s.to(F32).to(F64)
     idx = select_topk(s.to(F32), bias, top_k)
     ssel = torch.gather(s, 1, idx)
-    wgt = ssel / ssel.sum(1, keepdim=True)
+    den = ssel.sum(1, keepdim=True)
+    # a zero sum of the selected scores gives the uniform weights 1/k
+    wgt = torch.where(den == 0, torch.full_like(ssel, 1.0 / top_k), ssel / torch.where(den == 0, 1.0, den))
     ws = wgt * _f(w["expert_scale"])[idx]
     T, L = z.shape
     E = w["expert_scale"].numel()
@@ -195,7 +197,8 @@ def backward(fc: ForwardCache, w: Dict[str, torch.Tensor], dy: torch.Tensor, top
     # w_j = s_j / S over the selected experts
     dw = dw.view(T, top_k)
     S = fc.ssel.sum(1, keepdim=True)
-    dssel = (dw - (fc.w * dw).sum(1, keepdim=True)) / S
+    # where the selected scores sum to 0 the weights are the constant 1/k: no gradient
+    dssel = torch.where(S == 0, 0.0, (dw - (fc.w * dw).sum(1, keepdim=True)) / torch.where(S == 0, 1.0, S))
     ds = torch.zeros(T, E, dtype=F64).scatter_add_(1, fc.idx, dssel)
     # s = agg_r sigmoid(l_r), l_r = zx W_r^T
     wr = _f(w["w_router"])

@@ -149,13 +149,19 @@ def route_weights(s: torch.Tensor, idx: torch.Tensor, alpha: torch.Tensor):
 
     Renormalisation over the selected experts is an assumption; the per-expert
     learnable scalar multiplies the routing weight [derekhsu, Stable LatentMoE].
+    The renormalisation is undefined when the selected scores sum to 0 (every
+    selected sigmoid underflowed to 0 in fp32); the weights are then taken as
+    the uniform fp32(1/k), the limit of equal scores.
     Returns (w, w_scaled), both fp32 [T, k].
     """
     ssel = torch.gather(s.to(F32), 1, idx)
+    k = idx.shape[1]
     den = ssel[:, 0].clone()
-    for j in range(1, idx.shape[1]):
+    for j in range(1, k):
         den = den + ssel[:, j]
-    w = ssel / den[:, None]
+    zero = den == 0
+    w = ssel / torch.where(zero, torch.ones_like(den), den)[:, None]
+    w = torch.where(zero[:, None], torch.tensor(1.0, dtype=F32) / k, w)
     return w, w * alpha.to(F32)[idx]
 
 

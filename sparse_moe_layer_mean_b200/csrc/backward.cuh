@@ -701,7 +701,7 @@ constexpr int kBwdMaxRouters = 8;
 // token t.  The logits of the k selected experts are recomputed from the
 // latent the routers read (zx = z hi + z lo, fp32) as fp32 dot products.
 //   dw'_j = sum over d_ff slices of dwsp;  aw_j = w_j dw'_j (for dalpha);
-//   dw_j = alpha_{e_j} dw'_j;  ds_j = (dw_j - sum_i w_i dw_i) / sum_i s_i;
+//   dw_j = alpha_{e_j} dw'_j;  ds_j = (dw_j - sum_i w_i dw_i) / sum_i s_i (0 if that sum is 0);
 //   dp_{j,r} = ds_j / R (mean), ds_j (sum), ds_j [r = first argmax] (max);
 //   dl_{j,r} = dp_{j,r} p_{j,r} (1 - p_{j,r});
 //   dzx = sum_{j <= k} dzs[t][j] + sum_{j,r} dl_{j,r} W_router[r, e_j]  (in that order)
@@ -784,7 +784,8 @@ __global__ void __launch_bounds__(kBwdThreads) token_bwd_kernel(
   // (slot j, router r): dl
   if (threadIdx.x < k * R) {
     const int j = threadIdx.x / R, r = threadIdx.x - j * R;
-    const float ds = (s_dw[j] - s_tot[1]) / s_tot[0];
+    // selected scores that sum to 0 get the constant weights 1/k: no gradient
+    const float ds = s_tot[0] != 0.0f ? (s_dw[j] - s_tot[1]) / s_tot[0] : 0.0f;
     int rmax = 0;
     if (agg == 2)
       for (int q = 1; q < R; ++q)

@@ -484,7 +484,7 @@ cudaError_t launch_quant(const __nv_bfloat16 *in, long ld_in, int rows, int K, c
 
 // Top-k from fp32 scores with the running-list length that k needs.
 cudaError_t launch_topk_from_scores(const float *s, const float *bias, const float *alpha, int T, int E, int k,
-                                    int32_t *idx, float *w, float *wscaled, const uint32_t *status,
+                                    int32_t *idx, float *w, float *wscaled, uint32_t *status,
                                     cudaStream_t st) {
   const int wpb = 8;
   const int grid = (T + wpb - 1) / wpb;
@@ -618,10 +618,12 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
     if (p.parts > 1) {
       if (k <= kTopKNarrow)
         topk_merge_kernel<kTopKNarrow><<<(T + 127) / 128, 128, 0, st>>>(
-            P.cand_v, P.cand_s, P.cand_i, T, p.parts, k, w->expert_scale, P.topk_idx, P.topk_w, P.wscaled, P.status);
+            P.cand_v, P.cand_s, P.cand_i, T, E, p.parts, k, w->expert_scale, P.topk_idx, P.topk_w, P.wscaled,
+            P.status);
       else
         topk_merge_kernel<kTopKMax><<<(T + 127) / 128, 128, 0, st>>>(
-            P.cand_v, P.cand_s, P.cand_i, T, p.parts, k, w->expert_scale, P.topk_idx, P.topk_w, P.wscaled, P.status);
+            P.cand_v, P.cand_s, P.cand_i, T, E, p.parts, k, w->expert_scale, P.topk_idx, P.topk_w, P.wscaled,
+            P.status);
       MRL_TRY(cudaGetLastError());
     }
   }

@@ -238,8 +238,8 @@ struct RouterPolicyK {
     }
     if (sub == U.nsub - 1 && valid) {
       if (p.parts == 1) {
-        write_selection<KMAX>(st.tk.s, st.tk.i, p.k, static_cast<size_t>(t), p.alpha, p.topk_idx, p.topk_w,
-                                  p.wscaled);
+        write_selection<KMAX>(st.tk.s, st.tk.i, p.k, p.E, static_cast<size_t>(t), p.alpha, p.topk_idx, p.topk_w,
+                              p.wscaled, p.status);
       } else {
         const size_t o = (static_cast<size_t>(t) * p.parts + U.g) * p.k;
 #pragma unroll

@@ -16,9 +16,10 @@ constexpr int kChunk = 32;  // tokens per histogram chunk (one warp, one bit per
 // (larger biased score, then lower index) emit the selection in rank order,
 // and lane 0 writes it with its weights.
 template <int KMAX>
-__device__ __forceinline__ void warp_select_and_write(TopK<KMAX> &tk, int k, int lane, size_t t,
+__device__ __forceinline__ void warp_select_and_write(TopK<KMAX> &tk, int k, int E, int lane, size_t t,
                                                       const float *__restrict__ alpha, int32_t *__restrict__ topk_idx,
-                                                      float *__restrict__ topk_w, float *__restrict__ wscaled) {
+                                                      float *__restrict__ topk_w, float *__restrict__ wscaled,
+                                                      uint32_t *status) {
   float sel_s[KMAX];
   int sel_i[KMAX];
 #pragma unroll
@@ -38,7 +39,7 @@ __device__ __forceinline__ void warp_select_and_write(TopK<KMAX> &tk, int k, int
       sel_i[j] = bi;
     }
   }
-  if (lane == 0) write_selection<KMAX>(sel_s, sel_i, k, t, alpha, topk_idx, topk_w, wscaled);
+  if (lane == 0) write_selection<KMAX>(sel_s, sel_i, k, E, t, alpha, topk_idx, topk_w, wscaled, status);
 }
 
 // Top-k from caller-given fp32 scores s [T, E]: one warp per token (see
@@ -48,7 +49,7 @@ template <int KMAX>
 __global__ void topk_from_scores_kernel(const float *__restrict__ s, const float *__restrict__ bias,
                                         const float *__restrict__ alpha, int T, int E, int k,
                                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
-                                        float *__restrict__ wscaled, const uint32_t *status) {
+                                        float *__restrict__ wscaled, uint32_t *status) {
   if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -60,7 +61,7 @@ __global__ void topk_from_scores_kernel(const float *__restrict__ s, const float
     const float sv = __ldg(row + e);
     tk.offer(sv + __ldg(bias + e), e, sv);
   }
-  warp_select_and_write<KMAX>(tk, k, lane, static_cast<size_t>(warp), alpha, topk_idx, topk_w, wscaled);
+  warp_select_and_write<KMAX>(tk, k, E, lane, static_cast<size_t>(warp), alpha, topk_idx, topk_w, wscaled, status);
 }
 
 // Scores of the K-split router: part[ks][t][r*E + e] holds router r's logit
@@ -93,10 +94,10 @@ __global__ void router_split_scores_kernel(const float *__restrict__ part, int k
 // One thread per token keeps the best k of all parts (same ranking rule).
 template <int KMAX>
 __global__ void topk_merge_kernel(const float *__restrict__ cand_v, const float *__restrict__ cand_s,
-                                  const int32_t *__restrict__ cand_i, int T, int parts, int k,
+                                  const int32_t *__restrict__ cand_i, int T, int E, int parts, int k,
                                   const float *__restrict__ alpha, int32_t *__restrict__ topk_idx,
                                   float *__restrict__ topk_w, float *__restrict__ wscaled,
-                                  const uint32_t *status) {
+                                  uint32_t *status) {
   if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
@@ -105,15 +106,17 @@ __global__ void topk_merge_kernel(const float *__restrict__ cand_v, const float 
   const size_t base = static_cast<size_t>(t) * parts * k;
   for (int c = 0; c < parts * k; ++c)
     topk_offer_any<KMAX>(tk, __ldg(cand_v + base + c), __ldg(cand_i + base + c), __ldg(cand_s + base + c));
-  write_selection<KMAX>(tk.s, tk.i, k, static_cast<size_t>(t), alpha, topk_idx, topk_w, wscaled);
+  write_selection<KMAX>(tk.s, tk.i, k, E, static_cast<size_t>(t), alpha, topk_idx, topk_w, wscaled, status);
 }
 
 // ---------------------------------------------------------------------------
 // Histogram: for chunk c (tokens 32c .. 32c+31) and expert e, mask[c*E + e]
 // has bit i set iff token 32c+i selected e.  One warp per chunk; the warp's
-// table lives in shared memory (E <= 1024 words).
+// table lives in shared memory (E <= 1024 words).  An expert index outside
+// [0, E) is never used: it records DEV_CHECK, so the kernels after this one
+// do nothing.
 __global__ void expert_mask_kernel(const int32_t *__restrict__ topk_idx, int T, int E, int k,
-                                   uint32_t *__restrict__ mask, int nchunks, const uint32_t *status) {
+                                   uint32_t *__restrict__ mask, int nchunks, uint32_t *status) {
   extern __shared__ uint32_t tab_all[];
   if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int wib = threadIdx.x >> 5;
@@ -124,8 +127,16 @@ __global__ void expert_mask_kernel(const int32_t *__restrict__ topk_idx, int T, 
   for (int e = lane; e < E; e += 32) tab[e] = 0u;
   __syncwarp();
   const int t = c * kChunk + lane;
+  bool bad = false;
   if (t < T)
-    for (int j = 0; j < k; ++j) atomicOr(&tab[__ldg(topk_idx + static_cast<size_t>(t) * k + j)], 1u << lane);
+    for (int j = 0; j < k; ++j) {
+      const int e = __ldg(topk_idx + static_cast<size_t>(t) * k + j);
+      if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
+        atomicOr(&tab[e], 1u << lane);
+      else
+        bad = true;
+    }
+  if (bad && status) atomicCAS(status, DEV_OK, DEV_CHECK);
   __syncwarp();
   uint32_t *dst = mask + static_cast<size_t>(c) * E;
   for (int e = lane; e < E; e += 32) dst[e] = tab[e];
@@ -230,11 +241,14 @@ __global__ void expert_offsets_kernel(const int32_t *__restrict__ counts_in, int
 
 // Stable scatter: entry (t, j) with expert e goes to row
 // offsets[e] + base[c*E + e] + popc(mask[c*E + e] & lanes below t's lane):
-// expert-major, ascending tokens within an expert.
+// expert-major, ascending tokens within an expert.  An index outside [0, E)
+// is skipped and records DEV_CHECK (the mask kernel has already refused it,
+// so this kernel only runs on a record it accepted; the check keeps every
+// access in bounds on its own).
 __global__ void expert_scatter_kernel(const int32_t *__restrict__ topk_idx, const uint32_t *__restrict__ mask,
                                       const int32_t *__restrict__ base, const int32_t *__restrict__ offsets,
                                       int T, int E, int k, int nchunks, int32_t *__restrict__ perm,
-                                      int32_t *__restrict__ inv_perm, const uint32_t *status) {
+                                      int32_t *__restrict__ inv_perm, uint32_t *status) {
   if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int c = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -245,6 +259,10 @@ __global__ void expert_scatter_kernel(const int32_t *__restrict__ topk_idx, cons
   for (int j = 0; j < k; ++j) {
     const int flat = t * k + j;
     const int e = __ldg(topk_idx + flat);
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
+      if (status) atomicCAS(status, DEV_OK, DEV_CHECK);
+      continue;
+    }
     const size_t ce = static_cast<size_t>(c) * E + e;
     const int row = __ldg(offsets + e) + __ldg(base + ce) + __popc(__ldg(mask + ce) & below);
     perm[row] = flat;

@@ -2,6 +2,8 @@
 #pragma once
 #include <math.h>
 
+#include "common.cuh"
+
 namespace mrl {
 
 // Sorted (descending value) list of the best candidates seen so far.
@@ -85,26 +87,43 @@ __device__ __forceinline__ void topk_offer_any(TopK<KMAX> &tk, float cv, int ci,
 }
 
 // Final step of routing for one token: w_j = s_j / (s_0 + ... + s_{k-1})
-// (fp32, summed in rank order), w'_j = w_j * alpha[e_j].
+// (fp32, summed in rank order), w'_j = w_j * alpha[e_j].  A zero sum (every
+// selected score 0, e.g. sigmoids that underflowed) gives the uniform weights
+// 1/k.  A slot whose running list never admitted a candidate (fewer than k
+// experts with a biased score that is a number above -inf: NaN scores, or a
+// -inf bias on too many experts) is written as expert -1 with weight 0, and
+// the call's status word records DEV_CHECK, so the dispatch kernels that
+// follow do nothing and no index outside [0, E) is ever used.
 template <int KMAX>
-__device__ __forceinline__ void write_selection(const float (&sel_s)[KMAX], const int (&sel_i)[KMAX], int k,
+__device__ __forceinline__ void write_selection(const float (&sel_s)[KMAX], const int (&sel_i)[KMAX], int k, int E,
                                                 size_t t, const float *__restrict__ alpha,
                                                 int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
-                                                float *__restrict__ wscaled) {
+                                                float *__restrict__ wscaled, uint32_t *status) {
   float den = sel_s[0];
 #pragma unroll
   for (int j = 1; j < KMAX; ++j)
     if (j < k) den = den + sel_s[j];
+  const float uniform = 1.0f / static_cast<float>(k);
+  bool complete = true;
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     if (j < k) {
       const size_t o = t * k + j;
-      const float w = sel_s[j] / den;
-      topk_idx[o] = sel_i[j];
-      topk_w[o] = w;
-      wscaled[o] = w * __ldg(alpha + sel_i[j]);
+      const int e = sel_i[j];
+      if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+        const float w = den != 0.0f ? sel_s[j] / den : uniform;
+        topk_idx[o] = e;
+        topk_w[o] = w;
+        wscaled[o] = w * __ldg(alpha + e);
+      } else {
+        complete = false;
+        topk_idx[o] = -1;
+        topk_w[o] = 0.0f;
+        wscaled[o] = 0.0f;
+      }
     }
   }
+  if (!complete && status) atomicCAS(status, DEV_OK, DEV_CHECK);
 }
 
 }  // namespace mrl

@@ -58,15 +58,19 @@ def _scores_case(name, T, E, k):
         s = torch.where(u == 0, torch.tensor(0.0), torch.where(u == 1, torch.tensor(-0.0), torch.tensor(-1.0)))
         s[:, E // 2] = 0.75          # a positive selected score keeps the weights finite
         b = torch.zeros(E)
+    elif name == "all_zero":
+        # every selected score 0: the weights are the uniform fp32(1/k)
+        s = torch.zeros(T, E)
+        b = W.uniform((E,), -0.05, 0.05, 14, 201, "cpu")
+    elif name == "zipf_skew":
+        # the skewed workload's Zipf(1.1) selection bias on uniform scores
+        s = W.uniform((T, E), 0.0, 1.0, 15, 200, "cpu")
+        b = W.make_bias(W.CONFIGS["c3_skew"], "cpu")
     return s.float().contiguous(), b.float().contiguous()
 
 
-@pytest.mark.parametrize("case", ["uniform", "dyadic_ties", "all_equal", "signed_zeros"])
-@pytest.mark.parametrize("T,E,k", [(64, 16, 2), (1, 16, 2), (33, 512, 10), (1000, 512, 10),
-                                   (257, 1024, 16), (513, 512, 17), (300, 64, 24), (77, 32, 32)])
-def test_route_scores_in_bit_exact(case, T, E, k):
+def _route_scores_in_and_compare(T, E, k, s, b):
     shape = W.LayerShape("t", T=T, d_model=256, d_lat=128, n_experts=E, top_k=k, d_ff=128, n_routers=1)
-    s, b = _scores_case(case, T, E, k)
     alpha = W.uniform((E,), 0.5, 1.5, 3, 300, "cpu")
     dev = "cuda"
     w = {"w_router": torch.zeros(1, E, 128, dtype=torch.bfloat16, device=dev),
@@ -84,6 +88,27 @@ def test_route_scores_in_bit_exact(case, T, E, k):
     assert torch.equal(r["perm"].cpu().long(), ref.perm)
     assert torch.equal(r["inv_perm"].cpu().long(), ref.inv_perm)
     assert layer.device_status() == 0
+    return ref
+
+
+@pytest.mark.parametrize("case", ["uniform", "dyadic_ties", "all_equal", "signed_zeros", "all_zero"])
+@pytest.mark.parametrize("T,E,k", [(64, 16, 2), (1, 16, 2), (33, 512, 10), (1000, 512, 10),
+                                   (257, 1024, 16), (513, 512, 17), (300, 64, 24), (77, 32, 32)])
+def test_route_scores_in_bit_exact(case, T, E, k):
+    s, b = _scores_case(case, T, E, k)
+    _route_scores_in_and_compare(T, E, k, s, b)
+
+
+@pytest.mark.parametrize("case,T", [("uniform", 8192), ("dyadic_ties", 8192), ("uniform", 16384),
+                                    ("zipf_skew", 32768), ("dyadic_ties", 32768)])
+def test_route_scores_in_bit_exact_full_size(case, T):
+    # the workloads' token counts with 512 experts, top-10: 256 to 1024 token
+    # chunks per expert column, so the column scan runs 8 to 32 chunks per warp
+    s, b = _scores_case(case, T, 512, 10)
+    ref = _route_scores_in_and_compare(T, 512, 10, s, b)
+    if case == "zipf_skew":
+        counts = ref.counts.double()
+        assert counts.max() / counts.mean() > 10.0       # skewed loads really reached the scan
 
 
 # ------------------------------------------------------- full layer, tiny

@@ -237,6 +237,19 @@ def test_route_weights_sum_and_closed_form():
     assert w[0, 3].item() == np.float32(ssel[0, 3] / den)
 
 
+def test_route_weights_zero_sum_gives_uniform_weights():
+    # w = s / sum(s) is undefined when the selected scores sum to 0 (sigmoids
+    # that underflowed to 0 in fp32); the reading is the uniform fp32(1/k),
+    # the limit of equal scores.  Tokens with a non-zero sum are unaffected.
+    s = torch.tensor([[0.0, 0.0, 0.0, 0.0], [0.0, 0.5, 0.0, 0.25]], dtype=torch.float32)
+    idx = torch.tensor([[0, 1, 2], [1, 3, 0]])
+    w, ws = O.route_weights(s, idx, torch.tensor([2.0, 1.0, 0.5, 1.0]))
+    third = np.float32(1.0) / np.float32(3.0)
+    assert w[0].tolist() == [float(third)] * 3
+    assert ws[0].tolist() == [float(np.float32(third * np.float32(2.0))), float(third), float(np.float32(third * np.float32(0.5)))]
+    assert w[1].tolist() == [float(np.float32(0.5) / np.float32(0.75)), float(np.float32(0.25) / np.float32(0.75)), 0.0]
+
+
 # -------------------------------------------------------------- dispatch
 def test_permutation_golden():
     g = _gold("permutation_small.json")
