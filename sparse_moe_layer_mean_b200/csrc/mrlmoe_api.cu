@@ -6,6 +6,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "mrlmoe.h"
@@ -292,40 +293,68 @@ bool make_token_maps8(TokenMaps8 *t, const void *base, uint64_t inner, uint64_t 
          make_map(&t->m64, base, 1, inner, rows, 64) && make_map(&t->m128, base, 1, inner, rows, kF8Tile);
 }
 
-// Make the device that owns `p` current; reject host/unknown pointers.
-mrlmoe_status bind_device(const void *p, int *sm_count) {
+// The caller's current device, put back when an entry point returns (the
+// library switches to the device that owns the call's buffers for its
+// launches and leaves the caller's choice as it found it).
+struct DeviceRestore {
+  int prev = -1;
+  ~DeviceRestore() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+// SM count per device, looked up once per device; concurrent first calls
+// from several host threads may each look it up, and store the same value.
+std::atomic<int> g_sm_count[kMaxDevices];
+
+// Make the device that owns `p` current for the rest of the call (restored by
+// `restore` when the entry point returns); reject host/unknown pointers.
+mrlmoe_status bind_device(const void *p, int *sm_count, DeviceRestore *restore) {
   cudaPointerAttributes a;
   if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
     cudaGetLastError();
     return MRLMOE_ERR_CUDA;
   }
   if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return MRLMOE_ERR_INVALID_ARG;
-  int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess || cur != a.device)
-    if (cudaSetDevice(a.device) != cudaSuccess) return MRLMOE_ERR_CUDA;
-  static int sms[kMaxDevices] = {0};
   if (a.device < 0 || a.device >= kMaxDevices) return MRLMOE_ERR_UNSUPPORTED;
-  if (!sms[a.device]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, a.device) != cudaSuccess) return MRLMOE_ERR_CUDA;
-    sms[a.device] = n;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return MRLMOE_ERR_CUDA;
+  if (cur != a.device) {
+    if (cudaSetDevice(a.device) != cudaSuccess) return MRLMOE_ERR_CUDA;
+    restore->prev = cur;
   }
-  *sm_count = sms[a.device];
+  int n = g_sm_count[a.device].load(std::memory_order_relaxed);
+  if (!n) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, a.device) != cudaSuccess) return MRLMOE_ERR_CUDA;
+    g_sm_count[a.device].store(n, std::memory_order_relaxed);
+  }
+  *sm_count = n;
   return MRLMOE_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.  Several host
+// threads may race on a device's first launch; each then sets the same
+// attribute, which is harmless, and the flag is an atomic.
+template <class Kernel>
+cudaError_t set_smem_once(std::atomic<bool> (&done)[kMaxDevices], Kernel kern, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!done[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    done[dev].store(true, std::memory_order_release);
+  }
+  return cudaSuccess;
 }
 
 template <class P>
 cudaError_t launch_gemm(const typename P::Params &p, int grid, cudaStream_t st) {
   static_assert(GemmSmem<P>::kTotal <= 232448, "GEMM shared memory above the 227 KB per-block limit");
-  static bool configured[kMaxDevices] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         GemmSmem<P>::kTotal);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static std::atomic<bool> configured[kMaxDevices];
+  cudaError_t e = set_smem_once(configured, gemm_kernel<P>, GemmSmem<P>::kTotal);
+  if (e != cudaSuccess) return e;
   gemm_kernel<P><<<grid, kGemmThreads, GemmSmem<P>::kTotal, st>>>(p);
   return cudaGetLastError();
 }
@@ -333,15 +362,9 @@ cudaError_t launch_gemm(const typename P::Params &p, int grid, cudaStream_t st) 
 template <class P>
 cudaError_t launch_gemm_pair(const typename P::Params &p, int grid, cudaStream_t st) {
   static_assert(Gemm2Smem<P>::kTotal <= 232448, "GEMM shared memory above the 227 KB per-block limit");
-  static bool configured[kMaxDevices] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm2_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Gemm2Smem<P>::kTotal);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static std::atomic<bool> configured[kMaxDevices];
+  cudaError_t e = set_smem_once(configured, gemm2_kernel<P>, Gemm2Smem<P>::kTotal);
+  if (e != cudaSuccess) return e;
   gemm2_kernel<P><<<grid & ~1, kGemmThreads, Gemm2Smem<P>::kTotal, st>>>(p);
   return cudaGetLastError();
 }
@@ -498,15 +521,9 @@ cudaError_t launch_topk_from_scores(const float *s, const float *bias, const flo
 template <class P>
 cudaError_t launch_gemm8(const typename P::Params &p, int grid, cudaStream_t st) {
   static_assert(Gemm8Smem<P>::kTotal <= 232448, "GEMM shared memory above the 227 KB per-block limit");
-  static bool configured[kMaxDevices] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm8_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Gemm8Smem<P>::kTotal);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  static std::atomic<bool> configured[kMaxDevices];
+  cudaError_t e = set_smem_once(configured, gemm8_kernel<P>, Gemm8Smem<P>::kTotal);
+  if (e != cudaSuccess) return e;
   gemm8_kernel<P><<<grid, kF8Threads, Gemm8Smem<P>::kTotal, st>>>(p);
   return cudaGetLastError();
 }
@@ -648,7 +665,8 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
   if (ws_bytes < layout_of(*cfg, train).total) return MRLMOE_ERR_WORKSPACE;
   int sms = 0;
-  if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
+  DeviceRestore restore;
+  if ((s = bind_device(workspace, &sms, &restore)) != MRLMOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the training forward keeps the routing record in the workspace (the
   // backward reads it there) and copies it to route_out afterwards
@@ -848,7 +866,8 @@ mrlmoe_status backward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, c
   const Layout LT = layout_of(*cfg, true);
   if (ws_bytes < LT.total) return MRLMOE_ERR_WORKSPACE;
   int sms = 0;
-  if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
+  DeviceRestore restore;
+  if ((s = bind_device(workspace, &sms, &restore)) != MRLMOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ptrs P = carve(*cfg, workspace, nullptr);
   uint8_t *b = static_cast<uint8_t *>(workspace);
@@ -1074,7 +1093,8 @@ mrlmoe_status mrlmoe_route(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
   if (ws_bytes < layout_of(*cfg).total) return MRLMOE_ERR_WORKSPACE;
   int sms = 0;
-  if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
+  DeviceRestore restore;
+  if ((s = bind_device(workspace, &sms, &restore)) != MRLMOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Ptrs P = carve(*cfg, workspace, out);
   if ((s = init_header(P.status, cfg->hold, st)) != MRLMOE_OK) return s;
@@ -1133,7 +1153,8 @@ mrlmoe_status mrlmoe_bias_update(const mrlmoe_config *cfg, const int32_t *counts
   if (s != MRLMOE_OK) return s;
   if (!counts || !bias) return MRLMOE_ERR_INVALID_ARG;
   int sms = 0;
-  if ((s = bind_device(bias, &sms)) != MRLMOE_OK) return s;
+  DeviceRestore restore;
+  if ((s = bind_device(bias, &sms, &restore)) != MRLMOE_OK) return s;
   const int E = cfg->n_experts;
   bias_update_kernel<<<(E + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       counts, bias, E, static_cast<long long>(cfg->T) * cfg->top_k, gamma);
@@ -1145,7 +1166,8 @@ mrlmoe_status mrlmoe_linear(const void *a, const void *w, void *out, int M, int 
   if (!a || !w || !out || M < 1 || N < 128 || K < 128 || N % 128 || K % 128) return MRLMOE_ERR_INVALID_ARG;
   if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return MRLMOE_ERR_INVALID_ARG;
   int sms = 0;
-  mrlmoe_status s = bind_device(w, &sms);
+  DeviceRestore restore;
+  mrlmoe_status s = bind_device(w, &sms, &restore);
   if (s != MRLMOE_OK) return s;
   return launch_dense_bf16(a, w, static_cast<__nv_bfloat16 *>(out), nullptr, M, N, K, nullptr, sms,
                            static_cast<cudaStream_t>(stream));
@@ -1161,7 +1183,8 @@ mrlmoe_status mrlmoe_route_scores_static(const mrlmoe_config *cfg, const float *
   const StaticRouteLayout SL = static_route_layout(*cfg);
   if (SL.total > MRLMOE_STATIC_SCRATCH_BYTES) return MRLMOE_ERR_SCRATCH_LIMIT;
   int sms = 0;
-  if ((s = bind_device(out->scores, &sms)) != MRLMOE_OK) return s;
+  DeviceRestore restore;
+  if ((s = bind_device(out->scores, &sms, &restore)) != MRLMOE_OK) return s;
   int dev = 0;
   MRL_TRY(cudaGetDevice(&dev));
   uint8_t *b = static_scratch(dev);
@@ -1197,7 +1220,8 @@ mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, flo
       (reinterpret_cast<uintptr_t>(scale) & 3u))
     return MRLMOE_ERR_INVALID_ARG;
   int sms = 0;
-  mrlmoe_status s = bind_device(in, &sms);
+  DeviceRestore restore;
+  mrlmoe_status s = bind_device(in, &sms, &restore);
   if (s != MRLMOE_OK) return s;
   MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(in), K, rows, K, nullptr, 1, 0, static_cast<uint8_t *>(q),
                        scale, false, nullptr, static_cast<cudaStream_t>(stream)));
@@ -1231,7 +1255,8 @@ mrlmoe_status mrlmoe_check_routing(const mrlmoe_config *cfg, const mrlmoe_routin
   const bool full = ws_bytes >= layout_of(*cfg).total;
   if (ws_bytes < 256 || (!whole && !full)) return MRLMOE_ERR_WORKSPACE;
   int sms = 0;
-  if ((s = bind_device(workspace, &sms)) != MRLMOE_OK) return s;
+  DeviceRestore restore;
+  if ((s = bind_device(workspace, &sms, &restore)) != MRLMOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t *hdr = static_cast<uint32_t *>(workspace);
   // r's arrays where given, else the workspace copies that route/forward keep
