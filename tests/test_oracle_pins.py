@@ -414,6 +414,129 @@ def test_weight_dequant_blocks():
     assert torch.all(wd[:128] == 2.0) and torch.all(wd[128:] == 0.5)
 
 
+# ------------------------------------------------- FP8 layer composition
+def _fp8_fixture():
+    """The hand-worked FP8 layer of tests/golden/fp8_composition_small.json:
+    e4m3 codes of the listed values, block scales 1, everything else 0."""
+    g = _gold("fp8_composition_small.json")
+    sh, inp = g["shape"], g["inputs"]
+    D, L, F, E = sh["d_model"], sh["d_lat"], sh["d_ff"], sh["n_experts"]
+    enc = lambda v: int(O.e4m3_encode(torch.tensor([v], dtype=F64)))
+
+    def mat(rows, cols, entries):
+        m = torch.zeros(rows, cols, dtype=torch.uint8)
+        for i, j, v in entries:
+            m[i, j] = enc(v)
+        return m
+
+    def experts(rows, cols, entries):
+        m = torch.zeros(E, rows, cols, dtype=torch.uint8)
+        m[0] = mat(rows, cols, entries)
+        return m
+
+    w = {"w_down": mat(L, D, inp["w_down"]), "w_up": mat(D, L, inp["w_up"]),
+         "w_gate": experts(F, L, inp["w_gate_e0"]), "w_up_e": experts(F, L, inp["w_up_e_e0"]),
+         "w_down_e": experts(L, F, inp["w_down_e_e0"]),
+         "w_sh_gate": mat(F, L, inp["w_sh_gate"]), "w_sh_up": mat(F, L, inp["w_sh_up"]),
+         "w_sh_down": mat(L, F, inp["w_sh_down"])}
+    for nm in list(w):
+        w["s_" + nm[2:]] = torch.ones(*w[nm].shape[:-2], 1, 1) if w[nm].dim() == 3 else torch.ones(1, 1)
+    w["w_router"] = torch.zeros(sh["n_routers"], E, L, dtype=torch.bfloat16)
+    for r, e, j, v in inp["w_router"]:
+        w["w_router"][r, e, j] = v
+    w["expert_scale"] = torch.tensor(inp["expert_scale"], dtype=torch.float32)
+    gain = torch.full((L,), inp["rms_gain"]["default"], dtype=torch.float32)
+    for j, v in inp["rms_gain"].items():
+        if j != "default":
+            gain[int(j)] = v
+    w["rms_gain"] = gain
+    x = torch.zeros(1, D, dtype=torch.bfloat16)
+    for j, v in inp["x"].items():
+        x[0, int(j)] = v
+    return g, x, w, torch.tensor(inp["bias"], dtype=torch.float32)
+
+
+def _fp8_run(x, w, b, g, skip=None):
+    """The oracle's FP8 forward; with ``skip`` = i, its i-th activation
+    quantisation (0 x, 1/2 the routed expert's z/h, 3/4 the shared
+    expert's z/h, 5 n) is dropped: a planted mistake in the oracle."""
+    import oracle.mrlmoe_oracle as MO
+    real = MO.quantize_act_1x128
+    calls = [0]
+
+    def q(v):
+        i = calls[0]
+        calls[0] += 1
+        return v.to(F64) if i == skip else real(v)
+
+    MO.quantize_act_1x128 = q
+    try:
+        r = O.forward(x, w, b, g["shape"]["top_k"], g["shape"]["rms_eps"], fp8=True)
+    finally:
+        MO.quantize_act_1x128 = real
+    return r, calls[0]
+
+
+def test_fp8_layer_composition_hand_worked():
+    g, x, w, b = _fp8_fixture()
+    r, n_q = _fp8_run(x, w, b, g)
+    assert n_q == 6                      # x; z, h of the routed expert; z, h of the shared expert; n
+    ex = g["expected"]
+    n = len(ex["c"])
+    assert r.z[0, :4].tolist() == ex["z"]
+    assert r.s[0].tolist() == ex["s"]
+    assert r.topk_idx[0].tolist() == ex["topk_idx"] and r.topk_w[0].tolist() == ex["topk_w"]
+    assert r.c[0, :n].tolist() == ex["c"] and torch.all(r.c[0, n:] == 0)
+    assert r.n[0, :n].tolist() == ex["n"] and torch.all(r.n[0, n:] == 0)
+    assert r.y[0, :n].tolist() == ex["y"] and torch.all(r.y[0, n:] == 0)
+
+
+@pytest.mark.parametrize("skip", range(6))
+def test_fp8_fixture_detects_each_dropped_quantisation(skip):
+    # every quantisation point moves c or y of the hand-worked case: an
+    # oracle that dropped any one of them would fail the fixture
+    g, x, w, b = _fp8_fixture()
+    r, _ = _fp8_run(x, w, b, g, skip=skip)
+    ex = g["expected"]
+    n = len(ex["c"])
+    assert r.c[0, :n].tolist() != ex["c"] or r.y[0, :n].tolist() != ex["y"]
+
+
+def test_fp8_fixture_detects_quantisation_before_rounding():
+    # quantising h or n before their bf16 rounding changes the block scale,
+    # so the fixture's c and y also pin the order (round, then quantise)
+    g, _, _, _ = _fp8_fixture()
+    un = g["unrounded"]
+    for v_un, v_bf in ((un["h_routed_0"], 12.25), (un["n_0"], 7.0)):
+        a = torch.zeros(1, 128, dtype=F64)
+        a[0, 0] = v_un
+        bq = torch.zeros(1, 128, dtype=F64)
+        bq[0, 0] = v_bf
+        assert O.bf16_round(a)[0, 0].item() == v_bf
+        assert O.quantize_act_1x128(a)[0, 0].item() != O.quantize_act_1x128(bq)[0, 0].item() == v_bf
+
+
+# ---------------------------------------------------- top-k boundary gap
+def test_topk_boundary_gap_closed_forms():
+    # gap = sb_(k) - sb_(k+1) of the biased scores sb = fp32(s + b), sorted descending
+    gap = lambda s, b, k: O.topk_boundary_gap(torch.tensor([s], dtype=torch.float32),
+                                              torch.tensor(b, dtype=torch.float32), k)[0].item()
+    assert gap([0.5, 0.25, 0.75, 0.125], [0, 0, 0, 0], 2) == 0.25
+    assert gap([0.5, 0.25, 0.75, 0.125], [0, 0, 0, 0], 1) == 0.25
+    assert gap([0.5, 0.25, 0.75, 0.125], [0, 0, 0, 0], 3) == 0.125
+    assert gap([0.5, 0.5, 0.5, 0.1], [0, 0, 0, 0], 1) == 0.0          # a tie at the boundary
+    assert gap([0.5, 0.5, 0.5, 0.125], [0, 0, 0, 0], 3) == 0.375
+    assert gap([0.0, -0.0, 1.0], [0, 0, 0], 2) == 0.0                 # +0 and -0 tie
+    assert gap([0.5, 0.5], [0.0, 2 ** -10], 1) == 2 ** -10            # the bias decides
+    assert gap([0.25, 0.75], [0.5, -0.125], 1) == 0.125               # sb = (0.75, 0.625)
+    # sb is an fp32 sum: 1 + 2^-24 rounds to 1 (ties to even) before the difference
+    assert gap([1.0, 1.0 + 2 ** -23], [2 ** -24, 0.0], 1) == 2 ** -23
+    # the gap is taken row by row
+    s = torch.tensor([[0.9, 0.1, 0.5], [0.2, 0.2, 0.3]], dtype=torch.float32)
+    got = O.topk_boundary_gap(s, torch.zeros(3), 1)
+    assert got.tolist() == [float(np.float32(0.9)) - float(np.float32(0.5)), float(np.float32(0.3)) - float(np.float32(0.2))]
+
+
 # ------------------------------------------------------------- FP4 e2m1
 # OCP Microscaling Formats (MX) v1.0, FP4 E2M1: exponent bias 1, one mantissa
 # bit, exponent field 0 subnormal, no inf/NaN; the positive values are
