@@ -85,6 +85,52 @@ def check_dispatch_properties(r, T: int, E: int, k: int):
     assert torch.all(tok[1:][same] > tok[:-1][same])
 
 
+def hard_tokens(r, T: int, E: int, k: int, bn: int = 256, want: int = 64, seed: int = 0):
+    """Tokens whose dispatch rows sit where the grouped GEMMs are hardest,
+    read from the routing record: the first, last and ragged token tile of
+    the busiest expert, rows on both sides of the CTA-pair split of a tile
+    (half = round32(rows) / 2), groups of 1 to 16 rows, groups whose size
+    straddles the 64/32/16-row box sizes, and the shared expert's first and
+    last tiles; topped up with seeded random tokens to ``want``."""
+    counts = r["counts"].cpu().long()
+    offsets = r["offsets"].cpu().long()
+    perm = r["perm"].cpu().long()
+    rows = []
+
+    def tile_rows(e, t0, nv):
+        base = int(offsets[e]) + t0
+        half = ((nv + 31) // 32 * 32) // 2
+        for q in (0, 1, half - 1, half, nv - 1):
+            if 0 <= q < nv:
+                rows.append(base + q)
+
+    hot = int(torch.argmax(counts))
+    c = int(counts[hot])
+    nt = (c + bn - 1) // bn
+    tile_rows(hot, 0, min(bn, c))                                 # first tile
+    if nt > 1:
+        tile_rows(hot, (nt - 1) * bn, c - (nt - 1) * bn)          # last (ragged) tile
+        tile_rows(hot, (nt // 2) * bn, min(bn, c - (nt // 2) * bn))
+    small = [e for e in range(E) if 1 <= int(counts[e]) <= 16][:8]
+    for e in small:
+        tile_rows(e, 0, int(counts[e]))
+    for m in (16, 17, 31, 32, 33, 63, 64, 65, 96, 127, 128, 129):
+        hit = (counts % bn == m).nonzero().flatten()
+        if hit.numel():
+            e = int(hit[0])
+            t0 = (int(counts[e]) // bn) * bn
+            tile_rows(e, t0, m)
+    tok = set(int(perm[q]) // k for q in rows)
+    tok |= {0, 1, T - 1, min(255, T - 1), min(256, T - 1), max(T - 256, 0)}   # shared expert tiles
+    g = torch.Generator().manual_seed(seed)
+    extra = torch.randperm(T, generator=g).tolist()
+    for t in extra:
+        if len(tok) >= want:
+            break
+        tok.add(t)
+    return torch.tensor(sorted(tok))
+
+
 def train_loop_oracle(steps, lr=7.8125e-4, gamma=1e-3):
     """SGD on fp32 master weights (bf16 copies in the forward, as the layer
     stores them) towards a teacher layer's output, with the balancing-bias
