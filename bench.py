@@ -74,6 +74,8 @@ def parse_args():
     ap.add_argument("--routers", type=int, default=None, help="override the number of routers R")
     ap.add_argument("--no-train-summary", action="store_true",
                     help="leave the training-step summary out of the forward's line")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="leave the c1_decode / c3_skew / c4_fp8 summaries out of the headline's line")
     ap.add_argument("--train", action="store_true",
                     help="time a training step (forward that keeps its activations + backward) instead")
     ap.add_argument("--route-only", action="store_true",
@@ -224,13 +226,14 @@ def layer_bytes_flops(s, counts):
 
 
 def glu_kernel_bytes(s, touched):
-    """Algorithmic bytes of one gate/up + SiLU-GLU launch: gate and up weights
-    of the touched experts and the shared expert, the dispatched latent rows
-    read once, and h written once."""
-    rows = s.T * s.top_k + s.T
-    wb = 1 if s.fp8 else 2
-    we = 0.5 if s.fp4 else wb
-    return int((touched + 1) * 2 * s.d_ff * s.d_lat * we) + rows * s.d_lat * wb + rows * s.d_ff * 2
+    """Algorithmic bytes of one gate/up + SiLU-GLU launch, counted as the
+    layer's byte count counts them: the gate and up weights of the touched
+    experts and of the shared expert (one 128-wide d_ff slice of both per
+    unit, 2 * 128 * d_lat * 2 bytes in bf16).  The dispatched latent rows it
+    reads and the h it writes are intermediates and are not counted; the
+    profiled DRAM traffic shows them."""
+    we = 0.5 if s.fp4 else (1 if s.fp8 else 2)
+    return int((touched + 1) * 2 * s.d_ff * s.d_lat * we)
 
 
 def glu_kernel_flops(s):
@@ -266,6 +269,79 @@ def fp8_peak_probe(dev, n=8192, seconds=1.0):
                 "reps": reps}
     except (RuntimeError, AttributeError) as e:   # not available in this torch build
         return {"unavailable": str(e).splitlines()[0][:200]}
+
+
+OTHER_CONFIGS = ("c1_decode", "c3_skew", "c4_fp8")
+
+
+def config_summary(name, dev, bf16_weights, steps=20, warmup=3):
+    """One more workload, timed on its own after the headline's timed region:
+    ms per forward (CUDA events on the launching stream), tokens/s, the
+    layer's roofline fraction and the stage times; the skewed workload also
+    times its balancing-bias update.  The bf16 workloads reuse the headline's
+    weights (same layer shape); the e4m3 one draws its own."""
+    import torch
+    import sparse_moe_layer_mean_b200 as M
+    import workloads as W
+    try:
+        s = W.CONFIGS[name]
+        weights = W.make_layer_weights(s, dev) if s.fp8 else bf16_weights
+        x = W.make_x(s, dev)
+        bias = W.make_bias(s, dev)
+        layer = M.MRLMoELayer(s, weights, device=dev)
+        y = torch.empty(s.T, s.d_model, dtype=torch.bfloat16, device=dev)
+        routing = layer.routing_buffers()
+        for _ in range(max(3, warmup)):
+            layer(x, bias, y=y, routing=routing)
+        torch.cuda.synchronize()
+        if layer.device_status() != 0:
+            raise RuntimeError("device status non-zero after warm-up")
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(M._native.NUM_STAGE_EVENTS)]
+               for _ in range(steps)]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for i in range(steps):
+            M.mrlmoe_forward_timed(layer.cfg, layer.cw, bias, x, y, None, layer.workspace, layer.ws_bytes, evs[i])
+        stop.record()
+        torch.cuda.synchronize()
+        if layer.device_status() != 0:
+            raise RuntimeError("device status non-zero after the timed region")
+        ms = start.elapsed_time(stop) / steps
+        stage = [sum(r[j].elapsed_time(r[j + 1]) for r in evs) / steps for j in range(M._native.NUM_STAGE_EVENTS - 1)]
+        counts = routing["counts"].cpu()
+        byts, flops, touched = layer_bytes_flops(s, counts)
+        peaks, peak_kind = load_peaks()
+        tpeak = peaks["bf16_tflops_sustained"] * (2 if s.fp8 else 1)
+        t_bytes, t_flops = byts / (peaks["hbm_gbs"] * 1e9), flops / (tpeak * 1e12)
+        out = {"T": s.T, "dtype": "e4m3" if s.fp8 else "bf16", "ms_per_step": round(ms, 4),
+               "tokens_per_s": s.T / (ms * 1e-3), "steps": steps, "warmup": max(3, warmup),
+               "touched_experts": touched,
+               "layer_roofline": {"bound": "hbm" if t_bytes >= t_flops else "tensor",
+                                  "t_bytes_ms": round(t_bytes * 1e3, 4), "t_flops_ms": round(t_flops * 1e3, 4),
+                                  "frac": max(t_bytes, t_flops) / (ms * 1e-3),
+                                  "peaks": f"{peak_kind}" + ("; e4m3 peak taken as 2x sustained bf16" if s.fp8 else "")},
+               "stage_ms": dict(zip(M._native.STAGES, [round(v, 4) for v in stage])),
+               "gpu_launches": kernels_per_step(s, torch.cuda.get_device_properties(dev).multi_processor_count) * steps}
+        if s.bias_kind == "zipf":
+            c = counts.double()
+            out["max_over_mean_load"] = round(float(c.max() / c.mean()), 2)
+            b2 = bias.clone()
+            for _ in range(3):
+                M.mrlmoe_bias_update(layer.cfg, routing["counts"], b2, 1e-3)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(steps):
+                M.mrlmoe_bias_update(layer.cfg, routing["counts"], b2, 1e-3)
+            b.record()
+            torch.cuda.synchronize()
+            out["bias_update_ms"] = round(a.elapsed_time(b) / steps, 5)
+        del layer, routing, y, x
+        if s.fp8:
+            del weights
+        torch.cuda.empty_cache()
+        return out
+    except Exception as e:  # the headline line is printed either way
+        return {"error": str(e).splitlines()[0][:200] if str(e) else type(e).__name__}
 
 
 def cpu_baseline(s, weights_dev, x_dev, bias_dev, ntok):
@@ -776,6 +852,8 @@ def main():
             line["cpu_baseline"] = cpu_baseline(s, weights, x, bias, min(args.cpu_sample, s.T))
         if world == 1 and not s.fp8 and not args.no_train_summary:
             line["train_step"] = train_summary(s, dev, weights, x, bias)
+        if world == 1 and s.name == "c2_prefill" and not args.no_other_configs:
+            line["other_configs"] = {n: config_summary(n, dev, weights) for n in OTHER_CONFIGS}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier(device_ids=[local])
