@@ -298,6 +298,10 @@ def config_summary(name, dev, bf16_weights, steps=20, warmup=3):
             raise RuntimeError("device status non-zero after warm-up")
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(M._native.NUM_STAGE_EVENTS)]
                for _ in range(steps)]
+        for row in evs:          # torch creates the event handles on their first record
+            for e in row:
+                e.record()
+        torch.cuda.synchronize()
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         start.record()
         for i in range(steps):

@@ -332,6 +332,75 @@ mrlmoe_status mrlmoe_backward_timed(const mrlmoe_config *cfg, const mrlmoe_weigh
                                     void *workspace, size_t ws_bytes, void *stream,
                                     void *const *events, int n_events);
 
+/* ------------------------------------------------- expert parallelism
+ * The layer with its routed experts spread over n_ranks ranks.  The pages
+ * motivate the latent design by this layout: the experts compute in the
+ * 2048-d latent, so the rows that travel to another GPU's experts are latent
+ * wide (blog.derekhsu.net "ERNIE-5.5-Flash-Base", section "多路由潛在 MoE";
+ * aitest123.com, section "模型结构").  They give no layout; the library's:
+ * rank d owns the E/n_ranks consecutive routed experts [d E/n, (d+1) E/n);
+ * the projections, routers, shared expert and RMSNorm are replicated; every
+ * rank routes its own tokens.  The library computes each phase on one rank;
+ * the two exchanges are the caller's (an NCCL all-to-all, or copies):
+ *
+ *   1. mrlmoe_ep_dispatch: this rank's tokens routed, their dispatched latent
+ *      rows gathered expert-major into send_rows.  The rows for rank d are
+ *      the contiguous slice offsets[d E/n] .. offsets[(d+1) E/n], and
+ *      counts[d E/n .. (d+1) E/n) says how many belong to each of its experts.
+ *   2. exchange: rank s sends rank d that slice and those counts.
+ *   3. mrlmoe_ep_experts: on the owner, the received rows (sources in rank
+ *      order, each source's rows expert-major) through its experts; row r's
+ *      UNWEIGHTED output, fp32, goes to out_rows[r] (arrival order).
+ *   4. exchange back: each source gets the outputs of the rows it sent, in the
+ *      order it sent them, i.e. in its own dispatch order.
+ *   5. mrlmoe_ep_combine: on the source, each returned row times its weight
+ *      w' = w * alpha, the shared expert, the fixed-order combine, RMSNorm and
+ *      the up-projection.  The additions are the single-GPU layer's, in its
+ *      order and precision, so y equals mrlmoe_forward's y for the same tokens
+ *      whenever the expert GEMMs reproduce each row's products.
+ * bf16 mode only (else MRLMOE_ERR_UNSUPPORTED); E divisible by n_ranks,
+ * 1 <= n_ranks <= 64 (else MRLMOE_ERR_INVALID_ARG).  All three calls of a rank
+ * take the same cfg (cfg->T = this rank's tokens) and the same workspace, in
+ * this order on one stream; mrlmoe_ep_dispatch clears the workspace's status
+ * word and the other two continue it (read it with mrlmoe_get_device_status).
+ * The returned rows are fp32: rounding them to bf16 on the wire would add a
+ * rounding of every expert output that the single-GPU layer does not have.  */
+
+/* Workspace bytes for the three calls on one rank, whose owner receives rows
+ * from n_ranks ranks of at most cfg->T tokens each (0 if cfg or n_ranks is
+ * invalid).  Beyond mrlmoe_workspace_size: the received rows expert-major and
+ * their h, n_ranks * T * min(k, E/n_ranks) * (d_lat + d_ff) * 2 bytes.        */
+size_t mrlmoe_ep_workspace_size(const mrlmoe_config *cfg, int n_ranks);
+
+/* Phase 1.  x [T, d_model] bf16; bias [E]; w: w_down, w_router, expert_scale
+ * (the expert matrices are not read).  out->counts [E] and out->offsets [E+1]
+ * are required (the caller derives the split sizes from them); its other
+ * fields are optional copies of the record.  send_rows: [T*k, d_lat] bf16,
+ * 16-byte aligned, caller-owned.                                              */
+mrlmoe_status mrlmoe_ep_dispatch(const mrlmoe_config *cfg, const mrlmoe_weights *w,
+                                 const float *bias, const void *x, int n_ranks,
+                                 mrlmoe_routing *out, void *send_rows, void *workspace,
+                                 size_t ws_bytes, void *stream);
+
+/* Phase 3, on the owner of experts [rank E/n, (rank+1) E/n).  w_local:
+ * w_gate, w_up_e [E/n, d_ff, d_lat] and w_down_e [E/n, d_lat, d_ff] of the
+ * owner's experts only (other fields unused).  recv_rows [n_recv, d_lat]
+ * bf16; recv_counts: DEVICE int32 [n_ranks, E/n], rows of source s for local
+ * expert e; n_recv = their sum (the device checks it and the counts' signs:
+ * a mismatch is MRLMOE_ERR_CHECK in the status word, nothing is read through
+ * the bad counts).  out_rows [n_recv, d_lat] fp32.  n_recv = 0 enqueues
+ * nothing.  ws_bytes must cover n_recv rows (MRLMOE_ERR_WORKSPACE).           */
+mrlmoe_status mrlmoe_ep_experts(const mrlmoe_config *cfg, const mrlmoe_weights *w_local,
+                                int n_ranks, const void *recv_rows, const int32_t *recv_counts,
+                                int n_recv, float *out_rows, void *workspace, size_t ws_bytes,
+                                void *stream);
+
+/* Phase 5.  ret_rows [T*k, d_lat] fp32 in this rank's dispatch order; w:
+ * the shared expert, rms_gain, w_up and expert_scale; y [T, d_model] bf16.  */
+mrlmoe_status mrlmoe_ep_combine(const mrlmoe_config *cfg, const mrlmoe_weights *w,
+                                const float *ret_rows, void *y, void *workspace,
+                                size_t ws_bytes, void *stream);
+
 /* Synchronises `stream`, then returns the device status word of `workspace`
  * written by the last call that used it (MRLMOE_OK if none failed).          */
 mrlmoe_status mrlmoe_get_device_status(const void *workspace, void *stream);

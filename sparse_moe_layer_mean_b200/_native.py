@@ -27,7 +27,8 @@ EXPORTED = ("mrlmoe_workspace_size", "mrlmoe_route", "mrlmoe_forward", "mrlmoe_f
             "mrlmoe_bias_update", "mrlmoe_linear", "mrlmoe_get_device_status",
             "mrlmoe_status_string", "mrlmoe_route_scores_static", "mrlmoe_quantize_e4m3",
             "mrlmoe_check_routing", "mrlmoe_get_device_detail", "mrlmoe_train_workspace_size",
-            "mrlmoe_forward_train", "mrlmoe_backward", "mrlmoe_backward_timed")
+            "mrlmoe_forward_train", "mrlmoe_backward", "mrlmoe_backward_timed",
+            "mrlmoe_ep_workspace_size", "mrlmoe_ep_dispatch", "mrlmoe_ep_experts", "mrlmoe_ep_combine")
 STATIC_SCRATCH_BYTES = 2 * 1024 * 1024
 NUM_STAGE_EVENTS = 9
 NUM_BACKWARD_EVENTS = 11
@@ -130,6 +131,17 @@ def lib() -> ctypes.CDLL:
         L.mrlmoe_backward_timed.argtypes = [POINTER(Config), POINTER(Weights), c_void_p, c_void_p, POINTER(Grads),
                                             c_void_p, c_size_t, c_void_p, c_void_p, c_int]
         L.mrlmoe_backward_timed.restype = c_int
+        L.mrlmoe_ep_workspace_size.argtypes = [POINTER(Config), c_int]
+        L.mrlmoe_ep_workspace_size.restype = c_size_t
+        L.mrlmoe_ep_dispatch.argtypes = [POINTER(Config), POINTER(Weights), c_void_p, c_void_p, c_int,
+                                         POINTER(Routing), c_void_p, c_void_p, c_size_t, c_void_p]
+        L.mrlmoe_ep_dispatch.restype = c_int
+        L.mrlmoe_ep_experts.argtypes = [POINTER(Config), POINTER(Weights), c_int, c_void_p, c_void_p, c_int,
+                                        c_void_p, c_void_p, c_size_t, c_void_p]
+        L.mrlmoe_ep_experts.restype = c_int
+        L.mrlmoe_ep_combine.argtypes = [POINTER(Config), POINTER(Weights), c_void_p, c_void_p, c_void_p, c_size_t,
+                                        c_void_p]
+        L.mrlmoe_ep_combine.restype = c_int
         L.mrlmoe_status_string.argtypes = [c_int]
         L.mrlmoe_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -298,3 +310,27 @@ def mrlmoe_check_routing(cfg: Config, routing: Optional[Routing], workspace, ws_
     rp = ctypes.byref(routing) if routing is not None else None
     _check(lib().mrlmoe_check_routing(ctypes.byref(cfg), rp, _ptr(workspace), int(ws_bytes), int(bool(clear)),
                                       _stream_ptr(stream)), "mrlmoe_check_routing")
+
+
+# ------------------------------------------------------ expert parallelism
+def mrlmoe_ep_workspace_size(cfg: Config, n_ranks: int) -> int:
+    return int(lib().mrlmoe_ep_workspace_size(ctypes.byref(cfg), int(n_ranks)))
+
+
+def mrlmoe_ep_dispatch(cfg: Config, weights: Weights, bias, x, n_ranks: int, routing: Routing, send_rows,
+                       workspace, ws_bytes: int, stream=None) -> None:
+    _check(lib().mrlmoe_ep_dispatch(ctypes.byref(cfg), ctypes.byref(weights), _ptr(bias), _ptr(x), int(n_ranks),
+                                    ctypes.byref(routing), _ptr(send_rows), _ptr(workspace), int(ws_bytes),
+                                    _stream_ptr(stream)), "mrlmoe_ep_dispatch")
+
+
+def mrlmoe_ep_experts(cfg: Config, w_local: Weights, n_ranks: int, recv_rows, recv_counts, n_recv: int, out_rows,
+                      workspace, ws_bytes: int, stream=None) -> None:
+    _check(lib().mrlmoe_ep_experts(ctypes.byref(cfg), ctypes.byref(w_local), int(n_ranks), _ptr(recv_rows),
+                                   _ptr(recv_counts), int(n_recv), _ptr(out_rows), _ptr(workspace), int(ws_bytes),
+                                   _stream_ptr(stream)), "mrlmoe_ep_experts")
+
+
+def mrlmoe_ep_combine(cfg: Config, weights: Weights, ret_rows, y, workspace, ws_bytes: int, stream=None) -> None:
+    _check(lib().mrlmoe_ep_combine(ctypes.byref(cfg), ctypes.byref(weights), _ptr(ret_rows), _ptr(y),
+                                   _ptr(workspace), int(ws_bytes), _stream_ptr(stream)), "mrlmoe_ep_combine")

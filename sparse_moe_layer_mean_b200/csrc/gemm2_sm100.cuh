@@ -314,4 +314,58 @@ struct Down2Policy {
   }
 };
 
+// Dense bf16 projection over a CTA pair: out[M, N] = bf16(a[M, K] w[N, K]^T)
+// (and optionally the residual of that rounding), unit = (256-row M tile,
+// 256-column N tile).  CTA r loads A rows m*256 + r*128 (its 128 token rows)
+// and the 128 weight rows n0 + r*nv/2 ..; the pair's MMA (M = 256, N = nv)
+// leaves CTA r the accumulator of its 128 token rows x all nv columns.  Per
+// 64-deep K block a CTA stages 32 KB for 2*128*256*64 FLOPs instead of the
+// one-CTA 128 x 256 tile's 48 KB, so a stage crosses from L2 in two thirds
+// of the time.  A 128-row weight box is loaded even when nv = 128 (N not a
+// multiple of 256): the MMA then reads only its first 64 rows in each CTA.
+struct Dense2Policy {
+  static constexpr int kStages = 6;
+  static constexpr int kGroup = 2;
+  static constexpr int kBN = 256;
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBBytesMax = (kBN / 2) * 128;
+  static constexpr int kEpiSmem = 0;
+  static constexpr int kAuxSmem = 0;
+  using Params = DensePolicy::Params;  // m_tiles counts 256-row tiles here
+  static __device__ __forceinline__ void prefetch(const Params &p) {
+    prefetch_tmap(&p.ta);
+    prefetch_tmap(&p.tb);
+  }
+  static __device__ __forceinline__ void stage_aux(const Params &, uint8_t *) {}
+  static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *) { return p.m_tiles * p.n_tiles; }
+  static __device__ __forceinline__ int k_blocks(const Params &p) { return p.K / kBK; }
+  static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *) {
+    Unit U;
+    U.g = 0;
+    U.row0 = 0;
+    U.m = u / p.n_tiles;
+    U.n0 = (u % p.n_tiles) * kBN;
+    U.nv = min(kBN, p.N - U.n0);
+    U.nsub = 1;
+    return U;
+  }
+  static __device__ __forceinline__ uint32_t b_bytes_pair(const Params &, const Unit &) { return 2u * kBBytesMax; }
+  static __device__ __forceinline__ void load_a(const Params &p, const Unit &U, int kb, uint32_t sa, uint32_t bar_cl,
+                                                uint32_t rank) {
+    tma_load_2d_pair(sa, &p.ta, bar_cl, kb * kBK, U.m * 256 + static_cast<int>(rank) * 128);
+  }
+  static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb, uint32_t bar_cl,
+                                                uint32_t rank) {
+    tma_load_2d_pair(sb, &p.tb, bar_cl, kb * kBK, U.n0 + static_cast<int>(rank) * (U.nv >> 1));
+  }
+  static __device__ __forceinline__ uint32_t idesc(const Params &, const Unit &U) { return idesc_bf16(256, U.nv); }
+  static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, uint32_t taddr, int q, int lane, int,
+                                                  uint32_t rank, uint8_t *) {
+    Unit V = U;
+    V.m = U.m * 2 + static_cast<int>(rank);  // the CTA's 128-row M tile
+    DensePolicy::EpiState st;
+    DensePolicy::epilogue(p, V, 0, taddr, q, lane, 0, st, nullptr);
+  }
+};
+
 }  // namespace mrl

@@ -16,6 +16,7 @@
 #include "routing.cuh"
 #include "check.cuh"
 #include "backward.cuh"
+#include "ep.cuh"
 
 using namespace mrl;
 
@@ -566,12 +567,30 @@ mrlmoe_status launch_dense_with(const void *a, const void *w, __nv_bfloat16 *out
   return MRLMOE_OK;
 }
 
+// The same on CTA pairs (M = 256 per unit; Dense2Policy).
+mrlmoe_status launch_dense_pair(const void *a, const void *w, __nv_bfloat16 *out, __nv_bfloat16 *out_lo, int M, int N,
+                                int K, uint32_t *status, int sms, cudaStream_t st) {
+  Dense2Policy::Params p{};
+  if (!make_map(&p.ta, a, 2, K, M, 128) || !make_map(&p.tb, w, 2, K, N, Dense2Policy::kBN / 2)) return MRLMOE_ERR_CUDA;
+  p.out = out;
+  p.out_lo = out_lo;
+  p.ldo = N;
+  p.M = M; p.N = N; p.K = K;
+  p.m_tiles = (M + 255) / 256;
+  p.n_tiles = (N + Dense2Policy::kBN - 1) / Dense2Policy::kBN;
+  p.status = status;
+  MRL_TRY(launch_gemm_pair<Dense2Policy>(p, std::min(sms, 2 * p.m_tiles * p.n_tiles), st));
+  return MRLMOE_OK;
+}
+
+// bf16 projection: 64-column one-CTA tiles when 256-wide tiles would occupy
+// fewer than half the SMs (decode-sized M), else 256 x 256 tiles on CTA pairs.
 mrlmoe_status launch_dense_bf16(const void *a, const void *w, __nv_bfloat16 *out, __nv_bfloat16 *out_lo, int M,
                                 int N, int K, uint32_t *status, int sms, cudaStream_t st) {
   const int wide_tiles = ((M + 127) / 128) * ((N + DensePolicy::kBN - 1) / DensePolicy::kBN);
   if (2 * wide_tiles < sms && N % DenseNarrowPolicy::kBN == 0)
     return launch_dense_with<DenseNarrowPolicy>(a, w, out, out_lo, M, N, K, status, sms, st);
-  return launch_dense_with<DensePolicy>(a, w, out, out_lo, M, N, K, status, sms, st);
+  return launch_dense_pair(a, w, out, out_lo, M, N, K, status, sms, st);
 }
 
 // Routing from x: down-projection into the tail of zbuf, then the fused router.
@@ -1054,6 +1073,52 @@ uint8_t *static_scratch(int dev) {
   return addr[dev];
 }
 
+// ------------------------------------------------ expert parallelism
+// The region after the single-GPU workspace that the expert-parallel phases
+// add: fixed-size tables first (so the combine finds them whatever the owner
+// received), then the received rows, expert-major, and their h.
+struct EpLayout {
+  size_t ep_off, ep_cnt, ep_u1, ep_u2, src, dst, zero, c_off, c_cnt, c_u1, c_u2, fixed_end, out_row, rows, h, total;
+};
+
+bool ep_supported(const mrlmoe_config &c, int n) {
+  return c.dtype == MRLMOE_BF16 && n >= 1 && n <= kEpMaxRanks && c.n_experts % n == 0;
+}
+
+// Rows one owner can receive when every rank routes at most cfg.T tokens:
+// a token sends a rank at most min(k, E/n) rows.
+size_t ep_rows_max(const mrlmoe_config &c, int n) {
+  return static_cast<size_t>(n) * c.T * std::min(c.top_k, c.n_experts / n);
+}
+
+EpLayout ep_layout_of(const mrlmoe_config &c, int n, size_t rows) {
+  EpLayout L{};
+  size_t off = layout_of(c).total;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  };
+  const size_t E = c.n_experts, El = c.n_experts / std::max(n, 1);
+  L.ep_off = take((El + 2) * 4);
+  L.ep_cnt = take((El + 2) * 4);
+  L.ep_u1 = take((El + 2) * 4);
+  L.ep_u2 = take((El + 2) * 4);
+  L.src = take(E * 4);
+  L.dst = take(E * 4);
+  L.zero = take((E + 2) * 4);
+  L.c_off = take((E + 2) * 4);
+  L.c_cnt = take((E + 2) * 4);
+  L.c_u1 = take((E + 2) * 4);
+  L.c_u2 = take((E + 2) * 4);
+  L.fixed_end = off;
+  L.out_row = take(rows * 4);
+  L.rows = take(rows * c.d_lat * 2);
+  L.h = take(rows * c.d_ff * 2);
+  L.total = off;
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1277,6 +1342,197 @@ mrlmoe_status mrlmoe_check_routing(const mrlmoe_config *cfg, const mrlmoe_routin
                                                                           cfg->T, cfg->n_experts, cfg->top_k, hdr);
   MRL_TRY(cudaGetLastError());
   return MRLMOE_OK;
+}
+
+size_t mrlmoe_ep_workspace_size(const mrlmoe_config *cfg, int n_ranks) {
+  if (check_config(cfg) != MRLMOE_OK || !ep_supported(*cfg, n_ranks)) return 0;
+  return ep_layout_of(*cfg, n_ranks, ep_rows_max(*cfg, n_ranks)).total;
+}
+
+mrlmoe_status mrlmoe_ep_dispatch(const mrlmoe_config *cfg, const mrlmoe_weights *w, const float *bias, const void *x,
+                                 int n_ranks, mrlmoe_routing *out, void *send_rows, void *workspace, size_t ws_bytes,
+                                 void *stream) {
+  mrlmoe_status s = check_config(cfg);
+  if (s != MRLMOE_OK) return s;
+  if (!ep_supported(*cfg, n_ranks)) return cfg->dtype != MRLMOE_BF16 ? MRLMOE_ERR_UNSUPPORTED : MRLMOE_ERR_INVALID_ARG;
+  if (!bias || !x || !aligned16(x) || !send_rows || !aligned16(send_rows)) return MRLMOE_ERR_INVALID_ARG;
+  if (!out || !out->counts || !out->offsets) return MRLMOE_ERR_INVALID_ARG;
+  if ((s = check_weights_bf16(w, false)) != MRLMOE_OK) return s;
+  if (!w->w_down || !aligned16(w->w_down)) return MRLMOE_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
+  if (ws_bytes < layout_of(*cfg).total) return MRLMOE_ERR_WORKSPACE;
+  int sms = 0;
+  DeviceRestore restore;
+  if ((s = bind_device(workspace, &sms, &restore)) != MRLMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the record stays in the workspace (the combine reads it there) and is copied out
+  Ptrs P = carve(*cfg, workspace, nullptr);
+  P.scores = out->scores;
+  P.out_counts = out->counts;
+  P.out_offsets = out->offsets;
+  const int T = cfg->T, Ld = cfg->d_lat, k = cfg->top_k, Tk = T * k;
+  if ((s = init_header(P.status, cfg->hold, st)) != MRLMOE_OK) return s;
+  NvtxCall nvtx_call("mrlmoe_ep_dispatch");
+  nvtx_stage(kForwardStages[0]);
+  if ((s = launch_project_and_route(*cfg, w, bias, x, P, sms, st)) != MRLMOE_OK) return s;
+  nvtx_stage(kForwardStages[2]);
+  if ((s = launch_dispatch(*cfg, P, st)) != MRLMOE_OK) return s;
+  nvtx_stage(kForwardStages[3]);
+  const int row_u4 = Ld * 2 / 16;
+  gather_rows_kernel<<<(Tk * 32 + 255) / 256, 256, 0, st>>>(
+      P.perm, Tk, k, reinterpret_cast<const uint4 *>(P.zbuf + static_cast<size_t>(Tk) * Ld),
+      static_cast<uint4 *>(send_rows), row_u4, P.status);
+  MRL_TRY(cudaGetLastError());
+  const size_t n = static_cast<size_t>(Tk) * 4;
+  if (out->topk_idx) MRL_TRY(cudaMemcpyAsync(out->topk_idx, P.topk_idx, n, cudaMemcpyDeviceToDevice, st));
+  if (out->topk_w) MRL_TRY(cudaMemcpyAsync(out->topk_w, P.topk_w, n, cudaMemcpyDeviceToDevice, st));
+  if (out->perm) MRL_TRY(cudaMemcpyAsync(out->perm, P.perm, n, cudaMemcpyDeviceToDevice, st));
+  if (out->inv_perm) MRL_TRY(cudaMemcpyAsync(out->inv_perm, P.inv, n, cudaMemcpyDeviceToDevice, st));
+  return MRLMOE_OK;
+}
+
+mrlmoe_status mrlmoe_ep_experts(const mrlmoe_config *cfg, const mrlmoe_weights *w_local, int n_ranks,
+                                const void *recv_rows, const int32_t *recv_counts, int n_recv, float *out_rows,
+                                void *workspace, size_t ws_bytes, void *stream) {
+  mrlmoe_status s = check_config(cfg);
+  if (s != MRLMOE_OK) return s;
+  if (!ep_supported(*cfg, n_ranks)) return cfg->dtype != MRLMOE_BF16 ? MRLMOE_ERR_UNSUPPORTED : MRLMOE_ERR_INVALID_ARG;
+  if (n_recv < 0 || !recv_counts || !w_local) return MRLMOE_ERR_INVALID_ARG;
+  if (n_recv > 0 && (!recv_rows || !aligned16(recv_rows) || !out_rows || !aligned16(out_rows)))
+    return MRLMOE_ERR_INVALID_ARG;
+  {
+    const void *ps[] = {w_local->w_gate, w_local->w_up_e, w_local->w_down_e};
+    for (const void *p : ps)
+      if (!p || !aligned16(p)) return MRLMOE_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(n_recv) * 256 >= (1ll << 31)) return MRLMOE_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
+  const EpLayout EL = ep_layout_of(*cfg, n_ranks, static_cast<size_t>(n_recv));
+  if (ws_bytes < EL.total) return MRLMOE_ERR_WORKSPACE;
+  if (n_recv == 0) return MRLMOE_OK;  // nothing arrived: no work
+  int sms = 0;
+  DeviceRestore restore;
+  if ((s = bind_device(workspace, &sms, &restore)) != MRLMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *b = static_cast<uint8_t *>(workspace);
+  uint32_t *status = reinterpret_cast<uint32_t *>(b + layout_of(*cfg).status);  // continues the rank's status word
+  auto i32 = [&](size_t off) { return reinterpret_cast<int32_t *>(b + off); };
+  const int El = cfg->n_experts / n_ranks, Ld = cfg->d_lat, F = cfg->d_ff;
+  __nv_bfloat16 *rows = reinterpret_cast<__nv_bfloat16 *>(b + EL.rows);
+  __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(b + EL.h);
+  NvtxCall nvtx_call("mrlmoe_ep_experts");
+  nvtx_stage(kForwardStages[3]);
+  ep_layout_kernel<<<1, 1024, 0, st>>>(recv_counts, n_ranks, El, n_recv, kExpertBN, glu_m_tiles(*cfg),
+                                       down_m_tiles(*cfg), i32(EL.ep_off), i32(EL.ep_cnt), i32(EL.ep_u1),
+                                       i32(EL.ep_u2), i32(EL.src), i32(EL.dst), status);
+  MRL_TRY(cudaGetLastError());
+  ep_gather_kernel<<<n_ranks * El, 256, 0, st>>>(static_cast<const uint4 *>(recv_rows), Ld * 2 / 16, recv_counts,
+                                                 i32(EL.src), i32(EL.dst), reinterpret_cast<uint4 *>(rows),
+                                                 i32(EL.out_row), status);
+  MRL_TRY(cudaGetLastError());
+  nvtx_stage(kForwardStages[4]);
+  {
+    GluParams p{};
+    const uint64_t EF = static_cast<uint64_t>(El) * F;
+    // no shared-expert rows here: its maps are never used and stand in as the routed ones
+    if (!make_map(&p.wg, w_local->w_gate, 2, Ld, EF, 64) || !make_map(&p.wu, w_local->w_up_e, 2, Ld, EF, 64) ||
+        !make_map(&p.sg, w_local->w_gate, 2, Ld, EF, 64) || !make_map(&p.su, w_local->w_up_e, 2, Ld, EF, 64) ||
+        !make_token_maps(&p.tz, rows, Ld, static_cast<uint64_t>(n_recv)))
+      return MRLMOE_ERR_CUDA;
+    p.gt = GroupTable{i32(EL.ep_off), i32(EL.ep_cnt), i32(EL.ep_u1), El, glu_m_tiles(*cfg)};
+    p.h = h;
+    p.F = F; p.L = Ld; p.rows = n_recv;
+    p.status = status;
+    MRL_TRY(launch_gemm_pair<Glu2Policy>(p, sms, st));
+  }
+  nvtx_stage(kForwardStages[5]);
+  {
+    DownPolicy::Params p{};
+    const uint64_t EL_rows = static_cast<uint64_t>(El) * Ld;
+    if (!make_map(&p.wd, w_local->w_down_e, 2, F, EL_rows, 128) ||
+        !make_map(&p.sd, w_local->w_down_e, 2, F, EL_rows, 128) ||
+        !make_token_maps_blocked(&p.th, h, F, static_cast<uint64_t>(n_recv)))
+      return MRLMOE_ERR_CUDA;
+    p.gt = GroupTable{i32(EL.ep_off), i32(EL.ep_cnt), i32(EL.ep_u2), El, down_m_tiles(*cfg)};
+    p.out_row = i32(EL.out_row);
+    p.slots = out_rows;
+    p.L = Ld; p.F = F; p.k = cfg->top_k; p.Tk = 0;
+    p.status = status;
+    if (down_uses_pairs(*cfg))
+      MRL_TRY(launch_gemm_pair<Down2Policy>(p, sms, st));
+    else
+      MRL_TRY(launch_gemm<DownPolicy>(p, sms, st));
+  }
+  return MRLMOE_OK;
+}
+
+mrlmoe_status mrlmoe_ep_combine(const mrlmoe_config *cfg, const mrlmoe_weights *w, const float *ret_rows, void *y,
+                                void *workspace, size_t ws_bytes, void *stream) {
+  mrlmoe_status s = check_config(cfg);
+  if (s != MRLMOE_OK) return s;
+  if (cfg->dtype != MRLMOE_BF16) return MRLMOE_ERR_UNSUPPORTED;
+  if (!w || !w->expert_scale || !ret_rows || !aligned16(ret_rows) || !y || !aligned16(y)) return MRLMOE_ERR_INVALID_ARG;
+  {
+    const void *ps[] = {w->w_sh_gate, w->w_sh_up, w->w_sh_down, w->rms_gain, w->w_up};
+    for (const void *p : ps)
+      if (!p || !aligned16(p)) return MRLMOE_ERR_INVALID_ARG;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
+  const EpLayout EL = ep_layout_of(*cfg, 1, 0);
+  if (ws_bytes < EL.fixed_end) return MRLMOE_ERR_WORKSPACE;
+  int sms = 0;
+  DeviceRestore restore;
+  if ((s = bind_device(workspace, &sms, &restore)) != MRLMOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ptrs P = carve(*cfg, workspace, nullptr);  // the dispatch's record; its status word continues
+  uint8_t *b = static_cast<uint8_t *>(workspace);
+  auto i32 = [&](size_t off) { return reinterpret_cast<int32_t *>(b + off); };
+  const int T = cfg->T, D = cfg->d_model, Ld = cfg->d_lat, F = cfg->d_ff, E = cfg->n_experts, k = cfg->top_k;
+  const int Tk = T * k;
+  NvtxCall nvtx_call("mrlmoe_ep_combine");
+  nvtx_stage(kForwardStages[4]);
+  // group tables with the shared expert alone (every routed count 0)
+  MRL_TRY(cudaMemsetAsync(b + EL.zero, 0, (E + 2) * 4, st));
+  expert_offsets_kernel<<<1, 1024, 0, st>>>(i32(EL.zero), T, E, k, kExpertBN, glu_m_tiles(*cfg), down_m_tiles(*cfg),
+                                            i32(EL.c_off), i32(EL.c_cnt), i32(EL.c_u1), i32(EL.c_u2), nullptr,
+                                            nullptr, P.status);
+  MRL_TRY(cudaGetLastError());
+  {
+    GluParams p{};
+    if (!make_map(&p.wg, w->w_sh_gate, 2, Ld, F, 64) || !make_map(&p.wu, w->w_sh_up, 2, Ld, F, 64) ||
+        !make_map(&p.sg, w->w_sh_gate, 2, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 2, Ld, F, 64) ||
+        !make_token_maps(&p.tz, P.zbuf, Ld, static_cast<uint64_t>(Tk) + T))
+      return MRLMOE_ERR_CUDA;
+    p.gt = GroupTable{i32(EL.c_off), i32(EL.c_cnt), i32(EL.c_u1), E, glu_m_tiles(*cfg)};
+    p.h = P.hbuf;
+    p.F = F; p.L = Ld; p.rows = Tk + T;
+    p.status = P.status;
+    MRL_TRY(launch_gemm_pair<Glu2Policy>(p, sms, st));
+  }
+  nvtx_stage(kForwardStages[5]);
+  {
+    DownPolicy::Params p{};
+    if (!make_map(&p.wd, w->w_sh_down, 2, F, Ld, 128) || !make_map(&p.sd, w->w_sh_down, 2, F, Ld, 128) ||
+        !make_token_maps_blocked(&p.th, P.hbuf, F, static_cast<uint64_t>(Tk) + T))
+      return MRLMOE_ERR_CUDA;
+    p.gt = GroupTable{i32(EL.c_off), i32(EL.c_cnt), i32(EL.c_u2), E, down_m_tiles(*cfg)};
+    p.perm = P.perm;
+    p.wscaled = P.wscaled;
+    p.slots = P.slots;
+    p.L = Ld; p.F = F; p.k = k; p.Tk = Tk;
+    p.status = P.status;
+    if (down_uses_pairs(*cfg))
+      MRL_TRY(launch_gemm_pair<Down2Policy>(p, sms, st));
+    else
+      MRL_TRY(launch_gemm<DownPolicy>(p, sms, st));
+  }
+  nvtx_stage(kForwardStages[6]);
+  ep_combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(
+      reinterpret_cast<const float4 *>(ret_rows), P.inv, P.wscaled, reinterpret_cast<const float4 *>(P.slots), Ld, k,
+      cfg->rms_eps, reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf, P.status);
+  MRL_TRY(cudaGetLastError());
+  nvtx_stage(kForwardStages[7]);
+  return launch_dense_bf16(P.nbuf, w->w_up, static_cast<__nv_bfloat16 *>(y), nullptr, T, D, Ld, P.status, sms, st);
 }
 
 }  // extern "C"

@@ -451,6 +451,9 @@ struct DownPolicy {
     const int32_t *perm;
     const float *wscaled;
     float *slots;    // [T, k+1, L]
+    // expert-parallel owner: row r's unweighted output goes to row out_row[r]
+    // of `slots` (then [rows, L] fp32) instead of its token's weighted slot
+    const int32_t *out_row;
     int L, F, k, Tk;
     uint32_t *status;
   };
@@ -485,7 +488,8 @@ struct DownPolicy {
     umma_f16(d, a, b, id, acc);
   }
   // Lane = output dim l; column = token.  The unit's per-column slot row and
-  // weight are first staged in shared memory (one parallel pass over the
+  // weight (w', 1 for the shared expert and for the rows of an expert-parallel
+  // owner) are first staged in shared memory (one parallel pass over the
   // dispatch record), then for each token column the warp writes 32
   // consecutive fp32 of that token's slot row (128 B, coalesced).
   static __device__ __forceinline__ void epilogue(const Params &p, const Unit &U, int, uint32_t taddr, int q,
@@ -497,7 +501,10 @@ struct DownPolicy {
     const int row0 = U.row0;
     for (int c = etid; c < U.nv; c += 128) {
       const int row = row0 + c;
-      if (sh) {
+      if (p.out_row) {
+        s_slot[c] = __ldg(p.out_row + row);
+        s_wt[c] = 1.0f;
+      } else if (sh) {
         s_slot[c] = (row - p.Tk) * (p.k + 1) + p.k;
         s_wt[c] = 1.0f;
       } else {

@@ -367,28 +367,19 @@ __global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_kernel(
 constexpr int kCombineThreads = 256;
 constexpr int kCombineMaxV4 = 8;  // d_lat <= 8192
 
-__global__ void __launch_bounds__(kCombineThreads) combine_rmsnorm_kernel(
-    const float4 *__restrict__ slots, int L, int k, float eps, const float4 *__restrict__ gain,
-    __nv_bfloat16 *__restrict__ n, const uint32_t *status) {
-  __shared__ float red[kCombineThreads / 32];
-  if (call_failed(status)) return;  // an earlier kernel of the call failed
-  const int t = blockIdx.x;
+// The RMSNorm half of a combine kernel: c[v] holds the thread's float4s of
+// token t's combined row (element i = threadIdx.x + v * kCombineThreads);
+// sum of squares in a fixed order (per thread, then warp tree, then warps in
+// order), n = bf16(c * (1 / sqrt(mean(c^2) + eps)) * gain).
+__device__ __forceinline__ void rmsnorm_row(const float4 (&c)[kCombineMaxV4], int L, float eps,
+                                            const float4 *__restrict__ gain, __nv_bfloat16 *__restrict__ n_row,
+                                            float *red) {
   const int L4 = L >> 2;
-  const float4 *base = slots + static_cast<size_t>(t) * (k + 1) * L4;
-  float4 c[kCombineMaxV4];
   float ss = 0.f;
 #pragma unroll
   for (int v = 0; v < kCombineMaxV4; ++v) {
     const int i = threadIdx.x + v * kCombineThreads;
-    if (i < L4) {
-      float4 a = __ldg(base + i);
-      for (int j = 1; j <= k; ++j) {
-        const float4 b = __ldg(base + static_cast<size_t>(j) * L4 + i);
-        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-      }
-      c[v] = a;
-      ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
-    }
+    if (i < L4) ss += c[v].x * c[v].x + c[v].y * c[v].y + c[v].z * c[v].z + c[v].w * c[v].w;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
@@ -398,7 +389,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_rmsnorm_kernel(
 #pragma unroll
   for (int w = 0; w < kCombineThreads / 32; ++w) tot += red[w];
   const float inv = 1.0f / sqrtf(tot / static_cast<float>(L) + eps);
-  uint2 *dst = reinterpret_cast<uint2 *>(n + static_cast<size_t>(t) * L);
+  uint2 *dst = reinterpret_cast<uint2 *>(n_row);
 #pragma unroll
   for (int v = 0; v < kCombineMaxV4; ++v) {
     const int i = threadIdx.x + v * kCombineThreads;
@@ -410,6 +401,30 @@ __global__ void __launch_bounds__(kCombineThreads) combine_rmsnorm_kernel(
       dst[i] = o;
     }
   }
+}
+
+__global__ void __launch_bounds__(kCombineThreads) combine_rmsnorm_kernel(
+    const float4 *__restrict__ slots, int L, int k, float eps, const float4 *__restrict__ gain,
+    __nv_bfloat16 *__restrict__ n, const uint32_t *status) {
+  __shared__ float red[kCombineThreads / 32];
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
+  const int t = blockIdx.x;
+  const int L4 = L >> 2;
+  const float4 *base = slots + static_cast<size_t>(t) * (k + 1) * L4;
+  float4 c[kCombineMaxV4];
+#pragma unroll
+  for (int v = 0; v < kCombineMaxV4; ++v) {
+    const int i = threadIdx.x + v * kCombineThreads;
+    if (i < L4) {
+      float4 a = __ldg(base + i);
+      for (int j = 1; j <= k; ++j) {
+        const float4 b = __ldg(base + static_cast<size_t>(j) * L4 + i);
+        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+      }
+      c[v] = a;
+    }
+  }
+  rmsnorm_row(c, L, eps, gain, n + static_cast<size_t>(t) * L, red);
 }
 
 // bias[e] += gamma * sgn(T*k - E*counts[e]) (exact integer sign; sign(0) = 0).

@@ -208,6 +208,43 @@ def test_training_entry_points_reject_bad_arguments_before_cuda():
                                    None, None, N.NUM_BACKWARD_EVENTS) == 1
 
 
+def test_expert_parallel_entry_points_reject_bad_arguments_before_cuda():
+    L = N.lib()
+    cfg = _cfg()
+    base = M.mrlmoe_workspace_size(cfg)
+    ws4 = N.mrlmoe_ep_workspace_size(cfg, 4)
+    assert ws4 > base                                          # + received rows and their h
+    assert N.mrlmoe_ep_workspace_size(cfg, 8) > ws4            # more sources, more rows
+    assert N.mrlmoe_ep_workspace_size(cfg, 3) == 0             # E = 16 does not divide by 3
+    assert N.mrlmoe_ep_workspace_size(cfg, 0) == 0
+    assert N.mrlmoe_ep_workspace_size(cfg, 65) == 0
+    assert N.mrlmoe_ep_workspace_size(_cfg(dtype=1), 2) == 0   # bf16 only
+    w = N.Weights(*([4096] * 11 + [None] * 8))
+    r = N.Routing(*([4096] * 7))
+    disp = lambda c, n, x, r_, send, ws, nb: L.mrlmoe_ep_dispatch(
+        ctypes.byref(c), ctypes.byref(w), 4096, x, n, ctypes.byref(r_) if r_ is not None else None, send, ws, nb, None)
+    assert disp(cfg, 3, 4096, r, 4096, 4096, ws4) == 1               # ranks do not divide E
+    assert disp(_cfg(dtype=1), 2, 4096, r, 4096, 4096, ws4) == 2     # FP8: unsupported
+    assert disp(cfg, 4, None, r, 4096, 4096, ws4) == 1               # x
+    assert disp(cfg, 4, 4096, None, 4096, 4096, ws4) == 1            # record
+    no_counts = N.Routing(4096, 4096, None, 4096, 4096, 4096, 4096)
+    assert disp(cfg, 4, 4096, no_counts, 4096, 4096, ws4) == 1       # counts are required
+    assert disp(cfg, 4, 4096, r, 4096 + 8, 4096, ws4) == 1           # send rows misaligned
+    assert disp(cfg, 4, 4096, r, 4096, 4096, base - 1) == 3          # workspace too small
+    exp = lambda n, rows, counts, n_recv, out, ws, nb: L.mrlmoe_ep_experts(
+        ctypes.byref(cfg), ctypes.byref(w), n, rows, counts, n_recv, out, ws, nb, None)
+    assert exp(4, 4096, 4096, -1, 4096, 4096, ws4) == 1              # negative row count
+    assert exp(4, 4096, None, 10, 4096, 4096, ws4) == 1              # counts
+    assert exp(4, None, 4096, 10, 4096, 4096, ws4) == 1              # rows
+    assert exp(4, 4096, 4096, 10, 4096 + 4, 4096, ws4) == 1          # out misaligned
+    assert exp(4, 4096, 4096, 10 ** 6, 4096, 4096, ws4) == 3         # more rows than the workspace holds
+    assert exp(4, None, 4096, 0, None, 4096, ws4) == 0               # nothing arrived: nothing to do
+    comb = lambda ret, y, ws, nb: L.mrlmoe_ep_combine(ctypes.byref(cfg), ctypes.byref(w), ret, y, ws, nb, None)
+    assert comb(None, 4096, 4096, ws4) == 1
+    assert comb(4096, 4096 + 2, 4096, ws4) == 1
+    assert comb(4096, 4096, 4096, base) == 3                         # needs the expert-parallel tables
+
+
 def test_gradient_fields_cover_every_learnable_tensor():
     from oracle import mrlmoe_backward as OB
     # dx -> x, d_<name> -> <name>: the same twelve tensors as the oracle's backward

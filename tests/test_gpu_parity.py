@@ -25,7 +25,9 @@ def _gpu():
 
 # ------------------------------------------------------------------ linear
 @pytest.mark.parametrize("M_,N_,K_", [(1, 128, 128), (127, 256, 256), (129, 384, 640),
-                                      (300, 2048, 4096), (1000, 4096, 2048)])
+                                      (300, 2048, 4096), (1000, 4096, 2048),
+                                      # CTA-pair tiles: a ragged 256-row M tile, a 128-wide last N tile
+                                      (8229, 384, 256), (2100, 2048, 4096)])
 def test_linear_matches_oracle(M_, N_, K_):
     a = W.normal((M_, K_), 7, 100, "cuda")
     w = W.normal((N_, K_), 7, 101, "cuda", std=K_ ** -0.5)
