@@ -68,3 +68,33 @@ def test_forward_tiny_layer_k32():
     keep[bad] = False
     mx, mean = rel_errors(y.cpu()[keep], ref.y[keep])
     assert mx <= BF16_MAX_REL and mean <= BF16_MEAN_REL, (mx, mean)
+
+
+@pytest.mark.parametrize("T,R,k,agg", [(2500, 4, 10, "mean"), (2600, 4, 24, "mean"), (2401, 3, 10, "sum"),
+                                       (9300, 1, 10, "mean"), (1300, 8, 10, "max"), (1300, 8, 32, "sum")])
+def test_route_from_x_larger_T(T, R, k, agg):
+    # token counts above the K-split router's range: the router walks its
+    # expert chunks per token tile and the partial lists are merged; ragged
+    # last tiles, odd R, R = 1 (two chunks of 256 experts), R = 8, wide k
+    import dataclasses
+    s = dataclasses.replace(W.LayerShape("pair", T=T, d_model=256, d_lat=256, n_experts=512, top_k=k, d_ff=128,
+                                         n_routers=R), aggregation=agg)
+    w = W.make_routing_weights(s, "cuda")
+    x = W.make_x(s, "cuda")
+    bias = W.uniform((s.n_experts,), -0.02, 0.02, 3, 960, "cuda")
+    layer = M.MRLMoELayer(s, w)
+    r = layer.routing_buffers(scores=True)
+    layer.route(bias, x=x, routing=r)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    zx = x.cpu().double() @ w["w_down"].cpu().double().T
+    s_ref = O.router_scores(zx, w["w_router"].cpu(), agg)
+    sg = r["scores"].view(T, s.n_experts).cpu().double()
+    assert (sg - s_ref.double()).abs().max().item() < 1e-5 * (R if agg == "sum" else 1)
+    bad, gaps, _ = routing_audit(r["topk_idx"].view(-1, k), s_ref, bias, k)
+    assert torch.all(gaps < GAP_TOL), (bad, gaps)
+    check_dispatch_properties(r, T, s.n_experts, k)
+    good = torch.ones(T, dtype=torch.bool)
+    good[bad] = False
+    wg = r["topk_w"].view(T, k).cpu().double()[good]
+    assert (wg.sum(1) - 1).abs().max().item() < 1e-5
