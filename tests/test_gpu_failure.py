@@ -36,10 +36,11 @@ def _bias(E):
     return W.uniform((E,), -0.01, 0.01, 4, 920, "cuda")
 
 
-@pytest.mark.parametrize("family,config", [("gemm", "c0_tiny"), ("gemm_pair", "c0_tiny"),
-                                           ("gemm_fp8", "c0_fp8"), ("gemm_fp8", "c0_fp4")])
-def test_held_loads_run_out_the_bounded_waits(family, config):
-    s = W.CONFIGS[config]
+@pytest.mark.parametrize("family,config,T", [("gemm", "c0_tiny", None), ("gemm_pair", "c0_tiny", None),
+                                             ("gemm_fp8", "c0_fp8", None), ("gemm_fp8", "c0_fp4", None),
+                                             ("gemm_fp8", "c0_fp8", 1100)])
+def test_held_loads_run_out_the_bounded_waits(family, config, T):
+    s = W.CONFIGS[config] if T is None else W.CONFIGS[config].with_T(T)
     x = W.make_x(s, "cuda")
     bias = _bias(s.n_experts)
     layer = M.MRLMoELayer(s, device_weights(config))

@@ -296,6 +296,32 @@ def test_forward_fp8_tiny_ragged(T):
     _compare_fp8(s, x, bias, y, r, host_weights("c0_fp8"))
 
 
+@pytest.mark.parametrize("T", [1024, 1100, 10100])
+def test_forward_fp8_tiny_larger_T(T):
+    # the tiny FP8 layer at token counts whose experts average >= 128 rows
+    # (several 128-token e4m3 units per expert, ragged last units); at
+    # T = 10100 the projections run ~80 token tiles
+    s, x, bias, y, r, _ = _run_layer("c0_fp8", T=T, scores=False)
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+    tokens = None if T <= 1100 else hard_tokens(r, s.T, s.n_experts, s.top_k, bn=256, want=300, seed=5)
+    if tokens is not None:
+        tokens = torch.unique(torch.cat([tokens, torch.arange(T - 140, T)]))
+    _compare_fp8(s, x, bias, y, r, host_weights("c0_fp8"), tokens=tokens)
+
+
+def test_forward_fp8_groups_of_every_size_larger_T():
+    # expert 0 takes every token (1100 rows: eight full 128-token units and a
+    # ragged one), the others 1 to a few hundred rows
+    bias = torch.linspace(0.0, 0.05, 16, dtype=torch.float32)
+    bias[0] = 10.0
+    bias[5] += 0.2
+    s, x, bias, y, r, _ = _run_layer("c0_fp8", T=1100, bias=bias.cuda(), scores=False)
+    counts = r["counts"].cpu()
+    assert int(counts[0]) == 1100 and int(counts.min()) < 128
+    _compare_fp8(s, x, bias, y, r, host_weights("c0_fp8"))
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+
+
 def test_forward_c4_fp8_sampled_tokens():
     s, x, bias, y, r, _ = _run_layer("c4_fp8", scores=False)
     check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
