@@ -632,9 +632,12 @@ struct Down8Policy {
     const size_t blk = (static_cast<size_t>(sh ? 0 : U.g) * (p.L / 128) + U.m) * kbs;
     stage_token_scales(p.hs_t, p.rows, U.row0, U.nv, kbs, tok, lane);
     stage_weight_scales((sh ? p.sd_s : p.wd_s) + blk, nullptr, kbs, w, lane);
-    // [128] slot row, then [128] weight; the loads go out in two batches
-    // (all permutation entries, then all weights) rather than as four
-    // dependent pairs
+    stage_slots(p, U, extra, lane);
+  }
+  // [128] slot row, then [128] weight; the loads go out in two batches (all
+  // permutation entries, then all weights) rather than as four dependent pairs
+  static __device__ __forceinline__ void stage_slots(const Params &p, const Unit &U, float *extra, int lane) {
+    const bool sh = U.g == p.gt.E;
     int *slot = reinterpret_cast<int *>(extra);
     constexpr int C = kF8Tile / 32;
     int flat[C];

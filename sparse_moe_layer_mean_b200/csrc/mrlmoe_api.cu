@@ -13,6 +13,7 @@
 #include "policies.cuh"
 #include "gemm2_sm100.cuh"
 #include "gemm8_sm100.cuh"
+#include "gemm8w_sm100.cuh"
 #include "routing.cuh"
 #include "check.cuh"
 #include "backward.cuh"
@@ -448,8 +449,36 @@ constexpr int kExpertBN = 256;  // token tile of the bf16 grouped GEMMs (Glu2Pol
 struct GroupTiling {
   int bn, mt1, mt2;
 };
+// The 256-column e4m3 kernels lend registers between warpgroups
+// (setmaxnreg), which is only sound when the kernel was built with exactly
+// kW8LaunchRegs registers per thread: each instantiation's count is read once
+// from its attributes, and one built with another count is never launched
+// (the 128-column kernel runs instead).
+template <class P>
+bool wide8_ready() {
+  static const bool ok = [] {
+    cudaFuncAttributes a{};
+    if (cudaFuncGetAttributes(&a, gemm8w_kernel<P>) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return false;
+    }
+    return a.numRegs == kW8LaunchRegs;
+  }();
+  return ok;
+}
+
+// FP8 (not FP4) expert GEMMs on 256-column units: gate/up always, the expert
+// down GEMM when d_lat splits into 256-wide slices.
+bool fp8_wide_glu(const mrlmoe_config &c) {
+  return c.dtype == MRLMOE_FP8_E4M3_BLOCK128 && wide8_ready<Glu8WPolicy>();
+}
+bool fp8_wide_down(const mrlmoe_config &c) {
+  return c.dtype == MRLMOE_FP8_E4M3_BLOCK128 && c.d_lat % kW8N == 0 && wide8_ready<Down8WPolicy>();
+}
+
 GroupTiling group_tiling(const mrlmoe_config &c) {
-  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128) return {kF8Tile, c.d_ff / 64, c.d_lat / 128};
+  if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128)
+    return {kF8Tile, c.d_ff / (fp8_wide_glu(c) ? 128 : 64), c.d_lat / (fp8_wide_down(c) ? kW8N : 128)};
   if (c.dtype == MRLMOE_FP4_E2M1_BLOCK128) return {kF4TokTile, c.d_ff / 64, c.d_lat / 128};
   return {kExpertBN, glu_m_tiles(c), down_m_tiles(c)};
 }
@@ -529,6 +558,16 @@ cudaError_t launch_gemm8(const typename P::Params &p, int grid, cudaStream_t st)
   return cudaGetLastError();
 }
 
+template <class P>
+cudaError_t launch_gemm8w(const typename P::Params &p, int grid, cudaStream_t st) {
+  static_assert(Gemm8WSmem<P>::kTotal <= 232448, "GEMM shared memory above the 227 KB per-block limit");
+  static std::atomic<bool> configured[kMaxDevices];
+  cudaError_t e = set_smem_once(configured, gemm8w_kernel<P>, Gemm8WSmem<P>::kTotal);
+  if (e != cudaSuccess) return e;
+  gemm8w_kernel<P><<<grid, kF8Threads, Gemm8WSmem<P>::kTotal, st>>>(p);
+  return cudaGetLastError();
+}
+
 // FP8 projection out = bf16(q(a) w^T) from e4m3 codes + scales (as_t: the
 // activation scales transposed, [K/128, M]).
 mrlmoe_status launch_dense8(const uint8_t *aq, const float *as_t, const void *wq, const float *ws, int M, int N, int K,
@@ -542,8 +581,15 @@ mrlmoe_status launch_dense8(const uint8_t *aq, const float *as_t, const void *wq
   p.ldo = N;
   p.M = M; p.N = N; p.K = K;
   p.m_tiles = (M + 127) / 128;
-  p.n_tiles = (N + kF8Tile - 1) / kF8Tile;
   p.status = P.status;
+  // 256-column units when they alone fill the SMs, else 128-column ones
+  const int wide_units = p.m_tiles * ((N + kW8N - 1) / kW8N);
+  if (wide_units >= sms && wide8_ready<Dense8WPolicy>()) {
+    p.n_tiles = (N + kW8N - 1) / kW8N;
+    MRL_TRY(launch_gemm8w<Dense8WPolicy>(p, std::min(sms, wide_units), st));
+    return MRLMOE_OK;
+  }
+  p.n_tiles = (N + kF8Tile - 1) / kF8Tile;
   MRL_TRY(launch_gemm8<Dense8Policy>(p, std::min(sms, p.m_tiles * p.n_tiles), st));
   return MRLMOE_OK;
 }
@@ -799,7 +845,24 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
   auto wmap = [&](CUtensorMap *m, const void *base, uint64_t K, uint64_t rows, uint32_t box_rows) {
     return fp4 ? make_map_packed(m, base, K / 2, rows, box_rows) : make_map(m, base, 1, K, rows, box_rows);
   };
-  {
+  if (fp8_wide_glu(c)) {
+    // 128 gate + 128 up rows per unit; h is quantised in the epilogue
+    Glu8WPolicy::Params p{};
+    if (!make_map(&p.wg, w->w_gate, 1, Ld, static_cast<uint64_t>(E) * F, 128) ||
+        !make_map(&p.wu, w->w_up_e, 1, Ld, static_cast<uint64_t>(E) * F, 128) ||
+        !make_map(&p.sg, w->w_sh_gate, 1, Ld, F, 128) || !make_map(&p.su, w->w_sh_up, 1, Ld, F, 128) ||
+        !make_token_maps8(&p.tz, P.zq, Ld, static_cast<uint64_t>(Tk) + T))
+      return MRLMOE_ERR_CUDA;
+    p.wg_s = w->s_gate; p.wu_s = w->s_up_e; p.sg_s = w->s_sh_gate; p.su_s = w->s_sh_up;
+    p.zs_t = P.zs;
+    p.rows = Tk + T;
+    p.gt = GroupTable{P.grp_off, P.grp_cnt, P.unit1, E, gtl.mt1};
+    p.hq = P.hq;
+    p.hs_t = P.hs;
+    p.F = F; p.L = Ld;
+    p.status = P.status;
+    MRL_TRY(launch_gemm8w<Glu8WPolicy>(p, sms, st));
+  } else {
     Glu8Policy::Params p{};
     if (!wmap(&p.wg, w->w_gate, Ld, static_cast<uint64_t>(E) * F, 64) ||
         !wmap(&p.wu, w->w_up_e, Ld, static_cast<uint64_t>(E) * F, 64) ||
@@ -817,8 +880,8 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
       MRL_TRY(launch_gemm8<Glu4Policy>(p, sms, st));
     else
       MRL_TRY(launch_gemm8<Glu8Policy>(p, sms, st));
+    MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, nullptr, 1, 0, P.hq, P.hs, true, P.status, st));
   }
-  MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, nullptr, 1, 0, P.hq, P.hs, true, P.status, st));
   if (!mark(5)) return MRLMOE_ERR_CUDA;
   {
     Down8Policy::Params p{};
@@ -836,6 +899,8 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     p.status = P.status;
     if (fp4)
       MRL_TRY(launch_gemm8<Down4Policy>(p, sms, st));
+    else if (fp8_wide_down(c))
+      MRL_TRY(launch_gemm8w<Down8WPolicy>(p, sms, st));
     else
       MRL_TRY(launch_gemm8<Down8Policy>(p, sms, st));
   }

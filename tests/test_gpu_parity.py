@@ -322,6 +322,34 @@ def test_forward_fp8_groups_of_every_size_larger_T():
     check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
 
 
+def _fp8_mid_width(T):
+    # d_lat 512 (two 256-wide slices in the expert-down units), d_ff 384
+    # (three 128-wide gate/up slices), d_model 384 (the up-projection's last
+    # 256-column unit half outside N); at T = 10100 both projections run on
+    # 256-column units (79 token tiles x 2 column tiles)
+    return W.LayerShape("fp8_mid", T=T, d_model=384, d_lat=512, n_experts=16, top_k=2, d_ff=384, n_routers=2,
+                        fp8=True, outlier_frac=0.01)
+
+
+@pytest.mark.parametrize("T", [300, 10100])
+def test_forward_fp8_mid_width(T):
+    s = _fp8_mid_width(T)
+    w = W.make_layer_weights(s, "cuda", seed=0)
+    x = W.make_x(s, "cuda", seed=0)
+    bias = W.uniform((s.n_experts,), -0.01, 0.01, 4, 901, "cuda")
+    layer = M.MRLMoELayer(s, w)
+    r = layer.routing_buffers(scores=False)
+    y = layer(x, bias, routing=r)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+    tokens = None
+    if T > 300:
+        tokens = hard_tokens(r, s.T, s.n_experts, s.top_k, bn=128, want=300, seed=6)
+        tokens = torch.unique(torch.cat([tokens, torch.arange(T - 140, T)]))
+    _compare_fp8(s, x, bias, y, r, {k: v.cpu() for k, v in w.items()}, tokens=tokens)
+
+
 def test_forward_c4_fp8_sampled_tokens():
     s, x, bias, y, r, _ = _run_layer("c4_fp8", scores=False)
     check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
