@@ -45,13 +45,16 @@ def kernels_per_step(s, sms: int) -> int:
             break
     m_tiles = (s.T + 127) // 128
     chunks = s.n_experts // ec
+    # FP8 variant: the x and n quantisers replace nothing and the z quantiser
+    # replaces the gather; h is quantised in the e4m3 gate/up epilogue, except
+    # with FP4 expert weights, where a quantiser pass over h follows the GEMM
+    extra = (3 if s.fp4 else 2) if s.fp8 else 0
     if 2 * m_tiles * chunks <= 148 and s.d_lat // 64 % 2 == 0:
-        return KERNELS_PER_STEP + 2 + (3 if s.fp8 else 0)
+        return KERNELS_PER_STEP + 2 + extra
     parts = 1
     while parts * 2 <= chunks and chunks % (parts * 2) == 0 and m_tiles * parts * 2 <= sms:
         parts *= 2
-    # FP8 variant: the x, h and n quantisers replace nothing and the z quantiser replaces the gather
-    return KERNELS_PER_STEP + (1 if parts > 1 else 0) + (3 if s.fp8 else 0)
+    return KERNELS_PER_STEP + (1 if parts > 1 else 0) + extra
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -272,6 +275,34 @@ def fp8_peak_probe(dev, n=8192, seconds=1.0):
         return {"unavailable": str(e).splitlines()[0][:200]}
 
 
+_E4M3_PROBE = {}
+
+
+def e4m3_peak(dev, peaks, peak_kind):
+    """The tensor peak an e4m3 kernel is measured against: the vendor
+    library's sustained e4m3 GEMM rate on this GPU (fp8_peak_probe, taken once
+    per process), or 2 x the sustained bf16 peak where the probe cannot run."""
+    if dev not in _E4M3_PROBE:
+        _E4M3_PROBE[dev] = fp8_peak_probe(dev)
+    probe = _E4M3_PROBE[dev]
+    if "tflops" in probe:
+        return probe["tflops"], "measured (vendor e4m3 GEMM probe on this GPU: " + probe["gemm"] + ")", probe
+    return peaks["bf16_tflops_sustained"] * 2, f"of {peak_kind} (sustained bf16 x 2 for e4m3, assumed)", probe
+
+
+def glu_roofline(s, glu_ms, touched, peaks, peak_kind, dev):
+    """The gate/up kernel against its bound: e4m3 FLOPs against the e4m3 peak,
+    bf16 weight bytes against the measured HBM bandwidth."""
+    if s.fp8:
+        tpeak, kind, _ = e4m3_peak(dev, peaks, peak_kind)
+        achieved = glu_kernel_flops(s) / (glu_ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": tpeak, "unit": "TFLOP/s",
+                "frac": achieved / tpeak, "peak_kind": kind}
+    achieved = glu_kernel_bytes(s, touched) / (glu_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "peak_kind": f"of {peak_kind}"}
+
+
 OTHER_CONFIGS = ("c1_decode", "c3_skew", "c4_fp8")
 
 
@@ -316,7 +347,10 @@ def config_summary(name, dev, bf16_weights, steps=20, warmup=3):
         counts = routing["counts"].cpu()
         byts, flops, touched = layer_bytes_flops(s, counts)
         peaks, peak_kind = load_peaks()
-        tpeak = peaks["bf16_tflops_sustained"] * (2 if s.fp8 else 1)
+        if s.fp8:
+            tpeak, tkind, _ = e4m3_peak(dev, peaks, peak_kind)
+        else:
+            tpeak, tkind = peaks["bf16_tflops_sustained"], f"{peak_kind}"
         t_bytes, t_flops = byts / (peaks["hbm_gbs"] * 1e9), flops / (tpeak * 1e12)
         out = {"T": s.T, "dtype": "e4m3" if s.fp8 else "bf16", "ms_per_step": round(ms, 4),
                "tokens_per_s": s.T / (ms * 1e-3), "steps": steps, "warmup": max(3, warmup),
@@ -324,8 +358,10 @@ def config_summary(name, dev, bf16_weights, steps=20, warmup=3):
                "layer_roofline": {"bound": "hbm" if t_bytes >= t_flops else "tensor",
                                   "t_bytes_ms": round(t_bytes * 1e3, 4), "t_flops_ms": round(t_flops * 1e3, 4),
                                   "frac": max(t_bytes, t_flops) / (ms * 1e-3),
-                                  "peaks": f"{peak_kind}" + ("; e4m3 peak taken as 2x sustained bf16" if s.fp8 else "")},
+                                  "peaks": f"{peak_kind}" + (f"; e4m3 peak {tpeak} TFLOP/s {tkind}" if s.fp8 else "")},
                "stage_ms": dict(zip(M._native.STAGES, [round(v, 4) for v in stage])),
+               "gate_up_roofline": glu_roofline(s, stage[M._native.STAGES.index("gate_up_glu")], touched, peaks,
+                                                peak_kind, dev),
                "gpu_launches": kernels_per_step(s, torch.cuda.get_device_properties(dev).multi_processor_count) * steps}
         if s.bias_kind == "zipf":
             c = counts.double()
@@ -795,13 +831,16 @@ def main():
         glu_ms = stage_ms[M._native.STAGES.index("gate_up_glu")]
         glu_bytes = glu_kernel_bytes(s, touched)
         glu_flops = glu_kernel_flops(s)
-        # the gate/up kernel's bound: HBM bytes or tensor FLOPs (FP8 peak taken as 2x bf16)
-        tensor_peak = peaks["bf16_tflops_sustained"] * (2 if s.fp8 else 1)
+        # the gate/up kernel's bound: HBM bytes or tensor FLOPs (e4m3: the probe's peak)
+        if s.fp8:
+            tensor_peak, tensor_kind, probe = e4m3_peak(dev, peaks, peak_kind)
+        else:
+            tensor_peak, tensor_kind = peaks["bf16_tflops_sustained"], f"of {peak_kind} (sustained bf16)"
         glu_tensor_bound = glu_flops / (tensor_peak * 1e12) > glu_bytes / (peaks["hbm_gbs"] * 1e9)
         achieved = glu_bytes / (glu_ms * 1e-3) / 1e9
         step_s = ms / args.steps * 1e-3
         t_bytes = byts / (peaks["hbm_gbs"] * 1e9)
-        t_flops = flops / (peaks["bf16_tflops_sustained"] * (2 if s.fp8 else 1) * 1e12)
+        t_flops = flops / (tensor_peak * 1e12)
         workload = s.name
         line = {
             "metric": METRIC, "value": job_throughput(world, s.T, args.steps, ms), "unit": UNIT,
@@ -822,7 +861,8 @@ def main():
                                    "t_bytes_ms": t_bytes * 1e3, "t_flops_ms": t_flops * 1e3,
                                    "frac": max(t_bytes, t_flops) / step_s,
                                    "tensor_frac_of_bf16_peak": flops / step_s / (peaks["bf16_tflops"] * 1e12),
-                                   "peaks": peak_kind,
+                                   "peaks": peak_kind + (f"; e4m3 peak {tensor_peak} TFLOP/s {tensor_kind}"
+                                                         if s.fp8 else ""),
                                    # the same against the nominal datasheet figures (HBM 8 TB/s,
                                    # dense bf16 2.25 PFLOP/s, dense e4m3 4.5 PFLOP/s)
                                    "frac_nominal": max(byts / 8.0e12,
@@ -835,7 +875,7 @@ def main():
                           "frac": glu_flops / (glu_ms * 1e-3) / 1e12 / tensor_peak,
                           "traffic": profiled_traffic("gate_up_glu", workload),
                           "algorithmic_flops": glu_flops,
-                          "peak_kind": f"of {peak_kind} (sustained bf16" + (" x 2 for e4m3, assumed)" if s.fp8 else ")")}
+                          "peak_kind": tensor_kind}
                          if glu_tensor_bound else
                          {"kernel": "gate_up_glu (grouped tcgen05 GEMM, SiLU-GLU epilogue)",
                           "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
@@ -851,8 +891,8 @@ def main():
                            "h2d_bytes_per_step": e2e[1], "d2h_bytes_per_step": e2e[2]}
         if bias_ms is not None:
             line["config"]["bias_update_ms"] = bias_ms
-        if s.fp8 and world == 1:
-            line["config"]["e4m3_peak_probe"] = fp8_peak_probe(dev)
+        if s.fp8:
+            line["config"]["e4m3_peak_probe"] = probe
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(s, weights, x, bias, min(args.cpu_sample, s.T))
         if world == 1 and not s.fp8 and not args.no_train_summary:

@@ -64,6 +64,19 @@ __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// acc[OFF + i] += r[i] * s for the 32 values of one TMEM load, as packed
+// fp32x2 FMAs (round to nearest per lane: the same values as fmaf).
+template <int OFF>
+__device__ __forceinline__ void fold32(float (&acc)[kW8Cols], const uint32_t (&r)[32], float2 s) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float2 v = __ffma2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])), s,
+                                make_float2(acc[OFF + i], acc[OFF + i + 1]));
+    acc[OFF + i] = v.x;
+    acc[OFF + i + 1] = v.y;
+  }
+}
+
 template <class P>
 __global__ void __launch_bounds__(kF8Threads, 1) gemm8w_kernel(const __grid_constant__ typename P::Params p) {
   using L = Gemm8WSmem<P>;
@@ -198,7 +211,10 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8w_kernel(const __grid_cons
     for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++ul) {
       const int tb = ul & 1;
       const float *tok = tabs + tb * kF8TabFloats + q * 32 + lane;
-      const float *wsc = tabs + tb * kF8TabFloats + kF8MaxKB * kF8Tile + h * kF8MaxKB;
+      // weight scales of the thread's columns 0-63 and 64-127 (one weight
+      // block for both, or gate then up: P::kGateUp)
+      const float *wlo = tabs + tb * kF8TabFloats + kF8MaxKB * kF8Tile + (P::kGateUp ? 0 : h) * kF8MaxKB;
+      const float *whi = tabs + tb * kF8TabFloats + kF8MaxKB * kF8Tile + (P::kGateUp ? 1 : h) * kF8MaxKB;
       bool bad = !__all_sync(0xffffffffu, mbar_wait(sfull0 + 8 * tb, (ul >> 1) & 1, abort_flag, status));
       Unit U;
       {
@@ -220,30 +236,30 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8w_kernel(const __grid_cons
           if (lane == 0) mbar_arrive(free0 + 8 * b);
           continue;
         }
-        const float sc = tok[kb * kF8Tile] * wsc[kb];
-        const float2 s2 = make_float2(sc, sc);
+        const float ts = tok[kb * kF8Tile];
+        const float2 slo = make_float2(ts * wlo[kb], ts * wlo[kb]);
+        const float2 shi = make_float2(ts * whi[kb], ts * whi[kb]);
         const uint32_t taddr = tmem_base + b * kW8N + lane_off + h * kW8Cols;
         tc_fence_after();
-        // four 32-column loads: a load's 32 values and the 128 accumulators
-        // stay within the warpgroup's registers
-#pragma unroll
-        for (int c = 0; c < kW8Cols / 32; ++c) {
-          float v[32];
-          tmem_ld32_sync(taddr + 32 * c, v);
-          if (c == kW8Cols / 32 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(free0 + 8 * b);  // the partial is in registers
-          }
-          // packed fp32x2 FMAs (round to nearest per lane: the same values as fmaf)
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 r =
-                __ffma2_rn(make_float2(v[i], v[i + 1]), s2, make_float2(acc[32 * c + i], acc[32 * c + i + 1]));
-            acc[32 * c + i] = r.x;
-            acc[32 * c + i + 1] = r.y;
-          }
-        }
+        // four 32-column loads, each in flight while the previous one is
+        // folded (two load buffers and the 128 accumulators fit the
+        // warpgroup's registers)
+        uint32_t ra[32], rb[32];
+        tmem_ld32_nowait(taddr, ra);
+        tmem_wait_ld32(ra);
+        tmem_ld32_nowait(taddr + 32, rb);
+        fold32<0>(acc, ra, slo);
+        tmem_wait_ld32(rb);
+        tmem_ld32_nowait(taddr + 64, ra);
+        fold32<32>(acc, rb, slo);
+        tmem_wait_ld32(ra);
+        tmem_ld32_nowait(taddr + 96, rb);
+        fold32<64>(acc, ra, shi);
+        tmem_wait_ld32(rb);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(free0 + 8 * b);  // the partial is in registers
+        fold32<96>(acc, rb, shi);
       }
       if (bar_red_or(1, kF8PromoThreads, bad || *abort_flag)) goto done;
       P::epilogue_regs(p, U, acc, q, h, lane, epi_smem, tabs + tb * kF8TabFloats + kF8TabExtra);
@@ -272,6 +288,7 @@ done:
 
 // Projection out = bf16(a w^T): unit = (128-token tile m, 256-column tile n0).
 struct Dense8WPolicy : Dense8Policy {
+  static constexpr bool kGateUp = false;  // the thread's 128 columns share one weight block
   static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *) { return p.m_tiles * p.n_tiles; }
   static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *) {
     Unit U;
@@ -326,16 +343,23 @@ struct Dense8WPolicy : Dense8Policy {
   }
 };
 
-// gate/up: unit = (group, 128-wide d_ff slice m, <= 128 dispatched tokens);
-// B = the slice's 128 gate rows (column half 0) then its 128 up rows (half
-// 1).  The epilogue forms h = bf16(SiLU(g) * u) for the slice, which is
-// exactly one 128-wide K block of the down GEMM's input, and quantises it
-// there: amax over the block's bf16 values, scale amax / 448 (1 if amax is
-// 0), codes e4m3_rn_satfinite(v * (448 / amax)) in fp32, the arithmetic of
+// gate/up: unit = (group, 128-wide d_ff slice m, <= 128 dispatched tokens).
+// B interleaves gate and up rows in 64-row quarters: slice columns f 0-63 of
+// gate, then of up, then f 64-127 of gate, then of up.  So column half h of
+// the accumulator holds both factors of h for f = 64h .. 64h+63 (columns
+// 0-63 of the half gate, with the gate block's scale; 64-127 up, with the up
+// block's), and each promotion warp forms its 64 values of
+// h = bf16(SiLU(g) * u) from its own registers.  The slice is exactly one
+// 128-wide K block of the down GEMM's input, quantised here: amax over the
+// block's bf16 values (the two warps of a token quarter exchange their
+// halves' maxima), scale amax / 448 (1 if amax is 0), codes
+// e4m3_rn_satfinite(v * (448 / amax)) in fp32, the arithmetic of
 // quant_rows_kernel, so no separate pass over h is needed.
 struct Glu8WPolicy : Glu8Policy {
+  static constexpr bool kGateUp = true;  // columns 0-63 of a thread's half: gate block; 64-127: up block
+  static constexpr int kEpiSmem = 8 * 32 * 4 + 8 * 32 * 17 * 4;  // block maxima, then the code rows
   struct Params {
-    CUtensorMap wg, wu, sg, su;  // e4m3 [E*F, L] / [F, L], box 128 x 128
+    CUtensorMap wg, wu, sg, su;  // e4m3 [E*F, L] / [F, L], box 64 x 128
     TokenMaps8 tz;               // quantised dispatched z [(T*k+T), L]
     const float *wg_s, *wu_s, *sg_s, *su_s;  // [E, F/128, L/128] / [F/128, L/128]
     const float *zs_t;                        // [L/128, T*k+T] (transposed)
@@ -362,9 +386,12 @@ struct Glu8WPolicy : Glu8Policy {
   }
   static __device__ __forceinline__ void load_b(const Params &p, const Unit &U, int kb, uint32_t sb, uint32_t bar) {
     const bool sh = U.g == p.gt.E;
+    const CUtensorMap *mg = sh ? &p.sg : &p.wg, *mu = sh ? &p.su : &p.wu;
     const int row = (sh ? 0 : U.g * p.F) + U.m * kF8Tile;
-    tma_load_2d(sb, sh ? &p.sg : &p.wg, bar, kb * 128, row);
-    tma_load_2d(sb + kF8OpBytes, sh ? &p.su : &p.wu, bar, kb * 128, row);
+    tma_load_2d(sb, mg, bar, kb * 128, row);
+    tma_load_2d(sb + 64 * 128, mu, bar, kb * 128, row);
+    tma_load_2d(sb + 128 * 128, mg, bar, kb * 128, row + 64);
+    tma_load_2d(sb + 192 * 128, mu, bar, kb * 128, row + 64);
   }
   static __device__ __forceinline__ void stage_scales(const Params &p, const Unit &U, float *tok, float *w, float *,
                                                       int lane) {
@@ -374,41 +401,28 @@ struct Glu8WPolicy : Glu8Policy {
     stage_token_scales(p.zs_t, p.rows, U.row0, U.nv, kbs, tok, lane);
     stage_weight_scales((sh ? p.sg_s : p.wg_s) + blk, (sh ? p.su_s : p.wu_s) + blk, kbs, w, lane);
   }
-  // Warp (q, 0) holds its 32 tokens' 128 gate values, warp (q, 1) the up
-  // values.  In two rounds of 32 columns each hands its partner the half the
-  // partner needs (named barrier 3 + q, 64 threads); warp (q, 0) then owns h
-  // for columns 0..63 of the slice, warp (q, 1) columns 64..127.  The block
-  // amax goes through shared memory once more, and each warp writes its 64
-  // e4m3 codes per token through its own shared rows (one 16-byte store per
-  // lane covers a quarter of a token's 64 bytes, eight tokens per instruction).
+  // Warp (q, hh): h for its 32 tokens and f = 64hh .. 64hh+63 of the slice;
+  // the partner warp (q, 1-hh) holds the other 64 values of each token's
+  // block.  Each warp writes its 64 e4m3 codes per token through its own
+  // shared rows (one 16-byte store per lane covers a quarter of a token's 64
+  // bytes, eight tokens per instruction).
   static __device__ __forceinline__ void epilogue_regs(const Params &p, const Unit &U, float (&acc)[kW8Cols], int q,
                                                        int hh, int lane, uint8_t *epi, const float *) {
-    float *xb = reinterpret_cast<float *>(epi);  // [8 warps][32][33]
     const int pw = hh * 4 + q;
-    float *mine = xb + (pw * 32 + lane) * 33;
-    const float *other = xb + ((pw ^ 4) * 32 + lane) * 33;
+    float *bmax = reinterpret_cast<float *>(epi);  // [8 warps][32]
     float hv[64];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) mine[i] = hh == 0 ? acc[64 + 32 * r + i] : acc[32 * r + i];
-      named_bar_sync(3 + q, 64);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int f = 32 * r + i;                           // this warp's column f (+64 for warp (q, 1))
-        const float gv = hh == 0 ? acc[f] : other[i];
-        const float uv = hh == 0 ? other[i] : acc[64 + f];
-        hv[f] = __bfloat162float(__float2bfloat16_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
-      }
-      named_bar_sync(3 + q, 64);
-    }
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(hv[i]));
-    mine[0] = amax;
+    for (int i = 0; i < 64; ++i) {
+      const float gv = acc[i], uv = acc[64 + i];
+      hv[i] = __bfloat162float(__float2bfloat16_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
+      amax = fmaxf(amax, fabsf(hv[i]));
+    }
+    // the partner reads this slot before it passes the promotion warps'
+    // barrier at the end of the next unit, which comes before the next write
+    bmax[pw * 32 + lane] = amax;
     named_bar_sync(3 + q, 64);
-    amax = fmaxf(amax, other[0]);
-    named_bar_sync(3 + q, 64);  // both read the partner's amax before the rows are reused
+    amax = fmaxf(amax, bmax[(pw ^ 4) * 32 + lane]);
     float scale = 1.0f, inv = 0.0f;
     if (amax != 0.0f) {
       scale = amax / 448.0f;
@@ -416,7 +430,7 @@ struct Glu8WPolicy : Glu8Policy {
     }
     const int t = q * 32 + lane;
     if (hh == 0 && t < U.nv) p.hs_t[static_cast<size_t>(U.m) * p.rows + U.row0 + t] = scale;
-    uint32_t *wrow = reinterpret_cast<uint32_t *>(xb + pw * 32 * 33);  // this warp's rows: [32 tokens][17 words]
+    uint32_t *wrow = reinterpret_cast<uint32_t *>(epi + 8 * 32 * 4) + pw * 32 * 17;  // [32 tokens][17 words]
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const uint32_t lo = e4m3x2(hv[4 * i] * inv, hv[4 * i + 1] * inv);
@@ -439,7 +453,7 @@ struct Glu8WPolicy : Glu8Policy {
                                    chunk * 16) = w;
       }
     }
-    __syncwarp();  // the rows are rewritten by the next unit's exchange
+    __syncwarp();  // the rows are rewritten by the next unit's epilogue
   }
 };
 
@@ -448,6 +462,7 @@ struct Glu8WPolicy : Glu8Policy {
 // 2m + h).  The stager's slot table and the weighted, shared-memory-staged
 // slot stores are Down8Policy's, over four 32-column passes.
 struct Down8WPolicy : Down8Policy {
+  static constexpr bool kGateUp = false;  // the thread's 128 columns share one weight block
   static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
     return grouped_unit(p.gt, aux, u, kF8Tile);
   }

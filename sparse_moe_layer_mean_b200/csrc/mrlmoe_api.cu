@@ -846,11 +846,11 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     return fp4 ? make_map_packed(m, base, K / 2, rows, box_rows) : make_map(m, base, 1, K, rows, box_rows);
   };
   if (fp8_wide_glu(c)) {
-    // 128 gate + 128 up rows per unit; h is quantised in the epilogue
+    // 128 gate + 128 up rows per unit (64-row quarters); h is quantised in the epilogue
     Glu8WPolicy::Params p{};
-    if (!make_map(&p.wg, w->w_gate, 1, Ld, static_cast<uint64_t>(E) * F, 128) ||
-        !make_map(&p.wu, w->w_up_e, 1, Ld, static_cast<uint64_t>(E) * F, 128) ||
-        !make_map(&p.sg, w->w_sh_gate, 1, Ld, F, 128) || !make_map(&p.su, w->w_sh_up, 1, Ld, F, 128) ||
+    if (!make_map(&p.wg, w->w_gate, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !make_map(&p.wu, w->w_up_e, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
+        !make_map(&p.sg, w->w_sh_gate, 1, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 1, Ld, F, 64) ||
         !make_token_maps8(&p.tz, P.zq, Ld, static_cast<uint64_t>(Tk) + T))
       return MRLMOE_ERR_CUDA;
     p.wg_s = w->s_gate; p.wu_s = w->s_up_e; p.sg_s = w->s_sh_gate; p.su_s = w->s_sh_up;
