@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8w_kernel(const __grid_cons
             tc_fence_after();
             const uint32_t a_s = ring + s * L::kStageBytes;
             const uint32_t b_s = a_s + kF8OpBytes;
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               umma_f8(tmem_base + b * kW8N, sdesc_sw128(a_s + kk * 32), sdesc_sw128(b_s + kk * 32), idesc, kk != 0);
             umma_commit(empty0 + 8 * s);

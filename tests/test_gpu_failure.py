@@ -38,7 +38,10 @@ def _bias(E):
 
 @pytest.mark.parametrize("family,config,T", [("gemm", "c0_tiny", None), ("gemm_pair", "c0_tiny", None),
                                              ("gemm_fp8", "c0_fp8", None), ("gemm_fp8", "c0_fp4", None),
-                                             ("gemm_fp8", "c0_fp8", 1100)])
+                                             ("gemm_fp8", "c0_fp8", 1100),
+                                             # full width at T = 4096: the first e4m3 GEMM (the
+                                             # down-projection) runs on 256-column units
+                                             ("gemm_fp8", "c4_fp8", 4096)])
 def test_held_loads_run_out_the_bounded_waits(family, config, T):
     s = W.CONFIGS[config] if T is None else W.CONFIGS[config].with_T(T)
     x = W.make_x(s, "cuda")
