@@ -46,9 +46,10 @@ def kernels_per_step(s, sms: int) -> int:
     m_tiles = (s.T + 127) // 128
     chunks = s.n_experts // ec
     # FP8 variant: the x and n quantisers replace nothing and the z quantiser
-    # replaces the gather; h is quantised in the e4m3 gate/up epilogue, except
-    # with FP4 expert weights, where a quantiser pass over h follows the GEMM
-    extra = (3 if s.fp4 else 2) if s.fp8 else 0
+    # replaces the gather; h is quantised in the gate/up GEMM's epilogue,
+    # except with FP4 expert weights and a d_lat that does not split into
+    # 256-wide slices, where a quantiser pass over h follows the GEMM
+    extra = (3 if s.fp4 and s.d_lat % 256 else 2) if s.fp8 else 0
     if 2 * m_tiles * chunks <= 148 and s.d_lat // 64 % 2 == 0:
         return KERNELS_PER_STEP + 2 + extra
     parts = 1

@@ -68,11 +68,12 @@ typedef enum {
                                    matrices (routed gate/up/down, shared gate/up/
                                    down) hold e2m1 codes (OCP MX FP4), two per
                                    byte along K (lower index in the low nibble):
-                                   [.., out, in/2] bytes, 16-byte aligned, with
-                                   the same fp32 128x128 block scales s_*; the
+                                   [.., out, in/2] bytes, 32-byte aligned (the
+                                   tensor core reads the codes through the 4-bit
+                                   unpacking TMA type, which needs it), with the
+                                   same fp32 128x128 block scales s_*; the
                                    projections stay e4m3.  Reading of "the
-                                   release ships FP4 weights"; tuned for
-                                   decode-sized batches (token tiles of 64)   */
+                                   release ships FP4 weights"                 */
 } mrlmoe_dtype;
 
 /* How the R sigmoid router scores of a (token, expert) are aggregated into

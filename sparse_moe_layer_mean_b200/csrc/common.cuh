@@ -342,6 +342,16 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// kind::f8f6f4 operand formats (A at [7,10), B at [10,13)): e4m3 0, e2m1 5.
+// An e2m1 operand sits in shared memory as the 16U4_ALIGN16B TMA type writes
+// it: each 16 codes in the first 8 bytes of a 16-byte chunk, so the tile has
+// the e4m3 tile's footprint (128 bytes per 128-deep K row) and the MMA's
+// 32-deep K steps advance 32 bytes as for e4m3.
+constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
+__host__ __device__ constexpr uint32_t idesc_f8f6f4(int M, int N, uint32_t a_fmt, uint32_t b_fmt) {
+  return idesc_e4m3(M, N) | (a_fmt << 7) | (b_fmt << 10);
+}
+
 // 32 lanes x 32 consecutive fp32 columns: thread i of the warp gets lane
 // (32*(warp%4) + i) of the accumulator, columns [col, col+32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {

@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8w_kernel(const __grid_cons
   const int nunits = P::num_units(p, aux);
   const int kblocks = P::k_blocks(p);
   int issued = -1;  // MMA issuer: last committed K block
-  const uint32_t idesc = idesc_e4m3(kF8Tile, kW8N);
+  const uint32_t idesc = idesc_f8f6f4(kF8Tile, kW8N, kFmtE4M3, P::kWeightFormat);
   if (*abort_flag) goto done;
 
   if (warp < 4) {
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kF8Threads, 1) gemm8w_kernel(const __grid_cons
           for (int kb = 0; kb < kblocks; ++kb, ++g) {
             const uint32_t s = g % kW8Ring;
             if (g >= kW8Ring && !mbar_wait(empty0 + 8 * s, ((g / kW8Ring) - 1) & 1, abort_flag, status)) goto done;
-            mbar_arrive_expect_tx(full0 + 8 * s, isA ? P::a_bytes(U) : static_cast<uint32_t>(kW8BBytes));
+            mbar_arrive_expect_tx(full0 + 8 * s, isA ? P::a_bytes(U) : P::kWeightTxBytes);
             const uint32_t st = ring + s * L::kStageBytes;
             if (isA)
               P::load_a(p, U, kb, st, full0 + 8 * s);
@@ -288,6 +288,8 @@ done:
 
 // Projection out = bf16(a w^T): unit = (128-token tile m, 256-column tile n0).
 struct Dense8WPolicy : Dense8Policy {
+  static constexpr uint32_t kWeightFormat = kFmtE4M3;
+  static constexpr uint32_t kWeightTxBytes = kW8BBytes;  // bytes the weight loads of a K block complete
   static constexpr bool kGateUp = false;  // the thread's 128 columns share one weight block
   static __device__ __forceinline__ int num_units(const Params &p, const uint8_t *) { return p.m_tiles * p.n_tiles; }
   static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *) {
@@ -356,6 +358,8 @@ struct Dense8WPolicy : Dense8Policy {
 // e4m3_rn_satfinite(v * (448 / amax)) in fp32, the arithmetic of
 // quant_rows_kernel, so no separate pass over h is needed.
 struct Glu8WPolicy : Glu8Policy {
+  static constexpr uint32_t kWeightFormat = kFmtE4M3;
+  static constexpr uint32_t kWeightTxBytes = kW8BBytes;  // bytes the weight loads of a K block complete
   static constexpr bool kGateUp = true;  // columns 0-63 of a thread's half: gate block; 64-127: up block
   static constexpr int kEpiSmem = 8 * 32 * 4 + 8 * 32 * 17 * 4;  // block maxima, then the code rows
   struct Params {
@@ -462,6 +466,8 @@ struct Glu8WPolicy : Glu8Policy {
 // 2m + h).  The stager's slot table and the weighted, shared-memory-staged
 // slot stores are Down8Policy's, over four 32-column passes.
 struct Down8WPolicy : Down8Policy {
+  static constexpr uint32_t kWeightFormat = kFmtE4M3;
+  static constexpr uint32_t kWeightTxBytes = kW8BBytes;  // bytes the weight loads of a K block complete
   static constexpr bool kGateUp = false;  // the thread's 128 columns share one weight block
   static __device__ __forceinline__ Unit unit(const Params &p, int u, const uint8_t *aux) {
     return grouped_unit(p.gt, aux, u, kF8Tile);
@@ -507,6 +513,23 @@ struct Down8WPolicy : Down8Policy {
       __syncwarp();
     }
   }
+};
+
+// FP4 expert weights: the same units with each weight matrix given as packed
+// e2m1 codes (two per byte, the lower K index in the low nibble).  The weight
+// maps use the 16U4_ALIGN16B TMA type, which unpacks 16 codes into each 16
+// bytes of the shared tile (and completes half a byte per code on the
+// barrier), and the MMA reads B as e2m1 (every e2m1 value is an e4m3 value,
+// so the partial products equal those of the codes expanded to e4m3);
+// scales, promotion and epilogues are the e4m3 policies'.
+struct Glu4WPolicy : Glu8WPolicy {
+  static constexpr uint32_t kWeightFormat = kFmtE2M1;
+  static constexpr uint32_t kWeightTxBytes = kW8BBytes / 2;  // counted as packed codes, half a byte each
+};
+
+struct Down4WPolicy : Down8WPolicy {
+  static constexpr uint32_t kWeightFormat = kFmtE2M1;
+  static constexpr uint32_t kWeightTxBytes = kW8BBytes / 2;
 };
 
 }  // namespace mrl

@@ -289,6 +289,23 @@ bool make_map_packed(CUtensorMap *m, const void *base, uint64_t inner_bytes, uin
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed e2m1 codes [rows, K/2 bytes] read as K 4-bit elements per row and
+// unpacked by the TMA into 16-byte chunks of 16 codes (16U4_ALIGN16B; boxes of
+// 128 codes x box_rows rows, SWIZZLE_128B: the e4m3 tile's shared layout).
+// The type needs a 32-byte-aligned base, K a multiple of 128 and a row stride
+// that is a multiple of 32 bytes; the encoder refuses anything else.
+bool make_map_e2m1(CUtensorMap *m, const void *base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 31u)) return false;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K / 2};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The four box heights of an e4m3 token tensor [rows, inner] (load_token_rows8).
 bool make_token_maps8(TokenMaps8 *t, const void *base, uint64_t inner, uint64_t rows) {
   return make_map(&t->m16, base, 1, inner, rows, 16) && make_map(&t->m32, base, 1, inner, rows, 32) &&
@@ -475,11 +492,21 @@ bool fp8_wide_glu(const mrlmoe_config &c) {
 bool fp8_wide_down(const mrlmoe_config &c) {
   return c.dtype == MRLMOE_FP8_E4M3_BLOCK128 && c.d_lat % kW8N == 0 && wide8_ready<Down8WPolicy>();
 }
+// FP4 expert weights on the same 256-column units (the tensor core reads the
+// e2m1 codes) when d_lat splits into 256-wide slices; else the 128-column
+// kernel expands them to e4m3 in shared memory, with 64-token units.
+bool fp4_wide(const mrlmoe_config &c) {
+  return c.dtype == MRLMOE_FP4_E2M1_BLOCK128 && c.d_lat % kW8N == 0 && wide8_ready<Glu4WPolicy>() &&
+         wide8_ready<Down4WPolicy>();
+}
 
 GroupTiling group_tiling(const mrlmoe_config &c) {
   if (c.dtype == MRLMOE_FP8_E4M3_BLOCK128)
     return {kF8Tile, c.d_ff / (fp8_wide_glu(c) ? 128 : 64), c.d_lat / (fp8_wide_down(c) ? kW8N : 128)};
-  if (c.dtype == MRLMOE_FP4_E2M1_BLOCK128) return {kF4TokTile, c.d_ff / 64, c.d_lat / 128};
+  if (c.dtype == MRLMOE_FP4_E2M1_BLOCK128) {
+    if (fp4_wide(c)) return {kF8Tile, c.d_ff / 128, c.d_lat / kW8N};
+    return {kF4TokTile, c.d_ff / 64, c.d_lat / 128};
+  }
   return {kExpertBN, glu_m_tiles(c), down_m_tiles(c)};
 }
 
@@ -515,12 +542,17 @@ mrlmoe_status check_weights_bf16(const mrlmoe_weights *w, bool need_all) {
   return MRLMOE_OK;
 }
 
-mrlmoe_status check_weights_fp8(const mrlmoe_weights *w) {
+// FP8 / FP4 weights: every code matrix 16-byte aligned; with FP4 experts the
+// six expert matrices 32-byte aligned (the 4-bit unpacking TMA type).
+mrlmoe_status check_weights_fp8(const mrlmoe_weights *w, bool fp4) {
   if (!w || !w->w_router || !w->expert_scale || !w->rms_gain || !aligned16(w->w_router)) return MRLMOE_ERR_INVALID_ARG;
   const void *codes[] = {w->w_down, w->w_gate, w->w_up_e, w->w_down_e, w->w_sh_gate, w->w_sh_up, w->w_sh_down, w->w_up};
   const float *scales[] = {w->s_down, w->s_gate, w->s_up_e, w->s_down_e, w->s_sh_gate, w->s_sh_up, w->s_sh_down, w->s_up};
   for (const void *p : codes)
     if (!p || !aligned16(p)) return MRLMOE_ERR_INVALID_ARG;
+  if (fp4)
+    for (const void *p : {w->w_gate, w->w_up_e, w->w_down_e, w->w_sh_gate, w->w_sh_up, w->w_sh_down})
+      if (reinterpret_cast<uintptr_t>(p) & 31u) return MRLMOE_ERR_INVALID_ARG;
   for (const float *p : scales)
     if (!p) return MRLMOE_ERR_INVALID_ARG;
   return MRLMOE_OK;
@@ -726,7 +758,9 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   if (train && !train_supported(*cfg)) return MRLMOE_ERR_UNSUPPORTED;
   if (!bias || !x || !y || !aligned16(x) || !aligned16(y)) return MRLMOE_ERR_INVALID_ARG;
   const bool fp8 = cfg->dtype != MRLMOE_BF16;  // e4m3 projections and activations (FP8 and FP4 variants)
-  if ((s = fp8 ? check_weights_fp8(w) : check_weights_bf16(w, true)) != MRLMOE_OK) return s;
+  if ((s = fp8 ? check_weights_fp8(w, cfg->dtype == MRLMOE_FP4_E2M1_BLOCK128) : check_weights_bf16(w, true)) !=
+      MRLMOE_OK)
+    return s;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MRLMOE_ERR_WORKSPACE;
   if (ws_bytes < layout_of(*cfg, train).total) return MRLMOE_ERR_WORKSPACE;
   int sms = 0;
@@ -845,12 +879,16 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
   auto wmap = [&](CUtensorMap *m, const void *base, uint64_t K, uint64_t rows, uint32_t box_rows) {
     return fp4 ? make_map_packed(m, base, K / 2, rows, box_rows) : make_map(m, base, 1, K, rows, box_rows);
   };
-  if (fp8_wide_glu(c)) {
+  const bool wide4 = fp4_wide(c);
+  if (fp8_wide_glu(c) || wide4) {
     // 128 gate + 128 up rows per unit (64-row quarters); h is quantised in the epilogue
     Glu8WPolicy::Params p{};
-    if (!make_map(&p.wg, w->w_gate, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
-        !make_map(&p.wu, w->w_up_e, 1, Ld, static_cast<uint64_t>(E) * F, 64) ||
-        !make_map(&p.sg, w->w_sh_gate, 1, Ld, F, 64) || !make_map(&p.su, w->w_sh_up, 1, Ld, F, 64) ||
+    auto wmapw = [&](CUtensorMap *m, const void *base, uint64_t rows) {
+      return wide4 ? make_map_e2m1(m, base, Ld, rows, 64) : make_map(m, base, 1, Ld, rows, 64);
+    };
+    const uint64_t EF = static_cast<uint64_t>(E) * F;
+    if (!wmapw(&p.wg, w->w_gate, EF) || !wmapw(&p.wu, w->w_up_e, EF) || !wmapw(&p.sg, w->w_sh_gate, F) ||
+        !wmapw(&p.su, w->w_sh_up, F) ||
         !make_token_maps8(&p.tz, P.zq, Ld, static_cast<uint64_t>(Tk) + T))
       return MRLMOE_ERR_CUDA;
     p.wg_s = w->s_gate; p.wu_s = w->s_up_e; p.sg_s = w->s_sh_gate; p.su_s = w->s_sh_up;
@@ -861,7 +899,10 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     p.hs_t = P.hs;
     p.F = F; p.L = Ld;
     p.status = P.status;
-    MRL_TRY(launch_gemm8w<Glu8WPolicy>(p, sms, st));
+    if (wide4)
+      MRL_TRY(launch_gemm8w<Glu4WPolicy>(p, sms, st));
+    else
+      MRL_TRY(launch_gemm8w<Glu8WPolicy>(p, sms, st));
   } else {
     Glu8Policy::Params p{};
     if (!wmap(&p.wg, w->w_gate, Ld, static_cast<uint64_t>(E) * F, 64) ||
@@ -885,9 +926,12 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
   if (!mark(5)) return MRLMOE_ERR_CUDA;
   {
     Down8Policy::Params p{};
-    if (!wmap(&p.wd, w->w_down_e, F, static_cast<uint64_t>(E) * Ld, 128) || !wmap(&p.sd, w->w_sh_down, F, Ld, 128) ||
-        !make_token_maps8(&p.th, P.hq, F, static_cast<uint64_t>(Tk) + T))
+    if (wide4 ? !make_map_e2m1(&p.wd, w->w_down_e, F, static_cast<uint64_t>(E) * Ld, 128) ||
+                    !make_map_e2m1(&p.sd, w->w_sh_down, F, Ld, 128)
+              : !wmap(&p.wd, w->w_down_e, F, static_cast<uint64_t>(E) * Ld, 128) ||
+                    !wmap(&p.sd, w->w_sh_down, F, Ld, 128))
       return MRLMOE_ERR_CUDA;
+    if (!make_token_maps8(&p.th, P.hq, F, static_cast<uint64_t>(Tk) + T)) return MRLMOE_ERR_CUDA;
     p.wd_s = w->s_down_e; p.sd_s = w->s_sh_down;
     p.hs_t = P.hs;
     p.rows = Tk + T;
@@ -897,7 +941,9 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     p.slots = P.slots;
     p.L = Ld; p.F = F; p.k = k; p.Tk = Tk;
     p.status = P.status;
-    if (fp4)
+    if (wide4)
+      MRL_TRY(launch_gemm8w<Down4WPolicy>(p, sms, st));
+    else if (fp4)
       MRL_TRY(launch_gemm8<Down4Policy>(p, sms, st));
     else if (fp8_wide_down(c))
       MRL_TRY(launch_gemm8w<Down8WPolicy>(p, sms, st));

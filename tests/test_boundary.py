@@ -97,6 +97,15 @@ def test_forward_rejects_bad_arguments_before_cuda():
     assert _raw_forward(cfg8, full, 4096, 4096, 4096, 4096, need8) == 1
     full8 = N.Weights(*([4096] * 11 + [8192] * 8))
     assert _raw_forward(cfg8, full8, 4096, 4096, 4096, 4096, need8 - 1) == 3
+    # FP4 experts: the six expert code matrices must be 32-byte aligned (the
+    # 4-bit unpacking TMA type); 16 bytes is enough for the FP8 variant
+    cfg4 = _cfg(dtype=2)
+    need4 = M.mrlmoe_workspace_size(cfg4)
+    for i in range(2, 8):                                                 # w_gate .. w_sh_down
+        ptrs = [4096] * 11 + [8192] * 8
+        ptrs[i] = 4096 + 16
+        assert _raw_forward(cfg4, N.Weights(*ptrs), 4096, 4096, 4096, 4096, need4) == 1, N.WEIGHT_FIELDS[i]
+        assert _raw_forward(cfg8, N.Weights(*ptrs), 4096, 4096, 4096, 4096, need8 - 1) == 3
 
 
 def test_route_rejects_bad_arguments_before_cuda():

@@ -322,18 +322,20 @@ def test_forward_fp8_groups_of_every_size_larger_T():
     check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
 
 
-def _fp8_mid_width(T):
+def _fp8_mid_width(T, fp4=False):
     # d_lat 512 (two 256-wide slices in the expert-down units), d_ff 384
     # (three 128-wide gate/up slices), d_model 384 (the up-projection's last
     # 256-column unit half outside N); at T = 10100 both projections run on
-    # 256-column units (79 token tiles x 2 column tiles)
-    return W.LayerShape("fp8_mid", T=T, d_model=384, d_lat=512, n_experts=16, top_k=2, d_ff=384, n_routers=2,
-                        fp8=True, outlier_frac=0.01)
+    # 256-column units (79 token tiles x 2 column tiles).  With fp4 the six
+    # expert matrices are e2m1 codes, which the same units read through the
+    # 4-bit unpacking TMA type.
+    return W.LayerShape("fp4_mid" if fp4 else "fp8_mid", T=T, d_model=384, d_lat=512, n_experts=16, top_k=2,
+                        d_ff=384, n_routers=2, fp8=True, fp4=fp4, outlier_frac=0.01)
 
 
-@pytest.mark.parametrize("T", [300, 10100])
-def test_forward_fp8_mid_width(T):
-    s = _fp8_mid_width(T)
+@pytest.mark.parametrize("T,fp4", [(300, False), (10100, False), (300, True), (10100, True)])
+def test_forward_fp8_mid_width(T, fp4):
+    s = _fp8_mid_width(T, fp4)
     w = W.make_layer_weights(s, "cuda", seed=0)
     x = W.make_x(s, "cuda", seed=0)
     bias = W.uniform((s.n_experts,), -0.01, 0.01, 4, 901, "cuda")
