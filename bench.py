@@ -79,7 +79,7 @@ def parse_args():
     ap.add_argument("--no-train-summary", action="store_true",
                     help="leave the training-step summary out of the forward's line")
     ap.add_argument("--no-other-configs", action="store_true",
-                    help="leave the c1_decode / c3_skew / c4_fp8 summaries out of the headline's line")
+                    help="leave the c1_decode / c3_skew / c4_fp8 / c1_fp4 summaries out of the headline's line")
     ap.add_argument("--train", action="store_true",
                     help="time a training step (forward that keeps its activations + backward) instead")
     ap.add_argument("--route-only", action="store_true",
@@ -292,19 +292,25 @@ def e4m3_peak(dev, peaks, peak_kind):
 
 
 def glu_roofline(s, glu_ms, touched, peaks, peak_kind, dev):
-    """The gate/up kernel against its bound: e4m3 FLOPs against the e4m3 peak,
-    bf16 weight bytes against the measured HBM bandwidth."""
+    """The gate/up kernel against its bound, the larger of its two floors:
+    the touched experts' gate and up weight bytes at the measured HBM copy
+    rate, or its FLOPs at the tensor peak of its operand type (e4m3 / e2m1:
+    the vendor e4m3 GEMM probe; bf16: the measured sustained bf16 peak)."""
     if s.fp8:
-        tpeak, kind, _ = e4m3_peak(dev, peaks, peak_kind)
-        achieved = glu_kernel_flops(s) / (glu_ms * 1e-3) / 1e12
+        tpeak, tkind, _ = e4m3_peak(dev, peaks, peak_kind)
+    else:
+        tpeak, tkind = peaks["bf16_tflops_sustained"], f"of {peak_kind} (sustained bf16)"
+    byts, flops = glu_kernel_bytes(s, touched), glu_kernel_flops(s)
+    if flops / (tpeak * 1e12) > byts / (peaks["hbm_gbs"] * 1e9):
+        achieved = flops / (glu_ms * 1e-3) / 1e12
         return {"bound": "tensor", "achieved": achieved, "peak": tpeak, "unit": "TFLOP/s",
-                "frac": achieved / tpeak, "peak_kind": kind}
-    achieved = glu_kernel_bytes(s, touched) / (glu_ms * 1e-3) / 1e9
+                "frac": achieved / tpeak, "peak_kind": tkind}
+    achieved = byts / (glu_ms * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "peak_kind": f"of {peak_kind}"}
 
 
-OTHER_CONFIGS = ("c1_decode", "c3_skew", "c4_fp8")
+OTHER_CONFIGS = ("c1_decode", "c3_skew", "c4_fp8", "c1_fp4")
 
 
 def config_summary(name, dev, bf16_weights, steps=20, warmup=3):
