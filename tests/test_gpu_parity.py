@@ -333,8 +333,11 @@ def _fp8_mid_width(T, fp4=False):
                         d_ff=384, n_routers=2, fp8=True, fp4=fp4, outlier_frac=0.01)
 
 
-@pytest.mark.parametrize("T,fp4", [(300, False), (10100, False), (300, True), (10100, True)])
+@pytest.mark.parametrize("T,fp4", [(300, False), (10100, False), (300, True), (10100, True), (64, False),
+                                   (64, True)])
 def test_forward_fp8_mid_width(T, fp4):
+    # T = 64: 8 rows per expert on average (groups of 0 to ~20 rows, one
+    # 16- or 32-row token box each)
     s = _fp8_mid_width(T, fp4)
     w = W.make_layer_weights(s, "cuda", seed=0)
     x = W.make_x(s, "cuda", seed=0)
@@ -350,6 +353,28 @@ def test_forward_fp8_mid_width(T, fp4):
         tokens = hard_tokens(r, s.T, s.n_experts, s.top_k, bn=128, want=300, seed=6)
         tokens = torch.unique(torch.cat([tokens, torch.arange(T - 140, T)]))
     _compare_fp8(s, x, bias, y, r, {k: v.cpu() for k, v in w.items()}, tokens=tokens)
+
+
+@pytest.mark.parametrize("fp4", [False, True])
+def test_forward_fp8_small_batch_hot_expert(fp4):
+    # T = 64 with expert 0 taking every token (64 rows in one unit), expert 5
+    # favoured and the rest holding 0 to a few rows
+    s = _fp8_mid_width(64, fp4)
+    w = W.make_layer_weights(s, "cuda", seed=1)
+    x = W.make_x(s, "cuda", seed=1)
+    bias = torch.linspace(0.0, 0.05, s.n_experts, dtype=torch.float32)
+    bias[0] = 10.0
+    bias[5] += 0.2
+    bias = bias.cuda()
+    layer = M.MRLMoELayer(s, w)
+    r = layer.routing_buffers(scores=False)
+    y = layer(x, bias, routing=r)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    counts = r["counts"].cpu()
+    assert int(counts[0]) == 64 and int(counts.min()) < 8
+    check_dispatch_properties(r, s.T, s.n_experts, s.top_k)
+    _compare_fp8(s, x, bias, y, r, {k: v.cpu() for k, v in w.items()})
 
 
 def test_forward_c4_fp8_sampled_tokens():
