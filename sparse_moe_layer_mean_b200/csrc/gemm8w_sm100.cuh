@@ -414,12 +414,17 @@ struct Glu8WPolicy : Glu8Policy {
                                                        int hh, int lane, uint8_t *epi, const float *) {
     const int pw = hh * 4 + q;
     float *bmax = reinterpret_cast<float *>(epi);  // [8 warps][32]
+    // SiLU(g) = g / 2 * (1 + tanh(g / 2)): one special-function instruction
+    // per value (exp and reciprocal would take two), with tanh.approx's error
+    // (about 2^-11 relative) far below the e4m3 step h is quantised to next
     float hv[64];
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 64; ++i) {
-      const float gv = acc[i], uv = acc[64 + i];
-      hv[i] = __bfloat162float(__float2bfloat16_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
+      const float hg = 0.5f * acc[i], uv = acc[64 + i];
+      float th;
+      asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(hg));
+      hv[i] = __bfloat162float(__float2bfloat16_rn(fmaf(hg, th, hg) * uv));
       amax = fmaxf(amax, fabsf(hv[i]));
     }
     // the partner reads this slot before it passes the promotion warps'
@@ -463,8 +468,9 @@ struct Glu8WPolicy : Glu8Policy {
 
 // expert down: unit = (group, 256-wide d_lat slice m, <= 128 dispatched
 // tokens); column half h = d_lat rows 256m + 128h .. +127 (weight block
-// 2m + h).  The stager's slot table and the weighted, shared-memory-staged
-// slot stores are Down8Policy's, over four 32-column passes.
+// 2m + h).  The stager's slot table is Down8Policy's; the weighted slot
+// stores go through the warp's shared rows in four 32-column passes, so each
+// store instruction covers four tokens' 128 contiguous bytes.
 struct Down8WPolicy : Down8Policy {
   static constexpr uint32_t kWeightFormat = kFmtE4M3;
   static constexpr uint32_t kWeightTxBytes = kW8BBytes;  // bytes the weight loads of a K block complete
@@ -492,23 +498,27 @@ struct Down8WPolicy : Down8Policy {
                                                        int h, int lane, uint8_t *epi, const float *extra) {
     const int *slot = reinterpret_cast<const int *>(extra);
     const float *wt = extra + kF8Tile;
-    float *wrow = reinterpret_cast<float *>(epi) + (h * 4 + q) * 32 * 33;  // this warp's rows: [32 tokens][33]
+    // this warp's rows: [32 tokens][32 floats], 16-byte chunk c of row r at
+    // chunk c ^ (r & 7), so the 128-bit writes of a quarter-warp (eight rows)
+    // and its 128-bit reads (one row's eight chunks) both spread over all banks
+    float4 *wrow = reinterpret_cast<float4 *>(epi) + (h * 4 + q) * 32 * 8;
     const float my_wt = q * 32 + lane < U.nv ? wt[q * 32 + lane] : 0.f;
     const int part = lane & 7;  // 16-byte eighth of a token's 128 bytes
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) wrow[lane * 33 + i] = acc[pass * 32 + i] * my_wt;
+      for (int c = 0; c < 8; ++c) {
+        const float *a = acc + pass * 32 + 4 * c;
+        wrow[lane * 8 + (c ^ (lane & 7))] = make_float4(a[0] * my_wt, a[1] * my_wt, a[2] * my_wt, a[3] * my_wt);
+      }
       __syncwarp();
 #pragma unroll
       for (int it = 0; it < 8; ++it) {
         const int i = it * 4 + (lane >> 3);  // token within the warp
         const int t = q * 32 + i;
-        if (t < U.nv) {
-          const float *src = wrow + i * 33 + part * 4;
+        if (t < U.nv)
           *reinterpret_cast<float4 *>(p.slots + static_cast<size_t>(slot[t]) * p.L + U.m * kW8N + h * kW8Cols +
-                                      pass * 32 + part * 4) = make_float4(src[0], src[1], src[2], src[3]);
-        }
+                                      pass * 32 + part * 4) = wrow[i * 8 + (part ^ (i & 7))];
       }
       __syncwarp();
     }
