@@ -417,15 +417,24 @@ struct Glu8WPolicy : Glu8Policy {
     // SiLU(g) = g / 2 * (1 + tanh(g / 2)): one special-function instruction
     // per value (exp and reciprocal would take two), with tanh.approx's error
     // (about 2^-11 relative) far below the e4m3 step h is quantised to next
+    // (the bf16 rounding of h goes two values per conversion: cvt.rn.bf16x2
+    // rounds each half as the scalar conversion does)
     float hv[64];
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      const float hg = 0.5f * acc[i], uv = acc[64 + i];
-      float th;
-      asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(hg));
-      hv[i] = __bfloat162float(__float2bfloat16_rn(fmaf(hg, th, hg) * uv));
-      amax = fmaxf(amax, fabsf(hv[i]));
+    for (int i = 0; i < 64; i += 2) {
+      float v[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float hg = 0.5f * acc[i + e], uv = acc[64 + i + e];
+        float th;
+        asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(hg));
+        v[e] = fmaf(hg, th, hg) * uv;
+      }
+      const uint32_t b2 = pack_bf16x2(v[0], v[1]);
+      hv[i] = __uint_as_float(b2 << 16);
+      hv[i + 1] = __uint_as_float(b2 & 0xffff0000u);
+      amax = fmaxf(amax, fmaxf(fabsf(hv[i]), fabsf(hv[i + 1])));
     }
     // the partner reads this slot before it passes the promotion warps'
     // barrier at the end of the next unit, which comes before the next write
