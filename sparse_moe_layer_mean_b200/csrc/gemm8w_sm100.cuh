@@ -423,15 +423,13 @@ struct Glu8WPolicy : Glu8Policy {
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 64; i += 2) {
-      float v[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float hg = 0.5f * acc[i + e], uv = acc[64 + i + e];
-        float th;
-        asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(hg));
-        v[e] = fmaf(hg, th, hg) * uv;
-      }
-      const uint32_t b2 = pack_bf16x2(v[0], v[1]);
+      // packed fp32x2 arithmetic (round to nearest per lane)
+      const float2 hg = __fmul2_rn(make_float2(acc[i], acc[i + 1]), make_float2(0.5f, 0.5f));
+      float2 th;
+      asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(hg.x));
+      asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(hg.y));
+      const float2 v = __fmul2_rn(__ffma2_rn(hg, th, hg), make_float2(acc[64 + i], acc[64 + i + 1]));
+      const uint32_t b2 = pack_bf16x2(v.x, v.y);
       hv[i] = __uint_as_float(b2 << 16);
       hv[i + 1] = __uint_as_float(b2 & 0xffff0000u);
       amax = fmaxf(amax, fmaxf(fabsf(hv[i]), fabsf(hv[i + 1])));
@@ -451,8 +449,10 @@ struct Glu8WPolicy : Glu8Policy {
     uint32_t *wrow = reinterpret_cast<uint32_t *>(epi + 8 * 32 * 4) + pw * 32 * 17;  // [32 tokens][17 words]
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const uint32_t lo = e4m3x2(hv[4 * i] * inv, hv[4 * i + 1] * inv);
-      const uint32_t hi = e4m3x2(hv[4 * i + 2] * inv, hv[4 * i + 3] * inv);
+      const float2 a = __fmul2_rn(make_float2(hv[4 * i], hv[4 * i + 1]), make_float2(inv, inv));
+      const float2 b = __fmul2_rn(make_float2(hv[4 * i + 2], hv[4 * i + 3]), make_float2(inv, inv));
+      const uint32_t lo = e4m3x2(a.x, a.y);
+      const uint32_t hi = e4m3x2(b.x, b.y);
       wrow[lane * 17 + i] = lo | (hi << 16);
     }
     __syncwarp();
@@ -518,7 +518,9 @@ struct Down8WPolicy : Down8Policy {
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const float *a = acc + pass * 32 + 4 * c;
-        wrow[lane * 8 + (c ^ (lane & 7))] = make_float4(a[0] * my_wt, a[1] * my_wt, a[2] * my_wt, a[3] * my_wt);
+        const float2 lo = __fmul2_rn(make_float2(a[0], a[1]), make_float2(my_wt, my_wt));
+        const float2 hi = __fmul2_rn(make_float2(a[2], a[3]), make_float2(my_wt, my_wt));
+        wrow[lane * 8 + (c ^ (lane & 7))] = make_float4(lo.x, lo.y, hi.x, hi.y);
       }
       __syncwarp();
 #pragma unroll
