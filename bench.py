@@ -14,6 +14,7 @@ For N > 1 launch with torchrun; every rank runs its own batch on its own GPU
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import glob
 import json
@@ -313,17 +314,18 @@ def glu_roofline(s, glu_ms, touched, peaks, peak_kind, dev):
 OTHER_CONFIGS = ("c1_decode", "c3_skew", "c4_fp8", "c1_fp4")
 
 
-def config_summary(name, dev, bf16_weights, steps=20, warmup=3):
+def config_summary(name, dev, bf16_weights, steps=20, warmup=3, shape=None):
     """One more workload, timed on its own after the headline's timed region:
     ms per forward (CUDA events on the launching stream), tokens/s, the
     layer's roofline fraction and the stage times; the skewed workload also
     times its balancing-bias update.  The bf16 workloads reuse the headline's
-    weights (same layer shape); the e4m3 one draws its own."""
+    weights (same layer shape); the e4m3 one draws its own.  ``shape``
+    replaces the named config's (e.g. another router aggregation)."""
     import torch
     import sparse_moe_layer_mean_b200 as M
     import workloads as W
     try:
-        s = W.CONFIGS[name]
+        s = shape if shape is not None else W.CONFIGS[name]
         weights = W.make_layer_weights(s, dev) if s.fp8 else bf16_weights
         x = W.make_x(s, dev)
         bias = W.make_bias(s, dev)
@@ -388,6 +390,73 @@ def config_summary(name, dev, bf16_weights, steps=20, warmup=3):
             del weights
         torch.cuda.empty_cache()
         return out
+    except Exception as e:  # the headline line is printed either way
+        return {"error": str(e).splitlines()[0][:200] if str(e) else type(e).__name__}
+
+
+def ep_summary(n, dev, bf16_weights, T=4096, iters=5, steps=20):
+    """The expert-parallel form emulated on one GPU: n ranks in one process,
+    the headline's full-width weights, T tokens per rank.  Rank d routes its
+    own tokens, runs experts [d E/n, (d+1) E/n) on every rank's rows for them
+    and combines its tokens (sparse_moe_layer_mean_b200.ep.emulate_forward).
+    Each phase's device time per rank comes from CUDA events (median of
+    ``iters`` runs), next to the single-GPU forward of one rank's T tokens.
+    The exchanges are device copies of the slices here; on n GPUs they cross
+    NVLink, so the line gives the bytes each rank sends and receives, not a
+    transfer time (the exchange over NVLink is unmeasured: every GPU call on
+    this pool has one GPU)."""
+    import torch
+    import sparse_moe_layer_mean_b200 as M
+    import workloads as W
+    from sparse_moe_layer_mean_b200 import ep as EP
+    try:
+        s = W.CONFIGS["c2_prefill"].with_T(T)
+        ranks = [EP.ExpertParallelRank(s, bf16_weights, r, n, device=dev) for r in range(n)]
+        xs = [W.make_x(s, dev, seed=100 + r) for r in range(n)]
+        bias = W.make_bias(s, dev)
+        EP.emulate_forward(ranks, xs, bias)                      # warm-up
+        torch.cuda.synchronize()
+        runs, splits = [], None
+        for _ in range(iters):
+            ev = {}
+            EP.emulate_forward(ranks, xs, bias, events=ev)
+            torch.cuda.synchronize()
+            splits = ev.pop("splits")
+            runs.append({k: [a.elapsed_time(b) for a, b in v] for k, v in ev.items()})
+        if any(rk.status() != 0 for rk in ranks):
+            raise RuntimeError("device status non-zero after the expert-parallel runs")
+
+        def med(vals):
+            return sorted(vals)[len(vals) // 2]
+        phase = {ph: [round(med([r[ph][i] for r in runs]), 4) for i in range(n)]
+                 for ph in ("dispatch", "experts", "combine")}
+        per_rank = [phase["dispatch"][i] + phase["experts"][i] + phase["combine"][i] for i in range(n)]
+        del ranks
+        torch.cuda.empty_cache()
+        # the single-GPU forward of one rank's tokens, same weights
+        layer = M.MRLMoELayer(s, bf16_weights, device=dev)
+        y = torch.empty(T, s.d_model, dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            layer(xs[0], bias, y=y)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            layer(xs[0], bias, y=y)
+        b.record()
+        torch.cuda.synchronize()
+        if layer.device_status() != 0:
+            raise RuntimeError("device status non-zero after the single-GPU forward")
+        fwd = a.elapsed_time(b) / steps
+        L = s.d_lat
+        out_rows = [sum(splits[r][d] for d in range(n) if d != r) for r in range(n)]
+        in_rows = [sum(splits[q][r] for q in range(n) if q != r) for r in range(n)]
+        return {"n_ranks": n, "tokens_per_rank": T, "experts_per_rank": s.n_experts // n,
+                "phase_ms": phase, "compute_ms_per_rank_max": round(max(per_rank), 4),
+                "single_gpu_forward_ms": round(fwd, 4),
+                "emulated_exchange_copies_ms": {ph: round(med([r[ph][0] for r in runs]), 4) for ph in ("rows", "back")},
+                "bytes_per_rank_max": {"rows_out_bf16": max(out_rows) * L * 2, "rows_in_bf16": max(in_rows) * L * 2,
+                                       "outputs_back_fp32": max(in_rows) * L * 4},
+                "exchange": "unmeasured (one GPU): device copies stand in for the NVLink all-to-alls"}
     except Exception as e:  # the headline line is printed either way
         return {"error": str(e).splitlines()[0][:200] if str(e) else type(e).__name__}
 
@@ -906,6 +975,12 @@ def main():
             line["train_step"] = train_summary(s, dev, weights, x, bias)
         if world == 1 and s.name == "c2_prefill" and not args.no_other_configs:
             line["other_configs"] = {n: config_summary(n, dev, weights) for n in OTHER_CONFIGS}
+            # the router aggregation variants (sum, max) of the headline workload
+            line["aggregation_variants"] = {
+                agg: config_summary("c2_prefill", dev, weights,
+                                    shape=dataclasses.replace(s, aggregation=agg, name=f"c2_prefill_{agg}"))
+                for agg in ("sum", "max")}
+            line["ep_emulated"] = ep_summary(8, dev, weights)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier(device_ids=[local])

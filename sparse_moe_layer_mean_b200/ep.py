@@ -170,21 +170,43 @@ def forward_distributed(rank: ExpertParallelRank, x, bias, exchange: Optional[Di
     return rank.combine(ret)
 
 
-def emulate_forward(ranks: Sequence[ExpertParallelRank], xs: Sequence[object], bias):
+def emulate_forward(ranks: Sequence[ExpertParallelRank], xs: Sequence[object], bias, events: Optional[dict] = None):
     """All ranks in one process on one GPU: each exchange is a device copy of
     every (source, destination) slice into the destination's receive buffer.
-    Returns the list of y, one per rank."""
+    Returns the list of y, one per rank.  With ``events`` (a dict), CUDA
+    events are recorded around each rank's phases on the current stream:
+    events[phase] is a list of (start, end) pairs, phase one of "dispatch"
+    and "combine" (per source rank), "experts" (per owner), "rows" and
+    "back" (the two exchanges, all ranks' copies together); events["splits"]
+    holds the rows each rank sent each rank."""
     import torch
     n = len(ranks)
     E = ranks[0].E
     per = E // n
-    disp = [rk.dispatch(x, bias) for rk, x in zip(ranks, xs)]
+
+    def mark(phase):
+        if events is None:
+            return None
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        events.setdefault(phase, []).append((a, b))
+        a.record()
+        return b
+
+    disp = []
+    for rk, x in zip(ranks, xs):
+        e = mark("dispatch")
+        disp.append(rk.dispatch(x, bias))
+        if e is not None:
+            e.record()
     splits = [send_splits(d.offsets_host, E, n) for d in disp]       # splits[s][d]
+    if events is not None:
+        events["splits"] = splits
     starts = [[0] * n for _ in range(n)]
     for s in range(n):
         for d in range(1, n):
             starts[s][d] = starts[s][d - 1] + splits[s][d - 1]
-    outs = []
+    recvs, rcs = [], []
+    e = mark("rows")
     for d in range(n):
         rc = torch.stack([counts_by_destination(disp[s].counts, n)[d] for s in range(n)]).contiguous()
         n_in = sum(splits[s][d] for s in range(n))
@@ -194,9 +216,19 @@ def emulate_forward(ranks: Sequence[ExpertParallelRank], xs: Sequence[object], b
             m = splits[s][d]
             recv[a:a + m].copy_(disp[s].send_rows[starts[s][d]:starts[s][d] + m])
             a += m
-        outs.append(ranks[d].experts(recv, rc, n_in))
         assert rc.shape == (n, per)
-    ys = []
+        recvs.append(recv)
+        rcs.append(rc)
+    if e is not None:
+        e.record()
+    outs = []
+    for d in range(n):
+        e = mark("experts")
+        outs.append(ranks[d].experts(recvs[d], rcs[d], recvs[d].shape[0]))
+        if e is not None:
+            e.record()
+    rets = []
+    e = mark("back")
     for s in range(n):
         ret = torch.empty(disp[s].send_rows.shape[0], ranks[s].shape.d_lat, dtype=torch.float32,
                           device=disp[s].send_rows.device)
@@ -205,5 +237,13 @@ def emulate_forward(ranks: Sequence[ExpertParallelRank], xs: Sequence[object], b
             a = sum(splits[q][d] for q in range(s))
             m = splits[s][d]
             ret[starts[s][d]:starts[s][d] + m].copy_(outs[d][a:a + m])
-        ys.append(ranks[s].combine(ret))
+        rets.append(ret)
+    if e is not None:
+        e.record()
+    ys = []
+    for s in range(n):
+        e = mark("combine")
+        ys.append(ranks[s].combine(rets[s]))
+        if e is not None:
+            e.record()
     return ys
