@@ -1,5 +1,7 @@
 // gemm8w_sm100.cuh — the e4m3 block-scaled GEMM with 256 weight columns per
-// unit (prefill-sized FP8 layers).
+// unit: the FP8 layer's expert GEMMs and projections, and the expert GEMMs of
+// the FP4 variant (weights as e2m1 codes, read by the tensor core; see
+// Glu4WPolicy).
 //
 // The arithmetic is gemm8_sm100.cuh's: tokens on M (TMEM lanes), weights on
 // N, each 128-deep K block accumulated alone in a TMEM partial and folded by
