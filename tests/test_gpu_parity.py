@@ -334,10 +334,11 @@ def _fp8_mid_width(T, fp4=False):
 
 
 @pytest.mark.parametrize("T,fp4", [(300, False), (10100, False), (300, True), (10100, True), (64, False),
-                                   (64, True)])
+                                   (64, True), (1, False), (1, True)])
 def test_forward_fp8_mid_width(T, fp4):
     # T = 64: 8 rows per expert on average (groups of 0 to ~20 rows, one
-    # 16- or 32-row token box each)
+    # 16- or 32-row token box each); T = 1: three groups of one row, most
+    # CTAs without a unit
     s = _fp8_mid_width(T, fp4)
     w = W.make_layer_weights(s, "cuda", seed=0)
     x = W.make_x(s, "cuda", seed=0)
