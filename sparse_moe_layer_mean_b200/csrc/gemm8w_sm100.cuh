@@ -315,34 +315,58 @@ struct Dense8WPolicy : Dense8Policy {
     const float *ws0 = p.ws + static_cast<size_t>(U.n0 / 128) * kbs;
     stage_weight_scales(ws0, U.n0 + kF8Tile < p.N ? ws0 + kbs : nullptr, kbs, w, lane);
   }
+  // bf16 rows staged per warp: [2 outputs][32 tokens][4 chunks of 16 bytes]
+  static constexpr int kEpiSmem = 8 * 2 * 32 * 64;
+  // 16-byte chunk c of staged row r sits at c ^ ((r >> 1) & 3): the 128-bit
+  // writes of a quarter-warp (eight rows) and its reads (two rows' four
+  // chunks) both fall on distinct bank groups
+  static __device__ __forceinline__ int chunk_at(int r, int c) { return r * 4 + (c ^ ((r >> 1) & 3)); }
+  // Four passes of 32 columns: the warp's 32 tokens' bf16 values (and, for
+  // the down-projection, the residuals of that rounding) go through its
+  // shared rows so that each store instruction writes eight tokens' 64
+  // contiguous bytes.
   static __device__ __forceinline__ void epilogue_regs(const Params &p, const Unit &U, float (&acc)[kW8Cols], int q,
-                                                       int h, int lane, uint8_t *, const float *) {
-    const int t = q * 32 + lane;
+                                                       int h, int lane, uint8_t *epi, const float *) {
     const int col = U.n0 + h * kW8Cols;
-    if (t >= U.nv || col >= p.N) return;
-    const long row = U.row0 + t;
-    uint4 *dst = reinterpret_cast<uint4 *>(p.out + row * p.ldo + col);
-    uint4 *dlo = p.out_lo ? reinterpret_cast<uint4 *>(p.out_lo + row * p.ldo + col) : nullptr;
+    if (q * 32 >= U.nv || col >= p.N) return;  // the warp holds no token, or its columns lie past N
+    uint4 *rows_hi = reinterpret_cast<uint4 *>(epi) + (h * 4 + q) * 2 * 32 * 4;
+    uint4 *rows_lo = rows_hi + 32 * 4;
+    const bool lo = p.out_lo != nullptr;
 #pragma unroll
-    for (int i = 0; i < kW8Cols / 8; ++i) {
-      const float *v = acc + 8 * i;
-      uint4 w;
-      w.x = pack_bf16x2(v[0], v[1]);
-      w.y = pack_bf16x2(v[2], v[3]);
-      w.z = pack_bf16x2(v[4], v[5]);
-      w.w = pack_bf16x2(v[6], v[7]);
-      dst[i] = w;
-      if (dlo) {
-        float r[8];
+    for (int pass = 0; pass < 4; ++pass) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) r[e] = v[e] - __bfloat162float(__float2bfloat16_rn(v[e]));
-        uint4 l;
-        l.x = pack_bf16x2(r[0], r[1]);
-        l.y = pack_bf16x2(r[2], r[3]);
-        l.z = pack_bf16x2(r[4], r[5]);
-        l.w = pack_bf16x2(r[6], r[7]);
-        dlo[i] = l;
+      for (int c = 0; c < 4; ++c) {
+        const float *v = acc + pass * 32 + 8 * c;
+        uint4 w;
+        w.x = pack_bf16x2(v[0], v[1]);
+        w.y = pack_bf16x2(v[2], v[3]);
+        w.z = pack_bf16x2(v[4], v[5]);
+        w.w = pack_bf16x2(v[6], v[7]);
+        rows_hi[chunk_at(lane, c)] = w;
+        if (lo) {
+          // residual v - bf16(v), from the rounded halves just packed
+          const uint32_t hw[4] = {w.x, w.y, w.z, w.w};
+          uint32_t lw[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            lw[e] = pack_bf16x2(v[2 * e] - __uint_as_float(hw[e] << 16),
+                                v[2 * e + 1] - __uint_as_float(hw[e] & 0xffff0000u));
+          rows_lo[chunk_at(lane, c)] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
       }
+      __syncwarp();
+      const int chunk = lane & 3;  // 16-byte quarter of a token's 64 bytes
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int i = it * 8 + (lane >> 2);  // token within the warp
+        const int t = q * 32 + i;
+        if (t < U.nv) {
+          const size_t o = static_cast<size_t>(U.row0 + t) * p.ldo + col + pass * 32 + chunk * 8;
+          *reinterpret_cast<uint4 *>(p.out + o) = rows_hi[chunk_at(i, chunk)];
+          if (lo) *reinterpret_cast<uint4 *>(p.out_lo + o) = rows_lo[chunk_at(i, chunk)];
+        }
+      }
+      __syncwarp();
     }
   }
 };
