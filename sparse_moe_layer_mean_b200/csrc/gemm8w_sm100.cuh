@@ -66,6 +66,12 @@ __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Shared rows of 64 bytes staged for coalesced stores: 16-byte chunk c of row
+// r sits at chunk index c ^ ((r >> 1) & 3), so the 128-bit writes of a
+// quarter-warp (eight rows) and its reads (two rows' four chunks) both fall
+// on distinct bank groups.
+__device__ __forceinline__ int row64_chunk(int r, int c) { return r * 4 + (c ^ ((r >> 1) & 3)); }
+
 // acc[OFF + i] += r[i] * s for the 32 values of one TMEM load, as packed
 // fp32x2 FMAs (round to nearest per lane: the same values as fmaf).
 template <int OFF>
@@ -315,12 +321,8 @@ struct Dense8WPolicy : Dense8Policy {
     const float *ws0 = p.ws + static_cast<size_t>(U.n0 / 128) * kbs;
     stage_weight_scales(ws0, U.n0 + kF8Tile < p.N ? ws0 + kbs : nullptr, kbs, w, lane);
   }
-  // bf16 rows staged per warp: [2 outputs][32 tokens][4 chunks of 16 bytes]
+  // bf16 rows staged per warp: [2 outputs][32 tokens][64 bytes] (row64_chunk)
   static constexpr int kEpiSmem = 8 * 2 * 32 * 64;
-  // 16-byte chunk c of staged row r sits at c ^ ((r >> 1) & 3): the 128-bit
-  // writes of a quarter-warp (eight rows) and its reads (two rows' four
-  // chunks) both fall on distinct bank groups
-  static __device__ __forceinline__ int chunk_at(int r, int c) { return r * 4 + (c ^ ((r >> 1) & 3)); }
   // Four passes of 32 columns: the warp's 32 tokens' bf16 values (and, for
   // the down-projection, the residuals of that rounding) go through its
   // shared rows so that each store instruction writes eight tokens' 64
@@ -342,7 +344,7 @@ struct Dense8WPolicy : Dense8Policy {
         w.y = pack_bf16x2(v[2], v[3]);
         w.z = pack_bf16x2(v[4], v[5]);
         w.w = pack_bf16x2(v[6], v[7]);
-        rows_hi[chunk_at(lane, c)] = w;
+        rows_hi[row64_chunk(lane, c)] = w;
         if (lo) {
           // residual v - bf16(v), from the rounded halves just packed
           const uint32_t hw[4] = {w.x, w.y, w.z, w.w};
@@ -351,7 +353,7 @@ struct Dense8WPolicy : Dense8Policy {
           for (int e = 0; e < 4; ++e)
             lw[e] = pack_bf16x2(v[2 * e] - __uint_as_float(hw[e] << 16),
                                 v[2 * e + 1] - __uint_as_float(hw[e] & 0xffff0000u));
-          rows_lo[chunk_at(lane, c)] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          rows_lo[row64_chunk(lane, c)] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
       }
       __syncwarp();
@@ -362,8 +364,8 @@ struct Dense8WPolicy : Dense8Policy {
         const int t = q * 32 + i;
         if (t < U.nv) {
           const size_t o = static_cast<size_t>(U.row0 + t) * p.ldo + col + pass * 32 + chunk * 8;
-          *reinterpret_cast<uint4 *>(p.out + o) = rows_hi[chunk_at(i, chunk)];
-          if (lo) *reinterpret_cast<uint4 *>(p.out_lo + o) = rows_lo[chunk_at(i, chunk)];
+          *reinterpret_cast<uint4 *>(p.out + o) = rows_hi[row64_chunk(i, chunk)];
+          if (lo) *reinterpret_cast<uint4 *>(p.out_lo + o) = rows_lo[row64_chunk(i, chunk)];
         }
       }
       __syncwarp();
@@ -387,7 +389,7 @@ struct Glu8WPolicy : Glu8Policy {
   static constexpr uint32_t kWeightFormat = kFmtE4M3;
   static constexpr uint32_t kWeightTxBytes = kW8BBytes;  // bytes the weight loads of a K block complete
   static constexpr bool kGateUp = true;  // columns 0-63 of a thread's half: gate block; 64-127: up block
-  static constexpr int kEpiSmem = 8 * 32 * 4 + 8 * 32 * 17 * 4;  // block maxima, then the code rows
+  static constexpr int kEpiSmem = 8 * 32 * 4 + 8 * 32 * 64;  // block maxima, then the code rows (row64_chunk)
   struct Params {
     CUtensorMap wg, wu, sg, su;  // e4m3 [E*F, L] / [F, L], box 64 x 128
     TokenMaps8 tz;               // quantised dispatched z [(T*k+T), L]
@@ -472,14 +474,18 @@ struct Glu8WPolicy : Glu8Policy {
     }
     const int t = q * 32 + lane;
     if (hh == 0 && t < U.nv) p.hs_t[static_cast<size_t>(U.m) * p.rows + U.row0 + t] = scale;
-    uint32_t *wrow = reinterpret_cast<uint32_t *>(epi + 8 * 32 * 4) + pw * 32 * 17;  // [32 tokens][17 words]
+    uint4 *rows = reinterpret_cast<uint4 *>(epi + 8 * 32 * 4) + pw * 32 * 4;  // [32 tokens][64 bytes]
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float2 a = __fmul2_rn(make_float2(hv[4 * i], hv[4 * i + 1]), make_float2(inv, inv));
-      const float2 b = __fmul2_rn(make_float2(hv[4 * i + 2], hv[4 * i + 3]), make_float2(inv, inv));
-      const uint32_t lo = e4m3x2(a.x, a.y);
-      const uint32_t hi = e4m3x2(b.x, b.y);
-      wrow[lane * 17 + i] = lo | (hi << 16);
+    for (int c = 0; c < 4; ++c) {
+      uint32_t wd[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * c + e;  // word i: codes 4i .. 4i+3
+        const float2 a = __fmul2_rn(make_float2(hv[4 * i], hv[4 * i + 1]), make_float2(inv, inv));
+        const float2 b = __fmul2_rn(make_float2(hv[4 * i + 2], hv[4 * i + 3]), make_float2(inv, inv));
+        wd[e] = static_cast<uint32_t>(e4m3x2(a.x, a.y)) | (static_cast<uint32_t>(e4m3x2(b.x, b.y)) << 16);
+      }
+      rows[row64_chunk(lane, c)] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
     }
     __syncwarp();
     const int chunk = lane & 3;  // 16-byte quarter of a token's 64 bytes
@@ -487,15 +493,9 @@ struct Glu8WPolicy : Glu8Policy {
     for (int it = 0; it < 4; ++it) {
       const int i = it * 8 + (lane >> 2);  // token within the warp
       const int tt = q * 32 + i;
-      if (tt < U.nv) {
-        uint4 w;
-        w.x = wrow[i * 17 + chunk * 4 + 0];
-        w.y = wrow[i * 17 + chunk * 4 + 1];
-        w.z = wrow[i * 17 + chunk * 4 + 2];
-        w.w = wrow[i * 17 + chunk * 4 + 3];
+      if (tt < U.nv)
         *reinterpret_cast<uint4 *>(p.hq + static_cast<size_t>(U.row0 + tt) * p.F + U.m * kF8Tile + hh * 64 +
-                                   chunk * 16) = w;
-      }
+                                   chunk * 16) = rows[row64_chunk(i, chunk)];
     }
     __syncwarp();  // the rows are rewritten by the next unit's epilogue
   }
