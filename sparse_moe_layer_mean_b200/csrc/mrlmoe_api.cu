@@ -560,10 +560,10 @@ mrlmoe_status check_weights_fp8(const mrlmoe_weights *w, bool fp4) {
 
 // Scales go to sc[rows][K/128], or transposed to sc[K/128][rows] (the layout
 // the FP8 GEMMs read) when `transposed`.
-cudaError_t launch_quant(const __nv_bfloat16 *in, long ld_in, int rows, int K, const int32_t *perm, int k, int Tk,
-                         uint8_t *q, float *sc, bool transposed, const uint32_t *status, cudaStream_t st) {
+cudaError_t launch_quant(const __nv_bfloat16 *in, long ld_in, int rows, int K, uint8_t *q, float *sc,
+                         bool transposed, const uint32_t *status, cudaStream_t st) {
   quant_rows_kernel<<<(rows + kQuantWarps - 1) / kQuantWarps, kQuantWarps * 32, 0, st>>>(
-      in, ld_in, rows, K, perm, k, Tk, q, sc, transposed ? static_cast<long>(rows) : 0L, status);
+      in, ld_in, rows, K, q, sc, transposed ? static_cast<long>(rows) : 0L, status);
   return cudaGetLastError();
 }
 
@@ -678,8 +678,7 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
   const int T = c.T, D = c.d_model, Ld = c.d_lat, E = c.n_experts, R = c.n_routers, k = c.top_k;
   __nv_bfloat16 *z = P.zbuf + static_cast<size_t>(T) * k * Ld;  // z rows live after the T*k dispatched rows
   if (c.dtype != MRLMOE_BF16) {
-    MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(x), D, T, D, nullptr, 1, 0, P.xq, P.xs, true, P.status,
-                         st));
+    MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(x), D, T, D, P.xq, P.xs, true, P.status, st));
     mrlmoe_status s = launch_dense8(P.xq, P.xs, w->w_down, w->s_down, T, Ld, D, z, P.zlo, P, sms, st);
     if (s != MRLMOE_OK) return s;
   } else {
@@ -869,9 +868,11 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
     nvtx_stage(i < 8 ? kForwardStages[i] : nullptr);
     return !ev || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st) == cudaSuccess;
   };
-  // quantised dispatched latent rows (rows < T*k) and the shared expert's rows (all T tokens)
-  MRL_TRY(launch_quant(P.zbuf + static_cast<size_t>(Tk) * Ld, Ld, Tk + T, Ld, P.perm, k, Tk, P.zq, P.zs, true,
-                       P.status, st));
+  // quantised dispatched latent rows (rows < T*k) and the shared expert's rows
+  // (all T tokens): each token's latent row quantised once, written to its rows
+  quant_dispatch_rows_kernel<<<(T + kQuantWarps - 1) / kQuantWarps, kQuantWarps * 32, 0, st>>>(
+      P.zbuf + static_cast<size_t>(Tk) * Ld, T, Ld, P.inv, k, Tk, P.zq, P.zs, static_cast<long>(Tk) + T, P.status);
+  MRL_TRY(cudaGetLastError());
   if (!mark(4)) return MRLMOE_ERR_CUDA;
   const GroupTiling gtl = group_tiling(c);
   const bool fp4 = c.dtype == MRLMOE_FP4_E2M1_BLOCK128;  // expert matrices as packed e2m1 codes
@@ -921,7 +922,7 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
       MRL_TRY(launch_gemm8<Glu4Policy>(p, sms, st));
     else
       MRL_TRY(launch_gemm8<Glu8Policy>(p, sms, st));
-    MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, nullptr, 1, 0, P.hq, P.hs, true, P.status, st));
+    MRL_TRY(launch_quant(P.hbuf, F, Tk + T, F, P.hq, P.hs, true, P.status, st));
   }
   if (!mark(5)) return MRLMOE_ERR_CUDA;
   {
@@ -954,7 +955,7 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
   combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k, c.rms_eps,
                                                         reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf, P.status);
   MRL_TRY(cudaGetLastError());
-  MRL_TRY(launch_quant(P.nbuf, Ld, T, Ld, nullptr, 1, 0, P.nq, P.ns, true, P.status, st));
+  MRL_TRY(launch_quant(P.nbuf, Ld, T, Ld, P.nq, P.ns, true, P.status, st));
   if (!mark(7)) return MRLMOE_ERR_CUDA;
   return launch_dense8(P.nq, P.ns, w->w_up, w->s_up, T, D, Ld, static_cast<__nv_bfloat16 *>(y_out), nullptr, P, sms,
                        st);
@@ -1399,8 +1400,8 @@ mrlmoe_status mrlmoe_quantize_e4m3(const void *in, int rows, int K, void *q, flo
   DeviceRestore restore;
   mrlmoe_status s = bind_device(in, &sms, &restore);
   if (s != MRLMOE_OK) return s;
-  MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(in), K, rows, K, nullptr, 1, 0, static_cast<uint8_t *>(q),
-                       scale, false, nullptr, static_cast<cudaStream_t>(stream)));
+  MRL_TRY(launch_quant(static_cast<const __nv_bfloat16 *>(in), K, rows, K, static_cast<uint8_t *>(q), scale, false,
+                       nullptr, static_cast<cudaStream_t>(stream)));
   return MRLMOE_OK;
 }
 

@@ -289,9 +289,6 @@ __global__ void gather_rows_kernel(const int32_t *__restrict__ perm, int rows, i
 // block (16 lanes x 8 bf16: 16-byte loads, 8-byte code stores): amax over the
 // block's bf16 values; amax == 0 -> scale 1, codes 0; else scale = amax / 448
 // and code = e4m3_rn_satfinite(v * (448 / amax)) (fp32 IEEE ops).
-// With `perm`, output row r < Tk takes input row perm[r] / k (a dispatched
-// token) and rows Tk .. Tk+T-1 take input rows 0 .. T-1.  Scales go to
-// s[r][K/128] (s_ld == 0) or, transposed, to s[b * s_ld + r].
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));  // first source -> upper byte
@@ -301,21 +298,49 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 constexpr int kQuantWarps = 8;
 constexpr int kQuantBatch = 4;   // warp iterations whose loads are in flight together
 
-// A warp's loads are issued kQuantBatch iterations (8 blocks) at a time before
-// those blocks are reduced, so a warp waits for memory once per 8 blocks
-// while the block keeps few registers (and many warps per SM).
+// One 128-wide block, quantised by a half-warp: lane hl of the half holds
+// elements 8 hl .. 8 hl + 7 in raw and gets their 8 codes; every lane of the
+// half gets the block's scale.  (The amax reduction stays within the half.)
+__device__ __forceinline__ void quant_block128(uint4 raw, uint2 &codes, float &scale) {
+  float v[8];
+  const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __low2float(h2[i]);
+    v[2 * i + 1] = __high2float(h2[i]);
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  float inv = 0.0f;
+  scale = 1.0f;
+  if (amax != 0.0f) {
+    scale = amax / 448.0f;
+    inv = 448.0f / amax;
+  }
+  codes.x = static_cast<uint32_t>(e4m3x2(v[0] * inv, v[1] * inv)) |
+            (static_cast<uint32_t>(e4m3x2(v[2] * inv, v[3] * inv)) << 16);
+  codes.y = static_cast<uint32_t>(e4m3x2(v[4] * inv, v[5] * inv)) |
+            (static_cast<uint32_t>(e4m3x2(v[6] * inv, v[7] * inv)) << 16);
+}
+
+// Rows of in [rows, K] to codes q [rows, K] and scales s[r][K/128] (s_ld ==
+// 0) or, transposed, s[b * s_ld + r].  A warp's loads are issued kQuantBatch
+// iterations (8 blocks) at a time before those blocks are reduced, so a warp
+// waits for memory once per 8 blocks while the block keeps few registers
+// (and many warps per SM).
 __global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_kernel(
-    const __nv_bfloat16 *__restrict__ in, long ld_in, int rows, int K, const int32_t *__restrict__ perm, int k,
-    int Tk, uint8_t *__restrict__ q, float *__restrict__ s, long s_ld, const uint32_t *status) {
+    const __nv_bfloat16 *__restrict__ in, long ld_in, int rows, int K, uint8_t *__restrict__ q,
+    float *__restrict__ s, long s_ld, const uint32_t *status) {
   if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int kbs = K >> 7;
   const int r = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
   if (r >= rows) return;  // whole warps leave together
   const int lane = threadIdx.x & 31;
   const int half = lane >> 4, hl = lane & 15;
-  long src = r;
-  if (perm) src = r < Tk ? __ldg(perm + r) / k : r - Tk;
-  const __nv_bfloat16 *row_in = in + src * ld_in;
+  const __nv_bfloat16 *row_in = in + static_cast<long>(r) * ld_in;
   uint8_t *row_q = q + static_cast<long>(r) * K;
   for (int it0 = 0; 2 * it0 < kbs; it0 += kQuantBatch) {
     uint4 raw[kQuantBatch];
@@ -328,32 +353,55 @@ __global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_kernel(
     for (int j = 0; j < kQuantBatch; ++j) {
       if (2 * (it0 + j) >= kbs) break;  // uniform across the warp
       const int b = 2 * (it0 + j) + half;
-      const bool live = b < kbs;
-      float v[8];
-      const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[j]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __low2float(h2[i]);
-        v[2 * i + 1] = __high2float(h2[i]);
-      }
-      float amax = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-#pragma unroll
-      for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      float scale = 1.0f, inv = 0.0f;
-      if (amax != 0.0f) {
-        scale = amax / 448.0f;
-        inv = 448.0f / amax;
-      }
-      if (live) {
-        uint2 codes;
-        codes.x = static_cast<uint32_t>(e4m3x2(v[0] * inv, v[1] * inv)) |
-                  (static_cast<uint32_t>(e4m3x2(v[2] * inv, v[3] * inv)) << 16);
-        codes.y = static_cast<uint32_t>(e4m3x2(v[4] * inv, v[5] * inv)) |
-                  (static_cast<uint32_t>(e4m3x2(v[6] * inv, v[7] * inv)) << 16);
+      uint2 codes;
+      float scale;
+      quant_block128(raw[j], codes, scale);
+      if (b < kbs) {
         *reinterpret_cast<uint2 *>(row_q + b * 128 + hl * 8) = codes;
         if (hl == 0) s[s_ld ? b * s_ld + r : static_cast<long>(r) * kbs + b] = scale;
+      }
+    }
+  }
+}
+
+// The FP8 variant's quantised dispatch rows: one warp per token t quantises
+// its latent row z[t] once (the arithmetic above, so every copy holds the
+// codes and scales that quantising it would give) and writes them to each of
+// the token's k dispatch rows inv[t k + j] and to its shared-expert row
+// Tk + t; scales transposed, s[b * s_ld + row].  Each latent row is read
+// once instead of once per dispatch row.
+__global__ void __launch_bounds__(kQuantWarps * 32) quant_dispatch_rows_kernel(
+    const __nv_bfloat16 *__restrict__ z, int T, int K, const int32_t *__restrict__ inv, int k, int Tk,
+    uint8_t *__restrict__ q, float *__restrict__ s, long s_ld, const uint32_t *status) {
+  if (call_failed(status)) return;  // an earlier kernel of the call failed
+  const int kbs = K >> 7;
+  const int t = blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+  if (t >= T) return;  // whole warps leave together
+  const int lane = threadIdx.x & 31;
+  const int half = lane >> 4, hl = lane & 15;
+  // lane j < k holds the dispatch row of (t, j)
+  const int my_row = lane < k ? __ldg(inv + static_cast<size_t>(t) * k + lane) : -1;
+  const __nv_bfloat16 *row_in = z + static_cast<size_t>(t) * K;
+  for (int it0 = 0; 2 * it0 < kbs; it0 += kQuantBatch) {
+    uint4 raw[kQuantBatch];
+#pragma unroll
+    for (int j = 0; j < kQuantBatch; ++j) {
+      const int b = 2 * (it0 + j) + half;
+      raw[j] = b < kbs ? __ldg(reinterpret_cast<const uint4 *>(row_in + b * 128 + hl * 8)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < kQuantBatch; ++j) {
+      if (2 * (it0 + j) >= kbs) break;  // uniform across the warp
+      const int b = 2 * (it0 + j) + half;
+      uint2 codes;
+      float scale;
+      quant_block128(raw[j], codes, scale);
+      for (int d = 0; d <= k; ++d) {
+        const int r = d < k ? __shfl_sync(0xffffffffu, my_row, d) : Tk + t;
+        if (b < kbs && r >= 0 && r < Tk + T) {
+          *reinterpret_cast<uint2 *>(q + static_cast<size_t>(r) * K + b * 128 + hl * 8) = codes;
+          if (hl == 0) s[b * s_ld + r] = scale;
+        }
       }
     }
   }
