@@ -746,6 +746,20 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
 // FP8 variant after the dispatch record: quantised gather of the dispatched
 // latent rows, gate/up, quantised h, expert down, combine + RMSNorm,
 // quantised n, up-projection.  Stage events 4..7 as in the bf16 sequence.
+// The T*k dispatched bf16 latent rows, in dispatch order, into dst from z
+// (rows [T*k, T*k + T) of zbuf).  One warp per token while the batch gives
+// at least 16 warps per SM; a smaller batch splits each token's k
+// destinations over up to k warps.
+cudaError_t launch_copy_dispatch_rows(const Ptrs &P, int T, int Ld, int k, void *dst, int sms, cudaStream_t st) {
+  const int Tk = T * k;
+  const int nsplit = std::min(k, std::max(1, (16 * sms + T - 1) / T));
+  const long long warps = static_cast<long long>(T) * nsplit;
+  copy_dispatch_rows_kernel<<<static_cast<unsigned>((warps + kCopyWarps - 1) / kCopyWarps), kCopyWarps * 32, 0, st>>>(
+      reinterpret_cast<const uint4 *>(P.zbuf + static_cast<size_t>(Tk) * Ld), T, Ld * 2 / 16, P.inv, k, nsplit, Tk,
+      static_cast<uint4 *>(dst), P.status);
+  return cudaGetLastError();
+}
+
 mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *w, const Ptrs &P, int sms,
                                   cudaStream_t st, void *const *ev, void *y_out = nullptr);
 
@@ -803,13 +817,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
   }
 
   // gather the dispatched latent rows (rows [0, T*k) of zbuf) from z (rows [T*k, T*k+T))
-  {
-    const int row_u4 = Ld * 2 / 16;
-    gather_rows_kernel<<<(Tk * 32 + 255) / 256, 256, 0, st>>>(
-        P.perm, Tk, k, reinterpret_cast<const uint4 *>(P.zbuf + static_cast<size_t>(Tk) * Ld),
-        reinterpret_cast<uint4 *>(P.zbuf), row_u4, P.status);
-    MRL_TRY(cudaGetLastError());
-  }
+  MRL_TRY(launch_copy_dispatch_rows(P, T, Ld, k, P.zbuf, sms, st));
   if (!mark(4)) return MRLMOE_ERR_CUDA;
   GroupTable gt1{P.grp_off, P.grp_cnt, P.unit1, E, glu_m_tiles(*cfg)};
   GroupTable gt2{P.grp_off, P.grp_cnt, P.unit2, E, down_m_tiles(*cfg)};
@@ -1490,11 +1498,7 @@ mrlmoe_status mrlmoe_ep_dispatch(const mrlmoe_config *cfg, const mrlmoe_weights 
   nvtx_stage(kForwardStages[2]);
   if ((s = launch_dispatch(*cfg, P, st)) != MRLMOE_OK) return s;
   nvtx_stage(kForwardStages[3]);
-  const int row_u4 = Ld * 2 / 16;
-  gather_rows_kernel<<<(Tk * 32 + 255) / 256, 256, 0, st>>>(
-      P.perm, Tk, k, reinterpret_cast<const uint4 *>(P.zbuf + static_cast<size_t>(Tk) * Ld),
-      static_cast<uint4 *>(send_rows), row_u4, P.status);
-  MRL_TRY(cudaGetLastError());
+  MRL_TRY(launch_copy_dispatch_rows(P, T, Ld, k, send_rows, sms, st));
   const size_t n = static_cast<size_t>(Tk) * 4;
   if (out->topk_idx) MRL_TRY(cudaMemcpyAsync(out->topk_idx, P.topk_idx, n, cudaMemcpyDeviceToDevice, st));
   if (out->topk_w) MRL_TRY(cudaMemcpyAsync(out->topk_w, P.topk_w, n, cudaMemcpyDeviceToDevice, st));

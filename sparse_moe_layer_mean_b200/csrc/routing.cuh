@@ -270,18 +270,44 @@ __global__ void expert_scatter_kernel(const int32_t *__restrict__ topk_idx, cons
   }
 }
 
-// Row gather: zd[row] = zs[perm[row] / k] for row < T*k (one warp per row).
-__global__ void gather_rows_kernel(const int32_t *__restrict__ perm, int rows, int k,
-                                   const uint4 *__restrict__ zs, uint4 *__restrict__ zd, int row_u4,
-                                   const uint32_t *status) {
+// Dispatch-row copy: zd[inv[t*k + j]] = zs[t] for j < k.  Warp w takes token
+// t = w / nsplit and its destinations j = w % nsplit, + nsplit, ...: it reads
+// the token's row, 32 lanes x kCopyU4 uint4 at a time, and writes each chunk
+// to those dispatch rows (lane j < k holds the row of (t, j)), so the stores
+// of a chunk are in flight behind one round of loads.  nsplit = 1 reads each
+// row once; a small batch takes nsplit > 1 to occupy more warps.  A row
+// index outside [0, rows) is skipped.
+constexpr int kCopyWarps = 8;
+constexpr int kCopyU4 = 8;
+
+__global__ void __launch_bounds__(kCopyWarps * 32) copy_dispatch_rows_kernel(
+    const uint4 *__restrict__ zs, int T, int row_u4, const int32_t *__restrict__ inv, int k, int nsplit,
+    int rows, uint4 *__restrict__ zd, const uint32_t *status) {
   if (call_failed(status)) return;  // an earlier kernel of the call failed
-  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int w = blockIdx.x * kCopyWarps + (threadIdx.x >> 5);
+  const int t = w / nsplit, part = w - t * nsplit;
+  if (t >= T) return;  // whole warps leave together
   const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
-  const int t = __ldg(perm + r) / k;
+  const int my_row = lane < k ? __ldg(inv + static_cast<size_t>(t) * k + lane) : -1;
   const uint4 *src = zs + static_cast<size_t>(t) * row_u4;
-  uint4 *dst = zd + static_cast<size_t>(r) * row_u4;
-  for (int i = lane; i < row_u4; i += 32) dst[i] = __ldg(src + i);
+  for (int c0 = 0; c0 < row_u4; c0 += 32 * kCopyU4) {
+    uint4 v[kCopyU4];
+#pragma unroll
+    for (int j = 0; j < kCopyU4; ++j) {
+      const int i = c0 + j * 32 + lane;
+      v[j] = i < row_u4 ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int d = part; d < k; d += nsplit) {
+      const int r = __shfl_sync(0xffffffffu, my_row, d);
+      if (r < 0 || r >= rows) continue;  // uniform across the warp
+      uint4 *dst = zd + static_cast<size_t>(r) * row_u4;
+#pragma unroll
+      for (int j = 0; j < kCopyU4; ++j) {
+        const int i = c0 + j * 32 + lane;
+        if (i < row_u4) dst[i] = v[j];
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
