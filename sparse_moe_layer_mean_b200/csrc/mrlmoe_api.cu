@@ -746,6 +746,23 @@ mrlmoe_status launch_project_and_route(const mrlmoe_config &c, const mrlmoe_weig
 // FP8 variant after the dispatch record: quantised gather of the dispatched
 // latent rows, gate/up, quantised h, expert down, combine + RMSNorm,
 // quantised n, up-projection.  Stage events 4..7 as in the bf16 sequence.
+// Combine + RMSNorm of the T tokens' slots into nbuf, instantiated for the
+// float4s each of the 256 threads holds (d_lat <= 1024 / 2048 / 4096 / 8192).
+cudaError_t launch_combine(const Ptrs &P, int T, int Ld, int k, float eps, const void *gain, cudaStream_t st) {
+  const float4 *slots = reinterpret_cast<const float4 *>(P.slots);
+  const float4 *g = reinterpret_cast<const float4 *>(gain);
+  const int L4 = Ld / 4;
+  if (L4 <= kCombineThreads)
+    combine_rmsnorm_kernel<1><<<T, kCombineThreads, 0, st>>>(slots, Ld, k, eps, g, P.nbuf, P.status);
+  else if (L4 <= 2 * kCombineThreads)
+    combine_rmsnorm_kernel<2><<<T, kCombineThreads, 0, st>>>(slots, Ld, k, eps, g, P.nbuf, P.status);
+  else if (L4 <= 4 * kCombineThreads)
+    combine_rmsnorm_kernel<4><<<T, kCombineThreads, 0, st>>>(slots, Ld, k, eps, g, P.nbuf, P.status);
+  else
+    combine_rmsnorm_kernel<kCombineMaxV4><<<T, kCombineThreads, 0, st>>>(slots, Ld, k, eps, g, P.nbuf, P.status);
+  return cudaGetLastError();
+}
+
 // The T*k dispatched bf16 latent rows, in dispatch order, into dst from z
 // (rows [T*k, T*k + T) of zbuf).  One warp per token while the batch gives
 // at least 16 warps per SM; a smaller batch splits each token's k
@@ -854,10 +871,7 @@ mrlmoe_status forward_impl(const mrlmoe_config *cfg, const mrlmoe_weights *w, co
       MRL_TRY(launch_gemm<DownPolicy>(p, sms, st));
   }
   if (!mark(6)) return MRLMOE_ERR_CUDA;
-  combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k,
-                                                        cfg->rms_eps,
-                                                        reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf, P.status);
-  MRL_TRY(cudaGetLastError());
+  MRL_TRY(launch_combine(P, T, Ld, k, cfg->rms_eps, w->rms_gain, st));
   if (!mark(7)) return MRLMOE_ERR_CUDA;
   {
     mrlmoe_status s = launch_dense_bf16(P.nbuf, w->w_up, static_cast<__nv_bfloat16 *>(y), nullptr, T, D, Ld,
@@ -960,9 +974,7 @@ mrlmoe_status forward_experts_fp8(const mrlmoe_config &c, const mrlmoe_weights *
       MRL_TRY(launch_gemm8<Down8Policy>(p, sms, st));
   }
   if (!mark(6)) return MRLMOE_ERR_CUDA;
-  combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(reinterpret_cast<const float4 *>(P.slots), Ld, k, c.rms_eps,
-                                                        reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf, P.status);
-  MRL_TRY(cudaGetLastError());
+  MRL_TRY(launch_combine(P, T, Ld, k, c.rms_eps, w->rms_gain, st));
   MRL_TRY(launch_quant(P.nbuf, Ld, T, Ld, P.nq, P.ns, true, P.status, st));
   if (!mark(7)) return MRLMOE_ERR_CUDA;
   return launch_dense8(P.nq, P.ns, w->w_up, w->s_up, T, D, Ld, static_cast<__nv_bfloat16 *>(y_out), nullptr, P, sms,

@@ -445,13 +445,14 @@ constexpr int kCombineMaxV4 = 8;  // d_lat <= 8192
 // token t's combined row (element i = threadIdx.x + v * kCombineThreads);
 // sum of squares in a fixed order (per thread, then warp tree, then warps in
 // order), n = bf16(c * (1 / sqrt(mean(c^2) + eps)) * gain).
-__device__ __forceinline__ void rmsnorm_row(const float4 (&c)[kCombineMaxV4], int L, float eps,
+template <int NV>
+__device__ __forceinline__ void rmsnorm_row(const float4 (&c)[NV], int L, float eps,
                                             const float4 *__restrict__ gain, __nv_bfloat16 *__restrict__ n_row,
                                             float *red) {
   const int L4 = L >> 2;
   float ss = 0.f;
 #pragma unroll
-  for (int v = 0; v < kCombineMaxV4; ++v) {
+  for (int v = 0; v < NV; ++v) {
     const int i = threadIdx.x + v * kCombineThreads;
     if (i < L4) ss += c[v].x * c[v].x + c[v].y * c[v].y + c[v].z * c[v].z + c[v].w * c[v].w;
   }
@@ -465,7 +466,7 @@ __device__ __forceinline__ void rmsnorm_row(const float4 (&c)[kCombineMaxV4], in
   const float inv = 1.0f / sqrtf(tot / static_cast<float>(L) + eps);
   uint2 *dst = reinterpret_cast<uint2 *>(n_row);
 #pragma unroll
-  for (int v = 0; v < kCombineMaxV4; ++v) {
+  for (int v = 0; v < NV; ++v) {
     const int i = threadIdx.x + v * kCombineThreads;
     if (i < L4) {
       const float4 g = __ldg(gain + i);
@@ -477,25 +478,43 @@ __device__ __forceinline__ void rmsnorm_row(const float4 (&c)[kCombineMaxV4], in
   }
 }
 
+// NV = float4s per thread (L <= 4 * 256 * NV).  The k + 1 slot loads of a
+// thread are issued in batches of kJ per float4 before they are added, so
+// several loads are in flight per thread; the adds keep the slot order.
+template <int NV>
 __global__ void __launch_bounds__(kCombineThreads) combine_rmsnorm_kernel(
     const float4 *__restrict__ slots, int L, int k, float eps, const float4 *__restrict__ gain,
     __nv_bfloat16 *__restrict__ n, const uint32_t *status) {
+  constexpr int kJ = NV >= 8 ? 1 : 8 / NV;
   __shared__ float red[kCombineThreads / 32];
   if (call_failed(status)) return;  // an earlier kernel of the call failed
   const int t = blockIdx.x;
   const int L4 = L >> 2;
   const float4 *base = slots + static_cast<size_t>(t) * (k + 1) * L4;
-  float4 c[kCombineMaxV4];
+  float4 c[NV];
 #pragma unroll
-  for (int v = 0; v < kCombineMaxV4; ++v) {
+  for (int v = 0; v < NV; ++v) {
     const int i = threadIdx.x + v * kCombineThreads;
-    if (i < L4) {
-      float4 a = __ldg(base + i);
-      for (int j = 1; j <= k; ++j) {
-        const float4 b = __ldg(base + static_cast<size_t>(j) * L4 + i);
-        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    c[v] = i < L4 ? __ldg(base + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int j0 = 1; j0 <= k; j0 += kJ) {
+    float4 b[NV][kJ];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int i = threadIdx.x + v * kCombineThreads;
+#pragma unroll
+      for (int jj = 0; jj < kJ; ++jj)
+        b[v][jj] = i < L4 && j0 + jj <= k ? __ldg(base + static_cast<size_t>(j0 + jj) * L4 + i)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+#pragma unroll
+      for (int jj = 0; jj < kJ; ++jj) {
+        if (j0 + jj <= k) {
+          c[v].x += b[v][jj].x; c[v].y += b[v][jj].y; c[v].z += b[v][jj].z; c[v].w += b[v][jj].w;
+        }
       }
-      c[v] = a;
     }
   }
   rmsnorm_row(c, L, eps, gain, n + static_cast<size_t>(t) * L, red);
