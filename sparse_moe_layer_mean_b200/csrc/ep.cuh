@@ -102,7 +102,8 @@ __global__ void __launch_bounds__(1024) ep_layout_kernel(const int32_t *__restri
 
 // One block per (source, local expert): copies that run of received rows to
 // its expert-major position and records, for each expert-major row, the
-// arrival position its output goes back to.  Rows of d_lat bf16 (uint4s).
+// arrival position its output goes back to.  Rows of d_lat bf16 (uint4s); a
+// thread moves four uint4s per pass, loads first, so four are in flight.
 __global__ void ep_gather_kernel(const uint4 *__restrict__ recv, int row_u4, const int32_t *__restrict__ recv_counts,
                                  const int32_t *__restrict__ src, const int32_t *__restrict__ dst,
                                  uint4 *__restrict__ rows, int32_t *__restrict__ out_row, const uint32_t *status) {
@@ -114,7 +115,17 @@ __global__ void ep_gather_kernel(const uint4 *__restrict__ recv, int row_u4, con
   const long long total = static_cast<long long>(n) * row_u4;
   const uint4 *from = recv + static_cast<size_t>(a) * row_u4;
   uint4 *to = rows + static_cast<size_t>(b) * row_u4;
-  for (long long i = threadIdx.x; i < total; i += blockDim.x) to[i] = __ldg(from + i);
+  const long long bd = blockDim.x;
+  long long i = threadIdx.x;
+  for (; i + 3 * bd < total; i += 4 * bd) {
+    const uint4 v0 = __ldg(from + i), v1 = __ldg(from + i + bd), v2 = __ldg(from + i + 2 * bd),
+                v3 = __ldg(from + i + 3 * bd);
+    to[i] = v0;
+    to[i + bd] = v1;
+    to[i + 2 * bd] = v2;
+    to[i + 3 * bd] = v3;
+  }
+  for (; i < total; i += bd) to[i] = __ldg(from + i);
 }
 
 // Combine on the source rank from the returned rows (dispatch order) and the
@@ -126,10 +137,15 @@ __global__ void ep_gather_kernel(const uint4 *__restrict__ recv, int row_u4, con
 // The products are rounded to fp32 before each add (no fused multiply-add),
 // as the single-GPU down GEMM stores fp32(w' o) in its slot; the RMSNorm half
 // is the single-GPU combine's own (rmsnorm_row).
+// NV = float4s per thread; the returned rows' loads are issued in batches
+// of kJ per float4 before they are added (in dispatch-slot order), as in
+// the single-GPU combine.
+template <int NV>
 __global__ void __launch_bounds__(kCombineThreads) ep_combine_rmsnorm_kernel(
     const float4 *__restrict__ ret, const int32_t *__restrict__ inv, const float *__restrict__ wscaled,
     const float4 *__restrict__ slots, int L, int k, float eps, const float4 *__restrict__ gain,
     __nv_bfloat16 *__restrict__ n, const uint32_t *status) {
+  constexpr int kJ = NV >= 8 ? 1 : 8 / NV;
   __shared__ float red[kCombineThreads / 32];
   __shared__ int s_row[32];
   __shared__ float s_w[32];
@@ -142,26 +158,46 @@ __global__ void __launch_bounds__(kCombineThreads) ep_combine_rmsnorm_kernel(
   }
   __syncthreads();
   const float4 *sh = slots + (static_cast<size_t>(t) * (k + 1) + k) * L4;
-  float4 c[kCombineMaxV4];
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 c[NV];
+  {
+    const float w0 = s_w[0];
+    const float4 *r0 = ret + static_cast<size_t>(s_row[0]) * L4;
 #pragma unroll
-  for (int v = 0; v < kCombineMaxV4; ++v) {
-    const int i = threadIdx.x + v * kCombineThreads;
-    if (i < L4) {
-      const float4 o0 = __ldg(ret + static_cast<size_t>(s_row[0]) * L4 + i);
-      const float w0 = s_w[0];
-      float4 a = make_float4(__fmul_rn(o0.x, w0), __fmul_rn(o0.y, w0), __fmul_rn(o0.z, w0), __fmul_rn(o0.w, w0));
-      for (int j = 1; j < k; ++j) {
-        const float4 o = __ldg(ret + static_cast<size_t>(s_row[j]) * L4 + i);
-        const float wj = s_w[j];
-        a.x = __fadd_rn(a.x, __fmul_rn(o.x, wj));
-        a.y = __fadd_rn(a.y, __fmul_rn(o.y, wj));
-        a.z = __fadd_rn(a.z, __fmul_rn(o.z, wj));
-        a.w = __fadd_rn(a.w, __fmul_rn(o.w, wj));
-      }
-      const float4 b = __ldg(sh + i);
-      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-      c[v] = a;
+    for (int v = 0; v < NV; ++v) {
+      const int i = threadIdx.x + v * kCombineThreads;
+      const float4 o0 = i < L4 ? __ldg(r0 + i) : zero;
+      c[v] = make_float4(__fmul_rn(o0.x, w0), __fmul_rn(o0.y, w0), __fmul_rn(o0.z, w0), __fmul_rn(o0.w, w0));
     }
+  }
+  for (int j0 = 1; j0 < k; j0 += kJ) {
+    float4 b[NV][kJ];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int i = threadIdx.x + v * kCombineThreads;
+#pragma unroll
+      for (int jj = 0; jj < kJ; ++jj)
+        b[v][jj] = i < L4 && j0 + jj < k ? __ldg(ret + static_cast<size_t>(s_row[j0 + jj]) * L4 + i) : zero;
+    }
+#pragma unroll
+    for (int jj = 0; jj < kJ; ++jj) {
+      if (j0 + jj < k) {
+        const float wj = s_w[j0 + jj];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          c[v].x = __fadd_rn(c[v].x, __fmul_rn(b[v][jj].x, wj));
+          c[v].y = __fadd_rn(c[v].y, __fmul_rn(b[v][jj].y, wj));
+          c[v].z = __fadd_rn(c[v].z, __fmul_rn(b[v][jj].z, wj));
+          c[v].w = __fadd_rn(c[v].w, __fmul_rn(b[v][jj].w, wj));
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const int i = threadIdx.x + v * kCombineThreads;
+    const float4 b = i < L4 ? __ldg(sh + i) : zero;
+    c[v].x += b.x; c[v].y += b.y; c[v].z += b.z; c[v].w += b.w;
   }
   rmsnorm_row(c, L, eps, gain, n + static_cast<size_t>(t) * L, red);
 }

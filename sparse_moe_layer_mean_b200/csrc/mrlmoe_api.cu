@@ -1655,10 +1655,26 @@ mrlmoe_status mrlmoe_ep_combine(const mrlmoe_config *cfg, const mrlmoe_weights *
       MRL_TRY(launch_gemm<DownPolicy>(p, sms, st));
   }
   nvtx_stage(kForwardStages[6]);
-  ep_combine_rmsnorm_kernel<<<T, kCombineThreads, 0, st>>>(
-      reinterpret_cast<const float4 *>(ret_rows), P.inv, P.wscaled, reinterpret_cast<const float4 *>(P.slots), Ld, k,
-      cfg->rms_eps, reinterpret_cast<const float4 *>(w->rms_gain), P.nbuf, P.status);
-  MRL_TRY(cudaGetLastError());
+  {
+    const float4 *ret = reinterpret_cast<const float4 *>(ret_rows);
+    const float4 *slots = reinterpret_cast<const float4 *>(P.slots);
+    const float4 *g = reinterpret_cast<const float4 *>(w->rms_gain);
+    const float eps = cfg->rms_eps;
+    const int L4 = Ld / 4;
+    if (L4 <= kCombineThreads)
+      ep_combine_rmsnorm_kernel<1><<<T, kCombineThreads, 0, st>>>(ret, P.inv, P.wscaled, slots, Ld, k, eps, g,
+                                                                  P.nbuf, P.status);
+    else if (L4 <= 2 * kCombineThreads)
+      ep_combine_rmsnorm_kernel<2><<<T, kCombineThreads, 0, st>>>(ret, P.inv, P.wscaled, slots, Ld, k, eps, g,
+                                                                  P.nbuf, P.status);
+    else if (L4 <= 4 * kCombineThreads)
+      ep_combine_rmsnorm_kernel<4><<<T, kCombineThreads, 0, st>>>(ret, P.inv, P.wscaled, slots, Ld, k, eps, g,
+                                                                  P.nbuf, P.status);
+    else
+      ep_combine_rmsnorm_kernel<kCombineMaxV4><<<T, kCombineThreads, 0, st>>>(ret, P.inv, P.wscaled, slots, Ld, k,
+                                                                              eps, g, P.nbuf, P.status);
+    MRL_TRY(cudaGetLastError());
+  }
   nvtx_stage(kForwardStages[7]);
   return launch_dense_bf16(P.nbuf, w->w_up, static_cast<__nv_bfloat16 *>(y), nullptr, T, D, Ld, P.status, sms, st);
 }
