@@ -223,10 +223,10 @@ mrlmoe_status mrlmoe_bias_update(const mrlmoe_config *cfg, const int32_t *counts
 mrlmoe_status mrlmoe_linear(const void *a, const void *w, void *out,
                             int M, int N, int K, void *stream);
 
-/* Routing from caller-given fp32 scores WITHOUT a workspace (no counterpart in
- * the paper: an entry point for callers that cannot allocate device memory,
- * e.g. code running inside a framework that owns every allocation, or a
- * graph of pre-planned buffers).  Same results as mrlmoe_route with
+/* Routing from caller-given fp32 scores WITHOUT a workspace (no counterpart
+ * in the method's description: an entry point for callers that cannot
+ * allocate device memory, e.g. code running inside a framework that owns
+ * every allocation, or a graph of pre-planned buffers).  Same results as mrlmoe_route with
  * scores_in = 1: out->scores holds s [T, E]; out->topk_idx, topk_w, counts,
  * offsets, perm and inv_perm must all be non-NULL and receive the record.
  * Its scratch (per-chunk expert masks and prefixes, scaled weights, group
