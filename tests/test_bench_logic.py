@@ -68,3 +68,17 @@ def test_e4m3_peak_falls_back_to_twice_the_sustained_bf16_peak():
     peak, kind, _ = bench.e4m3_peak("dev", PEAKS, "measured")
     assert peak == 2500.0 and kind.startswith("measured")
     bench._E4M3_PROBE.clear()
+
+
+def test_profiled_traffic_only_on_the_sources_it_was_taken_on(tmp_path, monkeypatch):
+    # a committed summary carries the hash of csrc/ it was captured on; any
+    # other hash reads as "no traffic figure"
+    (tmp_path / "profiles").mkdir()
+    p = tmp_path / "profiles" / "k__w.json"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "csrc_hash", lambda: "abc")
+    p.write_text('{"csrc_hash": "abc", "dram_bytes_per_launch_full": 123.0}')
+    assert bench.profiled_traffic("k", "w") == 123.0
+    p.write_text('{"csrc_hash": "old", "dram_bytes_per_launch_full": 123.0}')
+    assert bench.profiled_traffic("k", "w") is None
+    assert bench.profiled_traffic("missing", "w") is None
